@@ -1,0 +1,208 @@
+"""fp64 CPU oracle of the Kimi Delta Attention forward pass.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this module.  It shares no code with
+the CUDA path and imports nothing from it.
+
+Three independent CPU computations of the same quantity:
+
+``recurrent``     the plain definition, token by token, in C (kda_recurrence.c,
+                  fp64, OpenMP over (sequence, head)).  This is the oracle.
+``brute_force``   the unrolled product form of the same recurrence for one
+                  (sequence, head) and T <= 8, written with explicit
+                  d_k x d_k transition matrices M_t = (I - b_t k_t k_t^T) Diag(a_t):
+                  S_t = M_t ... M_1 S_0 + sum_i (M_t ... M_{i+1}) b_i k_i v_i^T.
+                  Each prefix t is recomputed from scratch, so it is not the
+                  recurrence evaluated a second time.
+``chunked_debug`` an fp64 model of the chunkwise rewrite that the GPU prefill
+                  kernels use (decay prefix sums, the strictly-lower factor
+                  matrix A, T = (I + A)^-1 by forward substitution, W, U, the
+                  per-chunk state pass and the output).  Used to localise GPU
+                  stage errors; pinned to ``recurrent`` by the tests.
+
+Sources (paraphrased): the delta-rule read/error/write ("Kimi Delta Attention",
+akshathtiwari.co.in, delta-rule passage; "Attention? More like notation
+warfare", Key Points); the per-key-channel forget vector applied as
+Diag(alpha_t) ("Kimi Delta Attention", akshathtiwari.co.in, channel-wise gating
+passage; "Teacher guide - Kimi Delta Attention", Misconceptions table row 2;
+"The fourth layer remembers", forget-gate paragraph); the chunkwise
+reorganisation of the recurrence into matrix products ("You Could Have Come Up
+with Kimi Delta Attention", daily.dev, Summary; the explainer's remark on the
+Diagonal-Plus-Low-Rank chunkwise algorithm).
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build_oracle
+
+_libs = {}
+
+
+def _load(path=None):
+    """Load (building if needed) the oracle library, or another build of the
+    same source at ``path`` (the tests load deliberately broken copies)."""
+    if path is None:
+        path = build_oracle.build()
+    if path not in _libs:
+        lib = ctypes.CDLL(path)
+        P = ctypes.POINTER(ctypes.c_double)
+        I64 = ctypes.c_int64
+        lib.kda_oracle_recurrent.restype = ctypes.c_int
+        lib.kda_oracle_recurrent.argtypes = [
+            I64, ctypes.POINTER(I64), I64, I64, I64, P, P, P, P, P, P, P, P]
+        lib.kda_oracle_num_threads.restype = ctypes.c_int
+        lib.kda_oracle_num_threads.argtypes = []
+        _libs[path] = lib
+    return _libs[path]
+
+
+def num_threads() -> int:
+    """Threads the oracle's OpenMP region uses (OMP_NUM_THREADS or all cores)."""
+    return int(_load().kda_oracle_num_threads())
+
+
+def _f64(x):
+    if x is None:
+        return None
+    if hasattr(x, "detach"):  # a torch tensor on the host
+        x = x.detach().cpu().double().numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def recurrent(q, k, v, log_alpha, beta, initial_state=None, seq_offsets=None,
+              library=None):
+    """Token-by-token fp64 recurrence (the oracle).
+
+    Shapes: q, k, log_alpha [B, T, H, d_k] (or [T_total, H, d_k] with
+    ``seq_offsets``); v [.., H, d_v]; beta [.., H]; initial_state
+    [n_seqs, H, d_k, d_v] or None (zeros).  ``seq_offsets`` (n_seqs + 1 token
+    offsets into the packed token axis) selects the variable-length layout.
+    Returns (out [same leading shape, H, d_v], final_state [n_seqs, H, d_k, d_v]),
+    both float64.  ``library`` selects another build of the C source.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    la, b = _f64(log_alpha), _f64(beta)
+    s0 = _f64(initial_state)
+    lead = q.shape[:-2]
+    H, dk = q.shape[-2], q.shape[-1]
+    dv = v.shape[-1]
+    if seq_offsets is None:
+        if q.ndim != 4:
+            raise ValueError("without seq_offsets q must be [B, T, H, d_k]")
+        B, T = q.shape[0], q.shape[1]
+        offs = np.arange(B + 1, dtype=np.int64) * T
+    else:
+        if q.ndim == 4:
+            if q.shape[0] != 1:
+                raise ValueError("packed layout needs B == 1")
+        offs = np.ascontiguousarray(np.asarray(seq_offsets, dtype=np.int64))
+    n_seqs = len(offs) - 1
+    T_total = int(np.prod(lead))
+    if offs[0] != 0 or offs[-1] != T_total:
+        raise ValueError("seq_offsets must start at 0 and end at the token count")
+    if s0 is not None and s0.shape != (n_seqs, H, dk, dv):
+        raise ValueError(f"initial_state shape {s0.shape} != {(n_seqs, H, dk, dv)}")
+    out = np.zeros(lead + (H, dv), dtype=np.float64)
+    fin = np.zeros((n_seqs, H, dk, dv), dtype=np.float64)
+    rc = _load(library).kda_oracle_recurrent(
+        n_seqs, offs.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), H, dk, dv,
+        _ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(b), _ptr(s0), _ptr(out),
+        _ptr(fin))
+    if rc != 0:
+        raise RuntimeError(f"kda_oracle_recurrent failed ({rc})")
+    return out, fin
+
+
+def brute_force(q, k, v, log_alpha, beta, initial_state=None):
+    """Unrolled-product evaluation for ONE (sequence, head), T <= 8.
+
+    q, k, log_alpha [T, d_k]; v [T, d_v]; beta [T]; initial_state [d_k, d_v].
+    Returns (out [T, d_v], final_state [d_k, d_v]).
+    """
+    q, k, v, la, b = map(_f64, (q, k, v, log_alpha, beta))
+    T, dk = k.shape
+    dv = v.shape[1]
+    if T > 8:
+        raise ValueError("brute force is for T <= 8")
+    S0 = np.zeros((dk, dv)) if initial_state is None else _f64(initial_state)
+    eye = np.eye(dk)
+    M = [(eye - b[t] * np.outer(k[t], k[t])) @ np.diag(np.exp(la[t]))
+         for t in range(T)]
+
+    def prod(lo, hi):  # M_hi-1 @ ... @ M_lo  (identity when empty)
+        P = eye.copy()
+        for t in range(lo, hi):
+            P = M[t] @ P
+        return P
+
+    out = np.zeros((T, dv))
+    S_t = S0
+    for t in range(1, T + 1):
+        S_t = prod(0, t) @ S0
+        for i in range(t):
+            S_t = S_t + prod(i + 1, t) @ (b[i] * np.outer(k[i], v[i]))
+        out[t - 1] = S_t.T @ q[t - 1]
+    return out, S_t
+
+
+def _forward_substitution_inverse(A):
+    """(I + A)^-1 for strictly-lower A, one row at a time:
+    row r of X = e_r - sum_{i<r} A[r, i] * row i of X."""
+    n = A.shape[0]
+    X = np.zeros_like(A)
+    for r in range(n):
+        X[r, r] = 1.0
+        for i in range(r):
+            X[r, :] -= A[r, i] * X[i, :]
+    return X
+
+
+def chunked_debug(q, k, v, log_alpha, beta, initial_state=None, chunk=64):
+    """fp64 model of the chunkwise rewrite for ONE (sequence, head).
+
+    Per chunk of C tokens (positions r = 1..C), with chunk-start state S_0:
+      g_r   = sum_{i<=r} l_i                   (per key channel)
+      Kt    = k * exp(g)      Kb = k * exp(-g)      Qt = q * exp(g)
+      Kh    = k * exp(g_C - g)
+      A     = strictly_lower(Diag(beta) Kt Kb^T)
+      Tm    = (I + A)^-1      (forward substitution)
+      W     = Tm Diag(beta) Kt          U = Tm Diag(beta) V
+      Delta = U - W S_0
+      O     = Qt S_0 + lower_incl(Qt Kb^T) Delta
+      S_C   = Diag(exp(g_C)) S_0 + Kh^T Delta
+    The last chunk may be shorter than C.  Returns a dict with 'out', 'final'
+    and per-chunk lists 'g', 'A', 'Tm', 'W', 'U', 'S_start'.
+    """
+    q, k, v, la, b = map(_f64, (q, k, v, log_alpha, beta))
+    T, dk = k.shape
+    dv = v.shape[1]
+    S = np.zeros((dk, dv)) if initial_state is None else _f64(initial_state).copy()
+    out = np.zeros((T, dv))
+    rec = {k_: [] for k_ in ("g", "A", "Tm", "W", "U", "S_start")}
+    for c0 in range(0, T, chunk):
+        c1 = min(T, c0 + chunk)
+        kc, qc, vc, lc, bc = k[c0:c1], q[c0:c1], v[c0:c1], la[c0:c1], b[c0:c1]
+        g = np.cumsum(lc, axis=0)
+        Kt, Kb, Qt = kc * np.exp(g), kc * np.exp(-g), qc * np.exp(g)
+        Kh = kc * np.exp(g[-1][None, :] - g)
+        A = np.tril(bc[:, None] * (Kt @ Kb.T), -1)
+        Tm = _forward_substitution_inverse(A)
+        W = Tm @ (bc[:, None] * Kt)
+        U = Tm @ (bc[:, None] * vc)
+        Delta = U - W @ S
+        out[c0:c1] = Qt @ S + np.tril(Qt @ Kb.T, 0) @ Delta
+        for name, val in (("g", g), ("A", A), ("Tm", Tm), ("W", W), ("U", U),
+                          ("S_start", S.copy())):
+            rec[name].append(val)
+        S = np.exp(g[-1])[:, None] * S + Kh.T @ Delta
+    rec["out"] = out
+    rec["final"] = S
+    return rec
