@@ -1,0 +1,440 @@
+#!/usr/bin/env python
+"""Benchmark of the KDA forward on B200: chunkwise prefill tokens/s (with the
+fraction of the dense bf16 tensor peak and of HBM bandwidth) and the decode
+step's GB/s, one JSON line on rank 0.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kda|reference]
+
+Workloads (synthetic, seeded):
+  prefill  kda_chunk_fwd, B=2 sequences x T=8192 tokens, H=32 heads,
+           d_k=d_v=128, chunk 64, bf16 q/k/v/out, fp32 log_alpha/beta, zero
+           initial state, fp32 final state.  Inputs (~0.8 GB) exceed the
+           126 MB L2, so no flush is needed between iterations.
+  decode   kda_recurrent_step, 256 sequences x 32 heads, d=128, one token per
+           step, fp32 state (537 MB) updated in place.
+With N ranks each GPU runs its own copy of the workload (weak scaling, no
+collective on the data path); time is the max over ranks.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import kda_workloads as W  # noqa: E402
+
+METRIC = "KDA fwd tokens/s (H=32,d=128,bf16) + % tensor peak; decode GB/s vs HBM"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+PREFILL_CFG, DECODE_CFG = 2, 4
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def prefill_bytes(B, T, H, dk, dv, io_bytes=2, init_state=False):
+    """Algorithmic HBM bytes of one kda_chunk_fwd: q, k, v read and o written
+    once (io dtype), log_alpha (fp32) and beta (fp32) read once, the fp32
+    final state written (and the initial state read when given)."""
+    th = B * T * H
+    n = th * (2 * dk + 2 * dv) * io_bytes + th * dk * 4 + th * 4
+    n += B * H * dk * dv * 4 * (2 if init_state else 1)
+    return n
+
+
+def prefill_flops(B, T, H, dk, dv, C):
+    """Tile-count flops per launch: per token and head 6 d_k d_v (W.S, Q.S,
+    K^T.Delta) + 6 C d_k (A, Q.K^T, W) + 4 C d_v (U, P.Delta)."""
+    return B * T * H * (6 * dk * dv + 6 * C * dk + 4 * C * dv)
+
+
+def decode_bytes(N, H, dk, dv, io_bytes=2):
+    """Algorithmic HBM bytes of one decode step: the fp32 state read and
+    written, q, k, v, o (io dtype), log_alpha (fp32), beta (fp32)."""
+    return N * H * (2 * dk * dv * 4 + (2 * dk + 2 * dv) * io_bytes + dk * 4 + 4)
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,"
+              "clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.samples = []
+        self.windows = []
+        self.proc = None
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", uuid, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.th = threading.Thread(target=self._read, daemon=True)
+            self.th.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), line.strip()))
+
+    def mark(self, t0, t1):
+        self.windows.append((t0, t1))
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sms, maxes, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        for t, line in self.samples:
+            if not any(a - 0.15 <= t <= b + 0.15 for a, b in self.windows):
+                continue
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sms.append(float(parts[0]))
+                maxes.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sms:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [],
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxes),
+                "reasons": sorted(reasons), "samples": len(sms)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group(
+            "nccl", timeout=datetime.timedelta(seconds=180),
+            device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def oracle_inputs(units):
+    """fp64 host inputs for `units` whole (sequence, head) units of the
+    prefill workload (one sequence of T tokens with `units` heads)."""
+    cfg = W.CONFIGS[PREFILL_CFG]
+    d = W.draw((1, cfg["T"]), units, cfg["dk"], cfg["dv"], io="bf16",
+               scale_q=True, device="cpu", seed=W.seed_of(PREFILL_CFG))
+    return [d[n].double().numpy() for n in ("q", "k", "v", "log_alpha", "beta")]
+
+
+def oracle_time(args_, min_seconds):
+    """Run the fp64 CPU oracle on prepared inputs until `min_seconds` have
+    passed (at least once); returns (token-heads, seconds)."""
+    from oracle import kda_oracle
+    units, T = args_[0].shape[2], args_[0].shape[1]
+    done, t0 = 0, time.perf_counter()
+    while True:
+        kda_oracle.recurrent(*args_)
+        done += units * T
+        el = time.perf_counter() - t0
+        if el >= min_seconds:
+            return done, el
+
+
+def run_reference(args, world, rank):
+    """The reference arm: the fp64 CPU oracle as it stands, on host cores."""
+    if rank != 0:
+        return
+    from oracle import kda_oracle
+    cfg = W.CONFIGS[PREFILL_CFG]
+    T, H = cfg["T"], cfg["H"]
+    threads = kda_oracle.num_threads()
+    units = max(1, threads)
+    inp = oracle_inputs(units)
+    for _ in range(args.warmup):
+        oracle_time(inp, 0.0)
+    total, el = 0, 0.0
+    for _ in range(args.steps):
+        n, t = oracle_time(inp, 0.0)
+        total += n
+        el += t
+    value = total / el / H
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value,
+        "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * el / max(1, args.steps),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"prefill T={T} H={H} d_k=d_v={cfg['dk']} "
+                   "(each step: a bounded sample of whole (sequence, head) "
+                   "units; tokens/s = token-heads/s / H)",
+                   "sample_units_per_step": units},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads,
+                         "kind": "oracle",
+                         "sample": f"{units} (sequence, head) units of {T} "
+                                   f"tokens per step, {args.steps} steps"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def timed(fn, steps, stream):
+    """Run fn() `steps` times between CUDA events recorded on `stream`;
+    returns (total ms, per-step ms list)."""
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    ev[0].record(stream)
+    for i in range(steps):
+        fn(i)
+        ev[i + 1].record(stream)
+    ev[-1].synchronize()
+    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(steps)]
+    return ev[0].elapsed_time(ev[-1]), per
+
+
+def run_kda(args, world, rank, local):
+    from gated_delta_rule_156_b200 import build as kbuild
+    from gated_delta_rule_156_b200 import kda as K
+    kbuild.build()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    pk, pk_kind = peaks()
+    clocks = Clocks(dev)
+
+    # ---- prefill -------------------------------------------------------
+    cfg = W.CONFIGS[PREFILL_CFG]
+    B, T, H, dk, dv, C = cfg["B"], cfg["T"], cfg["H"], cfg["dk"], cfg["dv"], \
+        cfg["chunk"]
+    d = W.make(PREFILL_CFG, device=dev, seed=W.seed_of(PREFILL_CFG) + 97 * rank)
+    out = torch.empty((B, T, H, dv), dtype=torch.bfloat16, device=dev)
+    fin = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+
+    def prefill(_i):
+        K.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], None,
+                    None, chunk=C, out=out, final_state=fin)
+
+    for i in range(args.warmup):
+        prefill(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = time.time()
+    ms, per = timed(prefill, args.steps, stream)
+    torch.cuda.synchronize()
+    clocks.mark(t0, time.time())
+    barrier(world)
+    ms = max_over_ranks(ms, world)
+    ms_step = ms / args.steps
+    launch_ms = statistics.mean(per)
+    n_kernels = K.chunk_fwd_kernel_count(B, T, H, dk, dv, C, torch.bfloat16,
+                                         packed=False)
+    value = world * B * T / (ms_step * 1e-3)
+    pbytes = prefill_bytes(B, T, H, dk, dv)
+    pflops = prefill_flops(B, T, H, dk, dv, C)
+    achieved_gbs = pbytes / (launch_ms * 1e-3) / 1e9
+    achieved_tf = pflops / (launch_ms * 1e-3) / 1e12
+
+    # ---- decode --------------------------------------------------------
+    dc = W.CONFIGS[DECODE_CFG]
+    dd = W.make(DECODE_CFG, device=dev, seed=W.seed_of(DECODE_CFG) + 97 * rank)
+    state = dd["initial_state"]
+    S = dc["steps"]
+    steps_in = [tuple(dd[n][s][:, None] for n in
+                      ("q", "k", "v", "log_alpha", "beta")) for s in range(S)]
+    dout = torch.empty((dc["N"], 1, dc["H"], dc["dv"]), dtype=torch.bfloat16,
+                       device=dev)
+
+    def decode(i):
+        q, k, v, la, b = steps_in[i % S]
+        K.recurrent_step(q, k, v, la, b, state, out=dout)
+
+    for i in range(args.warmup):
+        decode(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = time.time()
+    dms, dper = timed(decode, args.steps, stream)
+    torch.cuda.synchronize()
+    clocks.mark(t0, time.time())
+    barrier(world)
+    dms = max_over_ranks(dms, world)
+    dbytes = decode_bytes(dc["N"], dc["H"], dc["dk"], dc["dv"])
+    d_step_ms = dms / args.steps
+    d_gbs = world * dbytes / (d_step_ms * 1e-3) / 1e9
+    d_launch_gbs = dbytes / (statistics.mean(dper) * 1e-3) / 1e9
+
+    # ---- end to end through the public API with host buffers ------------
+    host = {n: d[n].cpu().pin_memory() for n in
+            ("q", "k", "v", "log_alpha", "beta")}
+    dev_in = {n: torch.empty_like(d[n]) for n in host}
+    out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    fin_h = torch.empty(fin.shape, dtype=fin.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_h.numel() * out_h.element_size() + fin_h.numel() * fin_h.element_size()
+
+    def e2e(_i):
+        for n, t in host.items():
+            dev_in[n].copy_(t, non_blocking=True)
+        K.chunk_fwd(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["log_alpha"],
+                    dev_in["beta"], None, None, chunk=C, out=out,
+                    final_state=fin)
+        out_h.copy_(out, non_blocking=True)
+        fin_h.copy_(fin, non_blocking=True)
+
+    e2e_steps = max(1, min(args.steps, 10))
+    for i in range(min(args.warmup, 3)):
+        e2e(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    ems, _ = timed(e2e, e2e_steps, stream)
+    barrier(world)
+    ems = max_over_ranks(ems, world)
+    e2e_value = world * B * T / (ems / e2e_steps * 1e-3)
+
+    clk = clocks.stop()
+
+    # ---- CPU baseline (rank 0, N = 1 only) ------------------------------
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from oracle import kda_oracle
+        threads = kda_oracle.num_threads()
+        units = max(1, threads)
+        n, el = oracle_time(oracle_inputs(units), args.cpu_seconds)
+        cpu = {"value": n / el / H, "unit": "tokens/s", "cores": threads,
+               "kind": "oracle",
+               "sample": f"{n // T} whole (sequence, head) units of {T} tokens "
+                         f"(d_k=d_v={dk}) of the prefill workload in {el:.1f} s "
+                         f"on {threads} threads; tokens/s = token-heads/s / "
+                         f"H={H}"}
+
+    traffic = load_traffic()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {
+                "workload": f"kda_chunk_fwd prefill B={B} T={T} H={H} "
+                            f"d_k=d_v={dk} C={C} bf16 (Kimi-Linear-shaped "
+                            "layer), zero initial state",
+                "global_batch": B * world, "seq_len": T,
+                "parallelism": f"dp{world} (independent replicas)",
+                "l2": "inputs larger than L2 (no flush)",
+                "path": K.chunk_fwd_path(B, T, H, dk, dv, C, torch.bfloat16),
+            },
+            "tensor_peak_frac": achieved_tf / pk["bf16_tflops"],
+            "roofline": {
+                "bound": "hbm", "achieved": achieved_gbs,
+                "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved_gbs / pk["hbm_gbs"],
+                "traffic": traffic.get("prefill"),
+                "peak_source": pk_kind,
+                "algorithmic_bytes_per_launch": pbytes,
+                "launch_ms": launch_ms,
+                "tensor": {"achieved": achieved_tf, "peak": pk["bf16_tflops"],
+                           "unit": "TFLOP/s",
+                           "frac": achieved_tf / pk["bf16_tflops"],
+                           "flops_per_launch": pflops,
+                           "count": "tile (full CxC tiles)"},
+            },
+            "decode": {
+                "metric": "decode GB/s vs HBM", "value": d_gbs, "unit": "GB/s",
+                "us_per_step": d_step_ms * 1e3,
+                "workload": f"kda_recurrent_step N={dc['N']} H={dc['H']} "
+                            f"d={dc['dk']} bf16 io, fp32 state in place",
+                "roofline": {"bound": "hbm", "achieved": d_launch_gbs,
+                             "peak": pk["hbm_gbs"], "unit": "GB/s",
+                             "frac": d_launch_gbs / pk["hbm_gbs"],
+                             "traffic": traffic.get("decode"),
+                             "algorithmic_bytes_per_launch": dbytes},
+                "gpu_launches": args.steps,
+            },
+            "e2e": {"value": e2e_value, "unit": "tokens/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": e2e_steps},
+            "gpu_launches": n_kernels * args.steps,
+            "clocks": clk,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def load_traffic():
+    """Per-launch DRAM bytes from the committed ncu summaries, when the
+    kernels have not changed since (a small JSON beside the summaries)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return {}
+    try:
+        with open(p) as f:
+            return json.load(f)
+    except Exception:
+        return {}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["kda", "reference"], default="kda")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.impl == "reference":
+        run_reference(args, world, int(os.environ.get("RANK", "0")))
+        return
+    world, rank, local = dist_setup()
+    try:
+        run_kda(args, world, rank, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

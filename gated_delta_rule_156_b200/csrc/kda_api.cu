@@ -1,0 +1,251 @@
+// C-ABI boundary of libkda.so: argument validation, workspace, dispatch.
+// Every argument error is found here, on the host, before anything launches.
+#include <stdint.h>
+#include <string.h>
+
+#include <atomic>
+
+#include "../../include/kda.h"
+#include "kda_internal.h"
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+kda_status cuda_fail(cudaError_t e) {
+  g_last_cuda_error = (int)e;
+  return KDA_ERR_CUDA;
+}
+
+bool supported_dim(int d) { return d == 32 || d == 64 || d == 128; }
+bool supported_chunk(int c) { return c == 16 || c == 32 || c == 64; }
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+struct Range {
+  uintptr_t lo, hi;
+};
+Range span(const void* p, size_t bytes) {
+  return Range{(uintptr_t)p, (uintptr_t)p + bytes};
+}
+bool overlap(Range a, Range b) {
+  return a.lo != 0 && b.lo != 0 && a.lo < b.hi && b.lo < a.hi && a.hi > a.lo &&
+         b.hi > b.lo;
+}
+
+// Keep freed stream-ordered workspace in the device's pool instead of handing
+// it back to the driver at every synchronisation.
+void keep_pool_memory() {
+  static std::atomic<uint64_t> done_mask{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return;
+  const uint64_t bit = 1ull << dev;
+  if (done_mask.load() & bit) return;
+  cudaMemPool_t pool;
+  if (cudaDeviceGetDefaultMemPool(&pool, dev) == cudaSuccess) {
+    uint64_t thr = UINT64_MAX;
+    cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &thr);
+  }
+  done_mask.fetch_or(bit);
+}
+
+// Shape-only checks shared by the launch entry points and the planner.
+kda_status validate_chunk_shape(const kda_shape* s, bool packed, int* n_seqs) {
+  if (!s) return KDA_ERR_INVALID_ARG;
+  if (s->B < 0 || s->T < 0 || s->H < 1) return KDA_ERR_INVALID_ARG;
+  if (s->io_dtype != KDA_BF16 && s->io_dtype != KDA_F32)
+    return KDA_ERR_INVALID_ARG;
+  if (!supported_dim(s->dk) || !supported_dim(s->dv)) return KDA_ERR_UNSUPPORTED;
+  if (!supported_chunk(s->chunk)) return KDA_ERR_UNSUPPORTED;
+  *n_seqs = s->B;
+  if (packed) {
+    if (s->B != 1 || s->n_seqs < 1) return KDA_ERR_INVALID_ARG;
+    *n_seqs = s->n_seqs;
+  }
+  if ((size_t)s->B * (size_t)s->T > (size_t)INT32_MAX ||
+      (size_t)*n_seqs * (size_t)s->H > (size_t)INT32_MAX || s->H > 65535)
+    return KDA_ERR_UNSUPPORTED;
+  return KDA_OK;
+}
+
+void fill_args(const kda_shape* s, int n_seqs, kda::ChunkArgs* a) {
+  a->n_seqs = n_seqs;
+  a->T = s->T;
+  a->H = s->H;
+  a->dk = s->dk;
+  a->dv = s->dv;
+  a->chunk = s->chunk;
+  a->bf16 = s->io_dtype == KDA_BF16;
+}
+
+kda_status validate_chunk(const kda_shape* s, const void* q, const void* k,
+                          const void* v, const float* la, const float* beta,
+                          const float* s_init, const int32_t* cu, void* out,
+                          float* s_final, kda::ChunkArgs* a) {
+  int n_seqs = 0;
+  const kda_status st = validate_chunk_shape(s, cu != nullptr, &n_seqs);
+  if (st != KDA_OK) return st;
+  const size_t esz = s->io_dtype == KDA_BF16 ? 2 : 4;
+  const size_t tokens = (size_t)s->B * (size_t)s->T;
+  const size_t H = s->H;
+  const bool any_tokens = tokens > 0;
+  const bool any_state = n_seqs > 0;
+  if (any_tokens && (!q || !k || !v || !la || !beta || !out))
+    return KDA_ERR_INVALID_ARG;
+  if (any_state && !s_final) return KDA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, la, beta, s_init, cu, out, s_final};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
+  // The output may alias no input; the final state may only coincide exactly
+  // with the initial state (in-place update).
+  const Range rq = span(q, tokens * H * s->dk * esz),
+              rk = span(k, tokens * H * s->dk * esz),
+              rv = span(v, tokens * H * s->dv * esz),
+              rl = span(la, tokens * H * s->dk * 4),
+              rb = span(beta, tokens * H * 4),
+              ro = span(out, tokens * H * s->dv * esz),
+              rsi = span(s_init, (size_t)n_seqs * H * s->dk * s->dv * 4),
+              rsf = span(s_final, (size_t)n_seqs * H * s->dk * s->dv * 4),
+              rc = span(cu, cu ? 4 * ((size_t)n_seqs + 1) : 0);
+  for (Range r : {rq, rk, rv, rl, rb, rsi, rsf, rc})
+    if (any_tokens && overlap(ro, r)) return KDA_ERR_INVALID_ARG;
+  for (Range r : {rq, rk, rv, rl, rb, rc})
+    if (any_state && overlap(rsf, r)) return KDA_ERR_INVALID_ARG;
+  if (s_init && overlap(rsf, rsi) && s_init != s_final) return KDA_ERR_INVALID_ARG;
+
+  a->q = q;
+  a->k = k;
+  a->v = v;
+  a->log_alpha = la;
+  a->beta = beta;
+  a->initial_state = s_init;
+  a->cu_seqlens = cu;
+  a->out = out;
+  a->final_state = s_final;
+  fill_args(s, n_seqs, a);
+  return KDA_OK;
+}
+
+kda_status run_with_workspace(size_t bytes, cudaStream_t stream, bool fused,
+                              const kda::ChunkArgs& a) {
+  void* ws = nullptr;
+  cudaError_t e;
+  if (bytes) {
+    keep_pool_memory();
+    if ((e = cudaMallocAsync(&ws, bytes, stream)) != cudaSuccess)
+      return cuda_fail(e);
+  }
+  e = fused ? kda::launch_fused(a, ws, stream)
+            : kda::launch_staged(a, ws, stream);
+  if (ws) {
+    const cudaError_t f = cudaFreeAsync(ws, stream);
+    if (e == cudaSuccess) e = f;
+  }
+  return e == cudaSuccess ? KDA_OK : cuda_fail(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+kda_status kda_chunk_fwd(const kda_shape* shape, const void* q, const void* k,
+                         const void* v, const float* log_alpha,
+                         const float* beta, const float* initial_state,
+                         const int32_t* cu_seqlens, void* out,
+                         float* final_state, cudaStream_t stream) {
+  kda::ChunkArgs a{};
+  const kda_status st = validate_chunk(shape, q, k, v, log_alpha, beta,
+                                       initial_state, cu_seqlens, out,
+                                       final_state, &a);
+  if (st != KDA_OK) return st;
+  if (kda::fused_supported(a))
+    return run_with_workspace(kda::fused_workspace_bytes(a), stream, true, a);
+  return run_with_workspace(kda::staged_workspace_bytes(a), stream, false, a);
+}
+
+kda_status kda_chunk_fwd_staged(const kda_shape* shape, const void* q,
+                                const void* k, const void* v,
+                                const float* log_alpha, const float* beta,
+                                const float* initial_state,
+                                const int32_t* cu_seqlens, void* out,
+                                float* final_state, cudaStream_t stream) {
+  kda::ChunkArgs a{};
+  const kda_status st = validate_chunk(shape, q, k, v, log_alpha, beta,
+                                       initial_state, cu_seqlens, out,
+                                       final_state, &a);
+  if (st != KDA_OK) return st;
+  return run_with_workspace(kda::staged_workspace_bytes(a), stream, false, a);
+}
+
+kda_status kda_recurrent_step(const kda_shape* s, const void* q, const void* k,
+                              const void* v, const float* log_alpha,
+                              const float* beta, float* state_inout, void* out,
+                              cudaStream_t stream) {
+  if (!s) return KDA_ERR_INVALID_ARG;
+  if (s->B < 0 || s->T < 0 || s->H < 1) return KDA_ERR_INVALID_ARG;
+  if (s->io_dtype != KDA_BF16 && s->io_dtype != KDA_F32)
+    return KDA_ERR_INVALID_ARG;
+  if (!supported_dim(s->dk) || !supported_dim(s->dv)) return KDA_ERR_UNSUPPORTED;
+  const size_t esz = s->io_dtype == KDA_BF16 ? 2 : 4;
+  const size_t tokens = (size_t)s->B * (size_t)s->T, H = s->H;
+  if ((size_t)s->B * H > (size_t)INT32_MAX) return KDA_ERR_UNSUPPORTED;
+  if (s->B > 0 && !state_inout) return KDA_ERR_INVALID_ARG;
+  if (tokens > 0 && (!q || !k || !v || !log_alpha || !beta || !out))
+    return KDA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, log_alpha, beta, state_inout, out};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
+  const Range rq = span(q, tokens * H * s->dk * esz),
+              rk = span(k, tokens * H * s->dk * esz),
+              rv = span(v, tokens * H * s->dv * esz),
+              rl = span(log_alpha, tokens * H * s->dk * 4),
+              rb = span(beta, tokens * H * 4),
+              ro = span(out, tokens * H * s->dv * esz),
+              rs = span(state_inout, (size_t)s->B * H * s->dk * s->dv * 4);
+  for (Range r : {rq, rk, rv, rl, rb, rs})
+    if (tokens > 0 && overlap(ro, r)) return KDA_ERR_INVALID_ARG;
+  for (Range r : {rq, rk, rv, rl, rb})
+    if (s->B > 0 && overlap(rs, r)) return KDA_ERR_INVALID_ARG;
+
+  kda::RecurrentArgs a{q, k, v, log_alpha, beta, state_inout, out,
+                       s->B, s->T, s->H, s->dk, s->dv,
+                       s->io_dtype == KDA_BF16};
+  const cudaError_t e = kda::launch_recurrent(a, stream);
+  return e == cudaSuccess ? KDA_OK : cuda_fail(e);
+}
+
+kda_status kda_chunk_fwd_plan(const kda_shape* shape, int packed, int staged,
+                              int* path, int* kernels,
+                              size_t* workspace_bytes) {
+  int n_seqs = 0;
+  const kda_status st = validate_chunk_shape(shape, packed != 0, &n_seqs);
+  if (st != KDA_OK) return st;
+  kda::ChunkArgs a{};
+  fill_args(shape, n_seqs, &a);
+  a.cu_seqlens = packed ? reinterpret_cast<const int32_t*>(16) : nullptr;
+  const bool fused = !staged && kda::fused_supported(a);
+  if (path) *path = fused ? 1 : 0;
+  if (kernels) *kernels = fused ? kda::fused_kernel_count(a)
+                                : kda::staged_kernel_count(a);
+  if (workspace_bytes)
+    *workspace_bytes = fused ? kda::fused_workspace_bytes(a)
+                             : kda::staged_workspace_bytes(a);
+  return KDA_OK;
+}
+
+const char* kda_status_string(kda_status status) {
+  switch (status) {
+    case KDA_OK: return "KDA_OK";
+    case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG: invalid argument";
+    case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED: unsupported size";
+    case KDA_ERR_MISALIGNED: return "KDA_ERR_MISALIGNED: pointer not 16-byte aligned";
+    case KDA_ERR_CUDA: return "KDA_ERR_CUDA: a CUDA call failed";
+    case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT: a bounded device wait gave up";
+  }
+  return "unknown kda_status";
+}
+
+int kda_last_cuda_error(void) { return g_last_cuda_error; }
+
+int kda_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,66 @@
+// Internal launch interface between the C-ABI layer (kda_api.cu) and the
+// kernel files.  Not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace kda {
+
+struct RecurrentArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* log_alpha;
+  const float* beta;
+  float* state;
+  void* out;
+  int B, T, H, dk, dv;
+  bool bf16;
+};
+
+struct ChunkArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* log_alpha;
+  const float* beta;
+  const float* initial_state;  // may be null
+  const int32_t* cu_seqlens;   // may be null (dense layout)
+  void* out;
+  float* final_state;
+  int n_seqs;  // B for the dense layout
+  int T;       // tokens per sequence (dense) or total tokens (packed)
+  int H, dk, dv, chunk;
+  bool bf16;
+};
+
+// Token-by-token evaluation (kda_decode.cu).
+cudaError_t launch_recurrent(const RecurrentArgs& a, cudaStream_t stream);
+
+// Four-stage fp32 pipeline (kda_staged.cu).  `workspace` must hold
+// staged_workspace_bytes(a) bytes, 256-byte aligned.
+size_t staged_workspace_bytes(const ChunkArgs& a);
+int staged_kernel_count(const ChunkArgs& a);
+cudaError_t launch_staged(const ChunkArgs& a, void* workspace,
+                          cudaStream_t stream);
+
+// Fused tensor-core prefill (kda_fused_sm100.cu): bf16 io, dk, dv in
+// {64, 128}, chunk 64.  `workspace` must hold fused_workspace_bytes(a).
+bool fused_supported(const ChunkArgs& a);
+size_t fused_workspace_bytes(const ChunkArgs& a);
+int fused_kernel_count(const ChunkArgs& a);
+cudaError_t launch_fused(const ChunkArgs& a, void* workspace,
+                         cudaStream_t stream);
+
+// Upper bound on the number of chunks of a request (packed sequences may each
+// add one partial chunk).
+inline int64_t max_chunks(const ChunkArgs& a) {
+  const int64_t C = a.chunk;
+  if (a.cu_seqlens == nullptr)
+    return (int64_t)a.n_seqs * ((a.T + C - 1) / C);
+  return (a.T + C - 1) / C + a.n_seqs;
+}
+
+}  // namespace kda

@@ -1,0 +1,393 @@
+// Four-stage chunkwise KDA forward, all arithmetic in fp32 (SIMT).
+//
+// The recurrence S_t = (I - b_t k_t k_t^T) Diag(a_t) S_{t-1} + b_t k_t v_t^T,
+// o_t = S_t^T q_t, regrouped over chunks of C tokens (the chunkwise form that
+// turns the recurrence into matrix products, "You Could Have Come Up with Kimi
+// Delta Attention", daily.dev, Summary; the Diagonal-Plus-Low-Rank transition
+// of "Kimi Delta Attention", akshathtiwari.co.in).  Inside a chunk with start
+// state S_0 and positions r = 1..C:
+//   g_r  = sum_{i<=r} l_i                          (1) cumulative log-decay
+//   Kt   = k * exp(g), Kb = k * exp(-g), Qt = q * exp(g), Kh = k * exp(g_C - g)
+//   A    = strictly_lower(Diag(b) Kt Kb^T)         (2) intra-chunk factors
+//   Tm   = (I + A)^-1                              forward substitution
+//   W    = Tm Diag(b) Kt,  U = Tm Diag(b) V
+//   D    = U - W S_0                               (3) state pass (serial)
+//   S_C  = Diag(exp(g_C)) S_0 + Kh^T D
+//   O    = Qt S_0 + lower_incl(Qt Kb^T) D           (4) output
+// Each stage is its own kernel with its inputs and outputs in an HBM
+// workspace; stages (1), (2), (4) are parallel over (chunk, head), stage (3)
+// over (sequence, head, 32-column tile of d_v).  This is the all-fp32 mode and
+// the reference decomposition the fused tensor-core kernel is built from.
+#include "kda_common.cuh"
+#include "kda_internal.h"
+
+namespace kda {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kDvTile = 32;
+
+struct Ws {
+  int32_t* chunk_off;  // [n_seqs + 1] (packed layout only)
+  float* g;            // [tokens, H, dk]   cumulative log-decay within chunk
+  float* w;            // [tokens, H, dk]   W rows
+  float* u;            // [tokens, H, dv]   U rows, overwritten by D
+  float* s;            // [max_chunks, H, dk, dv]  chunk-start states
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+Ws carve(const ChunkArgs& a, void* base, size_t* total) {
+  const size_t tokens =
+      a.cu_seqlens ? (size_t)a.T : (size_t)a.n_seqs * (size_t)a.T;
+  const size_t H = a.H;
+  size_t off = 0;
+  Ws w{};
+  char* p = static_cast<char*>(base);
+  auto take = [&](size_t bytes) {
+    char* r = p ? p + off : nullptr;
+    off = align256(off + bytes);
+    return r;
+  };
+  w.chunk_off = reinterpret_cast<int32_t*>(take(4 * (size_t)(a.n_seqs + 1)));
+  w.g = reinterpret_cast<float*>(take(4 * tokens * H * a.dk));
+  w.w = reinterpret_cast<float*>(take(4 * tokens * H * a.dk));
+  w.u = reinterpret_cast<float*>(take(4 * tokens * H * a.dv));
+  w.s = reinterpret_cast<float*>(
+      take(4 * (size_t)max_chunks(a) * H * a.dk * a.dv));
+  if (total) *total = off;
+  return w;
+}
+
+// Packed layout: exclusive prefix sum of ceil(len_s / C) per sequence.
+__global__ void plan_kernel(const int32_t* __restrict__ cu, int n_seqs, int T,
+                            int C, int32_t* __restrict__ chunk_off) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  int acc = 0;
+  chunk_off[0] = 0;
+  for (int s = 0; s < n_seqs; ++s) {
+    int a, b;
+    seq_range(cu, s, T, &a, &b);
+    acc += (b - a + C - 1) / C;
+    chunk_off[s + 1] = acc;
+  }
+}
+
+// (1) g_r = sum_{i<=r} l_i within the chunk; one thread per key channel.
+__global__ void cumsum_kernel(const float* __restrict__ la, float* __restrict__ g,
+                              const int32_t* cu, const int32_t* chunk_off,
+                              int n_seqs, int T, int H, int dk, int C) {
+  int seq, tok0, L;
+  if (!locate_chunk(blockIdx.x, cu, chunk_off, n_seqs, T, C, &seq, &tok0, &L))
+    return;
+  const int h = blockIdx.y;
+  for (int c = threadIdx.x; c < dk; c += blockDim.x) {
+    float acc = 0.f;
+    for (int r = 0; r < L; ++r) {
+      const size_t idx = ((size_t)(tok0 + r) * H + h) * dk + c;
+      acc += la[idx];
+      g[idx] = acc;
+    }
+  }
+}
+
+// (2) A, Tm = (I + A)^-1, W = Tm Diag(b) Kt, U = Tm Diag(b) V.
+template <typename IO>
+__global__ void __launch_bounds__(kThreads)
+    intra_kernel(const IO* __restrict__ k, const IO* __restrict__ v,
+                 const float* __restrict__ beta, const float* __restrict__ g,
+                 float* __restrict__ w_out, float* __restrict__ u_out,
+                 const int32_t* cu, const int32_t* chunk_off, int n_seqs, int T,
+                 int H, int dk, int dv, int C) {
+  int seq, tok0, L;
+  if (!locate_chunk(blockIdx.x, cu, chunk_off, n_seqs, T, C, &seq, &tok0, &L))
+    return;
+  const int h = blockIdx.y, tid = threadIdx.x;
+  extern __shared__ float sm[];
+  float* Kt = sm;              // [C][dk]
+  float* Kb = Kt + C * dk;     // [C][dk]
+  float* V = Kb + C * dk;      // [C][dv]
+  float* A = V + C * dv;       // [C][C]
+  float* Tm = A + C * C;       // [C][C]
+  float* bs = Tm + C * C;      // [C]
+
+  for (int idx = tid; idx < C * dk; idx += kThreads) {
+    const int r = idx / dk, c = idx % dk;
+    float kt = 0.f, kb = 0.f;
+    if (r < L) {
+      const size_t gi = ((size_t)(tok0 + r) * H + h) * dk + c;
+      const float kv = to_f32(k[gi]), gv = g[gi];
+      kt = kv * __expf(gv);
+      kb = kv * __expf(-gv);
+    }
+    Kt[idx] = kt;
+    Kb[idx] = kb;
+  }
+  for (int idx = tid; idx < C * dv; idx += kThreads) {
+    const int r = idx / dv, j = idx % dv;
+    V[idx] = r < L ? to_f32(v[((size_t)(tok0 + r) * H + h) * dv + j]) : 0.f;
+  }
+  for (int r = tid; r < C; r += kThreads)
+    bs[r] = r < L ? beta[(size_t)(tok0 + r) * H + h] : 0.f;
+  __syncthreads();
+
+  for (int idx = tid; idx < C * C; idx += kThreads) {
+    const int r = idx / C, i = idx % C;
+    float acc = 0.f;
+    if (i < r) {
+      for (int c = 0; c < dk; ++c) acc += Kt[r * dk + c] * Kb[i * dk + c];
+      acc *= bs[r];
+    }
+    A[idx] = acc;
+  }
+  __syncthreads();
+
+  // Forward substitution, one column of Tm per thread:
+  // Tm[r][j] = [r == j] - sum_{j<=i<r} A[r][i] Tm[i][j].
+  for (int j = tid; j < C; j += kThreads) {
+    for (int r = 0; r < C; ++r) {
+      float t;
+      if (r < j) {
+        t = 0.f;
+      } else if (r == j) {
+        t = 1.f;
+      } else {
+        t = 0.f;
+        for (int i = j; i < r; ++i) t -= A[r * C + i] * Tm[i * C + j];
+      }
+      Tm[r * C + j] = t;
+    }
+  }
+  __syncthreads();
+
+  for (int idx = tid; idx < L * dk; idx += kThreads) {
+    const int r = idx / dk, c = idx % dk;
+    float acc = 0.f;
+    for (int i = 0; i <= r; ++i) acc += Tm[r * C + i] * bs[i] * Kt[i * dk + c];
+    w_out[((size_t)(tok0 + r) * H + h) * dk + c] = acc;
+  }
+  for (int idx = tid; idx < L * dv; idx += kThreads) {
+    const int r = idx / dv, j = idx % dv;
+    float acc = 0.f;
+    for (int i = 0; i <= r; ++i) acc += Tm[r * C + i] * bs[i] * V[i * dv + j];
+    u_out[((size_t)(tok0 + r) * H + h) * dv + j] = acc;
+  }
+}
+
+// (3) Sequential over the chunks of one sequence; one 32-column tile of S.
+//   D = U - W S ;  S <- Diag(exp(g_C)) S + Kh^T D.  Stores every chunk-start
+// state (for stage 4), D (over U), and the final state.
+template <typename IO>
+__global__ void __launch_bounds__(kThreads)
+    state_kernel(const IO* __restrict__ k, const float* __restrict__ g,
+                 const float* __restrict__ w, float* __restrict__ u,
+                 float* __restrict__ s_chunks,
+                 const float* __restrict__ s_init, float* __restrict__ s_final,
+                 const int32_t* cu, const int32_t* chunk_off, int n_seqs, int T,
+                 int H, int dk, int dv, int C) {
+  const int seq = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * kDvTile;
+  const int tid = threadIdx.x;
+  extern __shared__ float sm[];
+  float* S = sm;                  // [dk][kDvTile]
+  float* Wc = S + dk * kDvTile;   // [C][dk]
+  float* Kh = Wc + C * dk;        // [C][dk]
+  float* D = Kh + C * dk;         // [C][kDvTile]
+  float* gC = D + C * kDvTile;    // [dk]
+
+  const size_t sbase = ((size_t)seq * H + h) * dk * dv;
+  for (int idx = tid; idx < dk * kDvTile; idx += kThreads) {
+    const int c = idx / kDvTile, jj = idx % kDvTile;
+    S[idx] = s_init ? s_init[sbase + (size_t)c * dv + j0 + jj] : 0.f;
+  }
+  int start, end;
+  seq_range(cu, seq, T, &start, &end);
+  const int nch = (end - start + C - 1) / C;
+  const int cid0 = cu ? chunk_off[seq] : seq * ((T + C - 1) / C);
+  __syncthreads();
+
+  for (int ch = 0; ch < nch; ++ch) {
+    const int tok0 = start + ch * C, L = min(C, end - tok0);
+    const size_t cbase = ((size_t)(cid0 + ch) * H + h) * dk * dv;
+    for (int idx = tid; idx < dk * kDvTile; idx += kThreads) {
+      const int c = idx / kDvTile, jj = idx % kDvTile;
+      s_chunks[cbase + (size_t)c * dv + j0 + jj] = S[idx];
+    }
+    for (int c = tid; c < dk; c += kThreads)
+      gC[c] = g[((size_t)(tok0 + L - 1) * H + h) * dk + c];
+    __syncthreads();
+    for (int idx = tid; idx < C * dk; idx += kThreads) {
+      const int r = idx / dk, c = idx % dk;
+      float wv = 0.f, kh = 0.f;
+      if (r < L) {
+        const size_t gi = ((size_t)(tok0 + r) * H + h) * dk + c;
+        wv = w[gi];
+        kh = to_f32(k[gi]) * __expf(gC[c] - g[gi]);
+      }
+      Wc[idx] = wv;
+      Kh[idx] = kh;
+    }
+    for (int idx = tid; idx < C * kDvTile; idx += kThreads) {
+      const int r = idx / kDvTile, jj = idx % kDvTile;
+      D[idx] = r < L ? u[((size_t)(tok0 + r) * H + h) * dv + j0 + jj] : 0.f;
+    }
+    __syncthreads();
+    for (int idx = tid; idx < C * kDvTile; idx += kThreads) {
+      const int r = idx / kDvTile, jj = idx % kDvTile;
+      if (r < L) {
+        float acc = D[idx];
+        for (int c = 0; c < dk; ++c) acc -= Wc[r * dk + c] * S[c * kDvTile + jj];
+        D[idx] = acc;
+        u[((size_t)(tok0 + r) * H + h) * dv + j0 + jj] = acc;
+      }
+    }
+    __syncthreads();
+    for (int idx = tid; idx < dk * kDvTile; idx += kThreads) {
+      const int c = idx / kDvTile, jj = idx % kDvTile;
+      float acc = __expf(gC[c]) * S[idx];
+      for (int r = 0; r < L; ++r) acc += Kh[r * dk + c] * D[r * kDvTile + jj];
+      S[idx] = acc;
+    }
+    __syncthreads();
+  }
+  for (int idx = tid; idx < dk * kDvTile; idx += kThreads) {
+    const int c = idx / kDvTile, jj = idx % kDvTile;
+    s_final[sbase + (size_t)c * dv + j0 + jj] = S[idx];
+  }
+}
+
+// (4) O = Qt S_0 + lower_incl(Qt Kb^T) D, per chunk and 32-column tile.
+template <typename IO>
+__global__ void __launch_bounds__(kThreads)
+    output_kernel(const IO* __restrict__ q, const IO* __restrict__ k,
+                  const float* __restrict__ g, const float* __restrict__ d,
+                  const float* __restrict__ s_chunks, IO* __restrict__ out,
+                  const int32_t* cu, const int32_t* chunk_off, int n_seqs,
+                  int T, int H, int dk, int dv, int C) {
+  const int cid = blockIdx.x;
+  int seq, tok0, L;
+  if (!locate_chunk(cid, cu, chunk_off, n_seqs, T, C, &seq, &tok0, &L)) return;
+  const int h = blockIdx.y, j0 = blockIdx.z * kDvTile, tid = threadIdx.x;
+  extern __shared__ float sm[];
+  float* Qt = sm;                 // [C][dk]
+  float* Kb = Qt + C * dk;        // [C][dk]
+  float* P = Kb + C * dk;         // [C][C]
+  float* S = P + C * C;           // [dk][kDvTile]
+  float* D = S + dk * kDvTile;    // [C][kDvTile]
+
+  for (int idx = tid; idx < C * dk; idx += kThreads) {
+    const int r = idx / dk, c = idx % dk;
+    float qt = 0.f, kb = 0.f;
+    if (r < L) {
+      const size_t gi = ((size_t)(tok0 + r) * H + h) * dk + c;
+      const float gv = g[gi];
+      qt = to_f32(q[gi]) * __expf(gv);
+      kb = to_f32(k[gi]) * __expf(-gv);
+    }
+    Qt[idx] = qt;
+    Kb[idx] = kb;
+  }
+  const size_t cbase = ((size_t)cid * H + h) * dk * dv;
+  for (int idx = tid; idx < dk * kDvTile; idx += kThreads) {
+    const int c = idx / kDvTile, jj = idx % kDvTile;
+    S[idx] = s_chunks[cbase + (size_t)c * dv + j0 + jj];
+  }
+  for (int idx = tid; idx < C * kDvTile; idx += kThreads) {
+    const int r = idx / kDvTile, jj = idx % kDvTile;
+    D[idx] = r < L ? d[((size_t)(tok0 + r) * H + h) * dv + j0 + jj] : 0.f;
+  }
+  __syncthreads();
+  for (int idx = tid; idx < C * C; idx += kThreads) {
+    const int r = idx / C, i = idx % C;
+    float acc = 0.f;
+    if (i <= r)
+      for (int c = 0; c < dk; ++c) acc += Qt[r * dk + c] * Kb[i * dk + c];
+    P[idx] = acc;
+  }
+  __syncthreads();
+  for (int idx = tid; idx < L * kDvTile; idx += kThreads) {
+    const int r = idx / kDvTile, jj = idx % kDvTile;
+    float acc = 0.f;
+    for (int c = 0; c < dk; ++c) acc += Qt[r * dk + c] * S[c * kDvTile + jj];
+    for (int i = 0; i <= r; ++i) acc += P[r * C + i] * D[i * kDvTile + jj];
+    out[((size_t)(tok0 + r) * H + h) * dv + j0 + jj] = from_f32<IO>(acc);
+  }
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, size_t bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)bytes);
+}
+
+template <typename IO>
+cudaError_t run(const ChunkArgs& a, void* workspace, cudaStream_t stream) {
+  Ws w = carve(a, workspace, nullptr);
+  const int C = a.chunk, H = a.H, dk = a.dk, dv = a.dv;
+  const int64_t nch = max_chunks(a);
+  const int32_t* cu = a.cu_seqlens;
+  const IO* q = static_cast<const IO*>(a.q);
+  const IO* k = static_cast<const IO*>(a.k);
+  const IO* v = static_cast<const IO*>(a.v);
+  IO* out = static_cast<IO*>(a.out);
+  cudaError_t e;
+
+  if (cu) {
+    plan_kernel<<<1, 32, 0, stream>>>(cu, a.n_seqs, a.T, C, w.chunk_off);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if (nch > 0) {
+    const dim3 grid((unsigned)nch, H);
+    cumsum_kernel<<<grid, dk, 0, stream>>>(a.log_alpha, w.g, cu, w.chunk_off,
+                                          a.n_seqs, a.T, H, dk, C);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+    const size_t sm2 = 4 * ((size_t)2 * C * dk + (size_t)C * dv + 2 * C * C + C);
+    if ((e = set_smem(intra_kernel<IO>, sm2)) != cudaSuccess) return e;
+    intra_kernel<IO><<<grid, kThreads, sm2, stream>>>(
+        k, v, a.beta, w.g, w.w, w.u, cu, w.chunk_off, a.n_seqs, a.T, H, dk, dv,
+        C);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  const size_t sm3 =
+      4 * ((size_t)dk * kDvTile + 2 * (size_t)C * dk + C * kDvTile + dk);
+  if ((e = set_smem(state_kernel<IO>, sm3)) != cudaSuccess) return e;
+  state_kernel<IO><<<dim3(a.n_seqs, H, dv / kDvTile), kThreads, sm3, stream>>>(
+      k, w.g, w.w, w.u, w.s, a.initial_state, a.final_state, cu, w.chunk_off,
+      a.n_seqs, a.T, H, dk, dv, C);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+  if (nch > 0) {
+    const size_t sm4 = 4 * (2 * (size_t)C * dk + (size_t)C * C +
+                            (size_t)dk * kDvTile + (size_t)C * kDvTile);
+    if ((e = set_smem(output_kernel<IO>, sm4)) != cudaSuccess) return e;
+    output_kernel<IO><<<dim3((unsigned)nch, H, dv / kDvTile), kThreads, sm4,
+                        stream>>>(q, k, w.g, w.u, w.s, out, cu, w.chunk_off,
+                                  a.n_seqs, a.T, H, dk, dv, C);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace
+
+size_t staged_workspace_bytes(const ChunkArgs& a) {
+  size_t total = 0;
+  carve(a, nullptr, &total);
+  return total;
+}
+
+int staged_kernel_count(const ChunkArgs& a) {
+  if (a.n_seqs == 0) return 0;
+  const bool any_chunks = max_chunks(a) > 0;
+  return (a.cu_seqlens ? 1 : 0) + 1 + (any_chunks ? 3 : 0);
+}
+
+cudaError_t launch_staged(const ChunkArgs& a, void* workspace,
+                          cudaStream_t stream) {
+  if (a.n_seqs == 0 || a.H == 0) return cudaSuccess;
+  return a.bf16 ? run<__nv_bfloat16>(a, workspace, stream)
+                : run<float>(a, workspace, stream);
+}
+
+}  // namespace kda

@@ -1,0 +1,190 @@
+"""Thin Python binding of libkda.so (argument marshalling only).
+
+Every step of the forward pass runs in the library's CUDA kernels; torch only
+provides device memory and the current CUDA stream.  There is no fallback: if
+the library is missing or the tensors are not on a CUDA device the calls
+raise.
+"""
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+KDA_OK = 0
+KDA_BF16, KDA_F32 = 0, 1
+STATUS_NAMES = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED",
+                3: "KDA_ERR_MISALIGNED", 4: "KDA_ERR_CUDA", 5: "KDA_ERR_TIMEOUT"}
+
+# Entry points declared in include/kda.h (kept in sync by tests).
+EXPORTS = ("kda_chunk_fwd", "kda_chunk_fwd_staged", "kda_recurrent_step",
+           "kda_chunk_fwd_plan", "kda_status_string", "kda_last_cuda_error",
+           "kda_version")
+
+
+class KdaShape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int),
+                ("dk", ctypes.c_int), ("dv", ctypes.c_int),
+                ("chunk", ctypes.c_int), ("n_seqs", ctypes.c_int),
+                ("io_dtype", ctypes.c_int)]
+
+
+class KdaError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)} "
+                         f"({library().kda_status_string(status).decode()})"
+                         + (f" cuda error {library().kda_last_cuda_error()}"
+                            if status == 4 else ""))
+
+
+_lib = None
+
+
+def library_path():
+    return _build.LIB
+
+
+def library():
+    """The loaded libkda.so.  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        path = library_path()
+        if not os.path.exists(path):
+            raise RuntimeError(
+                f"libkda.so not found at {path}; build it with "
+                "`python -m gated_delta_rule_156_b200.build`")
+        lib = ctypes.CDLL(path)
+        vp, fp = ctypes.c_void_p, ctypes.c_void_p
+        chunk_args = [ctypes.POINTER(KdaShape), vp, vp, vp, fp, fp, fp, vp, vp,
+                      fp, vp]
+        for name in ("kda_chunk_fwd", "kda_chunk_fwd_staged"):
+            fn = getattr(lib, name)
+            fn.restype = ctypes.c_int
+            fn.argtypes = chunk_args
+        lib.kda_recurrent_step.restype = ctypes.c_int
+        lib.kda_recurrent_step.argtypes = [ctypes.POINTER(KdaShape), vp, vp, vp,
+                                           fp, fp, fp, vp, vp]
+        lib.kda_chunk_fwd_plan.restype = ctypes.c_int
+        lib.kda_chunk_fwd_plan.argtypes = [
+            ctypes.POINTER(KdaShape), ctypes.c_int, ctypes.c_int,
+            ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int),
+            ctypes.POINTER(ctypes.c_size_t)]
+        lib.kda_status_string.restype = ctypes.c_char_p
+        lib.kda_status_string.argtypes = [ctypes.c_int]
+        lib.kda_last_cuda_error.restype = ctypes.c_int
+        lib.kda_last_cuda_error.argtypes = []
+        lib.kda_version.restype = ctypes.c_int
+        lib.kda_version.argtypes = []
+        _lib = lib
+    return _lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _check_dev(name, t, dtype=None):
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor) or t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _io(q):
+    if q.dtype == torch.bfloat16:
+        return KDA_BF16
+    if q.dtype == torch.float32:
+        return KDA_F32
+    raise ValueError(f"unsupported io dtype {q.dtype}")
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
+              chunk=64, out=None, final_state=None, staged=False, stream=None):
+    """Chunkwise KDA forward (kda_chunk_fwd / kda_chunk_fwd_staged).
+
+    q, k [B, T, H, d_k]; v [B, T, H, d_v] (bf16 or fp32, same dtype);
+    log_alpha [B, T, H, d_k] fp32; beta [B, T, H] fp32; initial_state
+    [N, H, d_k, d_v] fp32 or None; cu_seqlens int32 [N + 1] or None (then
+    B == 1 and T is the packed total).  Returns (out, final_state).
+    """
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    n = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if final_state is None:
+        final_state = torch.empty((n, H, dk, dv), dtype=torch.float32,
+                                  device=q.device)
+    for name, t, dt in (("q", q, None), ("k", k, q.dtype), ("v", v, q.dtype),
+                        ("log_alpha", log_alpha, torch.float32),
+                        ("beta", beta, torch.float32),
+                        ("initial_state", initial_state, torch.float32),
+                        ("cu_seqlens", cu_seqlens, torch.int32),
+                        ("out", out, q.dtype),
+                        ("final_state", final_state, torch.float32)):
+        _check_dev(name, t, dt)
+    shape = KdaShape(B, T, H, dk, dv, chunk, n if cu_seqlens is not None else 0,
+                     _io(q))
+    fn = library().kda_chunk_fwd_staged if staged else library().kda_chunk_fwd
+    st = fn(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+            _ptr(beta), _ptr(initial_state), _ptr(cu_seqlens), _ptr(out),
+            _ptr(final_state), _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_chunk_fwd_staged" if staged else "kda_chunk_fwd")
+    return out, final_state
+
+
+def recurrent_step(q, k, v, log_alpha, beta, state, out=None, stream=None):
+    """Token-by-token KDA (kda_recurrent_step); ``state`` [B, H, d_k, d_v] fp32
+    is updated in place.  q, k [B, T, H, d_k] (T >= 1 tokens per sequence).
+    Returns out [B, T, H, d_v]."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    for name, t, dt in (("q", q, None), ("k", k, q.dtype), ("v", v, q.dtype),
+                        ("log_alpha", log_alpha, torch.float32),
+                        ("beta", beta, torch.float32),
+                        ("state", state, torch.float32), ("out", out, q.dtype)):
+        _check_dev(name, t, dt)
+    shape = KdaShape(B, T, H, dk, dv, 0, 0, _io(q))
+    st = library().kda_recurrent_step(
+        ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+        _ptr(beta), _ptr(state), _ptr(out), _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_recurrent_step")
+    return out
+
+
+def chunk_fwd_plan(B, T, H, dk, dv, chunk, dtype, packed=False, n_seqs=0,
+                   staged=False):
+    """(path, kernels, workspace_bytes) of a chunk_fwd call of this shape:
+    path is "fused" or "staged"; no device work is done."""
+    io = KDA_BF16 if dtype == torch.bfloat16 else KDA_F32
+    shape = KdaShape(B, T, H, dk, dv, chunk, n_seqs if packed else 0, io)
+    path, kern, ws = ctypes.c_int(), ctypes.c_int(), ctypes.c_size_t()
+    st = library().kda_chunk_fwd_plan(ctypes.byref(shape), int(packed),
+                                      int(staged), ctypes.byref(path),
+                                      ctypes.byref(kern), ctypes.byref(ws))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_chunk_fwd_plan")
+    return ("fused" if path.value == 1 else "staged"), kern.value, ws.value
+
+
+def chunk_fwd_kernel_count(B, T, H, dk, dv, chunk, dtype, packed=False):
+    return chunk_fwd_plan(B, T, H, dk, dv, chunk, dtype, packed, 1)[1]
+
+
+def chunk_fwd_path(B, T, H, dk, dv, chunk, dtype, packed=False):
+    return chunk_fwd_plan(B, T, H, dk, dv, chunk, dtype, packed, 1)[0]

@@ -1,0 +1,181 @@
+/*
+ * kda.h -- C ABI of the B200 (sm_100a) Kimi Delta Attention forward library.
+ *
+ * The operation (stated in this header's own words):
+ *   Per (sequence, head) a state S in R^{d_k x d_v} is carried across tokens.
+ *   For token t with query q_t, key k_t (in R^{d_k}), value v_t (in R^{d_v}),
+ *   write rate beta_t and per-key-channel forget vector alpha_t = exp(l_t):
+ *       S'  = Diag(alpha_t) S_{t-1}             decay each key channel (row)
+ *       S_t = S' + beta_t k_t (v_t - S'^T k_t)^T delta-rule write of the error
+ *       o_t = S_t^T q_t                          read with the query
+ *   i.e. S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T.
+ *   Sources: "Kimi Delta Attention" (akshathtiwari.co.in), the delta-rule and
+ *   channel-wise gating passages; "The fourth layer remembers"
+ *   (praveentn.live), section "What each kind of layer keeps"; "Teacher guide -
+ *   Kimi Delta Attention", section 12.1 and the Misconceptions table.
+ *   kda_chunk_fwd evaluates it chunkwise (the recurrence reorganised into
+ *   matrix products, "You Could Have Come Up with Kimi Delta Attention",
+ *   daily.dev, Summary); kda_recurrent_step evaluates it token by token with
+ *   constant memory and work per token ("The fourth layer remembers", the
+ *   paragraph after the forget gate).  Both give the same result up to
+ *   floating-point rounding.
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor pointers are DEVICE memory owned by the caller; the library
+ *     never frees or retains them.  Calls are asynchronous on `stream` and never
+ *     synchronise the host.  Temporary workspace, when a path needs it, is
+ *     stream-ordered (cudaMallocAsync / cudaFreeAsync on `stream`).
+ *   - Layouts are dense row-major:
+ *       q, k       [B, T, H, d_k]   io dtype (bf16 or fp32)
+ *       v, out     [B, T, H, d_v]   io dtype
+ *       log_alpha  [B, T, H, d_k]   fp32, l = log(alpha) <= 0 (no lower bound
+ *                                   is applied; the caller forms the gate)
+ *       beta       [B, T, H]        fp32
+ *       states     [N, H, d_k, d_v] fp32, N = B (or n_seqs with cu_seqlens)
+ *     q and k are used as given: any scaling or L2 normalisation is the
+ *     caller's.
+ *   - Every pointer must be 16-byte aligned (KDA_ERR_MISALIGNED otherwise).
+ *   - `out` must not alias an input.  Argument errors are detected on the host
+ *     before anything is launched; no exception crosses the ABI.
+ *   - Supported sizes: d_k, d_v in {32, 64, 128}; chunk in {16, 32, 64}.
+ *     Others return KDA_ERR_UNSUPPORTED.
+ *   - Numerical range: the chunkwise path factorises the decay inside a chunk,
+ *     which is exact for |sum of l over one chunk| up to about 80 per channel
+ *     (fp32 exponent range).  Gates stronger than that are not supported.
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define KDA_API __attribute__((visibility("default")))
+#else
+#define KDA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KDA_OK = 0,
+  KDA_ERR_INVALID_ARG = 1, /* null pointer, bad size, aliasing            */
+  KDA_ERR_UNSUPPORTED = 2, /* valid request outside the supported sizes    */
+  KDA_ERR_MISALIGNED = 3,  /* a pointer is not 16-byte aligned             */
+  KDA_ERR_CUDA = 4,        /* a CUDA call failed; see kda_last_cuda_error  */
+  KDA_ERR_TIMEOUT = 5      /* a bounded device-side wait gave up           */
+} kda_status;
+
+typedef enum { KDA_BF16 = 0, KDA_F32 = 1 } kda_dtype;
+
+typedef struct {
+  int B;      /* batch (number of sequences when cu_seqlens is NULL; 1 with it) */
+  int T;      /* tokens per sequence, or total packed tokens with cu_seqlens  */
+  int H;      /* heads                                                          */
+  int dk;     /* key / query head dimension                                     */
+  int dv;     /* value head dimension                                           */
+  int chunk;  /* chunk length C of the chunkwise evaluation (16, 32 or 64)      */
+  int n_seqs; /* number of packed sequences (used only with cu_seqlens)         */
+  kda_dtype io_dtype; /* dtype of q, k, v and out                               */
+} kda_shape;
+
+/*
+ * kda_chunk_fwd -- chunkwise prefill over whole sequences.
+ *
+ *   q, k, v, log_alpha, beta : inputs, layouts above.
+ *   initial_state : [N, H, d_k, d_v] fp32 start state, or NULL for zeros.
+ *   cu_seqlens    : NULL for the dense [B, T, ...] layout.  Otherwise int32
+ *                   device array of n_seqs + 1 token offsets into the packed
+ *                   token axis (B must be 1, T the total): sequence s owns tokens
+ *                   cu_seqlens[s] .. cu_seqlens[s+1]-1.  It must start at 0, be
+ *                   non-decreasing and end at T; it is device memory, so it is
+ *                   not checked on the host: the kernels clamp every offset into
+ *                   [0, T] (they stay in bounds), but results for a malformed
+ *                   array are unspecified.  Chunks never straddle sequences;
+ *                   a sequence's last chunk may be partial; empty sequences are
+ *                   allowed (their final state is their initial state).
+ *   out           : [B, T, H, d_v] io dtype, written.
+ *   final_state   : [N, H, d_k, d_v] fp32, written (may equal initial_state).
+ *
+ * bf16 inputs with d_k, d_v in {64, 128} and chunk = 64 run the fused
+ * tensor-core kernel; every other supported request runs the four-stage
+ * kernel pipeline of kda_chunk_fwd_staged.  fp32 state throughout.
+ */
+KDA_API kda_status kda_chunk_fwd(const kda_shape* shape, const void* q, const void* k,
+                         const void* v, const float* log_alpha,
+                         const float* beta, const float* initial_state,
+                         const int32_t* cu_seqlens, void* out,
+                         float* final_state, cudaStream_t stream);
+
+/*
+ * kda_chunk_fwd_staged -- same contract as kda_chunk_fwd, always evaluated as
+ * four kernels with an intermediate workspace in HBM:
+ *   (1) per-chunk cumulative log-decay g;  (2) intra-chunk factors: the
+ *   decay-scaled strictly-lower matrix A, T = (I + A)^-1 by forward
+ *   substitution, W = T Diag(beta) K~ and U = T Diag(beta) V;  (3) the
+ *   inter-chunk state pass, sequential over chunks, parallel over
+ *   (sequence, head, d_v tile);  (4) the output, q.S plus the masked
+ *   intra-chunk q.k^T term.  All arithmetic is fp32 (the all-fp32 mode).
+ * Workspace: about (2 d_k + d_v) * 4 bytes per token and head plus
+ * d_k * d_v * 4 bytes per chunk and head, allocated stream-ordered.
+ */
+KDA_API kda_status kda_chunk_fwd_staged(const kda_shape* shape, const void* q,
+                                const void* k, const void* v,
+                                const float* log_alpha, const float* beta,
+                                const float* initial_state,
+                                const int32_t* cu_seqlens, void* out,
+                                float* final_state, cudaStream_t stream);
+
+/*
+ * kda_recurrent_step -- token-by-token evaluation (decode).
+ *
+ *   shape->B  : number of independent sequences; shape->T : tokens per
+ *               sequence in this call (1 for one decode step; T > 1 runs T
+ *               steps with the state kept on chip); shape->chunk and n_seqs
+ *               are ignored; cu_seqlens is not supported here.
+ *   q, k, v, log_alpha, beta : [B, T, H, ...] as above.
+ *   state_inout : [B, H, d_k, d_v] fp32, read and overwritten in place.
+ *   out         : [B, T, H, d_v] io dtype.
+ * Streams each head's fp32 state through the SMs once per call.
+ */
+KDA_API kda_status kda_recurrent_step(const kda_shape* shape, const void* q,
+                              const void* k, const void* v,
+                              const float* log_alpha, const float* beta,
+                              float* state_inout, void* out,
+                              cudaStream_t stream);
+
+/*
+ * kda_chunk_fwd_plan -- how kda_chunk_fwd (staged = 0) or kda_chunk_fwd_staged
+ * (staged = 1) would evaluate a request of this shape; launches nothing and
+ * touches no device memory.
+ *   packed          : nonzero when cu_seqlens will be passed.
+ *   path            : out, 1 = fused tensor-core kernel, 0 = four-stage fp32
+ *                     pipeline (may be NULL).
+ *   kernels         : out, kernel launches one call makes (may be NULL).
+ *   workspace_bytes : out, stream-ordered workspace one call allocates (may be
+ *                     NULL).
+ * Returns KDA_OK, or the status the call itself would return for this shape.
+ */
+KDA_API kda_status kda_chunk_fwd_plan(const kda_shape* shape, int packed,
+                                      int staged, int* path, int* kernels,
+                                      size_t* workspace_bytes);
+
+/* Human-readable name of a status code (static string, never NULL). */
+KDA_API const char* kda_status_string(kda_status status);
+
+/* The cudaError_t value behind the most recent KDA_ERR_CUDA on this thread
+ * (0 if none). */
+KDA_API int kda_last_cuda_error(void);
+
+/* Library version as major * 10000 + minor * 100 + patch. */
+KDA_API int kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

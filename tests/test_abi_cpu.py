@@ -1,0 +1,106 @@
+"""The C-ABI library on the host: it loads without a GPU, exports every entry
+point include/*.h declares, and rejects bad arguments before launching
+anything (no compute call is made here)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from gated_delta_rule_156_b200 import build as kbuild
+from gated_delta_rule_156_b200 import kda as K
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    kbuild.build()
+    return K.library()
+
+
+def declared_entry_points():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        names += re.findall(r"KDA_API\s+[\w\s\*]+?\b(kda_\w+)\s*\(", src)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_entry_points()
+    assert "kda_chunk_fwd" in names and "kda_recurrent_step" in names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(K.EXPORTS) <= set(names)
+
+
+def test_status_strings(lib):
+    for code, name in K.STATUS_NAMES.items():
+        assert lib.kda_status_string(code).decode().startswith(name)
+    assert lib.kda_version() >= 100
+    assert lib.kda_last_cuda_error() == 0
+
+
+# Fake device addresses: validation rejects before any CUDA call is made.
+A = 0x7000_0000_0000
+
+
+def _p(i):
+    return ctypes.c_void_p(A + i * 0x1000_0000)
+
+
+def shape(**kw):
+    d = dict(B=1, T=64, H=2, dk=64, dv=64, chunk=64, n_seqs=0, io_dtype=0)
+    d.update(kw)
+    return K.KdaShape(**d)
+
+
+def chunk_call(lib, s, q=1, k=2, v=3, la=4, b=5, s0=6, cu=None, out=7, sf=8,
+               fn="kda_chunk_fwd"):
+    P = lambda i: None if i is None else (ctypes.c_void_p(i) if isinstance(i, int) and i > 1000 else _p(i))  # noqa: E731
+    return getattr(lib, fn)(None if s is None else ctypes.byref(s), P(q), P(k),
+                            P(v), P(la), P(b), P(s0), P(cu), P(out), P(sf), None)
+
+
+@pytest.mark.parametrize("fn", ["kda_chunk_fwd", "kda_chunk_fwd_staged"])
+def test_chunk_validation(lib, fn):
+    INV, UNS, MIS = 1, 2, 3
+    assert chunk_call(lib, None, fn=fn) == INV
+    assert chunk_call(lib, shape(H=0), fn=fn) == INV
+    assert chunk_call(lib, shape(T=-1), fn=fn) == INV
+    assert chunk_call(lib, shape(io_dtype=7), fn=fn) == INV
+    assert chunk_call(lib, shape(dk=96), fn=fn) == UNS
+    assert chunk_call(lib, shape(dv=256), fn=fn) == UNS
+    assert chunk_call(lib, shape(chunk=128), fn=fn) == UNS
+    assert chunk_call(lib, shape(), q=None, fn=fn) == INV
+    assert chunk_call(lib, shape(), sf=None, fn=fn) == INV
+    assert chunk_call(lib, shape(), out=A + 3 * 0x1000_0000 + 2, fn=fn) == MIS
+    assert chunk_call(lib, shape(), la=A + 4 * 0x1000_0000 + 8, fn=fn) == MIS
+    # out aliasing an input
+    assert chunk_call(lib, shape(), out=1, fn=fn) == INV
+    # final state overlapping (but not equal to) the initial state
+    assert chunk_call(lib, shape(), sf=A + 6 * 0x1000_0000 + 16, fn=fn) == INV
+    # packed layout needs B == 1 and n_seqs >= 1
+    assert chunk_call(lib, shape(B=2, n_seqs=2), cu=9, fn=fn) == INV
+    assert chunk_call(lib, shape(n_seqs=0), cu=9, fn=fn) == INV
+
+
+def test_recurrent_validation(lib):
+    INV, UNS, MIS = 1, 2, 3
+
+    def call(s, q=1, k=2, v=3, la=4, b=5, st=6, out=7):
+        P = lambda i: None if i is None else (ctypes.c_void_p(i) if i > 1000 else _p(i))  # noqa: E731
+        return lib.kda_recurrent_step(None if s is None else ctypes.byref(s),
+                                      P(q), P(k), P(v), P(la), P(b), P(st),
+                                      P(out), None)
+
+    assert call(None) == INV
+    assert call(shape(H=0)) == INV
+    assert call(shape(dk=48)) == UNS
+    assert call(shape(), st=None) == INV
+    assert call(shape(), v=None) == INV
+    assert call(shape(), q=A + 0x1000_0000 + 4) == MIS
+    assert call(shape(), out=6) == INV          # out aliases the state
+    assert call(shape(), st=2) == INV           # state aliases k
