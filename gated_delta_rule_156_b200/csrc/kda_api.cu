@@ -20,6 +20,7 @@ kda_status cuda_fail(cudaError_t e) {
 bool supported_dim(int d) { return d == 32 || d == 64 || d == 128; }
 bool supported_chunk(int c) { return c == 16 || c == 32 || c == 64; }
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+bool aligned4(const void* p) { return ((uintptr_t)p & 3u) == 0; }
 
 struct Range {
   uintptr_t lo, hi;
@@ -92,9 +93,11 @@ kda_status validate_chunk(const kda_shape* s, const void* q, const void* k,
   if (any_tokens && (!q || !k || !v || !la || !beta || !out))
     return KDA_ERR_INVALID_ARG;
   if (any_state && !s_final) return KDA_ERR_INVALID_ARG;
-  const void* ptrs[] = {q, k, v, la, beta, s_init, cu, out, s_final};
+  const void* ptrs[] = {q, k, v, la, s_init, out, s_final};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
+  if ((beta && !aligned4(beta)) || (cu && !aligned4(cu)))
+    return KDA_ERR_MISALIGNED;
   // The output may alias no input; the final state may only coincide exactly
   // with the initial state (in-place update).
   const Range rq = span(q, tokens * H * s->dk * esz),
@@ -191,9 +194,10 @@ kda_status kda_recurrent_step(const kda_shape* s, const void* q, const void* k,
   if (s->B > 0 && !state_inout) return KDA_ERR_INVALID_ARG;
   if (tokens > 0 && (!q || !k || !v || !log_alpha || !beta || !out))
     return KDA_ERR_INVALID_ARG;
-  const void* ptrs[] = {q, k, v, log_alpha, beta, state_inout, out};
+  const void* ptrs[] = {q, k, v, log_alpha, state_inout, out};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
+  if (beta && !aligned4(beta)) return KDA_ERR_MISALIGNED;
   const Range rq = span(q, tokens * H * s->dk * esz),
               rk = span(k, tokens * H * s->dk * esz),
               rv = span(v, tokens * H * s->dv * esz),

@@ -19,8 +19,8 @@ STATUS_NAMES = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED",
 
 # Entry points declared in include/kda.h (kept in sync by tests).
 EXPORTS = ("kda_chunk_fwd", "kda_chunk_fwd_staged", "kda_recurrent_step",
-           "kda_chunk_fwd_plan", "kda_status_string", "kda_last_cuda_error",
-           "kda_version")
+           "kda_chunk_fwd_plan", "kda_selftest_umma", "kda_status_string",
+           "kda_last_cuda_error", "kda_version")
 
 
 class KdaShape(ctypes.Structure):
@@ -71,6 +71,8 @@ def library():
             ctypes.POINTER(KdaShape), ctypes.c_int, ctypes.c_int,
             ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int),
             ctypes.POINTER(ctypes.c_size_t)]
+        lib.kda_selftest_umma.restype = ctypes.c_int
+        lib.kda_selftest_umma.argtypes = [ctypes.c_int] * 5 + [vp, vp, vp, vp]
         lib.kda_status_string.restype = ctypes.c_char_p
         lib.kda_status_string.argtypes = [ctypes.c_int]
         lib.kda_last_cuda_error.restype = ctypes.c_int
@@ -188,3 +190,21 @@ def chunk_fwd_kernel_count(B, T, H, dk, dv, chunk, dtype, packed=False):
 
 def chunk_fwd_path(B, T, H, dk, dv, chunk, dtype, packed=False):
     return chunk_fwd_plan(B, T, H, dk, dv, chunk, dtype, packed, 1)[0]
+
+
+def selftest_umma(A, B, a_mn, b_mn, panel_rows=None, stream=None):
+    """Diagnostic tensor-core product through the fused kernel's operand
+    layouts (kda_selftest_umma).  A is [128, K] (a_mn=False) or [K, 128]
+    (a_mn=True); B is [N, K] (b_mn=False) or [K, N] (b_mn=True); bf16.
+    Returns D = A_logical @ B_logical as [128, N] fp32."""
+    K = A.shape[1] if not a_mn else A.shape[0]
+    N = B.shape[0] if not b_mn else B.shape[1]
+    D = torch.empty((128, N), dtype=torch.float32, device=A.device)
+    for name, t in (("A", A), ("B", B)):
+        _check_dev(name, t, torch.bfloat16)
+    st = library().kda_selftest_umma(int(a_mn), int(b_mn), N, K,
+                                     panel_rows or K, _ptr(A), _ptr(B),
+                                     _ptr(D), _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_selftest_umma")
+    return D

@@ -34,7 +34,8 @@
  *       states     [N, H, d_k, d_v] fp32, N = B (or n_seqs with cu_seqlens)
  *     q and k are used as given: any scaling or L2 normalisation is the
  *     caller's.
- *   - Every pointer must be 16-byte aligned (KDA_ERR_MISALIGNED otherwise).
+ *   - q, k, v, log_alpha, out and the states must be 16-byte aligned; beta
+ *     and cu_seqlens 4-byte aligned (KDA_ERR_MISALIGNED otherwise).
  *   - `out` must not alias an input.  Argument errors are detected on the host
  *     before anything is launched; no exception crosses the ABI.
  *   - Supported sizes: d_k, d_v in {32, 64, 128}; chunk in {16, 32, 64}.
@@ -163,6 +164,22 @@ KDA_API kda_status kda_recurrent_step(const kda_shape* shape, const void* q,
 KDA_API kda_status kda_chunk_fwd_plan(const kda_shape* shape, int packed,
                                       int staged, int* path, int* kernels,
                                       size_t* workspace_bytes);
+
+/*
+ * kda_selftest_umma -- diagnostic, not part of the forward pass: one
+ * D[128 x N] = A[128 x K] * B[K x N] product (bf16 in, fp32 out) on the
+ * tensor cores through the same shared-memory layouts (128-byte swizzle),
+ * operand descriptors and TMEM read-back as the fused prefill kernel.
+ *   a_mn = 0: A is [128, K] row-major (K-major); 1: A is [K, 128] (M-major).
+ *   b_mn = 0: B is [N, K] row-major (K-major); 1: B is [K, N] (N-major).
+ *   N, K in {64, 128}; panel_rows (>= K, multiple of 8, <= 256) is the row
+ *   count of each M-/N-major shared-memory panel.  D is [128, N] row-major.
+ * One CTA, asynchronous on `stream`; device pointers owned by the caller.
+ */
+KDA_API kda_status kda_selftest_umma(int a_mn, int b_mn, int N, int K,
+                                     int panel_rows, const void* A,
+                                     const void* B, float* D,
+                                     cudaStream_t stream);
 
 /* Human-readable name of a status code (static string, never NULL). */
 KDA_API const char* kda_status_string(kda_status status);

@@ -78,6 +78,7 @@ def test_chunk_validation(lib, fn):
     assert chunk_call(lib, shape(), sf=None, fn=fn) == INV
     assert chunk_call(lib, shape(), out=A + 3 * 0x1000_0000 + 2, fn=fn) == MIS
     assert chunk_call(lib, shape(), la=A + 4 * 0x1000_0000 + 8, fn=fn) == MIS
+    assert chunk_call(lib, shape(), b=A + 5 * 0x1000_0000 + 2, fn=fn) == MIS
     # out aliasing an input
     assert chunk_call(lib, shape(), out=1, fn=fn) == INV
     # final state overlapping (but not equal to) the initial state
