@@ -248,6 +248,13 @@ const char* kda_status_string(kda_status status) {
   return "unknown kda_status";
 }
 
+kda_status kda_device_status(cudaStream_t stream) {
+  int flag = 0;
+  const cudaError_t e = kda::fused_take_timeout(stream, &flag);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return flag ? KDA_ERR_TIMEOUT : KDA_OK;
+}
+
 int kda_last_cuda_error(void) { return g_last_cuda_error; }
 
 int kda_version(void) { return 100; }

@@ -51,6 +51,9 @@ cudaError_t launch_staged(const ChunkArgs& a, void* workspace,
 bool fused_supported(const ChunkArgs& a);
 size_t fused_workspace_bytes(const ChunkArgs& a);
 int fused_kernel_count(const ChunkArgs& a);
+// Synchronises `stream`, then reads and clears the flag a fused kernel sets
+// when one of its bounded waits gave up.
+cudaError_t fused_take_timeout(cudaStream_t stream, int* flag);
 cudaError_t launch_fused(const ChunkArgs& a, void* workspace,
                          cudaStream_t stream);
 

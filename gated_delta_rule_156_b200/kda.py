@@ -19,8 +19,8 @@ STATUS_NAMES = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED",
 
 # Entry points declared in include/kda.h (kept in sync by tests).
 EXPORTS = ("kda_chunk_fwd", "kda_chunk_fwd_staged", "kda_recurrent_step",
-           "kda_chunk_fwd_plan", "kda_selftest_umma", "kda_status_string",
-           "kda_last_cuda_error", "kda_version")
+           "kda_chunk_fwd_plan", "kda_selftest_umma", "kda_device_status",
+           "kda_status_string", "kda_last_cuda_error", "kda_version")
 
 
 class KdaShape(ctypes.Structure):
@@ -73,6 +73,8 @@ def library():
             ctypes.POINTER(ctypes.c_size_t)]
         lib.kda_selftest_umma.restype = ctypes.c_int
         lib.kda_selftest_umma.argtypes = [ctypes.c_int] * 5 + [vp, vp, vp, vp]
+        lib.kda_device_status.restype = ctypes.c_int
+        lib.kda_device_status.argtypes = [vp]
         lib.kda_status_string.restype = ctypes.c_char_p
         lib.kda_status_string.argtypes = [ctypes.c_int]
         lib.kda_last_cuda_error.restype = ctypes.c_int
@@ -208,3 +210,9 @@ def selftest_umma(A, B, a_mn, b_mn, panel_rows=None, stream=None):
     if st != KDA_OK:
         raise KdaError(st, "kda_selftest_umma")
     return D
+
+
+def device_status(stream=None):
+    """Synchronise the stream and return the library's device-side status
+    code (0 = no bounded wait ran out since the last call)."""
+    return library().kda_device_status(_stream(stream))

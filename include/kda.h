@@ -184,6 +184,13 @@ KDA_API kda_status kda_selftest_umma(int a_mn, int b_mn, int N, int K,
 /* Human-readable name of a status code (static string, never NULL). */
 KDA_API const char* kda_status_string(kda_status status);
 
+/* Synchronises `stream` and reports whether any kernel of this library on
+ * this device gave up a bounded device-side wait since the last call
+ * (KDA_ERR_TIMEOUT; the flag is cleared), else KDA_OK.  The kernels never
+ * wait without a time limit; a wait that runs out abandons the rest of that
+ * CTA's work and leaves its outputs unspecified. */
+KDA_API kda_status kda_device_status(cudaStream_t stream);
+
 /* The cudaError_t value behind the most recent KDA_ERR_CUDA on this thread
  * (0 if none). */
 KDA_API int kda_last_cuda_error(void);

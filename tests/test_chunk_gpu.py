@@ -105,7 +105,8 @@ def test_zero_length_and_none_state(path):
 
 @pytest.mark.parametrize("path", PATHS)
 def test_state_handoff_and_in_place(path):
-    # one call over T == two calls joined by the state (T1 not a chunk multiple)
+    # one call over T == two calls joined by the state (T1 not a chunk
+    # multiple; the second call updates the state in place)
     d = W.draw((1, 300), 2, 128, 128, io="bf16", n_states=1, device=DEV, seed=5)
     out, fin = run(d, path, 64)
     part = lambda x, a, b: x[:, a:b].contiguous()  # noqa: E731
@@ -119,9 +120,12 @@ def test_state_handoff_and_in_place(path):
                         state, None, chunk=64, final_state=state,
                         staged=(path == "staged"))
     torch.cuda.synchronize()
-    ref = PY.host64(out)
-    PY.check("split out", PY.host64(torch.cat([o1, o2], 1)), ref, 2e-3)
-    PY.check("split state", PY.host64(state), PY.host64(fin), 2e-3)
+    ro, rs = PY.oracle_dense(d)
+    split = PY.host64(torch.cat([o1, o2], 1))
+    PY.check("split out vs oracle", split, ro, PY.TOL_BF16)
+    PY.check("split state vs oracle", PY.host64(state), rs, PY.TOL_BF16)
+    PY.check("one call out vs oracle", PY.host64(out), ro, PY.TOL_BF16)
+    PY.check("split vs one call", split, PY.host64(out), PY.TOL_BF16)
 
 
 @pytest.mark.parametrize("path", PATHS)
@@ -143,6 +147,18 @@ def test_exact_recall_fp32(path):
                          chunk=64, staged=(path == "staged"))
     torch.cuda.synchronize()
     PY.check("recall", PY.host64(out), PY.host64(d["v"]), 1e-4)
+
+
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 64), (64, 128), (128, 64)])
+def test_bf16_takes_fused_path(dk, dv):
+    path, kernels, _ = K.chunk_fwd_plan(1, 128, 2, dk, dv, 64, torch.bfloat16)
+    assert path == "fused" and kernels == 1
+    d = W.draw((2, 130), 2, dk, dv, io="bf16", n_states=2, device=DEV, seed=dk + dv)
+    out, fin = run(d, "auto", 64)
+    assert K.device_status() == 0
+    ro, rs = PY.oracle_dense(d)
+    PY.check("out", PY.host64(out), ro, PY.TOL_BF16)
+    PY.check("final", PY.host64(fin), rs, PY.TOL_BF16)
 
 
 def _sampled_check(d, out, fin, units, offsets=None):
