@@ -4,6 +4,7 @@
 #include <string.h>
 
 #include <atomic>
+#include <mutex>
 
 #include "../../include/kda.h"
 #include "kda_internal.h"
@@ -146,6 +147,43 @@ kda_status run_with_workspace(size_t bytes, cudaStream_t stream, bool fused,
   return e == cudaSuccess ? KDA_OK : cuda_fail(e);
 }
 
+// ---- fixed scratch for kda_chunk_fwd_staged_noalloc ----------------------
+// The four-stage pipeline's workspace for callers that cannot allocate device
+// memory.  Every GPU that loads this library holds the array until the
+// process exits.  Host code must not pass `g_noalloc_scratch` itself to a
+// kernel: on the host that name is only a stand-in, so its device address is
+// looked up once per device below.
+static __device__ __align__(256) unsigned char
+    g_noalloc_scratch[KDA_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch on the current device, looked up (with
+// that device current) the first time each device asks, then cached.
+void* noalloc_scratch(cudaError_t* err) {
+  static std::mutex mu;
+  static void* addr[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    *err = e;
+    return nullptr;
+  }
+  if (dev < 0 || dev >= 64) {
+    *err = cudaErrorInvalidDevice;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) {
+      *err = e;
+      return nullptr;
+    }
+    addr[dev] = p;
+  }
+  return addr[dev];
+}
+
 }  // namespace
 
 extern "C" {
@@ -177,6 +215,26 @@ kda_status kda_chunk_fwd_staged(const kda_shape* shape, const void* q,
                                        final_state, &a);
   if (st != KDA_OK) return st;
   return run_with_workspace(kda::staged_workspace_bytes(a), stream, false, a);
+}
+
+kda_status kda_chunk_fwd_staged_noalloc(
+    const kda_shape* shape, const void* q, const void* k, const void* v,
+    const float* log_alpha, const float* beta, const float* initial_state,
+    const int32_t* cu_seqlens, void* out, float* final_state,
+    cudaStream_t stream) {
+  kda::ChunkArgs a{};
+  const kda_status st = validate_chunk(shape, q, k, v, log_alpha, beta,
+                                       initial_state, cu_seqlens, out,
+                                       final_state, &a);
+  if (st != KDA_OK) return st;
+  // Too large for the fixed array: refuse before touching the device.
+  if (kda::staged_workspace_bytes(a) > (size_t)KDA_NOALLOC_SCRATCH_BYTES)
+    return KDA_ERR_UNSUPPORTED;
+  cudaError_t e = cudaSuccess;
+  void* ws = noalloc_scratch(&e);
+  if (!ws) return cuda_fail(e);
+  e = kda::launch_staged(a, ws, stream);
+  return e == cudaSuccess ? KDA_OK : cuda_fail(e);
 }
 
 kda_status kda_recurrent_step(const kda_shape* s, const void* q, const void* k,

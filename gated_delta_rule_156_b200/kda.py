@@ -20,7 +20,8 @@ STATUS_NAMES = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED",
 # Entry points declared in include/kda.h (kept in sync by tests).
 EXPORTS = ("kda_chunk_fwd", "kda_chunk_fwd_staged", "kda_recurrent_step",
            "kda_chunk_fwd_plan", "kda_selftest_umma", "kda_device_status",
-           "kda_status_string", "kda_last_cuda_error", "kda_version")
+           "kda_status_string", "kda_last_cuda_error", "kda_version",
+           "kda_chunk_fwd_staged_noalloc")
 
 
 class KdaShape(ctypes.Structure):
@@ -59,7 +60,8 @@ def library():
         vp, fp = ctypes.c_void_p, ctypes.c_void_p
         chunk_args = [ctypes.POINTER(KdaShape), vp, vp, vp, fp, fp, fp, vp, vp,
                       fp, vp]
-        for name in ("kda_chunk_fwd", "kda_chunk_fwd_staged"):
+        for name in ("kda_chunk_fwd", "kda_chunk_fwd_staged",
+                     "kda_chunk_fwd_staged_noalloc"):
             fn = getattr(lib, name)
             fn.restype = ctypes.c_int
             fn.argtypes = chunk_args
@@ -216,3 +218,41 @@ def device_status(stream=None):
     """Synchronise the stream and return the library's device-side status
     code (0 = no bounded wait ran out since the last call)."""
     return library().kda_device_status(_stream(stream))
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20  # KDA_NOALLOC_SCRATCH_BYTES in include/kda.h
+
+
+def chunk_fwd_noalloc(q, k, v, log_alpha, beta, initial_state=None,
+                      cu_seqlens=None, chunk=64, out=None, final_state=None,
+                      stream=None):
+    """kda_chunk_fwd_staged_noalloc: the four-stage fp32 pipeline with its
+    workspace in the library's fixed device array, for callers that must not
+    allocate device memory during the call.  ``out`` and ``final_state``
+    should be passed in by such callers (they are allocated here only when
+    omitted).  Calls that overlap on the GPU race on the shared array."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    n = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if final_state is None:
+        final_state = torch.empty((n, H, dk, dv), dtype=torch.float32,
+                                  device=q.device)
+    for name, t, dt in (("q", q, None), ("k", k, q.dtype), ("v", v, q.dtype),
+                        ("log_alpha", log_alpha, torch.float32),
+                        ("beta", beta, torch.float32),
+                        ("initial_state", initial_state, torch.float32),
+                        ("cu_seqlens", cu_seqlens, torch.int32),
+                        ("out", out, q.dtype),
+                        ("final_state", final_state, torch.float32)):
+        _check_dev(name, t, dt)
+    shape = KdaShape(B, T, H, dk, dv, chunk, n if cu_seqlens is not None else 0,
+                     _io(q))
+    st = library().kda_chunk_fwd_staged_noalloc(
+        ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+        _ptr(beta), _ptr(initial_state), _ptr(cu_seqlens), _ptr(out),
+        _ptr(final_state), _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_chunk_fwd_staged_noalloc")
+    return out, final_state

@@ -131,6 +131,46 @@ KDA_API kda_status kda_chunk_fwd_staged(const kda_shape* shape, const void* q,
                                 const int32_t* cu_seqlens, void* out,
                                 float* final_state, cudaStream_t stream);
 
+/* Size in bytes of the fixed device scratch array behind
+ * kda_chunk_fwd_staged_noalloc (16 MiB). */
+#define KDA_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/*
+ * kda_chunk_fwd_staged_noalloc -- kda_chunk_fwd_staged for callers that must
+ * not allocate device memory.  (The pages have no counterpart of this entry
+ * point: it is a deployment convenience of this library.)
+ *
+ * Who needs it: code whose device memory is owned and planned by someone
+ * else.  Examples are a plugin run inside an inference engine that hands it
+ * pre-planned buffers and forbids allocation in its execute path, a serving
+ * loop that must never stall or fail on an allocator under memory pressure,
+ * and a process whose HBM is already claimed by another caching allocator.
+ * kda_chunk_fwd_staged allocates its workspace stream-ordered on every call,
+ * which such callers cannot allow.
+ *
+ * What it does: exactly the kda_chunk_fwd_staged computation (same
+ * arguments, layouts and results), with the workspace taken from one static
+ * device array of KDA_NOALLOC_SCRATCH_BYTES that every GPU loading this library
+ * holds until the process exits.  It calls no cudaMalloc, cudaFree or other
+ * allocating routine.
+ *   - Size limit: requests whose workspace (kda_chunk_fwd_plan with staged = 1
+ *     reports it) exceeds KDA_NOALLOC_SCRATCH_BYTES return KDA_ERR_UNSUPPORTED
+ *     before anything is launched.
+ *   - First call on a device: it looks up the array's device address on the
+ *     current device (cudaGetSymbolAddress) and caches it.  Make that first
+ *     call before any stream capture.
+ *   - Sharing: every call on a device uses the same array, which keeps the
+ *     last call's contents.  Nothing in it has to start at zero (each call
+ *     writes every scratch byte before reading it).  Calls whose executions
+ *     overlap on the GPU (different streams, or without ordering between
+ *     them) race on the array and give wrong results: serialise them.
+ */
+KDA_API kda_status kda_chunk_fwd_staged_noalloc(
+    const kda_shape* shape, const void* q, const void* k, const void* v,
+    const float* log_alpha, const float* beta, const float* initial_state,
+    const int32_t* cu_seqlens, void* out, float* final_state,
+    cudaStream_t stream);
+
 /*
  * kda_recurrent_step -- token-by-token evaluation (decode).
  *
