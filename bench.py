@@ -239,6 +239,10 @@ def run_kda(args, world, rank, local):
     pk, pk_kind = peaks()
     clocks = Clocks(dev)
 
+    if args.only:
+        run_only(args, dev, stream)
+        return
+
     # ---- prefill -------------------------------------------------------
     cfg = W.CONFIGS[PREFILL_CFG]
     B, T, H, dk, dv, C = cfg["B"], cfg["T"], cfg["H"], cfg["dk"], cfg["dv"], \
@@ -400,6 +404,42 @@ def run_kda(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+def run_only(args, dev, stream):
+    """Warm-up plus `steps` launches of one workload, for a profiler to
+    capture; prints the mean launch time and nothing else."""
+    from gated_delta_rule_156_b200 import kda as K
+    if args.only == "prefill":
+        cfg = W.CONFIGS[PREFILL_CFG]
+        d = W.make(PREFILL_CFG, device=dev)
+        out = torch.empty((cfg["B"], cfg["T"], cfg["H"], cfg["dv"]),
+                          dtype=torch.bfloat16, device=dev)
+        fin = torch.empty((cfg["B"], cfg["H"], cfg["dk"], cfg["dv"]),
+                          dtype=torch.float32, device=dev)
+
+        def fn(_i):
+            K.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"],
+                        None, None, chunk=cfg["chunk"], out=out,
+                        final_state=fin)
+    else:
+        dc = W.CONFIGS[DECODE_CFG]
+        dd = W.make(DECODE_CFG, device=dev)
+        state = dd["initial_state"]
+        dout = torch.empty((dc["N"], 1, dc["H"], dc["dv"]),
+                           dtype=torch.bfloat16, device=dev)
+
+        def fn(i):
+            s_ = i % dc["steps"]
+            K.recurrent_step(*(dd[n][s_][:, None] for n in
+                               ("q", "k", "v", "log_alpha", "beta")), state,
+                             out=dout)
+    for i in range(args.warmup):
+        fn(i)
+    torch.cuda.synchronize()
+    ms, _ = timed(fn, args.steps, stream)
+    print(f"{args.only}: {ms / args.steps:.4f} ms per launch over "
+          f"{args.steps} launches", flush=True)
+
+
 def load_traffic():
     """Per-launch DRAM bytes from the committed ncu summaries, when the
     kernels have not changed since (a small JSON beside the summaries)."""
@@ -421,6 +461,9 @@ def main():
     ap.add_argument("--impl", choices=["kda", "reference"], default="kda")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--only", choices=["prefill", "decode"], default=None,
+                    help="profiling aid: run one workload's warm-up and timed "
+                         "launches only (no e2e, no CPU baseline, no JSON line)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -46,7 +46,7 @@ using namespace sm100;
 
 constexpr int kC = 64;        // chunk length
 constexpr int kDvt = 64;      // d_v columns per CTA
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;
 constexpr int kFS = 68;       // fp32 row stride (floats) of the A / Tm tiles
 
 template <int DK>
@@ -65,7 +65,7 @@ struct Layout {
   static constexpr uint32_t afp = dop + 8192;       // 64 x kFS fp32
   static constexpr uint32_t tfp = afp + 18432;      // 64 x kFS fp32
   static constexpr uint32_t msc = tfp + 18432;      // 3 x 256 fp32
-  static constexpr uint32_t misc = msc + 3072;      // beta, barriers, tmem
+  static constexpr uint32_t misc = msc + 3072;      // beta, exp(g_C), barriers
   static constexpr uint32_t bytes = misc + 1024;
   static constexpr uint32_t tx_in = 2 * NP * 8192 + (DK / 32) * 8192;
   // TMEM columns
@@ -86,20 +86,13 @@ struct FusedParams {
   int n_seqs, T, H, dv, n_tiles;
 };
 
-__device__ __forceinline__ float bf16_at(const uint8_t* panel, int row, int col) {
-  return __bfloat162float(
-      *reinterpret_cast<const __nv_bfloat16*>(panel + sw128_off(row, col)));
-}
-__device__ __forceinline__ void put_bf16(uint8_t* panel, int row, int col,
-                                         float x) {
-  *reinterpret_cast<__nv_bfloat16*>(panel + sw128_off(row, col)) =
-      __float2bfloat16_rn(x);
-}
-
 // (I + A)^-1 for the strictly-lower 64 x 64 A in `A` (row stride kFS) into
 // `X`: the four 16 x 16 diagonal blocks by forward substitution (one column
 // per thread), then the off-diagonal blocks by block forward substitution,
-// X_ij = -X_ii sum_{j<=k<i} A_ik X_kj, in order of distance i - j.
+// X_ij = -X_ii sum_{j<=k<i} A_ik X_kj, in order of distance d = i - j.  In
+// the block products a thread owns 4 rows x 1 column, reading rows as float4
+// (shared by the 16 threads of a row group); all loops are unrolled.  The
+// strictly-upper blocks of X are never written: the caller zeroes them once.
 __device__ __forceinline__ void invert_unit_lower(const float* A, float* X,
                                                   float* M, int tid) {
   if (tid < 64) {
@@ -107,36 +100,88 @@ __device__ __forceinline__ void invert_unit_lower(const float* A, float* X,
     float x[16];
 #pragma unroll
     for (int r = 0; r < 16; ++r) {
-      float acc = 0.f;
+      float a[16];
 #pragma unroll
-      for (int i = 0; i < r; ++i) acc -= A[(o + r) * kFS + o + i] * x[i];
-      x[r] = r < j ? 0.f : (r == j ? 1.f : acc);
+      for (int q4 = 0; q4 < 4; ++q4) {
+        if (4 * q4 < r) {
+          const float4 t =
+              *reinterpret_cast<const float4*>(A + (o + r) * kFS + o + 4 * q4);
+          a[4 * q4] = t.x; a[4 * q4 + 1] = t.y; a[4 * q4 + 2] = t.z;
+          a[4 * q4 + 3] = t.w;
+        }
+      }
+      float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+      for (int i = 0; i < r; ++i) {
+        if (i & 1) s1 -= a[i] * x[i];
+        else s0 -= a[i] * x[i];
+      }
+      x[r] = r < j ? 0.f : (r == j ? 1.f : s0 + s1);
     }
 #pragma unroll
     for (int r = 0; r < 16; ++r) X[(o + r) * kFS + o + j] = x[r];
   }
   __syncthreads();
-#pragma unroll 1
+#pragma unroll
   for (int d = 1; d < 4; ++d) {
-    const int n = 256 * (4 - d);
-    for (int e = tid; e < n; e += kThreads) {
-      const int blk = e >> 8, bi = d + blk, bj = bi - d;
-      const int r = (e >> 4) & 15, c = e & 15;
-      float acc = 0.f;
-      for (int kk = 16 * bj; kk < 16 * bi; ++kk)
-        acc += A[(16 * bi + r) * kFS + kk] * X[kk * kFS + 16 * bj + c];
-      M[blk * 256 + r * 16 + c] = acc;
+    const bool active = tid < 64 * (4 - d);
+    const int blk = tid >> 6, tr = (tid >> 4) & 3, tc = tid & 15;
+    const int bi = d + blk, bj = blk;
+    const int row0 = 16 * bi + 4 * tr;  // this thread's 4 rows
+    if (active) {  // M = sum_{bj<=k<bi} A_{bi,k} X_{k,bj}
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int kk = 0; kk < 16 * d; kk += 4) {
+        const int k0 = 16 * bj + kk;
+        float xv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) xv[u] = X[(k0 + u) * kFS + 16 * bj + tc];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float4 a4 =
+              *reinterpret_cast<const float4*>(A + (row0 + i) * kFS + k0);
+          acc[i] += a4.x * xv[0] + a4.y * xv[1] + a4.z * xv[2] + a4.w * xv[3];
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) M[blk * 256 + (4 * tr + i) * 16 + tc] = acc[i];
     }
     __syncthreads();
-    for (int e = tid; e < n; e += kThreads) {
-      const int blk = e >> 8, bi = d + blk, bj = bi - d;
-      const int r = (e >> 4) & 15, c = e & 15;
-      float acc = 0.f;
-      for (int rr = 0; rr <= r; ++rr)
-        acc -= X[(16 * bi + r) * kFS + 16 * bi + rr] * M[blk * 256 + rr * 16 + c];
-      X[(16 * bi + r) * kFS + 16 * bj + c] = acc;
+    if (active) {  // X_{bi,bj} = -X_{bi,bi} M
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int rr = 0; rr < 16; rr += 4) {
+        float mv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) mv[u] = M[blk * 256 + (rr + u) * 16 + tc];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float4 x4 = *reinterpret_cast<const float4*>(
+              X + (row0 + i) * kFS + 16 * bi + rr);
+          acc[i] -= x4.x * mv[0] + x4.y * mv[1] + x4.z * mv[2] + x4.w * mv[3];
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) X[(row0 + i) * kFS + 16 * bj + tc] = acc[i];
     }
     __syncthreads();
+  }
+}
+
+// Store `n` consecutive 16-byte chunks (8 bf16 each, starting at chunk
+// `c0`) of one row of a 128-byte-swizzled panel.
+template <int N>
+__device__ __forceinline__ void st_chunks_sw128(uint8_t* panel, int row, int c0,
+                                                const float* v) {
+#pragma unroll
+  for (int c = 0; c < N; ++c) {
+    uint4 w;
+    w.x = pack_bf16x2(v[8 * c + 0], v[8 * c + 1]);
+    w.y = pack_bf16x2(v[8 * c + 2], v[8 * c + 3]);
+    w.z = pack_bf16x2(v[8 * c + 4], v[8 * c + 5]);
+    w.w = pack_bf16x2(v[8 * c + 6], v[8 * c + 7]);
+    *reinterpret_cast<uint4*>(panel + row * 128 + (((c0 + c) ^ (row & 7)) << 4)) =
+        w;
   }
 }
 
@@ -164,13 +209,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* afp = reinterpret_cast<float*>(sm + Lay::afp);
   float* tfp = reinterpret_cast<float*>(sm + Lay::tfp);
   float* msc = reinterpret_cast<float*>(sm + Lay::msc);
+  float* red = afp;  // the prologue's partial sums (afp is free then)
   float* beta_s = reinterpret_cast<float*>(sm + Lay::misc);        // [64]
-  uint64_t* bar_in = reinterpret_cast<uint64_t*>(sm + Lay::misc + 256);
+  float* gexp_s = reinterpret_cast<float*>(sm + Lay::misc + 256);  // [DK]
+  uint64_t* bar_in = reinterpret_cast<uint64_t*>(sm + Lay::misc + 768);
   uint64_t* bar_v = bar_in + 1;
   uint64_t* bar_mma = bar_in + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_in + 3);
 
   const int tid = threadIdx.x, warp = tid >> 5;
+  // TMEM access: warp w reads lanes 32 (w % 4) .. +31; warps 0-3 take the
+  // first 32 columns of a 64-column accumulator, warps 4-7 the second.
+  const int row_t = tid & 127;  // this thread's TMEM lane / accumulator row
+  const int colh = warp >> 2;   // which 32-column half
+  const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+
   const int u = blockIdx.x;
   const int tile = u % p.n_tiles;
   const int h = (u / p.n_tiles) % p.H;
@@ -195,28 +248,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
+  for (int i = tid; i < 64 * kFS; i += kThreads) tfp[i] = 0.f;
   if (DK == 64) {  // channels 64-127 of the M = 128 Kh^T operand stay zero
     uint4* z = reinterpret_cast<uint4*>(kh + 8192);
     for (int i = tid; i < 512; i += kThreads) z[i] = make_uint4(0, 0, 0, 0);
   }
 
-  // The state tile: thread c owns row c (key channel c), 64 fp32 columns.
-  float s[kDvt];
+  // The state tile: thread t owns row row_t (key channel), columns
+  // 32 colh .. 32 colh + 31 of this CTA's 64-column tile, in fp32 registers.
+  const bool owns_state = row_t < DK;
+  float s[32];
   const size_t sbase = (((size_t)seq * p.H + h) * DK) * p.dv + j0;
-  if (tid < DK) {
+  if (owns_state) {
     if (p.s_init) {
-      const float4* src =
-          reinterpret_cast<const float4*>(p.s_init + sbase + (size_t)tid * p.dv);
+      const float4* src = reinterpret_cast<const float4*>(
+          p.s_init + sbase + (size_t)row_t * p.dv + 32 * colh);
 #pragma unroll
-      for (int i = 0; i < kDvt / 4; ++i) {
+      for (int i = 0; i < 8; ++i) {
         const float4 x = src[i];
         s[4 * i] = x.x; s[4 * i + 1] = x.y; s[4 * i + 2] = x.z; s[4 * i + 3] = x.w;
       }
     } else {
 #pragma unroll
-      for (int i = 0; i < kDvt; ++i) s[i] = 0.f;
+      for (int i = 0; i < 32; ++i) s[i] = 0.f;
     }
-    st_row_sw128(sop, tid, s);
+    st_chunks_sw128<4>(sop, row_t, 4 * colh, s);
   }
 
   auto issue_inputs = [&](int tok) {
@@ -240,7 +296,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
 
   if (tid == 0 && nch > 0) {
     issue_inputs(start);
@@ -252,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   uint32_t ph_in = 0, ph_v = 0, ph_mma = 0;
   bool failed = false;
-  bool in_flight = false;  // an input TMA was issued and not waited for
+  bool in_flight = false;    // an input TMA was issued and not waited for
   bool v_pending = nch > 0;  // (thread 0) a V TMA was issued, not waited for
 
   for (int n = 0; n < nch; ++n) {
@@ -272,35 +327,93 @@ __global__ void __launch_bounds__(kThreads, 1)
     in_flight = false;
     if (__syncthreads_or(!ok)) { failed = true; break; }
 
-    // ---- prologue: decay prefix sums and the four scaled copies of k, q
-    float gexp_c = 1.f;  // exp(g_C) of this thread's channel
-    if (tid < DK) {
-      const int c = tid, pnl = c >> 6, cc = c & 63;
-      const float* la = st_la + (c >> 5) * (64 * 32) + (c & 31);
-      float gC = 0.f;
-      for (int r = 0; r < L; ++r) gC += la[r * 32];
-      gexp_c = __expf(gC);
+    // ---- prologue: decay prefix sums and the four scaled copies of k, q.
+    // Thread = (4-channel group cg, block of RPT consecutive rows).  The
+    // products are formed in packed bf16 (the operands are bf16 anyway).
+    {
+      constexpr int NCG = DK / 4;                 // channel groups
+      constexpr int NRB = kThreads / NCG;         // row blocks
+      constexpr int RPT = kC / NRB;               // rows per thread
+      const int cg = tid % NCG, rb = tid / NCG;
+      const int pnl = cg >> 4;                    // 64-channel panel
+      const int ck = (cg >> 1) & 7;               // 16-byte chunk in the row
+      const int cb = (cg & 1) * 8;                // byte offset in the chunk
+      const float* la_base = st_la + (cg >> 3) * (64 * 32) + (cg & 7) * 4;
+      float part[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int i = 0; i < RPT; ++i) {
+        const int r = rb * RPT + i;
+        if (r < L) {
+          const float4 x = *reinterpret_cast<const float4*>(la_base + r * 32);
+          part[0] += x.x; part[1] += x.y; part[2] += x.z; part[3] += x.w;
+        }
+      }
+      *reinterpret_cast<float4*>(red + rb * DK + 4 * cg) =
+          make_float4(part[0], part[1], part[2], part[3]);
+      __syncthreads();
+      float g[4] = {0.f, 0.f, 0.f, 0.f}, tot[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int b2 = 0; b2 < NRB; ++b2) {
+        const float4 y = *reinterpret_cast<const float4*>(red + b2 * DK + 4 * cg);
+        if (b2 < rb) { g[0] += y.x; g[1] += y.y; g[2] += y.z; g[3] += y.w; }
+        tot[0] += y.x; tot[1] += y.y; tot[2] += y.z; tot[3] += y.w;
+      }
+      constexpr float kLog2e = 1.4426950408889634f;
+      float gct[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) gct[c] = ex2_approx(tot[c] * kLog2e);
+      if (rb == 0)
+        *reinterpret_cast<float4*>(gexp_s + 4 * cg) =
+            make_float4(gct[0], gct[1], gct[2], gct[3]);
+      const __nv_bfloat162 gc01 = __floats2bfloat162_rn(gct[0], gct[1]);
+      const __nv_bfloat162 gc23 = __floats2bfloat162_rn(gct[2], gct[3]);
       const uint8_t* pq = st_q + pnl * 8192;
       const uint8_t* pk = st_k + pnl * 8192;
       uint8_t* pkq = kq + pnl * 16384;
       uint8_t* pkb = kb + pnl * 8192;
       uint8_t* pkh = kh + pnl * 8192;
-      float g = 0.f;
-#pragma unroll 4
-      for (int r = 0; r < kC; ++r) {
+#pragma unroll
+      for (int i = 0; i < RPT; ++i) {
+        const int r = rb * RPT + i;
+        const uint32_t off = r * 128 + ((ck ^ (r & 7)) << 4) + cb;
         const bool valid = r < L;
-        g += valid ? la[r * 32] : 0.f;
-        const float e = valid ? __expf(g) : 0.f;
-        const float ie = valid ? __expf(-g) : 0.f;
-        const float kv = bf16_at(pk, r, cc), qv = bf16_at(pq, r, cc);
-        put_bf16(pkq, r, cc, kv * e);
-        put_bf16(pkq, 64 + r, cc, qv * e);
-        put_bf16(pkb, r, cc, kv * ie);
-        put_bf16(pkh, r, cc, kv * ie * gexp_c);
+        const uint2 kr = *reinterpret_cast<const uint2*>(pk + off);
+        const uint2 qr = *reinterpret_cast<const uint2*>(pq + off);
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (valid) x = *reinterpret_cast<const float4*>(la_base + r * 32);
+        g[0] += x.x; g[1] += x.y; g[2] += x.z; g[3] += x.w;
+        float e[4], ie[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const float t = g[c] * kLog2e;
+          e[c] = valid ? ex2_approx(t) : 0.f;
+          ie[c] = valid ? ex2_approx(-t) : 0.f;
+        }
+        const __nv_bfloat162 e01 = __floats2bfloat162_rn(e[0], e[1]);
+        const __nv_bfloat162 e23 = __floats2bfloat162_rn(e[2], e[3]);
+        const __nv_bfloat162 i01 = __floats2bfloat162_rn(ie[0], ie[1]);
+        const __nv_bfloat162 i23 = __floats2bfloat162_rn(ie[2], ie[3]);
+        const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kr);
+        const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&qr);
+        const __nv_bfloat162 kb01 = __hmul2(k2[0], i01), kb23 = __hmul2(k2[1], i23);
+        uint2 wt, wq, wb, wh;
+        *reinterpret_cast<__nv_bfloat162*>(&wt.x) = __hmul2(k2[0], e01);
+        *reinterpret_cast<__nv_bfloat162*>(&wt.y) = __hmul2(k2[1], e23);
+        *reinterpret_cast<__nv_bfloat162*>(&wq.x) = __hmul2(q2[0], e01);
+        *reinterpret_cast<__nv_bfloat162*>(&wq.y) = __hmul2(q2[1], e23);
+        *reinterpret_cast<__nv_bfloat162*>(&wb.x) = kb01;
+        *reinterpret_cast<__nv_bfloat162*>(&wb.y) = kb23;
+        *reinterpret_cast<__nv_bfloat162*>(&wh.x) = __hmul2(kb01, gc01);
+        *reinterpret_cast<__nv_bfloat162*>(&wh.y) = __hmul2(kb23, gc23);
+        *reinterpret_cast<uint2*>(pkq + off) = wt;
+        *reinterpret_cast<uint2*>(pkq + 64 * 128 + off) = wq;
+        *reinterpret_cast<uint2*>(pkb + off) = wb;
+        *reinterpret_cast<uint2*>(pkh + off) = wh;
       }
     }
     fence_proxy_async();
     __syncthreads();
+    const float gexp_c = owns_state ? gexp_s[row_t] : 1.f;
 
     // ---- MMA1: [Kt; Qt] . Kb^T ; then prefetch the next chunk's inputs
     if (tid == 0) {
@@ -315,9 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                  idesc, ks > 0);
       }
       mma_commit(bar_mma);
-      if (has_next) {
-        issue_inputs(tok0 + kC);
-      }
+      if (has_next) issue_inputs(tok0 + kC);
     }
     in_flight = has_next;
     ok = mbar_wait(bar_mma, ph_mma);
@@ -327,25 +438,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---- A (rows 0-63, fp32) and P (rows 64-127, bf16 into [T'; P])
     {
-      float v[64];
-      tmem_ld32(tmem + lane_base + Lay::t_d1, v);
-      tmem_ld32(tmem + lane_base + Lay::t_d1 + 32, v + 32);
-      if (tid < 64) {
-        const float b = beta_s[tid];
+      float v[32];
+      tmem_ld32(tmem + lane_base + Lay::t_d1 + 32 * colh, v);
+      if (row_t < 64) {
+        const float b = beta_s[row_t];
 #pragma unroll
-        for (int i = 0; i < 64; i += 4) {
+        for (int i = 0; i < 32; i += 4) {
+          const int c = 32 * colh + i;
           float4 w;
-          w.x = i + 0 < tid ? b * v[i + 0] : 0.f;
-          w.y = i + 1 < tid ? b * v[i + 1] : 0.f;
-          w.z = i + 2 < tid ? b * v[i + 2] : 0.f;
-          w.w = i + 3 < tid ? b * v[i + 3] : 0.f;
-          *reinterpret_cast<float4*>(afp + tid * kFS + i) = w;
+          w.x = c + 0 < row_t ? b * v[i + 0] : 0.f;
+          w.y = c + 1 < row_t ? b * v[i + 1] : 0.f;
+          w.z = c + 2 < row_t ? b * v[i + 2] : 0.f;
+          w.w = c + 3 < row_t ? b * v[i + 3] : 0.f;
+          *reinterpret_cast<float4*>(afp + row_t * kFS + c) = w;
         }
       } else {
-        const int r = tid - 64;
+        const int r = row_t - 64;
 #pragma unroll
-        for (int i = 0; i < 64; ++i) v[i] = i <= r ? v[i] : 0.f;
-        st_row_sw128(tpp, tid, v);
+        for (int i = 0; i < 32; ++i) v[i] = 32 * colh + i <= r ? v[i] : 0.f;
+        st_chunks_sw128<4>(tpp, row_t, 4 * colh, v);
       }
     }
     tc_fence_before();
@@ -353,12 +464,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     invert_unit_lower(afp, tfp, msc, tid);
 
-    if (tid < 64) {  // T' = Tm Diag(beta), row tid of [T'; P]
-      float v[64];
+    {  // T' = Tm Diag(beta): row tid % 64, 16 columns per thread
+      const int r = tid & 63, qc = tid >> 6;
+      float v[16];
 #pragma unroll
-      for (int i = 0; i < 64; ++i)
-        v[i] = i <= tid ? tfp[tid * kFS + i] * beta_s[i] : 0.f;
-      st_row_sw128(tpp, tid, v);
+      for (int i = 0; i < 16; i += 4) {
+        const float4 t =
+            *reinterpret_cast<const float4*>(tfp + r * kFS + 16 * qc + i);
+        const float4 b = *reinterpret_cast<const float4*>(beta_s + 16 * qc + i);
+        v[i] = t.x * b.x; v[i + 1] = t.y * b.y; v[i + 2] = t.z * b.z;
+        v[i + 3] = t.w * b.w;
+      }
+      st_chunks_sw128<2>(tpp, r, 2 * qc, v);
     }
     fence_proxy_async();
     __syncthreads();
@@ -390,13 +507,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
 
     // ---- W rows (bf16) over the Kt rows of [Kt; Qt] -> [W; Qt]
-    if (tid < 64) {
+    if (row_t < 64) {
 #pragma unroll
-      for (int pnl = 0; pnl < (int)Lay::NP; ++pnl) {
-        float v[64];
-        tmem_ld32(tmem + lane_base + Lay::t_w + pnl * 64, v);
-        tmem_ld32(tmem + lane_base + Lay::t_w + pnl * 64 + 32, v + 32);
-        st_row_sw128(kq + pnl * 16384, tid, v);
+      for (int j = 0; j < DK / 64; ++j) {
+        const int hh = colh * (DK / 64) + j;  // 32-column piece of the row
+        float v[32];
+        tmem_ld32(tmem + lane_base + Lay::t_w + 32 * hh, v);
+        st_chunks_sw128<4>(kq + (hh >> 1) * 16384, row_t, 4 * (hh & 1), v);
       }
     }
     tc_fence_before();
@@ -426,15 +543,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
 
     // ---- Delta = U - W S  (rows 0-63), bf16 into the MN-major Delta tile
-    if (tid < 64) {
-      float uu[64], ws[64];
-      tmem_ld32(tmem + lane_base + Lay::t_u, uu);
-      tmem_ld32(tmem + lane_base + Lay::t_u + 32, uu + 32);
-      tmem_ld32(tmem + lane_base + Lay::t_d3, ws);
-      tmem_ld32(tmem + lane_base + Lay::t_d3 + 32, ws + 32);
+    if (row_t < 64) {
+      float uu[32], ws[32];
+      tmem_ld32(tmem + lane_base + Lay::t_u + 32 * colh, uu);
+      tmem_ld32(tmem + lane_base + Lay::t_d3 + 32 * colh, ws);
 #pragma unroll
-      for (int i = 0; i < 64; ++i) uu[i] -= ws[i];
-      st_row_sw128(dop, tid, uu);
+      for (int i = 0; i < 32; ++i) uu[i] -= ws[i];
+      st_chunks_sw128<4>(dop, row_t, 4 * colh, uu);
     }
     tc_fence_before();
     fence_proxy_async();
@@ -462,16 +577,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
 
     // ---- outputs (rows 64-127) and the state update (row per channel)
-    if (tid >= 64) {
-      const int r = tid - 64;
-      float o[64];
-      tmem_ld32(tmem + lane_base + Lay::t_d3, o);
-      tmem_ld32(tmem + lane_base + Lay::t_d3 + 32, o + 32);
+    if (row_t >= 64) {
+      const int r = row_t - 64;
+      float o[32];
+      tmem_ld32(tmem + lane_base + Lay::t_d3 + 32 * colh, o);
       if (r < L) {
         uint4* dst = reinterpret_cast<uint4*>(
-            p.out + ((size_t)(tok0 + r) * p.H + h) * p.dv + j0);
+            p.out + ((size_t)(tok0 + r) * p.H + h) * p.dv + j0 + 32 * colh);
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
+        for (int ch = 0; ch < 4; ++ch) {
           uint4 w;
           w.x = pack_bf16x2(o[8 * ch + 0], o[8 * ch + 1]);
           w.y = pack_bf16x2(o[8 * ch + 2], o[8 * ch + 3]);
@@ -482,13 +596,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     {
-      float d4[64];
-      tmem_ld32(tmem + lane_base + Lay::t_d4, d4);
-      tmem_ld32(tmem + lane_base + Lay::t_d4 + 32, d4 + 32);
-      if (tid < DK) {
+      float d4[32];
+      tmem_ld32(tmem + lane_base + Lay::t_d4 + 32 * colh, d4);
+      if (owns_state) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i) s[i] = gexp_c * s[i] + d4[i];
-        st_row_sw128(sop, tid, s);
+        for (int i = 0; i < 32; ++i) s[i] = gexp_c * s[i] + d4[i];
+        st_chunks_sw128<4>(sop, row_t, 4 * colh, s);
       }
     }
     tc_fence_before();
@@ -500,12 +613,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) {
       atomicExch(&g_fused_timeout, 1);
       if (in_flight) mbar_wait(bar_in, ph_in, 100000000ull);
-      if (v_pending) mbar_wait(bar_v, v_pending ? ph_v : 0, 100000000ull);
+      if (v_pending) mbar_wait(bar_v, ph_v, 100000000ull);
     }
-  } else if (tid < DK) {
-    float4* dst = reinterpret_cast<float4*>(p.s_final + sbase + (size_t)tid * p.dv);
+  } else if (owns_state) {
+    float4* dst = reinterpret_cast<float4*>(p.s_final + sbase +
+                                            (size_t)row_t * p.dv + 32 * colh);
 #pragma unroll
-    for (int i = 0; i < kDvt / 4; ++i)
+    for (int i = 0; i < 8; ++i)
       dst[i] = make_float4(s[4 * i], s[4 * i + 1], s[4 * i + 2], s[4 * i + 3]);
   }
   tc_fence_before();

@@ -19,6 +19,13 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// 2^x by the SFU's approximate base-2 exponential (flush-to-zero).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)),
@@ -211,6 +218,21 @@ __device__ __forceinline__ void st_row_sw128(uint8_t* panel, int row,
     w.y = pack_bf16x2(v[8 * ch + 2], v[8 * ch + 3]);
     w.z = pack_bf16x2(v[8 * ch + 4], v[8 * ch + 5]);
     w.w = pack_bf16x2(v[8 * ch + 6], v[8 * ch + 7]);
+    *reinterpret_cast<uint4*>(panel + row * 128 + ((ch ^ (row & 7)) << 4)) = w;
+  }
+}
+
+// Write 32 floats as half (chunks 4*half .. 4*half+3) of a 128-byte bf16 row.
+__device__ __forceinline__ void st_half_row_sw128(uint8_t* panel, int row,
+                                                  int half, const float* v) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const int ch = 4 * half + c;
+    uint4 w;
+    w.x = pack_bf16x2(v[8 * c + 0], v[8 * c + 1]);
+    w.y = pack_bf16x2(v[8 * c + 2], v[8 * c + 3]);
+    w.z = pack_bf16x2(v[8 * c + 4], v[8 * c + 5]);
+    w.w = pack_bf16x2(v[8 * c + 6], v[8 * c + 7]);
     *reinterpret_cast<uint4*>(panel + row * 128 + ((ch ^ (row & 7)) << 4)) = w;
   }
 }
