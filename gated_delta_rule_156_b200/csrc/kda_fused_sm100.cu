@@ -64,8 +64,8 @@ struct Layout {
   static constexpr uint32_t dop = sop + DK * 128;   // 64 rows x 128 B
   static constexpr uint32_t afp = dop + 8192;       // 64 x kFS fp32
   static constexpr uint32_t tfp = afp + 18432;      // 64 x kFS fp32
-  static constexpr uint32_t msc = tfp + 18432;      // 3 x 256 fp32
-  static constexpr uint32_t misc = msc + 3072;      // beta, exp(g_C), barriers
+  static constexpr uint32_t msc = tfp + 18432;      // 1024 fp32 scratch
+  static constexpr uint32_t misc = msc + 4096;      // beta, exp(g_C), barriers
   static constexpr uint32_t bytes = misc + 1024;
   static constexpr uint32_t tx_in = 2 * NP * 8192 + (DK / 32) * 8192;
   // TMEM columns
@@ -87,12 +87,15 @@ struct FusedParams {
 };
 
 // (I + A)^-1 for the strictly-lower 64 x 64 A in `A` (row stride kFS) into
-// `X`: the four 16 x 16 diagonal blocks by forward substitution (one column
-// per thread), then the off-diagonal blocks by block forward substitution,
-// X_ij = -X_ii sum_{j<=k<i} A_ik X_kj, in order of distance d = i - j.  In
-// the block products a thread owns 4 rows x 1 column, reading rows as float4
-// (shared by the 16 threads of a row group); all loops are unrolled.  The
-// strictly-upper blocks of X are never written: the caller zeroes them once.
+// `X` (row stride kFS), by recursive doubling on unit-lower blocks:
+//   [L11 0; L21 L22]^-1 = [X11 0; -X22 L21 X11  X22].
+// Phase 0 inverts the four 16 x 16 diagonal blocks by forward substitution
+// (one column per thread).  Phases 1-2 form the two 16 x 16 blocks (1,0) and
+// (3,2) that complete the 32 x 32 diagonal halves; phases 3-4 form the
+// 32 x 32 block coupling the halves.  Every product phase uses all threads
+// with float4 operand loads.  `M` holds 1024 floats of scratch.  The
+// strictly-upper part of X outside the diagonal 16-blocks is never written:
+// the caller zeroes it once.
 __device__ __forceinline__ void invert_unit_lower(const float* A, float* X,
                                                   float* M, int tid) {
   if (tid < 64) {
@@ -122,50 +125,78 @@ __device__ __forceinline__ void invert_unit_lower(const float* A, float* X,
     for (int r = 0; r < 16; ++r) X[(o + r) * kFS + o + j] = x[r];
   }
   __syncthreads();
+  {  // blocks (1,0) and (3,2): thread = (block b, row r, column pair c)
+    const int b = tid >> 7, r = (tid >> 3) & 15, c = (tid & 7) * 2;
+    const int bi = 2 * b + 1, bj = 2 * b;  // rows of block bi, cols of bj
+    float m0 = 0.f, m1 = 0.f;
 #pragma unroll
-  for (int d = 1; d < 4; ++d) {
-    const bool active = tid < 64 * (4 - d);
-    const int blk = tid >> 6, tr = (tid >> 4) & 3, tc = tid & 15;
-    const int bi = d + blk, bj = blk;
-    const int row0 = 16 * bi + 4 * tr;  // this thread's 4 rows
-    if (active) {  // M = sum_{bj<=k<bi} A_{bi,k} X_{k,bj}
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int k = 0; k < 16; k += 4) {  // M = A_{bi,bj} X_{bj,bj}
+      const float4 a4 =
+          *reinterpret_cast<const float4*>(A + (16 * bi + r) * kFS + 16 * bj + k);
+      const float av[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
-      for (int kk = 0; kk < 16 * d; kk += 4) {
-        const int k0 = 16 * bj + kk;
-        float xv[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) xv[u] = X[(k0 + u) * kFS + 16 * bj + tc];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float4 a4 =
-              *reinterpret_cast<const float4*>(A + (row0 + i) * kFS + k0);
-          acc[i] += a4.x * xv[0] + a4.y * xv[1] + a4.z * xv[2] + a4.w * xv[3];
-        }
+      for (int u = 0; u < 4; ++u) {
+        const float2 x2 = *reinterpret_cast<const float2*>(
+            X + (16 * bj + k + u) * kFS + 16 * bj + c);
+        m0 += av[u] * x2.x;
+        m1 += av[u] * x2.y;
       }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) M[blk * 256 + (4 * tr + i) * 16 + tc] = acc[i];
     }
+    *reinterpret_cast<float2*>(M + b * 256 + r * 16 + c) = make_float2(m0, m1);
     __syncthreads();
-    if (active) {  // X_{bi,bj} = -X_{bi,bi} M
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    float y0 = 0.f, y1 = 0.f;
 #pragma unroll
-      for (int rr = 0; rr < 16; rr += 4) {
-        float mv[4];
+    for (int k = 0; k < 16; k += 4) {  // X_{bi,bj} = -X_{bi,bi} M
+      const float4 x4 =
+          *reinterpret_cast<const float4*>(X + (16 * bi + r) * kFS + 16 * bi + k);
+      const float xv[4] = {x4.x, x4.y, x4.z, x4.w};
 #pragma unroll
-        for (int u = 0; u < 4; ++u) mv[u] = M[blk * 256 + (rr + u) * 16 + tc];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float4 x4 = *reinterpret_cast<const float4*>(
-              X + (row0 + i) * kFS + 16 * bi + rr);
-          acc[i] -= x4.x * mv[0] + x4.y * mv[1] + x4.z * mv[2] + x4.w * mv[3];
-        }
+      for (int u = 0; u < 4; ++u) {
+        const float2 m2 =
+            *reinterpret_cast<const float2*>(M + b * 256 + (k + u) * 16 + c);
+        y0 -= xv[u] * m2.x;
+        y1 -= xv[u] * m2.y;
       }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) X[(row0 + i) * kFS + 16 * bj + tc] = acc[i];
     }
-    __syncthreads();
+    *reinterpret_cast<float2*>(X + (16 * bi + r) * kFS + 16 * bj + c) =
+        make_float2(y0, y1);
   }
+  __syncthreads();
+  {  // the 32 x 32 block (rows 32-63, cols 0-31): thread = (row r, 4 cols)
+    const int r = tid >> 3, c = (tid & 7) * 4;
+    float m[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int k = 0; k < 32; k += 4) {  // M = A_{21} X_{11}
+      const float4 a4 =
+          *reinterpret_cast<const float4*>(A + (32 + r) * kFS + k);
+      const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float4 x4 =
+            *reinterpret_cast<const float4*>(X + (k + u) * kFS + c);
+        m[0] += av[u] * x4.x; m[1] += av[u] * x4.y;
+        m[2] += av[u] * x4.z; m[3] += av[u] * x4.w;
+      }
+    }
+    *reinterpret_cast<float4*>(M + r * 32 + c) = make_float4(m[0], m[1], m[2], m[3]);
+    __syncthreads();
+    float y[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int k = 0; k < 32; k += 4) {  // X_{21} = -X_{22} M
+      const float4 x4 =
+          *reinterpret_cast<const float4*>(X + (32 + r) * kFS + 32 + k);
+      const float xv[4] = {x4.x, x4.y, x4.z, x4.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float4 m4 = *reinterpret_cast<const float4*>(M + (k + u) * 32 + c);
+        y[0] -= xv[u] * m4.x; y[1] -= xv[u] * m4.y;
+        y[2] -= xv[u] * m4.z; y[3] -= xv[u] * m4.w;
+      }
+    }
+    *reinterpret_cast<float4*>(X + (32 + r) * kFS + c) =
+        make_float4(y[0], y[1], y[2], y[3]);
+  }
+  __syncthreads();
 }
 
 // Store `n` consecutive 16-byte chunks (8 bf16 each, starting at chunk
