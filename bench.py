@@ -441,16 +441,24 @@ def run_only(args, dev, stream):
 
 
 def load_traffic():
-    """Per-launch DRAM bytes from the committed ncu summaries, when the
-    kernels have not changed since (a small JSON beside the summaries)."""
+    """Per-launch DRAM bytes from the committed ncu captures
+    (profiles/traffic.json), kept only while the kernel source still has the
+    hash the capture was taken on."""
+    import hashlib
     p = os.path.join(ROOT, "profiles", "traffic.json")
-    if not os.path.exists(p):
-        return {}
+    out = {}
     try:
         with open(p) as f:
-            return json.load(f)
+            d = json.load(f)
+        for name, rec in d.items():
+            if name.startswith("_"):
+                continue
+            with open(os.path.join(ROOT, rec["file"]), "rb") as src:
+                if hashlib.sha256(src.read()).hexdigest() == rec["sha256"]:
+                    out[name] = rec["bytes"]
     except Exception:
         return {}
+    return out
 
 
 def main():
