@@ -710,6 +710,21 @@ bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+}  // namespace
+
+// bf16 [tokens, H, d] tensor, box of 64 channels x 64 tokens, 128-byte swizzle.
+bool make_tile_map(CUtensorMap* m, const void* base, int d, int H, int tokens) {
+  return make_map(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, H, tokens, 64,
+                  CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+}  // namespace kda
+
+#include "kda_fused_ws_sm100.cuh"
+
+namespace kda {
+namespace {
+
 int64_t total_tokens(const ChunkArgs& a) {
   return a.cu_seqlens ? (int64_t)a.T : (int64_t)a.n_seqs * a.T;
 }
@@ -782,8 +797,15 @@ cudaError_t fused_take_timeout(cudaStream_t stream, int* flag) {
 
 cudaError_t launch_fused(const ChunkArgs& a, void* workspace,
                          cudaStream_t stream) {
-  return a.dk == 128 ? run<128>(a, workspace, stream)
-                     : run<64>(a, workspace, stream);
+  const int32_t* order = nullptr;
+  if (a.cu_seqlens) {
+    int32_t* o = static_cast<int32_t*>(workspace);
+    order_kernel<<<1, 1024, 0, stream>>>(a.cu_seqlens, a.n_seqs, a.T, o);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    order = o;
+  }
+  return ws::launch_fused_ws(a, order, stream);
 }
 
 }  // namespace kda

@@ -1,0 +1,787 @@
+// Warp-specialised fused chunkwise KDA prefill for sm_100a.
+//
+// Same mathematics as the single-role kernel (see kda_fused_sm100.cu), split
+// into two roles that work on different chunks at the same time:
+//   producer (warps 0-7, 256 threads): for chunk n it forms the decay-scaled
+//     operands (prologue), A and P (MMA1), T' = (I + A)^-1 Diag(beta) (blocked
+//     inverse), W = T' Kt and U = T' V (MMA2), and hands them over in operand
+//     slot n mod 2;
+//   consumer (warps 8-11, 128 threads): for chunk n it forms W S and Qt S
+//     (MMA3), Delta = U - W S, the state update and the output (MMA4, MMA5).
+// While the consumer runs the serial state chain of chunk n the producer
+// works on chunk n + 1.  The slots are handed over by full/empty mbarriers.
+//
+// The state stays in TMEM in fp32.  The consumer uses the identity
+//   S_C = Diag(exp(g_C)) S_0 + Kh^T Delta = Diag(exp(g_C)) (S_0 + Kb^T Delta),
+// since Kh = Kb Diag(exp(g_C)) row-wise.  MMA4 therefore accumulates
+// Kb^T Delta straight onto the state, and the epilogue rescales each state row
+// by exp(g_C) (tcgen05.ld / tcgen05.st).  The separate Kh operand is not
+// needed.  log(alpha) is prefetched into the producer's registers with plain
+// global loads one chunk ahead; q, k and V arrive by TMA.
+// Included by kda_fused_sm100.cu (same translation unit: it shares the
+// device-side timeout flag and the tensor-map helper).
+#pragma once
+
+namespace kda {
+namespace ws {
+
+using namespace sm100;
+
+constexpr int kC = 64;
+constexpr int kDvt = 64;
+constexpr int kProd = 256;  // producer threads (warps 0-7)
+constexpr int kCons = 128;  // consumer threads (warps 8-11)
+constexpr int kThreads = kProd + kCons;
+constexpr int kFS = 68;     // fp32 row stride of the A / Tm tiles
+constexpr int kBarProd = 1, kBarCons = 2;  // named barrier ids
+
+template <int DK>
+struct WsLayout {
+  static constexpr uint32_t NP = DK / 64;
+  // producer-private
+  static constexpr uint32_t stage_q = 0;                    // NP x 8 KB
+  static constexpr uint32_t stage_k = stage_q + NP * 8192;  // NP x 8 KB
+  static constexpr uint32_t vbuf = stage_k + NP * 8192;     // 8 KB
+  static constexpr uint32_t afp = vbuf + 8192;              // 64 x kFS fp32
+  static constexpr uint32_t tfp = afp + 64 * kFS * 4;       // 64 x kFS fp32
+  static constexpr uint32_t msc = tfp + 64 * kFS * 4;       // 1024 fp32
+  static constexpr uint32_t tp = msc + 4096;                // T', 64 rows
+  // slots (two of each)
+  static constexpr uint32_t kq = tp + 8192;                 // [Kt/W; Qt]
+  static constexpr uint32_t kq_stride = NP * 16384;
+  static constexpr uint32_t kb = kq + 2 * kq_stride;        // Kb, 2 panels
+  static constexpr uint32_t pp = kb + 2 * 16384;            // P, 64 rows
+  // consumer-private
+  static constexpr uint32_t sop = pp + 2 * 8192;            // S, DK rows
+  static constexpr uint32_t dop = sop + DK * 128;           // Delta, 64 rows
+  static constexpr uint32_t misc = dop + 8192;
+  static constexpr uint32_t bytes = misc + 2048;
+  static constexpr uint32_t tx_qk = 2 * NP * 8192;
+  // TMEM columns
+  static constexpr uint32_t t_d1 = 0;
+  static constexpr uint32_t t_w = 64;
+  static constexpr uint32_t t_u0 = 64 + DK;
+  static constexpr uint32_t t_d3 = 192 + DK;
+  static constexpr uint32_t t_s = 256 + DK;
+  static_assert(tp % 1024 == 0 && kq % 1024 == 0, "swizzle atoms");
+};
+
+struct WsParams {
+  const float* beta;
+  const float* log_alpha;
+  const float* s_init;
+  float* s_final;
+  __nv_bfloat16* out;
+  const int32_t* cu;
+  const int32_t* order;
+  int n_seqs, T, H, dv, n_tiles;
+};
+
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+// Barrier over `n` threads that also returns whether any thread's `pred`
+// was set.
+__device__ __forceinline__ bool named_sync_or(int id, int n, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+// Bounded wait that also gives up when the other role has failed.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity,
+                                              volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > 2000000000ull) return false;
+  }
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, "
+      "%31, %32};" ::"r"(taddr),
+      "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]),
+      "f"(v[6]), "f"(v[7]), "f"(v[8]), "f"(v[9]), "f"(v[10]), "f"(v[11]),
+      "f"(v[12]), "f"(v[13]), "f"(v[14]), "f"(v[15]), "f"(v[16]), "f"(v[17]),
+      "f"(v[18]), "f"(v[19]), "f"(v[20]), "f"(v[21]), "f"(v[22]), "f"(v[23]),
+      "f"(v[24]), "f"(v[25]), "f"(v[26]), "f"(v[27]), "f"(v[28]), "f"(v[29]),
+      "f"(v[30]), "f"(v[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void st_chunks(uint8_t* panel, int row, int c0,
+                                          const float* v) {
+#pragma unroll
+  for (int c = 0; c < N; ++c) {
+    uint4 w;
+    w.x = pack_bf16x2(v[8 * c + 0], v[8 * c + 1]);
+    w.y = pack_bf16x2(v[8 * c + 2], v[8 * c + 3]);
+    w.z = pack_bf16x2(v[8 * c + 4], v[8 * c + 5]);
+    w.w = pack_bf16x2(v[8 * c + 6], v[8 * c + 7]);
+    *reinterpret_cast<uint4*>(panel + row * 128 + (((c0 + c) ^ (row & 7)) << 4)) =
+        w;
+  }
+}
+
+// (I + A)^-1 of the strictly-lower 64 x 64 A (row stride kFS) into X by
+// recursive doubling on unit-lower blocks,
+//   [L11 0; L21 L22]^-1 = [X11 0; -X22 L21 X11  X22]:
+// the four 16 x 16 diagonal blocks by forward substitution, then blocks
+// (1,0) and (3,2), then the 32 x 32 coupling block.  256 producer threads;
+// X's strictly-upper part outside the diagonal blocks must be zero.
+__device__ __forceinline__ void invert_unit_lower(const float* A, float* X,
+                                                  float* M, int t) {
+  if (t < 64) {
+    const int o = (t >> 4) * 16, j = t & 15;
+    float x[16];
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+      float a[16];
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        if (4 * q4 < r) {
+          const float4 v =
+              *reinterpret_cast<const float4*>(A + (o + r) * kFS + o + 4 * q4);
+          a[4 * q4] = v.x; a[4 * q4 + 1] = v.y; a[4 * q4 + 2] = v.z;
+          a[4 * q4 + 3] = v.w;
+        }
+      }
+      float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+      for (int i = 0; i < r; ++i) {
+        if (i & 1) s1 -= a[i] * x[i];
+        else s0 -= a[i] * x[i];
+      }
+      x[r] = r < j ? 0.f : (r == j ? 1.f : s0 + s1);
+    }
+#pragma unroll
+    for (int r = 0; r < 16; ++r) X[(o + r) * kFS + o + j] = x[r];
+  }
+  named_sync(kBarProd, kProd);
+  {
+    const int b = t >> 7, r = (t >> 3) & 15, c = (t & 7) * 2;
+    const int bi = 2 * b + 1, bj = 2 * b;
+    float m0 = 0.f, m1 = 0.f;
+#pragma unroll
+    for (int k = 0; k < 16; k += 4) {
+      const float4 a4 =
+          *reinterpret_cast<const float4*>(A + (16 * bi + r) * kFS + 16 * bj + k);
+      const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float2 x2 = *reinterpret_cast<const float2*>(
+            X + (16 * bj + k + u) * kFS + 16 * bj + c);
+        m0 += av[u] * x2.x;
+        m1 += av[u] * x2.y;
+      }
+    }
+    *reinterpret_cast<float2*>(M + b * 256 + r * 16 + c) = make_float2(m0, m1);
+    named_sync(kBarProd, kProd);
+    float y0 = 0.f, y1 = 0.f;
+#pragma unroll
+    for (int k = 0; k < 16; k += 4) {
+      const float4 x4 =
+          *reinterpret_cast<const float4*>(X + (16 * bi + r) * kFS + 16 * bi + k);
+      const float xv[4] = {x4.x, x4.y, x4.z, x4.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float2 m2 =
+            *reinterpret_cast<const float2*>(M + b * 256 + (k + u) * 16 + c);
+        y0 -= xv[u] * m2.x;
+        y1 -= xv[u] * m2.y;
+      }
+    }
+    *reinterpret_cast<float2*>(X + (16 * bi + r) * kFS + 16 * bj + c) =
+        make_float2(y0, y1);
+  }
+  named_sync(kBarProd, kProd);
+  {
+    const int r = t >> 3, c = (t & 7) * 4;
+    float m[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int k = 0; k < 32; k += 4) {
+      const float4 a4 = *reinterpret_cast<const float4*>(A + (32 + r) * kFS + k);
+      const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float4 x4 = *reinterpret_cast<const float4*>(X + (k + u) * kFS + c);
+        m[0] += av[u] * x4.x; m[1] += av[u] * x4.y;
+        m[2] += av[u] * x4.z; m[3] += av[u] * x4.w;
+      }
+    }
+    *reinterpret_cast<float4*>(M + r * 32 + c) = make_float4(m[0], m[1], m[2], m[3]);
+    named_sync(kBarProd, kProd);
+    float y[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int k = 0; k < 32; k += 4) {
+      const float4 x4 =
+          *reinterpret_cast<const float4*>(X + (32 + r) * kFS + 32 + k);
+      const float xv[4] = {x4.x, x4.y, x4.z, x4.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float4 m4 = *reinterpret_cast<const float4*>(M + (k + u) * 32 + c);
+        y[0] -= xv[u] * m4.x; y[1] -= xv[u] * m4.y;
+        y[2] -= xv[u] * m4.z; y[3] -= xv[u] * m4.w;
+      }
+    }
+    *reinterpret_cast<float4*>(X + (32 + r) * kFS + c) =
+        make_float4(y[0], y[1], y[2], y[3]);
+  }
+  named_sync(kBarProd, kProd);
+}
+
+template <int DK>
+__global__ void __launch_bounds__(kThreads, 1)
+    fused_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
+                    const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v,
+                    const WsParams p) {
+  using Lay = WsLayout<DK>;
+  constexpr int NCG = DK / 4;        // producer prologue: 4-channel groups
+  constexpr int NRB = kProd / NCG;   // row blocks
+  constexpr int RPT = kC / NRB;      // rows per producer thread
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* st_q = sm + Lay::stage_q;
+  uint8_t* st_k = sm + Lay::stage_k;
+  uint8_t* vbuf = sm + Lay::vbuf;
+  float* afp = reinterpret_cast<float*>(sm + Lay::afp);
+  float* tfp = reinterpret_cast<float*>(sm + Lay::tfp);
+  float* msc = reinterpret_cast<float*>(sm + Lay::msc);
+  uint8_t* tp = sm + Lay::tp;
+  uint8_t* sop = sm + Lay::sop;
+  uint8_t* dop = sm + Lay::dop;
+  float* beta_s = reinterpret_cast<float*>(sm + Lay::misc);         // [64]
+  float* gcs = reinterpret_cast<float*>(sm + Lay::misc + 256);      // [2][DK]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Lay::misc + 1280);
+  uint64_t* bar_in = bars + 0;
+  uint64_t* bar_v = bars + 1;
+  uint64_t* bar_pm = bars + 2;
+  uint64_t* bar_cm = bars + 3;
+  uint64_t* full = bars + 4;   // [2]
+  uint64_t* empty = bars + 6;  // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 9);
+
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+  const int u = blockIdx.x;
+  const int tile = u % p.n_tiles;
+  const int h = (u / p.n_tiles) % p.H;
+  const int rank = u / (p.n_tiles * p.H);
+  const int seq = p.order ? p.order[rank] : rank;
+  const int j0 = tile * kDvt;
+  int start, end;
+  seq_range(p.cu, seq, p.T, &start, &end);
+  const int nch = (end - start + kC - 1) / kC;
+
+  if (tid == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+    mbar_init(bar_in, 1);
+    mbar_init(bar_v, 1);
+    mbar_init(bar_pm, 1);
+    mbar_init(bar_cm, 1);
+    mbar_init(full + 0, 1);
+    mbar_init(full + 1, 1);
+    mbar_init(empty + 0, 1);
+    mbar_init(empty + 1, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  for (int i = tid; i < 64 * kFS; i += kThreads) tfp[i] = 0.f;
+  if (DK == 64) {  // the second M-panel of each Kb slot stays zero
+    for (int i = tid; i < 2 * 512; i += kThreads) {
+      uint4* z = reinterpret_cast<uint4*>(sm + Lay::kb + (i >> 9) * 16384 + 8192);
+      z[i & 511] = make_uint4(0, 0, 0, 0);
+    }
+  }
+  fence_proxy_async();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  bool failed = false;
+
+  if (tid < kProd) {
+    // =================================================== producer role
+    const int t = tid;
+    const int colh = warp >> 2;  // 32-column half of a 64-column accumulator
+    const int row_t = t & 127;
+    const int cg = t % NCG, rb = t / NCG;
+    const int pnl = cg >> 4, ck = (cg >> 1) & 7, cb = (cg & 1) * 8;
+    const float* la_g = p.log_alpha + (size_t)h * DK + 4 * cg;
+    const size_t la_stride = (size_t)p.H * DK;
+
+    auto issue_qk = [&](int tok) {
+      mbar_arrive_expect_tx(bar_in, Lay::tx_qk);
+#pragma unroll
+      for (int q = 0; q < (int)Lay::NP; ++q) {
+        tma_load_3d(st_q + q * 8192, &tm_q, bar_in, q * 64, h, tok);
+        tma_load_3d(st_k + q * 8192, &tm_k, bar_in, q * 64, h, tok);
+      }
+    };
+    auto issue_v = [&](int tok) {
+      mbar_arrive_expect_tx(bar_v, 8192);
+      tma_load_3d(vbuf, &tm_v, bar_v, j0, h, tok);
+    };
+    float4 la_reg[RPT];
+    auto load_la = [&](int tok0, int L) {
+#pragma unroll
+      for (int i = 0; i < RPT; ++i) {
+        const int r = rb * RPT + i;
+        la_reg[i] = r < L ? __ldg(reinterpret_cast<const float4*>(
+                                la_g + (size_t)(tok0 + r) * la_stride))
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    };
+
+    if (t == 0 && nch > 0) {
+      issue_qk(start);
+      issue_v(start);
+    }
+    float beta_next = 0.f;
+    if (nch > 0) {
+      load_la(start, min(kC, end - start));
+      if (t < kC && t < end - start)
+        beta_next = p.beta[(size_t)(start + t) * p.H + h];
+    }
+    uint32_t ph_in = 0, ph_v = 0, ph_pm = 0;
+    bool in_flight = nch > 0, v_pending = nch > 0;
+
+    for (int n = 0; n < nch; ++n) {
+      const int s = n & 1, use = n >> 1;
+      const int tok0 = start + n * kC;
+      const int L = min(kC, end - tok0);
+      const bool has_next = n + 1 < nch;
+      uint8_t* kq = sm + Lay::kq + s * Lay::kq_stride;
+      uint8_t* kb = sm + Lay::kb + s * 16384;
+      uint8_t* pp = sm + Lay::pp + s * 8192;
+      float* gc = gcs + s * DK;
+      if (t < kC) {
+        beta_s[t] = beta_next;
+        beta_next = 0.f;
+        if (has_next && t < end - (tok0 + kC))
+          beta_next = p.beta[(size_t)(tok0 + kC + t) * p.H + h];
+      }
+      bool ok = true;
+      if (use >= 1) ok = wait_or_abort(empty + s, (use - 1) & 1, abort_flag);
+      ok = ok && wait_or_abort(bar_in, ph_in, abort_flag);
+      ph_in ^= 1;
+      in_flight = false;
+      if (named_sync_or(kBarProd, kProd, !ok)) { failed = true; break; }
+
+      // ---- prologue (log(alpha) rows already in registers)
+      {
+        float part[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int i = 0; i < RPT; ++i) {
+          part[0] += la_reg[i].x; part[1] += la_reg[i].y;
+          part[2] += la_reg[i].z; part[3] += la_reg[i].w;
+        }
+        float* red = afp;  // free until the A extraction below
+        *reinterpret_cast<float4*>(red + rb * DK + 4 * cg) =
+            make_float4(part[0], part[1], part[2], part[3]);
+        named_sync(kBarProd, kProd);
+        float g[4] = {0.f, 0.f, 0.f, 0.f}, tot[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int b2 = 0; b2 < NRB; ++b2) {
+          const float4 y = *reinterpret_cast<const float4*>(red + b2 * DK + 4 * cg);
+          if (b2 < rb) { g[0] += y.x; g[1] += y.y; g[2] += y.z; g[3] += y.w; }
+          tot[0] += y.x; tot[1] += y.y; tot[2] += y.z; tot[3] += y.w;
+        }
+        constexpr float kLog2e = 1.4426950408889634f;
+        if (rb == 0)
+          *reinterpret_cast<float4*>(gc + 4 * cg) =
+              make_float4(ex2_approx(tot[0] * kLog2e), ex2_approx(tot[1] * kLog2e),
+                          ex2_approx(tot[2] * kLog2e), ex2_approx(tot[3] * kLog2e));
+        const uint8_t* pq = st_q + pnl * 8192;
+        const uint8_t* pk = st_k + pnl * 8192;
+        uint8_t* pkq = kq + pnl * 16384;
+        uint8_t* pkb = kb + pnl * 8192;
+#pragma unroll
+        for (int i = 0; i < RPT; ++i) {
+          const int r = rb * RPT + i;
+          const uint32_t off = r * 128 + ((ck ^ (r & 7)) << 4) + cb;
+          const bool valid = r < L;
+          const uint2 kr = *reinterpret_cast<const uint2*>(pk + off);
+          const uint2 qr = *reinterpret_cast<const uint2*>(pq + off);
+          g[0] += la_reg[i].x; g[1] += la_reg[i].y;
+          g[2] += la_reg[i].z; g[3] += la_reg[i].w;
+          float e[4], ie[4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const float x = g[c] * kLog2e;
+            e[c] = valid ? ex2_approx(x) : 0.f;
+            ie[c] = valid ? ex2_approx(-x) : 0.f;
+          }
+          const __nv_bfloat162 e01 = __floats2bfloat162_rn(e[0], e[1]);
+          const __nv_bfloat162 e23 = __floats2bfloat162_rn(e[2], e[3]);
+          const __nv_bfloat162 i01 = __floats2bfloat162_rn(ie[0], ie[1]);
+          const __nv_bfloat162 i23 = __floats2bfloat162_rn(ie[2], ie[3]);
+          const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kr);
+          const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&qr);
+          uint2 wt, wq, wb;
+          *reinterpret_cast<__nv_bfloat162*>(&wt.x) = __hmul2(k2[0], e01);
+          *reinterpret_cast<__nv_bfloat162*>(&wt.y) = __hmul2(k2[1], e23);
+          *reinterpret_cast<__nv_bfloat162*>(&wq.x) = __hmul2(q2[0], e01);
+          *reinterpret_cast<__nv_bfloat162*>(&wq.y) = __hmul2(q2[1], e23);
+          *reinterpret_cast<__nv_bfloat162*>(&wb.x) = __hmul2(k2[0], i01);
+          *reinterpret_cast<__nv_bfloat162*>(&wb.y) = __hmul2(k2[1], i23);
+          *reinterpret_cast<uint2*>(pkq + off) = wt;
+          *reinterpret_cast<uint2*>(pkq + 64 * 128 + off) = wq;
+          *reinterpret_cast<uint2*>(pkb + off) = wb;
+        }
+      }
+      if (has_next) load_la(tok0 + kC, min(kC, end - (tok0 + kC)));
+      fence_proxy_async();
+      named_sync(kBarProd, kProd);
+
+      // ---- MMA1: [Kt; Qt] . Kb^T ; next chunk's q, k into the staging
+      if (t == 0) {
+        tc_fence_after();
+        const uint32_t idesc = idesc_bf16(128, 64, false, false);
+#pragma unroll
+        for (int ks = 0; ks < DK / 16; ++ks) {
+          const uint32_t off = (ks & 3) * 32;
+          mma_bf16(tmem + Lay::t_d1,
+                   desc_sw128(smem_u32(kq) + (ks >> 2) * 16384 + off, 16, 1024),
+                   desc_sw128(smem_u32(kb) + (ks >> 2) * 8192 + off, 16, 1024),
+                   idesc, ks > 0);
+        }
+        mma_commit(bar_pm);
+        if (has_next) issue_qk(tok0 + kC);
+      }
+      in_flight = has_next;
+      ok = wait_or_abort(bar_pm, ph_pm, abort_flag);
+      ph_pm ^= 1;
+      if (named_sync_or(kBarProd, kProd, !ok)) { failed = true; break; }
+      tc_fence_after();
+
+      // ---- A (fp32) and P (bf16 into the slot)
+      {
+        float v[32];
+        tmem_ld32(tmem + lane_base + Lay::t_d1 + 32 * colh, v);
+        if (row_t < 64) {
+          const float b = beta_s[row_t];
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            const int c = 32 * colh + i;
+            float4 w;
+            w.x = c + 0 < row_t ? b * v[i + 0] : 0.f;
+            w.y = c + 1 < row_t ? b * v[i + 1] : 0.f;
+            w.z = c + 2 < row_t ? b * v[i + 2] : 0.f;
+            w.w = c + 3 < row_t ? b * v[i + 3] : 0.f;
+            *reinterpret_cast<float4*>(afp + row_t * kFS + c) = w;
+          }
+        } else {
+          const int r = row_t - 64;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = 32 * colh + i <= r ? v[i] : 0.f;
+          st_chunks<4>(pp, r, 4 * colh, v);
+        }
+      }
+      tc_fence_before();
+      named_sync(kBarProd, kProd);
+
+      invert_unit_lower(afp, tfp, msc, t);
+
+      {  // T' = Tm Diag(beta), rows masked to the lower triangle
+        const int r = t & 63, qc = t >> 6;
+        float v[16];
+#pragma unroll
+        for (int i = 0; i < 16; i += 4) {
+          const int c = 16 * qc + i;
+          const float4 x = *reinterpret_cast<const float4*>(tfp + r * kFS + c);
+          const float4 b = *reinterpret_cast<const float4*>(beta_s + c);
+          v[i] = c + 0 <= r ? x.x * b.x : 0.f;
+          v[i + 1] = c + 1 <= r ? x.y * b.y : 0.f;
+          v[i + 2] = c + 2 <= r ? x.z * b.z : 0.f;
+          v[i + 3] = c + 3 <= r ? x.w * b.w : 0.f;
+        }
+        st_chunks<2>(tp, r, 2 * qc, v);
+      }
+      fence_proxy_async();
+      named_sync(kBarProd, kProd);
+
+      // ---- MMA2: W = T' Kt (N = DK), U = T' V (N = 64) into U slot s
+      if (t == 0) {
+        tc_fence_after();
+        ok = wait_or_abort(bar_v, ph_v, abort_flag);
+        ph_v ^= 1;
+        v_pending = !ok;
+        if (ok) {
+          const uint32_t iw = idesc_bf16(128, DK, false, true);
+          const uint32_t iu = idesc_bf16(128, 64, false, true);
+#pragma unroll
+          for (int ks = 0; ks < kC / 16; ++ks) {
+            const uint64_t a = desc_sw128(smem_u32(tp) + ks * 32, 16, 1024);
+            mma_bf16(tmem + Lay::t_w, a,
+                     desc_sw128(smem_u32(kq) + ks * 2048, 16384, 1024), iw,
+                     ks > 0);
+            mma_bf16(tmem + Lay::t_u0 + 64 * s, a,
+                     desc_sw128(smem_u32(vbuf) + ks * 2048, 8192, 1024), iu,
+                     ks > 0);
+          }
+          mma_commit(bar_pm);
+        }
+      }
+      if (named_sync_or(kBarProd, kProd, !ok)) { failed = true; break; }
+      ok = wait_or_abort(bar_pm, ph_pm, abort_flag);
+      ph_pm ^= 1;
+      if (named_sync_or(kBarProd, kProd, !ok)) { failed = true; break; }
+      tc_fence_after();
+      if (t == 0 && has_next) {
+        issue_v(tok0 + kC);
+        v_pending = true;
+      }
+
+      // ---- W rows (bf16) over the Kt rows of the slot's [Kt; Qt]
+      if (row_t < 64) {
+#pragma unroll
+        for (int j = 0; j < DK / 64; ++j) {
+          const int hh = colh * (DK / 64) + j;
+          float v[32];
+          tmem_ld32(tmem + lane_base + Lay::t_w + 32 * hh, v);
+          st_chunks<4>(kq + (hh >> 1) * 16384, row_t, 4 * (hh & 1), v);
+        }
+      }
+      tc_fence_before();
+      fence_proxy_async();
+      named_sync(kBarProd, kProd);
+      if (t == 0) mbar_arrive(full + s);
+    }
+    if (failed && t == 0) {
+      *abort_flag = 1;
+      atomicExch(&g_fused_timeout, 1);
+      if (in_flight) mbar_wait(bar_in, ph_in, 100000000ull);
+      if (v_pending) mbar_wait(bar_v, ph_v, 100000000ull);
+    }
+  } else {
+    // =================================================== consumer role
+    const int c = tid - kProd;  // TMEM lane = accumulator row
+    const bool owns_state = c < DK;
+    const size_t sbase = (((size_t)seq * p.H + h) * DK) * p.dv + j0;
+    if (owns_state) {  // initial state into TMEM (fp32) and the bf16 operand
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        float v[32];
+        if (p.s_init) {
+          const float4* src = reinterpret_cast<const float4*>(
+              p.s_init + sbase + (size_t)c * p.dv + 32 * hf);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float4 x = src[i];
+            v[4 * i] = x.x; v[4 * i + 1] = x.y; v[4 * i + 2] = x.z;
+            v[4 * i + 3] = x.w;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = 0.f;
+        }
+        tmem_st32(tmem + lane_base + Lay::t_s + 32 * hf, v);
+        st_chunks<4>(sop, c, 4 * hf, v);
+      }
+      tmem_wait_st();
+    }
+    tc_fence_before();
+    fence_proxy_async();
+    named_sync(kBarCons, kCons);
+    uint32_t ph_cm = 0;
+
+    for (int n = 0; n < nch; ++n) {
+      const int s = n & 1, use = n >> 1;
+      const int tok0 = start + n * kC;
+      const int L = min(kC, end - tok0);
+      uint8_t* kq = sm + Lay::kq + s * Lay::kq_stride;
+      uint8_t* kb = sm + Lay::kb + s * 16384;
+      uint8_t* pp = sm + Lay::pp + s * 8192;
+      bool ok = wait_or_abort(full + s, use & 1, abort_flag);
+      if (named_sync_or(kBarCons, kCons, !ok)) { failed = true; break; }
+      tc_fence_after();
+
+      // ---- MMA3: [W; Qt] . S
+      if (c == 0) {
+        const uint32_t idesc = idesc_bf16(128, 64, false, true);
+#pragma unroll
+        for (int ks = 0; ks < DK / 16; ++ks)
+          mma_bf16(tmem + Lay::t_d3,
+                   desc_sw128(smem_u32(kq) + (ks >> 2) * 16384 + (ks & 3) * 32,
+                              16, 1024),
+                   desc_sw128(smem_u32(sop) + ks * 2048, 8192, 1024), idesc,
+                   ks > 0);
+        mma_commit(bar_cm);
+      }
+      ok = wait_or_abort(bar_cm, ph_cm, abort_flag);
+      ph_cm ^= 1;
+      if (named_sync_or(kBarCons, kCons, !ok)) { failed = true; break; }
+      tc_fence_after();
+
+      // ---- Delta = U - W S (rows 0-63)
+      if (c < 64) {
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          float uu[32], ws[32];
+          tmem_ld32(tmem + lane_base + Lay::t_u0 + 64 * s + 32 * hf, uu);
+          tmem_ld32(tmem + lane_base + Lay::t_d3 + 32 * hf, ws);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) uu[i] -= ws[i];
+          st_chunks<4>(dop, c, 4 * hf, uu);
+        }
+      }
+      const float gamma = owns_state ? gcs[s * DK + c] : 1.f;
+      tc_fence_before();
+      fence_proxy_async();
+      named_sync(kBarCons, kCons);
+
+      // ---- MMA4: S += Kb^T Delta ; MMA5: rows 64-127 += P Delta
+      if (c == 0) {
+        tc_fence_after();
+        const uint32_t i4 = idesc_bf16(128, 64, true, true);
+        const uint32_t i5 = idesc_bf16(128, 64, false, true);
+#pragma unroll
+        for (int ks = 0; ks < kC / 16; ++ks) {
+          const uint64_t bd = desc_sw128(smem_u32(dop) + ks * 2048, 8192, 1024);
+          mma_bf16(tmem + Lay::t_s,
+                   desc_sw128(smem_u32(kb) + ks * 2048, 8192, 1024), bd, i4, 1u);
+          mma_bf16(tmem + Lay::t_d3,
+                   desc_sw128(smem_u32(pp) - 8192 + ks * 32, 16, 1024), bd, i5,
+                   1u);
+        }
+        mma_commit(bar_cm);
+      }
+      ok = wait_or_abort(bar_cm, ph_cm, abort_flag);
+      ph_cm ^= 1;
+      if (named_sync_or(kBarCons, kCons, !ok)) { failed = true; break; }
+      tc_fence_after();
+      if (c == 0) mbar_arrive(empty + s);  // slot s (and U slot s) consumed
+
+      // ---- outputs (rows 64-127) and the state rescale by exp(g_C)
+      if (c >= 64) {
+        const int r = c - 64;
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          float o[32];
+          tmem_ld32(tmem + lane_base + Lay::t_d3 + 32 * hf, o);
+          if (r < L) {
+            uint4* dst = reinterpret_cast<uint4*>(
+                p.out + ((size_t)(tok0 + r) * p.H + h) * p.dv + j0 + 32 * hf);
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+              uint4 w;
+              w.x = pack_bf16x2(o[8 * ch + 0], o[8 * ch + 1]);
+              w.y = pack_bf16x2(o[8 * ch + 2], o[8 * ch + 3]);
+              w.z = pack_bf16x2(o[8 * ch + 4], o[8 * ch + 5]);
+              w.w = pack_bf16x2(o[8 * ch + 6], o[8 * ch + 7]);
+              dst[ch] = w;
+            }
+          }
+        }
+      }
+      if (owns_state) {
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          float v[32];
+          tmem_ld32(tmem + lane_base + Lay::t_s + 32 * hf, v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] *= gamma;
+          tmem_st32(tmem + lane_base + Lay::t_s + 32 * hf, v);
+          st_chunks<4>(sop, c, 4 * hf, v);
+        }
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      fence_proxy_async();
+      named_sync(kBarCons, kCons);
+    }
+    if (failed) {
+      *abort_flag = 1;
+      if (c == 0) atomicExch(&g_fused_timeout, 1);
+    } else if (owns_state) {
+      tc_fence_after();
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        float v[32];
+        tmem_ld32(tmem + lane_base + Lay::t_s + 32 * hf, v);
+        float4* dst = reinterpret_cast<float4*>(p.s_final + sbase +
+                                                (size_t)c * p.dv + 32 * hf);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+// Host side: tensor maps for q, k, v and the launch, one CTA per (sequence,
+// head, 64-column d_v tile).
+template <int DK>
+cudaError_t run_ws(const ChunkArgs& a, const int32_t* order,
+                   cudaStream_t stream) {
+  using Lay = WsLayout<DK>;
+  const int tokens = a.cu_seqlens ? a.T : a.n_seqs * a.T;
+  CUtensorMap tq, tk, tv;
+  if (!make_tile_map(&tq, a.q, DK, a.H, tokens) ||
+      !make_tile_map(&tk, a.k, DK, a.H, tokens) ||
+      !make_tile_map(&tv, a.v, a.dv, a.H, tokens))
+    return cudaErrorInvalidValue;
+  WsParams p{};
+  p.beta = a.beta;
+  p.log_alpha = a.log_alpha;
+  p.s_init = a.initial_state;
+  p.s_final = a.final_state;
+  p.out = static_cast<__nv_bfloat16*>(a.out);
+  p.cu = a.cu_seqlens;
+  p.order = order;
+  p.n_seqs = a.n_seqs;
+  p.T = a.T;
+  p.H = a.H;
+  p.dv = a.dv;
+  p.n_tiles = a.dv / kDvt;
+  const size_t smem = Lay::bytes + 1024;
+  cudaError_t e = cudaFuncSetAttribute(
+      fused_ws_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      (int)smem);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = (unsigned)a.n_seqs * a.H * p.n_tiles;
+  fused_ws_kernel<DK><<<grid, kThreads, smem, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+inline cudaError_t launch_fused_ws(const ChunkArgs& a, const int32_t* order,
+                                   cudaStream_t stream) {
+  return a.dk == 128 ? run_ws<128>(a, order, stream)
+                     : run_ws<64>(a, order, stream);
+}
+
+}  // namespace ws
+}  // namespace kda
