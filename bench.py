@@ -306,6 +306,33 @@ def run_kda(args, world, rank, local):
     d_gbs = world * dbytes / (d_step_ms * 1e-3) / 1e9
     d_launch_gbs = dbytes / (statistics.mean(dper) * 1e-3) / 1e9
 
+    # ---- per-head gate (Gated DeltaNet layout): same shapes, 4 B of gate per
+    # token and head instead of 4 d_k B --------------------------------------
+    lh = d["log_alpha"][..., 0].contiguous()
+
+    def prefill_head(_i):
+        K.chunk_fwd(d["q"], d["k"], d["v"], lh, d["beta"], None, None,
+                    chunk=C, out=out, final_state=fin, gate="head")
+
+    for i in range(args.warmup):
+        prefill_head(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    hms, hper = timed(prefill_head, args.steps, stream)
+    barrier(world)
+    hms = max_over_ranks(hms, world)
+    hbytes = prefill_bytes(B, T, H, dk, dv) - B * T * H * dk * 4 + B * T * H * 4
+    h_launch = statistics.mean(hper)
+    head_gate = {
+        "value": world * B * T / (hms / args.steps * 1e-3), "unit": "tokens/s",
+        "ms_per_step": hms / args.steps,
+        "workload": "as the prefill, log_alpha [B,T,H] (one gate per head)",
+        "hbm": {"achieved": hbytes / (h_launch * 1e-3) / 1e9, "unit": "GB/s",
+                "frac": hbytes / (h_launch * 1e-3) / 1e9 / pk["hbm_gbs"],
+                "algorithmic_bytes_per_launch": hbytes},
+        "tensor_frac": pflops / (h_launch * 1e-3) / 1e12 / pk["bf16_tflops"],
+    }
+
     # ---- end to end through the public API with host buffers ------------
     host = {n: d[n].cpu().pin_memory() for n in
             ("q", "k", "v", "log_alpha", "beta")}
@@ -394,10 +421,13 @@ def run_kda(args, world, rank, local):
                              "algorithmic_bytes_per_launch": dbytes},
                 "gpu_launches": args.steps,
             },
+            "prefill_head_gate": head_gate,
             "e2e": {"value": e2e_value, "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": e2e_steps},
             "gpu_launches": n_kernels * args.steps,
+            "gpu_launches_note": "kernel launches inside the headline prefill "
+                                 "timed region (one fused kernel per call)",
             "clocks": clk,
             "cpu_baseline": cpu,
         }

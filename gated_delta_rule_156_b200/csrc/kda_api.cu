@@ -82,21 +82,28 @@ void fill_args(const kda_shape* s, int n_seqs, kda::ChunkArgs* a) {
 kda_status validate_chunk(const kda_shape* s, const void* q, const void* k,
                           const void* v, const float* la, const float* beta,
                           const float* s_init, const int32_t* cu, void* out,
-                          float* s_final, kda::ChunkArgs* a) {
+                          float* s_final, kda::ChunkArgs* a,
+                          int gate = kda::kGateChannel) {
   int n_seqs = 0;
   const kda_status st = validate_chunk_shape(s, cu != nullptr, &n_seqs);
   if (st != KDA_OK) return st;
+  if (gate != kda::kGateChannel && gate != kda::kGateHead &&
+      gate != kda::kGateNone)
+    return KDA_ERR_INVALID_ARG;
   const size_t esz = s->io_dtype == KDA_BF16 ? 2 : 4;
   const size_t tokens = (size_t)s->B * (size_t)s->T;
   const size_t H = s->H;
   const bool any_tokens = tokens > 0;
   const bool any_state = n_seqs > 0;
-  if (any_tokens && (!q || !k || !v || !la || !beta || !out))
-    return KDA_ERR_INVALID_ARG;
+  if (gate == kda::kGateNone) la = nullptr;  // alpha = 1: no gate tensor
+  if (any_tokens && (!q || !k || !v || !beta || !out)) return KDA_ERR_INVALID_ARG;
+  if (any_tokens && gate != kda::kGateNone && !la) return KDA_ERR_INVALID_ARG;
   if (any_state && !s_final) return KDA_ERR_INVALID_ARG;
-  const void* ptrs[] = {q, k, v, la, s_init, out, s_final};
+  const void* ptrs[] = {q, k, v, s_init, out, s_final};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
+  if (la && !(gate == kda::kGateChannel ? aligned16(la) : aligned4(la)))
+    return KDA_ERR_MISALIGNED;
   if ((beta && !aligned4(beta)) || (cu && !aligned4(cu)))
     return KDA_ERR_MISALIGNED;
   // The output may alias no input; the final state may only coincide exactly
@@ -104,7 +111,7 @@ kda_status validate_chunk(const kda_shape* s, const void* q, const void* k,
   const Range rq = span(q, tokens * H * s->dk * esz),
               rk = span(k, tokens * H * s->dk * esz),
               rv = span(v, tokens * H * s->dv * esz),
-              rl = span(la, tokens * H * s->dk * 4),
+              rl = span(la, tokens * H * (gate == kda::kGateChannel ? s->dk : 1) * 4),
               rb = span(beta, tokens * H * 4),
               ro = span(out, tokens * H * s->dv * esz),
               rsi = span(s_init, (size_t)n_seqs * H * s->dk * s->dv * 4),
@@ -126,6 +133,7 @@ kda_status validate_chunk(const kda_shape* s, const void* q, const void* k,
   a->out = out;
   a->final_state = s_final;
   fill_args(s, n_seqs, a);
+  a->gate = gate;
   return KDA_OK;
 }
 
@@ -217,6 +225,23 @@ kda_status kda_chunk_fwd_staged(const kda_shape* shape, const void* q,
   return run_with_workspace(kda::staged_workspace_bytes(a), stream, false, a);
 }
 
+kda_status kda_chunk_fwd_gated(const kda_shape* shape, int gate, const void* q,
+                               const void* k, const void* v,
+                               const float* log_gate, const float* beta,
+                               const float* initial_state,
+                               const int32_t* cu_seqlens, void* out,
+                               float* final_state, int staged,
+                               cudaStream_t stream) {
+  kda::ChunkArgs a{};
+  const kda_status st = validate_chunk(shape, q, k, v, log_gate, beta,
+                                       initial_state, cu_seqlens, out,
+                                       final_state, &a, gate);
+  if (st != KDA_OK) return st;
+  if (!staged && kda::fused_supported(a))
+    return run_with_workspace(kda::fused_workspace_bytes(a), stream, true, a);
+  return run_with_workspace(kda::staged_workspace_bytes(a), stream, false, a);
+}
+
 kda_status kda_chunk_fwd_staged_noalloc(
     const kda_shape* shape, const void* q, const void* k, const void* v,
     const float* log_alpha, const float* beta, const float* initial_state,
@@ -241,7 +266,19 @@ kda_status kda_recurrent_step(const kda_shape* s, const void* q, const void* k,
                               const void* v, const float* log_alpha,
                               const float* beta, float* state_inout, void* out,
                               cudaStream_t stream) {
+  return kda_recurrent_step_gated(s, KDA_GATE_CHANNEL, q, k, v, log_alpha,
+                                  beta, state_inout, out, stream);
+}
+
+kda_status kda_recurrent_step_gated(const kda_shape* s, int gate, const void* q,
+                                    const void* k, const void* v,
+                                    const float* log_alpha, const float* beta,
+                                    float* state_inout, void* out,
+                                    cudaStream_t stream) {
   if (!s) return KDA_ERR_INVALID_ARG;
+  if (gate != KDA_GATE_CHANNEL && gate != KDA_GATE_HEAD && gate != KDA_GATE_NONE)
+    return KDA_ERR_INVALID_ARG;
+  if (gate == KDA_GATE_NONE) log_alpha = nullptr;
   if (s->B < 0 || s->T < 0 || s->H < 1) return KDA_ERR_INVALID_ARG;
   if (s->io_dtype != KDA_BF16 && s->io_dtype != KDA_F32)
     return KDA_ERR_INVALID_ARG;
@@ -250,16 +287,21 @@ kda_status kda_recurrent_step(const kda_shape* s, const void* q, const void* k,
   const size_t tokens = (size_t)s->B * (size_t)s->T, H = s->H;
   if ((size_t)s->B * H > (size_t)INT32_MAX) return KDA_ERR_UNSUPPORTED;
   if (s->B > 0 && !state_inout) return KDA_ERR_INVALID_ARG;
-  if (tokens > 0 && (!q || !k || !v || !log_alpha || !beta || !out))
+  if (tokens > 0 && (!q || !k || !v || !beta || !out)) return KDA_ERR_INVALID_ARG;
+  if (tokens > 0 && gate != KDA_GATE_NONE && !log_alpha)
     return KDA_ERR_INVALID_ARG;
-  const void* ptrs[] = {q, k, v, log_alpha, state_inout, out};
+  const void* ptrs[] = {q, k, v, state_inout, out};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
+  if (log_alpha && !(gate == KDA_GATE_CHANNEL ? aligned16(log_alpha)
+                                               : aligned4(log_alpha)))
+    return KDA_ERR_MISALIGNED;
   if (beta && !aligned4(beta)) return KDA_ERR_MISALIGNED;
   const Range rq = span(q, tokens * H * s->dk * esz),
               rk = span(k, tokens * H * s->dk * esz),
               rv = span(v, tokens * H * s->dv * esz),
-              rl = span(log_alpha, tokens * H * s->dk * 4),
+              rl = span(log_alpha,
+                        tokens * H * (gate == KDA_GATE_CHANNEL ? s->dk : 1) * 4),
               rb = span(beta, tokens * H * 4),
               ro = span(out, tokens * H * s->dv * esz),
               rs = span(state_inout, (size_t)s->B * H * s->dk * s->dv * 4);
@@ -270,7 +312,7 @@ kda_status kda_recurrent_step(const kda_shape* s, const void* q, const void* k,
 
   kda::RecurrentArgs a{q, k, v, log_alpha, beta, state_inout, out,
                        s->B, s->T, s->H, s->dk, s->dv,
-                       s->io_dtype == KDA_BF16};
+                       s->io_dtype == KDA_BF16, gate};
   const cudaError_t e = kda::launch_recurrent(a, stream);
   return e == cudaSuccess ? KDA_OK : cuda_fail(e);
 }

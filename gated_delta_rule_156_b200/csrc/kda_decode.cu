@@ -16,7 +16,8 @@
 // every thread issues all of its state loads before it touches them.  The
 // column sums over d_k are a register partial per thread, then one pass over
 // the 8 row groups in shared memory.  With T > 1 the state stays in registers
-// across tokens and is written once at the end.
+// across tokens and is written once at the end.  The gate may also be one
+// value per head (Gated DeltaNet) or absent (alpha = 1, DeltaNet).
 #include "kda_common.cuh"
 #include "kda_internal.h"
 
@@ -32,7 +33,7 @@ __global__ void __launch_bounds__((DV / 4) * kRowGroups)
                      const IO* __restrict__ v,
                      const float* __restrict__ log_alpha,
                      const float* __restrict__ beta, float* __restrict__ state,
-                     IO* __restrict__ out, int T, int H) {
+                     IO* __restrict__ out, int T, int H, int gate) {
   constexpr int CG = DV / 4;          // float4 column groups
   constexpr int R = DK / kRowGroups;  // rows per thread
   constexpr int NT = CG * kRowGroups;
@@ -56,7 +57,9 @@ __global__ void __launch_bounds__((DV / 4) * kRowGroups)
     for (int c = tid; c < DK; c += NT) {
       s_k[c] = to_f32(k[ok + c]);
       s_q[c] = to_f32(q[ok + c]);
-      s_a[c] = __expf(log_alpha[ok + c]);
+      s_a[c] = gate == kGateChannel ? __expf(log_alpha[ok + c])
+               : gate == kGateHead  ? __expf(log_alpha[tok * H + h])
+                                    : 1.f;
     }
     for (int j = tid; j < DV; j += NT) s_v[j] = to_f32(v[ov + j]);
     if (tid < 32) {  // k . q, one warp
@@ -122,7 +125,7 @@ cudaError_t launch_dkdv(const RecurrentArgs& a, cudaStream_t stream) {
   recurrent_kernel<DK, DV, IO><<<grid, NT, 0, stream>>>(
       static_cast<const IO*>(a.q), static_cast<const IO*>(a.k),
       static_cast<const IO*>(a.v), a.log_alpha, a.beta, a.state,
-      static_cast<IO*>(a.out), a.T, a.H);
+      static_cast<IO*>(a.out), a.T, a.H, a.gate);
   return cudaGetLastError();
 }
 

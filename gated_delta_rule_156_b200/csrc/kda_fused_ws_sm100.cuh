@@ -55,14 +55,15 @@ struct WsLayout {
   static constexpr uint32_t sop = pp + 2 * 8192;            // S, DK rows
   static constexpr uint32_t dop = sop + DK * 128;           // Delta, 64 rows
   static constexpr uint32_t misc = dop + 8192;
-  static constexpr uint32_t bytes = misc + 2048;
+  static constexpr uint32_t bytes = misc + 2048;  // betas, gcs, barriers
   static constexpr uint32_t tx_qk = 2 * NP * 8192;
-  // TMEM columns
+  // TMEM columns: D1 (two buffers), W, U (two slots), D3, S
   static constexpr uint32_t t_d1 = 0;
-  static constexpr uint32_t t_w = 64;
-  static constexpr uint32_t t_u0 = 64 + DK;
-  static constexpr uint32_t t_d3 = 192 + DK;
-  static constexpr uint32_t t_s = 256 + DK;
+  static constexpr uint32_t t_w = 128;
+  static constexpr uint32_t t_u0 = 128 + DK;
+  static constexpr uint32_t t_d3 = 256 + DK;
+  static constexpr uint32_t t_s = 320 + DK;
+  static_assert(t_s + 64 <= 512, "TMEM columns");
   static_assert(tp % 1024 == 0 && kq % 1024 == 0, "swizzle atoms");
 };
 
@@ -98,13 +99,33 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar))
                : "memory");
 }
-// Bounded wait that also gives up when the other role has failed.
+// Bounded wait that also gives up when the other role has failed.  The
+// try_wait carries a suspend-time hint, so a waiting warp sleeps in the
+// barrier unit (issuing nothing) until the phase completes or 0.5 ms pass.
+__device__ __forceinline__ bool try_wait_sleep(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(500000u)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait, also abandoned when the other role has failed.  Waits on
+// the other role (slot full / empty) sleep in the barrier unit; waits on this
+// role's own MMAs and TMA copies, which end within microseconds, poll.
+template <bool kSleep>
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity,
                                               volatile int* abort_flag) {
-  if (mbar_try_wait(bar, parity)) return true;
+  auto once = [&]() {
+    return kSleep ? try_wait_sleep(bar, parity) : mbar_try_wait(bar, parity);
+  };
+  if (once()) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (once()) return true;
     if (*abort_flag) return false;
     if (globaltimer_ns() - t0 > 2000000000ull) return false;
   }
@@ -126,6 +147,26 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
 }
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Predicated loads into registers that keep their old value when `pred` is
+// false: no select follows the load, so nothing waits for it until the value
+// is used (the prefetches below are used one chunk later).
+__device__ __forceinline__ void ldg_f4_if(float4& v, const float* p, bool pred) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\t"
+      "setp.ne.u32 q, %4, 0;\n\t"
+      "@q ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%5];\n\t}"
+      : "+f"(v.x), "+f"(v.y), "+f"(v.z), "+f"(v.w)
+      : "r"((uint32_t)pred), "l"(p));
+}
+__device__ __forceinline__ void ldg_f1_if(float& v, const float* p, bool pred) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "@q ld.global.nc.f32 %0, [%2];\n\t}"
+      : "+f"(v)
+      : "r"((uint32_t)pred), "l"(p));
 }
 
 template <int N>
@@ -250,7 +291,7 @@ __device__ __forceinline__ void invert_unit_lower(const float* A, float* X,
   named_sync(kBarProd, kProd);
 }
 
-template <int DK>
+template <int DK, int GATE>
 __global__ void __launch_bounds__(kThreads, 1)
     fused_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
@@ -268,21 +309,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* vbuf = sm + Lay::vbuf;
   float* afp = reinterpret_cast<float*>(sm + Lay::afp);
   float* tfp = reinterpret_cast<float*>(sm + Lay::tfp);
-  float* msc = reinterpret_cast<float*>(sm + Lay::msc);
   uint8_t* tp = sm + Lay::tp;
   uint8_t* sop = sm + Lay::sop;
   uint8_t* dop = sm + Lay::dop;
-  float* beta_s = reinterpret_cast<float*>(sm + Lay::misc);         // [64]
-  float* gcs = reinterpret_cast<float*>(sm + Lay::misc + 256);      // [2][DK]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Lay::misc + 1280);
+  float* betas = reinterpret_cast<float*>(sm + Lay::misc);          // [2][64]
+  float* gcs = reinterpret_cast<float*>(sm + Lay::misc + 512);      // [2][DK]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Lay::misc + 1536);
   uint64_t* bar_in = bars + 0;
   uint64_t* bar_v = bars + 1;
-  uint64_t* bar_pm = bars + 2;
-  uint64_t* bar_cm = bars + 3;
-  uint64_t* full = bars + 4;   // [2]
-  uint64_t* empty = bars + 6;  // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 9);
+  uint64_t* bar_m1 = bars + 2;  // [2] MMA1 into D1 buffer b
+  uint64_t* bar_m2 = bars + 4;  // MMA2
+  uint64_t* bar_cm = bars + 5;
+  uint64_t* full = bars + 6;    // [2]
+  uint64_t* empty = bars + 8;   // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 11);
 
   const int tid = threadIdx.x, warp = tid >> 5;
   const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
@@ -302,7 +343,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tm_v);
     mbar_init(bar_in, 1);
     mbar_init(bar_v, 1);
-    mbar_init(bar_pm, 1);
+    mbar_init(bar_m1 + 0, 1);
+    mbar_init(bar_m1 + 1, 1);
+    mbar_init(bar_m2, 1);
     mbar_init(bar_cm, 1);
     mbar_init(full + 0, 1);
     mbar_init(full + 1, 1);
@@ -336,8 +379,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row_t = t & 127;
     const int cg = t % NCG, rb = t / NCG;
     const int pnl = cg >> 4, ck = (cg >> 1) & 7, cb = (cg & 1) * 8;
-    const float* la_g = p.log_alpha + (size_t)h * DK + 4 * cg;
-    const size_t la_stride = (size_t)p.H * DK;
+    // log(alpha): one value per key channel (four per thread), one per head
+    // (broadcast over the channels), or none (alpha = 1).
+    const float* la_g = GATE == kGateChannel ? p.log_alpha + (size_t)h * DK + 4 * cg
+                                             : p.log_alpha + h;
+    const size_t la_stride = GATE == kGateChannel ? (size_t)p.H * DK : (size_t)p.H;
 
     auto issue_qk = [&](int tok) {
       mbar_arrive_expect_tx(bar_in, Lay::tx_qk);
@@ -356,56 +402,63 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int i = 0; i < RPT; ++i) {
         const int r = rb * RPT + i;
-        la_reg[i] = r < L ? __ldg(reinterpret_cast<const float4*>(
-                                la_g + (size_t)(tok0 + r) * la_stride))
-                          : make_float4(0.f, 0.f, 0.f, 0.f);
+        la_reg[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (GATE == kGateChannel)
+          ldg_f4_if(la_reg[i], la_g + (size_t)(tok0 + r) * la_stride, r < L);
+        else if (GATE == kGateHead)
+          ldg_f1_if(la_reg[i].x, la_g + (size_t)(tok0 + r) * la_stride, r < L);
       }
     };
 
+    uint32_t ph_in = 0, ph_v = 0, ph_m2 = 0;
+    bool in_flight = nch > 0, v_pending = nch > 0;
+    float beta_next = 0.f;  // beta of the chunk whose prologue runs next
     if (t == 0 && nch > 0) {
       issue_qk(start);
       issue_v(start);
     }
-    float beta_next = 0.f;
     if (nch > 0) {
       load_la(start, min(kC, end - start));
-      if (t < kC && t < end - start)
-        beta_next = p.beta[(size_t)(start + t) * p.H + h];
+      ldg_f1_if(beta_next, p.beta + (size_t)(start + t) * p.H + h,
+                t < kC && t < end - start);
     }
-    uint32_t ph_in = 0, ph_v = 0, ph_pm = 0;
-    bool in_flight = nch > 0, v_pending = nch > 0;
 
-    for (int n = 0; n < nch; ++n) {
-      const int s = n & 1, use = n >> 1;
-      const int tok0 = start + n * kC;
+    // front(m): wait for slot m % 2 and the q, k of chunk m; prologue into
+    // the slot; issue MMA1(m) into D1 buffer m % 2 and the TMA of chunk m+1.
+    // It runs between back1 and back2 of the previous chunk, so MMA2's
+    // latency is spent on this prologue.
+    auto front = [&](int m) -> bool {
+      const int s = m & 1, use = m >> 1;
+      const int tok0 = start + m * kC;
       const int L = min(kC, end - tok0);
-      const bool has_next = n + 1 < nch;
+      const bool has_next = m + 1 < nch;
       uint8_t* kq = sm + Lay::kq + s * Lay::kq_stride;
       uint8_t* kb = sm + Lay::kb + s * 16384;
-      uint8_t* pp = sm + Lay::pp + s * 8192;
       float* gc = gcs + s * DK;
-      if (t < kC) {
-        beta_s[t] = beta_next;
-        beta_next = 0.f;
-        if (has_next && t < end - (tok0 + kC))
-          beta_next = p.beta[(size_t)(tok0 + kC + t) * p.H + h];
-      }
+      if (t < kC) betas[s * 64 + t] = beta_next;
+      beta_next = 0.f;
+      ldg_f1_if(beta_next, p.beta + (size_t)(tok0 + kC + t) * p.H + h,
+                t < kC && has_next && t < end - (tok0 + kC));
       bool ok = true;
-      if (use >= 1) ok = wait_or_abort(empty + s, (use - 1) & 1, abort_flag);
-      ok = ok && wait_or_abort(bar_in, ph_in, abort_flag);
+      if (use >= 1) ok = wait_or_abort<true>(empty + s, (use - 1) & 1, abort_flag);
+      ok = ok && wait_or_abort<false>(bar_in, ph_in, abort_flag);
       ph_in ^= 1;
       in_flight = false;
-      if (named_sync_or(kBarProd, kProd, !ok)) { failed = true; break; }
+      if (named_sync_or(kBarProd, kProd, !ok)) return false;
 
-      // ---- prologue (log(alpha) rows already in registers)
-      {
+      {  // prologue (log(alpha) rows already in registers)
+        if (GATE == kGateHead) {
+#pragma unroll
+          for (int i = 0; i < RPT; ++i)
+            la_reg[i].y = la_reg[i].z = la_reg[i].w = la_reg[i].x;
+        }
         float part[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int i = 0; i < RPT; ++i) {
           part[0] += la_reg[i].x; part[1] += la_reg[i].y;
           part[2] += la_reg[i].z; part[3] += la_reg[i].w;
         }
-        float* red = afp;  // free until the A extraction below
+        float* red = afp;  // free: back() of the previous chunk is done
         *reinterpret_cast<float4*>(red + rb * DK + 4 * cg) =
             make_float4(part[0], part[1], part[2], part[3]);
         named_sync(kBarProd, kProd);
@@ -435,11 +488,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           g[0] += la_reg[i].x; g[1] += la_reg[i].y;
           g[2] += la_reg[i].z; g[3] += la_reg[i].w;
           float e[4], ie[4];
+          if (GATE == kGateChannel) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const float x = g[c] * kLog2e;
-            e[c] = valid ? ex2_approx(x) : 0.f;
-            ie[c] = valid ? ex2_approx(-x) : 0.f;
+            for (int c = 0; c < 4; ++c) {
+              const float x = g[c] * kLog2e;
+              e[c] = valid ? ex2_approx(x) : 0.f;
+              ie[c] = valid ? ex2_approx(-x) : 0.f;
+            }
+          } else {  // one decay for the whole row: two exponentials per row
+            const float x = g[0] * kLog2e;
+            const float e0 = !valid ? 0.f : GATE == kGateHead ? ex2_approx(x) : 1.f;
+            const float i0 = !valid ? 0.f : GATE == kGateHead ? ex2_approx(-x) : 1.f;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              e[c] = e0;
+              ie[c] = i0;
+            }
           }
           const __nv_bfloat162 e01 = __floats2bfloat162_rn(e[0], e[1]);
           const __nv_bfloat162 e23 = __floats2bfloat162_rn(e[2], e[3]);
@@ -462,32 +526,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (has_next) load_la(tok0 + kC, min(kC, end - (tok0 + kC)));
       fence_proxy_async();
       named_sync(kBarProd, kProd);
-
-      // ---- MMA1: [Kt; Qt] . Kb^T ; next chunk's q, k into the staging
-      if (t == 0) {
+      if (t == 0) {  // MMA1: [Kt; Qt] . Kb^T ; then q, k of the next chunk
         tc_fence_after();
         const uint32_t idesc = idesc_bf16(128, 64, false, false);
 #pragma unroll
         for (int ks = 0; ks < DK / 16; ++ks) {
           const uint32_t off = (ks & 3) * 32;
-          mma_bf16(tmem + Lay::t_d1,
+          mma_bf16(tmem + Lay::t_d1 + 64 * s,
                    desc_sw128(smem_u32(kq) + (ks >> 2) * 16384 + off, 16, 1024),
                    desc_sw128(smem_u32(kb) + (ks >> 2) * 8192 + off, 16, 1024),
                    idesc, ks > 0);
         }
-        mma_commit(bar_pm);
+        mma_commit(bar_m1 + s);
         if (has_next) issue_qk(tok0 + kC);
       }
       in_flight = has_next;
-      ok = wait_or_abort(bar_pm, ph_pm, abort_flag);
-      ph_pm ^= 1;
-      if (named_sync_or(kBarProd, kProd, !ok)) { failed = true; break; }
-      tc_fence_after();
+      return true;
+    };
 
-      // ---- A (fp32) and P (bf16 into the slot)
-      {
+    // back1(n): A and P from D1, the inverse, T', then issue MMA2 (W, U)
+    // without waiting for it.
+    auto back1 = [&](int n) -> bool {
+      const int s = n & 1;
+      uint8_t* kq = sm + Lay::kq + s * Lay::kq_stride;
+      uint8_t* pp = sm + Lay::pp + s * 8192;
+      const float* beta_s = betas + s * 64;
+      bool ok = wait_or_abort<false>(bar_m1 + s, (n >> 1) & 1, abort_flag);
+      if (named_sync_or(kBarProd, kProd, !ok)) return false;
+      tc_fence_after();
+      {  // A (fp32) and P (bf16 into the slot)
         float v[32];
-        tmem_ld32(tmem + lane_base + Lay::t_d1 + 32 * colh, v);
+        tmem_ld32(tmem + lane_base + Lay::t_d1 + 64 * s + 32 * colh, v);
         if (row_t < 64) {
           const float b = beta_s[row_t];
 #pragma unroll
@@ -510,7 +579,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       named_sync(kBarProd, kProd);
 
-      invert_unit_lower(afp, tfp, msc, t);
+      invert_unit_lower(afp, tfp, reinterpret_cast<float*>(sm + Lay::msc), t);
 
       {  // T' = Tm Diag(beta), rows masked to the lower triangle
         const int r = t & 63, qc = t >> 6;
@@ -530,10 +599,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async();
       named_sync(kBarProd, kProd);
 
-      // ---- MMA2: W = T' Kt (N = DK), U = T' V (N = 64) into U slot s
-      if (t == 0) {
+      if (t == 0) {  // MMA2: W = T' Kt (N = DK), U = T' V (N = 64) into U slot s
         tc_fence_after();
-        ok = wait_or_abort(bar_v, ph_v, abort_flag);
+        ok = wait_or_abort<false>(bar_v, ph_v, abort_flag);
         ph_v ^= 1;
         v_pending = !ok;
         if (ok) {
@@ -549,21 +617,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                      desc_sw128(smem_u32(vbuf) + ks * 2048, 8192, 1024), iu,
                      ks > 0);
           }
-          mma_commit(bar_pm);
+          mma_commit(bar_m2);
         }
       }
-      if (named_sync_or(kBarProd, kProd, !ok)) { failed = true; break; }
-      ok = wait_or_abort(bar_pm, ph_pm, abort_flag);
-      ph_pm ^= 1;
-      if (named_sync_or(kBarProd, kProd, !ok)) { failed = true; break; }
+      return !named_sync_or(kBarProd, kProd, !ok);
+    };
+
+    // back2(n): wait for MMA2, W into the slot, hand slot n % 2 over.
+    auto back2 = [&](int n) -> bool {
+      const int s = n & 1;
+      const int tok0 = start + n * kC;
+      uint8_t* kq = sm + Lay::kq + s * Lay::kq_stride;
+      bool ok = wait_or_abort<false>(bar_m2, ph_m2, abort_flag);
+      ph_m2 ^= 1;
+      if (named_sync_or(kBarProd, kProd, !ok)) return false;
       tc_fence_after();
-      if (t == 0 && has_next) {
+      if (t == 0 && n + 1 < nch) {  // V is free once MMA2 has completed
         issue_v(tok0 + kC);
         v_pending = true;
       }
-
-      // ---- W rows (bf16) over the Kt rows of the slot's [Kt; Qt]
-      if (row_t < 64) {
+      if (row_t < 64) {  // W rows (bf16) over the Kt rows of the slot
 #pragma unroll
         for (int j = 0; j < DK / 64; ++j) {
           const int hh = colh * (DK / 64) + j;
@@ -576,6 +649,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async();
       named_sync(kBarProd, kProd);
       if (t == 0) mbar_arrive(full + s);
+      return true;
+    };
+
+    // Per chunk n: back1(n), then the next chunk's prologue and MMA1 while
+    // MMA2(n) runs, then back2(n).
+    if (nch > 0 && !front(0)) failed = true;
+    for (int n = 0; n < nch && !failed; ++n) {
+      if (!back1(n) || (n + 1 < nch && !front(n + 1)) || !back2(n))
+        failed = true;
     }
     if (failed && t == 0) {
       *abort_flag = 1;
@@ -622,7 +704,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint8_t* kq = sm + Lay::kq + s * Lay::kq_stride;
       uint8_t* kb = sm + Lay::kb + s * 16384;
       uint8_t* pp = sm + Lay::pp + s * 8192;
-      bool ok = wait_or_abort(full + s, use & 1, abort_flag);
+      bool ok = wait_or_abort<true>(full + s, use & 1, abort_flag);
       if (named_sync_or(kBarCons, kCons, !ok)) { failed = true; break; }
       tc_fence_after();
 
@@ -638,7 +720,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                    ks > 0);
         mma_commit(bar_cm);
       }
-      ok = wait_or_abort(bar_cm, ph_cm, abort_flag);
+      ok = wait_or_abort<false>(bar_cm, ph_cm, abort_flag);
       ph_cm ^= 1;
       if (named_sync_or(kBarCons, kCons, !ok)) { failed = true; break; }
       tc_fence_after();
@@ -676,7 +758,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mma_commit(bar_cm);
       }
-      ok = wait_or_abort(bar_cm, ph_cm, abort_flag);
+      ok = wait_or_abort<false>(bar_cm, ph_cm, abort_flag);
       ph_cm ^= 1;
       if (named_sync_or(kBarCons, kCons, !ok)) { failed = true; break; }
       tc_fence_after();
@@ -744,7 +826,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // Host side: tensor maps for q, k, v and the launch, one CTA per (sequence,
 // head, 64-column d_v tile).
-template <int DK>
+template <int DK, int GATE>
 cudaError_t run_ws(const ChunkArgs& a, const int32_t* order,
                    cudaStream_t stream) {
   using Lay = WsLayout<DK>;
@@ -769,18 +851,24 @@ cudaError_t run_ws(const ChunkArgs& a, const int32_t* order,
   p.n_tiles = a.dv / kDvt;
   const size_t smem = Lay::bytes + 1024;
   cudaError_t e = cudaFuncSetAttribute(
-      fused_ws_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      fused_ws_kernel<DK, GATE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
       (int)smem);
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)a.n_seqs * a.H * p.n_tiles;
-  fused_ws_kernel<DK><<<grid, kThreads, smem, stream>>>(tq, tk, tv, p);
+  fused_ws_kernel<DK, GATE><<<grid, kThreads, smem, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 
 inline cudaError_t launch_fused_ws(const ChunkArgs& a, const int32_t* order,
                                    cudaStream_t stream) {
-  return a.dk == 128 ? run_ws<128>(a, order, stream)
-                     : run_ws<64>(a, order, stream);
+  if (a.gate == kGateHead)
+    return a.dk == 128 ? run_ws<128, kGateHead>(a, order, stream)
+                       : run_ws<64, kGateHead>(a, order, stream);
+  if (a.gate == kGateNone)
+    return a.dk == 128 ? run_ws<128, kGateNone>(a, order, stream)
+                       : run_ws<64, kGateNone>(a, order, stream);
+  return a.dk == 128 ? run_ws<128, kGateChannel>(a, order, stream)
+                     : run_ws<64, kGateChannel>(a, order, stream);
 }
 
 }  // namespace ws

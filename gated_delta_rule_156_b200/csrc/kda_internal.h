@@ -8,6 +8,10 @@
 
 namespace kda {
 
+// Forget-gate layouts: one log(alpha) per key channel (KDA), one per head
+// (Gated DeltaNet), or none (alpha = 1, DeltaNet).
+enum GateMode { kGateChannel = 0, kGateHead = 1, kGateNone = 2 };
+
 struct RecurrentArgs {
   const void* q;
   const void* k;
@@ -18,6 +22,7 @@ struct RecurrentArgs {
   void* out;
   int B, T, H, dk, dv;
   bool bf16;
+  int gate = kGateChannel;
 };
 
 struct ChunkArgs {
@@ -34,6 +39,7 @@ struct ChunkArgs {
   int T;       // tokens per sequence (dense) or total tokens (packed)
   int H, dk, dv, chunk;
   bool bf16;
+  int gate = kGateChannel;
 };
 
 // Token-by-token evaluation (kda_decode.cu).

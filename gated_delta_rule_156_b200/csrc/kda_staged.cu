@@ -75,9 +75,11 @@ __global__ void plan_kernel(const int32_t* __restrict__ cu, int n_seqs, int T,
 }
 
 // (1) g_r = sum_{i<=r} l_i within the chunk; one thread per key channel.
+// With a per-head gate every channel reads the head's log(alpha); with no
+// gate (alpha = 1) g stays zero.
 __global__ void cumsum_kernel(const float* __restrict__ la, float* __restrict__ g,
                               const int32_t* cu, const int32_t* chunk_off,
-                              int n_seqs, int T, int H, int dk, int C) {
+                              int n_seqs, int T, int H, int dk, int C, int gate) {
   int seq, tok0, L;
   if (!locate_chunk(blockIdx.x, cu, chunk_off, n_seqs, T, C, &seq, &tok0, &L))
     return;
@@ -86,7 +88,9 @@ __global__ void cumsum_kernel(const float* __restrict__ la, float* __restrict__ 
     float acc = 0.f;
     for (int r = 0; r < L; ++r) {
       const size_t idx = ((size_t)(tok0 + r) * H + h) * dk + c;
-      acc += la[idx];
+      acc += gate == kGateChannel ? la[idx]
+             : gate == kGateHead  ? la[(size_t)(tok0 + r) * H + h]
+                                  : 0.f;
       g[idx] = acc;
     }
   }
@@ -339,7 +343,7 @@ cudaError_t run(const ChunkArgs& a, void* workspace, cudaStream_t stream) {
   if (nch > 0) {
     const dim3 grid((unsigned)nch, H);
     cumsum_kernel<<<grid, dk, 0, stream>>>(a.log_alpha, w.g, cu, w.chunk_off,
-                                          a.n_seqs, a.T, H, dk, C);
+                                          a.n_seqs, a.T, H, dk, C, a.gate);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
     const size_t sm2 = 4 * ((size_t)2 * C * dk + (size_t)C * dv + 2 * C * C + C);

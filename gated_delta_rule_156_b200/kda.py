@@ -21,7 +21,9 @@ STATUS_NAMES = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED",
 EXPORTS = ("kda_chunk_fwd", "kda_chunk_fwd_staged", "kda_recurrent_step",
            "kda_chunk_fwd_plan", "kda_selftest_umma", "kda_device_status",
            "kda_status_string", "kda_last_cuda_error", "kda_version",
-           "kda_chunk_fwd_staged_noalloc")
+           "kda_chunk_fwd_staged_noalloc", "kda_chunk_fwd_gated",
+           "kda_recurrent_step_gated")
+GATES = {"channel": 0, "head": 1, "none": 2}
 
 
 class KdaShape(ctypes.Structure):
@@ -65,6 +67,14 @@ def library():
             fn = getattr(lib, name)
             fn.restype = ctypes.c_int
             fn.argtypes = chunk_args
+        lib.kda_chunk_fwd_gated.restype = ctypes.c_int
+        lib.kda_chunk_fwd_gated.argtypes = [
+            ctypes.POINTER(KdaShape), ctypes.c_int, vp, vp, vp, fp, fp, fp, vp,
+            vp, fp, ctypes.c_int, vp]
+        lib.kda_recurrent_step_gated.restype = ctypes.c_int
+        lib.kda_recurrent_step_gated.argtypes = [
+            ctypes.POINTER(KdaShape), ctypes.c_int, vp, vp, vp, fp, fp, fp, vp,
+            vp]
         lib.kda_recurrent_step.restype = ctypes.c_int
         lib.kda_recurrent_step.argtypes = [ctypes.POINTER(KdaShape), vp, vp, vp,
                                            fp, fp, fp, vp, vp]
@@ -116,11 +126,14 @@ def _stream(stream):
 
 
 def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
-              chunk=64, out=None, final_state=None, staged=False, stream=None):
-    """Chunkwise KDA forward (kda_chunk_fwd / kda_chunk_fwd_staged).
+              chunk=64, out=None, final_state=None, staged=False, stream=None,
+              gate="channel"):
+    """Chunkwise KDA forward (kda_chunk_fwd / kda_chunk_fwd_staged, or
+    kda_chunk_fwd_gated when ``gate`` is not "channel").
 
     q, k [B, T, H, d_k]; v [B, T, H, d_v] (bf16 or fp32, same dtype);
-    log_alpha [B, T, H, d_k] fp32; beta [B, T, H] fp32; initial_state
+    log_alpha fp32 [B, T, H, d_k] (gate="channel"), [B, T, H] (gate="head")
+    or None (gate="none"); beta [B, T, H] fp32; initial_state
     [N, H, d_k, d_v] fp32 or None; cu_seqlens int32 [N + 1] or None (then
     B == 1 and T is the packed total).  Returns (out, final_state).
     """
@@ -142,6 +155,14 @@ def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
         _check_dev(name, t, dt)
     shape = KdaShape(B, T, H, dk, dv, chunk, n if cu_seqlens is not None else 0,
                      _io(q))
+    if gate != "channel":
+        st = library().kda_chunk_fwd_gated(
+            ctypes.byref(shape), GATES[gate], _ptr(q), _ptr(k), _ptr(v),
+            _ptr(log_alpha), _ptr(beta), _ptr(initial_state), _ptr(cu_seqlens),
+            _ptr(out), _ptr(final_state), int(staged), _stream(stream))
+        if st != KDA_OK:
+            raise KdaError(st, "kda_chunk_fwd_gated")
+        return out, final_state
     fn = library().kda_chunk_fwd_staged if staged else library().kda_chunk_fwd
     st = fn(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
             _ptr(beta), _ptr(initial_state), _ptr(cu_seqlens), _ptr(out),
@@ -151,9 +172,11 @@ def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
     return out, final_state
 
 
-def recurrent_step(q, k, v, log_alpha, beta, state, out=None, stream=None):
-    """Token-by-token KDA (kda_recurrent_step); ``state`` [B, H, d_k, d_v] fp32
-    is updated in place.  q, k [B, T, H, d_k] (T >= 1 tokens per sequence).
+def recurrent_step(q, k, v, log_alpha, beta, state, out=None, stream=None,
+                   gate="channel"):
+    """Token-by-token KDA (kda_recurrent_step, or kda_recurrent_step_gated
+    when ``gate`` is "head" or "none"); ``state`` [B, H, d_k, d_v] fp32 is
+    updated in place.  q, k [B, T, H, d_k] (T >= 1 tokens per sequence).
     Returns out [B, T, H, d_v]."""
     B, T, H, dk = q.shape
     dv = v.shape[-1]
@@ -165,9 +188,12 @@ def recurrent_step(q, k, v, log_alpha, beta, state, out=None, stream=None):
                         ("state", state, torch.float32), ("out", out, q.dtype)):
         _check_dev(name, t, dt)
     shape = KdaShape(B, T, H, dk, dv, 0, 0, _io(q))
-    st = library().kda_recurrent_step(
-        ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
-        _ptr(beta), _ptr(state), _ptr(out), _stream(stream))
+    st = library().kda_recurrent_step_gated(
+        ctypes.byref(shape), GATES[gate], _ptr(q), _ptr(k), _ptr(v),
+        _ptr(log_alpha), _ptr(beta), _ptr(state), _ptr(out), _stream(stream)) \
+        if gate != "channel" else library().kda_recurrent_step(
+            ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+            _ptr(beta), _ptr(state), _ptr(out), _stream(stream))
     if st != KDA_OK:
         raise KdaError(st, "kda_recurrent_step")
     return out

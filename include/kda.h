@@ -73,6 +73,14 @@ typedef enum {
 
 typedef enum { KDA_BF16 = 0, KDA_F32 = 1 } kda_dtype;
 
+/* Layout of the forget gate's log(alpha) for the *_gated entry points. */
+typedef enum {
+  KDA_GATE_CHANNEL = 0, /* [B, T, H, d_k]: one per key channel (KDA)          */
+  KDA_GATE_HEAD = 1,    /* [B, T, H]: one per head, all channels alike
+                           (Gated DeltaNet)                                   */
+  KDA_GATE_NONE = 2     /* no tensor, alpha = 1 (DeltaNet); pass NULL          */
+} kda_gate;
+
 typedef struct {
   int B;      /* batch (number of sequences when cu_seqlens is NULL; 1 with it) */
   int T;      /* tokens per sequence, or total packed tokens with cu_seqlens  */
@@ -130,6 +138,41 @@ KDA_API kda_status kda_chunk_fwd_staged(const kda_shape* shape, const void* q,
                                 const float* initial_state,
                                 const int32_t* cu_seqlens, void* out,
                                 float* final_state, cudaStream_t stream);
+
+/*
+ * kda_chunk_fwd_gated -- kda_chunk_fwd with the forget gate in one of the
+ * three layouts of kda_gate.  A channel-uniform gate is Gated DeltaNet, no
+ * gate is DeltaNet; both are special cases of the same recurrence ("Kimi
+ * Delta Attention", akshathtiwari.co.in: Gated DeltaNet's single per-head
+ * gate, sharpened by KDA into one gate per channel; "The fourth layer
+ * remembers": the earlier design's one decay number per head per token).
+ * With KDA_GATE_HEAD / KDA_GATE_NONE the kernels read 4 bytes / nothing per
+ * token and head instead of 4 d_k bytes and form one decay per row.
+ *   gate     : a kda_gate value.
+ *   log_gate : [B, T, H, d_k] (channel, 16-byte aligned), [B, T, H] (head,
+ *              4-byte aligned) or NULL (none).
+ *   staged   : nonzero forces the four-stage fp32 pipeline
+ *              (kda_chunk_fwd_staged); zero picks as kda_chunk_fwd does.
+ * Everything else as kda_chunk_fwd.
+ */
+KDA_API kda_status kda_chunk_fwd_gated(const kda_shape* shape, int gate,
+                                       const void* q, const void* k,
+                                       const void* v, const float* log_gate,
+                                       const float* beta,
+                                       const float* initial_state,
+                                       const int32_t* cu_seqlens, void* out,
+                                       float* final_state, int staged,
+                                       cudaStream_t stream);
+
+/* kda_recurrent_step with the forget gate in one of the kda_gate layouts
+ * (see kda_chunk_fwd_gated); everything else as kda_recurrent_step. */
+KDA_API kda_status kda_recurrent_step_gated(const kda_shape* shape, int gate,
+                                            const void* q, const void* k,
+                                            const void* v,
+                                            const float* log_gate,
+                                            const float* beta,
+                                            float* state_inout, void* out,
+                                            cudaStream_t stream);
 
 /* Size in bytes of the fixed device scratch array behind
  * kda_chunk_fwd_staged_noalloc (16 MiB). */

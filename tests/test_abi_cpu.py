@@ -105,3 +105,36 @@ def test_recurrent_validation(lib):
     assert call(shape(), q=A + 0x1000_0000 + 4) == MIS
     assert call(shape(), out=6) == INV          # out aliases the state
     assert call(shape(), st=2) == INV           # state aliases k
+
+
+def test_gated_validation(lib):
+    INV, MIS = 1, 3
+
+    def call(s, gate, la=4, **kw):
+        P = lambda i: None if i is None else (ctypes.c_void_p(i) if i > 1000 else _p(i))  # noqa: E731
+        args = dict(q=1, k=2, v=3, b=5, s0=6, cu=None, out=7, sf=8)
+        args.update(kw)
+        return lib.kda_chunk_fwd_gated(
+            ctypes.byref(s), gate, P(args["q"]), P(args["k"]), P(args["v"]),
+            P(la), P(args["b"]), P(args["s0"]), P(args["cu"]), P(args["out"]),
+            P(args["sf"]), 0, None)
+
+    assert call(shape(), 3) == INV                 # unknown gate layout
+    assert call(shape(), -1) == INV
+    assert call(shape(), 0, la=None) == INV        # channel gate needs a tensor
+    assert call(shape(), 1, la=None) == INV        # head gate needs a tensor
+    # a per-head gate needs only 4-byte alignment, a per-channel one 16
+    assert call(shape(), 0, la=A + 4 * 0x1000_0000 + 4) == MIS
+    assert call(shape(), 1, la=A + 4 * 0x1000_0000 + 2) == MIS
+    # the out buffer may not overlap a per-head gate either
+    assert call(shape(), 1, la=A + 7 * 0x1000_0000 + 64) == INV
+
+    def step(s, gate, la=4):
+        P = lambda i: None if i is None else (ctypes.c_void_p(i) if i > 1000 else _p(i))  # noqa: E731
+        return lib.kda_recurrent_step_gated(
+            ctypes.byref(s), gate, P(1), P(2), P(3), P(la), P(5), P(6), P(7),
+            None)
+
+    assert step(shape(), 5) == INV
+    assert step(shape(), 1, la=None) == INV
+    assert step(shape(), 0, la=A + 4 * 0x1000_0000 + 8) == MIS
