@@ -333,6 +333,37 @@ def run_kda(args, world, rank, local):
         "tensor_frac": pflops / (h_launch * 1e-3) / 1e12 / pk["bf16_tflops"],
     }
 
+    # ---- in-kernel input prologue on raw inputs: q, k L2-normalised (and q
+    # scaled) and log(alpha) = logsigmoid(x) / 16 from raw gate logits x ------
+    g_raw = torch.Generator(device=dev).manual_seed(4242 + rank)
+    q_raw = torch.randn(d["q"].shape, generator=g_raw, device=dev).bfloat16()
+    k_raw = torch.randn(d["k"].shape, generator=g_raw, device=dev).bfloat16()
+    x_raw = torch.randn(d["log_alpha"].shape, generator=g_raw, device=dev)
+    pro = dict(normalize_qk=True, q_scale=dk ** -0.5, gate_logits=True,
+               gate_scale=1 / 16)
+
+    def prefill_pro(_i):
+        K.chunk_fwd(q_raw, k_raw, d["v"], x_raw, d["beta"], None, None,
+                    chunk=C, out=out, final_state=fin, prologue=pro)
+
+    for i in range(args.warmup):
+        prefill_pro(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    rms, rper = timed(prefill_pro, args.steps, stream)
+    barrier(world)
+    rms = max_over_ranks(rms, world)
+    r_launch = statistics.mean(rper)
+    fused_prologue = {
+        "value": world * B * T / (rms / args.steps * 1e-3), "unit": "tokens/s",
+        "ms_per_step": rms / args.steps,
+        "workload": "as the prefill, from raw q, k and gate logits with the "
+                    "in-kernel prologue (L2 norm, q scale, logsigmoid/16)",
+        "hbm": {"achieved": pbytes / (r_launch * 1e-3) / 1e9, "unit": "GB/s",
+                "frac": pbytes / (r_launch * 1e-3) / 1e9 / pk["hbm_gbs"]},
+    }
+    del q_raw, k_raw, x_raw
+
     # ---- end to end through the public API with host buffers ------------
     host = {n: d[n].cpu().pin_memory() for n in
             ("q", "k", "v", "log_alpha", "beta")}
@@ -422,6 +453,7 @@ def run_kda(args, world, rank, local):
                 "gpu_launches": args.steps,
             },
             "prefill_head_gate": head_gate,
+            "prefill_fused_prologue": fused_prologue,
             "e2e": {"value": e2e_value, "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": e2e_steps},

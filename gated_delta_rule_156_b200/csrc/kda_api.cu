@@ -242,6 +242,42 @@ kda_status kda_chunk_fwd_gated(const kda_shape* shape, int gate, const void* q,
   return run_with_workspace(kda::staged_workspace_bytes(a), stream, false, a);
 }
 
+}  // extern "C"
+
+namespace {
+bool set_prologue(const kda_prologue* p, kda::Prologue* out) {
+  if (!p) return true;
+  if (!(p->q_scale == p->q_scale) || !(p->gate_scale == p->gate_scale))
+    return false;  // NaN scales
+  out->norm_qk = p->normalize_qk != 0;
+  out->q_scale = p->q_scale;
+  out->gate_logits = p->gate_logits != 0;
+  out->gate_scale = p->gate_scale;
+  return true;
+}
+}  // namespace
+
+extern "C" {
+
+kda_status kda_chunk_fwd_ex(const kda_shape* shape, int gate,
+                            const kda_prologue* prologue, const void* q,
+                            const void* k, const void* v,
+                            const float* gate_tensor, const float* beta,
+                            const float* initial_state,
+                            const int32_t* cu_seqlens, void* out,
+                            float* final_state, int staged,
+                            cudaStream_t stream) {
+  kda::ChunkArgs a{};
+  const kda_status st = validate_chunk(shape, q, k, v, gate_tensor, beta,
+                                       initial_state, cu_seqlens, out,
+                                       final_state, &a, gate);
+  if (st != KDA_OK) return st;
+  if (!set_prologue(prologue, &a.pro)) return KDA_ERR_INVALID_ARG;
+  if (!staged && kda::fused_supported(a))
+    return run_with_workspace(kda::fused_workspace_bytes(a), stream, true, a);
+  return run_with_workspace(kda::staged_workspace_bytes(a), stream, false, a);
+}
+
 kda_status kda_chunk_fwd_staged_noalloc(
     const kda_shape* shape, const void* q, const void* k, const void* v,
     const float* log_alpha, const float* beta, const float* initial_state,
@@ -275,7 +311,19 @@ kda_status kda_recurrent_step_gated(const kda_shape* s, int gate, const void* q,
                                     const float* log_alpha, const float* beta,
                                     float* state_inout, void* out,
                                     cudaStream_t stream) {
+  return kda_recurrent_step_ex(s, gate, nullptr, q, k, v, log_alpha, beta,
+                               state_inout, out, stream);
+}
+
+kda_status kda_recurrent_step_ex(const kda_shape* s, int gate,
+                                 const kda_prologue* prologue, const void* q,
+                                 const void* k, const void* v,
+                                 const float* log_alpha, const float* beta,
+                                 float* state_inout, void* out,
+                                 cudaStream_t stream) {
   if (!s) return KDA_ERR_INVALID_ARG;
+  kda::Prologue pro;
+  if (!set_prologue(prologue, &pro)) return KDA_ERR_INVALID_ARG;
   if (gate != KDA_GATE_CHANNEL && gate != KDA_GATE_HEAD && gate != KDA_GATE_NONE)
     return KDA_ERR_INVALID_ARG;
   if (gate == KDA_GATE_NONE) log_alpha = nullptr;
@@ -312,7 +360,7 @@ kda_status kda_recurrent_step_gated(const kda_shape* s, int gate, const void* q,
 
   kda::RecurrentArgs a{q, k, v, log_alpha, beta, state_inout, out,
                        s->B, s->T, s->H, s->dk, s->dv,
-                       s->io_dtype == KDA_BF16, gate};
+                       s->io_dtype == KDA_BF16, gate, pro};
   const cudaError_t e = kda::launch_recurrent(a, stream);
   return e == cudaSuccess ? KDA_OK : cuda_fail(e);
 }
@@ -353,6 +401,12 @@ kda_status kda_device_status(cudaStream_t stream) {
   const cudaError_t e = kda::fused_take_timeout(stream, &flag);
   if (e != cudaSuccess) return cuda_fail(e);
   return flag ? KDA_ERR_TIMEOUT : KDA_OK;
+}
+
+kda_status kda_selftest_timeout(int limit_us, cudaStream_t stream) {
+  if (limit_us < 1 || limit_us > 100000) return KDA_ERR_INVALID_ARG;
+  const cudaError_t e = kda::launch_timeout_probe(limit_us, stream);
+  return e == cudaSuccess ? KDA_OK : cuda_fail(e);
 }
 
 int kda_last_cuda_error(void) { return g_last_cuda_error; }

@@ -17,7 +17,9 @@
 // column sums over d_k are a register partial per thread, then one pass over
 // the 8 row groups in shared memory.  With T > 1 the state stays in registers
 // across tokens and is written once at the end.  The gate may also be one
-// value per head (Gated DeltaNet) or absent (alpha = 1, DeltaNet).
+// value per head (Gated DeltaNet) or absent (alpha = 1, DeltaNet), and an
+// optional prologue normalises q and k and turns gate logits into
+// log(alpha) = scale * logsigmoid(x) on the fly.
 #include "kda_common.cuh"
 #include "kda_internal.h"
 
@@ -27,13 +29,16 @@ namespace {
 
 constexpr int kRowGroups = 8;
 
-template <int DK, int DV, typename IO>
+// PLAIN: per-channel gate and no prologue (the common case, kept free of the
+// per-token selects and extra reductions of the general path).
+template <int DK, int DV, typename IO, bool PLAIN>
 __global__ void __launch_bounds__((DV / 4) * kRowGroups)
     recurrent_kernel(const IO* __restrict__ q, const IO* __restrict__ k,
                      const IO* __restrict__ v,
                      const float* __restrict__ log_alpha,
                      const float* __restrict__ beta, float* __restrict__ state,
-                     IO* __restrict__ out, int T, int H, int gate) {
+                     IO* __restrict__ out, int T, int H, int gate,
+                     Prologue pro) {
   constexpr int CG = DV / 4;          // float4 column groups
   constexpr int R = DK / kRowGroups;  // rows per thread
   constexpr int NT = CG * kRowGroups;
@@ -44,7 +49,7 @@ __global__ void __launch_bounds__((DV / 4) * kRowGroups)
 
   __shared__ float s_k[DK], s_q[DK], s_a[DK], s_v[DV];
   __shared__ float4 s_e[kRowGroups][CG], s_p[kRowGroups][CG];
-  __shared__ float s_kq, s_beta;
+  __shared__ float s_kq, s_beta, s_invk, s_invq;
 
   float4* st = reinterpret_cast<float4*>(state + (size_t)bh * DK * DV);
   float4 s[R];
@@ -57,29 +62,54 @@ __global__ void __launch_bounds__((DV / 4) * kRowGroups)
     for (int c = tid; c < DK; c += NT) {
       s_k[c] = to_f32(k[ok + c]);
       s_q[c] = to_f32(q[ok + c]);
-      s_a[c] = gate == kGateChannel ? __expf(log_alpha[ok + c])
-               : gate == kGateHead  ? __expf(log_alpha[tok * H + h])
-                                    : 1.f;
+      if (PLAIN) {
+        s_a[c] = __expf(log_alpha[ok + c]);
+      } else {
+        float l = gate == kGateChannel ? log_alpha[ok + c]
+                  : gate == kGateHead  ? log_alpha[tok * H + h]
+                                       : 0.f;
+        if (pro.gate_logits && gate != kGateNone)  // scale * logsigmoid(l)
+          l = pro.gate_scale * (fminf(l, 0.f) - log1pf(__expf(-fabsf(l))));
+        s_a[c] = __expf(l);
+      }
     }
     for (int j = tid; j < DV; j += NT) s_v[j] = to_f32(v[ov + j]);
-    if (tid < 32) {  // k . q, one warp
-      float acc = 0.f;
-      for (int c = tid; c < DK; c += 32)
-        acc += to_f32(k[ok + c]) * to_f32(q[ok + c]);
+    if (tid < 32) {  // k . q (and, with the prologue, the norms), one warp
+      float kq = 0.f, kk = 0.f, qq = 0.f;
+      for (int c = tid; c < DK; c += 32) {
+        const float kc = to_f32(k[ok + c]), qc = to_f32(q[ok + c]);
+        kq += kc * qc;
+        if (!PLAIN) {
+          kk += kc * kc;
+          qq += qc * qc;
+        }
+      }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      for (int o = 16; o > 0; o >>= 1) {
+        kq += __shfl_xor_sync(0xffffffffu, kq, o);
+        if (!PLAIN) {
+          kk += __shfl_xor_sync(0xffffffffu, kk, o);
+          qq += __shfl_xor_sync(0xffffffffu, qq, o);
+        }
+      }
       if (tid == 0) {
-        s_kq = acc;
+        const float ik = !PLAIN && pro.norm_qk ? rsqrtf(kk) : 1.f;
+        const float iq =
+            (!PLAIN && pro.norm_qk ? rsqrtf(qq) : 1.f) * (PLAIN ? 1.f : pro.q_scale);
+        s_invk = ik;
+        s_invq = iq;
+        s_kq = kq * ik * iq;
         s_beta = beta[tok * H + h];
       }
     }
     __syncthreads();
+    const float invk = PLAIN ? 1.f : s_invk, invq = PLAIN ? 1.f : s_invq;
 
     float4 e = make_float4(0.f, 0.f, 0.f, 0.f), p = e;
 #pragma unroll
     for (int i = 0; i < R; ++i) {
       const int r = rg * R + i;
-      const float a = s_a[r], kr = s_k[r], qr = s_q[r];
+      const float a = s_a[r], kr = s_k[r] * invk, qr = s_q[r] * invq;
       s[i].x *= a; s[i].y *= a; s[i].z *= a; s[i].w *= a;
       e.x += s[i].x * kr; e.y += s[i].y * kr; e.z += s[i].z * kr; e.w += s[i].w * kr;
       p.x += s[i].x * qr; p.y += s[i].y * qr; p.z += s[i].z * qr; p.w += s[i].w * qr;
@@ -109,7 +139,7 @@ __global__ void __launch_bounds__((DV / 4) * kRowGroups)
     }
 #pragma unroll
     for (int i = 0; i < R; ++i) {
-      const float kr = s_k[rg * R + i];
+      const float kr = s_k[rg * R + i] * invk;
       s[i].x += kr * d.x; s[i].y += kr * d.y; s[i].z += kr * d.z; s[i].w += kr * d.w;
     }
     __syncthreads();  // shared vectors are rewritten by the next token
@@ -122,10 +152,18 @@ template <int DK, int DV, typename IO>
 cudaError_t launch_dkdv(const RecurrentArgs& a, cudaStream_t stream) {
   constexpr int NT = (DV / 4) * kRowGroups;
   const unsigned grid = (unsigned)a.B * (unsigned)a.H;
-  recurrent_kernel<DK, DV, IO><<<grid, NT, 0, stream>>>(
-      static_cast<const IO*>(a.q), static_cast<const IO*>(a.k),
-      static_cast<const IO*>(a.v), a.log_alpha, a.beta, a.state,
-      static_cast<IO*>(a.out), a.T, a.H, a.gate);
+  const bool plain = a.gate == kGateChannel && !a.pro.norm_qk &&
+                     a.pro.q_scale == 1.f && !a.pro.gate_logits;
+  if (plain)
+    recurrent_kernel<DK, DV, IO, true><<<grid, NT, 0, stream>>>(
+        static_cast<const IO*>(a.q), static_cast<const IO*>(a.k),
+        static_cast<const IO*>(a.v), a.log_alpha, a.beta, a.state,
+        static_cast<IO*>(a.out), a.T, a.H, a.gate, a.pro);
+  else
+    recurrent_kernel<DK, DV, IO, false><<<grid, NT, 0, stream>>>(
+        static_cast<const IO*>(a.q), static_cast<const IO*>(a.k),
+        static_cast<const IO*>(a.v), a.log_alpha, a.beta, a.state,
+        static_cast<IO*>(a.out), a.T, a.H, a.gate, a.pro);
   return cudaGetLastError();
 }
 

@@ -119,6 +119,28 @@ size_t fused_workspace_bytes(const ChunkArgs& a) {
 
 int fused_kernel_count(const ChunkArgs& a) { return a.cu_seqlens ? 2 : 1; }
 
+namespace {
+// Waits on an mbarrier that nothing completes, with the same bounded wait the
+// fused kernel uses; when the limit runs out it sets the device status flag
+// and returns.  Exercises the timeout reporting without a fault or a hang.
+__global__ void timeout_probe_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(&bar, 1);
+    sm100::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !sm100::mbar_wait(&bar, 0, limit_ns))
+    atomicExch(&g_fused_timeout, 1);
+  __syncthreads();
+}
+}  // namespace
+
+cudaError_t launch_timeout_probe(int limit_us, cudaStream_t stream) {
+  timeout_probe_kernel<<<1, 32, 0, stream>>>((uint64_t)limit_us * 1000ull);
+  return cudaGetLastError();
+}
+
 cudaError_t fused_take_timeout(cudaStream_t stream, int* flag) {
   cudaError_t e = cudaStreamSynchronize(stream);
   if (e != cudaSuccess) return e;

@@ -68,6 +68,7 @@ struct WsLayout {
 };
 
 struct WsParams {
+  Prologue pro;
   const float* beta;
   const float* log_alpha;
   const float* s_init;
@@ -447,6 +448,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (named_sync_or(kBarProd, kProd, !ok)) return false;
 
       {  // prologue (log(alpha) rows already in registers)
+        if (GATE != kGateNone && p.pro.gate_logits) {
+          // raw logits x -> log(alpha) = scale * logsigmoid(x), valid rows only
+          const float sc = p.pro.gate_scale;
+          auto ls = [&](float x) {
+            return sc * (fminf(x, 0.f) - log1pf(__expf(-fabsf(x))));
+          };
+#pragma unroll
+          for (int i = 0; i < RPT; ++i) {
+            if (rb * RPT + i < L) {
+              la_reg[i].x = ls(la_reg[i].x);
+              if (GATE == kGateChannel) {
+                la_reg[i].y = ls(la_reg[i].y);
+                la_reg[i].z = ls(la_reg[i].z);
+                la_reg[i].w = ls(la_reg[i].w);
+              }
+            }
+          }
+        }
         if (GATE == kGateHead) {
 #pragma unroll
           for (int i = 0; i < RPT; ++i)
@@ -505,19 +524,46 @@ __global__ void __launch_bounds__(kThreads, 1)
               ie[c] = i0;
             }
           }
-          const __nv_bfloat162 e01 = __floats2bfloat162_rn(e[0], e[1]);
-          const __nv_bfloat162 e23 = __floats2bfloat162_rn(e[2], e[3]);
-          const __nv_bfloat162 i01 = __floats2bfloat162_rn(ie[0], ie[1]);
-          const __nv_bfloat162 i23 = __floats2bfloat162_rn(ie[2], ie[3]);
           const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kr);
           const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&qr);
           uint2 wt, wq, wb;
-          *reinterpret_cast<__nv_bfloat162*>(&wt.x) = __hmul2(k2[0], e01);
-          *reinterpret_cast<__nv_bfloat162*>(&wt.y) = __hmul2(k2[1], e23);
-          *reinterpret_cast<__nv_bfloat162*>(&wq.x) = __hmul2(q2[0], e01);
-          *reinterpret_cast<__nv_bfloat162*>(&wq.y) = __hmul2(q2[1], e23);
-          *reinterpret_cast<__nv_bfloat162*>(&wb.x) = __hmul2(k2[0], i01);
-          *reinterpret_cast<__nv_bfloat162*>(&wb.y) = __hmul2(k2[1], i23);
+          if (p.pro.norm_qk || p.pro.q_scale != 1.f) {
+            // optional prologue: L2-normalise the rows of q and k (the row's
+            // NCG threads reduce by shuffles) and scale q, in fp32
+            const float2 k01 = __bfloat1622float2(k2[0]), k23 = __bfloat1622float2(k2[1]);
+            const float2 q01 = __bfloat1622float2(q2[0]), q23 = __bfloat1622float2(q2[1]);
+            float kf[4] = {k01.x, k01.y, k23.x, k23.y};
+            float qf[4] = {q01.x, q01.y, q23.x, q23.y};
+            float ik = 1.f, iq = p.pro.q_scale;
+            if (p.pro.norm_qk) {
+              float sk = kf[0] * kf[0] + kf[1] * kf[1] + kf[2] * kf[2] + kf[3] * kf[3];
+              float sq = qf[0] * qf[0] + qf[1] * qf[1] + qf[2] * qf[2] + qf[3] * qf[3];
+#pragma unroll
+              for (int o = NCG / 2; o > 0; o >>= 1) {
+                sk += __shfl_xor_sync(0xffffffffu, sk, o);
+                sq += __shfl_xor_sync(0xffffffffu, sq, o);
+              }
+              ik = valid ? rsqrtf(sk) : 0.f;
+              iq = valid ? rsqrtf(sq) * p.pro.q_scale : 0.f;
+            }
+            wt.x = pack_bf16x2(kf[0] * ik * e[0], kf[1] * ik * e[1]);
+            wt.y = pack_bf16x2(kf[2] * ik * e[2], kf[3] * ik * e[3]);
+            wq.x = pack_bf16x2(qf[0] * iq * e[0], qf[1] * iq * e[1]);
+            wq.y = pack_bf16x2(qf[2] * iq * e[2], qf[3] * iq * e[3]);
+            wb.x = pack_bf16x2(kf[0] * ik * ie[0], kf[1] * ik * ie[1]);
+            wb.y = pack_bf16x2(kf[2] * ik * ie[2], kf[3] * ik * ie[3]);
+          } else {
+            const __nv_bfloat162 e01 = __floats2bfloat162_rn(e[0], e[1]);
+            const __nv_bfloat162 e23 = __floats2bfloat162_rn(e[2], e[3]);
+            const __nv_bfloat162 i01 = __floats2bfloat162_rn(ie[0], ie[1]);
+            const __nv_bfloat162 i23 = __floats2bfloat162_rn(ie[2], ie[3]);
+            *reinterpret_cast<__nv_bfloat162*>(&wt.x) = __hmul2(k2[0], e01);
+            *reinterpret_cast<__nv_bfloat162*>(&wt.y) = __hmul2(k2[1], e23);
+            *reinterpret_cast<__nv_bfloat162*>(&wq.x) = __hmul2(q2[0], e01);
+            *reinterpret_cast<__nv_bfloat162*>(&wq.y) = __hmul2(q2[1], e23);
+            *reinterpret_cast<__nv_bfloat162*>(&wb.x) = __hmul2(k2[0], i01);
+            *reinterpret_cast<__nv_bfloat162*>(&wb.y) = __hmul2(k2[1], i23);
+          }
           *reinterpret_cast<uint2*>(pkq + off) = wt;
           *reinterpret_cast<uint2*>(pkq + 64 * 128 + off) = wq;
           *reinterpret_cast<uint2*>(pkb + off) = wb;
@@ -837,6 +883,7 @@ cudaError_t run_ws(const ChunkArgs& a, const int32_t* order,
       !make_tile_map(&tv, a.v, a.dv, a.H, tokens))
     return cudaErrorInvalidValue;
   WsParams p{};
+  p.pro = a.pro;
   p.beta = a.beta;
   p.log_alpha = a.log_alpha;
   p.s_init = a.initial_state;

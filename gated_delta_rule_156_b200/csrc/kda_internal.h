@@ -12,6 +12,16 @@ namespace kda {
 // (Gated DeltaNet), or none (alpha = 1, DeltaNet).
 enum GateMode { kGateChannel = 0, kGateHead = 1, kGateNone = 2 };
 
+// Optional input prologue applied inside the kernels: per-token L2
+// normalisation of q and k over d_k, a scale on q, and log(alpha) formed as
+// gate_scale * logsigmoid(x) from raw gate logits x.
+struct Prologue {
+  bool norm_qk = false;
+  float q_scale = 1.f;
+  bool gate_logits = false;
+  float gate_scale = 1.f;
+};
+
 struct RecurrentArgs {
   const void* q;
   const void* k;
@@ -23,6 +33,7 @@ struct RecurrentArgs {
   int B, T, H, dk, dv;
   bool bf16;
   int gate = kGateChannel;
+  Prologue pro;
 };
 
 struct ChunkArgs {
@@ -40,6 +51,7 @@ struct ChunkArgs {
   int H, dk, dv, chunk;
   bool bf16;
   int gate = kGateChannel;
+  Prologue pro;
 };
 
 // Token-by-token evaluation (kda_decode.cu).
@@ -60,6 +72,8 @@ int fused_kernel_count(const ChunkArgs& a);
 // Synchronises `stream`, then reads and clears the flag a fused kernel sets
 // when one of its bounded waits gave up.
 cudaError_t fused_take_timeout(cudaStream_t stream, int* flag);
+// Diagnostic: one CTA whose bounded wait runs out after limit_us.
+cudaError_t launch_timeout_probe(int limit_us, cudaStream_t stream);
 cudaError_t launch_fused(const ChunkArgs& a, void* workspace,
                          cudaStream_t stream);
 

@@ -28,7 +28,15 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kDvTile = 32;
 
+bool has_prologue(const ChunkArgs& a) {
+  return a.pro.norm_qk || a.pro.q_scale != 1.f ||
+         (a.pro.gate_logits && a.gate != kGateNone);
+}
+
 struct Ws {
+  void* qn;            // prologue outputs (only with an input prologue):
+  void* kn;            //   normalised q, k [tokens, H, dk] in the io dtype,
+  float* lan;          //   log(alpha) [tokens, H, dk or 1]
   int32_t* chunk_off;  // [n_seqs + 1] (packed layout only)
   float* g;            // [tokens, H, dk]   cumulative log-decay within chunk
   float* w;            // [tokens, H, dk]   W rows
@@ -50,6 +58,13 @@ Ws carve(const ChunkArgs& a, void* base, size_t* total) {
     off = align256(off + bytes);
     return r;
   };
+  if (has_prologue(a)) {
+    const size_t esz = a.bf16 ? 2 : 4;
+    w.qn = take(esz * tokens * H * a.dk);
+    w.kn = take(esz * tokens * H * a.dk);
+    w.lan = reinterpret_cast<float*>(
+        take(4 * tokens * H * (a.gate == kGateChannel ? a.dk : 1)));
+  }
   w.chunk_off = reinterpret_cast<int32_t*>(take(4 * (size_t)(a.n_seqs + 1)));
   w.g = reinterpret_cast<float*>(take(4 * tokens * H * a.dk));
   w.w = reinterpret_cast<float*>(take(4 * tokens * H * a.dk));
@@ -58,6 +73,43 @@ Ws carve(const ChunkArgs& a, void* base, size_t* total) {
       take(4 * (size_t)max_chunks(a) * H * a.dk * a.dv));
   if (total) *total = off;
   return w;
+}
+
+// Optional input prologue, one warp per (token, head): q and k L2-normalised
+// over d_k (q also scaled), and raw gate logits turned into
+// log(alpha) = scale * logsigmoid(x); results go to the workspace.
+template <typename IO>
+__global__ void prologue_kernel(const IO* __restrict__ q, const IO* __restrict__ k,
+                                const float* __restrict__ la, IO* __restrict__ qn,
+                                IO* __restrict__ kn, float* __restrict__ lan,
+                                int H, int dk, int gate, Prologue pro) {
+  const size_t th = blockIdx.x;  // token * H + head
+  const int lane = threadIdx.x;
+  float sk = 0.f, sq = 0.f;
+  for (int c = lane; c < dk; c += 32) {
+    const float kc = to_f32(k[th * dk + c]), qc = to_f32(q[th * dk + c]);
+    sk += kc * kc;
+    sq += qc * qc;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    sk += __shfl_xor_sync(0xffffffffu, sk, o);
+    sq += __shfl_xor_sync(0xffffffffu, sq, o);
+  }
+  const float ik = pro.norm_qk ? rsqrtf(sk) : 1.f;
+  const float iq = (pro.norm_qk ? rsqrtf(sq) : 1.f) * pro.q_scale;
+  for (int c = lane; c < dk; c += 32) {
+    kn[th * dk + c] = from_f32<IO>(to_f32(k[th * dk + c]) * ik);
+    qn[th * dk + c] = from_f32<IO>(to_f32(q[th * dk + c]) * iq);
+  }
+  if (gate == kGateNone) return;
+  const int nl = gate == kGateChannel ? dk : 1;
+  for (int c = lane; c < nl; c += 32) {
+    float x = la[th * nl + c];
+    if (pro.gate_logits)
+      x = pro.gate_scale * (fminf(x, 0.f) - log1pf(__expf(-fabsf(x))));
+    lan[th * nl + c] = x;
+  }
 }
 
 // Packed layout: exclusive prefix sum of ceil(len_s / C) per sequence.
@@ -384,14 +436,55 @@ size_t staged_workspace_bytes(const ChunkArgs& a) {
 int staged_kernel_count(const ChunkArgs& a) {
   if (a.n_seqs == 0) return 0;
   const bool any_chunks = max_chunks(a) > 0;
-  return (a.cu_seqlens ? 1 : 0) + 1 + (any_chunks ? 3 : 0);
+  return (a.cu_seqlens ? 1 : 0) + 1 + (any_chunks ? 3 : 0) +
+         (has_prologue(a) && any_chunks ? 1 : 0);
 }
 
 cudaError_t launch_staged(const ChunkArgs& a, void* workspace,
                           cudaStream_t stream) {
   if (a.n_seqs == 0 || a.H == 0) return cudaSuccess;
-  return a.bf16 ? run<__nv_bfloat16>(a, workspace, stream)
-                : run<float>(a, workspace, stream);
+  if (!has_prologue(a))
+    return a.bf16 ? run<__nv_bfloat16>(a, workspace, stream)
+                  : run<float>(a, workspace, stream);
+  // Input prologue first, into the workspace; then the four stages read the
+  // prepared q, k and log(alpha).
+  Ws w = carve(a, workspace, nullptr);
+  const size_t tokens =
+      a.cu_seqlens ? (size_t)a.T : (size_t)a.n_seqs * (size_t)a.T;
+  if (tokens > 0) {
+    const unsigned grid = (unsigned)(tokens * a.H);
+    if (a.bf16)
+      prologue_kernel<__nv_bfloat16><<<grid, 32, 0, stream>>>(
+          static_cast<const __nv_bfloat16*>(a.q),
+          static_cast<const __nv_bfloat16*>(a.k), a.log_alpha,
+          static_cast<__nv_bfloat16*>(w.qn), static_cast<__nv_bfloat16*>(w.kn),
+          w.lan, a.H, a.dk, a.gate, a.pro);
+    else
+      prologue_kernel<float><<<grid, 32, 0, stream>>>(
+          static_cast<const float*>(a.q), static_cast<const float*>(a.k),
+          a.log_alpha, static_cast<float*>(w.qn), static_cast<float*>(w.kn),
+          w.lan, a.H, a.dk, a.gate, a.pro);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  ChunkArgs b = a;
+  b.q = w.qn;
+  b.k = w.kn;
+  b.log_alpha = a.gate == kGateNone ? nullptr : w.lan;
+  b.pro = Prologue{};
+  // b's workspace is the part of ours after the prologue outputs
+  size_t pre = 0;
+  {
+    ChunkArgs c = a;
+    c.pro = Prologue{};
+    size_t whole = 0, rest = 0;
+    carve(a, nullptr, &whole);
+    carve(c, nullptr, &rest);
+    pre = whole - rest;
+  }
+  void* rest_ws = static_cast<char*>(workspace) + pre;
+  return a.bf16 ? run<__nv_bfloat16>(b, rest_ws, stream)
+                : run<float>(b, rest_ws, stream);
 }
 
 }  // namespace kda

@@ -22,7 +22,8 @@ EXPORTS = ("kda_chunk_fwd", "kda_chunk_fwd_staged", "kda_recurrent_step",
            "kda_chunk_fwd_plan", "kda_selftest_umma", "kda_device_status",
            "kda_status_string", "kda_last_cuda_error", "kda_version",
            "kda_chunk_fwd_staged_noalloc", "kda_chunk_fwd_gated",
-           "kda_recurrent_step_gated")
+           "kda_recurrent_step_gated", "kda_chunk_fwd_ex",
+           "kda_recurrent_step_ex", "kda_selftest_timeout")
 GATES = {"channel": 0, "head": 1, "none": 2}
 
 
@@ -31,6 +32,21 @@ class KdaShape(ctypes.Structure):
                 ("dk", ctypes.c_int), ("dv", ctypes.c_int),
                 ("chunk", ctypes.c_int), ("n_seqs", ctypes.c_int),
                 ("io_dtype", ctypes.c_int)]
+
+
+class KdaPrologue(ctypes.Structure):
+    _fields_ = [("normalize_qk", ctypes.c_int), ("q_scale", ctypes.c_float),
+                ("gate_logits", ctypes.c_int), ("gate_scale", ctypes.c_float)]
+
+
+def _prologue(pro):
+    """dict(normalize_qk=bool, q_scale=float, gate_logits=bool,
+    gate_scale=float) -> KdaPrologue (missing keys: no-op defaults)."""
+    pro = dict(pro or {})
+    return KdaPrologue(int(bool(pro.get("normalize_qk", False))),
+                       float(pro.get("q_scale", 1.0)),
+                       int(bool(pro.get("gate_logits", False))),
+                       float(pro.get("gate_scale", 1.0)))
 
 
 class KdaError(RuntimeError):
@@ -75,6 +91,14 @@ def library():
         lib.kda_recurrent_step_gated.argtypes = [
             ctypes.POINTER(KdaShape), ctypes.c_int, vp, vp, vp, fp, fp, fp, vp,
             vp]
+        lib.kda_chunk_fwd_ex.restype = ctypes.c_int
+        lib.kda_chunk_fwd_ex.argtypes = [
+            ctypes.POINTER(KdaShape), ctypes.c_int, ctypes.POINTER(KdaPrologue),
+            vp, vp, vp, fp, fp, fp, vp, vp, fp, ctypes.c_int, vp]
+        lib.kda_recurrent_step_ex.restype = ctypes.c_int
+        lib.kda_recurrent_step_ex.argtypes = [
+            ctypes.POINTER(KdaShape), ctypes.c_int, ctypes.POINTER(KdaPrologue),
+            vp, vp, vp, fp, fp, fp, vp, vp]
         lib.kda_recurrent_step.restype = ctypes.c_int
         lib.kda_recurrent_step.argtypes = [ctypes.POINTER(KdaShape), vp, vp, vp,
                                            fp, fp, fp, vp, vp]
@@ -85,6 +109,8 @@ def library():
             ctypes.POINTER(ctypes.c_size_t)]
         lib.kda_selftest_umma.restype = ctypes.c_int
         lib.kda_selftest_umma.argtypes = [ctypes.c_int] * 5 + [vp, vp, vp, vp]
+        lib.kda_selftest_timeout.restype = ctypes.c_int
+        lib.kda_selftest_timeout.argtypes = [ctypes.c_int, vp]
         lib.kda_device_status.restype = ctypes.c_int
         lib.kda_device_status.argtypes = [vp]
         lib.kda_status_string.restype = ctypes.c_char_p
@@ -127,7 +153,7 @@ def _stream(stream):
 
 def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
               chunk=64, out=None, final_state=None, staged=False, stream=None,
-              gate="channel"):
+              gate="channel", prologue=None):
     """Chunkwise KDA forward (kda_chunk_fwd / kda_chunk_fwd_staged, or
     kda_chunk_fwd_gated when ``gate`` is not "channel").
 
@@ -135,7 +161,9 @@ def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
     log_alpha fp32 [B, T, H, d_k] (gate="channel"), [B, T, H] (gate="head")
     or None (gate="none"); beta [B, T, H] fp32; initial_state
     [N, H, d_k, d_v] fp32 or None; cu_seqlens int32 [N + 1] or None (then
-    B == 1 and T is the packed total).  Returns (out, final_state).
+    B == 1 and T is the packed total).  ``prologue`` (dict, see
+    kda_prologue) normalises q and k and/or maps gate logits in-kernel
+    (kda_chunk_fwd_ex).  Returns (out, final_state).
     """
     B, T, H, dk = q.shape
     dv = v.shape[-1]
@@ -155,6 +183,16 @@ def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
         _check_dev(name, t, dt)
     shape = KdaShape(B, T, H, dk, dv, chunk, n if cu_seqlens is not None else 0,
                      _io(q))
+    if prologue is not None:
+        pro = _prologue(prologue)
+        st = library().kda_chunk_fwd_ex(
+            ctypes.byref(shape), GATES[gate], ctypes.byref(pro), _ptr(q),
+            _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(initial_state),
+            _ptr(cu_seqlens), _ptr(out), _ptr(final_state), int(staged),
+            _stream(stream))
+        if st != KDA_OK:
+            raise KdaError(st, "kda_chunk_fwd_ex")
+        return out, final_state
     if gate != "channel":
         st = library().kda_chunk_fwd_gated(
             ctypes.byref(shape), GATES[gate], _ptr(q), _ptr(k), _ptr(v),
@@ -173,7 +211,7 @@ def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
 
 
 def recurrent_step(q, k, v, log_alpha, beta, state, out=None, stream=None,
-                   gate="channel"):
+                   gate="channel", prologue=None):
     """Token-by-token KDA (kda_recurrent_step, or kda_recurrent_step_gated
     when ``gate`` is "head" or "none"); ``state`` [B, H, d_k, d_v] fp32 is
     updated in place.  q, k [B, T, H, d_k] (T >= 1 tokens per sequence).
@@ -188,6 +226,15 @@ def recurrent_step(q, k, v, log_alpha, beta, state, out=None, stream=None,
                         ("state", state, torch.float32), ("out", out, q.dtype)):
         _check_dev(name, t, dt)
     shape = KdaShape(B, T, H, dk, dv, 0, 0, _io(q))
+    if prologue is not None:
+        pro = _prologue(prologue)
+        st = library().kda_recurrent_step_ex(
+            ctypes.byref(shape), GATES[gate], ctypes.byref(pro), _ptr(q),
+            _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(state),
+            _ptr(out), _stream(stream))
+        if st != KDA_OK:
+            raise KdaError(st, "kda_recurrent_step_ex")
+        return out
     st = library().kda_recurrent_step_gated(
         ctypes.byref(shape), GATES[gate], _ptr(q), _ptr(k), _ptr(v),
         _ptr(log_alpha), _ptr(beta), _ptr(state), _ptr(out), _stream(stream)) \
@@ -282,3 +329,11 @@ def chunk_fwd_noalloc(q, k, v, log_alpha, beta, initial_state=None,
     if st != KDA_OK:
         raise KdaError(st, "kda_chunk_fwd_staged_noalloc")
     return out, final_state
+
+
+def selftest_timeout(limit_us=1000, stream=None):
+    """Diagnostic (kda_selftest_timeout): a kernel whose bounded wait runs out
+    after limit_us; the next device_status() then reports KDA_ERR_TIMEOUT."""
+    st = library().kda_selftest_timeout(int(limit_us), _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_selftest_timeout")

@@ -174,6 +174,47 @@ KDA_API kda_status kda_recurrent_step_gated(const kda_shape* shape, int gate,
                                             float* state_inout, void* out,
                                             cudaStream_t stream);
 
+/*
+ * Optional input prologue for the *_ex entry points, applied inside the
+ * kernels so the caller needs no separate pass over q, k and the gate:
+ *   normalize_qk : nonzero -> q and k are L2-normalised per token and head
+ *                  over d_k (in fp32) before use.
+ *   q_scale      : q is multiplied by q_scale after normalisation (1 = none).
+ *   gate_logits  : nonzero -> the gate tensor holds raw logits x and
+ *                  log(alpha) = gate_scale * logsigmoid(x); zero -> it holds
+ *                  log(alpha) itself (gate_scale ignored).
+ * The pages leave the gate's parameterisation open ("The fourth layer
+ * remembers": a forget-gate module without a lower bound); logsigmoid of a
+ * logit is the plainest reading of such a gate.  A NULL prologue means none.
+ */
+typedef struct {
+  int normalize_qk;
+  float q_scale;
+  int gate_logits;
+  float gate_scale;
+} kda_prologue;
+
+/* kda_chunk_fwd_gated with an optional input prologue (see kda_prologue). */
+KDA_API kda_status kda_chunk_fwd_ex(const kda_shape* shape, int gate,
+                                    const kda_prologue* prologue,
+                                    const void* q, const void* k,
+                                    const void* v, const float* gate_tensor,
+                                    const float* beta,
+                                    const float* initial_state,
+                                    const int32_t* cu_seqlens, void* out,
+                                    float* final_state, int staged,
+                                    cudaStream_t stream);
+
+/* kda_recurrent_step_gated with an optional input prologue. */
+KDA_API kda_status kda_recurrent_step_ex(const kda_shape* shape, int gate,
+                                         const kda_prologue* prologue,
+                                         const void* q, const void* k,
+                                         const void* v,
+                                         const float* gate_tensor,
+                                         const float* beta,
+                                         float* state_inout, void* out,
+                                         cudaStream_t stream);
+
 /* Size in bytes of the fixed device scratch array behind
  * kda_chunk_fwd_staged_noalloc (16 MiB). */
 #define KDA_NOALLOC_SCRATCH_BYTES (16u << 20)
@@ -273,6 +314,14 @@ KDA_API const char* kda_status_string(kda_status status);
  * wait without a time limit; a wait that runs out abandons the rest of that
  * CTA's work and leaves its outputs unspecified. */
 KDA_API kda_status kda_device_status(cudaStream_t stream);
+
+/* kda_selftest_timeout -- diagnostic of the failure reporting, not part of
+ * the forward pass: launches one CTA that waits on a device barrier nothing
+ * completes, using the library's bounded wait with a limit of limit_us
+ * microseconds (1 .. 100000).  The wait gives up, the CTA sets the device
+ * status flag and exits normally (no fault, no hang), so the next
+ * kda_device_status on this stream returns KDA_ERR_TIMEOUT. */
+KDA_API kda_status kda_selftest_timeout(int limit_us, cudaStream_t stream);
 
 /* The cudaError_t value behind the most recent KDA_ERR_CUDA on this thread
  * (0 if none). */

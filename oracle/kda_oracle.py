@@ -206,3 +206,25 @@ def chunked_debug(q, k, v, log_alpha, beta, initial_state=None, chunk=64):
     rec["out"] = out
     rec["final"] = S
     return rec
+
+
+def prologue(q, k, gate, normalize_qk=True, q_scale=1.0, gate_logits=True,
+             gate_scale=1.0):
+    """The optional input prologue, in fp64, as its plain definition:
+      q <- q_scale * q / ||q||,  k <- k / ||k||   (L2 norm over d_k, per token
+                                                 and head; only if normalize_qk)
+      log(alpha) <- gate_scale * logsigmoid(gate) (only if gate_logits), with
+      logsigmoid(x) = log(1 / (1 + exp(-x))).
+    ``gate`` may be a per-channel [.., d_k], per-head [..] tensor, or None.
+    Returns (q, k, log_alpha) as float64 arrays (log_alpha None if gate is).
+    """
+    q, k = _f64(q), _f64(k)
+    if normalize_qk:
+        q = q_scale * q / np.sqrt(np.sum(q * q, axis=-1, keepdims=True))
+        k = k / np.sqrt(np.sum(k * k, axis=-1, keepdims=True))
+    elif q_scale != 1.0:
+        q = q_scale * q
+    la = None if gate is None else _f64(gate)
+    if la is not None and gate_logits:
+        la = gate_scale * -np.logaddexp(0.0, -la)
+    return q, k, la

@@ -138,3 +138,15 @@ def test_gated_validation(lib):
     assert step(shape(), 5) == INV
     assert step(shape(), 1, la=None) == INV
     assert step(shape(), 0, la=A + 4 * 0x1000_0000 + 8) == MIS
+
+
+def test_prologue_validation(lib):
+    pro = K.KdaPrologue(1, float("nan"), 1, 1.0)
+    s = shape()
+    P = lambda i: None if i is None else _p(i)  # noqa: E731
+    st = lib.kda_chunk_fwd_ex(ctypes.byref(s), 0, ctypes.byref(pro), P(1), P(2),
+                              P(3), P(4), P(5), P(6), None, P(7), P(8), 0, None)
+    assert st == 1  # NaN scale rejected before any launch
+    st = lib.kda_recurrent_step_ex(ctypes.byref(s), 0, ctypes.byref(pro), P(1),
+                                   P(2), P(3), P(4), P(5), P(6), P(7), None)
+    assert st == 1

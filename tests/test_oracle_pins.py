@@ -82,3 +82,23 @@ def test_pins_catch_planted_mistake(name, tmp_path):
     failed = P.failing_pins(rec)
     assert failed, f"no pin caught the planted mistake {name!r}"
     os.remove(lib)
+
+
+def test_prologue_closed_forms():
+    # logsigmoid: 0 -> -log 2; large positive -> 0; large negative -> x;
+    # L2 normalisation gives unit (or q_scale) norms and keeps direction.
+    rng = np.random.default_rng(30)
+    q = rng.standard_normal((3, 5, 2, 8))
+    k = rng.standard_normal((3, 5, 2, 8))
+    g = np.array([0.0, 40.0, -40.0, 1.0])
+    qn, kn, la = kda_oracle.prologue(q, k, g, q_scale=0.25, gate_scale=0.5)
+    assert np.allclose(np.linalg.norm(qn, axis=-1), 0.25)
+    assert np.allclose(np.linalg.norm(kn, axis=-1), 1.0)
+    assert np.allclose(np.sum(kn * k, axis=-1), np.linalg.norm(k, axis=-1))
+    assert np.isclose(la[0], -0.5 * np.log(2.0))
+    assert abs(la[1]) < 1e-15 and np.isclose(la[2], -20.0)
+    assert np.isclose(la[3], 0.5 * np.log(1.0 / (1.0 + np.exp(-1.0))))
+    # no normalisation: only the scale; no logits: the gate passes through
+    q2, k2, la2 = kda_oracle.prologue(q, k, g, normalize_qk=False, q_scale=2.0,
+                                      gate_logits=False)
+    assert np.allclose(q2, 2.0 * q) and np.allclose(k2, k) and np.allclose(la2, g)
