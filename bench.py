@@ -515,9 +515,12 @@ def load_traffic():
         for name, rec in d.items():
             if name.startswith("_"):
                 continue
-            with open(os.path.join(ROOT, rec["file"]), "rb") as src:
-                if hashlib.sha256(src.read()).hexdigest() == rec["sha256"]:
-                    out[name] = rec["bytes"]
+            h = hashlib.sha256()
+            for fn in rec["files"]:  # the kernel's sources, in order
+                with open(os.path.join(ROOT, fn), "rb") as src:
+                    h.update(src.read())
+            if h.hexdigest() == rec["sha256"]:
+                out[name] = rec["bytes"]
     except Exception:
         return {}
     return out
