@@ -98,6 +98,7 @@ bool make_tile_map(CUtensorMap* m, const void* base, int d, int H, int tokens) {
 }  // namespace kda
 
 #include "kda_fused_ws_sm100.cuh"
+#include "kda_fused_pair_sm100.cuh"
 
 namespace kda {
 namespace {
@@ -161,6 +162,9 @@ cudaError_t launch_fused(const ChunkArgs& a, void* workspace,
     if (e != cudaSuccess) return e;
     order = o;
   }
+  // d_v = 128: the two 64-column tiles of a head share the per-chunk
+  // factorisation as a cluster pair; d_v = 64: one CTA per head.
+  if (a.dv == 2 * ws::kDvt) return pair::launch_fused_pair(a, order, stream);
   return ws::launch_fused_ws(a, order, stream);
 }
 

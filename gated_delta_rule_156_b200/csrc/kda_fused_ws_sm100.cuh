@@ -292,6 +292,144 @@ __device__ __forceinline__ void invert_unit_lower(const float* A, float* X,
   named_sync(kBarProd, kProd);
 }
 
+// The producer prologue of one chunk, over all 256 producer threads: turns
+// the log(alpha) rows held in registers (raw gate logits with the prologue)
+// into the running decay g, writes exp(g_C) per channel to gc, and the
+// decay-scaled bf16 operands Kt = k e^g and Qt = q e^g (rows 0-63 and 64-127
+// of the [Kt; Qt] panel pkq) and Kb = k e^-g (panel pkb) from the raw q and k
+// rows at pq and pk.  Thread t owns channels 4 cg .. 4 cg + 3 of rows
+// rb RPT .. rb RPT + RPT - 1; rows at or past L are written as zeros.  pq and
+// pk may be the same bytes as the destination rows (in-place transform): each
+// element is read and rewritten by the same thread.  `red` is DK * NRB
+// floats of scratch.
+template <int DK, int GATE>
+__device__ __forceinline__ void prologue_rows(float4* la_reg, float* red,
+                                              float* gc, const uint8_t* pq,
+                                              const uint8_t* pk, uint8_t* pkq,
+                                              uint8_t* pkb, int L,
+                                              const Prologue& pro, int t) {
+  constexpr int NCG = DK / 4;
+  constexpr int NRB = kProd / NCG;
+  constexpr int RPT = kC / NRB;
+  const int cg = t % NCG, rb = t / NCG;
+  const int ck = (cg >> 1) & 7, cb = (cg & 1) * 8;
+  if (GATE != kGateNone && pro.gate_logits) {
+    // raw logits x -> log(alpha) = scale * logsigmoid(x), valid rows only
+    const float sc = pro.gate_scale;
+    auto ls = [&](float x) {
+      return sc * (fminf(x, 0.f) - log1pf(__expf(-fabsf(x))));
+    };
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) {
+      if (rb * RPT + i < L) {
+        la_reg[i].x = ls(la_reg[i].x);
+        if (GATE == kGateChannel) {
+          la_reg[i].y = ls(la_reg[i].y);
+          la_reg[i].z = ls(la_reg[i].z);
+          la_reg[i].w = ls(la_reg[i].w);
+        }
+      }
+    }
+  }
+  if (GATE == kGateHead) {
+#pragma unroll
+    for (int i = 0; i < RPT; ++i)
+      la_reg[i].y = la_reg[i].z = la_reg[i].w = la_reg[i].x;
+  }
+  float part[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int i = 0; i < RPT; ++i) {
+    part[0] += la_reg[i].x; part[1] += la_reg[i].y;
+    part[2] += la_reg[i].z; part[3] += la_reg[i].w;
+  }
+  *reinterpret_cast<float4*>(red + rb * DK + 4 * cg) =
+      make_float4(part[0], part[1], part[2], part[3]);
+  named_sync(kBarProd, kProd);
+  float g[4] = {0.f, 0.f, 0.f, 0.f}, tot[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int b2 = 0; b2 < NRB; ++b2) {
+    const float4 y = *reinterpret_cast<const float4*>(red + b2 * DK + 4 * cg);
+    if (b2 < rb) { g[0] += y.x; g[1] += y.y; g[2] += y.z; g[3] += y.w; }
+    tot[0] += y.x; tot[1] += y.y; tot[2] += y.z; tot[3] += y.w;
+  }
+  constexpr float kLog2e = 1.4426950408889634f;
+  if (rb == 0)
+    *reinterpret_cast<float4*>(gc + 4 * cg) =
+        make_float4(ex2_approx(tot[0] * kLog2e), ex2_approx(tot[1] * kLog2e),
+                    ex2_approx(tot[2] * kLog2e), ex2_approx(tot[3] * kLog2e));
+#pragma unroll
+  for (int i = 0; i < RPT; ++i) {
+    const int r = rb * RPT + i;
+    const uint32_t off = r * 128 + ((ck ^ (r & 7)) << 4) + cb;
+    const bool valid = r < L;
+    const uint2 kr = *reinterpret_cast<const uint2*>(pk + off);
+    const uint2 qr = *reinterpret_cast<const uint2*>(pq + off);
+    g[0] += la_reg[i].x; g[1] += la_reg[i].y;
+    g[2] += la_reg[i].z; g[3] += la_reg[i].w;
+    float e[4], ie[4];
+    if (GATE == kGateChannel) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const float x = g[c] * kLog2e;
+        e[c] = valid ? ex2_approx(x) : 0.f;
+        ie[c] = valid ? ex2_approx(-x) : 0.f;
+      }
+    } else {  // one decay for the whole row: two exponentials per row
+      const float x = g[0] * kLog2e;
+      const float e0 = !valid ? 0.f : GATE == kGateHead ? ex2_approx(x) : 1.f;
+      const float i0 = !valid ? 0.f : GATE == kGateHead ? ex2_approx(-x) : 1.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        e[c] = e0;
+        ie[c] = i0;
+      }
+    }
+    const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kr);
+    const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&qr);
+    uint2 wt, wq, wb;
+    if (pro.norm_qk || pro.q_scale != 1.f) {
+      // optional prologue: L2-normalise the rows of q and k (the row's NCG
+      // threads reduce by shuffles) and scale q, in fp32
+      const float2 k01 = __bfloat1622float2(k2[0]), k23 = __bfloat1622float2(k2[1]);
+      const float2 q01 = __bfloat1622float2(q2[0]), q23 = __bfloat1622float2(q2[1]);
+      float kf[4] = {k01.x, k01.y, k23.x, k23.y};
+      float qf[4] = {q01.x, q01.y, q23.x, q23.y};
+      float ik = 1.f, iq = pro.q_scale;
+      if (pro.norm_qk) {
+        float sk = kf[0] * kf[0] + kf[1] * kf[1] + kf[2] * kf[2] + kf[3] * kf[3];
+        float sq = qf[0] * qf[0] + qf[1] * qf[1] + qf[2] * qf[2] + qf[3] * qf[3];
+#pragma unroll
+        for (int o = NCG / 2; o > 0; o >>= 1) {
+          sk += __shfl_xor_sync(0xffffffffu, sk, o);
+          sq += __shfl_xor_sync(0xffffffffu, sq, o);
+        }
+        ik = valid ? rsqrtf(sk) : 0.f;
+        iq = valid ? rsqrtf(sq) * pro.q_scale : 0.f;
+      }
+      wt.x = pack_bf16x2(kf[0] * ik * e[0], kf[1] * ik * e[1]);
+      wt.y = pack_bf16x2(kf[2] * ik * e[2], kf[3] * ik * e[3]);
+      wq.x = pack_bf16x2(qf[0] * iq * e[0], qf[1] * iq * e[1]);
+      wq.y = pack_bf16x2(qf[2] * iq * e[2], qf[3] * iq * e[3]);
+      wb.x = pack_bf16x2(kf[0] * ik * ie[0], kf[1] * ik * ie[1]);
+      wb.y = pack_bf16x2(kf[2] * ik * ie[2], kf[3] * ik * ie[3]);
+    } else {
+      const __nv_bfloat162 e01 = __floats2bfloat162_rn(e[0], e[1]);
+      const __nv_bfloat162 e23 = __floats2bfloat162_rn(e[2], e[3]);
+      const __nv_bfloat162 i01 = __floats2bfloat162_rn(ie[0], ie[1]);
+      const __nv_bfloat162 i23 = __floats2bfloat162_rn(ie[2], ie[3]);
+      *reinterpret_cast<__nv_bfloat162*>(&wt.x) = __hmul2(k2[0], e01);
+      *reinterpret_cast<__nv_bfloat162*>(&wt.y) = __hmul2(k2[1], e23);
+      *reinterpret_cast<__nv_bfloat162*>(&wq.x) = __hmul2(q2[0], e01);
+      *reinterpret_cast<__nv_bfloat162*>(&wq.y) = __hmul2(q2[1], e23);
+      *reinterpret_cast<__nv_bfloat162*>(&wb.x) = __hmul2(k2[0], i01);
+      *reinterpret_cast<__nv_bfloat162*>(&wb.y) = __hmul2(k2[1], i23);
+    }
+    *reinterpret_cast<uint2*>(pkq + off) = wt;
+    *reinterpret_cast<uint2*>(pkq + 64 * 128 + off) = wq;
+    *reinterpret_cast<uint2*>(pkb + off) = wb;
+  }
+}
+
 template <int DK, int GATE>
 __global__ void __launch_bounds__(kThreads, 1)
     fused_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -379,7 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int colh = warp >> 2;  // 32-column half of a 64-column accumulator
     const int row_t = t & 127;
     const int cg = t % NCG, rb = t / NCG;
-    const int pnl = cg >> 4, ck = (cg >> 1) & 7, cb = (cg & 1) * 8;
+    const int pnl = cg >> 4;
     // log(alpha): one value per key channel (four per thread), one per head
     // (broadcast over the channels), or none (alpha = 1).
     const float* la_g = GATE == kGateChannel ? p.log_alpha + (size_t)h * DK + 4 * cg
@@ -447,128 +585,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       in_flight = false;
       if (named_sync_or(kBarProd, kProd, !ok)) return false;
 
-      {  // prologue (log(alpha) rows already in registers)
-        if (GATE != kGateNone && p.pro.gate_logits) {
-          // raw logits x -> log(alpha) = scale * logsigmoid(x), valid rows only
-          const float sc = p.pro.gate_scale;
-          auto ls = [&](float x) {
-            return sc * (fminf(x, 0.f) - log1pf(__expf(-fabsf(x))));
-          };
-#pragma unroll
-          for (int i = 0; i < RPT; ++i) {
-            if (rb * RPT + i < L) {
-              la_reg[i].x = ls(la_reg[i].x);
-              if (GATE == kGateChannel) {
-                la_reg[i].y = ls(la_reg[i].y);
-                la_reg[i].z = ls(la_reg[i].z);
-                la_reg[i].w = ls(la_reg[i].w);
-              }
-            }
-          }
-        }
-        if (GATE == kGateHead) {
-#pragma unroll
-          for (int i = 0; i < RPT; ++i)
-            la_reg[i].y = la_reg[i].z = la_reg[i].w = la_reg[i].x;
-        }
-        float part[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int i = 0; i < RPT; ++i) {
-          part[0] += la_reg[i].x; part[1] += la_reg[i].y;
-          part[2] += la_reg[i].z; part[3] += la_reg[i].w;
-        }
-        float* red = afp;  // free: back() of the previous chunk is done
-        *reinterpret_cast<float4*>(red + rb * DK + 4 * cg) =
-            make_float4(part[0], part[1], part[2], part[3]);
-        named_sync(kBarProd, kProd);
-        float g[4] = {0.f, 0.f, 0.f, 0.f}, tot[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int b2 = 0; b2 < NRB; ++b2) {
-          const float4 y = *reinterpret_cast<const float4*>(red + b2 * DK + 4 * cg);
-          if (b2 < rb) { g[0] += y.x; g[1] += y.y; g[2] += y.z; g[3] += y.w; }
-          tot[0] += y.x; tot[1] += y.y; tot[2] += y.z; tot[3] += y.w;
-        }
-        constexpr float kLog2e = 1.4426950408889634f;
-        if (rb == 0)
-          *reinterpret_cast<float4*>(gc + 4 * cg) =
-              make_float4(ex2_approx(tot[0] * kLog2e), ex2_approx(tot[1] * kLog2e),
-                          ex2_approx(tot[2] * kLog2e), ex2_approx(tot[3] * kLog2e));
-        const uint8_t* pq = st_q + pnl * 8192;
-        const uint8_t* pk = st_k + pnl * 8192;
-        uint8_t* pkq = kq + pnl * 16384;
-        uint8_t* pkb = kb + pnl * 8192;
-#pragma unroll
-        for (int i = 0; i < RPT; ++i) {
-          const int r = rb * RPT + i;
-          const uint32_t off = r * 128 + ((ck ^ (r & 7)) << 4) + cb;
-          const bool valid = r < L;
-          const uint2 kr = *reinterpret_cast<const uint2*>(pk + off);
-          const uint2 qr = *reinterpret_cast<const uint2*>(pq + off);
-          g[0] += la_reg[i].x; g[1] += la_reg[i].y;
-          g[2] += la_reg[i].z; g[3] += la_reg[i].w;
-          float e[4], ie[4];
-          if (GATE == kGateChannel) {
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              const float x = g[c] * kLog2e;
-              e[c] = valid ? ex2_approx(x) : 0.f;
-              ie[c] = valid ? ex2_approx(-x) : 0.f;
-            }
-          } else {  // one decay for the whole row: two exponentials per row
-            const float x = g[0] * kLog2e;
-            const float e0 = !valid ? 0.f : GATE == kGateHead ? ex2_approx(x) : 1.f;
-            const float i0 = !valid ? 0.f : GATE == kGateHead ? ex2_approx(-x) : 1.f;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              e[c] = e0;
-              ie[c] = i0;
-            }
-          }
-          const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kr);
-          const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&qr);
-          uint2 wt, wq, wb;
-          if (p.pro.norm_qk || p.pro.q_scale != 1.f) {
-            // optional prologue: L2-normalise the rows of q and k (the row's
-            // NCG threads reduce by shuffles) and scale q, in fp32
-            const float2 k01 = __bfloat1622float2(k2[0]), k23 = __bfloat1622float2(k2[1]);
-            const float2 q01 = __bfloat1622float2(q2[0]), q23 = __bfloat1622float2(q2[1]);
-            float kf[4] = {k01.x, k01.y, k23.x, k23.y};
-            float qf[4] = {q01.x, q01.y, q23.x, q23.y};
-            float ik = 1.f, iq = p.pro.q_scale;
-            if (p.pro.norm_qk) {
-              float sk = kf[0] * kf[0] + kf[1] * kf[1] + kf[2] * kf[2] + kf[3] * kf[3];
-              float sq = qf[0] * qf[0] + qf[1] * qf[1] + qf[2] * qf[2] + qf[3] * qf[3];
-#pragma unroll
-              for (int o = NCG / 2; o > 0; o >>= 1) {
-                sk += __shfl_xor_sync(0xffffffffu, sk, o);
-                sq += __shfl_xor_sync(0xffffffffu, sq, o);
-              }
-              ik = valid ? rsqrtf(sk) : 0.f;
-              iq = valid ? rsqrtf(sq) * p.pro.q_scale : 0.f;
-            }
-            wt.x = pack_bf16x2(kf[0] * ik * e[0], kf[1] * ik * e[1]);
-            wt.y = pack_bf16x2(kf[2] * ik * e[2], kf[3] * ik * e[3]);
-            wq.x = pack_bf16x2(qf[0] * iq * e[0], qf[1] * iq * e[1]);
-            wq.y = pack_bf16x2(qf[2] * iq * e[2], qf[3] * iq * e[3]);
-            wb.x = pack_bf16x2(kf[0] * ik * ie[0], kf[1] * ik * ie[1]);
-            wb.y = pack_bf16x2(kf[2] * ik * ie[2], kf[3] * ik * ie[3]);
-          } else {
-            const __nv_bfloat162 e01 = __floats2bfloat162_rn(e[0], e[1]);
-            const __nv_bfloat162 e23 = __floats2bfloat162_rn(e[2], e[3]);
-            const __nv_bfloat162 i01 = __floats2bfloat162_rn(ie[0], ie[1]);
-            const __nv_bfloat162 i23 = __floats2bfloat162_rn(ie[2], ie[3]);
-            *reinterpret_cast<__nv_bfloat162*>(&wt.x) = __hmul2(k2[0], e01);
-            *reinterpret_cast<__nv_bfloat162*>(&wt.y) = __hmul2(k2[1], e23);
-            *reinterpret_cast<__nv_bfloat162*>(&wq.x) = __hmul2(q2[0], e01);
-            *reinterpret_cast<__nv_bfloat162*>(&wq.y) = __hmul2(q2[1], e23);
-            *reinterpret_cast<__nv_bfloat162*>(&wb.x) = __hmul2(k2[0], i01);
-            *reinterpret_cast<__nv_bfloat162*>(&wb.y) = __hmul2(k2[1], i23);
-          }
-          *reinterpret_cast<uint2*>(pkq + off) = wt;
-          *reinterpret_cast<uint2*>(pkq + 64 * 128 + off) = wq;
-          *reinterpret_cast<uint2*>(pkb + off) = wb;
-        }
-      }
+      prologue_rows<DK, GATE>(la_reg, afp, gc,
+                              st_q + pnl * 8192, st_k + pnl * 8192,
+                              kq + pnl * 16384, kb + pnl * 8192, L, p.pro, t);
       if (has_next) load_la(tok0 + kC, min(kC, end - (tok0 + kC)));
       fence_proxy_async();
       named_sync(kBarProd, kProd);
