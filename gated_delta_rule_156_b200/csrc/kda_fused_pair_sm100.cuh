@@ -20,16 +20,22 @@
 // consumer's order.  The raw q and k of an own chunk are loaded by TMA
 // straight into its slot and transformed in place, and that load is issued
 // by the consumer as soon as it has used the peer chunk before it in the same
-// slot.
+// slot.  The package crosses to the peer as bulk shared-to-shared copies
+// (distributed shared memory runs at about 35 GB/s between the two SMs of a
+// pair, so 64.5 KB take about 2 us): Qt, Kb, P and exp(g_C) as soon as the
+// peer's slot is free, T' after the inverse, W at the hand-over.
 //
 // Barriers per CTA: bar_in[s] (q, k of an own chunk landed in slot s),
-// full[s] (slot s holds the next chunk: a local arrive for an own chunk, the
-// peer's expect-tx arrive plus the copy's byte count for a peer chunk),
-// send_ok[s] (the peer's slot s may receive this CTA's next chunk: arrivals
-// from the peer's consumer, done with the chunk there, and from the peer's
-// producer, whose outgoing copy of it has been read).  Every wait is bounded;
-// a failed CTA also raises its peer's abort flag, and both CTAs meet at a
-// final cluster barrier only after all their copies have completed.
+// full[s] (an own chunk is ready in slot s: local arrive), pfull[s] (a peer
+// chunk has fully arrived in slot s: the peer's expect-tx arrive plus the
+// copies' byte counts), send_ok[s] (this CTA's consumer is done with its own
+// chunk in slot s, so the peer may send the next chunk there).  The peer's
+// slot is free for a send once the peer's consumer has released its own
+// chunk there (send_ok, signalled remotely) and the peer's copy of that chunk
+// to this CTA has been read out, which its complete arrival here (pfull)
+// proves.  Every wait is bounded; a failed CTA also raises its peer's abort
+// flag, and both CTAs meet at a final cluster barrier only after all their
+// outgoing copies have completed.
 #pragma once
 
 namespace kda {
@@ -97,11 +103,30 @@ __device__ __forceinline__ void copy_to_peer(uint32_t dst, const void* src,
 __device__ __forceinline__ void bulk_commit() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
-__device__ __forceinline__ void bulk_wait_read() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
 __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+// Non-blocking test of a phase (cluster-scope acquire).
+__device__ __forceinline__ bool test_wait_cluster(uint64_t* bar,
+                                                  uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Pull one TMA box into L2 ahead of its load.
+__device__ __forceinline__ void prefetch_box_l2(const void* tmap, int c0, int c1,
+                                                int c2) {
+  asm volatile(
+      "cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+          reinterpret_cast<uint64_t>(tmap)),
+      "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
 }
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile(
@@ -150,6 +175,14 @@ struct PairLayout {
   static constexpr uint32_t s_gc = s_tp + 8192;     // exp(g_C), DK floats
   static constexpr uint32_t copy_bytes = s_gc + DK * 4;
   static constexpr uint32_t slot = (copy_bytes + 1023) & ~1023u;
+  // The package goes to the peer in three parts, each as soon as it exists
+  // and the peer's slot is free: Qt, Kb, P and exp(g_C) (early), T' (after
+  // the inverse), W (last).  Kb's second panel is all zero when DK = 64 and
+  // stays out (zero in every slot from the start).
+  static constexpr uint32_t kb_bytes = DK == 64 ? 8192 : 16384;
+  static constexpr uint32_t push_bytes =
+      NP * 8192 /* Qt */ + kb_bytes + 8192 /* P */ + DK * 4 + 8192 /* T' */ +
+      NP * 8192 /* W */;
   // producer-private
   static constexpr uint32_t afp = 2 * slot;         // 64 x kFS fp32
   static constexpr uint32_t tfp = afp + 64 * kFS * 4;
@@ -171,7 +204,8 @@ struct PairLayout {
   static_assert(slot % 1024 == 0 && sop % 1024 == 0 && dop % 1024 == 0 &&
                     vbuf % 1024 == 0,
                 "swizzle atoms");
-  static_assert(copy_bytes % 16 == 0, "bulk copy size");
+  static_assert(copy_bytes % 16 == 0 && push_bytes < (1u << 20), "push size");
+  static_assert((DK * 4) % 16 == 0, "exp(g_C) copy size");
   static_assert(bytes + 1024 <= 232448, "shared memory");
 };
 
@@ -196,16 +230,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   float* betas = reinterpret_cast<float*>(sm + Lay::misc);  // [64]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Lay::misc + 256);
   uint64_t* bar_in = bars + 0;   // [2]
-  uint64_t* full = bars + 2;     // [2]
-  uint64_t* send_ok = bars + 4;  // [2]
-  uint64_t* bar_v = bars + 6;    // [2]
-  uint64_t* bar_m1 = bars + 8;
-  uint64_t* bar_m2 = bars + 9;
-  uint64_t* bar_cm = bars + 10;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 12);
+  uint64_t* full = bars + 2;     // [2] own chunk ready (local arrive)
+  uint64_t* pfull = bars + 4;    // [2] peer chunk arrived (peer's pushes)
+  uint64_t* send_ok = bars + 6;  // [2]
+  uint64_t* bar_v = bars + 8;    // [2]
+  uint64_t* bar_m1 = bars + 10;
+  uint64_t* bar_m2 = bars + 11;
+  uint64_t* bar_cm = bars + 12;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 14);
   // q/k loads issued per slot: [0..1] by the producer, [2..3] by the consumer
-  int* issued = reinterpret_cast<int*>(bars + 13);
+  int* issued = reinterpret_cast<int*>(bars + 15);
 
   const int tid = threadIdx.x, warp = tid >> 5;
   const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
@@ -227,7 +262,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar_in + s, 1);
       mbar_init(full + s, 1);
-      mbar_init(send_ok + s, 2);
+      mbar_init(pfull + s, 1);
+      mbar_init(send_ok + s, 1);
       mbar_init(bar_v + s, 1);
     }
     mbar_init(bar_m1, 1);
@@ -254,7 +290,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   tc_fence_after();
   cluster_sync_all();  // both CTAs' barriers exist before any remote access
   const uint32_t tmem = *tmem_slot;
-  const uint32_t peer_full = peer_addr(full, peer);
+  const uint32_t peer_pfull = peer_addr(pfull, peer);
   const uint32_t peer_ok = peer_addr(send_ok, peer);
   const uint32_t peer_slots = peer_addr(sm, peer);
   const uint32_t peer_abort = peer_addr((const void*)abort_flag, peer);
@@ -316,8 +352,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 t < kC && t < end - tok0);
     }
     uint32_t ph_m1 = 0, ph_m2 = 0;
-    int ack_slot = -1;       // own slot whose outgoing copy awaits its ack
-    bool send_fail = false;  // thread 0: a wait for the peer's slot gave up
+    // thread 0's push state for the current chunk
+    bool send_fail = false;  // a wait for the peer's slot gave up
+    bool slot_ok = false, sent_early = false, sent_tp = false;
 
     for (int j = 0; j < n_own; ++j) {
       const int n = (int)r + 2 * j;
@@ -335,6 +372,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       beta_next = 0.f;
       ldg_f1_if(beta_next, p.beta + (size_t)(tok0 + 2 * kC + t) * p.H + h,
                 t < kC && has_next && t < end - (tok0 + 2 * kC));
+      if (t == 0 && has_next) {  // the next own chunk's q and k into L2
+#pragma unroll
+        for (int q = 0; q < (int)Lay::NP; ++q) {
+          prefetch_box_l2(&tm_q, q * 64, h, tok0 + 2 * kC);
+          prefetch_box_l2(&tm_k, q * 64, h, tok0 + 2 * kC);
+        }
+      }
       const uint32_t wn = s ? waited1 : waited0;
       bool ok = wait_or_abort<true>(bar_in + s, wn & 1u, abort_flag);
       if (ok) {
@@ -345,6 +389,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         failed = true;
         break;
       }
+      const uint32_t ps = (uint32_t)j & 1u;  // the peer's slot for this chunk
+      const uint32_t pdst = peer_slots + ps * Lay::slot;
+      const uint32_t pbar = peer_pfull + 8u * ps;
+      // The peer's slot ps is free once the peer's consumer has used the
+      // peer's own chunk before this one there (send_ok) and the peer's copy
+      // of that chunk to this CTA has been read out, which the arrival of
+      // all its bytes here (pfull) proves.  The first chunks find it free.
+      auto peer_slot_free = [&](bool block) {
+        const int ip = j + (int)r - 1;  // that chunk, as this CTA's peer chunk
+        if (ip < 0) return true;
+        const uint32_t par = (uint32_t)(ip >> 1) & 1u;
+        uint64_t* pf = pfull + (ip & 1);
+        return block ? wait_cluster(send_ok + ps, par, abort_flag) &&
+                           wait_cluster(pf, par, abort_flag)
+                     : test_wait_cluster(send_ok + ps, par) &&
+                           test_wait_cluster(pf, par);
+      };
+      auto push_early = [&]() {  // Qt, Kb, P, exp(g_C)
+        remote_arrive_tx(pbar, Lay::push_bytes);
+#pragma unroll
+        for (int q = 0; q < (int)Lay::NP; ++q)
+          copy_to_peer(pdst + q * 16384 + 8192, slot + q * 16384 + 8192, 8192,
+                       pbar);
+        copy_to_peer(pdst + Lay::s_kb, slot + Lay::s_kb, Lay::kb_bytes, pbar);
+        copy_to_peer(pdst + Lay::s_pp, slot + Lay::s_pp, 8192, pbar);
+        copy_to_peer(pdst + Lay::s_gc, slot + Lay::s_gc, DK * 4, pbar);
+        sent_early = true;
+      };
+      if (t == 0) slot_ok = sent_early = sent_tp = false;
 
       // ---- prologue, in place over the raw q and k in the slot
       prologue_rows<DK, GATE>(la_reg, afp, gc, kq + pnl * 16384 + 8192,
@@ -365,11 +438,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                    idesc, ks > 0);
         }
         mma_commit(bar_m1);
-        if (ack_slot >= 0) {  // the previous outgoing copy has long been read
-          bulk_wait_read();
-          remote_arrive(peer_ok + 8u * (uint32_t)ack_slot);
-          ack_slot = -1;
-        }
       }
 
       // ---- A (fp32) and P (bf16 into the slot)
@@ -403,7 +471,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
       }
       tc_fence_before();
+      fence_proxy_async();  // P, to the copy engine
       named_sync(kBarProd, kProd);
+      if (t == 0) {
+        slot_ok = peer_slot_free(false);
+        if (slot_ok) push_early();
+      }
 
       invert_unit_lower(afp, tfp, reinterpret_cast<float*>(sm + Lay::msc), t);
 
@@ -425,6 +498,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       fence_proxy_async();
       named_sync(kBarProd, kProd);
       if (t == 0) {  // MMA2: W = T' Kt (N = DK)
+        if (!slot_ok) slot_ok = peer_slot_free(false);
+        if (slot_ok) {
+          if (!sent_early) push_early();
+          copy_to_peer(pdst + Lay::s_tp, tp, 8192, pbar);
+          sent_tp = true;
+        }
         tc_fence_after();
         const uint32_t iw = idesc_bf16(128, DK, false, true);
 #pragma unroll
@@ -456,30 +535,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       named_sync(kBarProd, kProd);
       if (t == 0) {
         mbar_arrive(full + s);  // to this CTA's consumer
-        // to the peer: its slot j & 1, once the peer's chunk before it there
-        // has been used and its copy read
-        const uint32_t ps = (uint32_t)j & 1u;
-        bool sent = true;
-        if (j - 1 + (int)r >= 0)
-          sent = wait_cluster(send_ok + ps, (uint32_t)((j + (int)r - 1) >> 1) & 1u,
-                              abort_flag);
-        if (sent) {
-          remote_arrive_tx(peer_full + 8u * ps, Lay::copy_bytes);
-          copy_to_peer(peer_slots + ps * Lay::slot, slot, Lay::copy_bytes,
-                       peer_full + 8u * ps);
+        if (!slot_ok) slot_ok = peer_slot_free(true);
+        if (slot_ok) {  // the rest of the package: (Qt, Kb, P, T') and W
+          if (!sent_early) push_early();
+          if (!sent_tp) copy_to_peer(pdst + Lay::s_tp, tp, 8192, pbar);
+#pragma unroll
+          for (int q = 0; q < (int)Lay::NP; ++q)
+            copy_to_peer(pdst + q * 16384, slot + q * 16384, 8192, pbar);
           bulk_commit();
-          ack_slot = s;
         } else {
           send_fail = true;
         }
       }
     }
     failed = named_sync_or(kBarProd, kProd, failed || send_fail);
-    if (t == 0 && !failed && ack_slot >= 0) {
-      bulk_wait_read();
-      remote_arrive(peer_ok + 8u * (uint32_t)ack_slot);
-    }
-    if (failed && t == 0) raise_abort();
+    if (t == 0 && failed) raise_abort();
   } else {
     // =================================================== consumer role
     const int c = tid - kProd;  // TMEM lane = accumulator row
@@ -518,7 +588,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     int v_issued = 0;
     if (c == 0 && nch > 0) issue_v(0);
     v_issued = nch > 0 ? 1 : 0;
-    uint32_t ph_cm = 0, fph = 0u;  // bit s: parity of slot s's next fill
+    uint32_t ph_cm = 0;
     int n = 0;
     for (; n < nch; ++n) {
       const int s = ((n + (int)r) >> 1) & 1;
@@ -536,8 +606,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (c == 0) issue_v(n + 1);
         v_issued = n + 2;
       }
-      bool ok = wait_cluster(full + s, (fph >> s) & 1u, abort_flag);
-      fph ^= 1u << s;
+      // own chunk j = n >> 1 is the (j >> 1)-th own use of its slot; peer
+      // chunk i = n >> 1 the (i >> 1)-th peer use
+      const uint32_t par = (uint32_t)(n >> 2) & 1u;
+      bool ok = wait_cluster((own ? full : pfull) + s, par, abort_flag);
       ok = ok && wait_or_abort<false>(bar_v + (n & 1), (uint32_t)(n >> 1) & 1u,
                                       abort_flag);
       if (named_sync_or(kBarCons, kCons, !ok)) {
@@ -548,6 +620,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
       // ---- U = T' V ; [W; Qt] . S
       if (c == 0) {
+        if (!own) fence_proxy_async();  // the peer's stores, to the MMA reads
         const uint32_t idesc = idesc_bf16(128, 64, false, true);
 #pragma unroll
         for (int ks = 0; ks < kC / 16; ++ks)
@@ -689,9 +762,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (uint32_t m = done; m < (uint32_t)(issued[s] + issued[2 + s]); ++m)
         mbar_wait(bar_in + s, m & 1u, 100000000ull);
     }
+    bulk_commit();  // copies issued before a failure cut the chunk short
     bulk_wait_all();  // outgoing copies complete before the peer may leave
   }
-  __syncthreads();
   cluster_sync_all();
   if (warp == 0) tmem_dealloc(tmem, 512);
 }
