@@ -352,7 +352,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 t < kC && t < end - tok0);
     }
     uint32_t ph_m1 = 0, ph_m2 = 0;
-    // thread 0's push state for the current chunk
+    // Thread 32 (the copier) sends the package to the peer, so that the
+    // copies' issue never holds up thread 0's MMAs; its state per chunk:
+    const bool copier = t == 32;
     bool send_fail = false;  // a wait for the peer's slot gave up
     bool slot_ok = false, sent_early = false, sent_tp = false;
 
@@ -417,7 +419,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         copy_to_peer(pdst + Lay::s_gc, slot + Lay::s_gc, DK * 4, pbar);
         sent_early = true;
       };
-      if (t == 0) slot_ok = sent_early = sent_tp = false;
+      if (copier) slot_ok = sent_early = sent_tp = false;
 
       // ---- prologue, in place over the raw q and k in the slot
       prologue_rows<DK, GATE>(la_reg, afp, gc, kq + pnl * 16384 + 8192,
@@ -473,10 +475,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tc_fence_before();
       fence_proxy_async();  // P, to the copy engine
       named_sync(kBarProd, kProd);
-      if (t == 0) {
-        slot_ok = peer_slot_free(false);
-        if (slot_ok) push_early();
-      }
 
       invert_unit_lower(afp, tfp, reinterpret_cast<float*>(sm + Lay::msc), t);
 
@@ -497,13 +495,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       fence_proxy_async();
       named_sync(kBarProd, kProd);
-      if (t == 0) {  // MMA2: W = T' Kt (N = DK)
-        if (!slot_ok) slot_ok = peer_slot_free(false);
+      if (copier) {  // early parts to the peer while MMA2 runs
+        slot_ok = peer_slot_free(false);
         if (slot_ok) {
-          if (!sent_early) push_early();
+          push_early();
           copy_to_peer(pdst + Lay::s_tp, tp, 8192, pbar);
           sent_tp = true;
         }
+      }
+      if (t == 0) {  // MMA2: W = T' Kt (N = DK)
         tc_fence_after();
         const uint32_t iw = idesc_bf16(128, DK, false, true);
 #pragma unroll
@@ -533,8 +533,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tc_fence_before();
       fence_proxy_async();
       named_sync(kBarProd, kProd);
-      if (t == 0) {
-        mbar_arrive(full + s);  // to this CTA's consumer
+      if (t == 0) mbar_arrive(full + s);  // to this CTA's consumer
+      if (copier) {
         if (!slot_ok) slot_ok = peer_slot_free(true);
         if (slot_ok) {  // the rest of the package: (Qt, Kb, P, T') and W
           if (!sent_early) push_early();
@@ -550,6 +550,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     failed = named_sync_or(kBarProd, kProd, failed || send_fail);
     if (t == 0 && failed) raise_abort();
+    if (copier) {
+      bulk_commit();  // copies issued before a failure cut the chunk short
+      bulk_wait_all();  // outgoing copies complete before the peer may leave
+    }
   } else {
     // =================================================== consumer role
     const int c = tid - kProd;  // TMEM lane = accumulator row
@@ -762,8 +766,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (uint32_t m = done; m < (uint32_t)(issued[s] + issued[2 + s]); ++m)
         mbar_wait(bar_in + s, m & 1u, 100000000ull);
     }
-    bulk_commit();  // copies issued before a failure cut the chunk short
-    bulk_wait_all();  // outgoing copies complete before the peer may leave
   }
   cluster_sync_all();
   if (warp == 0) tmem_dealloc(tmem, 512);
