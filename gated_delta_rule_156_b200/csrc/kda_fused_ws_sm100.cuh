@@ -185,11 +185,66 @@ __device__ __forceinline__ void st_chunks(uint8_t* panel, int row, int c0,
   }
 }
 
+// C = A B (or -A B) for 32 x 32 fp32 tiles in shared memory (leading
+// dimensions in floats), on 256 threads: each thread accumulates a 4 x 4
+// block of C over a quarter of K, the four quarters sit on lanes l, l ^ 8,
+// l ^ 16, l ^ 24 and are summed with shuffles, and each of the four lanes
+// then stores one row of the block.  Four 128-bit loads of A and four of B
+// feed 64 FMAs, which keeps the shared-memory load bytes per FMA low.
+template <bool NEG>
+__device__ __forceinline__ void mm32_tiles(const float* Ab, int lda,
+                                           const float* Bb, int ldb, float* Cb,
+                                           int ldc, int t) {
+  const int q = (t >> 3) & 3;
+  const int tile = (t >> 5) * 8 + (t & 7);
+  const int tr = tile >> 3, tc = tile & 7;
+  float m[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) m[i][j] = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < 8; kk += 4) {
+    const int k4 = q * 8 + kk;
+    float4 a[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      a[i] = *reinterpret_cast<const float4*>(Ab + (4 * tr + i) * lda + k4);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float4 x = *reinterpret_cast<const float4*>(Bb + (k4 + u) * ldb + 4 * tc);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float av = u == 0 ? a[i].x : u == 1 ? a[i].y : u == 2 ? a[i].z : a[i].w;
+        m[i][0] += av * x.x; m[i][1] += av * x.y;
+        m[i][2] += av * x.z; m[i][3] += av * x.w;
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      m[i][j] += __shfl_xor_sync(0xffffffffu, m[i][j], 8);
+      m[i][j] += __shfl_xor_sync(0xffffffffu, m[i][j], 16);
+    }
+  float4 w;
+  w.x = q == 0 ? m[0][0] : q == 1 ? m[1][0] : q == 2 ? m[2][0] : m[3][0];
+  w.y = q == 0 ? m[0][1] : q == 1 ? m[1][1] : q == 2 ? m[2][1] : m[3][1];
+  w.z = q == 0 ? m[0][2] : q == 1 ? m[1][2] : q == 2 ? m[2][2] : m[3][2];
+  w.w = q == 0 ? m[0][3] : q == 1 ? m[1][3] : q == 2 ? m[2][3] : m[3][3];
+  if (NEG) {
+    w.x = -w.x; w.y = -w.y; w.z = -w.z; w.w = -w.w;
+  }
+  *reinterpret_cast<float4*>(Cb + (4 * tr + q) * ldc + 4 * tc) = w;
+}
+
 // (I + A)^-1 of the strictly-lower 64 x 64 A (row stride kFS) into X by
 // recursive doubling on unit-lower blocks,
 //   [L11 0; L21 L22]^-1 = [X11 0; -X22 L21 X11  X22]:
 // the four 16 x 16 diagonal blocks by forward substitution, then blocks
-// (1,0) and (3,2), then the 32 x 32 coupling block.  256 producer threads;
+// (1,0) and (3,2), then the 32 x 32 coupling block (register-tiled products,
+// mm32_tiles).  256 producer threads;
 // X's strictly-upper part outside the diagonal blocks must be zero.
 __device__ __forceinline__ void invert_unit_lower(const float* A, float* X,
                                                   float* M, int t) {
@@ -257,38 +312,9 @@ __device__ __forceinline__ void invert_unit_lower(const float* A, float* X,
         make_float2(y0, y1);
   }
   named_sync(kBarProd, kProd);
-  {
-    const int r = t >> 3, c = (t & 7) * 4;
-    float m[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int k = 0; k < 32; k += 4) {
-      const float4 a4 = *reinterpret_cast<const float4*>(A + (32 + r) * kFS + k);
-      const float av[4] = {a4.x, a4.y, a4.z, a4.w};
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float4 x4 = *reinterpret_cast<const float4*>(X + (k + u) * kFS + c);
-        m[0] += av[u] * x4.x; m[1] += av[u] * x4.y;
-        m[2] += av[u] * x4.z; m[3] += av[u] * x4.w;
-      }
-    }
-    *reinterpret_cast<float4*>(M + r * 32 + c) = make_float4(m[0], m[1], m[2], m[3]);
-    named_sync(kBarProd, kProd);
-    float y[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int k = 0; k < 32; k += 4) {
-      const float4 x4 =
-          *reinterpret_cast<const float4*>(X + (32 + r) * kFS + 32 + k);
-      const float xv[4] = {x4.x, x4.y, x4.z, x4.w};
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float4 m4 = *reinterpret_cast<const float4*>(M + (k + u) * 32 + c);
-        y[0] -= xv[u] * m4.x; y[1] -= xv[u] * m4.y;
-        y[2] -= xv[u] * m4.z; y[3] -= xv[u] * m4.w;
-      }
-    }
-    *reinterpret_cast<float4*>(X + (32 + r) * kFS + c) =
-        make_float4(y[0], y[1], y[2], y[3]);
-  }
+  mm32_tiles<false>(A + 32 * kFS, kFS, X, kFS, M, 32, t);  // M = L21 X11
+  named_sync(kBarProd, kProd);
+  mm32_tiles<true>(X + 32 * kFS + 32, kFS, M, 32, X + 32 * kFS, kFS, t);
   named_sync(kBarProd, kProd);
 }
 
