@@ -364,6 +364,47 @@ def run_kda(args, world, rank, local):
     }
     del q_raw, k_raw, x_raw
 
+    # ---- packed variable-length batch with one long context: 16 sequences
+    # of 256..16384 tokens and one of 131072 (H = 32, d = 128, with initial
+    # states), the workload whose long serial chunk chain bounds the time ---
+    d3 = W.make(3, device=dev, seed=W.seed_of(3) + 97 * rank)
+    T3 = d3["q"].shape[1]
+    n3 = len(d3["lengths"])
+    c3 = W.CONFIGS[3]
+    out3 = torch.empty_like(d3["v"])
+    fin3 = torch.empty_like(d3["initial_state"])
+
+    def prefill_packed(_i):
+        K.chunk_fwd(d3["q"], d3["k"], d3["v"], d3["log_alpha"], d3["beta"],
+                    d3["initial_state"], d3["cu_seqlens"], chunk=C, out=out3,
+                    final_state=fin3)
+
+    for i in range(2):
+        prefill_packed(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    p3_steps = max(2, min(args.steps, 5))
+    p3ms, p3per = timed(prefill_packed, p3_steps, stream)
+    barrier(world)
+    p3ms = max_over_ranks(p3ms, world)
+    state_b = c3["H"] * c3["dk"] * c3["dv"] * 4
+    p3bytes = (prefill_bytes(1, T3, c3["H"], c3["dk"], c3["dv"]) - state_b
+               + 2 * n3 * state_b)  # every sequence's state read and written
+    p3_launch = statistics.mean(p3per)
+    packed_long = {
+        "value": world * T3 / (p3ms / p3_steps * 1e-3), "unit": "tokens/s",
+        "ms_per_step": p3ms / p3_steps, "steps": p3_steps,
+        "workload": f"kda_chunk_fwd packed: {n3 - 1} sequences of "
+                    f"{c3['len_lo']}..{c3['len_hi']} tokens + one of "
+                    f"{c3['long_len']} ({T3} tokens), H=32 d=128 bf16, "
+                    "initial states in, final states out",
+        "hbm": {"achieved": p3bytes / (p3_launch * 1e-3) / 1e9, "unit": "GB/s",
+                "frac": p3bytes / (p3_launch * 1e-3) / 1e9 / pk["hbm_gbs"],
+                "algorithmic_bytes_per_launch": p3bytes},
+        "serial_chain_chunks": max(d3["lengths"]) // C,
+    }
+    del d3, out3, fin3
+
     # ---- end to end through the public API with host buffers ------------
     host = {n: d[n].cpu().pin_memory() for n in
             ("q", "k", "v", "log_alpha", "beta")}
@@ -453,6 +494,7 @@ def run_kda(args, world, rank, local):
                 "gpu_launches": args.steps,
             },
             "prefill_head_gate": head_gate,
+            "prefill_packed_long": packed_long,
             "prefill_fused_prologue": fused_prologue,
             "e2e": {"value": e2e_value, "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
