@@ -4,7 +4,8 @@ TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
 CPU-baseline leg of ``bench.py`` may import this module.  It shares no code with
 the CUDA path and imports nothing from it.
 
-Three independent CPU computations of the same quantity:
+Three independent CPU computations of the same forward quantity, and its
+gradients:
 
 ``recurrent``     the plain definition, token by token, in C (kda_recurrence.c,
                   fp64, OpenMP over (sequence, head)).  This is the oracle.
@@ -14,6 +15,9 @@ Three independent CPU computations of the same quantity:
                   S_t = M_t ... M_1 S_0 + sum_i (M_t ... M_{i+1}) b_i k_i v_i^T.
                   Each prefix t is recomputed from scratch, so it is not the
                   recurrence evaluated a second time.
+``recurrent_bwd`` the reverse-mode gradients of ``recurrent`` (the chain rule
+                  applied line by line to the token step, in C, fp64), pinned
+                  by central finite differences of ``recurrent``.
 ``chunked_debug`` an fp64 model of the chunkwise rewrite that the GPU prefill
                   kernels use (decay prefix sums, the strictly-lower factor
                   matrix A, T = (I + A)^-1 by forward substitution, W, U, the
@@ -52,6 +56,9 @@ def _load(path=None):
         lib.kda_oracle_recurrent.restype = ctypes.c_int
         lib.kda_oracle_recurrent.argtypes = [
             I64, ctypes.POINTER(I64), I64, I64, I64, P, P, P, P, P, P, P, P]
+        lib.kda_oracle_recurrent_bwd.restype = ctypes.c_int
+        lib.kda_oracle_recurrent_bwd.argtypes = [
+            I64, ctypes.POINTER(I64), I64, I64, I64] + [P] * 14
         lib.kda_oracle_num_threads.restype = ctypes.c_int
         lib.kda_oracle_num_threads.argtypes = []
         _libs[path] = lib
@@ -119,6 +126,54 @@ def recurrent(q, k, v, log_alpha, beta, initial_state=None, seq_offsets=None,
     if rc != 0:
         raise RuntimeError(f"kda_oracle_recurrent failed ({rc})")
     return out, fin
+
+
+def recurrent_bwd(q, k, v, log_alpha, beta, initial_state, d_out,
+                  d_final_state=None, seq_offsets=None, library=None):
+    """Gradients of the token-by-token recurrence (reverse mode, fp64) for
+    L = sum(d_out * out) + sum(d_final_state * final_state), in C
+    (kda_recurrence.c, ``kda_oracle_recurrent_bwd``).
+
+    Shapes as ``recurrent``; d_out like the output, d_final_state like the
+    final state (None = zero).  Returns (dq, dk, dv, dlog_alpha, dbeta,
+    d_initial_state), float64, in the shapes of the corresponding inputs
+    (d_initial_state [n_seqs, H, d_k, d_v] whether or not a state was given).
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    la, b = _f64(log_alpha), _f64(beta)
+    s0, do, dsT = _f64(initial_state), _f64(d_out), _f64(d_final_state)
+    lead = q.shape[:-2]
+    H, dk = q.shape[-2], q.shape[-1]
+    dv = v.shape[-1]
+    if seq_offsets is None:
+        if q.ndim != 4:
+            raise ValueError("without seq_offsets q must be [B, T, H, d_k]")
+        B, T = q.shape[0], q.shape[1]
+        offs = np.arange(B + 1, dtype=np.int64) * T
+    else:
+        if q.ndim == 4 and q.shape[0] != 1:
+            raise ValueError("packed layout needs B == 1")
+        offs = np.ascontiguousarray(np.asarray(seq_offsets, dtype=np.int64))
+    n_seqs = len(offs) - 1
+    if offs[0] != 0 or offs[-1] != int(np.prod(lead)):
+        raise ValueError("seq_offsets must start at 0 and end at the token count")
+    if do.shape != lead + (H, dv):
+        raise ValueError(f"d_out shape {do.shape} != {lead + (H, dv)}")
+    for name, st in (("initial_state", s0), ("d_final_state", dsT)):
+        if st is not None and st.shape != (n_seqs, H, dk, dv):
+            raise ValueError(f"{name} shape {st.shape} != {(n_seqs, H, dk, dv)}")
+    dq, dkk, dla = (np.zeros(lead + (H, dk)) for _ in range(3))
+    dvv = np.zeros(lead + (H, dv))
+    dbeta = np.zeros(lead + (H,))
+    ds0 = np.zeros((n_seqs, H, dk, dv))
+    rc = _load(library).kda_oracle_recurrent_bwd(
+        n_seqs, offs.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), H, dk, dv,
+        _ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(b), _ptr(s0), _ptr(do),
+        _ptr(dsT), _ptr(dq), _ptr(dkk), _ptr(dvv), _ptr(dla), _ptr(dbeta),
+        _ptr(ds0))
+    if rc != 0:
+        raise RuntimeError(f"kda_oracle_recurrent_bwd failed ({rc})")
+    return dq, dkk, dvv, dla, dbeta, ds0
 
 
 def brute_force(q, k, v, log_alpha, beta, initial_state=None):
