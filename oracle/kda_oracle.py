@@ -263,6 +263,90 @@ def chunked_debug(q, k, v, log_alpha, beta, initial_state=None, chunk=64):
     return rec
 
 
+def chunked_bwd_debug(q, k, v, log_alpha, beta, initial_state, d_out,
+                      d_final_state=None, chunk=64):
+    """fp64 model of the chunkwise backward for ONE (sequence, head): the chain
+    rule applied to each line of ``chunked_debug``, chunk by chunk in reverse.
+
+    Per chunk, with G = Diag(exp(g_C)) dS_C (dS_C the gradient of the state
+    leaving the chunk):
+      S_C = Diag(exp(g_C)) (S_0 + Kb^T Delta):
+          dS_0 = G, dDelta = Kb G, dKb = Delta G^T,
+          d exp(g_C) = rowsum((S_0 + Kb^T Delta) * dS_C)
+      O = Qt S_0 + P Delta, P = lower_incl(Qt Kb^T):
+          dQt = dO S_0^T + dP Kb, dS_0 += Qt^T dO, dDelta += P^T dO,
+          dP = lower_incl(dO Delta^T), dKb += dP^T Qt
+      Delta = U - W S_0:  dU = dDelta, dW = -dDelta S_0^T, dS_0 -= W^T dDelta
+      W = Tm Diag(b) Kt, U = Tm Diag(b) V:
+          dTm = dW (b Kt)^T + dU (b V)^T, dKt = b Tm^T dW, dV = b Tm^T dU,
+          db = rowsum(Tm^T dW * Kt) + rowsum(Tm^T dU * V)
+      Tm = (I + A)^-1:  dA = strictly_lower(-Tm^T dTm Tm^T)
+      A = strictly_lower(Diag(b) Kt Kb^T):
+          db += rowsum(dA * Kt Kb^T), dKt += (b dA) Kb, dKb += (b dA)^T Kt
+      Kt = k e^g, Kb = k e^-g, Qt = q e^g:
+          dk = dKt e^g + dKb e^-g, dq = dQt e^g,
+          dg = dKt * Kt + dQt * Qt - dKb * Kb  (+ exp(g_C) d exp(g_C) on row C)
+      g = cumsum(l):  dl = reverse cumsum of dg within the chunk
+    and dS_0 becomes the previous chunk's dS_C.  Returns (dq, dk, dv,
+    dlog_alpha, dbeta, d_initial_state) in float64.  Used to check the
+    chunkwise algebra the GPU backward follows; pinned to ``recurrent_bwd``.
+    """
+    q, k, v, la, b, do = map(_f64, (q, k, v, log_alpha, beta, d_out))
+    T, dk = k.shape
+    dv = v.shape[1]
+    fwd = chunked_debug(q, k, v, la, b, initial_state, chunk)
+    dq, dkk, dla = np.zeros((T, dk)), np.zeros((T, dk)), np.zeros((T, dk))
+    dvv, db = np.zeros((T, dv)), np.zeros(T)
+    dS = np.zeros((dk, dv)) if d_final_state is None else _f64(d_final_state).copy()
+    for ci in reversed(range(len(fwd["g"]))):
+        c0 = ci * chunk
+        c1 = min(T, c0 + chunk)
+        kc, qc, vc, bc, doc = k[c0:c1], q[c0:c1], v[c0:c1], b[c0:c1], do[c0:c1]
+        g, Tm, W, U, S0 = (fwd[n][ci] for n in ("g", "Tm", "W", "U", "S_start"))
+        eg, emg = np.exp(g), np.exp(-g)
+        Kt, Kb, Qt = kc * eg, kc * emg, qc * eg
+        gam = eg[-1]
+        Delta = U - W @ S0
+        P = np.tril(Qt @ Kb.T, 0)
+        # S_C = Diag(gam) (S_0 + Kb^T Delta)
+        G = gam[:, None] * dS
+        dS0 = G.copy()
+        dDelta = Kb @ G
+        dKb = Delta @ G.T
+        dgam = ((S0 + Kb.T @ Delta) * dS).sum(axis=1)
+        # O = Qt S_0 + P Delta
+        dQt = doc @ S0.T
+        dS0 += Qt.T @ doc
+        dP = np.tril(doc @ Delta.T, 0)
+        dDelta += P.T @ doc
+        dQt += dP @ Kb
+        dKb += dP.T @ Qt
+        # Delta = U - W S_0
+        dW = -dDelta @ S0.T
+        dS0 -= W.T @ dDelta
+        # W = Tm (b Kt), U = Tm (b V)
+        BK, BV = bc[:, None] * Kt, bc[:, None] * vc
+        dTm = dW @ BK.T + dDelta @ BV.T
+        dBK, dBV = Tm.T @ dW, Tm.T @ dDelta
+        dKt = bc[:, None] * dBK
+        dvv[c0:c1] = bc[:, None] * dBV
+        db[c0:c1] = (dBK * Kt).sum(axis=1) + (dBV * vc).sum(axis=1)
+        # Tm = (I + A)^-1, A = strictly_lower(b Kt Kb^T)
+        dA = np.tril(-Tm.T @ dTm @ Tm.T, -1)
+        db[c0:c1] += (dA * (Kt @ Kb.T)).sum(axis=1)
+        dM = bc[:, None] * dA
+        dKt += dM @ Kb
+        dKb += dM.T @ Kt
+        # Kt = k e^g, Kb = k e^-g, Qt = q e^g, g = cumsum(l)
+        dkk[c0:c1] = dKt * eg + dKb * emg
+        dq[c0:c1] = dQt * eg
+        dg = dKt * Kt + dQt * Qt - dKb * Kb
+        dg[-1] += dgam * gam
+        dla[c0:c1] = np.cumsum(dg[::-1], axis=0)[::-1]
+        dS = dS0
+    return dq, dkk, dvv, dla, db, dS
+
+
 def prologue(q, k, gate, normalize_qk=True, q_scale=1.0, gate_logits=True,
              gate_scale=1.0):
     """The optional input prologue, in fp64, as its plain definition:

@@ -144,3 +144,18 @@ def test_backward_pins_catch_planted_mistake(name, tmp_path):
     inputs, do, dsT = case(rng, (1, 6), 1, 3, 2, 1)
     assert fd_error(inputs, do, dsT, library=lib) > 1e-3, name
     os.remove(lib)
+
+
+@pytest.mark.parametrize("T,C", [(150, 64), (150, 32), (37, 16), (1, 16)])
+def test_chunked_backward_model_matches_oracle(T, C):
+    # the chunkwise backward algebra (the GPU backward's recipe) against the
+    # token-level gradients
+    rng = np.random.default_rng(50 + T + C)
+    (q, k, v, la, b, s0), do, dsT = case(rng, (1, T), 1, 6, 5, 1)
+    ref = kda_oracle.recurrent_bwd(q, k, v, la, b, s0, do, dsT)
+    got = kda_oracle.chunked_bwd_debug(q[0, :, 0], k[0, :, 0], v[0, :, 0],
+                                       la[0, :, 0], b[0, :, 0], s0[0, 0],
+                                       do[0, :, 0], dsT[0, 0], chunk=C)
+    refs = [r[0, :, 0] for r in ref[:5]] + [ref[5][0, 0]]
+    for g, r in zip(got, refs):
+        np.testing.assert_allclose(g, r, rtol=1e-10, atol=1e-10)
