@@ -225,6 +225,99 @@ kda_status kda_chunk_fwd_staged(const kda_shape* shape, const void* q,
   return run_with_workspace(kda::staged_workspace_bytes(a), stream, false, a);
 }
 
+kda_status kda_chunk_bwd(const kda_shape* shape, const void* q, const void* k,
+                         const void* v, const float* log_alpha,
+                         const float* beta, const float* initial_state,
+                         const int32_t* cu_seqlens, const void* d_out,
+                         const float* d_final_state, void* dq, void* dk,
+                         void* dv, float* d_log_alpha, float* d_beta,
+                         float* d_initial_state, cudaStream_t stream) {
+  int n_seqs = 0;
+  kda_status st = validate_chunk_shape(shape, cu_seqlens != nullptr, &n_seqs);
+  if (st != KDA_OK) return st;
+  const size_t esz = shape->io_dtype == KDA_BF16 ? 2 : 4;
+  const size_t tokens = (size_t)shape->B * (size_t)shape->T;
+  const size_t H = shape->H, dkk = shape->dk, dvv = shape->dv;
+  if (tokens > 0 && (!q || !k || !v || !log_alpha || !beta || !d_out || !dq ||
+                     !dk || !dv || !d_log_alpha || !d_beta))
+    return KDA_ERR_INVALID_ARG;
+  const void* p16[] = {q, k, v, initial_state, d_out, d_final_state, dq, dk,
+                       dv, d_initial_state};
+  for (const void* p : p16)
+    if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
+  const void* p4[] = {log_alpha, beta, cu_seqlens, d_log_alpha, d_beta};
+  for (const void* p : p4)
+    if (p && !aligned4(p)) return KDA_ERR_MISALIGNED;
+  // No output may overlap an input or another output.
+  const size_t sbytes = (size_t)n_seqs * H * dkk * dvv * 4;
+  const Range ins[] = {span(q, tokens * H * dkk * esz),
+                       span(k, tokens * H * dkk * esz),
+                       span(v, tokens * H * dvv * esz),
+                       span(log_alpha, tokens * H * dkk * 4),
+                       span(beta, tokens * H * 4),
+                       span(initial_state, sbytes),
+                       span(cu_seqlens, cu_seqlens ? 4 * ((size_t)n_seqs + 1) : 0),
+                       span(d_out, tokens * H * dvv * esz),
+                       span(d_final_state, sbytes)};
+  const Range outs[] = {span(dq, tokens * H * dkk * esz),
+                        span(dk, tokens * H * dkk * esz),
+                        span(dv, tokens * H * dvv * esz),
+                        span(d_log_alpha, tokens * H * dkk * 4),
+                        span(d_beta, tokens * H * 4),
+                        span(d_initial_state, sbytes)};
+  for (size_t i = 0; i < 6; ++i) {
+    for (const Range& r : ins)
+      if (overlap(outs[i], r)) return KDA_ERR_INVALID_ARG;
+    for (size_t j = i + 1; j < 6; ++j)
+      if (overlap(outs[i], outs[j])) return KDA_ERR_INVALID_ARG;
+  }
+  kda::BwdArgs b{};
+  b.f.q = q;
+  b.f.k = k;
+  b.f.v = v;
+  b.f.log_alpha = log_alpha;
+  b.f.beta = beta;
+  b.f.initial_state = initial_state;
+  b.f.cu_seqlens = cu_seqlens;
+  fill_args(shape, n_seqs, &b.f);
+  b.d_out = d_out;
+  b.d_final_state = d_final_state;
+  b.dq = dq;
+  b.dk = dk;
+  b.dv = dv;
+  b.d_log_alpha = d_log_alpha;
+  b.d_beta = d_beta;
+  b.d_initial_state = d_initial_state;
+  void* ws = nullptr;
+  cudaError_t e;
+  const size_t bytes = kda::bwd_workspace_bytes(b);
+  if (bytes) {
+    keep_pool_memory();
+    if ((e = cudaMallocAsync(&ws, bytes, stream)) != cudaSuccess)
+      return cuda_fail(e);
+  }
+  e = kda::launch_bwd(b, ws, stream);
+  if (ws) {
+    const cudaError_t f = cudaFreeAsync(ws, stream);
+    if (e == cudaSuccess) e = f;
+  }
+  return e == cudaSuccess ? KDA_OK : cuda_fail(e);
+}
+
+kda_status kda_chunk_bwd_plan(const kda_shape* shape, int packed, int* kernels,
+                              size_t* workspace_bytes) {
+  int n_seqs = 0;
+  const kda_status st = validate_chunk_shape(shape, packed != 0, &n_seqs);
+  if (st != KDA_OK) return st;
+  kda::BwdArgs b{};
+  fill_args(shape, n_seqs, &b.f);
+  static const int32_t kTag = 0;  // only tells the planner the layout
+  b.f.cu_seqlens = packed ? &kTag : nullptr;
+  if (kernels) *kernels = kda::bwd_kernel_count(b);
+  if (workspace_bytes) *workspace_bytes = kda::bwd_workspace_bytes(b);
+  return KDA_OK;
+}
+
 kda_status kda_chunk_fwd_gated(const kda_shape* shape, int gate, const void* q,
                                const void* k, const void* v,
                                const float* log_gate, const float* beta,

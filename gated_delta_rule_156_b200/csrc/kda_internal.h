@@ -63,6 +63,38 @@ size_t staged_workspace_bytes(const ChunkArgs& a);
 int staged_kernel_count(const ChunkArgs& a);
 cudaError_t launch_staged(const ChunkArgs& a, void* workspace,
                           cudaStream_t stream);
+// Stages (1)-(3) only (no outputs; the final state still goes to
+// a.final_state), leaving in the workspace what the backward pass reads:
+// the packed-layout chunk offsets, g = cumulative log-decay [tokens, H, dk],
+// W [tokens, H, dk], Delta = U - W S_0 [tokens, H, dv] and every chunk-start
+// state [max_chunks, H, dk, dv], all fp32.  Channel gate, no prologue.
+struct StagedView {
+  const int32_t* chunk_off;
+  const float* g;
+  const float* w;
+  const float* d;
+  const float* s;
+};
+cudaError_t launch_staged_state(const ChunkArgs& a, void* workspace,
+                                StagedView* view, cudaStream_t stream);
+
+// Chunkwise backward pass (kda_backward.cu): the gradients of
+// L = <d_out, out> + <d_final_state, final_state> with respect to q, k, v,
+// log(alpha), beta and the initial state, all arithmetic in fp32.
+struct BwdArgs {
+  ChunkArgs f;                  // forward arguments; f.out, f.final_state unused
+  const void* d_out;            // [tokens, H, dv], io dtype
+  const float* d_final_state;   // [n_seqs, H, dk, dv] or null (zero)
+  void* dq;                     // [tokens, H, dk], io dtype
+  void* dk;                     // [tokens, H, dk], io dtype
+  void* dv;                     // [tokens, H, dv], io dtype
+  float* d_log_alpha;           // [tokens, H, dk]
+  float* d_beta;                // [tokens, H]
+  float* d_initial_state;       // [n_seqs, H, dk, dv] or null (not wanted)
+};
+size_t bwd_workspace_bytes(const BwdArgs& a);
+int bwd_kernel_count(const BwdArgs& a);
+cudaError_t launch_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream);
 
 // Fused tensor-core prefill (kda_fused_sm100.cu): bf16 io, dk, dv in
 // {64, 128}, chunk 64.  `workspace` must hold fused_workspace_bytes(a).

@@ -377,7 +377,8 @@ cudaError_t set_smem(K kernel, size_t bytes) {
 }
 
 template <typename IO>
-cudaError_t run(const ChunkArgs& a, void* workspace, cudaStream_t stream) {
+cudaError_t run(const ChunkArgs& a, void* workspace, cudaStream_t stream,
+                bool outputs = true) {
   Ws w = carve(a, workspace, nullptr);
   const int C = a.chunk, H = a.H, dk = a.dk, dv = a.dv;
   const int64_t nch = max_chunks(a);
@@ -413,7 +414,7 @@ cudaError_t run(const ChunkArgs& a, void* workspace, cudaStream_t stream) {
       a.n_seqs, a.T, H, dk, dv, C);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
-  if (nch > 0) {
+  if (nch > 0 && outputs) {
     const size_t sm4 = 4 * (2 * (size_t)C * dk + (size_t)C * C +
                             (size_t)dk * kDvTile + (size_t)C * kDvTile);
     if ((e = set_smem(output_kernel<IO>, sm4)) != cudaSuccess) return e;
@@ -438,6 +439,19 @@ int staged_kernel_count(const ChunkArgs& a) {
   const bool any_chunks = max_chunks(a) > 0;
   return (a.cu_seqlens ? 1 : 0) + 1 + (any_chunks ? 3 : 0) +
          (has_prologue(a) && any_chunks ? 1 : 0);
+}
+
+cudaError_t launch_staged_state(const ChunkArgs& a, void* workspace,
+                                StagedView* view, cudaStream_t stream) {
+  Ws w = carve(a, workspace, nullptr);
+  view->chunk_off = w.chunk_off;
+  view->g = w.g;
+  view->w = w.w;
+  view->d = w.u;
+  view->s = w.s;
+  if (a.n_seqs == 0 || a.H == 0) return cudaSuccess;
+  return a.bf16 ? run<__nv_bfloat16>(a, workspace, stream, false)
+                : run<float>(a, workspace, stream, false);
 }
 
 cudaError_t launch_staged(const ChunkArgs& a, void* workspace,

@@ -23,7 +23,8 @@ EXPORTS = ("kda_chunk_fwd", "kda_chunk_fwd_staged", "kda_recurrent_step",
            "kda_status_string", "kda_last_cuda_error", "kda_version",
            "kda_chunk_fwd_staged_noalloc", "kda_chunk_fwd_gated",
            "kda_recurrent_step_gated", "kda_chunk_fwd_ex",
-           "kda_recurrent_step_ex", "kda_selftest_timeout")
+           "kda_recurrent_step_ex", "kda_selftest_timeout", "kda_chunk_bwd",
+           "kda_chunk_bwd_plan")
 GATES = {"channel": 0, "head": 1, "none": 2}
 
 
@@ -106,6 +107,12 @@ def library():
         lib.kda_chunk_fwd_plan.argtypes = [
             ctypes.POINTER(KdaShape), ctypes.c_int, ctypes.c_int,
             ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int),
+            ctypes.POINTER(ctypes.c_size_t)]
+        lib.kda_chunk_bwd.restype = ctypes.c_int
+        lib.kda_chunk_bwd.argtypes = [ctypes.POINTER(KdaShape)] + [vp] * 16
+        lib.kda_chunk_bwd_plan.restype = ctypes.c_int
+        lib.kda_chunk_bwd_plan.argtypes = [
+            ctypes.POINTER(KdaShape), ctypes.c_int, ctypes.POINTER(ctypes.c_int),
             ctypes.POINTER(ctypes.c_size_t)]
         lib.kda_selftest_umma.restype = ctypes.c_int
         lib.kda_selftest_umma.argtypes = [ctypes.c_int] * 5 + [vp, vp, vp, vp]
@@ -208,6 +215,57 @@ def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
     if st != KDA_OK:
         raise KdaError(st, "kda_chunk_fwd_staged" if staged else "kda_chunk_fwd")
     return out, final_state
+
+
+def chunk_bwd(q, k, v, log_alpha, beta, initial_state, cu_seqlens, d_out,
+              d_final_state=None, chunk=64, want_initial_state=True,
+              stream=None):
+    """Backward pass of chunk_fwd (kda_chunk_bwd; per-channel gate, no input
+    prologue): the gradients of sum(d_out * out) + sum(d_final_state *
+    final_state).  Shapes as chunk_fwd; d_out like out; d_final_state fp32
+    [N, H, d_k, d_v] or None.  Returns (dq, dk, dv, dlog_alpha, dbeta,
+    d_initial_state) with d_initial_state None unless want_initial_state.
+    """
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    n = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    for name, t, dt in (("q", q, None), ("k", k, q.dtype), ("v", v, q.dtype),
+                        ("log_alpha", log_alpha, torch.float32),
+                        ("beta", beta, torch.float32),
+                        ("initial_state", initial_state, torch.float32),
+                        ("cu_seqlens", cu_seqlens, torch.int32),
+                        ("d_out", d_out, q.dtype),
+                        ("d_final_state", d_final_state, torch.float32)):
+        _check_dev(name, t, dt)
+    dq = torch.empty_like(q)
+    dkk = torch.empty_like(k)
+    dvv = torch.empty_like(v)
+    dla = torch.empty((B, T, H, dk), dtype=torch.float32, device=q.device)
+    dbeta = torch.empty((B, T, H), dtype=torch.float32, device=q.device)
+    ds0 = (torch.empty((n, H, dk, dv), dtype=torch.float32, device=q.device)
+           if want_initial_state else None)
+    shape = KdaShape(B, T, H, dk, dv, chunk, n if cu_seqlens is not None else 0,
+                     _io(q))
+    st = library().kda_chunk_bwd(
+        ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+        _ptr(beta), _ptr(initial_state), _ptr(cu_seqlens), _ptr(d_out),
+        _ptr(d_final_state), _ptr(dq), _ptr(dkk), _ptr(dvv), _ptr(dla),
+        _ptr(dbeta), _ptr(ds0), _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_chunk_bwd")
+    return dq, dkk, dvv, dla, dbeta, ds0
+
+
+def chunk_bwd_plan(B, T, H, dk, dv, chunk, dtype, packed=False, n_seqs=0):
+    """(kernels, workspace_bytes) of a chunk_bwd call of this shape."""
+    io = KDA_BF16 if dtype == torch.bfloat16 else KDA_F32
+    shape = KdaShape(B, T, H, dk, dv, chunk, n_seqs if packed else 0, io)
+    kern, ws = ctypes.c_int(), ctypes.c_size_t()
+    st = library().kda_chunk_bwd_plan(ctypes.byref(shape), int(packed),
+                                      ctypes.byref(kern), ctypes.byref(ws))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_chunk_bwd_plan")
+    return kern.value, ws.value
 
 
 def recurrent_step(q, k, v, log_alpha, beta, state, out=None, stream=None,

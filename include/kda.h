@@ -315,6 +315,48 @@ KDA_API const char* kda_status_string(kda_status status);
  * CTA's work and leaves its outputs unspecified. */
 KDA_API kda_status kda_device_status(cudaStream_t stream);
 
+/* kda_chunk_bwd -- the backward pass of kda_chunk_fwd (per-key-channel gate,
+ * no input prologue): for the scalar
+ *     L = sum(d_out * out) + sum(d_final_state * final_state)
+ * it writes dL/dq, dL/dk, dL/dv, dL/dlog_alpha, dL/dbeta and (when
+ * d_initial_state is not NULL) dL/dinitial_state.  The gradient follows the
+ * chunkwise factorisation of the forward ("You Could Have Come Up with Kimi
+ * Delta Attention", daily.dev, Summary); the pages print no gradient, so it
+ * is the chain rule applied to that factorisation, checked against an fp64
+ * reverse-mode evaluation of the token recurrence.
+ *
+ * Arguments: shape, q, k, v, log_alpha, beta, initial_state (may be NULL =
+ * zeros), cu_seqlens (may be NULL) exactly as for kda_chunk_fwd (shape's
+ * chunk in {16, 32, 64}, dims in {32, 64, 128});
+ *   d_out          [tokens, H, d_v]    io dtype, the gradient of out
+ *   d_final_state  [n_seqs, H, d_k, d_v] fp32 or NULL (zero)
+ *   dq, dk         [tokens, H, d_k]    io dtype (written)
+ *   dv             [tokens, H, d_v]    io dtype (written)
+ *   d_log_alpha    [tokens, H, d_k]    fp32 (written)
+ *   d_beta         [tokens, H]         fp32 (written)
+ *   d_initial_state [n_seqs, H, d_k, d_v] fp32 (written) or NULL.
+ * All pointers are device pointers owned by the caller; io-dtype tensors and
+ * states 16-byte aligned, the other fp32 tensors and cu_seqlens 4-byte
+ * aligned (KDA_ERR_MISALIGNED otherwise).  No output may overlap an input or
+ * another output (KDA_ERR_INVALID_ARG).  All arithmetic is fp32; the call
+ * re-runs the forward's chunk stages and allocates its fp32 workspace from
+ * the stream-ordered pool (kda_chunk_bwd_plan reports its size).  Stream
+ * ordered: returns after queueing the kernels. */
+KDA_API kda_status kda_chunk_bwd(const kda_shape* shape, const void* q,
+                                 const void* k, const void* v,
+                                 const float* log_alpha, const float* beta,
+                                 const float* initial_state,
+                                 const int32_t* cu_seqlens, const void* d_out,
+                                 const float* d_final_state, void* dq, void* dk,
+                                 void* dv, float* d_log_alpha, float* d_beta,
+                                 float* d_initial_state, cudaStream_t stream);
+
+/* kda_chunk_bwd_plan -- kernels a kda_chunk_bwd call of this shape launches
+ * and the workspace bytes it allocates; no device work.  `packed` selects the
+ * cu_seqlens layout (then shape->n_seqs sequences). */
+KDA_API kda_status kda_chunk_bwd_plan(const kda_shape* shape, int packed,
+                                      int* kernels, size_t* workspace_bytes);
+
 /* kda_selftest_timeout -- diagnostic of the failure reporting, not part of
  * the forward pass: launches one CTA that waits on a device barrier nothing
  * completes, using the library's bounded wait with a limit of limit_us

@@ -150,3 +150,48 @@ def test_prologue_validation(lib):
     st = lib.kda_recurrent_step_ex(ctypes.byref(s), 0, ctypes.byref(pro), P(1),
                                    P(2), P(3), P(4), P(5), P(6), P(7), None)
     assert st == 1
+
+
+def bwd_call(lib, s, **kw):
+    """kda_chunk_bwd with fake, disjoint addresses; keyword overrides take a
+    slot index (an address) or None."""
+    names = ["q", "k", "v", "la", "b", "s0", "cu", "do", "dsT", "dq", "dk",
+             "dv", "dla", "db", "ds0"]
+    slots = {n: i + 1 for i, n in enumerate(names)}
+    slots["cu"] = None
+    slots.update(kw)
+    args = [_p(slots[n]) if isinstance(slots[n], int) else slots[n]
+            for n in names]
+    return lib.kda_chunk_bwd(ctypes.byref(s), *args, None)
+
+
+INVALID, UNSUPPORTED, MISALIGNED = 1, 2, 3
+
+
+def test_backward_validation(lib):
+    # unsupported sizes, missing tensors, misalignment and overlapping
+    # outputs are all rejected before any launch
+    assert bwd_call(lib, shape(dk=48)) == UNSUPPORTED
+    assert bwd_call(lib, shape(chunk=128)) == UNSUPPORTED
+    assert bwd_call(lib, shape(), dq=None) == INVALID
+    assert bwd_call(lib, shape(), la=None) == INVALID
+    assert bwd_call(lib, shape(), do=None) == INVALID
+    bad = ctypes.c_void_p(A + 0x1000_0000 + 8)
+    assert bwd_call(lib, shape(), dk=bad) == MISALIGNED
+    odd = ctypes.c_void_p(A + 3 * 0x1000_0000 + 2)
+    assert bwd_call(lib, shape(), db=odd) == MISALIGNED
+    # an output over an input, or over another output
+    assert bwd_call(lib, shape(), dq=1) == INVALID
+    assert bwd_call(lib, shape(), dv=10) == INVALID
+    # the packed layout needs B == 1 and n_seqs >= 1
+    assert bwd_call(lib, shape(B=2, n_seqs=2), cu=7) == INVALID
+
+
+def test_backward_plan(lib):
+    import torch
+    kern, ws = K.chunk_bwd_plan(2, 8192, 32, 128, 128, 64, torch.bfloat16)
+    # forward stages (1)-(3), the reverse chain, prep, 14 products, final
+    assert kern == 20 and ws > 0
+    kern_p, _ = K.chunk_bwd_plan(1, 300, 2, 64, 64, 32, torch.float32,
+                                 packed=True, n_seqs=3)
+    assert kern_p == 21
