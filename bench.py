@@ -405,6 +405,42 @@ def run_kda(args, world, rank, local):
     }
     del d3, out3, fin3
 
+    # ---- backward pass of the prefill workload: every input's gradient for
+    # a random output gradient (fp32 arithmetic, chunkwise) ----------------
+    gdo = torch.randn(d["v"].shape, generator=torch.Generator(device=dev)
+                      .manual_seed(77 + rank), device=dev).bfloat16()
+
+    def backward(_i):
+        K.chunk_bwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], None,
+                    None, gdo, None, chunk=C, want_initial_state=False)
+
+    for i in range(2):
+        backward(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    bw_steps = max(2, min(args.steps, 5))
+    bwms, bwper = timed(backward, bw_steps, stream)
+    barrier(world)
+    bwms = max_over_ranks(bwms, world)
+    th = B * T * H
+    # algorithmic bytes: q, k, v, log_alpha, beta and dO read once; dq, dk,
+    # dv, dlog_alpha, dbeta written once
+    bw_bytes = th * ((2 * dk + dv) * 2 + dk * 4 + 4 + dv * 2) + \
+        th * ((2 * dk + dv) * 2 + dk * 4 + 4)
+    bw_launch = statistics.mean(bwper)
+    kern_bw, ws_bw = K.chunk_bwd_plan(B, T, H, dk, dv, C, torch.bfloat16)
+    backward_line = {
+        "value": world * B * T / (bwms / bw_steps * 1e-3), "unit": "tokens/s",
+        "ms_per_step": bwms / bw_steps, "steps": bw_steps,
+        "workload": "kda_chunk_bwd on the prefill workload (dq, dk, dv, "
+                    "dlog_alpha, dbeta), fp32 arithmetic",
+        "hbm": {"achieved": bw_bytes / (bw_launch * 1e-3) / 1e9, "unit": "GB/s",
+                "frac": bw_bytes / (bw_launch * 1e-3) / 1e9 / pk["hbm_gbs"],
+                "algorithmic_bytes_per_launch": bw_bytes},
+        "kernels_per_call": kern_bw, "workspace_bytes": ws_bw,
+    }
+    del gdo
+
     # ---- end to end through the public API with host buffers ------------
     host = {n: d[n].cpu().pin_memory() for n in
             ("q", "k", "v", "log_alpha", "beta")}
@@ -495,6 +531,7 @@ def run_kda(args, world, rank, local):
             },
             "prefill_head_gate": head_gate,
             "prefill_packed_long": packed_long,
+            "backward": backward_line,
             "prefill_fused_prologue": fused_prologue,
             "e2e": {"value": e2e_value, "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -524,6 +561,16 @@ def run_only(args, dev, stream):
             K.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"],
                         None, None, chunk=cfg["chunk"], out=out,
                         final_state=fin)
+    elif args.only == "backward":
+        cfg = W.CONFIGS[PREFILL_CFG]
+        d = W.make(PREFILL_CFG, device=dev)
+        gdo = torch.randn(d["v"].shape, generator=torch.Generator(
+            device=dev).manual_seed(77), device=dev).bfloat16()
+
+        def fn(_i):
+            K.chunk_bwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"],
+                        None, None, gdo, None, chunk=cfg["chunk"],
+                        want_initial_state=False)
     else:
         dc = W.CONFIGS[DECODE_CFG]
         dd = W.make(DECODE_CFG, device=dev)
@@ -576,7 +623,8 @@ def main():
     ap.add_argument("--impl", choices=["kda", "reference"], default="kda")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--only", choices=["prefill", "decode"], default=None,
+    ap.add_argument("--only", choices=["prefill", "decode", "backward"],
+                    default=None,
                     help="profiling aid: run one workload's warm-up and timed "
                          "launches only (no e2e, no CPU baseline, no JSON line)")
     args = ap.parse_args()

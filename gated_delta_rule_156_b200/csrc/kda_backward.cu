@@ -32,6 +32,7 @@
 // combines them into the input gradients.  Channel gate, no input prologue.
 #include "kda_common.cuh"
 #include "kda_internal.h"
+#include "kda_inverse.cuh"
 
 namespace kda {
 
@@ -114,12 +115,14 @@ __global__ void __launch_bounds__(kThreads)
   if (!locate_chunk(cid, cu, chunk_off, n_seqs, T, C, &seq, &tok0, &L)) return;
   const int h = blockIdx.y, tid = threadIdx.x;
   extern __shared__ float sm[];
-  float* Kt = sm;              // [C][dk]
-  float* Kb = Kt + C * dk;     // [C][dk]
-  float* Qt = Kb + C * dk;     // [C][dk]
-  float* M = Qt + C * dk;      // [C][C]
-  float* Tm = M + C * C;       // [C][C]
-  float* bs = Tm + C * C;      // [C]
+  const int ldk = dk + 1;          // padded rows: no bank conflicts
+  float* Kt = sm;                  // [C][ldk]
+  float* Kb = Kt + C * ldk;        // [C][ldk]
+  float* Qt = Kb + C * ldk;        // [C][ldk]
+  float* A = Qt + C * ldk;         // [64][kFS] b M, zero-padded past C
+  float* Tm = A + 64 * ws::kFS;    // [64][kFS]
+  float* Msc = Tm + 64 * ws::kFS;  // [1024] scratch of the inverse
+  float* bs = Msc + 1024;          // [C]
 
   for (int r = tid; r < C; r += kThreads)
     bs[r] = r < L ? beta[(size_t)(tok0 + r) * H + h] : 0.f;
@@ -139,9 +142,9 @@ __global__ void __launch_bounds__(kThreads)
       w.qt[gi] = qt;
       w.bkt[gi] = bs[r] * kt;
     }
-    Kt[idx] = kt;
-    Kb[idx] = kb;
-    Qt[idx] = qt;
+    Kt[r * ldk + c] = kt;
+    Kb[r * ldk + c] = kb;
+    Qt[r * ldk + c] = qt;
   }
   for (int idx = tid; idx < L * dv; idx += kThreads) {
     const int r = idx / dv, j = idx % dv;
@@ -156,64 +159,65 @@ __global__ void __launch_bounds__(kThreads)
         __expf(g[((size_t)(tok0 + L - 1) * H + h) * dk + c]);
   __syncthreads();
   const size_t sqb = ((size_t)cid * H + h) * C * C;
+  for (int idx = tid; idx < 64 * ws::kFS; idx += kThreads) {
+    A[idx] = 0.f;
+    Tm[idx] = 0.f;
+  }
+  __syncthreads();
   for (int idx = tid; idx < C * C; idx += kThreads) {
     const int r = idx / C, i = idx % C;
     float m = 0.f, pv = 0.f;
     if (r < L && i <= r) {
-      for (int c = 0; c < dk; ++c) pv += Qt[r * dk + c] * Kb[i * dk + c];
+      for (int c = 0; c < dk; ++c) pv += Qt[r * ldk + c] * Kb[i * ldk + c];
       if (i < r)
-        for (int c = 0; c < dk; ++c) m += Kt[r * dk + c] * Kb[i * dk + c];
+        for (int c = 0; c < dk; ++c) m += Kt[r * ldk + c] * Kb[i * ldk + c];
     }
-    M[idx] = m;
+    A[r * ws::kFS + i] = bs[r] * m;
     w.mm[sqb + idx] = m;
     w.pp[sqb + idx] = i <= r ? pv : 0.f;
   }
   __syncthreads();
-  // Tm[r][j] = [r == j] - sum_{j<=i<r} b_r M[r][i] Tm[i][j]
-  for (int j = tid; j < C; j += kThreads) {
-    for (int r = 0; r < C; ++r) {
-      float t;
-      if (r < j) {
-        t = 0.f;
-      } else if (r == j) {
-        t = 1.f;
-      } else {
-        t = 0.f;
-        for (int i = j; i < r; ++i) t -= bs[r] * M[r * C + i] * Tm[i * C + j];
-      }
-      Tm[r * C + j] = t;
-    }
-  }
+  // Tm = (I + Diag(b) M)^-1 by recursive doubling (identity past C)
+  ws::invert_unit_lower(A, Tm, Msc, tid);
   __syncthreads();
-  for (int idx = tid; idx < C * C; idx += kThreads) w.tm[sqb + idx] = Tm[idx];
+  for (int idx = tid; idx < C * C; idx += kThreads)
+    w.tm[sqb + idx] = Tm[(idx / C) * ws::kFS + idx % C];
 }
 
 // The reverse chain over one sequence's chunks for one head and one 32-column
 // tile of d_v.  Per chunk (last first), with dS the gradient of the state
 // leaving it: partial d gam, G = Diag(gam) dS (stored), dDelta = Kb G + P^T dO
-// (stored), then dS <- G + Qt^T dO - W^T dDelta.
+// (stored), then dS <- G + Qt^T dO - W^T dDelta.  Each product gives every
+// thread a block of outputs (rows strided by 32, columns by 8) so that the
+// sums over the contraction index run as independent chains; the shared rows
+// are padded (33 floats for the 32-wide tiles, d_k + 1 for the token rows)
+// so both access directions are free of bank conflicts.
+constexpr int kTp = kDvTile + 1;
+
 __global__ void __launch_bounds__(kThreads)
     chain_kernel(BwdWs w, const float* __restrict__ d_final,
                  float* __restrict__ d_init, const int32_t* cu, int n_seqs,
                  int T, int H, int dk, int dv, int C) {
   const int seq = blockIdx.x, h = blockIdx.y, tile = blockIdx.z;
   const int j0 = tile * kDvTile, tid = threadIdx.x, ntile = dv / kDvTile;
+  const int dkp = dk + 1, NA = dk / 32;
+  const int g8 = tid >> 3, j8 = tid & 7;  // row group, column group
   extern __shared__ float sm[];
-  float* dS = sm;                    // [dk][32]
-  float* S0 = dS + dk * kDvTile;     // [dk][32]
-  float* Kb = S0 + dk * kDvTile;     // [C][dk]
-  float* Qt = Kb + C * dk;           // [C][dk]
-  float* Wc = Qt + C * dk;           // [C][dk]
-  float* P = Wc + C * dk;            // [C][C]
-  float* dO = P + C * C;             // [C][32]
-  float* De = dO + C * kDvTile;      // [C][32] Delta
-  float* dD = De + C * kDvTile;      // [C][32] dDelta
-  float* gC = dD + C * kDvTile;      // [dk]
+  float* dS = sm;                    // [dk][kTp]
+  float* S0 = dS + dk * kTp;         // [dk][kTp]
+  float* Kb = S0 + dk * kTp;         // [C][dkp]
+  float* Qt = Kb + C * dkp;          // [C][dkp]
+  float* Wc = Qt + C * dkp;          // [C][dkp]
+  float* P = Wc + C * dkp;           // [C][C]
+  float* dO = P + C * C;             // [C][kTp]
+  float* De = dO + C * kTp;          // [C][kTp] Delta
+  float* dD = De + C * kTp;          // [C][kTp] dDelta
+  float* gC = dD + C * kTp;          // [dk]
 
   const size_t sbase = ((size_t)seq * H + h) * dk * dv;
   for (int idx = tid; idx < dk * kDvTile; idx += kThreads) {
     const int c = idx / kDvTile, jj = idx % kDvTile;
-    dS[idx] = d_final ? d_final[sbase + (size_t)c * dv + j0 + jj] : 0.f;
+    dS[c * kTp + jj] = d_final ? d_final[sbase + (size_t)c * dv + j0 + jj] : 0.f;
   }
   int start, end;
   seq_range(cu, seq, T, &start, &end);
@@ -233,9 +237,9 @@ __global__ void __launch_bounds__(kThreads)
         qt = w.qt[gi];
         wv = w.fv.w[gi];
       }
-      Kb[idx] = kb;
-      Qt[idx] = qt;
-      Wc[idx] = wv;
+      Kb[r * dkp + c] = kb;
+      Qt[r * dkp + c] = qt;
+      Wc[r * dkp + c] = wv;
     }
     for (int idx = tid; idx < C * C; idx += kThreads)
       P[idx] = w.pp[((size_t)cid * H + h) * C * C + idx];
@@ -247,58 +251,150 @@ __global__ void __launch_bounds__(kThreads)
         o = w.do32[gi];
         de = w.fv.d[gi];
       }
-      dO[idx] = o;
-      De[idx] = de;
+      dO[r * kTp + jj] = o;
+      De[r * kTp + jj] = de;
     }
     for (int idx = tid; idx < dk * kDvTile; idx += kThreads) {
       const int c = idx / kDvTile, jj = idx % kDvTile;
-      S0[idx] = w.fv.s[cbase + (size_t)c * dv + j0 + jj];
+      S0[c * kTp + jj] = w.fv.s[cbase + (size_t)c * dv + j0 + jj];
     }
     for (int c = tid; c < dk; c += kThreads)
       gC[c] = w.gam[((size_t)cid * H + h) * dk + c];
     __syncthreads();
+
     // partial d gam over this tile: rowsum((S_0 + Kb^T Delta) * dS)
-    for (int c = tid; c < dk; c += kThreads) {
-      float acc = 0.f;
-      for (int jj = 0; jj < kDvTile; ++jj) {
-        float x = S0[c * kDvTile + jj];
-        for (int r = 0; r < L; ++r) x += Kb[r * dk + c] * De[r * kDvTile + jj];
-        acc += x * dS[c * kDvTile + jj];
+    {
+      float x[4][4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) x[a][b] = 0.f;
+      for (int r = 0; r < L; ++r) {
+        float de[4];
+#pragma unroll
+        for (int b = 0; b < 4; ++b) de[b] = De[r * kTp + j8 + 8 * b];
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          if (a < NA) {
+            const float kb = Kb[r * dkp + g8 + 32 * a];
+#pragma unroll
+            for (int b = 0; b < 4; ++b) x[a][b] += kb * de[b];
+          }
+        }
       }
-      w.dgam[(((size_t)cid * H + h) * ntile + tile) * dk + c] = acc;
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        if (a < NA) {
+          const int c = g8 + 32 * a;
+          float part = 0.f;
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const int jj = j8 + 8 * b;
+            part += (S0[c * kTp + jj] + x[a][b]) * dS[c * kTp + jj];
+          }
+          part += __shfl_xor_sync(0xffffffffu, part, 1);
+          part += __shfl_xor_sync(0xffffffffu, part, 2);
+          part += __shfl_xor_sync(0xffffffffu, part, 4);
+          if (j8 == 0)
+            w.dgam[(((size_t)cid * H + h) * ntile + tile) * dk + c] = part;
+        }
+      }
     }
     __syncthreads();
     for (int idx = tid; idx < dk * kDvTile; idx += kThreads) {
       const int c = idx / kDvTile, jj = idx % kDvTile;
-      const float gv = gC[c] * dS[idx];
-      dS[idx] = gv;
+      const float gv = gC[c] * dS[c * kTp + jj];
+      dS[c * kTp + jj] = gv;
       w.gst[cbase + (size_t)c * dv + j0 + jj] = gv;
     }
     __syncthreads();
-    for (int idx = tid; idx < C * kDvTile; idx += kThreads) {
-      const int r = idx / kDvTile, jj = idx % kDvTile;
-      float acc = 0.f;
-      if (r < L) {
-        for (int c = 0; c < dk; ++c) acc += Kb[r * dk + c] * dS[c * kDvTile + jj];
-        for (int i = r; i < L; ++i) acc += P[i * C + r] * dO[i * kDvTile + jj];
-        w.dd[((size_t)(tok0 + r) * H + h) * dv + j0 + jj] = acc;
+    // dDelta = Kb G + P^T dO  (rows g8, g8 + 32)
+    {
+      float acc[2][4];
+#pragma unroll
+      for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+      for (int c = 0; c < dk; ++c) {
+        float gv[4];
+#pragma unroll
+        for (int b = 0; b < 4; ++b) gv[b] = dS[c * kTp + j8 + 8 * b];
+#pragma unroll
+        for (int a = 0; a < 2; ++a) {
+          const int r = g8 + 32 * a;  // Kb rows past L are zero, past C absent
+          const float kb = r < C ? Kb[r * dkp + c] : 0.f;
+#pragma unroll
+          for (int b = 0; b < 4; ++b) acc[a][b] += kb * gv[b];
+        }
       }
-      dD[idx] = acc;
+      for (int i = 0; i < L; ++i) {
+        float o[4];
+#pragma unroll
+        for (int b = 0; b < 4; ++b) o[b] = dO[i * kTp + j8 + 8 * b];
+#pragma unroll
+        for (int a = 0; a < 2; ++a) {
+          const int r = g8 + 32 * a;
+          const float pv = r < C ? P[i * C + r] : 0.f;
+#pragma unroll
+          for (int b = 0; b < 4; ++b) acc[a][b] += pv * o[b];
+        }
+      }
+#pragma unroll
+      for (int a = 0; a < 2; ++a) {
+        const int r = g8 + 32 * a;
+        if (r < C) {
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const int jj = j8 + 8 * b;
+            const float v = r < L ? acc[a][b] : 0.f;
+            dD[r * kTp + jj] = v;
+            if (r < L) w.dd[((size_t)(tok0 + r) * H + h) * dv + j0 + jj] = v;
+          }
+        }
+      }
     }
     __syncthreads();
-    for (int idx = tid; idx < dk * kDvTile; idx += kThreads) {
-      const int c = idx / kDvTile, jj = idx % kDvTile;
-      float acc = dS[idx];
-      for (int r = 0; r < L; ++r)
-        acc += Qt[r * dk + c] * dO[r * kDvTile + jj] - Wc[r * dk + c] * dD[r * kDvTile + jj];
-      dS[idx] = acc;
+    // dS <- G + Qt^T dO - W^T dDelta
+    {
+      float acc[4][4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+      for (int r = 0; r < L; ++r) {
+        float o[4], dd[4];
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          o[b] = dO[r * kTp + j8 + 8 * b];
+          dd[b] = dD[r * kTp + j8 + 8 * b];
+        }
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          if (a < NA) {
+            const float qt = Qt[r * dkp + g8 + 32 * a];
+            const float wv = Wc[r * dkp + g8 + 32 * a];
+#pragma unroll
+            for (int b = 0; b < 4; ++b) acc[a][b] += qt * o[b] - wv * dd[b];
+          }
+        }
+      }
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        if (a < NA) {
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const int i = (g8 + 32 * a) * kTp + j8 + 8 * b;
+            dS[i] += acc[a][b];
+          }
+        }
+      }
     }
     __syncthreads();
   }
   if (d_init) {
     for (int idx = tid; idx < dk * kDvTile; idx += kThreads) {
       const int c = idx / kDvTile, jj = idx % kDvTile;
-      d_init[sbase + (size_t)c * dv + j0 + jj] = dS[idx];
+      d_init[sbase + (size_t)c * dv + j0 + jj] = dS[c * kTp + jj];
     }
   }
 }
@@ -352,17 +448,29 @@ __global__ void __launch_bounds__(kThreads)
   const int m = dim_of(op.m, L, dk, dv), n = dim_of(op.n, L, dk, dv);
   const int kk = dim_of(op.k, L, dk, dv);
   extern __shared__ float sm[];
-  float* As = sm;            // [m][kk]
-  float* Bs = sm + m * kk;   // [kk][n]
-  for (int idx = tid; idx < m * kk; idx += kThreads) {
-    const int i = idx / kk, t = idx % kk;
-    const int r = op.a.trans ? t : i, c = op.a.trans ? i : t;
-    As[idx] = op.a.p[elem_off(op.a, r, c, cid, h, tok0, H, C, dk)];
+  const int la = kk + 1, lb = n + 1;  // padded rows: conflict-free transposes
+  float* As = sm;            // [m][la]
+  float* Bs = sm + m * la;   // [kk][lb]
+  // Both operands are read in their memory order (consecutive threads read
+  // consecutive elements of a source row) and transposed, where asked, on
+  // the way into shared memory.
+  {
+    const int rows = op.a.trans ? kk : m, cols = op.a.trans ? m : kk;
+    for (int idx = tid; idx < rows * cols; idx += kThreads) {
+      const int r = idx / cols, c = idx % cols;
+      const float x = op.a.p[elem_off(op.a, r, c, cid, h, tok0, H, C, dk)];
+      if (op.a.trans) As[c * la + r] = x;
+      else As[r * la + c] = x;
+    }
   }
-  for (int idx = tid; idx < kk * n; idx += kThreads) {
-    const int t = idx / n, j = idx % n;
-    const int r = op.b.trans ? j : t, c = op.b.trans ? t : j;
-    Bs[idx] = op.b.p[elem_off(op.b, r, c, cid, h, tok0, H, C, dk)];
+  {
+    const int rows = op.b.trans ? n : kk, cols = op.b.trans ? kk : n;
+    for (int idx = tid; idx < rows * cols; idx += kThreads) {
+      const int r = idx / cols, c = idx % cols;
+      const float x = op.b.p[elem_off(op.b, r, c, cid, h, tok0, H, C, dk)];
+      if (op.b.trans) Bs[c * lb + r] = x;
+      else Bs[r * lb + c] = x;
+    }
   }
   __syncthreads();
   const int ti = tid >> 4, tj = tid & 15;
@@ -376,12 +484,12 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
     for (int a = 0; a < 8; ++a) {
       const int i = ti + 16 * a;
-      av[a] = i < m ? As[i * kk + t] : 0.f;
+      av[a] = i < m ? As[i * la + t] : 0.f;
     }
 #pragma unroll
     for (int b = 0; b < 8; ++b) {
       const int j = tj + 16 * b;
-      bv[b] = j < n ? Bs[t * n + j] : 0.f;
+      bv[b] = j < n ? Bs[t * lb + j] : 0.f;
     }
 #pragma unroll
     for (int a = 0; a < 8; ++a)
@@ -480,7 +588,7 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
   const dim3 grid((unsigned)(nch > 0 ? nch : 1), H);
 
   if (nch > 0) {
-    const size_t smp = 4 * (3 * (size_t)C * dk + 2 * (size_t)C * C + C);
+    const size_t smp = 4 * (3 * (size_t)C * (dk + 1) + 2 * 64 * ws::kFS + 1024 + C);
     if ((e = set_smem(prep_kernel<IO>, smp)) != cudaSuccess) return e;
     prep_kernel<IO><<<grid, kThreads, smp, stream>>>(
         static_cast<const IO*>(f.q), static_cast<const IO*>(f.k),
@@ -488,15 +596,15 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
         w.fv.g, w, cu, co, f.n_seqs, f.T, H, dk, dv, C);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  const size_t smc = 4 * (2 * (size_t)dk * kDvTile + 3 * (size_t)C * dk +
-                          (size_t)C * C + 3 * (size_t)C * kDvTile + dk);
+  const size_t smc = 4 * (2 * (size_t)dk * kTp + 3 * (size_t)C * (dk + 1) +
+                          (size_t)C * C + 3 * (size_t)C * kTp + dk);
   if ((e = set_smem(chain_kernel, smc)) != cudaSuccess) return e;
   chain_kernel<<<dim3(f.n_seqs, H, dv / kDvTile), kThreads, smc, stream>>>(
       w, a.d_final_state, a.d_initial_state, cu, f.n_seqs, f.T, H, dk, dv, C);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (nch == 0) return cudaSuccess;
 
-  if ((e = set_smem(bmm_kernel, 4 * 2 * 128 * 128)) != cudaSuccess) return e;
+  if ((e = set_smem(bmm_kernel, 4 * 2 * 128 * 129)) != cudaSuccess) return e;
   auto tok = [](float* p, int cols, int t = 0) { return MatRef{p, kTok, cols, t}; };
   auto sq = [&](float* p, int t = 0) { return MatRef{p, kSq, C, t}; };
   auto stt = [&](const float* p, int t = 0) {
@@ -507,7 +615,7 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
                  float alpha, int accumulate) {
     const BmmOp op{o, x, y, m, n, k, mask, alpha, accumulate};
     const size_t smem =
-        4 * (size_t)(dmax(m) * dmax(k) + dmax(k) * dmax(n));
+        4 * (size_t)(dmax(m) * (dmax(k) + 1) + dmax(k) * (dmax(n) + 1));
     bmm_kernel<<<grid, kThreads, smem, stream>>>(op, cu, co, f.n_seqs, f.T, H,
                                                  dk, dv, C);
     return cudaGetLastError();

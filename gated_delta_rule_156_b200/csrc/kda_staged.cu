@@ -20,6 +20,7 @@
 // the reference decomposition the fused tensor-core kernel is built from.
 #include "kda_common.cuh"
 #include "kda_internal.h"
+#include "kda_inverse.cuh"
 
 namespace kda {
 
@@ -161,12 +162,14 @@ __global__ void __launch_bounds__(kThreads)
     return;
   const int h = blockIdx.y, tid = threadIdx.x;
   extern __shared__ float sm[];
-  float* Kt = sm;              // [C][dk]
-  float* Kb = Kt + C * dk;     // [C][dk]
-  float* V = Kb + C * dk;      // [C][dv]
-  float* A = V + C * dv;       // [C][C]
-  float* Tm = A + C * C;       // [C][C]
-  float* bs = Tm + C * C;      // [C]
+  const int ldk = dk + 1;          // padded rows: no bank conflicts
+  float* Kt = sm;                  // [C][ldk]
+  float* Kb = Kt + C * ldk;        // [C][ldk]
+  float* V = Kb + C * ldk;         // [C][dv]
+  float* A = V + C * dv;           // [64][kFS], zero-padded past C
+  float* Tm = A + 64 * ws::kFS;    // [64][kFS], (I + A)^-1
+  float* Msc = Tm + 64 * ws::kFS;  // [1024] scratch of the inverse
+  float* bs = Msc + 1024;          // [C]
 
   for (int idx = tid; idx < C * dk; idx += kThreads) {
     const int r = idx / dk, c = idx % dk;
@@ -177,8 +180,8 @@ __global__ void __launch_bounds__(kThreads)
       kt = kv * __expf(gv);
       kb = kv * __expf(-gv);
     }
-    Kt[idx] = kt;
-    Kb[idx] = kb;
+    Kt[r * ldk + c] = kt;
+    Kb[r * ldk + c] = kb;
   }
   for (int idx = tid; idx < C * dv; idx += kThreads) {
     const int r = idx / dv, j = idx % dv;
@@ -188,45 +191,32 @@ __global__ void __launch_bounds__(kThreads)
     bs[r] = r < L ? beta[(size_t)(tok0 + r) * H + h] : 0.f;
   __syncthreads();
 
-  for (int idx = tid; idx < C * C; idx += kThreads) {
-    const int r = idx / C, i = idx % C;
+  for (int idx = tid; idx < 64 * ws::kFS; idx += kThreads) {
+    const int r = idx / ws::kFS, i = idx % ws::kFS;
     float acc = 0.f;
-    if (i < r) {
-      for (int c = 0; c < dk; ++c) acc += Kt[r * dk + c] * Kb[i * dk + c];
+    if (i < r && r < C) {
+      for (int c = 0; c < dk; ++c) acc += Kt[r * ldk + c] * Kb[i * ldk + c];
       acc *= bs[r];
     }
     A[idx] = acc;
+    Tm[idx] = 0.f;
   }
   __syncthreads();
-
-  // Forward substitution, one column of Tm per thread:
-  // Tm[r][j] = [r == j] - sum_{j<=i<r} A[r][i] Tm[i][j].
-  for (int j = tid; j < C; j += kThreads) {
-    for (int r = 0; r < C; ++r) {
-      float t;
-      if (r < j) {
-        t = 0.f;
-      } else if (r == j) {
-        t = 1.f;
-      } else {
-        t = 0.f;
-        for (int i = j; i < r; ++i) t -= A[r * C + i] * Tm[i * C + j];
-      }
-      Tm[r * C + j] = t;
-    }
-  }
+  // Tm = (I + A)^-1 by recursive doubling on 16 x 16 blocks (the rows and
+  // columns past C are zero in A, so they stay identity in Tm)
+  ws::invert_unit_lower(A, Tm, Msc, tid);
   __syncthreads();
 
   for (int idx = tid; idx < L * dk; idx += kThreads) {
     const int r = idx / dk, c = idx % dk;
     float acc = 0.f;
-    for (int i = 0; i <= r; ++i) acc += Tm[r * C + i] * bs[i] * Kt[i * dk + c];
+    for (int i = 0; i <= r; ++i) acc += Tm[r * ws::kFS + i] * bs[i] * Kt[i * ldk + c];
     w_out[((size_t)(tok0 + r) * H + h) * dk + c] = acc;
   }
   for (int idx = tid; idx < L * dv; idx += kThreads) {
     const int r = idx / dv, j = idx % dv;
     float acc = 0.f;
-    for (int i = 0; i <= r; ++i) acc += Tm[r * C + i] * bs[i] * V[i * dv + j];
+    for (int i = 0; i <= r; ++i) acc += Tm[r * ws::kFS + i] * bs[i] * V[i * dv + j];
     u_out[((size_t)(tok0 + r) * H + h) * dv + j] = acc;
   }
 }
@@ -325,9 +315,10 @@ __global__ void __launch_bounds__(kThreads)
   if (!locate_chunk(cid, cu, chunk_off, n_seqs, T, C, &seq, &tok0, &L)) return;
   const int h = blockIdx.y, j0 = blockIdx.z * kDvTile, tid = threadIdx.x;
   extern __shared__ float sm[];
-  float* Qt = sm;                 // [C][dk]
-  float* Kb = Qt + C * dk;        // [C][dk]
-  float* P = Kb + C * dk;         // [C][C]
+  const int ldk = dk + 1;         // padded rows: no bank conflicts
+  float* Qt = sm;                 // [C][ldk]
+  float* Kb = Qt + C * ldk;       // [C][ldk]
+  float* P = Kb + C * ldk;        // [C][C]
   float* S = P + C * C;           // [dk][kDvTile]
   float* D = S + dk * kDvTile;    // [C][kDvTile]
 
@@ -340,8 +331,8 @@ __global__ void __launch_bounds__(kThreads)
       qt = to_f32(q[gi]) * __expf(gv);
       kb = to_f32(k[gi]) * __expf(-gv);
     }
-    Qt[idx] = qt;
-    Kb[idx] = kb;
+    Qt[r * ldk + c] = qt;
+    Kb[r * ldk + c] = kb;
   }
   const size_t cbase = ((size_t)cid * H + h) * dk * dv;
   for (int idx = tid; idx < dk * kDvTile; idx += kThreads) {
@@ -357,14 +348,14 @@ __global__ void __launch_bounds__(kThreads)
     const int r = idx / C, i = idx % C;
     float acc = 0.f;
     if (i <= r)
-      for (int c = 0; c < dk; ++c) acc += Qt[r * dk + c] * Kb[i * dk + c];
+      for (int c = 0; c < dk; ++c) acc += Qt[r * ldk + c] * Kb[i * ldk + c];
     P[idx] = acc;
   }
   __syncthreads();
   for (int idx = tid; idx < L * kDvTile; idx += kThreads) {
     const int r = idx / kDvTile, jj = idx % kDvTile;
     float acc = 0.f;
-    for (int c = 0; c < dk; ++c) acc += Qt[r * dk + c] * S[c * kDvTile + jj];
+    for (int c = 0; c < dk; ++c) acc += Qt[r * ldk + c] * S[c * kDvTile + jj];
     for (int i = 0; i <= r; ++i) acc += P[r * C + i] * D[i * kDvTile + jj];
     out[((size_t)(tok0 + r) * H + h) * dv + j0 + jj] = from_f32<IO>(acc);
   }
@@ -399,7 +390,8 @@ cudaError_t run(const ChunkArgs& a, void* workspace, cudaStream_t stream,
                                           a.n_seqs, a.T, H, dk, C, a.gate);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
-    const size_t sm2 = 4 * ((size_t)2 * C * dk + (size_t)C * dv + 2 * C * C + C);
+    const size_t sm2 = 4 * ((size_t)2 * C * (dk + 1) + (size_t)C * dv +
+                            2 * 64 * ws::kFS + 1024 + C);
     if ((e = set_smem(intra_kernel<IO>, sm2)) != cudaSuccess) return e;
     intra_kernel<IO><<<grid, kThreads, sm2, stream>>>(
         k, v, a.beta, w.g, w.w, w.u, cu, w.chunk_off, a.n_seqs, a.T, H, dk, dv,
@@ -415,7 +407,7 @@ cudaError_t run(const ChunkArgs& a, void* workspace, cudaStream_t stream,
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
   if (nch > 0 && outputs) {
-    const size_t sm4 = 4 * (2 * (size_t)C * dk + (size_t)C * C +
+    const size_t sm4 = 4 * (2 * (size_t)C * (dk + 1) + (size_t)C * C +
                             (size_t)dk * kDvTile + (size_t)C * kDvTile);
     if ((e = set_smem(output_kernel<IO>, sm4)) != cudaSuccess) return e;
     output_kernel<IO><<<dim3((unsigned)nch, H, dv / kDvTile), kThreads, sm4,
