@@ -228,35 +228,67 @@ __global__ void __launch_bounds__(kThreads)
   for (int ch = nch - 1; ch >= 0; --ch) {
     const int cid = cid0 + ch, tok0 = start + ch * C, L = min(C, end - tok0);
     const size_t cbase = ((size_t)cid * H + h) * dk * dv;
-    for (int idx = tid; idx < C * dk; idx += kThreads) {
-      const int r = idx / dk, c = idx % dk;
-      float kb = 0.f, qt = 0.f, wv = 0.f;
-      if (r < L) {
-        const size_t gi = ((size_t)(tok0 + r) * H + h) * dk + c;
-        kb = w.kb[gi];
-        qt = w.qt[gi];
-        wv = w.fv.w[gi];
+    // staging loads batched eight deep so their latencies overlap
+    for (int base = 0; base < C * dk; base += 8 * kThreads) {
+      float kb[8], qt[8], wv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int idx = base + u * kThreads + tid;
+        const int r = idx / dk, c = idx % dk;
+        kb[u] = qt[u] = wv[u] = 0.f;
+        if (idx < C * dk && r < L) {
+          const size_t gi = ((size_t)(tok0 + r) * H + h) * dk + c;
+          kb[u] = w.kb[gi];
+          qt[u] = w.qt[gi];
+          wv[u] = w.fv.w[gi];
+        }
       }
-      Kb[r * dkp + c] = kb;
-      Qt[r * dkp + c] = qt;
-      Wc[r * dkp + c] = wv;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int idx = base + u * kThreads + tid;
+        if (idx < C * dk) {
+          const int r = idx / dk, c = idx % dk;
+          Kb[r * dkp + c] = kb[u];
+          Qt[r * dkp + c] = qt[u];
+          Wc[r * dkp + c] = wv[u];
+        }
+      }
     }
     for (int idx = tid; idx < C * C; idx += kThreads)
       P[idx] = w.pp[((size_t)cid * H + h) * C * C + idx];
-    for (int idx = tid; idx < C * kDvTile; idx += kThreads) {
-      const int r = idx / kDvTile, jj = idx % kDvTile;
-      float o = 0.f, de = 0.f;
-      if (r < L) {
-        const size_t gi = ((size_t)(tok0 + r) * H + h) * dv + j0 + jj;
-        o = w.do32[gi];
-        de = w.fv.d[gi];
+    {
+      float o[8], de[8], s0[16];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {  // C * 32 <= 8 * kThreads
+        const int idx = u * kThreads + tid;
+        const int r = idx / kDvTile, jj = idx % kDvTile;
+        o[u] = de[u] = 0.f;
+        if (idx < C * kDvTile && r < L) {
+          const size_t gi = ((size_t)(tok0 + r) * H + h) * dv + j0 + jj;
+          o[u] = w.do32[gi];
+          de[u] = w.fv.d[gi];
+        }
       }
-      dO[r * kTp + jj] = o;
-      De[r * kTp + jj] = de;
-    }
-    for (int idx = tid; idx < dk * kDvTile; idx += kThreads) {
-      const int c = idx / kDvTile, jj = idx % kDvTile;
-      S0[c * kTp + jj] = w.fv.s[cbase + (size_t)c * dv + j0 + jj];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {  // dk * 32 <= 16 * kThreads
+        const int idx = u * kThreads + tid;
+        const int c = idx / kDvTile, jj = idx % kDvTile;
+        s0[u] = idx < dk * kDvTile ? w.fv.s[cbase + (size_t)c * dv + j0 + jj] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int idx = u * kThreads + tid;
+        if (idx < C * kDvTile) {
+          const int r = idx / kDvTile, jj = idx % kDvTile;
+          dO[r * kTp + jj] = o[u];
+          De[r * kTp + jj] = de[u];
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int idx = u * kThreads + tid;
+        if (idx < dk * kDvTile) S0[(idx / kDvTile) * kTp + idx % kDvTile] = s0[u];
+      }
     }
     for (int c = tid; c < dk; c += kThreads)
       gC[c] = w.gam[((size_t)cid * H + h) * dk + c];

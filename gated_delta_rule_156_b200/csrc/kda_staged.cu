@@ -262,16 +262,30 @@ __global__ void __launch_bounds__(kThreads)
     for (int c = tid; c < dk; c += kThreads)
       gC[c] = g[((size_t)(tok0 + L - 1) * H + h) * dk + c];
     __syncthreads();
-    for (int idx = tid; idx < C * dk; idx += kThreads) {
-      const int r = idx / dk, c = idx % dk;
-      float wv = 0.f, kh = 0.f;
-      if (r < L) {
-        const size_t gi = ((size_t)(tok0 + r) * H + h) * dk + c;
-        wv = w[gi];
-        kh = to_f32(k[gi]) * __expf(gC[c] - g[gi]);
+    // staging loads batched eight deep so their latencies overlap
+    for (int base = 0; base < C * dk; base += 8 * kThreads) {
+      float wv[8], kv[8], gv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int idx = base + u * kThreads + tid;
+        const int r = idx / dk;
+        wv[u] = kv[u] = gv[u] = 0.f;
+        if (idx < C * dk && r < L) {
+          const size_t gi = ((size_t)(tok0 + r) * H + h) * dk + idx % dk;
+          wv[u] = w[gi];
+          kv[u] = to_f32(k[gi]);
+          gv[u] = g[gi];
+        }
       }
-      Wc[idx] = wv;
-      Kh[idx] = kh;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int idx = base + u * kThreads + tid;
+        if (idx < C * dk) {
+          const int r = idx / dk, c = idx % dk;
+          Wc[idx] = wv[u];
+          Kh[idx] = r < L ? kv[u] * __expf(gC[c] - gv[u]) : 0.f;
+        }
+      }
     }
     for (int idx = tid; idx < C * kDvTile; idx += kThreads) {
       const int r = idx / kDvTile, jj = idx % kDvTile;
