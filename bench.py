@@ -130,15 +130,18 @@ class Clocks:
                 "reasons": sorted(reasons), "samples": len(sms)}
 
 
-def dist_setup():
+def dist_setup(backend="nccl"):
+    """Join the process group torchrun describes in the environment (one rank
+    per GPU over NCCL; gloo for host-only use).  Returns (world, rank,
+    local_rank)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
+        kw = {"device_id": torch.device("cuda", local)} if backend == "nccl" else {}
         torch.distributed.init_process_group(
-            "nccl", timeout=datetime.timedelta(seconds=180),
-            device_id=torch.device("cuda", local))
+            backend, timeout=datetime.timedelta(seconds=180), **kw)
     return world, rank, local
 
 
@@ -147,10 +150,11 @@ def barrier(world):
         torch.distributed.barrier()
 
 
-def max_over_ranks(x, world):
+def max_over_ranks(x, world, device="cuda"):
+    """The largest of every rank's x (each rank's device time), on every rank."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
 
