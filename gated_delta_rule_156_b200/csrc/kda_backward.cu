@@ -452,10 +452,11 @@ struct MatRef {
 
 struct BmmOp {
   MatRef out, a, b;
-  int m, n, k;  // Dim codes
+  int m, n, k;     // Dim codes
   int mask;
   float alpha;
   int accumulate;
+  int md, nd, kd;  // the largest m, n, k can be (row widths of the staging)
 };
 
 __device__ __forceinline__ int dim_of(int code, int L, int dk, int dv) {
@@ -470,6 +471,11 @@ __device__ __forceinline__ size_t elem_off(const MatRef& x, int r, int c,
   return (((size_t)cid * H + h) * dk + r) * x.cols + c;
 }
 
+// op(A) is staged transposed (AT[t][i]) and op(B) as is (Bs[t][j]), both in
+// the order the source is laid out in memory, with rows padded to a multiple
+// of four floats; each thread then owns the 8 x 8 block of Out at rows
+// 8 ti .. 8 ti + 7 and columns 8 tj .. 8 tj + 7, and every step of the
+// contraction is four 16-byte shared loads for 64 FMAs.
 __global__ void __launch_bounds__(kThreads)
     bmm_kernel(BmmOp op, const int32_t* cu, const int32_t* chunk_off, int n_seqs,
                int T, int H, int dk, int dv, int C) {
@@ -479,20 +485,18 @@ __global__ void __launch_bounds__(kThreads)
   const int h = blockIdx.y, tid = threadIdx.x;
   const int m = dim_of(op.m, L, dk, dv), n = dim_of(op.n, L, dk, dv);
   const int kk = dim_of(op.k, L, dk, dv);
-  extern __shared__ float sm[];
-  const int la = kk + 1, lb = n + 1;  // padded rows: conflict-free transposes
-  float* As = sm;            // [m][la]
-  float* Bs = sm + m * la;   // [kk][lb]
-  // Both operands are read in their memory order (consecutive threads read
-  // consecutive elements of a source row) and transposed, where asked, on
-  // the way into shared memory.
+  const int la = op.md + 4, lb = op.nd + 4;
+  extern __shared__ __align__(16) float sm[];
+  float* AT = sm;                 // [kd][la]
+  float* Bs = sm + op.kd * la;    // [kd][lb]
   {
+    // op(A)(i, t) = A(i, t) or A(t, i); walk the source row by row
     const int rows = op.a.trans ? kk : m, cols = op.a.trans ? m : kk;
     for (int idx = tid; idx < rows * cols; idx += kThreads) {
       const int r = idx / cols, c = idx % cols;
       const float x = op.a.p[elem_off(op.a, r, c, cid, h, tok0, H, C, dk)];
-      if (op.a.trans) As[c * la + r] = x;
-      else As[r * la + c] = x;
+      if (op.a.trans) AT[r * la + c] = x;   // r = t, c = i
+      else AT[c * la + r] = x;              // r = i, c = t
     }
   }
   {
@@ -500,29 +504,27 @@ __global__ void __launch_bounds__(kThreads)
     for (int idx = tid; idx < rows * cols; idx += kThreads) {
       const int r = idx / cols, c = idx % cols;
       const float x = op.b.p[elem_off(op.b, r, c, cid, h, tok0, H, C, dk)];
-      if (op.b.trans) Bs[c * lb + r] = x;
-      else Bs[r * lb + c] = x;
+      if (op.b.trans) Bs[c * lb + r] = x;   // r = j, c = t
+      else Bs[r * lb + c] = x;              // r = t, c = j
     }
   }
   __syncthreads();
   const int ti = tid >> 4, tj = tid & 15;
+  if (8 * ti >= m || 8 * tj >= n) return;
   float acc[8][8];
 #pragma unroll
   for (int a = 0; a < 8; ++a)
 #pragma unroll
     for (int b = 0; b < 8; ++b) acc[a][b] = 0.f;
+  const float* ap = AT + 8 * ti;
+  const float* bp = Bs + 8 * tj;
   for (int t = 0; t < kk; ++t) {
-    float av[8], bv[8];
-#pragma unroll
-    for (int a = 0; a < 8; ++a) {
-      const int i = ti + 16 * a;
-      av[a] = i < m ? As[i * la + t] : 0.f;
-    }
-#pragma unroll
-    for (int b = 0; b < 8; ++b) {
-      const int j = tj + 16 * b;
-      bv[b] = j < n ? Bs[t * lb + j] : 0.f;
-    }
+    const float4 a0 = *reinterpret_cast<const float4*>(ap + t * la);
+    const float4 a1 = *reinterpret_cast<const float4*>(ap + t * la + 4);
+    const float4 b0 = *reinterpret_cast<const float4*>(bp + t * lb);
+    const float4 b1 = *reinterpret_cast<const float4*>(bp + t * lb + 4);
+    const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+    const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
     for (int a = 0; a < 8; ++a)
 #pragma unroll
@@ -530,11 +532,11 @@ __global__ void __launch_bounds__(kThreads)
   }
 #pragma unroll
   for (int a = 0; a < 8; ++a) {
-    const int i = ti + 16 * a;
+    const int i = 8 * ti + a;
     if (i >= m) continue;
 #pragma unroll
     for (int b = 0; b < 8; ++b) {
-      const int j = tj + 16 * b;
+      const int j = 8 * tj + b;
       if (j >= n) continue;
       float x = op.alpha * acc[a][b];
       if ((op.mask == kMaskLowerIncl && j > i) ||
@@ -636,7 +638,7 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (nch == 0) return cudaSuccess;
 
-  if ((e = set_smem(bmm_kernel, 4 * 2 * 128 * 129)) != cudaSuccess) return e;
+  if ((e = set_smem(bmm_kernel, 4 * 2 * 128 * 132)) != cudaSuccess) return e;
   auto tok = [](float* p, int cols, int t = 0) { return MatRef{p, kTok, cols, t}; };
   auto sq = [&](float* p, int t = 0) { return MatRef{p, kSq, C, t}; };
   auto stt = [&](const float* p, int t = 0) {
@@ -645,9 +647,10 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
   auto dmax = [&](int code) { return code == kDimL ? C : code == kDimDk ? dk : dv; };
   auto bmm = [&](MatRef o, MatRef x, MatRef y, int m, int n, int k, int mask,
                  float alpha, int accumulate) {
-    const BmmOp op{o, x, y, m, n, k, mask, alpha, accumulate};
+    const BmmOp op{o,     x,    y,          m,       n,       k,
+                   mask,  alpha, accumulate, dmax(m), dmax(n), dmax(k)};
     const size_t smem =
-        4 * (size_t)(dmax(m) * (dmax(k) + 1) + dmax(k) * (dmax(n) + 1));
+        4 * (size_t)(dmax(k) * (dmax(m) + 4) + dmax(k) * (dmax(n) + 4));
     bmm_kernel<<<grid, kThreads, smem, stream>>>(op, cu, co, f.n_seqs, f.T, H,
                                                  dk, dv, C);
     return cudaGetLastError();

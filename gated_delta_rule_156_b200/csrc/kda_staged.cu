@@ -234,17 +234,24 @@ __global__ void __launch_bounds__(kThreads)
                  int H, int dk, int dv, int C) {
   const int seq = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * kDvTile;
   const int tid = threadIdx.x;
+  // Shared rows padded (kTp = 33 floats for the 32-wide tiles, dk + 1 for the
+  // token rows) so the products below are free of bank conflicts; each thread
+  // owns a block of outputs (rows strided by 32, columns by 8) whose sums run
+  // as independent chains.
+  constexpr int kTp = kDvTile + 1;
+  const int dkp = dk + 1, NA = dk / 32;
+  const int g8 = tid >> 3, j8 = tid & 7;
   extern __shared__ float sm[];
-  float* S = sm;                  // [dk][kDvTile]
-  float* Wc = S + dk * kDvTile;   // [C][dk]
-  float* Kh = Wc + C * dk;        // [C][dk]
-  float* D = Kh + C * dk;         // [C][kDvTile]
-  float* gC = D + C * kDvTile;    // [dk]
+  float* S = sm;                  // [dk][kTp]
+  float* Wc = S + dk * kTp;       // [C][dkp]
+  float* Kh = Wc + C * dkp;       // [C][dkp]
+  float* D = Kh + C * dkp;        // [C][kTp]
+  float* gC = D + C * kTp;        // [dk]
 
   const size_t sbase = ((size_t)seq * H + h) * dk * dv;
   for (int idx = tid; idx < dk * kDvTile; idx += kThreads) {
     const int c = idx / kDvTile, jj = idx % kDvTile;
-    S[idx] = s_init ? s_init[sbase + (size_t)c * dv + j0 + jj] : 0.f;
+    S[c * kTp + jj] = s_init ? s_init[sbase + (size_t)c * dv + j0 + jj] : 0.f;
   }
   int start, end;
   seq_range(cu, seq, T, &start, &end);
@@ -257,7 +264,7 @@ __global__ void __launch_bounds__(kThreads)
     const size_t cbase = ((size_t)(cid0 + ch) * H + h) * dk * dv;
     for (int idx = tid; idx < dk * kDvTile; idx += kThreads) {
       const int c = idx / kDvTile, jj = idx % kDvTile;
-      s_chunks[cbase + (size_t)c * dv + j0 + jj] = S[idx];
+      s_chunks[cbase + (size_t)c * dv + j0 + jj] = S[c * kTp + jj];
     }
     for (int c = tid; c < dk; c += kThreads)
       gC[c] = g[((size_t)(tok0 + L - 1) * H + h) * dk + c];
@@ -282,37 +289,86 @@ __global__ void __launch_bounds__(kThreads)
         const int idx = base + u * kThreads + tid;
         if (idx < C * dk) {
           const int r = idx / dk, c = idx % dk;
-          Wc[idx] = wv[u];
-          Kh[idx] = r < L ? kv[u] * __expf(gC[c] - gv[u]) : 0.f;
+          Wc[r * dkp + c] = wv[u];
+          Kh[r * dkp + c] = r < L ? kv[u] * __expf(gC[c] - gv[u]) : 0.f;
         }
       }
     }
     for (int idx = tid; idx < C * kDvTile; idx += kThreads) {
       const int r = idx / kDvTile, jj = idx % kDvTile;
-      D[idx] = r < L ? u[((size_t)(tok0 + r) * H + h) * dv + j0 + jj] : 0.f;
+      D[r * kTp + jj] = r < L ? u[((size_t)(tok0 + r) * H + h) * dv + j0 + jj] : 0.f;
     }
     __syncthreads();
-    for (int idx = tid; idx < C * kDvTile; idx += kThreads) {
-      const int r = idx / kDvTile, jj = idx % kDvTile;
-      if (r < L) {
-        float acc = D[idx];
-        for (int c = 0; c < dk; ++c) acc -= Wc[r * dk + c] * S[c * kDvTile + jj];
-        D[idx] = acc;
-        u[((size_t)(tok0 + r) * H + h) * dv + j0 + jj] = acc;
+    {  // D = U - W S   (rows g8, g8 + 32; columns j8 + 8 b)
+      float acc[2][4];
+#pragma unroll
+      for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+      for (int c = 0; c < dk; ++c) {
+        float sv[4];
+#pragma unroll
+        for (int b = 0; b < 4; ++b) sv[b] = S[c * kTp + j8 + 8 * b];
+#pragma unroll
+        for (int a = 0; a < 2; ++a) {
+          const int r = g8 + 32 * a;
+          const float wv = r < C ? Wc[r * dkp + c] : 0.f;
+#pragma unroll
+          for (int b = 0; b < 4; ++b) acc[a][b] += wv * sv[b];
+        }
+      }
+#pragma unroll
+      for (int a = 0; a < 2; ++a) {
+        const int r = g8 + 32 * a;
+        if (r < L) {
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const int jj = j8 + 8 * b;
+            const float dvl = D[r * kTp + jj] - acc[a][b];
+            D[r * kTp + jj] = dvl;
+            u[((size_t)(tok0 + r) * H + h) * dv + j0 + jj] = dvl;
+          }
+        }
       }
     }
     __syncthreads();
-    for (int idx = tid; idx < dk * kDvTile; idx += kThreads) {
-      const int c = idx / kDvTile, jj = idx % kDvTile;
-      float acc = __expf(gC[c]) * S[idx];
-      for (int r = 0; r < L; ++r) acc += Kh[r * dk + c] * D[r * kDvTile + jj];
-      S[idx] = acc;
+    {  // S <- Diag(exp(g_C)) S + Kh^T D   (rows g8 + 32 a; columns j8 + 8 b)
+      float acc[4][4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+      for (int r = 0; r < L; ++r) {
+        float dvv[4];
+#pragma unroll
+        for (int b = 0; b < 4; ++b) dvv[b] = D[r * kTp + j8 + 8 * b];
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          if (a < NA) {
+            const float kh = Kh[r * dkp + g8 + 32 * a];
+#pragma unroll
+            for (int b = 0; b < 4; ++b) acc[a][b] += kh * dvv[b];
+          }
+        }
+      }
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        if (a < NA) {
+          const int c = g8 + 32 * a;
+          const float ga = __expf(gC[c]);
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const int i = c * kTp + j8 + 8 * b;
+            S[i] = ga * S[i] + acc[a][b];
+          }
+        }
+      }
     }
     __syncthreads();
   }
   for (int idx = tid; idx < dk * kDvTile; idx += kThreads) {
     const int c = idx / kDvTile, jj = idx % kDvTile;
-    s_final[sbase + (size_t)c * dv + j0 + jj] = S[idx];
+    s_final[sbase + (size_t)c * dv + j0 + jj] = S[c * kTp + jj];
   }
 }
 
@@ -412,8 +468,8 @@ cudaError_t run(const ChunkArgs& a, void* workspace, cudaStream_t stream,
         C);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  const size_t sm3 =
-      4 * ((size_t)dk * kDvTile + 2 * (size_t)C * dk + C * kDvTile + dk);
+  const size_t sm3 = 4 * ((size_t)dk * (kDvTile + 1) + 2 * (size_t)C * (dk + 1) +
+                          (size_t)C * (kDvTile + 1) + dk);
   if ((e = set_smem(state_kernel<IO>, sm3)) != cudaSuccess) return e;
   state_kernel<IO><<<dim3(a.n_seqs, H, dv / kDvTile), kThreads, sm3, stream>>>(
       k, w.g, w.w, w.u, w.s, a.initial_state, a.final_state, cu, w.chunk_off,
