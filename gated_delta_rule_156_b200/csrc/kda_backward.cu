@@ -39,7 +39,6 @@ namespace kda {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kDvTile = 32;
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -91,7 +90,7 @@ BwdWs carve_bwd(const BwdArgs& a, void* base, size_t* total) {
   w.tm = take(sq); w.mm = take(sq); w.pp = take(sq);
   w.gam = take(4 * nch * H * dk);
   w.gst = take(st);
-  w.dgam = take(4 * nch * H * (dv / kDvTile) * dk);
+  w.dgam = take(4 * nch * H * (dv / 32) * dk);
   w.dp = take(sq); w.dtm = take(sq); w.tmp = take(sq); w.da = take(sq);
   w.dqt = take(tdk); w.dkb = take(tdk); w.dw = take(tdk); w.dbk = take(tdk);
   w.y1 = take(tdk);
@@ -164,17 +163,45 @@ __global__ void __launch_bounds__(kThreads)
     Tm[idx] = 0.f;
   }
   __syncthreads();
-  for (int idx = tid; idx < C * C; idx += kThreads) {
-    const int r = idx / C, i = idx % C;
-    float m = 0.f, pv = 0.f;
-    if (r < L && i <= r) {
-      for (int c = 0; c < dk; ++c) pv += Qt[r * ldk + c] * Kb[i * ldk + c];
-      if (i < r)
-        for (int c = 0; c < dk; ++c) m += Kt[r * ldk + c] * Kb[i * ldk + c];
+  {
+    // M and P together: thread (ti, tj) owns rows ti + 16 a and columns
+    // tj + 16 b (a, b < C / 16), so the padded rows give conflict-free loads
+    const int ti = tid >> 4, tj = tid & 15, nr = C / 16;
+    float m[4][4], pv[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) m[a][b] = pv[a][b] = 0.f;
+#pragma unroll 2
+    for (int c = 0; c < dk; ++c) {
+      float kt[4], qt[4], kb[4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        const bool in = a < nr;
+        kt[a] = in ? Kt[(ti + 16 * a) * ldk + c] : 0.f;
+        qt[a] = in ? Qt[(ti + 16 * a) * ldk + c] : 0.f;
+        kb[a] = in ? Kb[(tj + 16 * a) * ldk + c] : 0.f;
+      }
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          m[a][b] += kt[a] * kb[b];
+          pv[a][b] += qt[a] * kb[b];
+        }
     }
-    A[r * ws::kFS + i] = bs[r] * m;
-    w.mm[sqb + idx] = m;
-    w.pp[sqb + idx] = i <= r ? pv : 0.f;
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        if (a < nr && b < nr) {
+          const int r = ti + 16 * a, i = tj + 16 * b;
+          const float mv = (r < L && i < r) ? m[a][b] : 0.f;
+          A[r * ws::kFS + i] = bs[r] * mv;
+          w.mm[sqb + r * C + i] = mv;
+          w.pp[sqb + r * C + i] = (r < L && i <= r) ? pv[a][b] : 0.f;
+        }
+      }
   }
   __syncthreads();
   // Tm = (I + Diag(b) M)^-1 by recursive doubling (identity past C)
@@ -184,40 +211,43 @@ __global__ void __launch_bounds__(kThreads)
     w.tm[sqb + idx] = Tm[(idx / C) * ws::kFS + idx % C];
 }
 
-// The reverse chain over one sequence's chunks for one head and one 32-column
-// tile of d_v.  Per chunk (last first), with dS the gradient of the state
-// leaving it: partial d gam, G = Diag(gam) dS (stored), dDelta = Kb G + P^T dO
-// (stored), then dS <- G + Qt^T dO - W^T dDelta.  Each product gives every
-// thread a block of outputs (rows strided by 32, columns by 8) so that the
-// sums over the contraction index run as independent chains; the shared rows
-// are padded (33 floats for the 32-wide tiles, d_k + 1 for the token rows)
-// so both access directions are free of bank conflicts.
-constexpr int kTp = kDvTile + 1;
+// The reverse chain over one sequence's chunks for one head and one TILE-wide
+// column tile of d_v (64, or 32 when d_v = 32, so that a d = 128 layer runs
+// one wave of CTAs).  Per chunk (last first), with dS the gradient of the
+// state leaving it: partial d gam, G = Diag(gam) dS (stored), dDelta = Kb G +
+// P^T dO (stored), then dS <- G + Qt^T dO - W^T dDelta.  Each product gives
+// every thread a block of outputs (rows strided by 32, columns by 8) so that
+// the sums over the contraction index run as independent chains; the shared
+// rows are padded (TILE + 1 floats for the tiles, d_k + 1 for the token rows)
+// so both access directions are free of bank conflicts.  The chunk-start
+// state enters only the d gam sum and is read there straight from memory.
+__host__ __device__ constexpr int chain_tile(int dv) { return dv >= 64 ? 64 : 32; }
 
+template <int TILE>
 __global__ void __launch_bounds__(kThreads)
     chain_kernel(BwdWs w, const float* __restrict__ d_final,
                  float* __restrict__ d_init, const int32_t* cu, int n_seqs,
                  int T, int H, int dk, int dv, int C) {
+  constexpr int TP = TILE + 1, NB = TILE / 8;
   const int seq = blockIdx.x, h = blockIdx.y, tile = blockIdx.z;
-  const int j0 = tile * kDvTile, tid = threadIdx.x, ntile = dv / kDvTile;
+  const int j0 = tile * TILE, tid = threadIdx.x, ntile = dv / TILE;
   const int dkp = dk + 1, NA = dk / 32;
   const int g8 = tid >> 3, j8 = tid & 7;  // row group, column group
   extern __shared__ float sm[];
-  float* dS = sm;                    // [dk][kTp]
-  float* S0 = dS + dk * kTp;         // [dk][kTp]
-  float* Kb = S0 + dk * kTp;         // [C][dkp]
+  float* dS = sm;                    // [dk][TP]
+  float* Kb = dS + dk * TP;          // [C][dkp]
   float* Qt = Kb + C * dkp;          // [C][dkp]
   float* Wc = Qt + C * dkp;          // [C][dkp]
   float* P = Wc + C * dkp;           // [C][C]
-  float* dO = P + C * C;             // [C][kTp]
-  float* De = dO + C * kTp;          // [C][kTp] Delta
-  float* dD = De + C * kTp;          // [C][kTp] dDelta
-  float* gC = dD + C * kTp;          // [dk]
+  float* dO = P + C * C;             // [C][TP]
+  float* De = dO + C * TP;           // [C][TP] Delta
+  float* dD = De + C * TP;           // [C][TP] dDelta
+  float* gC = dD + C * TP;           // [dk]
 
   const size_t sbase = ((size_t)seq * H + h) * dk * dv;
-  for (int idx = tid; idx < dk * kDvTile; idx += kThreads) {
-    const int c = idx / kDvTile, jj = idx % kDvTile;
-    dS[c * kTp + jj] = d_final ? d_final[sbase + (size_t)c * dv + j0 + jj] : 0.f;
+  for (int idx = tid; idx < dk * TILE; idx += kThreads) {
+    const int c = idx / TILE, jj = idx % TILE;
+    dS[c * TP + jj] = d_final ? d_final[sbase + (size_t)c * dv + j0 + jj] : 0.f;
   }
   int start, end;
   seq_range(cu, seq, T, &start, &end);
@@ -257,37 +287,27 @@ __global__ void __launch_bounds__(kThreads)
     for (int idx = tid; idx < C * C; idx += kThreads)
       P[idx] = w.pp[((size_t)cid * H + h) * C * C + idx];
     {
-      float o[8], de[8], s0[16];
+      constexpr int NU = 64 * TILE / kThreads;  // C * TILE <= NU * kThreads
+      float o[NU], de[NU];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {  // C * 32 <= 8 * kThreads
+      for (int u = 0; u < NU; ++u) {
         const int idx = u * kThreads + tid;
-        const int r = idx / kDvTile, jj = idx % kDvTile;
+        const int r = idx / TILE, jj = idx % TILE;
         o[u] = de[u] = 0.f;
-        if (idx < C * kDvTile && r < L) {
+        if (idx < C * TILE && r < L) {
           const size_t gi = ((size_t)(tok0 + r) * H + h) * dv + j0 + jj;
           o[u] = w.do32[gi];
           de[u] = w.fv.d[gi];
         }
       }
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {  // dk * 32 <= 16 * kThreads
+      for (int u = 0; u < NU; ++u) {
         const int idx = u * kThreads + tid;
-        const int c = idx / kDvTile, jj = idx % kDvTile;
-        s0[u] = idx < dk * kDvTile ? w.fv.s[cbase + (size_t)c * dv + j0 + jj] : 0.f;
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int idx = u * kThreads + tid;
-        if (idx < C * kDvTile) {
-          const int r = idx / kDvTile, jj = idx % kDvTile;
-          dO[r * kTp + jj] = o[u];
-          De[r * kTp + jj] = de[u];
+        if (idx < C * TILE) {
+          const int r = idx / TILE, jj = idx % TILE;
+          dO[r * TP + jj] = o[u];
+          De[r * TP + jj] = de[u];
         }
-      }
-#pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int idx = u * kThreads + tid;
-        if (idx < dk * kDvTile) S0[(idx / kDvTile) * kTp + idx % kDvTile] = s0[u];
       }
     }
     for (int c = tid; c < dk; c += kThreads)
@@ -296,21 +316,26 @@ __global__ void __launch_bounds__(kThreads)
 
     // partial d gam over this tile: rowsum((S_0 + Kb^T Delta) * dS)
     {
-      float x[4][4];
+      float s0[4][NB], x[4][NB];
 #pragma unroll
       for (int a = 0; a < 4; ++a)
 #pragma unroll
-        for (int b = 0; b < 4; ++b) x[a][b] = 0.f;
+        for (int b = 0; b < NB; ++b) {
+          x[a][b] = 0.f;
+          s0[a][b] = a < NA ? w.fv.s[cbase + (size_t)(g8 + 32 * a) * dv + j0 +
+                                     j8 + 8 * b]
+                            : 0.f;
+        }
       for (int r = 0; r < L; ++r) {
-        float de[4];
+        float de[NB];
 #pragma unroll
-        for (int b = 0; b < 4; ++b) de[b] = De[r * kTp + j8 + 8 * b];
+        for (int b = 0; b < NB; ++b) de[b] = De[r * TP + j8 + 8 * b];
 #pragma unroll
         for (int a = 0; a < 4; ++a) {
           if (a < NA) {
             const float kb = Kb[r * dkp + g8 + 32 * a];
 #pragma unroll
-            for (int b = 0; b < 4; ++b) x[a][b] += kb * de[b];
+            for (int b = 0; b < NB; ++b) x[a][b] += kb * de[b];
           }
         }
       }
@@ -320,10 +345,8 @@ __global__ void __launch_bounds__(kThreads)
           const int c = g8 + 32 * a;
           float part = 0.f;
 #pragma unroll
-          for (int b = 0; b < 4; ++b) {
-            const int jj = j8 + 8 * b;
-            part += (S0[c * kTp + jj] + x[a][b]) * dS[c * kTp + jj];
-          }
+          for (int b = 0; b < NB; ++b)
+            part += (s0[a][b] + x[a][b]) * dS[c * TP + j8 + 8 * b];
           part += __shfl_xor_sync(0xffffffffu, part, 1);
           part += __shfl_xor_sync(0xffffffffu, part, 2);
           part += __shfl_xor_sync(0xffffffffu, part, 4);
@@ -333,42 +356,42 @@ __global__ void __launch_bounds__(kThreads)
       }
     }
     __syncthreads();
-    for (int idx = tid; idx < dk * kDvTile; idx += kThreads) {
-      const int c = idx / kDvTile, jj = idx % kDvTile;
-      const float gv = gC[c] * dS[c * kTp + jj];
-      dS[c * kTp + jj] = gv;
+    for (int idx = tid; idx < dk * TILE; idx += kThreads) {
+      const int c = idx / TILE, jj = idx % TILE;
+      const float gv = gC[c] * dS[c * TP + jj];
+      dS[c * TP + jj] = gv;
       w.gst[cbase + (size_t)c * dv + j0 + jj] = gv;
     }
     __syncthreads();
     // dDelta = Kb G + P^T dO  (rows g8, g8 + 32)
     {
-      float acc[2][4];
+      float acc[2][NB];
 #pragma unroll
       for (int a = 0; a < 2; ++a)
 #pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+        for (int b = 0; b < NB; ++b) acc[a][b] = 0.f;
       for (int c = 0; c < dk; ++c) {
-        float gv[4];
+        float gv[NB];
 #pragma unroll
-        for (int b = 0; b < 4; ++b) gv[b] = dS[c * kTp + j8 + 8 * b];
+        for (int b = 0; b < NB; ++b) gv[b] = dS[c * TP + j8 + 8 * b];
 #pragma unroll
         for (int a = 0; a < 2; ++a) {
           const int r = g8 + 32 * a;  // Kb rows past L are zero, past C absent
           const float kb = r < C ? Kb[r * dkp + c] : 0.f;
 #pragma unroll
-          for (int b = 0; b < 4; ++b) acc[a][b] += kb * gv[b];
+          for (int b = 0; b < NB; ++b) acc[a][b] += kb * gv[b];
         }
       }
       for (int i = 0; i < L; ++i) {
-        float o[4];
+        float o[NB];
 #pragma unroll
-        for (int b = 0; b < 4; ++b) o[b] = dO[i * kTp + j8 + 8 * b];
+        for (int b = 0; b < NB; ++b) o[b] = dO[i * TP + j8 + 8 * b];
 #pragma unroll
         for (int a = 0; a < 2; ++a) {
           const int r = g8 + 32 * a;
           const float pv = r < C ? P[i * C + r] : 0.f;
 #pragma unroll
-          for (int b = 0; b < 4; ++b) acc[a][b] += pv * o[b];
+          for (int b = 0; b < NB; ++b) acc[a][b] += pv * o[b];
         }
       }
 #pragma unroll
@@ -376,10 +399,10 @@ __global__ void __launch_bounds__(kThreads)
         const int r = g8 + 32 * a;
         if (r < C) {
 #pragma unroll
-          for (int b = 0; b < 4; ++b) {
+          for (int b = 0; b < NB; ++b) {
             const int jj = j8 + 8 * b;
             const float v = r < L ? acc[a][b] : 0.f;
-            dD[r * kTp + jj] = v;
+            dD[r * TP + jj] = v;
             if (r < L) w.dd[((size_t)(tok0 + r) * H + h) * dv + j0 + jj] = v;
           }
         }
@@ -388,17 +411,17 @@ __global__ void __launch_bounds__(kThreads)
     __syncthreads();
     // dS <- G + Qt^T dO - W^T dDelta
     {
-      float acc[4][4];
+      float acc[4][NB];
 #pragma unroll
       for (int a = 0; a < 4; ++a)
 #pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+        for (int b = 0; b < NB; ++b) acc[a][b] = 0.f;
       for (int r = 0; r < L; ++r) {
-        float o[4], dd[4];
+        float o[NB], dd[NB];
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          o[b] = dO[r * kTp + j8 + 8 * b];
-          dd[b] = dD[r * kTp + j8 + 8 * b];
+        for (int b = 0; b < NB; ++b) {
+          o[b] = dO[r * TP + j8 + 8 * b];
+          dd[b] = dD[r * TP + j8 + 8 * b];
         }
 #pragma unroll
         for (int a = 0; a < 4; ++a) {
@@ -406,7 +429,7 @@ __global__ void __launch_bounds__(kThreads)
             const float qt = Qt[r * dkp + g8 + 32 * a];
             const float wv = Wc[r * dkp + g8 + 32 * a];
 #pragma unroll
-            for (int b = 0; b < 4; ++b) acc[a][b] += qt * o[b] - wv * dd[b];
+            for (int b = 0; b < NB; ++b) acc[a][b] += qt * o[b] - wv * dd[b];
           }
         }
       }
@@ -414,8 +437,8 @@ __global__ void __launch_bounds__(kThreads)
       for (int a = 0; a < 4; ++a) {
         if (a < NA) {
 #pragma unroll
-          for (int b = 0; b < 4; ++b) {
-            const int i = (g8 + 32 * a) * kTp + j8 + 8 * b;
+          for (int b = 0; b < NB; ++b) {
+            const int i = (g8 + 32 * a) * TP + j8 + 8 * b;
             dS[i] += acc[a][b];
           }
         }
@@ -424,21 +447,20 @@ __global__ void __launch_bounds__(kThreads)
     __syncthreads();
   }
   if (d_init) {
-    for (int idx = tid; idx < dk * kDvTile; idx += kThreads) {
-      const int c = idx / kDvTile, jj = idx % kDvTile;
-      d_init[sbase + (size_t)c * dv + j0 + jj] = dS[c * kTp + jj];
+    for (int idx = tid; idx < dk * TILE; idx += kThreads) {
+      const int c = idx / TILE, jj = idx % TILE;
+      d_init[sbase + (size_t)c * dv + j0 + jj] = dS[c * TP + jj];
     }
   }
 }
 
 // ---------------------------------------------------------------------------
-// Batched small products over every (chunk, head): Out (m x n) = alpha op(A)
-// op(B) (+ Out), with op = transpose or not and an optional lower-triangular
-// mask on Out.  An operand is one of: token rows [tokens, H, cols] (rows are
-// the chunk's tokens, zero past its length), a per-chunk square [chunks, H,
-// C, C], or a per-chunk state [chunks, H, dk, dv].  Both operands are staged
-// whole in shared memory (m, n, k <= 128); each thread owns an up to 8 x 8
-// block of Out strided by 16 in both directions.
+// Batched small products over every (chunk, head): Out (m x n) = alpha sum of
+// op(A) op(B) over one or two terms (+ Out), with op = transpose or not and an
+// optional lower-triangular mask on Out.  An operand is one of: token rows
+// [tokens, H, cols] (rows are the chunk's tokens), a per-chunk square
+// [chunks, H, C, C], or a per-chunk state [chunks, H, dk, dv].  Every m is the
+// chunk length L; n and the contraction length are L, d_k or d_v.
 enum MatKind { kTok = 0, kSq = 1, kState = 2 };
 enum Dim { kDimL = 0, kDimDk = 1, kDimDv = 2 };
 enum Mask { kMaskNone = 0, kMaskLowerIncl = 1, kMaskStrictLower = 2 };
@@ -450,32 +472,144 @@ struct MatRef {
   int trans;
 };
 
+struct BmmTerm {
+  MatRef a, b;
+  int kd;      // the padded contraction length (C, d_k or d_v)
+};
+
 struct BmmOp {
-  MatRef out, a, b;
-  int m, n, k;     // Dim codes
+  MatRef out;
+  BmmTerm term[2];
+  int nterms;
+  int n;       // Dim code of n (m is always L)
+  int nd;      // padded n
   int mask;
   float alpha;
   int accumulate;
-  int md, nd, kd;  // the largest m, n, k can be (row widths of the staging)
 };
 
 __device__ __forceinline__ int dim_of(int code, int L, int dk, int dv) {
   return code == kDimL ? L : code == kDimDk ? dk : dv;
 }
 
-__device__ __forceinline__ size_t elem_off(const MatRef& x, int r, int c,
-                                           int cid, int h, int tok0, int H,
-                                           int C, int dk) {
-  if (x.kind == kTok) return ((size_t)(tok0 + r) * H + h) * x.cols + c;
-  if (x.kind == kSq) return (((size_t)cid * H + h) * C + r) * C + c;
-  return (((size_t)cid * H + h) * dk + r) * x.cols + c;
+// One operand source as a row-major matrix: row 0 and the row stride, plus
+// the valid extent (token rows and square entries past L read as zero).
+struct Src {
+  float* p;
+  size_t stride;
+  int vrows, vcols;
+};
+
+__device__ __forceinline__ Src src_of(const MatRef& x, int cid, int h,
+                                      int tok0, int L, int H, int C, int dk) {
+  if (x.kind == kTok)
+    return Src{x.p + ((size_t)tok0 * H + h) * x.cols, (size_t)H * x.cols, L,
+               x.cols};
+  if (x.kind == kSq)
+    return Src{x.p + ((size_t)cid * H + h) * C * C, (size_t)C, L, L};
+  return Src{x.p + ((size_t)cid * H + h) * dk * x.cols, (size_t)x.cols, dk,
+             x.cols};
 }
 
-// op(A) is staged transposed (AT[t][i]) and op(B) as is (Bs[t][j]), both in
-// the order the source is laid out in memory, with rows padded to a multiple
-// of four floats; each thread then owns the 8 x 8 block of Out at rows
-// 8 ti .. 8 ti + 7 and columns 8 tj .. 8 tj + 7, and every step of the
-// contraction is four 16-byte shared loads for 64 FMAs.
+// Four consecutive entries (r, c .. c + 3), c a multiple of four.  A square's
+// last valid vector can be partial; its tail lies inside the C x C
+// allocation and is zeroed.
+__device__ __forceinline__ float4 ld_src4(const Src& s, int r, int c) {
+  float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (r < s.vrows && c < s.vcols) {
+    v = *reinterpret_cast<const float4*>(s.p + (size_t)r * s.stride + c);
+    if (c + 1 >= s.vcols) v.y = 0.f;
+    if (c + 2 >= s.vcols) v.z = 0.f;
+    if (c + 3 >= s.vcols) v.w = 0.f;
+  }
+  return v;
+}
+
+// dst[r * ld + c] = src(r, c) over the padded rows x cols (multiples of 16):
+// consecutive threads take consecutive 16-byte vectors of a row.
+__device__ __forceinline__ void stage_direct(const Src& s, int rows, int cols,
+                                             float* dst, int ld, int tid) {
+  const int cv = cols >> 2, units = rows * cv;
+  for (int base = 0; base < units; base += 4 * kThreads) {
+    float4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int idx = base + u * kThreads + tid;
+      v[u] = idx < units ? ld_src4(s, idx / cv, (idx % cv) * 4)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int idx = base + u * kThreads + tid;
+      if (idx < units)
+        *reinterpret_cast<float4*>(dst + (idx / cv) * ld + (idx % cv) * 4) = v[u];
+    }
+  }
+}
+
+// dst[c * ld + r] = src(r, c): consecutive threads take consecutive rows, each
+// reading 32 contiguous bytes, so the scattered shared stores of a warp fall
+// in distinct banks.
+__device__ __forceinline__ void stage_transposed(const Src& s, int rows,
+                                                 int cols, float* dst, int ld,
+                                                 int tid) {
+  const int units = rows * (cols >> 3);
+  for (int base = 0; base < units; base += 2 * kThreads) {
+    float4 v[2][2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int idx = base + u * kThreads + tid;
+      const int r = idx % rows, c = (idx / rows) * 8;
+      const bool in = idx < units;
+      v[u][0] = in ? ld_src4(s, r, c) : make_float4(0.f, 0.f, 0.f, 0.f);
+      v[u][1] = in ? ld_src4(s, r, c + 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int idx = base + u * kThreads + tid;
+      if (idx < units) {
+        const int r = idx % rows, c = (idx / rows) * 8;
+        float* d = dst + c * ld + r;
+        d[0 * ld] = v[u][0].x;
+        d[1 * ld] = v[u][0].y;
+        d[2 * ld] = v[u][0].z;
+        d[3 * ld] = v[u][0].w;
+        d[4 * ld] = v[u][1].x;
+        d[5 * ld] = v[u][1].y;
+        d[6 * ld] = v[u][1].z;
+        d[7 * ld] = v[u][1].w;
+      }
+    }
+  }
+}
+
+template <int N>
+__device__ __forceinline__ void lds_vec(const float* p, float* v) {
+  if constexpr (N >= 4) {
+#pragma unroll
+    for (int q = 0; q < N / 4; ++q) {
+      const float4 x = *reinterpret_cast<const float4*>(p + 4 * q);
+      v[4 * q] = x.x;
+      v[4 * q + 1] = x.y;
+      v[4 * q + 2] = x.z;
+      v[4 * q + 3] = x.w;
+    }
+  } else if constexpr (N == 2) {
+    const float2 x = *reinterpret_cast<const float2*>(p);
+    v[0] = x.x;
+    v[1] = x.y;
+  } else {
+    v[0] = p[0];
+  }
+}
+
+// op(A) is staged transposed (AT[t][i]) and op(B) as is (Bs[t][j]), zero past
+// the valid extent, rows padded by four floats.  The 256 threads form a
+// 16 x 16 grid over the padded C x nd output; thread (ti, tj) owns the RM x RN
+// block at rows RM ti.., columns RN tj.. (RM = C / 16, RN = nd / 16), so every
+// thread works and each step of the contraction is RM / 4 + RN / 4 vector
+// shared loads for RM x RN FMAs.
+template <int RM, int RN>
 __global__ void __launch_bounds__(kThreads)
     bmm_kernel(BmmOp op, const int32_t* cu, const int32_t* chunk_off, int n_seqs,
                int T, int H, int dk, int dv, int C) {
@@ -483,67 +617,76 @@ __global__ void __launch_bounds__(kThreads)
   int seq, tok0, L;
   if (!locate_chunk(cid, cu, chunk_off, n_seqs, T, C, &seq, &tok0, &L)) return;
   const int h = blockIdx.y, tid = threadIdx.x;
-  const int m = dim_of(op.m, L, dk, dv), n = dim_of(op.n, L, dk, dv);
-  const int kk = dim_of(op.k, L, dk, dv);
-  const int la = op.md + 4, lb = op.nd + 4;
+  const int md = 16 * RM, nd = 16 * RN;
+  const int la = md + 4, lb = nd + 4;
   extern __shared__ __align__(16) float sm[];
-  float* AT = sm;                 // [kd][la]
-  float* Bs = sm + op.kd * la;    // [kd][lb]
-  {
-    // op(A)(i, t) = A(i, t) or A(t, i); walk the source row by row
-    const int rows = op.a.trans ? kk : m, cols = op.a.trans ? m : kk;
-    for (int idx = tid; idx < rows * cols; idx += kThreads) {
-      const int r = idx / cols, c = idx % cols;
-      const float x = op.a.p[elem_off(op.a, r, c, cid, h, tok0, H, C, dk)];
-      if (op.a.trans) AT[r * la + c] = x;   // r = t, c = i
-      else AT[c * la + r] = x;              // r = i, c = t
-    }
-  }
-  {
-    const int rows = op.b.trans ? n : kk, cols = op.b.trans ? kk : n;
-    for (int idx = tid; idx < rows * cols; idx += kThreads) {
-      const int r = idx / cols, c = idx % cols;
-      const float x = op.b.p[elem_off(op.b, r, c, cid, h, tok0, H, C, dk)];
-      if (op.b.trans) Bs[c * lb + r] = x;   // r = j, c = t
-      else Bs[r * lb + c] = x;              // r = t, c = j
-    }
-  }
-  __syncthreads();
   const int ti = tid >> 4, tj = tid & 15;
-  if (8 * ti >= m || 8 * tj >= n) return;
-  float acc[8][8];
+  float acc[RM][RN];
 #pragma unroll
-  for (int a = 0; a < 8; ++a)
+  for (int a = 0; a < RM; ++a)
 #pragma unroll
-    for (int b = 0; b < 8; ++b) acc[a][b] = 0.f;
-  const float* ap = AT + 8 * ti;
-  const float* bp = Bs + 8 * tj;
-  for (int t = 0; t < kk; ++t) {
-    const float4 a0 = *reinterpret_cast<const float4*>(ap + t * la);
-    const float4 a1 = *reinterpret_cast<const float4*>(ap + t * la + 4);
-    const float4 b0 = *reinterpret_cast<const float4*>(bp + t * lb);
-    const float4 b1 = *reinterpret_cast<const float4*>(bp + t * lb + 4);
-    const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-    const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+    for (int b = 0; b < RN; ++b) acc[a][b] = 0.f;
+  for (int term = 0; term < op.nterms; ++term) {
+    const BmmTerm tm = term == 0 ? op.term[0] : op.term[1];
+    const int kd = tm.kd;
+    float* AT = sm;            // [kd][la]
+    float* Bs = sm + kd * la;  // [kd][lb]
+    if (term > 0) __syncthreads();  // the previous term's reads are done
+    const Src sa = src_of(tm.a, cid, h, tok0, L, H, C, dk);
+    const Src sb = src_of(tm.b, cid, h, tok0, L, H, C, dk);
+    if (tm.a.trans) stage_direct(sa, kd, md, AT, la, tid);  // source A[t][i]
+    else stage_transposed(sa, md, kd, AT, la, tid);         // source A[i][t]
+    if (tm.b.trans) stage_transposed(sb, nd, kd, Bs, lb, tid);  // B[j][t]
+    else stage_direct(sb, kd, nd, Bs, lb, tid);                 // B[t][j]
+    __syncthreads();
+    const float* ap = AT + RM * ti;
+    const float* bp = Bs + RN * tj;
+#pragma unroll 4
+    for (int t = 0; t < kd; ++t) {
+      float av[RM], bv[RN];
+      lds_vec<RM>(ap + t * la, av);
+      lds_vec<RN>(bp + t * lb, bv);
 #pragma unroll
-    for (int a = 0; a < 8; ++a)
+      for (int a = 0; a < RM; ++a)
 #pragma unroll
-      for (int b = 0; b < 8; ++b) acc[a][b] += av[a] * bv[b];
+        for (int b = 0; b < RN; ++b) acc[a][b] += av[a] * bv[b];
+    }
   }
+  const int m = L, n = dim_of(op.n, L, dk, dv);
+  const Src so = src_of(op.out, cid, h, tok0, L, H, C, dk);
+  const int j0 = RN * tj;
 #pragma unroll
-  for (int a = 0; a < 8; ++a) {
-    const int i = 8 * ti + a;
-    if (i >= m) continue;
+  for (int a = 0; a < RM; ++a) {
+    const int i = RM * ti + a;
+    if (i >= m || j0 >= n) continue;
+    float x[RN];
 #pragma unroll
-    for (int b = 0; b < 8; ++b) {
-      const int j = 8 * tj + b;
-      if (j >= n) continue;
-      float x = op.alpha * acc[a][b];
+    for (int b = 0; b < RN; ++b) {
+      const int j = j0 + b;
+      x[b] = op.alpha * acc[a][b];
       if ((op.mask == kMaskLowerIncl && j > i) ||
           (op.mask == kMaskStrictLower && j >= i))
-        x = 0.f;
-      float* o = op.out.p + elem_off(op.out, i, j, cid, h, tok0, H, C, dk);
-      *o = op.accumulate ? *o + x : x;
+        x[b] = 0.f;
+    }
+    float* o = so.p + (size_t)i * so.stride + j0;
+    if (RN >= 4 && j0 + RN <= n) {
+#pragma unroll
+      for (int q = 0; q < RN / 4; ++q) {
+        float4* o4 = reinterpret_cast<float4*>(o + 4 * q);
+        float4 y = make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
+        if (op.accumulate) {
+          const float4 z = *o4;
+          y.x += z.x;
+          y.y += z.y;
+          y.z += z.z;
+          y.w += z.w;
+        }
+        *o4 = y;
+      }
+    } else {
+#pragma unroll
+      for (int b = 0; b < RN; ++b)
+        if (j0 + b < n) o[b] = op.accumulate ? o[b] + x[b] : x[b];
     }
   }
 }
@@ -560,7 +703,7 @@ __global__ void __launch_bounds__(kThreads)
   const int cid = blockIdx.x;
   int seq, tok0, L;
   if (!locate_chunk(cid, cu, chunk_off, n_seqs, T, C, &seq, &tok0, &L)) return;
-  const int h = blockIdx.y, tid = threadIdx.x, ntile = dv / kDvTile;
+  const int h = blockIdx.y, tid = threadIdx.x, ntile = dv / chain_tile(dv);
   extern __shared__ float sm[];
   float* dg = sm;  // [C][dk]
   for (int idx = tid; idx < L * dk; idx += kThreads) {
@@ -609,6 +752,46 @@ cudaError_t set_smem(K kernel, size_t bytes) {
                               (int)bytes);
 }
 
+// Launch one batched product with the thread blocking its padded shape asks
+// for: RM = C / 16 rows and RN = nd / 16 columns per thread.
+template <int RM, int RN>
+cudaError_t launch_bmm_t(const BmmOp& op, size_t smem, dim3 grid,
+                         cudaStream_t stream, const int32_t* cu,
+                         const int32_t* co, int n_seqs, int T, int H, int dk,
+                         int dv, int C) {
+  cudaError_t e = set_smem(bmm_kernel<RM, RN>, smem);
+  if (e != cudaSuccess) return e;
+  bmm_kernel<RM, RN><<<grid, kThreads, smem, stream>>>(op, cu, co, n_seqs, T, H,
+                                                       dk, dv, C);
+  return cudaGetLastError();
+}
+
+template <int RM>
+cudaError_t launch_bmm_n(const BmmOp& op, int C, size_t smem, dim3 grid,
+                         cudaStream_t stream, const int32_t* cu,
+                         const int32_t* co, int n_seqs, int T, int H, int dk,
+                         int dv) {
+  switch (op.nd) {
+    case 16: return launch_bmm_t<RM, 1>(op, smem, grid, stream, cu, co, n_seqs, T, H, dk, dv, C);
+    case 32: return launch_bmm_t<RM, 2>(op, smem, grid, stream, cu, co, n_seqs, T, H, dk, dv, C);
+    case 64: return launch_bmm_t<RM, 4>(op, smem, grid, stream, cu, co, n_seqs, T, H, dk, dv, C);
+    case 128: return launch_bmm_t<RM, 8>(op, smem, grid, stream, cu, co, n_seqs, T, H, dk, dv, C);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_bmm(const BmmOp& op, int C, size_t smem, dim3 grid,
+                       cudaStream_t stream, const int32_t* cu,
+                       const int32_t* co, int n_seqs, int T, int H, int dk,
+                       int dv) {
+  switch (C) {
+    case 16: return launch_bmm_n<1>(op, C, smem, grid, stream, cu, co, n_seqs, T, H, dk, dv);
+    case 32: return launch_bmm_n<2>(op, C, smem, grid, stream, cu, co, n_seqs, T, H, dk, dv);
+    case 64: return launch_bmm_n<4>(op, C, smem, grid, stream, cu, co, n_seqs, T, H, dk, dv);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 template <typename IO>
 cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
   BwdWs w = carve_bwd(a, workspace, nullptr);
@@ -630,71 +813,90 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
         w.fv.g, w, cu, co, f.n_seqs, f.T, H, dk, dv, C);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  const size_t smc = 4 * (2 * (size_t)dk * kTp + 3 * (size_t)C * (dk + 1) +
-                          (size_t)C * C + 3 * (size_t)C * kTp + dk);
-  if ((e = set_smem(chain_kernel, smc)) != cudaSuccess) return e;
-  chain_kernel<<<dim3(f.n_seqs, H, dv / kDvTile), kThreads, smc, stream>>>(
-      w, a.d_final_state, a.d_initial_state, cu, f.n_seqs, f.T, H, dk, dv, C);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  {
+    const int tile = chain_tile(dv), tp = tile + 1;
+    const size_t smc = 4 * ((size_t)dk * tp + 3 * (size_t)C * (dk + 1) +
+                            (size_t)C * C + 3 * (size_t)C * tp + dk);
+    const dim3 cgrid(f.n_seqs, H, dv / tile);
+    if (tile == 64) {
+      if ((e = set_smem(chain_kernel<64>, smc)) != cudaSuccess) return e;
+      chain_kernel<64><<<cgrid, kThreads, smc, stream>>>(
+          w, a.d_final_state, a.d_initial_state, cu, f.n_seqs, f.T, H, dk, dv, C);
+    } else {
+      if ((e = set_smem(chain_kernel<32>, smc)) != cudaSuccess) return e;
+      chain_kernel<32><<<cgrid, kThreads, smc, stream>>>(
+          w, a.d_final_state, a.d_initial_state, cu, f.n_seqs, f.T, H, dk, dv, C);
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   if (nch == 0) return cudaSuccess;
 
-  if ((e = set_smem(bmm_kernel, 4 * 2 * 128 * 132)) != cudaSuccess) return e;
   auto tok = [](float* p, int cols, int t = 0) { return MatRef{p, kTok, cols, t}; };
   auto sq = [&](float* p, int t = 0) { return MatRef{p, kSq, C, t}; };
   auto stt = [&](const float* p, int t = 0) {
     return MatRef{const_cast<float*>(p), kState, dv, t};
   };
   auto dmax = [&](int code) { return code == kDimL ? C : code == kDimDk ? dk : dv; };
-  auto bmm = [&](MatRef o, MatRef x, MatRef y, int m, int n, int k, int mask,
+  auto term = [&](MatRef x, MatRef y, int k) { return BmmTerm{x, y, dmax(k)}; };
+  auto bmm2 = [&](MatRef o, BmmTerm t0, BmmTerm t1, int nterms, int n,
+                  int mask, float alpha, int accumulate) {
+    BmmOp op{};
+    op.out = o;
+    op.term[0] = t0;
+    op.term[1] = t1;
+    op.nterms = nterms;
+    op.n = n;
+    op.nd = dmax(n);
+    op.mask = mask;
+    op.alpha = alpha;
+    op.accumulate = accumulate;
+    const int kd = max(t0.kd, nterms > 1 ? t1.kd : 0);
+    const size_t smem = 4 * (size_t)kd * ((C + 4) + (op.nd + 4));
+    return launch_bmm(op, C, smem, grid, stream, cu, co, f.n_seqs, f.T, H, dk,
+                      dv);
+  };
+  auto bmm = [&](MatRef o, MatRef x, MatRef y, int n, int k, int mask,
                  float alpha, int accumulate) {
-    const BmmOp op{o,     x,    y,          m,       n,       k,
-                   mask,  alpha, accumulate, dmax(m), dmax(n), dmax(k)};
-    const size_t smem =
-        4 * (size_t)(dmax(k) * (dmax(m) + 4) + dmax(k) * (dmax(n) + 4));
-    bmm_kernel<<<grid, kThreads, smem, stream>>>(op, cu, co, f.n_seqs, f.T, H,
-                                                 dk, dv, C);
-    return cudaGetLastError();
+    const BmmTerm t = term(x, y, k);
+    return bmm2(o, t, t, 1, n, mask, alpha, accumulate);
   };
   float* De = const_cast<float*>(w.fv.d);  // Delta
   const float* S0 = w.fv.s;
 #define KDA_BMM(...) \
-  if ((e = bmm(__VA_ARGS__)) != cudaSuccess) return e;
+  if ((e = __VA_ARGS__) != cudaSuccess) return e;
   // dP = lower_incl(dO Delta^T)
-  KDA_BMM(sq(w.dp), tok(w.do32, dv), tok(De, dv, 1), kDimL, kDimL, kDimDv,
-          kMaskLowerIncl, 1.f, 0)
+  KDA_BMM(bmm(sq(w.dp), tok(w.do32, dv), tok(De, dv, 1), kDimL, kDimDv,
+              kMaskLowerIncl, 1.f, 0))
   // dQt = dO S_0^T + dP Kb
-  KDA_BMM(tok(w.dqt, dk), tok(w.do32, dv), stt(S0, 1), kDimL, kDimDk, kDimDv,
-          kMaskNone, 1.f, 0)
-  KDA_BMM(tok(w.dqt, dk), sq(w.dp), tok(w.kb, dk), kDimL, kDimDk, kDimL,
-          kMaskNone, 1.f, 1)
+  KDA_BMM(bmm2(tok(w.dqt, dk), term(tok(w.do32, dv), stt(S0, 1), kDimDv),
+               term(sq(w.dp), tok(w.kb, dk), kDimL), 2, kDimDk, kMaskNone, 1.f,
+               0))
   // dKb = Delta G^T + dP^T Qt  (+ dA^T b Kt below)
-  KDA_BMM(tok(w.dkb, dk), tok(De, dv), stt(w.gst, 1), kDimL, kDimDk, kDimDv,
-          kMaskNone, 1.f, 0)
-  KDA_BMM(tok(w.dkb, dk), sq(w.dp, 1), tok(w.qt, dk), kDimL, kDimDk, kDimL,
-          kMaskNone, 1.f, 1)
+  KDA_BMM(bmm2(tok(w.dkb, dk), term(tok(De, dv), stt(w.gst, 1), kDimDv),
+               term(sq(w.dp, 1), tok(w.qt, dk), kDimL), 2, kDimDk, kMaskNone,
+               1.f, 0))
   // dW = -dDelta S_0^T
-  KDA_BMM(tok(w.dw, dk), tok(w.dd, dv), stt(S0, 1), kDimL, kDimDk, kDimDv,
-          kMaskNone, -1.f, 0)
+  KDA_BMM(bmm(tok(w.dw, dk), tok(w.dd, dv), stt(S0, 1), kDimDk, kDimDv,
+              kMaskNone, -1.f, 0))
   // dTm = dW (b Kt)^T + dDelta (b V)^T
-  KDA_BMM(sq(w.dtm), tok(w.dw, dk), tok(w.bkt, dk, 1), kDimL, kDimL, kDimDk,
-          kMaskNone, 1.f, 0)
-  KDA_BMM(sq(w.dtm), tok(w.dd, dv), tok(w.bv, dv, 1), kDimL, kDimL, kDimDv,
-          kMaskNone, 1.f, 1)
+  KDA_BMM(bmm2(sq(w.dtm), term(tok(w.dw, dk), tok(w.bkt, dk, 1), kDimDk),
+               term(tok(w.dd, dv), tok(w.bv, dv, 1), kDimDv), 2, kDimL,
+               kMaskNone, 1.f, 0))
   // Tm^T dW, Tm^T dDelta, Tm^T dTm
-  KDA_BMM(tok(w.dbk, dk), sq(w.tm, 1), tok(w.dw, dk), kDimL, kDimDk, kDimL,
-          kMaskNone, 1.f, 0)
-  KDA_BMM(tok(w.dbv, dv), sq(w.tm, 1), tok(w.dd, dv), kDimL, kDimDv, kDimL,
-          kMaskNone, 1.f, 0)
-  KDA_BMM(sq(w.tmp), sq(w.tm, 1), sq(w.dtm), kDimL, kDimL, kDimL, kMaskNone,
-          1.f, 0)
+  KDA_BMM(bmm(tok(w.dbk, dk), sq(w.tm, 1), tok(w.dw, dk), kDimDk, kDimL,
+              kMaskNone, 1.f, 0))
+  KDA_BMM(bmm(tok(w.dbv, dv), sq(w.tm, 1), tok(w.dd, dv), kDimDv, kDimL,
+              kMaskNone, 1.f, 0))
+  KDA_BMM(bmm(sq(w.tmp), sq(w.tm, 1), sq(w.dtm), kDimL, kDimL, kMaskNone, 1.f,
+              0))
   // dA = strictly_lower(-(Tm^T dTm) Tm^T)
-  KDA_BMM(sq(w.da), sq(w.tmp), sq(w.tm, 1), kDimL, kDimL, kDimL,
-          kMaskStrictLower, -1.f, 0)
+  KDA_BMM(bmm(sq(w.da), sq(w.tmp), sq(w.tm, 1), kDimL, kDimL, kMaskStrictLower,
+              -1.f, 0))
   // dA Kb, and dKb += dA^T (b Kt)
-  KDA_BMM(tok(w.y1, dk), sq(w.da), tok(w.kb, dk), kDimL, kDimDk, kDimL,
-          kMaskNone, 1.f, 0)
-  KDA_BMM(tok(w.dkb, dk), sq(w.da, 1), tok(w.bkt, dk), kDimL, kDimDk, kDimL,
-          kMaskNone, 1.f, 1)
+  KDA_BMM(bmm(tok(w.y1, dk), sq(w.da), tok(w.kb, dk), kDimDk, kDimL, kMaskNone,
+              1.f, 0))
+  KDA_BMM(bmm(tok(w.dkb, dk), sq(w.da, 1), tok(w.bkt, dk), kDimDk, kDimL,
+              kMaskNone, 1.f, 1))
 #undef KDA_BMM
   const size_t smf = 4 * (size_t)C * dk;
   if ((e = set_smem(final_kernel<IO>, smf)) != cudaSuccess) return e;
@@ -705,7 +907,7 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-constexpr int kBmmOps = 14;
+constexpr int kBmmOps = 11;
 
 }  // namespace
 

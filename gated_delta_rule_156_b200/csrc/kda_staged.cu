@@ -192,32 +192,91 @@ __global__ void __launch_bounds__(kThreads)
   __syncthreads();
 
   for (int idx = tid; idx < 64 * ws::kFS; idx += kThreads) {
-    const int r = idx / ws::kFS, i = idx % ws::kFS;
-    float acc = 0.f;
-    if (i < r && r < C) {
-      for (int c = 0; c < dk; ++c) acc += Kt[r * ldk + c] * Kb[i * ldk + c];
-      acc *= bs[r];
-    }
-    A[idx] = acc;
+    A[idx] = 0.f;
     Tm[idx] = 0.f;
+  }
+  __syncthreads();
+  // Thread (ti, tj) owns rows ti + 16 a and columns tj + 16 b of each
+  // product: with the padded rows every shared load is conflict-free or a
+  // broadcast, and a step of the contraction feeds a block of FMAs.
+  const int ti = tid >> 4, tj = tid & 15, nr = C / 16;
+  {
+    float m[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) m[a][b] = 0.f;
+#pragma unroll 2
+    for (int c = 0; c < dk; ++c) {
+      float kt[4], kb[4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        kt[a] = a < nr ? Kt[(ti + 16 * a) * ldk + c] : 0.f;
+        kb[a] = a < nr ? Kb[(tj + 16 * a) * ldk + c] : 0.f;
+      }
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) m[a][b] += kt[a] * kb[b];
+    }
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const int r = ti + 16 * a, i = tj + 16 * b;
+        if (a < nr && b < nr && i < r) A[r * ws::kFS + i] = m[a][b] * bs[r];
+      }
   }
   __syncthreads();
   // Tm = (I + A)^-1 by recursive doubling on 16 x 16 blocks (the rows and
   // columns past C are zero in A, so they stay identity in Tm)
   ws::invert_unit_lower(A, Tm, Msc, tid);
   __syncthreads();
-
-  for (int idx = tid; idx < L * dk; idx += kThreads) {
-    const int r = idx / dk, c = idx % dk;
-    float acc = 0.f;
-    for (int i = 0; i <= r; ++i) acc += Tm[r * ws::kFS + i] * bs[i] * Kt[i * ldk + c];
-    w_out[((size_t)(tok0 + r) * H + h) * dk + c] = acc;
+  // Tm Diag(b), in place (Tm is lower triangular, zero above the diagonal)
+  for (int idx = tid; idx < C * C; idx += kThreads) {
+    const int r = idx / C, i = idx % C;
+    Tm[r * ws::kFS + i] *= bs[i];
   }
-  for (int idx = tid; idx < L * dv; idx += kThreads) {
-    const int r = idx / dv, j = idx % dv;
-    float acc = 0.f;
-    for (int i = 0; i <= r; ++i) acc += Tm[r * ws::kFS + i] * bs[i] * V[i * dv + j];
-    u_out[((size_t)(tok0 + r) * H + h) * dv + j] = acc;
+  __syncthreads();
+  // W = (Tm Diag(b)) Kt and U = (Tm Diag(b)) V over i = 0 .. C - 1 (the
+  // terms above the diagonal are exact zeros)
+  {
+    const int nw = dk / 16, nu = dv / 16;
+    float aw[4][8], au[4][8];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 8; ++b) aw[a][b] = au[a][b] = 0.f;
+    for (int i = 0; i < C; ++i) {
+      float t[4], kt[8], vv[8];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) t[a] = a < nr ? Tm[(ti + 16 * a) * ws::kFS + i] : 0.f;
+#pragma unroll
+      for (int b = 0; b < 8; ++b) {
+        kt[b] = b < nw ? Kt[i * ldk + tj + 16 * b] : 0.f;
+        vv[b] = b < nu ? V[i * dv + tj + 16 * b] : 0.f;
+      }
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+          aw[a][b] += t[a] * kt[b];
+          au[a][b] += t[a] * vv[b];
+        }
+    }
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const int r = ti + 16 * a;
+      if (a < nr && r < L) {
+        const size_t rw = ((size_t)(tok0 + r) * H + h) * dk;
+        const size_t ru = ((size_t)(tok0 + r) * H + h) * dv;
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+          if (b < nw) w_out[rw + tj + 16 * b] = aw[a][b];
+          if (b < nu) u_out[ru + tj + 16 * b] = au[a][b];
+        }
+      }
+    }
   }
 }
 
