@@ -51,10 +51,12 @@ struct BwdWs {
   float *tm, *mm, *pp;            // [chunks, H, C, C]
   float *gam;                     // [chunks, H, dk]
   float *gst;                     // G = Diag(gam) dS_C, [chunks, H, dk, dv]
-  float *dgam;                    // [chunks, H, dv / 32, dk] partial sums
+  float *dgam;                    // [chunks, H, dv / 32, dk] partials of gam * d gam
   float *dp, *dtm, *tmp, *da;     // [chunks, H, C, C]
   float *dqt, *dkb, *dw, *dbk, *y1;  // [tokens, H, dk]
   float *dbv;                     // [tokens, H, dv]
+  float *qdo;                     // Qt^T dO, [chunks, H, dk, dv]
+  float *pdo;                     // P^T dO, [tokens, H, dv]
 };
 
 ChunkArgs forward_args(const BwdArgs& a, float* fin) {
@@ -95,19 +97,23 @@ BwdWs carve_bwd(const BwdArgs& a, void* base, size_t* total) {
   w.dqt = take(tdk); w.dkb = take(tdk); w.dw = take(tdk); w.dbk = take(tdk);
   w.y1 = take(tdk);
   w.dbv = take(tdv);
+  w.qdo = take(st);
+  w.pdo = take(tdv);
   if (total) *total = off;
   return w;
 }
 
 // Per (chunk, head): Kt, Kb, Qt, b Kt and fp32 copies of V, b V, dO; gam;
-// M = Kt Kb^T (strictly lower), P = lower_incl(Qt Kb^T) and
-// Tm = (I + Diag(b) M)^-1 by forward substitution (one column per thread).
+// M = Kt Kb^T (strictly lower), P = lower_incl(Qt Kb^T), Tm = (I + Diag(b)
+// M)^-1 by recursive doubling, and the forward's W = Tm Diag(b) Kt and U =
+// Tm Diag(b) V for the state pass.
 template <typename IO>
 __global__ void __launch_bounds__(kThreads)
     prep_kernel(const IO* __restrict__ q, const IO* __restrict__ k,
                 const IO* __restrict__ v, const float* __restrict__ beta,
                 const IO* __restrict__ dout, const float* __restrict__ g,
-                BwdWs w, const int32_t* cu, const int32_t* chunk_off, int n_seqs,
+                BwdWs w, float* __restrict__ w_out, float* __restrict__ u_out,
+                const int32_t* cu, const int32_t* chunk_off, int n_seqs,
                 int T, int H, int dk, int dv, int C) {
   const int cid = blockIdx.x;
   int seq, tok0, L;
@@ -117,14 +123,19 @@ __global__ void __launch_bounds__(kThreads)
   const int ldk = dk + 1;          // padded rows: no bank conflicts
   float* Kt = sm;                  // [C][ldk]
   float* Kb = Kt + C * ldk;        // [C][ldk]
-  float* Qt = Kb + C * ldk;        // [C][ldk]
-  float* A = Qt + C * ldk;         // [64][kFS] b M, zero-padded past C
+  float* Qt = Kb + C * ldk;        // [C][ldk]; V [C][dv] once P is formed
+  float* V = Qt;
+  float* A = Qt + C * max(ldk, dv);  // [64][kFS] b M, zero-padded past C
   float* Tm = A + 64 * ws::kFS;    // [64][kFS]
   float* Msc = Tm + 64 * ws::kFS;  // [1024] scratch of the inverse
   float* bs = Msc + 1024;          // [C]
 
   for (int r = tid; r < C; r += kThreads)
     bs[r] = r < L ? beta[(size_t)(tok0 + r) * H + h] : 0.f;
+  for (int idx = tid; idx < 64 * ws::kFS; idx += kThreads) {
+    A[idx] = 0.f;
+    Tm[idx] = 0.f;
+  }
   __syncthreads();
   for (int idx = tid; idx < C * dk; idx += kThreads) {
     const int r = idx / dk, c = idx % dk;
@@ -145,28 +156,31 @@ __global__ void __launch_bounds__(kThreads)
     Kb[r * ldk + c] = kb;
     Qt[r * ldk + c] = qt;
   }
-  for (int idx = tid; idx < L * dv; idx += kThreads) {
-    const int r = idx / dv, j = idx % dv;
-    const size_t gi = ((size_t)(tok0 + r) * H + h) * dv + j;
-    const float vv = to_f32(v[gi]);
-    w.v32[gi] = vv;
-    w.bv[gi] = bs[r] * vv;
-    w.do32[gi] = to_f32(dout[gi]);
+  // V and dO: fp32 copies out now, V held in registers until P is formed
+  constexpr int kVU = 64 * 128 / kThreads;  // C * dv <= kVU * kThreads
+  float vr[kVU];
+#pragma unroll
+  for (int u = 0; u < kVU; ++u) {
+    const int idx = u * kThreads + tid;
+    const int r = idx / dv;
+    vr[u] = 0.f;
+    if (idx < C * dv && r < L) {
+      const size_t gi = ((size_t)(tok0 + r) * H + h) * dv + idx % dv;
+      vr[u] = to_f32(v[gi]);
+      w.v32[gi] = vr[u];
+      w.bv[gi] = bs[r] * vr[u];
+      w.do32[gi] = to_f32(dout[gi]);
+    }
   }
   for (int c = tid; c < dk; c += kThreads)
     w.gam[((size_t)cid * H + h) * dk + c] =
         __expf(g[((size_t)(tok0 + L - 1) * H + h) * dk + c]);
   __syncthreads();
   const size_t sqb = ((size_t)cid * H + h) * C * C;
-  for (int idx = tid; idx < 64 * ws::kFS; idx += kThreads) {
-    A[idx] = 0.f;
-    Tm[idx] = 0.f;
-  }
-  __syncthreads();
+  // Thread (ti, tj) owns rows ti + 16 a and columns tj + 16 b of each
+  // product, so the padded rows give conflict-free loads.
+  const int ti = tid >> 4, tj = tid & 15, nr = C / 16;
   {
-    // M and P together: thread (ti, tj) owns rows ti + 16 a and columns
-    // tj + 16 b (a, b < C / 16), so the padded rows give conflict-free loads
-    const int ti = tid >> 4, tj = tid & 15, nr = C / 16;
     float m[4][4], pv[4][4];
 #pragma unroll
     for (int a = 0; a < 4; ++a)
@@ -203,24 +217,84 @@ __global__ void __launch_bounds__(kThreads)
         }
       }
   }
-  __syncthreads();
-  // Tm = (I + Diag(b) M)^-1 by recursive doubling (identity past C)
+  __syncthreads();  // Qt is dead: V takes its place
+#pragma unroll
+  for (int u = 0; u < kVU; ++u) {
+    const int idx = u * kThreads + tid;
+    if (idx < C * dv) V[idx] = vr[u];
+  }
+  // Tm = (I + Diag(b) M)^-1 by recursive doubling (identity past C); V is
+  // read only after the barriers below
   ws::invert_unit_lower(A, Tm, Msc, tid);
   __syncthreads();
-  for (int idx = tid; idx < C * C; idx += kThreads)
-    w.tm[sqb + idx] = Tm[(idx / C) * ws::kFS + idx % C];
+  for (int idx = tid; idx < C * C; idx += kThreads) {
+    const int r = idx / C, i = idx % C;
+    w.tm[sqb + idx] = Tm[r * ws::kFS + i];
+  }
+  __syncthreads();
+  // Tm Diag(b), in place (Tm is lower triangular, zero above the diagonal)
+  for (int idx = tid; idx < C * C; idx += kThreads) {
+    const int r = idx / C, i = idx % C;
+    Tm[r * ws::kFS + i] *= bs[i];
+  }
+  __syncthreads();
+  // W = (Tm Diag(b)) Kt and U = (Tm Diag(b)) V over i = 0 .. C - 1 (the
+  // terms above the diagonal are exact zeros)
+  {
+    const int nw = dk / 16, nu = dv / 16;
+    float aw[4][8], au[4][8];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 8; ++b) aw[a][b] = au[a][b] = 0.f;
+    for (int i = 0; i < C; ++i) {
+      float t[4], kt[8], vv[8];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) t[a] = a < nr ? Tm[(ti + 16 * a) * ws::kFS + i] : 0.f;
+#pragma unroll
+      for (int b = 0; b < 8; ++b) {
+        kt[b] = b < nw ? Kt[i * ldk + tj + 16 * b] : 0.f;
+        vv[b] = b < nu ? V[i * dv + tj + 16 * b] : 0.f;
+      }
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+          aw[a][b] += t[a] * kt[b];
+          au[a][b] += t[a] * vv[b];
+        }
+    }
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const int r = ti + 16 * a;
+      if (a < nr && r < L) {
+        const size_t rw = ((size_t)(tok0 + r) * H + h) * dk;
+        const size_t ru = ((size_t)(tok0 + r) * H + h) * dv;
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+          if (b < nw) w_out[rw + tj + 16 * b] = aw[a][b];
+          if (b < nu) u_out[ru + tj + 16 * b] = au[a][b];
+        }
+      }
+    }
+  }
 }
 
 // The reverse chain over one sequence's chunks for one head and one TILE-wide
 // column tile of d_v (64, or 32 when d_v = 32, so that a d = 128 layer runs
 // one wave of CTAs).  Per chunk (last first), with dS the gradient of the
-// state leaving it: partial d gam, G = Diag(gam) dS (stored), dDelta = Kb G +
-// P^T dO (stored), then dS <- G + Qt^T dO - W^T dDelta.  Each product gives
-// every thread a block of outputs (rows strided by 32, columns by 8) so that
-// the sums over the contraction index run as independent chains; the shared
-// rows are padded (TILE + 1 floats for the tiles, d_k + 1 for the token rows)
-// so both access directions are free of bank conflicts.  The chunk-start
-// state enters only the d gam sum and is read there straight from memory.
+// state leaving it:
+//   gam * d gam (partial over the tile) = rowsum(S_next * dS), S_next being
+//     the state leaving the chunk (= gam (S_0 + Kb^T Delta)): the next
+//     chunk's stored start state, or the final state;
+//   G = Diag(gam) dS (stored);
+//   dDelta = Kb G + P^T dO (stored), P^T dO precomputed;
+//   dS <- G + Qt^T dO - W^T dDelta, Qt^T dO precomputed.
+// Only the two products with dS on their path are left in the serial loop.
+// Each gives every thread a block of outputs (rows strided by 32, columns by
+// 8) whose sums over the contraction index run as independent chains; the
+// shared rows are padded (TILE + 1 floats for the tiles, d_k + 1 for the
+// token rows) so both access directions are free of bank conflicts.
 __host__ __device__ constexpr int chain_tile(int dv) { return dv >= 64 ? 64 : 32; }
 
 template <int TILE>
@@ -236,12 +310,8 @@ __global__ void __launch_bounds__(kThreads)
   extern __shared__ float sm[];
   float* dS = sm;                    // [dk][TP]
   float* Kb = dS + dk * TP;          // [C][dkp]
-  float* Qt = Kb + C * dkp;          // [C][dkp]
-  float* Wc = Qt + C * dkp;          // [C][dkp]
-  float* P = Wc + C * dkp;           // [C][C]
-  float* dO = P + C * C;             // [C][TP]
-  float* De = dO + C * TP;           // [C][TP] Delta
-  float* dD = De + C * TP;           // [C][TP] dDelta
+  float* Wc = Kb + C * dkp;          // [C][dkp]
+  float* dD = Wc + C * dkp;          // [C][TP] dDelta
   float* gC = dD + C * TP;           // [dk]
 
   const size_t sbase = ((size_t)seq * H + h) * dk * dv;
@@ -258,18 +328,38 @@ __global__ void __launch_bounds__(kThreads)
   for (int ch = nch - 1; ch >= 0; --ch) {
     const int cid = cid0 + ch, tok0 = start + ch * C, L = min(C, end - tok0);
     const size_t cbase = ((size_t)cid * H + h) * dk * dv;
+    // per-thread operands straight to registers: S_next, P^T dO, Qt^T dO
+    const float* snx = ch + 1 < nch ? w.fv.s + cbase + (size_t)H * dk * dv
+                                    : w.fin + sbase;
+    float sn[4][NB], dacc[2][NB], sacc[4][NB];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        const size_t o = (size_t)(g8 + 32 * a) * dv + j0 + j8 + 8 * b;
+        sn[a][b] = a < NA ? snx[o] : 0.f;
+        sacc[a][b] = a < NA ? w.qdo[cbase + o] : 0.f;
+      }
+#pragma unroll
+    for (int a = 0; a < 2; ++a) {
+      const int r = g8 + 32 * a;
+#pragma unroll
+      for (int b = 0; b < NB; ++b)
+        dacc[a][b] = r < L ? w.pdo[((size_t)(tok0 + r) * H + h) * dv + j0 +
+                                   j8 + 8 * b]
+                           : 0.f;
+    }
     // staging loads batched eight deep so their latencies overlap
     for (int base = 0; base < C * dk; base += 8 * kThreads) {
-      float kb[8], qt[8], wv[8];
+      float kb[8], wv[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const int idx = base + u * kThreads + tid;
         const int r = idx / dk, c = idx % dk;
-        kb[u] = qt[u] = wv[u] = 0.f;
+        kb[u] = wv[u] = 0.f;
         if (idx < C * dk && r < L) {
           const size_t gi = ((size_t)(tok0 + r) * H + h) * dk + c;
           kb[u] = w.kb[gi];
-          qt[u] = w.qt[gi];
           wv[u] = w.fv.w[gi];
         }
       }
@@ -279,80 +369,25 @@ __global__ void __launch_bounds__(kThreads)
         if (idx < C * dk) {
           const int r = idx / dk, c = idx % dk;
           Kb[r * dkp + c] = kb[u];
-          Qt[r * dkp + c] = qt[u];
           Wc[r * dkp + c] = wv[u];
-        }
-      }
-    }
-    for (int idx = tid; idx < C * C; idx += kThreads)
-      P[idx] = w.pp[((size_t)cid * H + h) * C * C + idx];
-    {
-      constexpr int NU = 64 * TILE / kThreads;  // C * TILE <= NU * kThreads
-      float o[NU], de[NU];
-#pragma unroll
-      for (int u = 0; u < NU; ++u) {
-        const int idx = u * kThreads + tid;
-        const int r = idx / TILE, jj = idx % TILE;
-        o[u] = de[u] = 0.f;
-        if (idx < C * TILE && r < L) {
-          const size_t gi = ((size_t)(tok0 + r) * H + h) * dv + j0 + jj;
-          o[u] = w.do32[gi];
-          de[u] = w.fv.d[gi];
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < NU; ++u) {
-        const int idx = u * kThreads + tid;
-        if (idx < C * TILE) {
-          const int r = idx / TILE, jj = idx % TILE;
-          dO[r * TP + jj] = o[u];
-          De[r * TP + jj] = de[u];
         }
       }
     }
     for (int c = tid; c < dk; c += kThreads)
       gC[c] = w.gam[((size_t)cid * H + h) * dk + c];
-    __syncthreads();
-
-    // partial d gam over this tile: rowsum((S_0 + Kb^T Delta) * dS)
-    {
-      float s0[4][NB], x[4][NB];
+    // gam * d gam over this tile (dS is only read here)
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
+    for (int a = 0; a < 4; ++a) {
+      if (a < NA) {
+        const int c = g8 + 32 * a;
+        float part = 0.f;
 #pragma unroll
-        for (int b = 0; b < NB; ++b) {
-          x[a][b] = 0.f;
-          s0[a][b] = a < NA ? w.fv.s[cbase + (size_t)(g8 + 32 * a) * dv + j0 +
-                                     j8 + 8 * b]
-                            : 0.f;
-        }
-      for (int r = 0; r < L; ++r) {
-        float de[NB];
-#pragma unroll
-        for (int b = 0; b < NB; ++b) de[b] = De[r * TP + j8 + 8 * b];
-#pragma unroll
-        for (int a = 0; a < 4; ++a) {
-          if (a < NA) {
-            const float kb = Kb[r * dkp + g8 + 32 * a];
-#pragma unroll
-            for (int b = 0; b < NB; ++b) x[a][b] += kb * de[b];
-          }
-        }
-      }
-#pragma unroll
-      for (int a = 0; a < 4; ++a) {
-        if (a < NA) {
-          const int c = g8 + 32 * a;
-          float part = 0.f;
-#pragma unroll
-          for (int b = 0; b < NB; ++b)
-            part += (s0[a][b] + x[a][b]) * dS[c * TP + j8 + 8 * b];
-          part += __shfl_xor_sync(0xffffffffu, part, 1);
-          part += __shfl_xor_sync(0xffffffffu, part, 2);
-          part += __shfl_xor_sync(0xffffffffu, part, 4);
-          if (j8 == 0)
-            w.dgam[(((size_t)cid * H + h) * ntile + tile) * dk + c] = part;
-        }
+        for (int b = 0; b < NB; ++b) part += sn[a][b] * dS[c * TP + j8 + 8 * b];
+        part += __shfl_xor_sync(0xffffffffu, part, 1);
+        part += __shfl_xor_sync(0xffffffffu, part, 2);
+        part += __shfl_xor_sync(0xffffffffu, part, 4);
+        if (j8 == 0)
+          w.dgam[(((size_t)cid * H + h) * ntile + tile) * dk + c] = part;
       }
     }
     __syncthreads();
@@ -363,84 +398,54 @@ __global__ void __launch_bounds__(kThreads)
       w.gst[cbase + (size_t)c * dv + j0 + jj] = gv;
     }
     __syncthreads();
-    // dDelta = Kb G + P^T dO  (rows g8, g8 + 32)
-    {
-      float acc[2][NB];
+    // dDelta = P^T dO + Kb G  (rows g8, g8 + 32)
+    for (int c = 0; c < dk; ++c) {
+      float gv[NB];
 #pragma unroll
-      for (int a = 0; a < 2; ++a)
-#pragma unroll
-        for (int b = 0; b < NB; ++b) acc[a][b] = 0.f;
-      for (int c = 0; c < dk; ++c) {
-        float gv[NB];
-#pragma unroll
-        for (int b = 0; b < NB; ++b) gv[b] = dS[c * TP + j8 + 8 * b];
-#pragma unroll
-        for (int a = 0; a < 2; ++a) {
-          const int r = g8 + 32 * a;  // Kb rows past L are zero, past C absent
-          const float kb = r < C ? Kb[r * dkp + c] : 0.f;
-#pragma unroll
-          for (int b = 0; b < NB; ++b) acc[a][b] += kb * gv[b];
-        }
-      }
-      for (int i = 0; i < L; ++i) {
-        float o[NB];
-#pragma unroll
-        for (int b = 0; b < NB; ++b) o[b] = dO[i * TP + j8 + 8 * b];
-#pragma unroll
-        for (int a = 0; a < 2; ++a) {
-          const int r = g8 + 32 * a;
-          const float pv = r < C ? P[i * C + r] : 0.f;
-#pragma unroll
-          for (int b = 0; b < NB; ++b) acc[a][b] += pv * o[b];
-        }
-      }
+      for (int b = 0; b < NB; ++b) gv[b] = dS[c * TP + j8 + 8 * b];
 #pragma unroll
       for (int a = 0; a < 2; ++a) {
-        const int r = g8 + 32 * a;
-        if (r < C) {
+        const int r = g8 + 32 * a;  // Kb rows past L are zero, past C absent
+        const float kb = r < C ? Kb[r * dkp + c] : 0.f;
 #pragma unroll
-          for (int b = 0; b < NB; ++b) {
-            const int jj = j8 + 8 * b;
-            const float v = r < L ? acc[a][b] : 0.f;
-            dD[r * TP + jj] = v;
-            if (r < L) w.dd[((size_t)(tok0 + r) * H + h) * dv + j0 + jj] = v;
-          }
+        for (int b = 0; b < NB; ++b) dacc[a][b] += kb * gv[b];
+      }
+    }
+#pragma unroll
+    for (int a = 0; a < 2; ++a) {
+      const int r = g8 + 32 * a;
+      if (r < C) {
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          const int jj = j8 + 8 * b;
+          const float v = r < L ? dacc[a][b] : 0.f;
+          dD[r * TP + jj] = v;
+          if (r < L) w.dd[((size_t)(tok0 + r) * H + h) * dv + j0 + jj] = v;
         }
       }
     }
     __syncthreads();
     // dS <- G + Qt^T dO - W^T dDelta
-    {
-      float acc[4][NB];
+    for (int r = 0; r < L; ++r) {
+      float dd[NB];
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b = 0; b < NB; ++b) acc[a][b] = 0.f;
-      for (int r = 0; r < L; ++r) {
-        float o[NB], dd[NB];
-#pragma unroll
-        for (int b = 0; b < NB; ++b) {
-          o[b] = dO[r * TP + j8 + 8 * b];
-          dd[b] = dD[r * TP + j8 + 8 * b];
-        }
-#pragma unroll
-        for (int a = 0; a < 4; ++a) {
-          if (a < NA) {
-            const float qt = Qt[r * dkp + g8 + 32 * a];
-            const float wv = Wc[r * dkp + g8 + 32 * a];
-#pragma unroll
-            for (int b = 0; b < NB; ++b) acc[a][b] += qt * o[b] - wv * dd[b];
-          }
-        }
-      }
+      for (int b = 0; b < NB; ++b) dd[b] = dD[r * TP + j8 + 8 * b];
 #pragma unroll
       for (int a = 0; a < 4; ++a) {
         if (a < NA) {
+          const float wv = Wc[r * dkp + g8 + 32 * a];
 #pragma unroll
-          for (int b = 0; b < NB; ++b) {
-            const int i = (g8 + 32 * a) * TP + j8 + 8 * b;
-            dS[i] += acc[a][b];
-          }
+          for (int b = 0; b < NB; ++b) sacc[a][b] -= wv * dd[b];
+        }
+      }
+    }
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      if (a < NA) {
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          const int i = (g8 + 32 * a) * TP + j8 + 8 * b;
+          dS[i] += sacc[a][b];
         }
       }
     }
@@ -459,8 +464,8 @@ __global__ void __launch_bounds__(kThreads)
 // op(A) op(B) over one or two terms (+ Out), with op = transpose or not and an
 // optional lower-triangular mask on Out.  An operand is one of: token rows
 // [tokens, H, cols] (rows are the chunk's tokens), a per-chunk square
-// [chunks, H, C, C], or a per-chunk state [chunks, H, dk, dv].  Every m is the
-// chunk length L; n and the contraction length are L, d_k or d_v.
+// [chunks, H, C, C], or a per-chunk state [chunks, H, dk, dv].  m, n and the
+// contraction length are each L, d_k or d_v.
 enum MatKind { kTok = 0, kSq = 1, kState = 2 };
 enum Dim { kDimL = 0, kDimDk = 1, kDimDv = 2 };
 enum Mask { kMaskNone = 0, kMaskLowerIncl = 1, kMaskStrictLower = 2 };
@@ -481,8 +486,8 @@ struct BmmOp {
   MatRef out;
   BmmTerm term[2];
   int nterms;
-  int n;       // Dim code of n (m is always L)
-  int nd;      // padded n
+  int m, n;    // Dim codes
+  int md, nd;  // padded m and n
   int mask;
   float alpha;
   int accumulate;
@@ -605,9 +610,9 @@ __device__ __forceinline__ void lds_vec(const float* p, float* v) {
 
 // op(A) is staged transposed (AT[t][i]) and op(B) as is (Bs[t][j]), zero past
 // the valid extent, rows padded by four floats.  The 256 threads form a
-// 16 x 16 grid over the padded C x nd output; thread (ti, tj) owns the RM x RN
-// block at rows RM ti.., columns RN tj.. (RM = C / 16, RN = nd / 16), so every
-// thread works and each step of the contraction is RM / 4 + RN / 4 vector
+// 16 x 16 grid over the padded md x nd output; thread (ti, tj) owns the
+// RM x RN block at rows RM ti.., columns RN tj.. (RM = md / 16, RN = nd / 16),
+// so every thread works and each step of the contraction is a few vector
 // shared loads for RM x RN FMAs.
 template <int RM, int RN>
 __global__ void __launch_bounds__(kThreads)
@@ -652,7 +657,7 @@ __global__ void __launch_bounds__(kThreads)
         for (int b = 0; b < RN; ++b) acc[a][b] += av[a] * bv[b];
     }
   }
-  const int m = L, n = dim_of(op.n, L, dk, dv);
+  const int m = dim_of(op.m, L, dk, dv), n = dim_of(op.n, L, dk, dv);
   const Src so = src_of(op.out, cid, h, tok0, L, H, C, dk);
   const int j0 = RN * tj;
 #pragma unroll
@@ -727,7 +732,7 @@ __global__ void __launch_bounds__(kThreads)
     float dgm = 0.f;
     for (int t = 0; t < ntile; ++t)
       dgm += w.dgam[(((size_t)cid * H + h) * ntile + t) * dk + c];
-    dg[(L - 1) * dk + c] += w.gam[((size_t)cid * H + h) * dk + c] * dgm;
+    dg[(L - 1) * dk + c] += dgm;  // the partials already carry gam
     float acc = 0.f;
     for (int r = L - 1; r >= 0; --r) {
       acc += dg[r * dk + c];
@@ -735,14 +740,19 @@ __global__ void __launch_bounds__(kThreads)
     }
   }
   const size_t sqb = ((size_t)cid * H + h) * C * C;
-  for (int r = tid; r < L; r += kThreads) {
+  // d beta: one warp per row, lanes across the row, then a shuffle sum
+  const int warp = tid >> 5, lane = tid & 31;
+  for (int r = warp; r < L; r += kThreads / 32) {
     const size_t rk = ((size_t)(tok0 + r) * H + h) * dk;
     const size_t rv = ((size_t)(tok0 + r) * H + h) * dv;
     float acc = 0.f;
-    for (int c = 0; c < dk; ++c) acc += w.dbk[rk + c] * w.kt[rk + c];
-    for (int j = 0; j < dv; ++j) acc += w.dbv[rv + j] * w.v32[rv + j];
-    for (int i = 0; i < r; ++i) acc += w.da[sqb + r * C + i] * w.mm[sqb + r * C + i];
-    dbeta[(size_t)(tok0 + r) * H + h] = acc;
+    for (int c = lane; c < dk; c += 32) acc += w.dbk[rk + c] * w.kt[rk + c];
+    for (int j = lane; j < dv; j += 32) acc += w.dbv[rv + j] * w.v32[rv + j];
+    for (int i = lane; i < r; i += 32)
+      acc += w.da[sqb + r * C + i] * w.mm[sqb + r * C + i];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) dbeta[(size_t)(tok0 + r) * H + h] = acc;
   }
 }
 
@@ -753,7 +763,7 @@ cudaError_t set_smem(K kernel, size_t bytes) {
 }
 
 // Launch one batched product with the thread blocking its padded shape asks
-// for: RM = C / 16 rows and RN = nd / 16 columns per thread.
+// for: RM = md / 16 rows and RN = nd / 16 columns per thread.
 template <int RM, int RN>
 cudaError_t launch_bmm_t(const BmmOp& op, size_t smem, dim3 grid,
                          cudaStream_t stream, const int32_t* cu,
@@ -784,10 +794,11 @@ cudaError_t launch_bmm(const BmmOp& op, int C, size_t smem, dim3 grid,
                        cudaStream_t stream, const int32_t* cu,
                        const int32_t* co, int n_seqs, int T, int H, int dk,
                        int dv) {
-  switch (C) {
+  switch (op.md) {
     case 16: return launch_bmm_n<1>(op, C, smem, grid, stream, cu, co, n_seqs, T, H, dk, dv);
     case 32: return launch_bmm_n<2>(op, C, smem, grid, stream, cu, co, n_seqs, T, H, dk, dv);
     case 64: return launch_bmm_n<4>(op, C, smem, grid, stream, cu, co, n_seqs, T, H, dk, dv);
+    case 128: return launch_bmm_n<8>(op, C, smem, grid, stream, cu, co, n_seqs, T, H, dk, dv);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -796,7 +807,8 @@ template <typename IO>
 cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
   BwdWs w = carve_bwd(a, workspace, nullptr);
   const ChunkArgs f = forward_args(a, w.fin);
-  cudaError_t e = launch_staged_state(f, w.staged, &w.fv, stream);
+  // the forward's plan and cumulative log-decay
+  cudaError_t e = launch_staged_part(f, w.staged, &w.fv, false, stream);
   if (e != cudaSuccess) return e;
   const int C = f.chunk, H = f.H, dk = f.dk, dv = f.dv;
   const int64_t nch = max_chunks(f);
@@ -805,18 +817,67 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
   const dim3 grid((unsigned)(nch > 0 ? nch : 1), H);
 
   if (nch > 0) {
-    const size_t smp = 4 * (3 * (size_t)C * (dk + 1) + 2 * 64 * ws::kFS + 1024 + C);
+    const size_t smp =
+        4 * (2 * (size_t)C * (dk + 1) + (size_t)C * max(dk + 1, dv) +
+             2 * 64 * ws::kFS + 1024 + C);
     if ((e = set_smem(prep_kernel<IO>, smp)) != cudaSuccess) return e;
     prep_kernel<IO><<<grid, kThreads, smp, stream>>>(
         static_cast<const IO*>(f.q), static_cast<const IO*>(f.k),
         static_cast<const IO*>(f.v), f.beta, static_cast<const IO*>(a.d_out),
-        w.fv.g, w, cu, co, f.n_seqs, f.T, H, dk, dv, C);
+        w.fv.g, w, w.fv.w, w.fv.d, cu, co, f.n_seqs, f.T, H, dk, dv, C);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  // the forward's serial state pass: chunk-start states, Delta over U, and
+  // the final state
+  if ((e = launch_staged_part(f, w.staged, &w.fv, true, stream)) != cudaSuccess)
+    return e;
+
+  auto tok = [](float* p, int cols, int t = 0) { return MatRef{p, kTok, cols, t}; };
+  auto sq = [&](float* p, int t = 0) { return MatRef{p, kSq, C, t}; };
+  auto stt = [&](const float* p, int t = 0) {
+    return MatRef{const_cast<float*>(p), kState, dv, t};
+  };
+  auto dmax = [&](int code) { return code == kDimL ? C : code == kDimDk ? dk : dv; };
+  auto term = [&](MatRef x, MatRef y, int k) { return BmmTerm{x, y, dmax(k)}; };
+  auto bmm2 = [&](MatRef o, BmmTerm t0, BmmTerm t1, int nterms, int m, int n,
+                  int mask, float alpha, int accumulate) {
+    BmmOp op{};
+    op.out = o;
+    op.term[0] = t0;
+    op.term[1] = t1;
+    op.nterms = nterms;
+    op.m = m;
+    op.n = n;
+    op.md = dmax(m);
+    op.nd = dmax(n);
+    op.mask = mask;
+    op.alpha = alpha;
+    op.accumulate = accumulate;
+    const int kd = max(t0.kd, nterms > 1 ? t1.kd : 0);
+    const size_t smem = 4 * (size_t)kd * ((op.md + 4) + (op.nd + 4));
+    return launch_bmm(op, C, smem, grid, stream, cu, co, f.n_seqs, f.T, H, dk,
+                      dv);
+  };
+  auto bmm = [&](MatRef o, MatRef x, MatRef y, int n, int k, int mask,
+                 float alpha, int accumulate) {
+    const BmmTerm t = term(x, y, k);
+    return bmm2(o, t, t, 1, kDimL, n, mask, alpha, accumulate);
+  };
+  float* De = w.fv.d;  // Delta
+  const float* S0 = w.fv.s;
+#define KDA_BMM(...) \
+  if ((e = __VA_ARGS__) != cudaSuccess) return e;
+  if (nch > 0) {
+    // the chain's terms that do not depend on dS: Qt^T dO and P^T dO
+    const BmmTerm tq = term(tok(w.qt, dk, 1), tok(w.do32, dv), kDimL);
+    KDA_BMM(bmm2(stt(w.qdo), tq, tq, 1, kDimDk, kDimDv, kMaskNone, 1.f, 0))
+    KDA_BMM(bmm(tok(w.pdo, dv), sq(w.pp, 1), tok(w.do32, dv), kDimDv, kDimL,
+                kMaskNone, 1.f, 0))
   }
   {
     const int tile = chain_tile(dv), tp = tile + 1;
-    const size_t smc = 4 * ((size_t)dk * tp + 3 * (size_t)C * (dk + 1) +
-                            (size_t)C * C + 3 * (size_t)C * tp + dk);
+    const size_t smc = 4 * ((size_t)dk * tp + 2 * (size_t)C * (dk + 1) +
+                            (size_t)C * tp + dk);
     const dim3 cgrid(f.n_seqs, H, dv / tile);
     if (tile == 64) {
       if ((e = set_smem(chain_kernel<64>, smc)) != cudaSuccess) return e;
@@ -831,56 +892,23 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
   }
   if (nch == 0) return cudaSuccess;
 
-  auto tok = [](float* p, int cols, int t = 0) { return MatRef{p, kTok, cols, t}; };
-  auto sq = [&](float* p, int t = 0) { return MatRef{p, kSq, C, t}; };
-  auto stt = [&](const float* p, int t = 0) {
-    return MatRef{const_cast<float*>(p), kState, dv, t};
-  };
-  auto dmax = [&](int code) { return code == kDimL ? C : code == kDimDk ? dk : dv; };
-  auto term = [&](MatRef x, MatRef y, int k) { return BmmTerm{x, y, dmax(k)}; };
-  auto bmm2 = [&](MatRef o, BmmTerm t0, BmmTerm t1, int nterms, int n,
-                  int mask, float alpha, int accumulate) {
-    BmmOp op{};
-    op.out = o;
-    op.term[0] = t0;
-    op.term[1] = t1;
-    op.nterms = nterms;
-    op.n = n;
-    op.nd = dmax(n);
-    op.mask = mask;
-    op.alpha = alpha;
-    op.accumulate = accumulate;
-    const int kd = max(t0.kd, nterms > 1 ? t1.kd : 0);
-    const size_t smem = 4 * (size_t)kd * ((C + 4) + (op.nd + 4));
-    return launch_bmm(op, C, smem, grid, stream, cu, co, f.n_seqs, f.T, H, dk,
-                      dv);
-  };
-  auto bmm = [&](MatRef o, MatRef x, MatRef y, int n, int k, int mask,
-                 float alpha, int accumulate) {
-    const BmmTerm t = term(x, y, k);
-    return bmm2(o, t, t, 1, n, mask, alpha, accumulate);
-  };
-  float* De = const_cast<float*>(w.fv.d);  // Delta
-  const float* S0 = w.fv.s;
-#define KDA_BMM(...) \
-  if ((e = __VA_ARGS__) != cudaSuccess) return e;
   // dP = lower_incl(dO Delta^T)
   KDA_BMM(bmm(sq(w.dp), tok(w.do32, dv), tok(De, dv, 1), kDimL, kDimDv,
               kMaskLowerIncl, 1.f, 0))
   // dQt = dO S_0^T + dP Kb
   KDA_BMM(bmm2(tok(w.dqt, dk), term(tok(w.do32, dv), stt(S0, 1), kDimDv),
-               term(sq(w.dp), tok(w.kb, dk), kDimL), 2, kDimDk, kMaskNone, 1.f,
-               0))
+               term(sq(w.dp), tok(w.kb, dk), kDimL), 2, kDimL, kDimDk,
+               kMaskNone, 1.f, 0))
   // dKb = Delta G^T + dP^T Qt  (+ dA^T b Kt below)
   KDA_BMM(bmm2(tok(w.dkb, dk), term(tok(De, dv), stt(w.gst, 1), kDimDv),
-               term(sq(w.dp, 1), tok(w.qt, dk), kDimL), 2, kDimDk, kMaskNone,
-               1.f, 0))
+               term(sq(w.dp, 1), tok(w.qt, dk), kDimL), 2, kDimL, kDimDk,
+               kMaskNone, 1.f, 0))
   // dW = -dDelta S_0^T
   KDA_BMM(bmm(tok(w.dw, dk), tok(w.dd, dv), stt(S0, 1), kDimDk, kDimDv,
               kMaskNone, -1.f, 0))
   // dTm = dW (b Kt)^T + dDelta (b V)^T
   KDA_BMM(bmm2(sq(w.dtm), term(tok(w.dw, dk), tok(w.bkt, dk, 1), kDimDk),
-               term(tok(w.dd, dv), tok(w.bv, dv, 1), kDimDv), 2, kDimL,
+               term(tok(w.dd, dv), tok(w.bv, dv, 1), kDimDv), 2, kDimL, kDimL,
                kMaskNone, 1.f, 0))
   // Tm^T dW, Tm^T dDelta, Tm^T dTm
   KDA_BMM(bmm(tok(w.dbk, dk), sq(w.tm, 1), tok(w.dw, dk), kDimDk, kDimL,
@@ -907,7 +935,7 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-constexpr int kBmmOps = 11;
+constexpr int kBmmOps = 13;
 
 }  // namespace
 
@@ -921,10 +949,10 @@ int bwd_kernel_count(const BwdArgs& a) {
   const ChunkArgs f = forward_args(a, nullptr);
   if (f.n_seqs == 0 || f.H == 0) return 0;
   const bool any = max_chunks(f) > 0;
-  // the forward's stages (1)-(3), the reverse chain, then prep, the batched
-  // products and the final combination
-  return staged_kernel_count(f) - (any ? 1 : 0) + 1 +
-         (any ? 1 + kBmmOps + 1 : 0);
+  // the plan (packed layout), the forward's state pass and the reverse
+  // chain always; with any chunk also the cumulative log-decay, prep, the
+  // batched products and the final combination
+  return (f.cu_seqlens ? 1 : 0) + 2 + (any ? 1 + 1 + kBmmOps + 1 : 0);
 }
 
 cudaError_t launch_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {

@@ -63,20 +63,24 @@ size_t staged_workspace_bytes(const ChunkArgs& a);
 int staged_kernel_count(const ChunkArgs& a);
 cudaError_t launch_staged(const ChunkArgs& a, void* workspace,
                           cudaStream_t stream);
-// Stages (1)-(3) only (no outputs; the final state still goes to
-// a.final_state), leaving in the workspace what the backward pass reads:
-// the packed-layout chunk offsets, g = cumulative log-decay [tokens, H, dk],
-// W [tokens, H, dk], Delta = U - W S_0 [tokens, H, dv] and every chunk-start
-// state [max_chunks, H, dk, dv], all fp32.  Channel gate, no prologue.
+// The staged pipeline's pieces the backward pass wraps around its own
+// per-chunk preparation.  With state_pass false: the packed-layout chunk
+// offsets and g = cumulative log-decay [tokens, H, dk].  The caller then
+// writes W [tokens, H, dk] into view->w and U [tokens, H, dv] into view->d.
+// With state_pass true: the serial state pass, which turns U into
+// Delta = U - W S_0 in place, stores every chunk-start state
+// [max_chunks, H, dk, dv] in view->s and the final state in a.final_state.
+// All fp32; channel gate, no prologue.
 struct StagedView {
   const int32_t* chunk_off;
   const float* g;
-  const float* w;
-  const float* d;
+  float* w;
+  float* d;
   const float* s;
 };
-cudaError_t launch_staged_state(const ChunkArgs& a, void* workspace,
-                                StagedView* view, cudaStream_t stream);
+cudaError_t launch_staged_part(const ChunkArgs& a, void* workspace,
+                               StagedView* view, bool state_pass,
+                               cudaStream_t stream);
 
 // Chunkwise backward pass (kda_backward.cu): the gradients of
 // L = <d_out, out> + <d_final_state, final_state> with respect to q, k, v,

@@ -496,9 +496,14 @@ cudaError_t set_smem(K kernel, size_t bytes) {
                               (int)bytes);
 }
 
+// Which stages run: all four (the forward), or the pieces the backward pass
+// wraps around its own per-chunk preparation (the plan and the cumulative
+// log-decay first, the state pass after W and U are in place).
+enum class Part { kAll, kPrefix, kStatePass };
+
 template <typename IO>
 cudaError_t run(const ChunkArgs& a, void* workspace, cudaStream_t stream,
-                bool outputs = true) {
+                Part part = Part::kAll) {
   Ws w = carve(a, workspace, nullptr);
   const int C = a.chunk, H = a.H, dk = a.dk, dv = a.dv;
   const int64_t nch = max_chunks(a);
@@ -509,15 +514,20 @@ cudaError_t run(const ChunkArgs& a, void* workspace, cudaStream_t stream,
   IO* out = static_cast<IO*>(a.out);
   cudaError_t e;
 
-  if (cu) {
-    plan_kernel<<<1, 32, 0, stream>>>(cu, a.n_seqs, a.T, C, w.chunk_off);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (part != Part::kStatePass) {
+    if (cu) {
+      plan_kernel<<<1, 32, 0, stream>>>(cu, a.n_seqs, a.T, C, w.chunk_off);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if (nch > 0) {
+      cumsum_kernel<<<dim3((unsigned)nch, H), dk, 0, stream>>>(
+          a.log_alpha, w.g, cu, w.chunk_off, a.n_seqs, a.T, H, dk, C, a.gate);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if (part == Part::kPrefix) return cudaSuccess;
   }
-  if (nch > 0) {
+  if (part == Part::kAll && nch > 0) {
     const dim3 grid((unsigned)nch, H);
-    cumsum_kernel<<<grid, dk, 0, stream>>>(a.log_alpha, w.g, cu, w.chunk_off,
-                                          a.n_seqs, a.T, H, dk, C, a.gate);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
     const size_t sm2 = 4 * ((size_t)2 * C * (dk + 1) + (size_t)C * dv +
                             2 * 64 * ws::kFS + 1024 + C);
@@ -535,7 +545,7 @@ cudaError_t run(const ChunkArgs& a, void* workspace, cudaStream_t stream,
       a.n_seqs, a.T, H, dk, dv, C);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
-  if (nch > 0 && outputs) {
+  if (nch > 0 && part == Part::kAll) {
     const size_t sm4 = 4 * (2 * (size_t)C * (dk + 1) + (size_t)C * C +
                             (size_t)dk * kDvTile + (size_t)C * kDvTile);
     if ((e = set_smem(output_kernel<IO>, sm4)) != cudaSuccess) return e;
@@ -562,8 +572,9 @@ int staged_kernel_count(const ChunkArgs& a) {
          (has_prologue(a) && any_chunks ? 1 : 0);
 }
 
-cudaError_t launch_staged_state(const ChunkArgs& a, void* workspace,
-                                StagedView* view, cudaStream_t stream) {
+cudaError_t launch_staged_part(const ChunkArgs& a, void* workspace,
+                               StagedView* view, bool state_pass,
+                               cudaStream_t stream) {
   Ws w = carve(a, workspace, nullptr);
   view->chunk_off = w.chunk_off;
   view->g = w.g;
@@ -571,8 +582,9 @@ cudaError_t launch_staged_state(const ChunkArgs& a, void* workspace,
   view->d = w.u;
   view->s = w.s;
   if (a.n_seqs == 0 || a.H == 0) return cudaSuccess;
-  return a.bf16 ? run<__nv_bfloat16>(a, workspace, stream, false)
-                : run<float>(a, workspace, stream, false);
+  const Part part = state_pass ? Part::kStatePass : Part::kPrefix;
+  return a.bf16 ? run<__nv_bfloat16>(a, workspace, stream, part)
+                : run<float>(a, workspace, stream, part);
 }
 
 cudaError_t launch_staged(const ChunkArgs& a, void* workspace,
