@@ -105,15 +105,15 @@ BwdWs carve_bwd(const BwdArgs& a, void* base, size_t* total) {
 
 // Per (chunk, head): Kt, Kb, Qt, b Kt and fp32 copies of V, b V, dO; gam;
 // M = Kt Kb^T (strictly lower), P = lower_incl(Qt Kb^T), Tm = (I + Diag(b)
-// M)^-1 by recursive doubling, and the forward's W = Tm Diag(b) Kt and U =
-// Tm Diag(b) V for the state pass.
+// M)^-1 by recursive doubling, and the forward's W = Tm Diag(b) Kt, U =
+// Tm Diag(b) V and Kh = k exp(g_C - g) for the state pass.
 template <typename IO>
 __global__ void __launch_bounds__(kThreads)
     prep_kernel(const IO* __restrict__ q, const IO* __restrict__ k,
                 const IO* __restrict__ v, const float* __restrict__ beta,
                 const IO* __restrict__ dout, const float* __restrict__ g,
                 BwdWs w, float* __restrict__ w_out, float* __restrict__ u_out,
-                const int32_t* cu, const int32_t* chunk_off, int n_seqs,
+                float* __restrict__ kh_out, const int32_t* cu, const int32_t* chunk_off, int n_seqs,
                 int T, int H, int dk, int dv, int C) {
   const int cid = blockIdx.x;
   int seq, tok0, L;
@@ -129,9 +129,12 @@ __global__ void __launch_bounds__(kThreads)
   float* Tm = A + 64 * ws::kFS;    // [64][kFS]
   float* Msc = Tm + 64 * ws::kFS;  // [1024] scratch of the inverse
   float* bs = Msc + 1024;          // [C]
+  float* gl = bs + C;              // [dk] g at the chunk's last row
 
   for (int r = tid; r < C; r += kThreads)
     bs[r] = r < L ? beta[(size_t)(tok0 + r) * H + h] : 0.f;
+  for (int c = tid; c < dk; c += kThreads)
+    gl[c] = g[((size_t)(tok0 + L - 1) * H + h) * dk + c];
   for (int idx = tid; idx < 64 * ws::kFS; idx += kThreads) {
     A[idx] = 0.f;
     Tm[idx] = 0.f;
@@ -151,6 +154,7 @@ __global__ void __launch_bounds__(kThreads)
       w.kb[gi] = kb;
       w.qt[gi] = qt;
       w.bkt[gi] = bs[r] * kt;
+      kh_out[gi] = kv * __expf(gl[c] - gv);
     }
     Kt[r * ldk + c] = kt;
     Kb[r * ldk + c] = kb;
@@ -173,8 +177,7 @@ __global__ void __launch_bounds__(kThreads)
     }
   }
   for (int c = tid; c < dk; c += kThreads)
-    w.gam[((size_t)cid * H + h) * dk + c] =
-        __expf(g[((size_t)(tok0 + L - 1) * H + h) * dk + c]);
+    w.gam[((size_t)cid * H + h) * dk + c] = __expf(gl[c]);
   __syncthreads();
   const size_t sqb = ((size_t)cid * H + h) * C * C;
   // Thread (ti, tj) owns rows ti + 16 a and columns tj + 16 b of each
@@ -819,12 +822,13 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
   if (nch > 0) {
     const size_t smp =
         4 * (2 * (size_t)C * (dk + 1) + (size_t)C * max(dk + 1, dv) +
-             2 * 64 * ws::kFS + 1024 + C);
+             2 * 64 * ws::kFS + 1024 + C + dk);
     if ((e = set_smem(prep_kernel<IO>, smp)) != cudaSuccess) return e;
     prep_kernel<IO><<<grid, kThreads, smp, stream>>>(
         static_cast<const IO*>(f.q), static_cast<const IO*>(f.k),
         static_cast<const IO*>(f.v), f.beta, static_cast<const IO*>(a.d_out),
-        w.fv.g, w, w.fv.w, w.fv.d, cu, co, f.n_seqs, f.T, H, dk, dv, C);
+        w.fv.g, w, w.fv.w, w.fv.d, w.fv.kh, cu, co, f.n_seqs, f.T, H, dk, dv,
+        C);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   // the forward's serial state pass: chunk-start states, Delta over U, and

@@ -66,7 +66,9 @@ cudaError_t launch_staged(const ChunkArgs& a, void* workspace,
 // The staged pipeline's pieces the backward pass wraps around its own
 // per-chunk preparation.  With state_pass false: the packed-layout chunk
 // offsets and g = cumulative log-decay [tokens, H, dk].  The caller then
-// writes W [tokens, H, dk] into view->w and U [tokens, H, dv] into view->d.
+// writes W [tokens, H, dk] into view->w, U [tokens, H, dv] into view->d and
+// Kh = k exp(g_C - g) [tokens, H, dk] (g_C: g at the chunk's last token)
+// into view->kh.
 // With state_pass true: the serial state pass, which turns U into
 // Delta = U - W S_0 in place, stores every chunk-start state
 // [max_chunks, H, dk, dv] in view->s and the final state in a.final_state.
@@ -76,6 +78,7 @@ struct StagedView {
   const float* g;
   float* w;
   float* d;
+  float* kh;
   const float* s;
 };
 cudaError_t launch_staged_part(const ChunkArgs& a, void* workspace,

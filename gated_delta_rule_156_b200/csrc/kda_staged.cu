@@ -42,6 +42,7 @@ struct Ws {
   float* g;            // [tokens, H, dk]   cumulative log-decay within chunk
   float* w;            // [tokens, H, dk]   W rows
   float* u;            // [tokens, H, dv]   U rows, overwritten by D
+  float* kh;           // [tokens, H, dk]   Kh = k exp(g_C - g)
   float* s;            // [max_chunks, H, dk, dv]  chunk-start states
 };
 
@@ -70,6 +71,7 @@ Ws carve(const ChunkArgs& a, void* base, size_t* total) {
   w.g = reinterpret_cast<float*>(take(4 * tokens * H * a.dk));
   w.w = reinterpret_cast<float*>(take(4 * tokens * H * a.dk));
   w.u = reinterpret_cast<float*>(take(4 * tokens * H * a.dv));
+  w.kh = reinterpret_cast<float*>(take(4 * tokens * H * a.dk));
   w.s = reinterpret_cast<float*>(
       take(4 * (size_t)max_chunks(a) * H * a.dk * a.dv));
   if (total) *total = off;
@@ -149,12 +151,14 @@ __global__ void cumsum_kernel(const float* __restrict__ la, float* __restrict__ 
   }
 }
 
-// (2) A, Tm = (I + A)^-1, W = Tm Diag(b) Kt, U = Tm Diag(b) V.
+// (2) A, Tm = (I + A)^-1, W = Tm Diag(b) Kt, U = Tm Diag(b) V, and the
+// state pass's Kh = k exp(g_C - g).
 template <typename IO>
 __global__ void __launch_bounds__(kThreads)
     intra_kernel(const IO* __restrict__ k, const IO* __restrict__ v,
                  const float* __restrict__ beta, const float* __restrict__ g,
                  float* __restrict__ w_out, float* __restrict__ u_out,
+                 float* __restrict__ kh_out,
                  const int32_t* cu, const int32_t* chunk_off, int n_seqs, int T,
                  int H, int dk, int dv, int C) {
   int seq, tok0, L;
@@ -170,7 +174,11 @@ __global__ void __launch_bounds__(kThreads)
   float* Tm = A + 64 * ws::kFS;    // [64][kFS], (I + A)^-1
   float* Msc = Tm + 64 * ws::kFS;  // [1024] scratch of the inverse
   float* bs = Msc + 1024;          // [C]
+  float* gl = bs + C;              // [dk] g at the chunk's last row
 
+  for (int c = tid; c < dk; c += kThreads)
+    gl[c] = g[((size_t)(tok0 + L - 1) * H + h) * dk + c];
+  __syncthreads();
   for (int idx = tid; idx < C * dk; idx += kThreads) {
     const int r = idx / dk, c = idx % dk;
     float kt = 0.f, kb = 0.f;
@@ -179,6 +187,7 @@ __global__ void __launch_bounds__(kThreads)
       const float kv = to_f32(k[gi]), gv = g[gi];
       kt = kv * __expf(gv);
       kb = kv * __expf(-gv);
+      kh_out[gi] = kv * __expf(gl[c] - gv);
     }
     Kt[r * ldk + c] = kt;
     Kb[r * ldk + c] = kb;
@@ -280,100 +289,110 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
-// (3) Sequential over the chunks of one sequence; one 32-column tile of S.
-//   D = U - W S ;  S <- Diag(exp(g_C)) S + Kh^T D.  Stores every chunk-start
-// state (for stage 4), D (over U), and the final state.
-template <typename IO>
+// (3) Sequential over the chunks of one sequence; one TILE-wide column tile
+// of S (64, or 32 when d_v = 32, so that a d = 128 layer is one wave of CTAs).
+//   D = U - W S ;  S <- Diag(exp(g_C)) S + Kh^T D,  Kh = k exp(g_C - g) from
+// stage (2).  Stores every chunk-start state (for stage 4), D (over U), and
+// the final state.  The next chunk's W, Kh, U tile and decay are loaded into
+// registers while the current chunk computes, so the serial loop does not
+// wait on memory.  Shared rows are padded (TILE + 1 floats for the tiles,
+// dk + 1 for the token rows) so the products are free of bank conflicts; each
+// thread owns a block of outputs (rows strided by 32, columns by 8) whose sums
+// run as independent chains.
+template <int TILE>
 __global__ void __launch_bounds__(kThreads)
-    state_kernel(const IO* __restrict__ k, const float* __restrict__ g,
-                 const float* __restrict__ w, float* __restrict__ u,
+    state_kernel(const float* __restrict__ g, const float* __restrict__ w,
+                 const float* __restrict__ kh, float* __restrict__ u,
                  float* __restrict__ s_chunks,
                  const float* __restrict__ s_init, float* __restrict__ s_final,
                  const int32_t* cu, const int32_t* chunk_off, int n_seqs, int T,
                  int H, int dk, int dv, int C) {
-  const int seq = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * kDvTile;
+  constexpr int TP = TILE + 1, NB = TILE / 8;
+  constexpr int NP = 64 * 128 / kThreads;   // C * dk <= NP * kThreads
+  constexpr int NU = 64 * TILE / kThreads;  // C * TILE <= NU * kThreads
+  const int seq = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * TILE;
   const int tid = threadIdx.x;
-  // Shared rows padded (kTp = 33 floats for the 32-wide tiles, dk + 1 for the
-  // token rows) so the products below are free of bank conflicts; each thread
-  // owns a block of outputs (rows strided by 32, columns by 8) whose sums run
-  // as independent chains.
-  constexpr int kTp = kDvTile + 1;
   const int dkp = dk + 1, NA = dk / 32;
   const int g8 = tid >> 3, j8 = tid & 7;
   extern __shared__ float sm[];
-  float* S = sm;                  // [dk][kTp]
-  float* Wc = S + dk * kTp;       // [C][dkp]
+  float* S = sm;                  // [dk][TP]
+  float* Wc = S + dk * TP;        // [C][dkp]
   float* Kh = Wc + C * dkp;       // [C][dkp]
-  float* D = Kh + C * dkp;        // [C][kTp]
-  float* gC = D + C * kTp;        // [dk]
+  float* D = Kh + C * dkp;        // [C][TP]
+  float* gam = D + C * TP;        // [dk] exp(g_C)
 
   const size_t sbase = ((size_t)seq * H + h) * dk * dv;
-  for (int idx = tid; idx < dk * kDvTile; idx += kThreads) {
-    const int c = idx / kDvTile, jj = idx % kDvTile;
-    S[c * kTp + jj] = s_init ? s_init[sbase + (size_t)c * dv + j0 + jj] : 0.f;
+  for (int idx = tid; idx < dk * TILE; idx += kThreads) {
+    const int c = idx / TILE, jj = idx % TILE;
+    S[c * TP + jj] = s_init ? s_init[sbase + (size_t)c * dv + j0 + jj] : 0.f;
   }
   int start, end;
   seq_range(cu, seq, T, &start, &end);
   const int nch = (end - start + C - 1) / C;
   const int cid0 = cu ? chunk_off[seq] : seq * ((T + C - 1) / C);
+
+  float pw[NP], pk[NP], pu[NU], pg = 0.f;
+  auto fetch = [&](int ch) {
+    const int tok0 = start + ch * C, L = min(C, end - tok0);
+#pragma unroll
+    for (int q = 0; q < NP; ++q) {
+      const int idx = q * kThreads + tid, r = idx / dk;
+      const bool in = idx < C * dk && r < L;
+      const size_t gi = ((size_t)(tok0 + r) * H + h) * dk + idx % dk;
+      pw[q] = in ? w[gi] : 0.f;
+      pk[q] = in ? kh[gi] : 0.f;
+    }
+#pragma unroll
+    for (int q = 0; q < NU; ++q) {
+      const int idx = q * kThreads + tid, r = idx / TILE;
+      const bool in = idx < C * TILE && r < L;
+      pu[q] = in ? u[((size_t)(tok0 + r) * H + h) * dv + j0 + idx % TILE] : 0.f;
+    }
+    pg = tid < dk ? g[((size_t)(tok0 + L - 1) * H + h) * dk + tid] : 0.f;
+  };
+  if (nch > 0) fetch(0);
   __syncthreads();
 
   for (int ch = 0; ch < nch; ++ch) {
     const int tok0 = start + ch * C, L = min(C, end - tok0);
     const size_t cbase = ((size_t)(cid0 + ch) * H + h) * dk * dv;
-    for (int idx = tid; idx < dk * kDvTile; idx += kThreads) {
-      const int c = idx / kDvTile, jj = idx % kDvTile;
-      s_chunks[cbase + (size_t)c * dv + j0 + jj] = S[c * kTp + jj];
+    for (int idx = tid; idx < dk * TILE; idx += kThreads) {
+      const int c = idx / TILE, jj = idx % TILE;
+      s_chunks[cbase + (size_t)c * dv + j0 + jj] = S[c * TP + jj];
     }
-    for (int c = tid; c < dk; c += kThreads)
-      gC[c] = g[((size_t)(tok0 + L - 1) * H + h) * dk + c];
-    __syncthreads();
-    // staging loads batched eight deep so their latencies overlap
-    for (int base = 0; base < C * dk; base += 8 * kThreads) {
-      float wv[8], kv[8], gv[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int idx = base + u * kThreads + tid;
-        const int r = idx / dk;
-        wv[u] = kv[u] = gv[u] = 0.f;
-        if (idx < C * dk && r < L) {
-          const size_t gi = ((size_t)(tok0 + r) * H + h) * dk + idx % dk;
-          wv[u] = w[gi];
-          kv[u] = to_f32(k[gi]);
-          gv[u] = g[gi];
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int idx = base + u * kThreads + tid;
-        if (idx < C * dk) {
-          const int r = idx / dk, c = idx % dk;
-          Wc[r * dkp + c] = wv[u];
-          Kh[r * dkp + c] = r < L ? kv[u] * __expf(gC[c] - gv[u]) : 0.f;
-        }
+    for (int q = 0; q < NP; ++q) {
+      const int idx = q * kThreads + tid;
+      if (idx < C * dk) {
+        const int r = idx / dk, c = idx % dk;
+        Wc[r * dkp + c] = pw[q];
+        Kh[r * dkp + c] = pk[q];
       }
     }
-    for (int idx = tid; idx < C * kDvTile; idx += kThreads) {
-      const int r = idx / kDvTile, jj = idx % kDvTile;
-      D[r * kTp + jj] = r < L ? u[((size_t)(tok0 + r) * H + h) * dv + j0 + jj] : 0.f;
+#pragma unroll
+    for (int q = 0; q < NU; ++q) {
+      const int idx = q * kThreads + tid;
+      if (idx < C * TILE) D[(idx / TILE) * TP + idx % TILE] = pu[q];
     }
+    if (tid < dk) gam[tid] = __expf(pg);
     __syncthreads();
+    if (ch + 1 < nch) fetch(ch + 1);
     {  // D = U - W S   (rows g8, g8 + 32; columns j8 + 8 b)
-      float acc[2][4];
+      float acc[2][NB];
 #pragma unroll
       for (int a = 0; a < 2; ++a)
 #pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+        for (int b = 0; b < NB; ++b) acc[a][b] = 0.f;
       for (int c = 0; c < dk; ++c) {
-        float sv[4];
+        float sv[NB];
 #pragma unroll
-        for (int b = 0; b < 4; ++b) sv[b] = S[c * kTp + j8 + 8 * b];
+        for (int b = 0; b < NB; ++b) sv[b] = S[c * TP + j8 + 8 * b];
 #pragma unroll
         for (int a = 0; a < 2; ++a) {
           const int r = g8 + 32 * a;
           const float wv = r < C ? Wc[r * dkp + c] : 0.f;
 #pragma unroll
-          for (int b = 0; b < 4; ++b) acc[a][b] += wv * sv[b];
+          for (int b = 0; b < NB; ++b) acc[a][b] += wv * sv[b];
         }
       }
 #pragma unroll
@@ -381,10 +400,10 @@ __global__ void __launch_bounds__(kThreads)
         const int r = g8 + 32 * a;
         if (r < L) {
 #pragma unroll
-          for (int b = 0; b < 4; ++b) {
+          for (int b = 0; b < NB; ++b) {
             const int jj = j8 + 8 * b;
-            const float dvl = D[r * kTp + jj] - acc[a][b];
-            D[r * kTp + jj] = dvl;
+            const float dvl = D[r * TP + jj] - acc[a][b];
+            D[r * TP + jj] = dvl;
             u[((size_t)(tok0 + r) * H + h) * dv + j0 + jj] = dvl;
           }
         }
@@ -392,21 +411,21 @@ __global__ void __launch_bounds__(kThreads)
     }
     __syncthreads();
     {  // S <- Diag(exp(g_C)) S + Kh^T D   (rows g8 + 32 a; columns j8 + 8 b)
-      float acc[4][4];
+      float acc[4][NB];
 #pragma unroll
       for (int a = 0; a < 4; ++a)
 #pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+        for (int b = 0; b < NB; ++b) acc[a][b] = 0.f;
       for (int r = 0; r < L; ++r) {
-        float dvv[4];
+        float dvv[NB];
 #pragma unroll
-        for (int b = 0; b < 4; ++b) dvv[b] = D[r * kTp + j8 + 8 * b];
+        for (int b = 0; b < NB; ++b) dvv[b] = D[r * TP + j8 + 8 * b];
 #pragma unroll
         for (int a = 0; a < 4; ++a) {
           if (a < NA) {
-            const float kh = Kh[r * dkp + g8 + 32 * a];
+            const float khv = Kh[r * dkp + g8 + 32 * a];
 #pragma unroll
-            for (int b = 0; b < 4; ++b) acc[a][b] += kh * dvv[b];
+            for (int b = 0; b < NB; ++b) acc[a][b] += khv * dvv[b];
           }
         }
       }
@@ -414,10 +433,10 @@ __global__ void __launch_bounds__(kThreads)
       for (int a = 0; a < 4; ++a) {
         if (a < NA) {
           const int c = g8 + 32 * a;
-          const float ga = __expf(gC[c]);
+          const float ga = gam[c];
 #pragma unroll
-          for (int b = 0; b < 4; ++b) {
-            const int i = c * kTp + j8 + 8 * b;
+          for (int b = 0; b < NB; ++b) {
+            const int i = c * TP + j8 + 8 * b;
             S[i] = ga * S[i] + acc[a][b];
           }
         }
@@ -425,9 +444,9 @@ __global__ void __launch_bounds__(kThreads)
     }
     __syncthreads();
   }
-  for (int idx = tid; idx < dk * kDvTile; idx += kThreads) {
-    const int c = idx / kDvTile, jj = idx % kDvTile;
-    s_final[sbase + (size_t)c * dv + j0 + jj] = S[c * kTp + jj];
+  for (int idx = tid; idx < dk * TILE; idx += kThreads) {
+    const int c = idx / TILE, jj = idx % TILE;
+    s_final[sbase + (size_t)c * dv + j0 + jj] = S[c * TP + jj];
   }
 }
 
@@ -530,20 +549,31 @@ cudaError_t run(const ChunkArgs& a, void* workspace, cudaStream_t stream,
     const dim3 grid((unsigned)nch, H);
 
     const size_t sm2 = 4 * ((size_t)2 * C * (dk + 1) + (size_t)C * dv +
-                            2 * 64 * ws::kFS + 1024 + C);
+                            2 * 64 * ws::kFS + 1024 + C + dk);
     if ((e = set_smem(intra_kernel<IO>, sm2)) != cudaSuccess) return e;
     intra_kernel<IO><<<grid, kThreads, sm2, stream>>>(
-        k, v, a.beta, w.g, w.w, w.u, cu, w.chunk_off, a.n_seqs, a.T, H, dk, dv,
-        C);
+        k, v, a.beta, w.g, w.w, w.u, w.kh, cu, w.chunk_off, a.n_seqs, a.T, H,
+        dk, dv, C);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  const size_t sm3 = 4 * ((size_t)dk * (kDvTile + 1) + 2 * (size_t)C * (dk + 1) +
-                          (size_t)C * (kDvTile + 1) + dk);
-  if ((e = set_smem(state_kernel<IO>, sm3)) != cudaSuccess) return e;
-  state_kernel<IO><<<dim3(a.n_seqs, H, dv / kDvTile), kThreads, sm3, stream>>>(
-      k, w.g, w.w, w.u, w.s, a.initial_state, a.final_state, cu, w.chunk_off,
-      a.n_seqs, a.T, H, dk, dv, C);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  {
+    const int tile = dv >= 64 ? 64 : 32, tp = tile + 1;
+    const size_t sm3 = 4 * ((size_t)dk * tp + 2 * (size_t)C * (dk + 1) +
+                            (size_t)C * tp + dk);
+    const dim3 sgrid(a.n_seqs, H, dv / tile);
+    if (tile == 64) {
+      if ((e = set_smem(state_kernel<64>, sm3)) != cudaSuccess) return e;
+      state_kernel<64><<<sgrid, kThreads, sm3, stream>>>(
+          w.g, w.w, w.kh, w.u, w.s, a.initial_state, a.final_state, cu,
+          w.chunk_off, a.n_seqs, a.T, H, dk, dv, C);
+    } else {
+      if ((e = set_smem(state_kernel<32>, sm3)) != cudaSuccess) return e;
+      state_kernel<32><<<sgrid, kThreads, sm3, stream>>>(
+          w.g, w.w, w.kh, w.u, w.s, a.initial_state, a.final_state, cu,
+          w.chunk_off, a.n_seqs, a.T, H, dk, dv, C);
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
 
   if (nch > 0 && part == Part::kAll) {
     const size_t sm4 = 4 * (2 * (size_t)C * (dk + 1) + (size_t)C * C +
@@ -580,6 +610,7 @@ cudaError_t launch_staged_part(const ChunkArgs& a, void* workspace,
   view->g = w.g;
   view->w = w.w;
   view->d = w.u;
+  view->kh = w.kh;
   view->s = w.s;
   if (a.n_seqs == 0 || a.H == 0) return cudaSuccess;
   const Part part = state_pass ? Part::kStatePass : Part::kPrefix;
