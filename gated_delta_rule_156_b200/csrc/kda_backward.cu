@@ -20,7 +20,8 @@
 //   dTm = dW (b Kt)^T + dDelta (b V)^T
 //   dA  = strictly_lower(-Tm^T dTm Tm^T)
 //   dKt = b (Tm^T dW + dA Kb),  dV = b Tm^T dDelta
-//   db  = rowsum(Tm^T dW * Kt) + rowsum(Tm^T dDelta * V) + rowsum(dA * M)
+//   db  = rowsum(Tm^T dW * Kt) + rowsum(Tm^T dDelta * V) + rowsum(dA * M),
+//         where rowsum(dA * M) = rowsum((dA Kb) * Kt) since M = Kt Kb^T
 //   dk  = dKt e^g + dKb e^-g,  dq = dQt e^g
 //   dg  = dKt * Kt + dQt * Qt - dKb * Kb  (+ gam * d gam on the last row)
 //   dlog_alpha = reverse cumulative sum of dg within the chunk
@@ -48,12 +49,12 @@ struct BwdWs {
   float* fin;                     // scratch final state of the forward
   float *kt, *kb, *qt, *bkt;      // [tokens, H, dk]
   float *v32, *bv, *do32, *dd;    // [tokens, H, dv]
-  float *tm, *mm, *pp;            // [chunks, H, C, C]
+  float *tm, *pp;                 // [chunks, H, C, C]
   float *gam;                     // [chunks, H, dk]
   float *gst;                     // G = Diag(gam) dS_C, [chunks, H, dk, dv]
   float *dgam;                    // [chunks, H, dv / 32, dk] partials of gam * d gam
   float *dp, *dtm, *tmp, *da;     // [chunks, H, C, C]
-  float *dqt, *dkb, *dw, *dbk, *y1;  // [tokens, H, dk]
+  float *dqt, *dkb, *dw, *dbk;    // [tokens, H, dk]; dbk = Tm^T dW + dA Kb
   float *dbv;                     // [tokens, H, dv]
   float *qdo;                     // Qt^T dO, [chunks, H, dk, dv]
   float *pdo;                     // P^T dO, [tokens, H, dv]
@@ -89,13 +90,12 @@ BwdWs carve_bwd(const BwdArgs& a, void* base, size_t* total) {
   const size_t sq = 4 * nch * H * C * C, st = 4 * nch * H * dk * dv;
   w.kt = take(tdk); w.kb = take(tdk); w.qt = take(tdk); w.bkt = take(tdk);
   w.v32 = take(tdv); w.bv = take(tdv); w.do32 = take(tdv); w.dd = take(tdv);
-  w.tm = take(sq); w.mm = take(sq); w.pp = take(sq);
+  w.tm = take(sq); w.pp = take(sq);
   w.gam = take(4 * nch * H * dk);
   w.gst = take(st);
   w.dgam = take(4 * nch * H * (dv / 32) * dk);
   w.dp = take(sq); w.dtm = take(sq); w.tmp = take(sq); w.da = take(sq);
   w.dqt = take(tdk); w.dkb = take(tdk); w.dw = take(tdk); w.dbk = take(tdk);
-  w.y1 = take(tdk);
   w.dbv = take(tdv);
   w.qdo = take(st);
   w.pdo = take(tdv);
@@ -103,8 +103,17 @@ BwdWs carve_bwd(const BwdArgs& a, void* base, size_t* total) {
   return w;
 }
 
+// Floats in each of prep's three shared regions: a [C][d_k + 1] or [C][d_v]
+// token tile, or the inverse's 64 x kFS tile (plus its scratch).
+__host__ __device__ constexpr int prep_region(int C, int dk, int dv) {
+  return C * (dk + 1 > dv ? dk + 1 : dv) > 64 * ws::kFS + 1024
+             ? C * (dk + 1 > dv ? dk + 1 : dv)
+             : 64 * ws::kFS + 1024;
+}
+
 // Per (chunk, head): Kt, Kb, Qt, b Kt and fp32 copies of V, b V, dO; gam;
-// M = Kt Kb^T (strictly lower), P = lower_incl(Qt Kb^T), Tm = (I + Diag(b)
+// M = Kt Kb^T (strictly lower, kept only on chip), P = lower_incl(Qt Kb^T),
+// Tm = (I + Diag(b)
 // M)^-1 by recursive doubling, and the forward's W = Tm Diag(b) Kt, U =
 // Tm Diag(b) V and Kh = k exp(g_C - g) for the state pass.
 template <typename IO>
@@ -120,25 +129,25 @@ __global__ void __launch_bounds__(kThreads)
   if (!locate_chunk(cid, cu, chunk_off, n_seqs, T, C, &seq, &tok0, &L)) return;
   const int h = blockIdx.y, tid = threadIdx.x;
   extern __shared__ float sm[];
+  // Three [C][ldk] regions, reused as the chunk moves on so that two CTAs
+  // fit on an SM: Kt, then V (once W is formed); Kb, then A and the
+  // inverse's scratch (once M and P are formed); Qt, then Tm.
   const int ldk = dk + 1;          // padded rows: no bank conflicts
+  const int reg = prep_region(C, dk, dv);
   float* Kt = sm;                  // [C][ldk]
-  float* Kb = Kt + C * ldk;        // [C][ldk]
-  float* Qt = Kb + C * ldk;        // [C][ldk]; V [C][dv] once P is formed
-  float* V = Qt;
-  float* A = Qt + C * max(ldk, dv);  // [64][kFS] b M, zero-padded past C
-  float* Tm = A + 64 * ws::kFS;    // [64][kFS]
-  float* Msc = Tm + 64 * ws::kFS;  // [1024] scratch of the inverse
-  float* bs = Msc + 1024;          // [C]
+  float* V = Kt;                   // [C][dv]
+  float* Kb = Kt + reg;            // [C][ldk]
+  float* A = Kb;                   // [64][kFS] b M, zero-padded past C
+  float* Msc = A + 64 * ws::kFS;   // [1024] scratch of the inverse
+  float* Qt = Kb + reg;            // [C][ldk]
+  float* Tm = Qt;                  // [64][kFS]
+  float* bs = Qt + reg;            // [C]
   float* gl = bs + C;              // [dk] g at the chunk's last row
 
   for (int r = tid; r < C; r += kThreads)
     bs[r] = r < L ? beta[(size_t)(tok0 + r) * H + h] : 0.f;
   for (int c = tid; c < dk; c += kThreads)
     gl[c] = g[((size_t)(tok0 + L - 1) * H + h) * dk + c];
-  for (int idx = tid; idx < 64 * ws::kFS; idx += kThreads) {
-    A[idx] = 0.f;
-    Tm[idx] = 0.f;
-  }
   __syncthreads();
   for (int idx = tid; idx < C * dk; idx += kThreads) {
     const int r = idx / dk, c = idx % dk;
@@ -160,7 +169,7 @@ __global__ void __launch_bounds__(kThreads)
     Kb[r * ldk + c] = kb;
     Qt[r * ldk + c] = qt;
   }
-  // V and dO: fp32 copies out now, V held in registers until P is formed
+  // V and dO: fp32 copies out now, V held in registers until W is formed
   constexpr int kVU = 64 * 128 / kThreads;  // C * dv <= kVU * kThreads
   float vr[kVU];
 #pragma unroll
@@ -183,8 +192,9 @@ __global__ void __launch_bounds__(kThreads)
   // Thread (ti, tj) owns rows ti + 16 a and columns tj + 16 b of each
   // product, so the padded rows give conflict-free loads.
   const int ti = tid >> 4, tj = tid & 15, nr = C / 16;
+  float m[4][4];
   {
-    float m[4][4], pv[4][4];
+    float pv[4][4];
 #pragma unroll
     for (int a = 0; a < 4; ++a)
 #pragma unroll
@@ -213,21 +223,26 @@ __global__ void __launch_bounds__(kThreads)
       for (int b = 0; b < 4; ++b) {
         if (a < nr && b < nr) {
           const int r = ti + 16 * a, i = tj + 16 * b;
-          const float mv = (r < L && i < r) ? m[a][b] : 0.f;
-          A[r * ws::kFS + i] = bs[r] * mv;
-          w.mm[sqb + r * C + i] = mv;
+          m[a][b] = (r < L && i < r) ? m[a][b] : 0.f;
           w.pp[sqb + r * C + i] = (r < L && i <= r) ? pv[a][b] : 0.f;
         }
       }
   }
-  __syncthreads();  // Qt is dead: V takes its place
-#pragma unroll
-  for (int u = 0; u < kVU; ++u) {
-    const int idx = u * kThreads + tid;
-    if (idx < C * dv) V[idx] = vr[u];
+  __syncthreads();  // Kb and Qt are dead: A and Tm take their places
+  for (int idx = tid; idx < 64 * ws::kFS; idx += kThreads) {
+    A[idx] = 0.f;
+    Tm[idx] = 0.f;
   }
-  // Tm = (I + Diag(b) M)^-1 by recursive doubling (identity past C); V is
-  // read only after the barriers below
+  __syncthreads();
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int r = ti + 16 * a, i = tj + 16 * b;
+      if (a < nr && b < nr) A[r * ws::kFS + i] = bs[r] * m[a][b];
+    }
+  __syncthreads();
+  // Tm = (I + Diag(b) M)^-1 by recursive doubling (identity past C)
   ws::invert_unit_lower(A, Tm, Msc, tid);
   __syncthreads();
   for (int idx = tid; idx < C * C; idx += kThreads) {
@@ -241,51 +256,55 @@ __global__ void __launch_bounds__(kThreads)
     Tm[r * ws::kFS + i] *= bs[i];
   }
   __syncthreads();
-  // W = (Tm Diag(b)) Kt and U = (Tm Diag(b)) V over i = 0 .. C - 1 (the
-  // terms above the diagonal are exact zeros)
-  {
-    const int nw = dk / 16, nu = dv / 16;
-    float aw[4][8], au[4][8];
+  // W = (Tm Diag(b)) Kt, then U = (Tm Diag(b)) V with V over Kt, each over
+  // i = 0 .. C - 1 (the terms above the diagonal are exact zeros)
+  for (int pass = 0; pass < 2; ++pass) {
+    const float* X = pass == 0 ? Kt : V;
+    const int ldx = pass == 0 ? ldk : dv;
+    const int nx = (pass == 0 ? dk : dv) / 16, cols = pass == 0 ? dk : dv;
+    float* out = pass == 0 ? w_out : u_out;
+    if (pass == 1) {
+      __syncthreads();  // every read of Kt is done
+#pragma unroll
+      for (int u = 0; u < kVU; ++u) {
+        const int idx = u * kThreads + tid;
+        if (idx < C * dv) V[idx] = vr[u];
+      }
+      __syncthreads();
+    }
+    float acc[4][8];
 #pragma unroll
     for (int a = 0; a < 4; ++a)
 #pragma unroll
-      for (int b = 0; b < 8; ++b) aw[a][b] = au[a][b] = 0.f;
+      for (int b = 0; b < 8; ++b) acc[a][b] = 0.f;
+#pragma unroll 2
     for (int i = 0; i < C; ++i) {
-      float t[4], kt[8], vv[8];
+      float t[4], xv[8];
 #pragma unroll
       for (int a = 0; a < 4; ++a) t[a] = a < nr ? Tm[(ti + 16 * a) * ws::kFS + i] : 0.f;
 #pragma unroll
-      for (int b = 0; b < 8; ++b) {
-        kt[b] = b < nw ? Kt[i * ldk + tj + 16 * b] : 0.f;
-        vv[b] = b < nu ? V[i * dv + tj + 16 * b] : 0.f;
-      }
+      for (int b = 0; b < 8; ++b) xv[b] = b < nx ? X[i * ldx + tj + 16 * b] : 0.f;
 #pragma unroll
       for (int a = 0; a < 4; ++a)
 #pragma unroll
-        for (int b = 0; b < 8; ++b) {
-          aw[a][b] += t[a] * kt[b];
-          au[a][b] += t[a] * vv[b];
-        }
+        for (int b = 0; b < 8; ++b) acc[a][b] += t[a] * xv[b];
     }
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
       const int r = ti + 16 * a;
       if (a < nr && r < L) {
-        const size_t rw = ((size_t)(tok0 + r) * H + h) * dk;
-        const size_t ru = ((size_t)(tok0 + r) * H + h) * dv;
+        const size_t ro = ((size_t)(tok0 + r) * H + h) * cols;
 #pragma unroll
-        for (int b = 0; b < 8; ++b) {
-          if (b < nw) w_out[rw + tj + 16 * b] = aw[a][b];
-          if (b < nu) u_out[ru + tj + 16 * b] = au[a][b];
-        }
+        for (int b = 0; b < 8; ++b)
+          if (b < nx) out[ro + tj + 16 * b] = acc[a][b];
       }
     }
   }
 }
 
-// The reverse chain over one sequence's chunks for one head and one TILE-wide
-// column tile of d_v (64, or 32 when d_v = 32, so that a d = 128 layer runs
-// one wave of CTAs).  Per chunk (last first), with dS the gradient of the
+// The reverse chain over one sequence's chunks for one head and one 32-wide
+// column tile of d_v (92 KB of shared memory at d = 128, so two CTAs share an
+// SM and a B=2, H=32 layer's 256 CTAs run as one wave).  Per chunk (last first), with dS the gradient of the
 // state leaving it:
 //   gam * d gam (partial over the tile) = rowsum(S_next * dS), S_next being
 //     the state leaving the chunk (= gam (S_0 + Kb^T Delta)): the next
@@ -298,7 +317,7 @@ __global__ void __launch_bounds__(kThreads)
 // 8) whose sums over the contraction index run as independent chains; the
 // shared rows are padded (TILE + 1 floats for the tiles, d_k + 1 for the
 // token rows) so both access directions are free of bank conflicts.
-__host__ __device__ constexpr int chain_tile(int dv) { return dv >= 64 ? 64 : 32; }
+constexpr int kChainTile = 32;
 
 template <int TILE>
 __global__ void __launch_bounds__(kThreads)
@@ -402,6 +421,7 @@ __global__ void __launch_bounds__(kThreads)
     }
     __syncthreads();
     // dDelta = P^T dO + Kb G  (rows g8, g8 + 32)
+    #pragma unroll 4
     for (int c = 0; c < dk; ++c) {
       float gv[NB];
 #pragma unroll
@@ -429,6 +449,7 @@ __global__ void __launch_bounds__(kThreads)
     }
     __syncthreads();
     // dS <- G + Qt^T dO - W^T dDelta
+    #pragma unroll 4
     for (int r = 0; r < L; ++r) {
       float dd[NB];
 #pragma unroll
@@ -464,7 +485,7 @@ __global__ void __launch_bounds__(kThreads)
 
 // ---------------------------------------------------------------------------
 // Batched small products over every (chunk, head): Out (m x n) = alpha sum of
-// op(A) op(B) over one or two terms (+ Out), with op = transpose or not and an
+// op(A) op(B) over one to three terms (+ Out), with op = transpose or not and an
 // optional lower-triangular mask on Out.  An operand is one of: token rows
 // [tokens, H, cols] (rows are the chunk's tokens), a per-chunk square
 // [chunks, H, C, C], or a per-chunk state [chunks, H, dk, dv].  m, n and the
@@ -487,7 +508,7 @@ struct BmmTerm {
 
 struct BmmOp {
   MatRef out;
-  BmmTerm term[2];
+  BmmTerm term[3];
   int nterms;
   int m, n;    // Dim codes
   int md, nd;  // padded m and n
@@ -616,9 +637,10 @@ __device__ __forceinline__ void lds_vec(const float* p, float* v) {
 // 16 x 16 grid over the padded md x nd output; thread (ti, tj) owns the
 // RM x RN block at rows RM ti.., columns RN tj.. (RM = md / 16, RN = nd / 16),
 // so every thread works and each step of the contraction is a few vector
-// shared loads for RM x RN FMAs.
+// shared loads for RM x RN FMAs.  Up to 4 x 8 blocks the registers are capped
+// so that three CTAs share an SM and hide each other's staging.
 template <int RM, int RN>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, RM * RN >= 64 ? 1 : 3)
     bmm_kernel(BmmOp op, const int32_t* cu, const int32_t* chunk_off, int n_seqs,
                int T, int H, int dk, int dv, int C) {
   const int cid = blockIdx.x;
@@ -635,7 +657,8 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
     for (int b = 0; b < RN; ++b) acc[a][b] = 0.f;
   for (int term = 0; term < op.nterms; ++term) {
-    const BmmTerm tm = term == 0 ? op.term[0] : op.term[1];
+    const BmmTerm tm = term == 0 ? op.term[0]
+                       : term == 1 ? op.term[1] : op.term[2];
     const int kd = tm.kd;
     float* AT = sm;            // [kd][la]
     float* Bs = sm + kd * la;  // [kd][lb]
@@ -711,14 +734,14 @@ __global__ void __launch_bounds__(kThreads)
   const int cid = blockIdx.x;
   int seq, tok0, L;
   if (!locate_chunk(cid, cu, chunk_off, n_seqs, T, C, &seq, &tok0, &L)) return;
-  const int h = blockIdx.y, tid = threadIdx.x, ntile = dv / chain_tile(dv);
+  const int h = blockIdx.y, tid = threadIdx.x, ntile = dv / kChainTile;
   extern __shared__ float sm[];
   float* dg = sm;  // [C][dk]
   for (int idx = tid; idx < L * dk; idx += kThreads) {
     const int r = idx / dk;
     const size_t gi = ((size_t)(tok0 + r) * H + h) * dk + idx % dk;
     const float b = beta[(size_t)(tok0 + r) * H + h];
-    const float dKt = b * (w.dbk[gi] + w.y1[gi]);
+    const float dKt = b * w.dbk[gi];
     const float dKb = w.dkb[gi], dQt = w.dqt[gi];
     const float gv = g[gi], e = __expf(gv), ie = __expf(-gv);
     dk_out[gi] = from_f32<IO>(dKt * e + dKb * ie);
@@ -742,7 +765,6 @@ __global__ void __launch_bounds__(kThreads)
       dla[((size_t)(tok0 + r) * H + h) * dk + c] = acc;
     }
   }
-  const size_t sqb = ((size_t)cid * H + h) * C * C;
   // d beta: one warp per row, lanes across the row, then a shuffle sum
   const int warp = tid >> 5, lane = tid & 31;
   for (int r = warp; r < L; r += kThreads / 32) {
@@ -751,8 +773,6 @@ __global__ void __launch_bounds__(kThreads)
     float acc = 0.f;
     for (int c = lane; c < dk; c += 32) acc += w.dbk[rk + c] * w.kt[rk + c];
     for (int j = lane; j < dv; j += 32) acc += w.dbv[rv + j] * w.v32[rv + j];
-    for (int i = lane; i < r; i += 32)
-      acc += w.da[sqb + r * C + i] * w.mm[sqb + r * C + i];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     if (lane == 0) dbeta[(size_t)(tok0 + r) * H + h] = acc;
@@ -820,9 +840,7 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
   const dim3 grid((unsigned)(nch > 0 ? nch : 1), H);
 
   if (nch > 0) {
-    const size_t smp =
-        4 * (2 * (size_t)C * (dk + 1) + (size_t)C * max(dk + 1, dv) +
-             2 * 64 * ws::kFS + 1024 + C + dk);
+    const size_t smp = 4 * (3 * (size_t)prep_region(C, dk, dv) + C + dk);
     if ((e = set_smem(prep_kernel<IO>, smp)) != cudaSuccess) return e;
     prep_kernel<IO><<<grid, kThreads, smp, stream>>>(
         static_cast<const IO*>(f.q), static_cast<const IO*>(f.k),
@@ -843,12 +861,13 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
   };
   auto dmax = [&](int code) { return code == kDimL ? C : code == kDimDk ? dk : dv; };
   auto term = [&](MatRef x, MatRef y, int k) { return BmmTerm{x, y, dmax(k)}; };
-  auto bmm2 = [&](MatRef o, BmmTerm t0, BmmTerm t1, int nterms, int m, int n,
-                  int mask, float alpha, int accumulate) {
+  auto bmm3 = [&](MatRef o, BmmTerm t0, BmmTerm t1, BmmTerm t2, int nterms,
+                  int m, int n, int mask, float alpha, int accumulate) {
     BmmOp op{};
     op.out = o;
     op.term[0] = t0;
     op.term[1] = t1;
+    op.term[2] = t2;
     op.nterms = nterms;
     op.m = m;
     op.n = n;
@@ -857,10 +876,14 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
     op.mask = mask;
     op.alpha = alpha;
     op.accumulate = accumulate;
-    const int kd = max(t0.kd, nterms > 1 ? t1.kd : 0);
+    const int kd = max(t0.kd, max(nterms > 1 ? t1.kd : 0, nterms > 2 ? t2.kd : 0));
     const size_t smem = 4 * (size_t)kd * ((op.md + 4) + (op.nd + 4));
     return launch_bmm(op, C, smem, grid, stream, cu, co, f.n_seqs, f.T, H, dk,
                       dv);
+  };
+  auto bmm2 = [&](MatRef o, BmmTerm t0, BmmTerm t1, int nterms, int m, int n,
+                  int mask, float alpha, int accumulate) {
+    return bmm3(o, t0, t1, t1, nterms, m, n, mask, alpha, accumulate);
   };
   auto bmm = [&](MatRef o, MatRef x, MatRef y, int n, int k, int mask,
                  float alpha, int accumulate) {
@@ -879,19 +902,14 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
                 kMaskNone, 1.f, 0))
   }
   {
-    const int tile = chain_tile(dv), tp = tile + 1;
+    constexpr int tp = kChainTile + 1;
     const size_t smc = 4 * ((size_t)dk * tp + 2 * (size_t)C * (dk + 1) +
                             (size_t)C * tp + dk);
-    const dim3 cgrid(f.n_seqs, H, dv / tile);
-    if (tile == 64) {
-      if ((e = set_smem(chain_kernel<64>, smc)) != cudaSuccess) return e;
-      chain_kernel<64><<<cgrid, kThreads, smc, stream>>>(
-          w, a.d_final_state, a.d_initial_state, cu, f.n_seqs, f.T, H, dk, dv, C);
-    } else {
-      if ((e = set_smem(chain_kernel<32>, smc)) != cudaSuccess) return e;
-      chain_kernel<32><<<cgrid, kThreads, smc, stream>>>(
-          w, a.d_final_state, a.d_initial_state, cu, f.n_seqs, f.T, H, dk, dv, C);
-    }
+    if ((e = set_smem(chain_kernel<kChainTile>, smc)) != cudaSuccess) return e;
+    chain_kernel<kChainTile><<<dim3(f.n_seqs, H, dv / kChainTile), kThreads,
+                               smc, stream>>>(w, a.d_final_state,
+                                              a.d_initial_state, cu, f.n_seqs,
+                                              f.T, H, dk, dv, C);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if (nch == 0) return cudaSuccess;
@@ -903,10 +921,6 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
   KDA_BMM(bmm2(tok(w.dqt, dk), term(tok(w.do32, dv), stt(S0, 1), kDimDv),
                term(sq(w.dp), tok(w.kb, dk), kDimL), 2, kDimL, kDimDk,
                kMaskNone, 1.f, 0))
-  // dKb = Delta G^T + dP^T Qt  (+ dA^T b Kt below)
-  KDA_BMM(bmm2(tok(w.dkb, dk), term(tok(De, dv), stt(w.gst, 1), kDimDv),
-               term(sq(w.dp, 1), tok(w.qt, dk), kDimL), 2, kDimL, kDimDk,
-               kMaskNone, 1.f, 0))
   // dW = -dDelta S_0^T
   KDA_BMM(bmm(tok(w.dw, dk), tok(w.dd, dv), stt(S0, 1), kDimDk, kDimDv,
               kMaskNone, -1.f, 0))
@@ -914,9 +928,7 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
   KDA_BMM(bmm2(sq(w.dtm), term(tok(w.dw, dk), tok(w.bkt, dk, 1), kDimDk),
                term(tok(w.dd, dv), tok(w.bv, dv, 1), kDimDv), 2, kDimL, kDimL,
                kMaskNone, 1.f, 0))
-  // Tm^T dW, Tm^T dDelta, Tm^T dTm
-  KDA_BMM(bmm(tok(w.dbk, dk), sq(w.tm, 1), tok(w.dw, dk), kDimDk, kDimL,
-              kMaskNone, 1.f, 0))
+  // Tm^T dDelta and Tm^T dTm
   KDA_BMM(bmm(tok(w.dbv, dv), sq(w.tm, 1), tok(w.dd, dv), kDimDv, kDimL,
               kMaskNone, 1.f, 0))
   KDA_BMM(bmm(sq(w.tmp), sq(w.tm, 1), sq(w.dtm), kDimL, kDimL, kMaskNone, 1.f,
@@ -924,11 +936,15 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
   // dA = strictly_lower(-(Tm^T dTm) Tm^T)
   KDA_BMM(bmm(sq(w.da), sq(w.tmp), sq(w.tm, 1), kDimL, kDimL, kMaskStrictLower,
               -1.f, 0))
-  // dA Kb, and dKb += dA^T (b Kt)
-  KDA_BMM(bmm(tok(w.y1, dk), sq(w.da), tok(w.kb, dk), kDimDk, kDimL, kMaskNone,
-              1.f, 0))
-  KDA_BMM(bmm(tok(w.dkb, dk), sq(w.da, 1), tok(w.bkt, dk), kDimDk, kDimL,
-              kMaskNone, 1.f, 1))
+  // dKt / b = Tm^T dW + dA Kb
+  KDA_BMM(bmm2(tok(w.dbk, dk), term(sq(w.tm, 1), tok(w.dw, dk), kDimL),
+               term(sq(w.da), tok(w.kb, dk), kDimL), 2, kDimL, kDimDk,
+               kMaskNone, 1.f, 0))
+  // dKb = Delta G^T + dP^T Qt + dA^T (b Kt)
+  KDA_BMM(bmm3(tok(w.dkb, dk), term(tok(De, dv), stt(w.gst, 1), kDimDv),
+               term(sq(w.dp, 1), tok(w.qt, dk), kDimL),
+               term(sq(w.da, 1), tok(w.bkt, dk), kDimL), 3, kDimL, kDimDk,
+               kMaskNone, 1.f, 0))
 #undef KDA_BMM
   const size_t smf = 4 * (size_t)C * dk;
   if ((e = set_smem(final_kernel<IO>, smf)) != cudaSuccess) return e;
@@ -939,7 +955,7 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-constexpr int kBmmOps = 13;
+constexpr int kBmmOps = 11;
 
 }  // namespace
 

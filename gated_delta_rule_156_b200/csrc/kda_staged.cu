@@ -256,6 +256,7 @@ __global__ void __launch_bounds__(kThreads)
     for (int a = 0; a < 4; ++a)
 #pragma unroll
       for (int b = 0; b < 8; ++b) aw[a][b] = au[a][b] = 0.f;
+#pragma unroll 2
     for (int i = 0; i < C; ++i) {
       float t[4], kt[8], vv[8];
 #pragma unroll
@@ -383,6 +384,7 @@ __global__ void __launch_bounds__(kThreads)
       for (int a = 0; a < 2; ++a)
 #pragma unroll
         for (int b = 0; b < NB; ++b) acc[a][b] = 0.f;
+      #pragma unroll 4
       for (int c = 0; c < dk; ++c) {
         float sv[NB];
 #pragma unroll
@@ -416,6 +418,7 @@ __global__ void __launch_bounds__(kThreads)
       for (int a = 0; a < 4; ++a)
 #pragma unroll
         for (int b = 0; b < NB; ++b) acc[a][b] = 0.f;
+      #pragma unroll 4
       for (int r = 0; r < L; ++r) {
         float dvv[NB];
 #pragma unroll

@@ -190,8 +190,8 @@ def test_backward_validation(lib):
 def test_backward_plan(lib):
     import torch
     kern, ws = K.chunk_bwd_plan(2, 8192, 32, 128, 128, 64, torch.bfloat16)
-    # cumsum, prep, the state pass, 2 + 11 products, the chain, final
-    assert kern == 18 and ws > 0
+    # cumsum, prep, the state pass, 2 + 9 products, the chain, final
+    assert kern == 16 and ws > 0
     kern_p, _ = K.chunk_bwd_plan(1, 300, 2, 64, 64, 32, torch.float32,
                                  packed=True, n_seqs=3)
-    assert kern_p == 19
+    assert kern_p == 17
