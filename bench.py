@@ -553,9 +553,10 @@ def run_only(args, dev, stream):
     """Warm-up plus `steps` launches of one workload, for a profiler to
     capture; prints the mean launch time and nothing else."""
     from gated_delta_rule_156_b200 import kda as K
+    over = {"T": args.seq_len} if args.seq_len else {}
     if args.only == "prefill":
-        cfg = W.CONFIGS[PREFILL_CFG]
-        d = W.make(PREFILL_CFG, device=dev)
+        cfg = dict(W.CONFIGS[PREFILL_CFG], **over)
+        d = W.make(PREFILL_CFG, device=dev, **over)
         out = torch.empty((cfg["B"], cfg["T"], cfg["H"], cfg["dv"]),
                           dtype=torch.bfloat16, device=dev)
         fin = torch.empty((cfg["B"], cfg["H"], cfg["dk"], cfg["dv"]),
@@ -566,8 +567,8 @@ def run_only(args, dev, stream):
                         None, None, chunk=cfg["chunk"], out=out,
                         final_state=fin)
     elif args.only == "backward":
-        cfg = W.CONFIGS[PREFILL_CFG]
-        d = W.make(PREFILL_CFG, device=dev)
+        cfg = dict(W.CONFIGS[PREFILL_CFG], **over)
+        d = W.make(PREFILL_CFG, device=dev, **over)
         gdo = torch.randn(d["v"].shape, generator=torch.Generator(
             device=dev).manual_seed(77), device=dev).bfloat16()
 
@@ -631,6 +632,10 @@ def main():
                     default=None,
                     help="profiling aid: run one workload's warm-up and timed "
                          "launches only (no e2e, no CPU baseline, no JSON line)")
+    ap.add_argument("--seq-len", type=int, default=None,
+                    help="with --only prefill/backward: tokens per sequence "
+                         "(default: the prefill workload's 8192), for a "
+                         "smaller profiler capture")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
