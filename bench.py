@@ -409,6 +409,49 @@ def run_kda(args, world, rank, local):
     }
     del d3, out3, fin3
 
+    # ---- one long sequence (131072 tokens, d = 128, bf16, with a start
+    # state): the plain prefill's serial chain of 2048 chunks against the
+    # sequence split into segments joined by a scan, with few heads (H = 8,
+    # most SMs idle) and with H = 32 (the GPU already full) ----------------
+    prefill_split = {}
+    for Hs, nseg in ((8, 4), (32, 2)):
+        ds = W.draw((1, 131072), Hs, 128, 128, io="bf16", scale_q=True,
+                    n_states=1, device=dev, seed=1234 + Hs + 97 * rank)
+        outs = torch.empty_like(ds["v"])
+        fins = torch.empty_like(ds["initial_state"])
+
+        def plain(_i):
+            K.chunk_fwd(ds["q"], ds["k"], ds["v"], ds["log_alpha"], ds["beta"],
+                        ds["initial_state"], None, chunk=C, out=outs,
+                        final_state=fins)
+
+        def split(_i):
+            K.chunk_fwd_split(ds["q"], ds["k"], ds["v"], ds["log_alpha"],
+                              ds["beta"], ds["initial_state"],
+                              n_segments=nseg, chunk=C, out=outs,
+                              final_state=fins)
+
+        for fn in (plain, split):
+            fn(0)
+            fn(1)
+        torch.cuda.synchronize()
+        barrier(world)
+        sp_steps = max(2, min(args.steps, 3))
+        pms, _ = timed(plain, sp_steps, stream)
+        sms, _ = timed(split, sp_steps, stream)
+        barrier(world)
+        pms = max_over_ranks(pms, world) / sp_steps
+        sms = max_over_ranks(sms, world) / sp_steps
+        prefill_split[f"H{Hs}"] = {
+            "value": world * 131072 / (sms * 1e-3), "unit": "tokens/s",
+            "ms_per_step": sms, "steps": sp_steps, "segments": nseg,
+            "unsplit_ms_per_step": pms, "speedup_vs_unsplit": pms / sms,
+            "workload": f"kda_chunk_fwd_split, one sequence of 131072 tokens, "
+                        f"H={Hs} d=128 bf16, start state in, final state out; "
+                        "unsplit = kda_chunk_fwd on the same inputs",
+        }
+        del ds, outs, fins
+
     # ---- backward pass of the prefill workload: every input's gradient for
     # a random output gradient (fp32 arithmetic, chunkwise) ----------------
     gdo = torch.randn(d["v"].shape, generator=torch.Generator(device=dev)
@@ -535,6 +578,7 @@ def run_kda(args, world, rank, local):
             },
             "prefill_head_gate": head_gate,
             "prefill_packed_long": packed_long,
+            "prefill_split": prefill_split,
             "backward": backward_line,
             "prefill_fused_prologue": fused_prologue,
             "e2e": {"value": e2e_value, "unit": "tokens/s",

@@ -211,6 +211,57 @@ kda_status kda_chunk_fwd(const kda_shape* shape, const void* q, const void* k,
   return run_with_workspace(kda::staged_workspace_bytes(a), stream, false, a);
 }
 
+kda_status kda_chunk_fwd_split(const kda_shape* shape, int gate, const void* q,
+                               const void* k, const void* v,
+                               const float* gate_tensor, const float* beta,
+                               const float* initial_state, void* out,
+                               float* final_state, int n_segments,
+                               cudaStream_t stream) {
+  if (!shape || shape->B != 1 || n_segments < 1 || n_segments > 64)
+    return KDA_ERR_INVALID_ARG;
+  kda::ChunkArgs a{};
+  const kda_status st = validate_chunk(shape, q, k, v, gate_tensor, beta,
+                                       initial_state, nullptr, out,
+                                       final_state, &a, gate);
+  if (st != KDA_OK) return st;
+  const kda::SplitGeom g = kda::split_geometry(a, n_segments);
+  const size_t bytes = kda::split_workspace_bytes(a, g);
+  void* ws = nullptr;
+  cudaError_t e;
+  if (bytes) {
+    keep_pool_memory();
+    if ((e = cudaMallocAsync(&ws, bytes, stream)) != cudaSuccess)
+      return cuda_fail(e);
+  }
+  e = kda::launch_split(a, g, ws, stream);
+  if (ws) {
+    const cudaError_t f = cudaFreeAsync(ws, stream);
+    if (e == cudaSuccess) e = f;
+  }
+  return e == cudaSuccess ? KDA_OK : cuda_fail(e);
+}
+
+kda_status kda_chunk_fwd_split_plan(const kda_shape* shape, int gate,
+                                    int n_segments, int* segments, int* kernels,
+                                    size_t* workspace_bytes) {
+  if (!shape || shape->B != 1 || n_segments < 1 || n_segments > 64)
+    return KDA_ERR_INVALID_ARG;
+  if (gate != kda::kGateChannel && gate != kda::kGateHead &&
+      gate != kda::kGateNone)
+    return KDA_ERR_INVALID_ARG;
+  int n_seqs = 0;
+  const kda_status st = validate_chunk_shape(shape, false, &n_seqs);
+  if (st != KDA_OK) return st;
+  kda::ChunkArgs a{};
+  fill_args(shape, n_seqs, &a);
+  a.gate = gate;
+  const kda::SplitGeom g = kda::split_geometry(a, n_segments);
+  if (segments) *segments = g.k;
+  if (kernels) *kernels = kda::split_kernel_count(a, g);
+  if (workspace_bytes) *workspace_bytes = kda::split_workspace_bytes(a, g);
+  return KDA_OK;
+}
+
 kda_status kda_chunk_fwd_staged(const kda_shape* shape, const void* q,
                                 const void* k, const void* v,
                                 const float* log_alpha, const float* beta,

@@ -85,6 +85,21 @@ cudaError_t launch_staged_part(const ChunkArgs& a, void* workspace,
                                StagedView* view, bool state_pass,
                                cudaStream_t stream);
 
+// Sequence-split prefill of one long sequence (kda_split.cu): k segments of
+// Ls tokens (a multiple of the chunk; the last one takes the rest) evaluated
+// side by side and joined by a scan of their state transitions.  k = 1 is
+// the plain chunkwise forward.  `a` is a dense single-sequence request
+// (n_seqs = 1, no cu_seqlens).
+struct SplitGeom {
+  int Ls;
+  int k;
+};
+SplitGeom split_geometry(const ChunkArgs& a, int n_segments);
+size_t split_workspace_bytes(const ChunkArgs& a, const SplitGeom& g);
+int split_kernel_count(const ChunkArgs& a, const SplitGeom& g);
+cudaError_t launch_split(const ChunkArgs& a, const SplitGeom& g, void* workspace,
+                         cudaStream_t stream);
+
 // Chunkwise backward pass (kda_backward.cu): the gradients of
 // L = <d_out, out> + <d_final_state, final_state> with respect to q, k, v,
 // log(alpha), beta and the initial state, all arithmetic in fp32.

@@ -1,0 +1,407 @@
+// Sequence-split prefill: one long sequence evaluated as n segments side by
+// side, joined by a scan of the segments' state transitions.
+//
+// The recurrence's state update is affine in the state ("Kimi Delta
+// Attention", akshathtiwari.co.in, the delta-rule passage: S_t = (I - beta_t
+// k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T).  Inside a segment that
+// starts from S_in, with M_t the product of the token transitions from the
+// segment start to token t and |0 marking the evaluation from a zero state:
+//     S_t = M_t S_in + S_t|0,        o_t = o_t|0 + S_in^T (M_t^T q_t).
+// M_t is itself the state of the same recurrence run with v = 0 from the
+// identity, and M_t^T q_t that run's output.  So:
+//   (1) value run: every segment at once as a packed batch, segment 0 from the
+//       true initial state, the others from zero;
+//   (2) transition run (on a second stream, concurrently): segments 1..n-1
+//       with v = 0, d_v = d_k and the identity as start state, giving
+//       X_t = M_t^T q_t and each segment's transition M_end;
+//   (3) scan: S_in(1) = S_end(0); S_in(j+1) = M_end(j) S_in(j) + S_end|0(j);
+//       the last step gives the final state;
+//   (4) correction: o_t += S_in(j)^T X_t for the tokens of segments 1..n-1.
+// Steps (1) and (2) run the library's own prefill kernels (fused or
+// four-stage, as kda_chunk_fwd would pick for their shapes); (3) and (4) are
+// the fp32 kernels below.
+#include <mutex>
+
+#include "kda_common.cuh"
+#include "kda_internal.h"
+
+namespace kda {
+
+namespace {
+
+constexpr int kThreads = 256;
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct SplitWs {
+  int32_t* cu_val;   // [k + 1] segment offsets of the value run
+  int32_t* cu_tr;    // [k] offsets of the transition run (segments 1..k-1)
+  float* init_val;   // [k, H, dk, dv] start states of the value run
+  float* end_val;    // [k, H, dk, dv] its end states
+  float* ident;      // [k - 1, H, dk, dk] identity start states
+  float* trans;      // [k - 1, H, dk, dk] segment transitions M_end
+  float* s_in;       // [k - 1, H, dk, dv] entry states of segments 1..k-1
+  void* vzero;       // [T - Ls, H, dk] io dtype, zeros
+  void* x;           // [T - Ls, H, dk] io dtype, M_t^T q_t
+  void* ws_val;      // the value run's own workspace
+  void* ws_tr;       // the transition run's own workspace
+};
+
+ChunkArgs value_args(const ChunkArgs& a, const SplitGeom& g, const SplitWs& w) {
+  ChunkArgs v = a;
+  v.cu_seqlens = w.cu_val;
+  v.n_seqs = g.k;
+  v.initial_state = w.init_val;
+  v.final_state = w.end_val;
+  return v;
+}
+
+ChunkArgs trans_args(const ChunkArgs& a, const SplitGeom& g, const SplitWs& w) {
+  ChunkArgs t = a;
+  const size_t esz = a.bf16 ? 2 : 4;
+  const size_t off = (size_t)g.Ls * a.H;  // token-heads before segment 1
+  const char* q = static_cast<const char*>(a.q);
+  const char* k = static_cast<const char*>(a.k);
+  t.q = q ? q + off * a.dk * esz : nullptr;
+  t.k = k ? k + off * a.dk * esz : nullptr;
+  t.v = w.vzero;
+  t.log_alpha = a.log_alpha
+                    ? a.log_alpha + off * (a.gate == kGateChannel ? a.dk : 1)
+                    : nullptr;
+  t.beta = a.beta ? a.beta + off : nullptr;
+  t.cu_seqlens = w.cu_tr;
+  t.n_seqs = g.k - 1;
+  t.T = a.T - g.Ls;
+  t.dv = a.dk;
+  t.initial_state = w.ident;
+  t.out = w.x;
+  t.final_state = w.trans;
+  return t;
+}
+
+size_t run_workspace(const ChunkArgs& a) {
+  return fused_supported(a) ? fused_workspace_bytes(a)
+                            : staged_workspace_bytes(a);
+}
+
+int run_kernels(const ChunkArgs& a) {
+  return fused_supported(a) ? fused_kernel_count(a) : staged_kernel_count(a);
+}
+
+cudaError_t run_forward(const ChunkArgs& a, void* ws, cudaStream_t s) {
+  return fused_supported(a) ? launch_fused(a, ws, s) : launch_staged(a, ws, s);
+}
+
+// Sizes and kernel counts depend on whether cu_seqlens is present, not on its
+// contents: while planning (no workspace yet) the offsets point at a tag.
+const int32_t kPlanTag = 0;
+SplitWs tagged(SplitWs w) {
+  if (!w.cu_val) w.cu_val = const_cast<int32_t*>(&kPlanTag);
+  if (!w.cu_tr) w.cu_tr = const_cast<int32_t*>(&kPlanTag);
+  return w;
+}
+
+SplitWs carve_split(const ChunkArgs& a, const SplitGeom& g, void* base,
+                    size_t* total) {
+  const size_t esz = a.bf16 ? 2 : 4;
+  const size_t H = a.H, dk = a.dk, dv = a.dv, k = g.k;
+  const size_t rest = (size_t)(a.T - g.Ls) * H * dk;  // token-head-channels
+  size_t off = 0;
+  char* p = static_cast<char*>(base);
+  auto take = [&](size_t bytes) {
+    char* r = p ? p + off : nullptr;
+    off = align256(off + bytes);
+    return static_cast<void*>(r);
+  };
+  SplitWs w{};
+  w.cu_val = static_cast<int32_t*>(take(4 * (k + 1)));
+  w.cu_tr = static_cast<int32_t*>(take(4 * k));
+  w.init_val = static_cast<float*>(take(4 * k * H * dk * dv));
+  w.end_val = static_cast<float*>(take(4 * k * H * dk * dv));
+  w.ident = static_cast<float*>(take(4 * (k - 1) * H * dk * dk));
+  w.trans = static_cast<float*>(take(4 * (k - 1) * H * dk * dk));
+  w.s_in = static_cast<float*>(take(4 * (k - 1) * H * dk * dv));
+  w.vzero = take(esz * rest);
+  w.x = take(esz * rest);
+  // the two runs' own workspaces: sized for the packed layout they run in
+  const SplitWs probe = tagged(w);
+  w.ws_val = take(run_workspace(value_args(a, g, probe)));
+  w.ws_tr = take(run_workspace(trans_args(a, g, probe)));
+  if (total) *total = off;
+  return w;
+}
+
+// Offsets, start states and the zero values of both runs, in one grid-stride
+// pass: cu_val = {0, Ls, 2 Ls, .., T}; cu_tr the same shifted by Ls;
+// init_val = {S_0 or 0, 0, ..}; ident = identity per (segment, head); vzero
+// = 0.
+__global__ void __launch_bounds__(kThreads)
+    split_setup_kernel(SplitWs w, const float* __restrict__ s0, int T, int Ls,
+                       int k, int H, int dk, int dv, size_t vzero_words) {
+  const size_t tid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  if (tid <= (size_t)k) w.cu_val[tid] = min((int)tid * Ls, T);
+  if (tid < (size_t)k) w.cu_tr[tid] = min((int)tid * Ls, T - Ls);
+  const size_t nstate = (size_t)H * dk * dv;
+  for (size_t i = tid; i < (size_t)k * nstate; i += stride)
+    w.init_val[i] = (i < nstate && s0) ? s0[i] : 0.f;
+  const size_t nid = (size_t)(k - 1) * H * dk * dk;
+  for (size_t i = tid; i < nid; i += stride) {
+    const size_t rc = i % ((size_t)dk * dk);
+    w.ident[i] = (rc / dk == rc % dk) ? 1.f : 0.f;
+  }
+  uint4* z = static_cast<uint4*>(w.vzero);
+  for (size_t i = tid; i < vzero_words; i += stride) z[i] = make_uint4(0, 0, 0, 0);
+}
+
+// (3) Per (head, 32-column tile of d_v): S = S_end(0); for j = 1 .. k-1:
+// S_in(j) = S, S <- M_end(j) S + S_end|0(j); the final S is the final state.
+// M_end(j) is staged whole in shared memory (rows padded to d_k + 1), the
+// tile of S beside it; thread (g8, j8) owns rows g8 + 32 a, columns j8 + 8 b.
+constexpr int kScanTile = 32, kScanTp = kScanTile + 1;
+
+__global__ void __launch_bounds__(kThreads)
+    split_scan_kernel(SplitWs w, float* __restrict__ final_state, int k, int H,
+                      int dk, int dv) {
+  const int h = blockIdx.x, j0 = blockIdx.y * kScanTile, tid = threadIdx.x;
+  const int dkp = dk + 1, NA = dk / 32, g8 = tid >> 3, j8 = tid & 7;
+  extern __shared__ float sm[];
+  float* S = sm;              // [dk][kScanTp]
+  float* M = S + dk * kScanTp;  // [dk][dkp]
+  const size_t nst = (size_t)H * dk * dv;
+  for (int idx = tid; idx < dk * kScanTile; idx += kThreads) {
+    const int c = idx / kScanTile, jj = idx % kScanTile;
+    S[c * kScanTp + jj] = w.end_val[(size_t)h * dk * dv + (size_t)c * dv + j0 + jj];
+  }
+  for (int j = 1; j < k; ++j) {
+    const float* Mj = w.trans + ((size_t)(j - 1) * H + h) * dk * dk;
+    const float* Ej = w.end_val + (size_t)j * nst + (size_t)h * dk * dv;
+    float* Sin = w.s_in + (size_t)(j - 1) * nst + (size_t)h * dk * dv;
+    for (int idx = tid; idx < dk * dk; idx += kThreads)
+      M[(idx / dk) * dkp + idx % dk] = Mj[idx];
+    __syncthreads();
+    for (int idx = tid; idx < dk * kScanTile; idx += kThreads) {
+      const int c = idx / kScanTile, jj = idx % kScanTile;
+      Sin[(size_t)c * dv + j0 + jj] = S[c * kScanTp + jj];
+    }
+    float acc[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+#pragma unroll 4
+    for (int c = 0; c < dk; ++c) {
+      float sv[4];
+#pragma unroll
+      for (int b = 0; b < 4; ++b) sv[b] = S[c * kScanTp + j8 + 8 * b];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        if (a < NA) {
+          const float m = M[(g8 + 32 * a) * dkp + c];
+#pragma unroll
+          for (int b = 0; b < 4; ++b) acc[a][b] += m * sv[b];
+        }
+      }
+    }
+    __syncthreads();  // every read of S and M is done
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      if (a < NA) {
+        const int r = g8 + 32 * a;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          const int jj = j8 + 8 * b;
+          S[r * kScanTp + jj] = acc[a][b] + Ej[(size_t)r * dv + j0 + jj];
+        }
+      }
+    }
+    __syncthreads();
+  }
+  for (int idx = tid; idx < dk * kScanTile; idx += kThreads) {
+    const int c = idx / kScanTile, jj = idx % kScanTile;
+    final_state[(size_t)h * dk * dv + (size_t)c * dv + j0 + jj] =
+        S[c * kScanTp + jj];
+  }
+}
+
+// (4) Per (chunk of segments 1..k-1, head): out[t] += S_in(j)^T X[t] for its
+// C tokens (a chunk never straddles segments, whose length is a multiple of
+// C).  X rows and S_in(j) are staged in shared memory; thread (ti, tj) owns
+// rows ti + 16 a and columns tj + 16 b.
+template <typename IO>
+__global__ void __launch_bounds__(kThreads)
+    split_fix_kernel(SplitWs w, IO* __restrict__ out, int T, int Ls, int k,
+                     int H, int dk, int dv, int C) {
+  const int t0 = Ls + blockIdx.x * C, h = blockIdx.y, tid = threadIdx.x;
+  const int L = min(C, T - t0);
+  const int j = min(t0 / Ls, k - 1);
+  const int dkp = dk + 1;
+  extern __shared__ float sm[];
+  float* X = sm;             // [C][dkp]
+  float* S = X + C * dkp;    // [dk][dv]
+  const IO* x = static_cast<const IO*>(w.x);
+  for (int idx = tid; idx < C * dk; idx += kThreads) {
+    const int r = idx / dk, c = idx % dk;
+    X[r * dkp + c] =
+        r < L ? to_f32(x[((size_t)(t0 - Ls + r) * H + h) * dk + c]) : 0.f;
+  }
+  const float* Sin = w.s_in + ((size_t)(j - 1) * H + h) * dk * dv;
+  for (int idx = tid; idx < dk * dv; idx += kThreads) S[idx] = Sin[idx];
+  __syncthreads();
+  const int ti = tid >> 4, tj = tid & 15, nr = C / 16, nc = dv / 16;
+  float acc[4][8];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 8; ++b) acc[a][b] = 0.f;
+#pragma unroll 2
+  for (int c = 0; c < dk; ++c) {
+    float xv[4], sv[8];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) xv[a] = a < nr ? X[(ti + 16 * a) * dkp + c] : 0.f;
+#pragma unroll
+    for (int b = 0; b < 8; ++b) sv[b] = b < nc ? S[c * dv + tj + 16 * b] : 0.f;
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 8; ++b) acc[a][b] += xv[a] * sv[b];
+  }
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    const int r = ti + 16 * a;
+    if (a < nr && r < L) {
+      IO* o = out + ((size_t)(t0 + r) * H + h) * dv;
+#pragma unroll
+      for (int b = 0; b < 8; ++b) {
+        if (b < nc) {
+          const int jj = tj + 16 * b;
+          o[jj] = from_f32<IO>(to_f32(o[jj]) + acc[a][b]);
+        }
+      }
+    }
+  }
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, size_t bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)bytes);
+}
+
+// A non-blocking stream per device for the transition run, created on first
+// use and kept for the life of the process.
+cudaError_t side_stream(cudaStream_t* out) {
+  static std::mutex mu;
+  static cudaStream_t streams[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!streams[dev]) {
+    e = cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking);
+    if (e != cudaSuccess) {
+      streams[dev] = nullptr;
+      return e;
+    }
+  }
+  *out = streams[dev];
+  return cudaSuccess;
+}
+
+template <typename IO>
+cudaError_t run_split(const ChunkArgs& a, const SplitGeom& g, void* workspace,
+                      cudaStream_t stream) {
+  SplitWs w = carve_split(a, g, workspace, nullptr);
+  const size_t esz = a.bf16 ? 2 : 4;
+  const size_t vz_words = esz * (size_t)(a.T - g.Ls) * a.H * a.dk / 16;
+  cudaError_t e;
+  split_setup_kernel<<<4 * 148, kThreads, 0, stream>>>(
+      w, a.initial_state, a.T, g.Ls, g.k, a.H, a.dk, a.dv, vz_words);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+  // (1) on `stream`, (2) on the side stream, joined by events
+  cudaStream_t side = nullptr;
+  if ((e = side_stream(&side)) != cudaSuccess) return e;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  if ((e = cudaEventCreateWithFlags(&fork, cudaEventDisableTiming)) != cudaSuccess)
+    return e;
+  if ((e = cudaEventCreateWithFlags(&join, cudaEventDisableTiming)) != cudaSuccess) {
+    cudaEventDestroy(fork);
+    return e;
+  }
+  auto done = [&](cudaError_t r) {
+    cudaEventDestroy(fork);
+    cudaEventDestroy(join);
+    return r;
+  };
+  if ((e = cudaEventRecord(fork, stream)) != cudaSuccess) return done(e);
+  if ((e = cudaStreamWaitEvent(side, fork, 0)) != cudaSuccess) return done(e);
+  // whatever fails below, `stream` waits for the side stream before the
+  // caller can release the workspace
+  const cudaError_t e_tr = run_forward(trans_args(a, g, w), w.ws_tr, side);
+  const cudaError_t e_rec = cudaEventRecord(join, side);
+  const cudaError_t e_val =
+      e_tr == cudaSuccess ? run_forward(value_args(a, g, w), w.ws_val, stream)
+                          : cudaSuccess;
+  const cudaError_t e_wait =
+      e_rec == cudaSuccess ? cudaStreamWaitEvent(stream, join, 0) : e_rec;
+  for (cudaError_t r : {e_tr, e_rec, e_val, e_wait})
+    if (r != cudaSuccess) return done(r);
+  done(cudaSuccess);
+
+  // (3) scan, (4) correction
+  const int dk = a.dk, dv = a.dv, H = a.H, C = a.chunk;
+  const size_t sms = 4 * ((size_t)dk * kScanTp + (size_t)dk * (dk + 1));
+  if ((e = set_smem(split_scan_kernel, sms)) != cudaSuccess) return e;
+  split_scan_kernel<<<dim3(H, dv / kScanTile), kThreads, sms, stream>>>(
+      w, a.final_state, g.k, H, dk, dv);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const size_t smf = 4 * ((size_t)C * (dk + 1) + (size_t)dk * dv);
+  if ((e = set_smem(split_fix_kernel<IO>, smf)) != cudaSuccess) return e;
+  const unsigned nblk = (unsigned)((a.T - g.Ls + C - 1) / C);
+  split_fix_kernel<IO><<<dim3(nblk, H), kThreads, smf, stream>>>(
+      w, static_cast<IO*>(a.out), a.T, g.Ls, g.k, H, dk, dv, C);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+SplitGeom split_geometry(const ChunkArgs& a, int n_segments) {
+  SplitGeom g{};
+  const int C = a.chunk;
+  const int nch = (a.T + C - 1) / C;
+  const int n = n_segments < nch ? n_segments : nch;
+  if (n <= 1) {
+    g.k = 1;
+    g.Ls = a.T;
+    return g;
+  }
+  g.Ls = ((nch + n - 1) / n) * C;
+  g.k = (a.T + g.Ls - 1) / g.Ls;
+  return g;
+}
+
+size_t split_workspace_bytes(const ChunkArgs& a, const SplitGeom& g) {
+  if (g.k <= 1) return run_workspace(a);
+  size_t total = 0;
+  carve_split(a, g, nullptr, &total);
+  return total;
+}
+
+int split_kernel_count(const ChunkArgs& a, const SplitGeom& g) {
+  if (g.k <= 1) return run_kernels(a);
+  const SplitWs w = tagged(SplitWs{});
+  // setup, the two runs, scan, correction
+  return 1 + run_kernels(value_args(a, g, w)) + run_kernels(trans_args(a, g, w)) +
+         2;
+}
+
+cudaError_t launch_split(const ChunkArgs& a, const SplitGeom& g, void* workspace,
+                         cudaStream_t stream) {
+  if (g.k <= 1) return run_forward(a, workspace, stream);
+  return a.bf16 ? run_split<__nv_bfloat16>(a, g, workspace, stream)
+                : run_split<float>(a, g, workspace, stream);
+}
+
+}  // namespace kda

@@ -24,7 +24,8 @@ EXPORTS = ("kda_chunk_fwd", "kda_chunk_fwd_staged", "kda_recurrent_step",
            "kda_chunk_fwd_staged_noalloc", "kda_chunk_fwd_gated",
            "kda_recurrent_step_gated", "kda_chunk_fwd_ex",
            "kda_recurrent_step_ex", "kda_selftest_timeout", "kda_chunk_bwd",
-           "kda_chunk_bwd_plan")
+           "kda_chunk_bwd_plan", "kda_chunk_fwd_split",
+           "kda_chunk_fwd_split_plan")
 GATES = {"channel": 0, "head": 1, "none": 2}
 
 
@@ -105,6 +106,15 @@ def library():
                                            fp, fp, fp, vp, vp]
         lib.kda_chunk_fwd_plan.restype = ctypes.c_int
         lib.kda_chunk_fwd_plan.argtypes = [
+            ctypes.POINTER(KdaShape), ctypes.c_int, ctypes.c_int,
+            ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int),
+            ctypes.POINTER(ctypes.c_size_t)]
+        lib.kda_chunk_fwd_split.restype = ctypes.c_int
+        lib.kda_chunk_fwd_split.argtypes = [
+            ctypes.POINTER(KdaShape), ctypes.c_int, vp, vp, vp, fp, fp, fp, vp,
+            fp, ctypes.c_int, vp]
+        lib.kda_chunk_fwd_split_plan.restype = ctypes.c_int
+        lib.kda_chunk_fwd_split_plan.argtypes = [
             ctypes.POINTER(KdaShape), ctypes.c_int, ctypes.c_int,
             ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int),
             ctypes.POINTER(ctypes.c_size_t)]
@@ -215,6 +225,51 @@ def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
     if st != KDA_OK:
         raise KdaError(st, "kda_chunk_fwd_staged" if staged else "kda_chunk_fwd")
     return out, final_state
+
+
+def chunk_fwd_split(q, k, v, log_alpha, beta, initial_state=None,
+                    n_segments=2, chunk=64, out=None, final_state=None,
+                    gate="channel", stream=None):
+    """Prefill of one long sequence as ``n_segments`` segments evaluated side
+    by side and joined by a scan of their state transitions
+    (kda_chunk_fwd_split).  Shapes as chunk_fwd with B == 1 and no
+    cu_seqlens.  Returns (out, final_state)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if final_state is None:
+        final_state = torch.empty((B, H, dk, dv), dtype=torch.float32,
+                                  device=q.device)
+    for name, t, dt in (("q", q, None), ("k", k, q.dtype), ("v", v, q.dtype),
+                        ("log_alpha", log_alpha, torch.float32),
+                        ("beta", beta, torch.float32),
+                        ("initial_state", initial_state, torch.float32),
+                        ("out", out, q.dtype),
+                        ("final_state", final_state, torch.float32)):
+        _check_dev(name, t, dt)
+    shape = KdaShape(B, T, H, dk, dv, chunk, 0, _io(q))
+    st = library().kda_chunk_fwd_split(
+        ctypes.byref(shape), GATES[gate], _ptr(q), _ptr(k), _ptr(v),
+        _ptr(log_alpha), _ptr(beta), _ptr(initial_state), _ptr(out),
+        _ptr(final_state), int(n_segments), _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_chunk_fwd_split")
+    return out, final_state
+
+
+def chunk_fwd_split_plan(T, H, dk, dv, chunk, dtype, n_segments,
+                         gate="channel"):
+    """(segments, kernels, workspace_bytes) of a chunk_fwd_split call."""
+    io = KDA_BF16 if dtype == torch.bfloat16 else KDA_F32
+    shape = KdaShape(1, T, H, dk, dv, chunk, 0, io)
+    seg, kern, ws = ctypes.c_int(), ctypes.c_int(), ctypes.c_size_t()
+    st = library().kda_chunk_fwd_split_plan(
+        ctypes.byref(shape), GATES[gate], int(n_segments), ctypes.byref(seg),
+        ctypes.byref(kern), ctypes.byref(ws))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_chunk_fwd_split_plan")
+    return seg.value, kern.value, ws.value
 
 
 def chunk_bwd(q, k, v, log_alpha, beta, initial_state, cu_seqlens, d_out,

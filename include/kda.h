@@ -357,6 +357,61 @@ KDA_API kda_status kda_chunk_bwd(const kda_shape* shape, const void* q,
 KDA_API kda_status kda_chunk_bwd_plan(const kda_shape* shape, int packed,
                                       int* kernels, size_t* workspace_bytes);
 
+/*
+ * kda_chunk_fwd_split -- the chunkwise prefill of ONE long sequence (dense
+ * layout, shape->B == 1, no cu_seqlens), evaluated as n_segments segments
+ * side by side instead of one serial chain of chunks, then joined by a scan
+ * over the segments.
+ *
+ * Why it is exact: the state update is affine in the state ("Kimi Delta
+ * Attention", akshathtiwari.co.in, the delta-rule passage).  Inside a segment
+ * entered with state S_in, and with M_t the product of the token transitions
+ * (I - beta k k^T) Diag(alpha) from the segment start to token t,
+ *     S_t = M_t S_in + S_t|0,      o_t = o_t|0 + S_in^T (M_t^T q_t),
+ * where |0 is the evaluation from a zero state.  M_t is the state of the same
+ * recurrence run with v = 0 from the identity, and M_t^T q_t is its output.
+ * The call:
+ *   1. evaluates all segments at once as a packed batch: segment 0 from
+ *      initial_state, the others from zero (outputs go to `out`);
+ *   2. concurrently, on a second stream it joins before returning, evaluates
+ *      segments 1..n-1 with v = 0, d_v = d_k and the identity as start state;
+ *   3. scans: S_in(1) = S_end(0), S_in(j+1) = M_end(j) S_in(j) + S_end|0(j);
+ *      the last step writes final_state;
+ *   4. adds S_in(j)^T (M_t^T q_t) to the outputs of segments 1..n-1.
+ * Steps 1 and 2 run the path kda_chunk_fwd picks for their shapes; steps 3
+ * and 4 are fp32.  Segments are ceil(chunks / n_segments) chunks long (the
+ * last takes the rest; n_segments above the chunk count is reduced to it).
+ * With bf16 io, step 1's outputs and step 2's M_t^T q_t pass through bf16:
+ * the result agrees with kda_chunk_fwd to the bf16 tolerance, not bit for bit.
+ *
+ * When it pays: steps 1 and 2 run 2n - 1 chains of T/n tokens side by side,
+ * so the call shortens the serial chain when one sequence leaves most SMs
+ * idle (few heads).  When the GPU is already full, the extra work of step 2
+ * makes it slower than kda_chunk_fwd.
+ *
+ * Arguments: as kda_chunk_fwd_gated with B = 1 and cu_seqlens = NULL, plus
+ * n_segments in 1 .. 64 (1 runs kda_chunk_fwd_gated's evaluation).  Errors:
+ * as kda_chunk_fwd_gated; B != 1 or n_segments out of range ->
+ * KDA_ERR_INVALID_ARG.  Workspace: stream-ordered (kda_chunk_fwd_split_plan
+ * reports it).  The call queues work on `stream` and on a library-owned
+ * stream and makes `stream` wait for all of it.
+ */
+KDA_API kda_status kda_chunk_fwd_split(const kda_shape* shape, int gate,
+                                       const void* q, const void* k,
+                                       const void* v, const float* gate_tensor,
+                                       const float* beta,
+                                       const float* initial_state, void* out,
+                                       float* final_state, int n_segments,
+                                       cudaStream_t stream);
+
+/* kda_chunk_fwd_split_plan -- the segments (after the reduction above), kernel
+ * launches and workspace bytes of a kda_chunk_fwd_split call; no device
+ * work.  Any out pointer may be NULL. */
+KDA_API kda_status kda_chunk_fwd_split_plan(const kda_shape* shape, int gate,
+                                            int n_segments, int* segments,
+                                            int* kernels,
+                                            size_t* workspace_bytes);
+
 /* kda_selftest_timeout -- diagnostic of the failure reporting, not part of
  * the forward pass: launches one CTA that waits on a device barrier nothing
  * completes, using the library's bounded wait with a limit of limit_us

@@ -195,3 +195,38 @@ def test_backward_plan(lib):
     kern_p, _ = K.chunk_bwd_plan(1, 300, 2, 64, 64, 32, torch.float32,
                                  packed=True, n_seqs=3)
     assert kern_p == 17
+
+
+def split_call(lib, s, gate=0, n=2, **kw):
+    """kda_chunk_fwd_split with fake, disjoint addresses."""
+    names = ["q", "k", "v", "la", "b", "s0", "out", "sf"]
+    slots = {nm: i + 1 for i, nm in enumerate(names)}
+    slots.update(kw)
+    args = [_p(slots[nm]) if isinstance(slots[nm], int) else slots[nm]
+            for nm in names]
+    return lib.kda_chunk_fwd_split(ctypes.byref(s), gate, *args, n, None)
+
+
+def test_split_validation_and_plan(lib):
+    import torch
+    # one dense sequence only, and 1 .. 64 segments
+    assert split_call(lib, shape(B=2)) == INVALID
+    assert split_call(lib, shape(), n=0) == INVALID
+    assert split_call(lib, shape(), n=65) == INVALID
+    assert split_call(lib, shape(dk=48)) == UNSUPPORTED
+    assert split_call(lib, shape(), out=None) == INVALID
+    assert split_call(lib, shape(), out=1) == INVALID       # out over q
+    bad = ctypes.c_void_p(A + 0x1000_0000 + 8)
+    assert split_call(lib, shape(), q=bad) == MISALIGNED
+    assert split_call(lib, shape(), gate=7) == INVALID
+    # plan: segments of ceil(chunks / n) chunks; the kernels are the setup,
+    # both runs (two launches each on the fused packed path), scan and fix
+    seg, kern, ws = K.chunk_fwd_split_plan(131072, 8, 128, 128, 64,
+                                           torch.bfloat16, 4)
+    assert seg == 4 and kern == 1 + 2 + 2 + 2 and ws > 0
+    seg, kern, ws = K.chunk_fwd_split_plan(1000, 2, 64, 64, 64,
+                                           torch.bfloat16, 7)
+    assert seg == 6  # 16 chunks in segments of 3
+    seg, kern, ws = K.chunk_fwd_split_plan(100, 2, 64, 64, 64,
+                                           torch.bfloat16, 1)
+    assert (seg, kern, ws) == (1, 1, 0)
