@@ -411,10 +411,14 @@ def run_kda(args, world, rank, local):
 
     # ---- one long sequence (131072 tokens, d = 128, bf16, with a start
     # state): the plain prefill's serial chain of 2048 chunks against the
-    # sequence split into segments joined by a scan, with few heads (H = 8,
-    # most SMs idle) and with H = 32 (the GPU already full) ----------------
+    # sequence split into segments joined by a scan, with the segment count
+    # the library picks for this GPU (n_segments = 0): few heads (H = 8, most
+    # SMs idle) and H = 32 (the GPU already full: not split) ----------------
     prefill_split = {}
-    for Hs, nseg in ((8, 4), (32, 2)):
+    n_sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    for Hs in (8, 32):
+        nseg = K.chunk_fwd_split_plan(131072, Hs, 128, 128, C, torch.bfloat16,
+                                      0, num_sms=n_sms)[0]
         ds = W.draw((1, 131072), Hs, 128, 128, io="bf16", scale_q=True,
                     n_states=1, device=dev, seed=1234 + Hs + 97 * rank)
         outs = torch.empty_like(ds["v"])
@@ -427,9 +431,8 @@ def run_kda(args, world, rank, local):
 
         def split(_i):
             K.chunk_fwd_split(ds["q"], ds["k"], ds["v"], ds["log_alpha"],
-                              ds["beta"], ds["initial_state"],
-                              n_segments=nseg, chunk=C, out=outs,
-                              final_state=fins)
+                              ds["beta"], ds["initial_state"], n_segments=0,
+                              chunk=C, out=outs, final_state=fins)
 
         for fn in (plain, split):
             fn(0)
@@ -446,7 +449,8 @@ def run_kda(args, world, rank, local):
             "value": world * 131072 / (sms * 1e-3), "unit": "tokens/s",
             "ms_per_step": sms, "steps": sp_steps, "segments": nseg,
             "unsplit_ms_per_step": pms, "speedup_vs_unsplit": pms / sms,
-            "workload": f"kda_chunk_fwd_split, one sequence of 131072 tokens, "
+            "workload": f"kda_chunk_fwd_split (segment count picked for "
+                        f"{n_sms} SMs), one sequence of 131072 tokens, "
                         f"H={Hs} d=128 bf16, start state in, final state out; "
                         "unsplit = kda_chunk_fwd on the same inputs",
         }

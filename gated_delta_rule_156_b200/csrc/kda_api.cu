@@ -217,13 +217,21 @@ kda_status kda_chunk_fwd_split(const kda_shape* shape, int gate, const void* q,
                                const float* initial_state, void* out,
                                float* final_state, int n_segments,
                                cudaStream_t stream) {
-  if (!shape || shape->B != 1 || n_segments < 1 || n_segments > 64)
+  if (!shape || shape->B != 1 || n_segments < 0 || n_segments > 64)
     return KDA_ERR_INVALID_ARG;
   kda::ChunkArgs a{};
   const kda_status st = validate_chunk(shape, q, k, v, gate_tensor, beta,
                                        initial_state, nullptr, out,
                                        final_state, &a, gate);
   if (st != KDA_OK) return st;
+  if (n_segments == 0) {
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess)
+      e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    n_segments = kda::split_auto_segments(a, sms);
+  }
   const kda::SplitGeom g = kda::split_geometry(a, n_segments);
   const size_t bytes = kda::split_workspace_bytes(a, g);
   void* ws = nullptr;
@@ -242,10 +250,11 @@ kda_status kda_chunk_fwd_split(const kda_shape* shape, int gate, const void* q,
 }
 
 kda_status kda_chunk_fwd_split_plan(const kda_shape* shape, int gate,
-                                    int n_segments, int* segments, int* kernels,
-                                    size_t* workspace_bytes) {
-  if (!shape || shape->B != 1 || n_segments < 1 || n_segments > 64)
+                                    int n_segments, int num_sms, int* segments,
+                                    int* kernels, size_t* workspace_bytes) {
+  if (!shape || shape->B != 1 || n_segments < 0 || n_segments > 64)
     return KDA_ERR_INVALID_ARG;
+  if (n_segments == 0 && num_sms < 1) return KDA_ERR_INVALID_ARG;
   if (gate != kda::kGateChannel && gate != kda::kGateHead &&
       gate != kda::kGateNone)
     return KDA_ERR_INVALID_ARG;
@@ -255,6 +264,7 @@ kda_status kda_chunk_fwd_split_plan(const kda_shape* shape, int gate,
   kda::ChunkArgs a{};
   fill_args(shape, n_seqs, &a);
   a.gate = gate;
+  if (n_segments == 0) n_segments = kda::split_auto_segments(a, num_sms);
   const kda::SplitGeom g = kda::split_geometry(a, n_segments);
   if (segments) *segments = g.k;
   if (kernels) *kernels = kda::split_kernel_count(a, g);

@@ -95,6 +95,9 @@ struct SplitGeom {
   int k;
 };
 SplitGeom split_geometry(const ChunkArgs& a, int n_segments);
+// The segment count the call picks when asked for none: the largest k whose
+// 2k - 1 concurrent chains (k value, k - 1 transition) fit on num_sms SMs.
+int split_auto_segments(const ChunkArgs& a, int num_sms);
 size_t split_workspace_bytes(const ChunkArgs& a, const SplitGeom& g);
 int split_kernel_count(const ChunkArgs& a, const SplitGeom& g);
 cudaError_t launch_split(const ChunkArgs& a, const SplitGeom& g, void* workspace,

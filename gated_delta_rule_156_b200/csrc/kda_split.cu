@@ -367,6 +367,17 @@ cudaError_t run_split(const ChunkArgs& a, const SplitGeom& g, void* workspace,
 
 }  // namespace
 
+int split_auto_segments(const ChunkArgs& a, int num_sms) {
+  // CTAs one segment's chain occupies: one per head and 64-wide value tile
+  // (the paired kernel's two CTAs at d_v = 128); the transition run has
+  // d_v = d_k, so take the wider of the two
+  const int wide = a.dv > a.dk ? a.dv : a.dk;
+  const int per_seg = a.H * (wide > 64 ? wide / 64 : 1);
+  int k = 1;
+  while (k < 64 && (2 * (k + 1) - 1) * per_seg <= num_sms) ++k;
+  return k;
+}
+
 SplitGeom split_geometry(const ChunkArgs& a, int n_segments) {
   SplitGeom g{};
   const int C = a.chunk;

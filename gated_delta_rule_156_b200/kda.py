@@ -115,7 +115,7 @@ def library():
             fp, ctypes.c_int, vp]
         lib.kda_chunk_fwd_split_plan.restype = ctypes.c_int
         lib.kda_chunk_fwd_split_plan.argtypes = [
-            ctypes.POINTER(KdaShape), ctypes.c_int, ctypes.c_int,
+            ctypes.POINTER(KdaShape), ctypes.c_int, ctypes.c_int, ctypes.c_int,
             ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int),
             ctypes.POINTER(ctypes.c_size_t)]
         lib.kda_chunk_bwd.restype = ctypes.c_int
@@ -232,8 +232,9 @@ def chunk_fwd_split(q, k, v, log_alpha, beta, initial_state=None,
                     gate="channel", stream=None):
     """Prefill of one long sequence as ``n_segments`` segments evaluated side
     by side and joined by a scan of their state transitions
-    (kda_chunk_fwd_split).  Shapes as chunk_fwd with B == 1 and no
-    cu_seqlens.  Returns (out, final_state)."""
+    (kda_chunk_fwd_split; ``n_segments=0`` lets the library pick the count
+    from the SM count).  Shapes as chunk_fwd with B == 1 and no cu_seqlens.
+    Returns (out, final_state)."""
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     if out is None:
@@ -259,14 +260,15 @@ def chunk_fwd_split(q, k, v, log_alpha, beta, initial_state=None,
 
 
 def chunk_fwd_split_plan(T, H, dk, dv, chunk, dtype, n_segments,
-                         gate="channel"):
-    """(segments, kernels, workspace_bytes) of a chunk_fwd_split call."""
+                         gate="channel", num_sms=148):
+    """(segments, kernels, workspace_bytes) of a chunk_fwd_split call
+    (``num_sms`` matters only for ``n_segments=0``)."""
     io = KDA_BF16 if dtype == torch.bfloat16 else KDA_F32
     shape = KdaShape(1, T, H, dk, dv, chunk, 0, io)
     seg, kern, ws = ctypes.c_int(), ctypes.c_int(), ctypes.c_size_t()
     st = library().kda_chunk_fwd_split_plan(
-        ctypes.byref(shape), GATES[gate], int(n_segments), ctypes.byref(seg),
-        ctypes.byref(kern), ctypes.byref(ws))
+        ctypes.byref(shape), GATES[gate], int(n_segments), int(num_sms),
+        ctypes.byref(seg), ctypes.byref(kern), ctypes.byref(ws))
     if st != KDA_OK:
         raise KdaError(st, "kda_chunk_fwd_split_plan")
     return seg.value, kern.value, ws.value

@@ -390,8 +390,11 @@ KDA_API kda_status kda_chunk_bwd_plan(const kda_shape* shape, int packed,
  * makes it slower than kda_chunk_fwd.
  *
  * Arguments: as kda_chunk_fwd_gated with B = 1 and cu_seqlens = NULL, plus
- * n_segments in 1 .. 64 (1 runs kda_chunk_fwd_gated's evaluation).  Errors:
- * as kda_chunk_fwd_gated; B != 1 or n_segments out of range ->
+ * n_segments in 0 .. 64.  1 runs kda_chunk_fwd_gated's evaluation.  0 picks
+ * the count: the largest k whose 2k - 1 concurrent chains fit on the
+ * device's SMs, each chain taking one CTA per head and 64 columns of the
+ * wider of d_k and d_v (so H = 32, d = 128 is not split at all on a B200).
+ * Errors: as kda_chunk_fwd_gated; B != 1 or n_segments out of range ->
  * KDA_ERR_INVALID_ARG.  Workspace: stream-ordered (kda_chunk_fwd_split_plan
  * reports it).  The call queues work on `stream` and on a library-owned
  * stream and makes `stream` wait for all of it.
@@ -406,10 +409,12 @@ KDA_API kda_status kda_chunk_fwd_split(const kda_shape* shape, int gate,
 
 /* kda_chunk_fwd_split_plan -- the segments (after the reduction above), kernel
  * launches and workspace bytes of a kda_chunk_fwd_split call; no device
- * work.  Any out pointer may be NULL. */
+ * work.  num_sms stands in for the device's SM count when n_segments is 0
+ * (it must then be >= 1; otherwise it is ignored).  Any out pointer may be
+ * NULL. */
 KDA_API kda_status kda_chunk_fwd_split_plan(const kda_shape* shape, int gate,
-                                            int n_segments, int* segments,
-                                            int* kernels,
+                                            int n_segments, int num_sms,
+                                            int* segments, int* kernels,
                                             size_t* workspace_bytes);
 
 /* kda_selftest_timeout -- diagnostic of the failure reporting, not part of

@@ -211,7 +211,7 @@ def test_split_validation_and_plan(lib):
     import torch
     # one dense sequence only, and 1 .. 64 segments
     assert split_call(lib, shape(B=2)) == INVALID
-    assert split_call(lib, shape(), n=0) == INVALID
+    assert split_call(lib, shape(), n=-1) == INVALID
     assert split_call(lib, shape(), n=65) == INVALID
     assert split_call(lib, shape(dk=48)) == UNSUPPORTED
     assert split_call(lib, shape(), out=None) == INVALID
@@ -230,3 +230,12 @@ def test_split_validation_and_plan(lib):
     seg, kern, ws = K.chunk_fwd_split_plan(100, 2, 64, 64, 64,
                                            torch.bfloat16, 1)
     assert (seg, kern, ws) == (1, 1, 0)
+    # n_segments = 0 picks the largest k with (2k - 1) chains of H x (width
+    # / 64) CTAs within the SMs: H = 8, d = 128 -> 16 CTAs a chain -> k = 5;
+    # H = 32 -> 64 a chain -> 1 (not split)
+    assert K.chunk_fwd_split_plan(131072, 8, 128, 128, 64, torch.bfloat16, 0,
+                                  num_sms=148)[0] == 5
+    assert K.chunk_fwd_split_plan(131072, 32, 128, 128, 64, torch.bfloat16, 0,
+                                  num_sms=148)[0] == 1
+    assert K.chunk_fwd_split_plan(131072, 4, 64, 64, 64, torch.bfloat16, 0,
+                                  num_sms=148)[0] == 19

@@ -104,3 +104,17 @@ def test_split_without_initial_state_long():
                          None)
     PY.check("out vs unsplit", PY.host64(out), PY.host64(o2), PY.TOL_BF16)
     PY.check("final vs unsplit", PY.host64(fin), PY.host64(f2), PY.TOL_BF16)
+
+
+def test_split_auto_segment_count():
+    # n_segments = 0: the library picks the count from the SM count (two
+    # heads of d = 128 leave most SMs idle, so it splits)
+    d = case(4000, 2, 128, 128, "bf16", seed=44)
+    n_sms = torch.cuda.get_device_properties(0).multi_processor_count
+    seg = K.chunk_fwd_split_plan(4000, 2, 128, 128, 64, torch.bfloat16, 0,
+                                 num_sms=n_sms)[0]
+    assert seg > 1
+    out, fin = K.chunk_fwd_split(d["q"], d["k"], d["v"], d["log_alpha"],
+                                 d["beta"], d["initial_state"], n_segments=0)
+    assert K.device_status() == 0
+    against_oracle(d, out, fin, PY.TOL_BF16)
