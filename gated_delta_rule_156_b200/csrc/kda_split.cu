@@ -224,58 +224,71 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
-// (4) Per (chunk of segments 1..k-1, head): out[t] += S_in(j)^T X[t] for its
-// C tokens (a chunk never straddles segments, whose length is a multiple of
-// C).  X rows and S_in(j) are staged in shared memory; thread (ti, tj) owns
-// rows ti + 16 a and columns tj + 16 b.
+// (4) Per (group of kFixChunks chunks of segments 1..k-1, head): out[t] +=
+// S_in(j)^T X[t] for each chunk's C tokens (a chunk never straddles segments,
+// whose length is a multiple of C).  S_in(j) is staged in shared memory once
+// per segment the group touches, each chunk's X rows beside it; thread
+// (ti, tj) owns rows ti + 16 a and columns tj + 16 b.
+constexpr int kFixChunks = 8;
+
 template <typename IO>
 __global__ void __launch_bounds__(kThreads)
     split_fix_kernel(SplitWs w, IO* __restrict__ out, int T, int Ls, int k,
                      int H, int dk, int dv, int C) {
-  const int t0 = Ls + blockIdx.x * C, h = blockIdx.y, tid = threadIdx.x;
-  const int L = min(C, T - t0);
-  const int j = min(t0 / Ls, k - 1);
+  const int h = blockIdx.y, tid = threadIdx.x;
+  const int n_rest = (T - Ls + C - 1) / C;  // chunks after segment 0
+  const int c_begin = blockIdx.x * kFixChunks;
+  const int c_end = min(c_begin + kFixChunks, n_rest);
   const int dkp = dk + 1;
   extern __shared__ float sm[];
   float* X = sm;             // [C][dkp]
   float* S = X + C * dkp;    // [dk][dv]
   const IO* x = static_cast<const IO*>(w.x);
-  for (int idx = tid; idx < C * dk; idx += kThreads) {
-    const int r = idx / dk, c = idx % dk;
-    X[r * dkp + c] =
-        r < L ? to_f32(x[((size_t)(t0 - Ls + r) * H + h) * dk + c]) : 0.f;
-  }
-  const float* Sin = w.s_in + ((size_t)(j - 1) * H + h) * dk * dv;
-  for (int idx = tid; idx < dk * dv; idx += kThreads) S[idx] = Sin[idx];
-  __syncthreads();
   const int ti = tid >> 4, tj = tid & 15, nr = C / 16, nc = dv / 16;
-  float acc[4][8];
-#pragma unroll
-  for (int a = 0; a < 4; ++a)
-#pragma unroll
-    for (int b = 0; b < 8; ++b) acc[a][b] = 0.f;
-#pragma unroll 2
-  for (int c = 0; c < dk; ++c) {
-    float xv[4], sv[8];
-#pragma unroll
-    for (int a = 0; a < 4; ++a) xv[a] = a < nr ? X[(ti + 16 * a) * dkp + c] : 0.f;
-#pragma unroll
-    for (int b = 0; b < 8; ++b) sv[b] = b < nc ? S[c * dv + tj + 16 * b] : 0.f;
+  int j_staged = -1;
+  for (int cc = c_begin; cc < c_end; ++cc) {
+    const int t0 = Ls + cc * C, L = min(C, T - t0);
+    const int j = min(t0 / Ls, k - 1);
+    __syncthreads();  // the previous chunk's reads are done
+    for (int idx = tid; idx < C * dk; idx += kThreads) {
+      const int r = idx / dk, c = idx % dk;
+      X[r * dkp + c] =
+          r < L ? to_f32(x[((size_t)(t0 - Ls + r) * H + h) * dk + c]) : 0.f;
+    }
+    if (j != j_staged) {
+      const float* Sin = w.s_in + ((size_t)(j - 1) * H + h) * dk * dv;
+      for (int idx = tid; idx < dk * dv; idx += kThreads) S[idx] = Sin[idx];
+      j_staged = j;
+    }
+    __syncthreads();
+    float acc[4][8];
 #pragma unroll
     for (int a = 0; a < 4; ++a)
 #pragma unroll
-      for (int b = 0; b < 8; ++b) acc[a][b] += xv[a] * sv[b];
-  }
+      for (int b = 0; b < 8; ++b) acc[a][b] = 0.f;
+#pragma unroll 2
+    for (int c = 0; c < dk; ++c) {
+      float xv[4], sv[8];
 #pragma unroll
-  for (int a = 0; a < 4; ++a) {
-    const int r = ti + 16 * a;
-    if (a < nr && r < L) {
-      IO* o = out + ((size_t)(t0 + r) * H + h) * dv;
+      for (int a = 0; a < 4; ++a) xv[a] = a < nr ? X[(ti + 16 * a) * dkp + c] : 0.f;
 #pragma unroll
-      for (int b = 0; b < 8; ++b) {
-        if (b < nc) {
-          const int jj = tj + 16 * b;
-          o[jj] = from_f32<IO>(to_f32(o[jj]) + acc[a][b]);
+      for (int b = 0; b < 8; ++b) sv[b] = b < nc ? S[c * dv + tj + 16 * b] : 0.f;
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 8; ++b) acc[a][b] += xv[a] * sv[b];
+    }
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const int r = ti + 16 * a;
+      if (a < nr && r < L) {
+        IO* o = out + ((size_t)(t0 + r) * H + h) * dv;
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+          if (b < nc) {
+            const int jj = tj + 16 * b;
+            o[jj] = from_f32<IO>(to_f32(o[jj]) + acc[a][b]);
+          }
         }
       }
     }
@@ -359,7 +372,8 @@ cudaError_t run_split(const ChunkArgs& a, const SplitGeom& g, void* workspace,
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const size_t smf = 4 * ((size_t)C * (dk + 1) + (size_t)dk * dv);
   if ((e = set_smem(split_fix_kernel<IO>, smf)) != cudaSuccess) return e;
-  const unsigned nblk = (unsigned)((a.T - g.Ls + C - 1) / C);
+  const int n_rest = (a.T - g.Ls + C - 1) / C;
+  const unsigned nblk = (unsigned)((n_rest + kFixChunks - 1) / kFixChunks);
   split_fix_kernel<IO><<<dim3(nblk, H), kThreads, smf, stream>>>(
       w, static_cast<IO*>(a.out), a.T, g.Ls, g.k, H, dk, dv, C);
   return cudaGetLastError();
