@@ -624,6 +624,14 @@ def run_only(args, dev, stream):
             K.chunk_bwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"],
                         None, None, gdo, None, chunk=cfg["chunk"],
                         want_initial_state=False)
+    elif args.only == "split":
+        Ts = args.seq_len or 131072
+        ds = W.draw((1, Ts), 8, 128, 128, io="bf16", scale_q=True, n_states=1,
+                    device=dev, seed=1242)
+
+        def fn(_i):
+            K.chunk_fwd_split(ds["q"], ds["k"], ds["v"], ds["log_alpha"],
+                              ds["beta"], ds["initial_state"], n_segments=0)
     else:
         dc = W.CONFIGS[DECODE_CFG]
         dd = W.make(DECODE_CFG, device=dev)
@@ -676,14 +684,15 @@ def main():
     ap.add_argument("--impl", choices=["kda", "reference"], default="kda")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--only", choices=["prefill", "decode", "backward"],
+    ap.add_argument("--only", choices=["prefill", "decode", "backward", "split"],
                     default=None,
                     help="profiling aid: run one workload's warm-up and timed "
                          "launches only (no e2e, no CPU baseline, no JSON line)")
     ap.add_argument("--seq-len", type=int, default=None,
-                    help="with --only prefill/backward: tokens per sequence "
-                         "(default: the prefill workload's 8192), for a "
-                         "smaller profiler capture")
+                    help="with --only prefill/backward/split: tokens per "
+                         "sequence (default: the workload's own, 8192 for "
+                         "prefill and backward, 131072 for the split's one "
+                         "sequence of H=8), for a smaller profiler capture")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -224,72 +224,158 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
-// (4) Per (group of kFixChunks chunks of segments 1..k-1, head): out[t] +=
-// S_in(j)^T X[t] for each chunk's C tokens (a chunk never straddles segments,
-// whose length is a multiple of C).  S_in(j) is staged in shared memory once
-// per segment the group touches, each chunk's X rows beside it; thread
-// (ti, tj) owns rows ti + 16 a and columns tj + 16 b.
-constexpr int kFixChunks = 8;
+// (4) Per (chunk of segments 1..k-1, head): out[t] += S_in(j)^T X[t] for its
+// C tokens (a chunk never straddles segments, whose length is a multiple of
+// C).  X is staged transposed (XT[c][r], lanes walking down the rows so the
+// scattered stores hit distinct banks) and S_in(j) as is, both with rows
+// padded by four floats; thread (ti, tj) of a 16 x 16 grid owns the RM x RN
+// block at rows RM ti.., columns RN tj.. (RM = C / 16, RN = d_v / 16), so
+// each step of the contraction is a few 16-byte shared loads for RM x RN
+// FMAs.
+template <int N>
+__device__ __forceinline__ void lds_run(const float* p, float* v) {
+  if constexpr (N >= 4) {
+#pragma unroll
+    for (int q = 0; q < N / 4; ++q) {
+      const float4 x = *reinterpret_cast<const float4*>(p + 4 * q);
+      v[4 * q] = x.x;
+      v[4 * q + 1] = x.y;
+      v[4 * q + 2] = x.z;
+      v[4 * q + 3] = x.w;
+    }
+  } else if constexpr (N == 2) {
+    const float2 x = *reinterpret_cast<const float2*>(p);
+    v[0] = x.x;
+    v[1] = x.y;
+  } else {
+    v[0] = p[0];
+  }
+}
 
-template <typename IO>
+// Eight consecutive io-dtype elements as fp32 (one 16-byte load for bf16,
+// two for fp32), and back.
+__device__ __forceinline__ void ld8(const __nv_bfloat16* p, float* v) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 f = __bfloat1622float2(h[e]);
+    v[2 * e] = f.x;
+    v[2 * e + 1] = f.y;
+  }
+}
+__device__ __forceinline__ void ld8(const float* p, float* v) {
+  const float4 a = *reinterpret_cast<const float4*>(p);
+  const float4 b = *reinterpret_cast<const float4*>(p + 4);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ void st8(__nv_bfloat16* p, const float* v) {
+  uint4 u;
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) h[e] = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+  *reinterpret_cast<uint4*>(p) = u;
+}
+__device__ __forceinline__ void st8(float* p, const float* v) {
+  *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  *reinterpret_cast<float4*>(p + 4) = make_float4(v[4], v[5], v[6], v[7]);
+}
+
+template <typename IO, int RM, int RN>
 __global__ void __launch_bounds__(kThreads)
     split_fix_kernel(SplitWs w, IO* __restrict__ out, int T, int Ls, int k,
-                     int H, int dk, int dv, int C) {
-  const int h = blockIdx.y, tid = threadIdx.x;
-  const int n_rest = (T - Ls + C - 1) / C;  // chunks after segment 0
-  const int c_begin = blockIdx.x * kFixChunks;
-  const int c_end = min(c_begin + kFixChunks, n_rest);
-  const int dkp = dk + 1;
-  extern __shared__ float sm[];
-  float* X = sm;             // [C][dkp]
-  float* S = X + C * dkp;    // [dk][dv]
+                     int H, int dk, int dv) {
+  constexpr int C = 16 * RM, DV = 16 * RN, LX = C + 4, LS = DV + 4;
+  const int t0 = Ls + blockIdx.x * C, h = blockIdx.y, tid = threadIdx.x;
+  const int L = min(C, T - t0);
+  const int j = min(t0 / Ls, k - 1);
+  extern __shared__ __align__(16) float sm[];
+  float* XT = sm;              // [dk][LX]
+  float* S = XT + dk * LX;     // [dk][LS]
   const IO* x = static_cast<const IO*>(w.x);
-  const int ti = tid >> 4, tj = tid & 15, nr = C / 16, nc = dv / 16;
-  int j_staged = -1;
-  for (int cc = c_begin; cc < c_end; ++cc) {
-    const int t0 = Ls + cc * C, L = min(C, T - t0);
-    const int j = min(t0 / Ls, k - 1);
-    __syncthreads();  // the previous chunk's reads are done
-    for (int idx = tid; idx < C * dk; idx += kThreads) {
-      const int r = idx / dk, c = idx % dk;
-      X[r * dkp + c] =
-          r < L ? to_f32(x[((size_t)(t0 - Ls + r) * H + h) * dk + c]) : 0.f;
-    }
-    if (j != j_staged) {
-      const float* Sin = w.s_in + ((size_t)(j - 1) * H + h) * dk * dv;
-      for (int idx = tid; idx < dk * dv; idx += kThreads) S[idx] = Sin[idx];
-      j_staged = j;
-    }
-    __syncthreads();
-    float acc[4][8];
+  // XT[c][r] = X[r][c]: thread (r, 8-column group), rows past L zero; all
+  // of a thread's loads are issued before its stores
+  {
+    constexpr int NX = 64 * 128 / 8 / kThreads;  // C * dk / 8 <= NX * kThreads
+    float v[NX][8];
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
+    for (int u = 0; u < NX; ++u) {
+      const int idx = u * kThreads + tid;
+      const int r = idx % C, c = (idx / C) * 8;
 #pragma unroll
-      for (int b = 0; b < 8; ++b) acc[a][b] = 0.f;
-#pragma unroll 2
-    for (int c = 0; c < dk; ++c) {
-      float xv[4], sv[8];
-#pragma unroll
-      for (int a = 0; a < 4; ++a) xv[a] = a < nr ? X[(ti + 16 * a) * dkp + c] : 0.f;
-#pragma unroll
-      for (int b = 0; b < 8; ++b) sv[b] = b < nc ? S[c * dv + tj + 16 * b] : 0.f;
-#pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b = 0; b < 8; ++b) acc[a][b] += xv[a] * sv[b];
+      for (int e = 0; e < 8; ++e) v[u][e] = 0.f;
+      if (idx < C * (dk / 8) && r < L)
+        ld8(x + ((size_t)(t0 - Ls + r) * H + h) * dk + c, v[u]);
     }
 #pragma unroll
-    for (int a = 0; a < 4; ++a) {
-      const int r = ti + 16 * a;
-      if (a < nr && r < L) {
-        IO* o = out + ((size_t)(t0 + r) * H + h) * dv;
+    for (int u = 0; u < NX; ++u) {
+      const int idx = u * kThreads + tid;
+      if (idx < C * (dk / 8)) {
+        const int r = idx % C, c = (idx / C) * 8;
 #pragma unroll
-        for (int b = 0; b < 8; ++b) {
-          if (b < nc) {
-            const int jj = tj + 16 * b;
-            o[jj] = from_f32<IO>(to_f32(o[jj]) + acc[a][b]);
-          }
+        for (int e = 0; e < 8; ++e) XT[(c + e) * LX + r] = v[u][e];
+      }
+    }
+  }
+  // S_in(j), sixteen 16-byte loads in flight per thread at a time
+  {
+    const float* Sin = w.s_in + ((size_t)(j - 1) * H + h) * dk * dv;
+    const int units = dk * (DV / 4);
+    for (int base = 0; base < units; base += 16 * kThreads) {
+      float4 v[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int idx = base + u * kThreads + tid;
+        if (idx < units) {
+          const int c = idx / (DV / 4), q = idx % (DV / 4);
+          v[u] = *reinterpret_cast<const float4*>(Sin + (size_t)c * dv + 4 * q);
         }
+      }
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int idx = base + u * kThreads + tid;
+        if (idx < units) {
+          const int c = idx / (DV / 4), q = idx % (DV / 4);
+          *reinterpret_cast<float4*>(S + c * LS + 4 * q) = v[u];
+        }
+      }
+    }
+  }
+  __syncthreads();
+  const int ti = tid >> 4, tj = tid & 15;
+  float acc[RM][RN];
+#pragma unroll
+  for (int a = 0; a < RM; ++a)
+#pragma unroll
+    for (int b = 0; b < RN; ++b) acc[a][b] = 0.f;
+  const float* ap = XT + RM * ti;
+  const float* bp = S + RN * tj;
+#pragma unroll 4
+  for (int c = 0; c < dk; ++c) {
+    float av[RM], bv[RN];
+    lds_run<RM>(ap + c * LX, av);
+    lds_run<RN>(bp + c * LS, bv);
+#pragma unroll
+    for (int a = 0; a < RM; ++a)
+#pragma unroll
+      for (int b = 0; b < RN; ++b) acc[a][b] += av[a] * bv[b];
+  }
+#pragma unroll
+  for (int a = 0; a < RM; ++a) {
+    const int r = RM * ti + a;
+    if (r < L) {
+      IO* o = out + ((size_t)(t0 + r) * H + h) * dv + RN * tj;
+      if constexpr (RN == 8) {  // one 16-byte read and write per row (bf16)
+        float y[8];
+        ld8(o, y);
+#pragma unroll
+        for (int b = 0; b < 8; ++b) y[b] += acc[a][b];
+        st8(o, y);
+      } else {
+#pragma unroll
+        for (int b = 0; b < RN; ++b)
+          o[b] = from_f32<IO>(to_f32(o[b]) + acc[a][b]);
       }
     }
   }
@@ -320,6 +406,40 @@ cudaError_t side_stream(cudaStream_t* out) {
   }
   *out = streams[dev];
   return cudaSuccess;
+}
+
+template <typename IO, int RM, int RN>
+cudaError_t launch_fix_t(const SplitWs& w, IO* out, const ChunkArgs& a,
+                         const SplitGeom& g, dim3 grid, cudaStream_t stream) {
+  const size_t smem = 4 * (size_t)a.dk * ((16 * RM + 4) + (16 * RN + 4));
+  cudaError_t e = set_smem(split_fix_kernel<IO, RM, RN>, smem);
+  if (e != cudaSuccess) return e;
+  split_fix_kernel<IO, RM, RN><<<grid, kThreads, smem, stream>>>(
+      w, out, a.T, g.Ls, g.k, a.H, a.dk, a.dv);
+  return cudaGetLastError();
+}
+
+template <typename IO, int RM>
+cudaError_t launch_fix_n(const SplitWs& w, IO* out, const ChunkArgs& a,
+                         const SplitGeom& g, dim3 grid, cudaStream_t stream) {
+  switch (a.dv) {
+    case 32: return launch_fix_t<IO, RM, 2>(w, out, a, g, grid, stream);
+    case 64: return launch_fix_t<IO, RM, 4>(w, out, a, g, grid, stream);
+    case 128: return launch_fix_t<IO, RM, 8>(w, out, a, g, grid, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+// The correction with the register blocking its chunk length and d_v ask for.
+template <typename IO>
+cudaError_t launch_fix(const SplitWs& w, IO* out, const ChunkArgs& a,
+                       const SplitGeom& g, dim3 grid, cudaStream_t stream) {
+  switch (a.chunk) {
+    case 16: return launch_fix_n<IO, 1>(w, out, a, g, grid, stream);
+    case 32: return launch_fix_n<IO, 2>(w, out, a, g, grid, stream);
+    case 64: return launch_fix_n<IO, 4>(w, out, a, g, grid, stream);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 template <typename IO>
@@ -370,13 +490,9 @@ cudaError_t run_split(const ChunkArgs& a, const SplitGeom& g, void* workspace,
   split_scan_kernel<<<dim3(H, dv / kScanTile), kThreads, sms, stream>>>(
       w, a.final_state, g.k, H, dk, dv);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const size_t smf = 4 * ((size_t)C * (dk + 1) + (size_t)dk * dv);
-  if ((e = set_smem(split_fix_kernel<IO>, smf)) != cudaSuccess) return e;
-  const int n_rest = (a.T - g.Ls + C - 1) / C;
-  const unsigned nblk = (unsigned)((n_rest + kFixChunks - 1) / kFixChunks);
-  split_fix_kernel<IO><<<dim3(nblk, H), kThreads, smf, stream>>>(
-      w, static_cast<IO*>(a.out), a.T, g.Ls, g.k, H, dk, dv, C);
-  return cudaGetLastError();
+  const unsigned nblk = (unsigned)((a.T - g.Ls + C - 1) / C);
+  return launch_fix<IO>(w, static_cast<IO*>(a.out), a, g, dim3(nblk, H),
+                        stream);
 }
 
 }  // namespace
