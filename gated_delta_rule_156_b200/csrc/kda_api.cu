@@ -551,10 +551,11 @@ const char* kda_status_string(kda_status status) {
 }
 
 kda_status kda_device_status(cudaStream_t stream) {
-  int flag = 0;
-  const cudaError_t e = kda::fused_take_timeout(stream, &flag);
+  int flag = 0, split_flag = 0;
+  cudaError_t e = kda::fused_take_timeout(stream, &flag);
+  if (e == cudaSuccess) e = kda::split_take_timeout(stream, &split_flag);
   if (e != cudaSuccess) return cuda_fail(e);
-  return flag ? KDA_ERR_TIMEOUT : KDA_OK;
+  return flag || split_flag ? KDA_ERR_TIMEOUT : KDA_OK;
 }
 
 kda_status kda_selftest_timeout(int limit_us, cudaStream_t stream) {

@@ -129,6 +129,8 @@ int fused_kernel_count(const ChunkArgs& a);
 // Synchronises `stream`, then reads and clears the flag a fused kernel sets
 // when one of its bounded waits gave up.
 cudaError_t fused_take_timeout(cudaStream_t stream, int* flag);
+// The same for the sequence split's tensor-core correction (kda_split.cu).
+cudaError_t split_take_timeout(cudaStream_t stream, int* flag);
 // Diagnostic: one CTA whose bounded wait runs out after limit_us.
 cudaError_t launch_timeout_probe(int limit_us, cudaStream_t stream);
 cudaError_t launch_fused(const ChunkArgs& a, void* workspace,

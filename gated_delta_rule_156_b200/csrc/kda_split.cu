@@ -21,11 +21,17 @@
 // four-stage, as kda_chunk_fwd would pick for their shapes); (3) and (4) are
 // the fp32 kernels below.
 #include <mutex>
+#include <type_traits>
 
 #include "kda_common.cuh"
 #include "kda_internal.h"
+#include "sm100_ptx.cuh"
 
 namespace kda {
+
+// Set by the tensor-core correction when its bounded MMA wait gives up; read
+// and cleared by kda_device_status.
+__device__ int g_split_timeout = 0;
 
 namespace {
 
@@ -41,6 +47,9 @@ struct SplitWs {
   float* ident;      // [k - 1, H, dk, dk] identity start states
   float* trans;      // [k - 1, H, dk, dk] segment transitions M_end
   float* s_in;       // [k - 1, H, dk, dv] entry states of segments 1..k-1
+  __nv_bfloat16* s_in_bf;  // the same in bf16, as the tensor-core correction's
+                           // MN-major operand: [k - 1, H, dv / 64, dk, 64],
+                           // each [dk, 64] panel 128-byte swizzled
   void* vzero;       // [T - Ls, H, dk] io dtype, zeros
   void* x;           // [T - Ls, H, dk] io dtype, M_t^T q_t
   void* ws_val;      // the value run's own workspace
@@ -121,6 +130,7 @@ SplitWs carve_split(const ChunkArgs& a, const SplitGeom& g, void* base,
   w.ident = static_cast<float*>(take(4 * (k - 1) * H * dk * dk));
   w.trans = static_cast<float*>(take(4 * (k - 1) * H * dk * dk));
   w.s_in = static_cast<float*>(take(4 * (k - 1) * H * dk * dv));
+  w.s_in_bf = static_cast<__nv_bfloat16*>(take(2 * (k - 1) * H * dk * dv));
   w.vzero = take(esz * rest);
   w.x = take(esz * rest);
   // the two runs' own workspaces: sized for the packed layout they run in
@@ -162,7 +172,7 @@ constexpr int kScanTile = 32, kScanTp = kScanTile + 1;
 
 __global__ void __launch_bounds__(kThreads)
     split_scan_kernel(SplitWs w, float* __restrict__ final_state, int k, int H,
-                      int dk, int dv) {
+                      int dk, int dv, int bf_panels) {
   const int h = blockIdx.x, j0 = blockIdx.y * kScanTile, tid = threadIdx.x;
   const int dkp = dk + 1, NA = dk / 32, g8 = tid >> 3, j8 = tid & 7;
   extern __shared__ float sm[];
@@ -180,9 +190,19 @@ __global__ void __launch_bounds__(kThreads)
     for (int idx = tid; idx < dk * dk; idx += kThreads)
       M[(idx / dk) * dkp + idx % dk] = Mj[idx];
     __syncthreads();
+    uint8_t* Sbf = reinterpret_cast<uint8_t*>(w.s_in_bf) +
+                   2 * ((size_t)(j - 1) * H + h) * dk * dv;
     for (int idx = tid; idx < dk * kScanTile; idx += kThreads) {
       const int c = idx / kScanTile, jj = idx % kScanTile;
-      Sin[(size_t)c * dv + j0 + jj] = S[c * kScanTp + jj];
+      const float sv = S[c * kScanTp + jj];
+      Sin[(size_t)c * dv + j0 + jj] = sv;
+      if (bf_panels) {  // element (c, n) of panel n / 64, swizzled
+        const int n = j0 + jj, nn = n & 63;
+        *reinterpret_cast<__nv_bfloat16*>(
+            Sbf + (size_t)(n >> 6) * dk * 128 + c * 128 +
+            ((((nn >> 3) ^ (c & 7)) << 4) | ((nn & 7) << 1))) =
+            __float2bfloat16_rn(sv);
+      }
     }
     float acc[4][4];
 #pragma unroll
@@ -381,6 +401,156 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
+// (4') The correction on the tensor cores, for bf16 io with d_k, d_v in
+// {64, 128}: per (chunk, head) one M = 128, N = d_v, K = d_k product of the
+// chunk's X rows (K-major, 128-byte-swizzled panels of 128 rows; rows past the
+// chunk are never read back) and S_in(j) rounded to bf16 (MN-major panels of
+// d_k rows), accumulated in TMEM.  The two warps that own TMEM lanes 0-63
+// then add the rows into the output, 16 bytes at a time.  The MMA wait is
+// bounded; if it gives up the block writes nothing and raises the library's
+// timeout flag.
+template <int DK, int DV>
+__global__ void __launch_bounds__(128)
+    split_fix_tc_kernel(SplitWs w, __nv_bfloat16* __restrict__ out, int T,
+                        int Ls, int k, int H, int C, int* timeout_flag) {
+  using namespace sm100;
+  constexpr uint32_t kApanel = 128 * 128;  // 128 rows of 64 bf16
+  constexpr uint32_t kBpanel = DK * 128;   // DK K-rows of 64 bf16
+  extern __shared__ __align__(1024) uint8_t sm_raw[];
+  uint8_t* sA = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sB = sA + (DK / 64) * kApanel;
+  constexpr uint32_t kBbytes = (DV / 64) * kBpanel;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sB + kBbytes);  // [0] B, [1] MMA
+  uint32_t* tbase = reinterpret_cast<uint32_t*>(bar + 2);
+  const int t0 = Ls + blockIdx.x * C, h = blockIdx.y, tid = threadIdx.x;
+  const int L = min(C, T - t0);
+  const int j = min(t0 / Ls, k - 1);
+  // B = S_in(j) in bf16, already in its swizzled N-major panels: one bulk
+  // copy (no multicast) completing on bar[0], while the threads stage A
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    mbar_init(bar + 1, 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(bar, kBbytes);
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(w.s_in_bf) +
+                         2 * ((size_t)(j - 1) * H + h) * DK * DV;
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes "
+        "[%0], [%1], %2, [%3];" ::"r"(smem_u32(sB)),
+        "l"(reinterpret_cast<uint64_t>(src)), "r"(kBbytes), "r"(smem_u32(bar))
+        : "memory");
+  }
+  // A[r][c] = X[r][c]: every load of the thread in flight before its stores
+  const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(w.x);
+  {
+    constexpr int NA = 64 * (DK / 8) / 128;
+    uint4 v[NA];
+#pragma unroll
+    for (int u = 0; u < NA; ++u) {
+      const int idx = u * 128 + tid;
+      const int r = idx / (DK / 8), pc = idx % (DK / 8);
+      v[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (r < L)
+        v[u] = *reinterpret_cast<const uint4*>(
+            x + ((size_t)(t0 - Ls + r) * H + h) * DK + pc * 8);
+    }
+#pragma unroll
+    for (int u = 0; u < NA; ++u) {
+      const int idx = u * 128 + tid;
+      const int r = idx / (DK / 8), pc = idx % (DK / 8);
+      *reinterpret_cast<uint4*>(sA + (pc / 8) * kApanel + r * 128 +
+                                (((pc % 8) ^ (r & 7)) << 4)) = v[u];
+    }
+  }
+  if (tid < 32) {
+    tmem_alloc(tbase, 128);
+    tmem_relinquish();
+  }
+  fence_proxy_async();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tbase;
+  bool ok = true;
+  if (tid == 0) {
+    ok = mbar_wait(bar, 0);  // B has landed
+    if (ok) {
+      const uint32_t idesc = idesc_bf16(128, DV, false, true);
+      const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
+#pragma unroll
+      for (int ks = 0; ks < DK / 16; ++ks)
+        mma_bf16(tmem,
+                 desc_sw128(a0 + (ks / 4) * kApanel + (ks % 4) * 32, 16, 1024),
+                 desc_sw128(b0 + ks * 2048, kBpanel, 1024), idesc,
+                 ks > 0 ? 1u : 0u);
+      mma_commit(bar + 1);
+    } else {
+      mbar_wait(bar, 0, 100000000ull);  // the copy, before the block leaves
+    }
+  }
+  ok = __syncthreads_and(ok) != 0;
+  if (ok) ok = mbar_wait(bar + 1, 0);
+  tc_fence_after();
+  const int warp = tid >> 5;
+  if (warp < 2) {  // TMEM lane = row of the chunk
+    const int r = tid;
+#pragma unroll
+    for (int c = 0; c < DV; c += 32) {
+      float v[32];
+      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + c, v);
+      if (ok && r < L) {
+        __nv_bfloat16* o = out + ((size_t)(t0 + r) * H + h) * DV + c;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          float y[8];
+          ld8(o + 8 * q, y);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) y[e] += v[8 * q + e];
+          st8(o + 8 * q, y);
+        }
+      }
+    }
+  }
+  if (!ok && tid == 0) atomicExch(timeout_flag, 1);
+  tc_fence_before();
+  __syncthreads();
+  if (tid < 32) tmem_dealloc(tmem, 128);
+}
+
+template <int DK, int DV>
+cudaError_t launch_fix_tc_t(const SplitWs& w, __nv_bfloat16* out,
+                            const ChunkArgs& a, const SplitGeom& g, dim3 grid,
+                            int* flag, cudaStream_t stream) {
+  const size_t smem = 1024 + (DK / 64) * 128 * 128 + (DV / 64) * DK * 128 + 64;
+  static_assert(((DV / 64) * DK * 128) % 16 == 0, "bulk copy size");
+  cudaError_t e = cudaFuncSetAttribute(split_fix_tc_kernel<DK, DV>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  split_fix_tc_kernel<DK, DV><<<grid, 128, smem, stream>>>(
+      w, out, a.T, g.Ls, g.k, a.H, a.chunk, flag);
+  return cudaGetLastError();
+}
+
+bool fix_on_tensor_cores(const ChunkArgs& a) {
+  return a.bf16 && (a.dk == 64 || a.dk == 128) && (a.dv == 64 || a.dv == 128);
+}
+
+cudaError_t launch_fix_tc(const SplitWs& w, __nv_bfloat16* out,
+                          const ChunkArgs& a, const SplitGeom& g, dim3 grid,
+                          cudaStream_t stream) {
+  int* flag = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&flag),
+                                       g_split_timeout);
+  if (e != cudaSuccess) return e;
+  if (a.dk == 64)
+    return a.dv == 64 ? launch_fix_tc_t<64, 64>(w, out, a, g, grid, flag, stream)
+                      : launch_fix_tc_t<64, 128>(w, out, a, g, grid, flag, stream);
+  return a.dv == 64 ? launch_fix_tc_t<128, 64>(w, out, a, g, grid, flag, stream)
+                    : launch_fix_tc_t<128, 128>(w, out, a, g, grid, flag, stream);
+}
+
 template <typename K>
 cudaError_t set_smem(K kernel, size_t bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -488,9 +658,14 @@ cudaError_t run_split(const ChunkArgs& a, const SplitGeom& g, void* workspace,
   const size_t sms = 4 * ((size_t)dk * kScanTp + (size_t)dk * (dk + 1));
   if ((e = set_smem(split_scan_kernel, sms)) != cudaSuccess) return e;
   split_scan_kernel<<<dim3(H, dv / kScanTile), kThreads, sms, stream>>>(
-      w, a.final_state, g.k, H, dk, dv);
+      w, a.final_state, g.k, H, dk, dv, fix_on_tensor_cores(a) ? 1 : 0);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const unsigned nblk = (unsigned)((a.T - g.Ls + C - 1) / C);
+  if constexpr (std::is_same<IO, __nv_bfloat16>::value) {
+    if (fix_on_tensor_cores(a))
+      return launch_fix_tc(w, static_cast<IO*>(a.out), a, g, dim3(nblk, H),
+                           stream);
+  }
   return launch_fix<IO>(w, static_cast<IO*>(a.out), a, g, dim3(nblk, H),
                         stream);
 }
@@ -506,6 +681,16 @@ int split_auto_segments(const ChunkArgs& a, int num_sms) {
   int k = 1;
   while (k < 64 && (2 * (k + 1) - 1) * per_seg <= num_sms) ++k;
   return k;
+}
+
+cudaError_t split_take_timeout(cudaStream_t stream, int* flag) {
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return e;
+  int zero = 0;
+  if ((e = cudaMemcpyFromSymbol(flag, g_split_timeout, sizeof(int))) !=
+      cudaSuccess)
+    return e;
+  return cudaMemcpyToSymbol(g_split_timeout, &zero, sizeof(int));
 }
 
 SplitGeom split_geometry(const ChunkArgs& a, int n_segments) {
