@@ -18,8 +18,9 @@
 //       the last step gives the final state;
 //   (4) correction: o_t += S_in(j)^T X_t for the tokens of segments 1..n-1.
 // Steps (1) and (2) run the library's own prefill kernels (fused or
-// four-stage, as kda_chunk_fwd would pick for their shapes); (3) and (4) are
-// the fp32 kernels below.
+// four-stage, as kda_chunk_fwd would pick for their shapes); (3) is an fp32
+// kernel below, and (4) a tcgen05 product for bf16 io with d in {64, 128}
+// (an fp32 register-blocked product otherwise).
 #include <mutex>
 #include <type_traits>
 

@@ -378,11 +378,14 @@ KDA_API kda_status kda_chunk_bwd_plan(const kda_shape* shape, int packed,
  *   3. scans: S_in(1) = S_end(0), S_in(j+1) = M_end(j) S_in(j) + S_end|0(j);
  *      the last step writes final_state;
  *   4. adds S_in(j)^T (M_t^T q_t) to the outputs of segments 1..n-1.
- * Steps 1 and 2 run the path kda_chunk_fwd picks for their shapes; steps 3
- * and 4 are fp32.  Segments are ceil(chunks / n_segments) chunks long (the
+ * Steps 1 and 2 run the path kda_chunk_fwd picks for their shapes.  Step 3
+ * is fp32.  Step 4 runs on the tensor cores (bf16 operands, fp32
+ * accumulation) for bf16 io with d_k, d_v in {64, 128}, and in fp32
+ * otherwise.  Segments are ceil(chunks / n_segments) chunks long (the
  * last takes the rest; n_segments above the chunk count is reduced to it).
- * With bf16 io, step 1's outputs and step 2's M_t^T q_t pass through bf16:
- * the result agrees with kda_chunk_fwd to the bf16 tolerance, not bit for bit.
+ * With bf16 io, step 1's outputs, step 2's M_t^T q_t and step 4's S_in pass
+ * through bf16: the result agrees with kda_chunk_fwd to the bf16 tolerance,
+ * not bit for bit.
  *
  * When it pays: steps 1 and 2 run 2n - 1 chains of T/n tokens side by side,
  * so the call shortens the serial chain when one sequence leaves most SMs
