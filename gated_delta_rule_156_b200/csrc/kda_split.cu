@@ -428,7 +428,7 @@ __global__ void __launch_bounds__(128)
   const int L = min(C, T - t0);
   const int j = min(t0 / Ls, k - 1);
   // B = S_in(j) in bf16, already in its swizzled N-major panels: one bulk
-  // copy (no multicast) completing on bar[0], while the threads stage A
+  // single-destination copy completing on bar[0], while the threads stage A
   if (tid == 0) {
     mbar_init(bar, 1);
     mbar_init(bar + 1, 1);
