@@ -493,32 +493,71 @@ def run_kda(args, world, rank, local):
     del gdo
 
     # ---- end to end through the public API with host buffers ------------
+    # Every step uploads its inputs from pinned host memory, runs the prefill
+    # and downloads its outputs; two buffer sets and three streams (upload,
+    # compute, download, ordered by events) let step i+1's upload overlap
+    # step i's compute and download, as a serving loop would.
     host = {n: d[n].cpu().pin_memory() for n in
             ("q", "k", "v", "log_alpha", "beta")}
-    dev_in = {n: torch.empty_like(d[n]) for n in host}
-    out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-    fin_h = torch.empty(fin.shape, dtype=fin.dtype, pin_memory=True)
+    dev_in = [{n: torch.empty_like(d[n]) for n in host} for _ in range(2)]
+    outs_e = [torch.empty_like(out) for _ in range(2)]
+    fins_e = [torch.empty_like(fin) for _ in range(2)]
+    out_h = [torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+             for _ in range(2)]
+    fin_h = [torch.empty(fin.shape, dtype=fin.dtype, pin_memory=True)
+             for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = out_h.numel() * out_h.element_size() + fin_h.numel() * fin_h.element_size()
+    d2h = out_h[0].numel() * out_h[0].element_size() + \
+        fin_h[0].numel() * fin_h[0].element_size()
+    s_up = torch.cuda.Stream(dev)
+    s_down = torch.cuda.Stream(dev)
+    ev_up = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_down = [torch.cuda.Event() for _ in range(2)]
 
-    def e2e(_i):
-        for n, t in host.items():
-            dev_in[n].copy_(t, non_blocking=True)
-        K.chunk_fwd(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["log_alpha"],
-                    dev_in["beta"], None, None, chunk=C, out=out,
-                    final_state=fin)
-        out_h.copy_(out, non_blocking=True)
-        fin_h.copy_(fin, non_blocking=True)
+    def e2e(i):
+        sl = i % 2
+        s_up.wait_event(ev_comp[sl])  # the compute that last read this set
+        with torch.cuda.stream(s_up):
+            for n, t in host.items():
+                dev_in[sl][n].copy_(t, non_blocking=True)
+        ev_up[sl].record(s_up)
+        stream.wait_event(ev_up[sl])
+        stream.wait_event(ev_down[sl])  # the download that last read outputs
+        x = dev_in[sl]
+        K.chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], None,
+                    None, chunk=C, out=outs_e[sl], final_state=fins_e[sl],
+                    stream=stream)
+        ev_comp[sl].record(stream)
+        s_down.wait_event(ev_comp[sl])
+        with torch.cuda.stream(s_down):
+            out_h[sl].copy_(outs_e[sl], non_blocking=True)
+            fin_h[sl].copy_(fins_e[sl], non_blocking=True)
+        ev_down[sl].record(s_down)
 
-    e2e_steps = max(1, min(args.steps, 10))
-    for i in range(min(args.warmup, 3)):
+    def e2e_timed(steps):
+        t0, t1 = (torch.cuda.Event(enable_timing=True) for _ in range(2))
+        t0.record(stream)
+        s_up.wait_event(t0)
+        s_down.wait_event(t0)
+        for i in range(steps):
+            e2e(i)
+        for sl in range(2):  # every download inside the timed region
+            stream.wait_event(ev_down[sl])
+        t1.record(stream)
+        t1.synchronize()
+        return t0.elapsed_time(t1)
+
+    e2e_steps = max(2, min(args.steps, 10))
+    for i in range(min(args.warmup, 4)):
         e2e(i)
     torch.cuda.synchronize()
     barrier(world)
-    ems, _ = timed(e2e, e2e_steps, stream)
+    ems = e2e_timed(e2e_steps)
     barrier(world)
     ems = max_over_ranks(ems, world)
     e2e_value = world * B * T / (ems / e2e_steps * 1e-3)
+    del dev_in, outs_e, fins_e
 
     clk = clocks.stop()
 
@@ -587,7 +626,9 @@ def run_kda(args, world, rank, local):
             "prefill_fused_prologue": fused_prologue,
             "e2e": {"value": e2e_value, "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "steps": e2e_steps},
+                    "steps": e2e_steps,
+                    "pipeline": "two buffer sets; step i+1's upload overlaps "
+                                "step i's compute and download"},
             "gpu_launches": n_kernels * args.steps,
             "gpu_launches_note": "kernel launches inside the headline prefill "
                                  "timed region (one fused kernel per call)",
