@@ -40,6 +40,13 @@ constexpr int kThreads = 256;
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// The output correction runs on the tensor cores for bf16 io with d_k, d_v in
+// {64, 128}, in tiles of kFixTile tokens (the MMA's M).
+constexpr int kFixTile = 128;
+bool fix_on_tensor_cores(const ChunkArgs& a) {
+  return a.bf16 && (a.dk == 64 || a.dk == 128) && (a.dv == 64 || a.dv == 128);
+}
+
 struct SplitWs {
   int32_t* cu_val;   // [k + 1] segment offsets of the value run
   int32_t* cu_tr;    // [k] offsets of the transition run (segments 1..k-1)
@@ -403,11 +410,12 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 // (4') The correction on the tensor cores, for bf16 io with d_k, d_v in
-// {64, 128}: per (chunk, head) one M = 128, N = d_v, K = d_k product of the
-// chunk's X rows (K-major, 128-byte-swizzled panels of 128 rows; rows past the
-// chunk are never read back) and S_in(j) rounded to bf16 (MN-major panels of
-// d_k rows), accumulated in TMEM.  The two warps that own TMEM lanes 0-63
-// then add the rows into the output, 16 bytes at a time.  The MMA wait is
+// {64, 128}: per (128-token tile, head) one M = 128, N = d_v, K = d_k product
+// of the tile's X rows (K-major, 128-byte-swizzled panels; rows past the
+// sequence are zero) and S_in(j) rounded to bf16 (MN-major panels of d_k
+// rows), accumulated in TMEM.  Segments are whole tiles on this path, so a
+// tile never straddles two.  Each thread owns one TMEM lane, i.e. one token,
+// and adds its row into the output 16 bytes at a time.  The MMA wait is
 // bounded; if it gives up the block writes nothing and raises the library's
 // timeout flag.
 template <int DK, int DV>
@@ -424,8 +432,8 @@ __global__ void __launch_bounds__(128)
   constexpr uint32_t kBbytes = (DV / 64) * kBpanel;
   uint64_t* bar = reinterpret_cast<uint64_t*>(sB + kBbytes);  // [0] B, [1] MMA
   uint32_t* tbase = reinterpret_cast<uint32_t*>(bar + 2);
-  const int t0 = Ls + blockIdx.x * C, h = blockIdx.y, tid = threadIdx.x;
-  const int L = min(C, T - t0);
+  const int t0 = Ls + blockIdx.x * kFixTile, h = blockIdx.y, tid = threadIdx.x;
+  const int L = min(kFixTile, T - t0);
   const int j = min(t0 / Ls, k - 1);
   // B = S_in(j) in bf16, already in its swizzled N-major panels: one bulk
   // single-destination copy completing on bar[0], while the threads stage A
@@ -445,7 +453,7 @@ __global__ void __launch_bounds__(128)
   // A[r][c] = X[r][c]: every load of the thread in flight before its stores
   const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(w.x);
   {
-    constexpr int NA = 64 * (DK / 8) / 128;
+    constexpr int NA = kFixTile * (DK / 8) / 128;
     uint4 v[NA];
 #pragma unroll
     for (int u = 0; u < NA; ++u) {
@@ -494,7 +502,7 @@ __global__ void __launch_bounds__(128)
   if (ok) ok = mbar_wait(bar + 1, 0);
   tc_fence_after();
   const int warp = tid >> 5;
-  if (warp < 2) {  // TMEM lane = row of the chunk
+  {  // TMEM lane = row of the tile
     const int r = tid;
 #pragma unroll
     for (int c = 0; c < DV; c += 32) {
@@ -534,9 +542,6 @@ cudaError_t launch_fix_tc_t(const SplitWs& w, __nv_bfloat16* out,
   return cudaGetLastError();
 }
 
-bool fix_on_tensor_cores(const ChunkArgs& a) {
-  return a.bf16 && (a.dk == 64 || a.dk == 128) && (a.dv == 64 || a.dv == 128);
-}
 
 cudaError_t launch_fix_tc(const SplitWs& w, __nv_bfloat16* out,
                           const ChunkArgs& a, const SplitGeom& g, dim3 grid,
@@ -663,9 +668,11 @@ cudaError_t run_split(const ChunkArgs& a, const SplitGeom& g, void* workspace,
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const unsigned nblk = (unsigned)((a.T - g.Ls + C - 1) / C);
   if constexpr (std::is_same<IO, __nv_bfloat16>::value) {
-    if (fix_on_tensor_cores(a))
-      return launch_fix_tc(w, static_cast<IO*>(a.out), a, g, dim3(nblk, H),
+    if (fix_on_tensor_cores(a)) {
+      const unsigned ntile = (unsigned)((a.T - g.Ls + kFixTile - 1) / kFixTile);
+      return launch_fix_tc(w, static_cast<IO*>(a.out), a, g, dim3(ntile, H),
                            stream);
+    }
   }
   return launch_fix<IO>(w, static_cast<IO*>(a.out), a, g, dim3(nblk, H),
                         stream);
@@ -705,7 +712,13 @@ SplitGeom split_geometry(const ChunkArgs& a, int n_segments) {
     return g;
   }
   g.Ls = ((nch + n - 1) / n) * C;
+  if (fix_on_tensor_cores(a))  // whole 128-token correction tiles per segment
+    g.Ls = (g.Ls + kFixTile - 1) / kFixTile * kFixTile;
   g.k = (a.T + g.Ls - 1) / g.Ls;
+  if (g.k <= 1) {
+    g.k = 1;
+    g.Ls = a.T;
+  }
   return g;
 }
 

@@ -381,8 +381,10 @@ KDA_API kda_status kda_chunk_bwd_plan(const kda_shape* shape, int packed,
  * Steps 1 and 2 run the path kda_chunk_fwd picks for their shapes.  Step 3
  * is fp32.  Step 4 runs on the tensor cores (bf16 operands, fp32
  * accumulation) for bf16 io with d_k, d_v in {64, 128}, and in fp32
- * otherwise.  Segments are ceil(chunks / n_segments) chunks long (the
- * last takes the rest; n_segments above the chunk count is reduced to it).
+ * otherwise.  Segments are ceil(chunks / n_segments) chunks long, rounded
+ * up to a multiple of 128 tokens when step 4 runs on the tensor cores; the
+ * last takes the rest, and fewer segments result when the rounding or the
+ * chunk count leaves fewer.
  * With bf16 io, step 1's outputs, step 2's M_t^T q_t and step 4's S_in pass
  * through bf16: the result agrees with kda_chunk_fwd to the bf16 tolerance,
  * not bit for bit.

@@ -225,8 +225,13 @@ def test_split_validation_and_plan(lib):
                                            torch.bfloat16, 4)
     assert seg == 4 and kern == 1 + 2 + 2 + 2 and ws > 0
     seg, kern, ws = K.chunk_fwd_split_plan(1000, 2, 64, 64, 64,
-                                           torch.bfloat16, 7)
+                                           torch.float32, 7)
     assert seg == 6  # 16 chunks in segments of 3
+    # bf16 with d in {64, 128}: segments rounded up to 128-token tiles
+    # (3 chunks = 192 tokens -> 256), so 4 segments
+    seg, kern, ws = K.chunk_fwd_split_plan(1000, 2, 64, 64, 64,
+                                           torch.bfloat16, 7)
+    assert seg == 4
     seg, kern, ws = K.chunk_fwd_split_plan(100, 2, 64, 64, 64,
                                            torch.bfloat16, 1)
     assert (seg, kern, ws) == (1, 1, 0)

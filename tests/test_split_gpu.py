@@ -82,14 +82,16 @@ def test_split_one_segment_is_chunk_fwd():
 
 
 def test_split_more_segments_than_chunks_and_short():
-    # 3 chunks asked to split 10 ways: three one-chunk segments; a sequence
-    # shorter than one chunk is not split at all
+    # 3 chunks asked to split 10 ways: one-chunk segments, rounded up to the
+    # 128-token tiles of the tensor-core correction (bf16, d = 64), so two
+    # segments; a sequence shorter than one chunk is not split at all
     for T, n in ((150, 10), (40, 4)):
         d = case(T, 2, 64, 64, "bf16", seed=T)
         out, fin = K.chunk_fwd_split(d["q"], d["k"], d["v"], d["log_alpha"],
                                      d["beta"], d["initial_state"], n_segments=n)
         against_oracle(d, out, fin, PY.TOL_BF16)
-    assert K.chunk_fwd_split_plan(150, 2, 64, 64, 64, torch.bfloat16, 10)[0] == 3
+    assert K.chunk_fwd_split_plan(150, 2, 64, 64, 64, torch.bfloat16, 10)[0] == 2
+    assert K.chunk_fwd_split_plan(150, 2, 64, 64, 64, torch.float32, 10)[0] == 3
     assert K.chunk_fwd_split_plan(40, 2, 64, 64, 64, torch.bfloat16, 4)[0] == 1
 
 
