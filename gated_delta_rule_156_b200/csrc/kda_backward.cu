@@ -25,12 +25,20 @@
 //   dk  = dKt e^g + dKb e^-g,  dq = dQt e^g
 //   dg  = dKt * Kt + dQt * Qt - dKb * Kb  (+ gam * d gam on the last row)
 //   dlog_alpha = reverse cumulative sum of dg within the chunk
-// The forward quantities come from stages (1)-(3) of the four-stage forward
-// (g, W, Delta, chunk-start states).  A prep kernel forms Kt, Kb, Qt, M, P and
-// Tm per chunk; the reverse chain runs per (sequence, head, 32-column d_v
-// tile); the remaining products are batched small matrix products over every
-// (chunk, head) with all operands staged in shared memory; a last kernel
-// combines them into the input gradients.  Channel gate, no input prologue.
+// Launch order:
+//   - stage (1) of the four-stage forward (g);
+//   - a prep kernel per (chunk, head): Kt, Kb, Qt, b Kt, P and Tm, plus the
+//     forward's own W, U and Kh, so the forward's stage (2) is not run;
+//   - the forward's state pass (stage 3): Delta and every chunk-start state;
+//   - the two products that do not depend on dS, Qt^T dO and P^T dO;
+//   - the reverse chain per (sequence, head, 32-column d_v tile), which
+//     keeps only dDelta and the dS update in its serial loop and takes
+//     gam * d gam = rowsum(S_next * dS_C) from the next chunk's start state
+//     (S_next = Diag(gam)(S_0 + Kb^T Delta));
+//   - the remaining products, batched over every (chunk, head) with their
+//     operands staged in shared memory and merged into multi-term launches;
+//   - a last kernel that combines them into the input gradients.
+// Channel gate, no input prologue.
 #include "kda_common.cuh"
 #include "kda_internal.h"
 #include "kda_inverse.cuh"
