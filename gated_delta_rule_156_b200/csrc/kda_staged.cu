@@ -9,15 +9,16 @@
 //   g_r  = sum_{i<=r} l_i                          (1) cumulative log-decay
 //   Kt   = k * exp(g), Kb = k * exp(-g), Qt = q * exp(g), Kh = k * exp(g_C - g)
 //   A    = strictly_lower(Diag(b) Kt Kb^T)         (2) intra-chunk factors
-//   Tm   = (I + A)^-1                              forward substitution
+//   Tm   = (I + A)^-1                              by recursive doubling
 //   W    = Tm Diag(b) Kt,  U = Tm Diag(b) V
 //   D    = U - W S_0                               (3) state pass (serial)
 //   S_C  = Diag(exp(g_C)) S_0 + Kh^T D
 //   O    = Qt S_0 + lower_incl(Qt Kb^T) D           (4) output
 // Each stage is its own kernel with its inputs and outputs in an HBM
 // workspace; stages (1), (2), (4) are parallel over (chunk, head), stage (3)
-// over (sequence, head, 32-column tile of d_v).  This is the all-fp32 mode and
-// the reference decomposition the fused tensor-core kernel is built from.
+// over (sequence, head, 64-column tile of d_v; 32 when d_v = 32), and stage
+// (4) over 32-column tiles.  This is the all-fp32 mode and the reference
+// decomposition the fused tensor-core kernel is built from.
 #include "kda_common.cuh"
 #include "kda_internal.h"
 #include "kda_inverse.cuh"
