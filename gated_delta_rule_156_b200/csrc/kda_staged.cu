@@ -9,7 +9,8 @@
 //   g_r  = sum_{i<=r} l_i                          (1) cumulative log-decay
 //   Kt   = k * exp(g), Kb = k * exp(-g), Qt = q * exp(g), Kh = k * exp(g_C - g)
 //   A    = strictly_lower(Diag(b) Kt Kb^T)         (2) intra-chunk factors
-//   Tm   = (I + A)^-1                              by recursive doubling
+//   Tm   = (I + A)^-1    blocked: 16 x 16 diagonal blocks by forward
+//                        substitution, the blocks below by recursive doubling
 //   W    = Tm Diag(b) Kt,  U = Tm Diag(b) V
 //   D    = U - W S_0                               (3) state pass (serial)
 //   S_C  = Diag(exp(g_C)) S_0 + Kh^T D
