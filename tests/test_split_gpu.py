@@ -120,3 +120,16 @@ def test_split_auto_segment_count():
                                  d["beta"], d["initial_state"], n_segments=0)
     assert K.device_status() == 0
     against_oracle(d, out, fin, PY.TOL_BF16)
+
+
+@pytest.mark.parametrize("dk,dv,C", [(64, 128, 32), (32, 128, 16), (128, 32, 64)])
+def test_split_bf16_other_paths(dk, dv, C):
+    # bf16 io off the fused path (C < 64, or d = 32): the value and transition
+    # runs take the four-stage pipeline; the correction runs on the tensor
+    # cores when d_k, d_v are in {64, 128} (first case) and in fp32 otherwise
+    d = case(613, 2, dk, dv, "bf16", seed=dk + dv + C)
+    out, fin = K.chunk_fwd_split(d["q"], d["k"], d["v"], d["log_alpha"],
+                                 d["beta"], d["initial_state"], n_segments=3,
+                                 chunk=C)
+    assert K.device_status() == 0
+    against_oracle(d, out, fin, PY.TOL_BF16)
