@@ -244,3 +244,46 @@ def test_split_validation_and_plan(lib):
                                   num_sms=148)[0] == 1
     assert K.chunk_fwd_split_plan(131072, 4, 64, 64, 64, torch.bfloat16, 0,
                                   num_sms=148)[0] == 19
+
+
+C_CALLER = r"""
+#include <stdio.h>
+#include "kda.h"
+int main(void) {
+  kda_shape s = {1, 64, 2, 48, 64, 64, 0, KDA_BF16};  /* d_k = 48 */
+  int kern = 0, path = 0, seg = 0;
+  size_t ws = 0;
+  if (kda_version() < 100) return 1;
+  if (kda_chunk_fwd_plan(&s, 0, 0, &path, &kern, &ws) != KDA_ERR_UNSUPPORTED)
+    return 2;
+  s.dk = 128;
+  s.dv = 128;
+  s.T = 131072;
+  s.H = 8;
+  if (kda_chunk_fwd_split_plan(&s, KDA_GATE_CHANNEL, 0, 148, &seg, &kern, &ws)
+      != KDA_OK || seg != 5)
+    return 3;
+  printf("%s\n", kda_status_string(KDA_OK));
+  return 0;
+}
+"""
+
+
+@pytest.mark.skipif(__import__("shutil").which("gcc") is None, reason="needs gcc")
+def test_plain_c_caller_links_and_runs(lib, tmp_path):
+    # the boundary is a C ABI: a C99 program includes include/kda.h, links
+    # libkda.so and calls its host-side entry points (no GPU needed)
+    import subprocess
+    from torch.utils.cpp_extension import CUDA_HOME
+    cuda_inc = os.path.join(CUDA_HOME or "/usr/local/cuda", "include")
+    src = tmp_path / "caller.c"
+    src.write_text(C_CALLER)
+    libdir = os.path.join(ROOT, "gated_delta_rule_156_b200")
+    exe = tmp_path / "caller"
+    subprocess.check_call(
+        ["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+         "-I", cuda_inc, str(src), "-L", libdir, "-lkda",
+         "-Wl,-rpath," + libdir, "-o", str(exe)])
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0, (out.returncode, out.stdout, out.stderr)
+    assert out.stdout.startswith("KDA_OK")
