@@ -241,8 +241,10 @@ KDA_API kda_status kda_recurrent_step_ex(const kda_shape* shape, int gate,
  *     reports it) exceeds KDA_NOALLOC_SCRATCH_BYTES return KDA_ERR_UNSUPPORTED
  *     before anything is launched.
  *   - First call on a device: it looks up the array's device address on the
- *     current device (cudaGetSymbolAddress) and caches it.  Make that first
- *     call before any stream capture.
+ *     current device (cudaGetSymbolAddress) and caches it until the process
+ *     exits.  Make that first call before any stream capture.  Resetting the
+ *     device (cudaDeviceReset, or any teardown of its primary context)
+ *     between calls is not supported: the cached address would be stale.
  *   - Sharing: every call on a device uses the same array, which keeps the
  *     last call's contents.  Nothing in it has to start at zero (each call
  *     writes every scratch byte before reading it).  Calls whose executions

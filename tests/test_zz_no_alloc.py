@@ -6,16 +6,15 @@ library's fixed device array; its results must equal those of
 kda_chunk_fwd_staged, which allocates its workspace per call.
 
 This file is collected last on purpose, so a stop-at-first-failure run has
-already run every other test before these."""
-import ctypes
-
+already run every other test before these.  The size limit is checked on
+the host; that check is exercised in fake_address_abi.py, in a process that
+sees no GPU."""
 import numpy as np
 import pytest
 import torch
 
 import kda_workloads as W
 import parity as PY
-from gated_delta_rule_156_b200 import build as kbuild
 from gated_delta_rule_156_b200 import kda as K
 
 DEV = "cuda"
@@ -58,16 +57,3 @@ def test_noalloc_matches_allocating_entry_point_twice():
                      PY.host64(ref_o), tol)
             PY.check(f"{name} call {call} state", PY.host64(fin),
                      PY.host64(ref_s), tol)
-
-
-def test_noalloc_rejects_requests_beyond_the_scratch_size():
-    # Validation and the size check happen on the host before any CUDA call,
-    # so fake (never dereferenced) device addresses are enough here.
-    kbuild.build()
-    lib = K.library()
-    shape = K.KdaShape(1, 1 << 20, 32, 128, 128, 64, 0, 0)  # ~1.9 GB needed
-    base = 0x7000_0000_0000
-    ptrs = [ctypes.c_void_p(base + i * (1 << 34)) for i in range(9)]
-    st = lib.kda_chunk_fwd_staged_noalloc(ctypes.byref(shape), *ptrs[:5],
-                                          None, None, ptrs[5], ptrs[6], None)
-    assert st == 2  # KDA_ERR_UNSUPPORTED
