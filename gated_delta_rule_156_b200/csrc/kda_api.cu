@@ -546,16 +546,23 @@ const char* kda_status_string(kda_status status) {
     case KDA_ERR_MISALIGNED: return "KDA_ERR_MISALIGNED: pointer not 16-byte aligned";
     case KDA_ERR_CUDA: return "KDA_ERR_CUDA: a CUDA call failed";
     case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT: a bounded device wait gave up";
+    case KDA_ERR_RANGE:
+      return "KDA_ERR_RANGE: a chunk's decay exceeded the supported range";
   }
   return "unknown kda_status";
 }
 
 kda_status kda_device_status(cudaStream_t stream) {
-  int flag = 0, split_flag = 0;
+  int flag = 0, split_flag = 0, range_fused = 0, range_staged = 0,
+      range_bwd = 0;
   cudaError_t e = kda::fused_take_timeout(stream, &flag);
   if (e == cudaSuccess) e = kda::split_take_timeout(stream, &split_flag);
+  if (e == cudaSuccess) e = kda::fused_take_range(stream, &range_fused);
+  if (e == cudaSuccess) e = kda::staged_take_range(stream, &range_staged);
+  if (e == cudaSuccess) e = kda::bwd_take_range(stream, &range_bwd);
   if (e != cudaSuccess) return cuda_fail(e);
-  return flag || split_flag ? KDA_ERR_TIMEOUT : KDA_OK;
+  if (flag || split_flag) return KDA_ERR_TIMEOUT;
+  return range_fused || range_staged || range_bwd ? KDA_ERR_RANGE : KDA_OK;
 }
 
 kda_status kda_selftest_timeout(int limit_us, cudaStream_t stream) {

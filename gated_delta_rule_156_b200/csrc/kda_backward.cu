@@ -45,6 +45,12 @@
 
 namespace kda {
 
+// Set when a chunk's decay exceeds the backward's range (read and cleared on
+// the host).  The backward keeps the chunk-start factorisation (k e^g and
+// k e^-g), which stays inside the fp32 range while |g_C| <= kBwdDecayMax.
+__device__ int g_bwd_range = 0;
+constexpr float kBwdDecayMax = 80.f;
+
 namespace {
 
 constexpr int kThreads = 256;
@@ -154,8 +160,10 @@ __global__ void __launch_bounds__(kThreads)
 
   for (int r = tid; r < C; r += kThreads)
     bs[r] = r < L ? beta[(size_t)(tok0 + r) * H + h] : 0.f;
-  for (int c = tid; c < dk; c += kThreads)
+  for (int c = tid; c < dk; c += kThreads) {
     gl[c] = g[((size_t)(tok0 + L - 1) * H + h) * dk + c];
+    if (fabsf(gl[c]) > kBwdDecayMax) atomicExch(&g_bwd_range, 1);
+  }
   __syncthreads();
   for (int idx = tid; idx < C * dk; idx += kThreads) {
     const int r = idx / dk, c = idx % dk;
@@ -966,6 +974,15 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
 constexpr int kBmmOps = 11;
 
 }  // namespace
+
+cudaError_t bwd_take_range(cudaStream_t stream, int* flag) {
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return e;
+  if ((e = cudaMemcpyFromSymbol(flag, g_bwd_range, sizeof(int))) != cudaSuccess)
+    return e;
+  const int zero = 0;
+  return cudaMemcpyToSymbol(g_bwd_range, &zero, sizeof(int));
+}
 
 size_t bwd_workspace_bytes(const BwdArgs& a) {
   size_t total = 0;

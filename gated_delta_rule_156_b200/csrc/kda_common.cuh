@@ -80,4 +80,19 @@ __device__ __forceinline__ bool locate_chunk(int cid, const int32_t* cu,
   return *len > 0;
 }
 
+// Reference point of the decay factorisation inside a chunk.  The products
+// A and P need exp(g_r - g_i) for i <= r, formed as exp(g_r - rho) *
+// exp(rho - g_i) from one operand per row and one per column.  With rho = 0
+// (the chunk start) the column factor exp(-g_i) grows like exp(|g_C|); with
+// rho = g_C / 2 both factors stay within exp(|g_C| / 2).  A channel whose
+// decay over the chunk is moderate keeps rho = 0 (its operands are then
+// exactly the chunk-start ones); a strong one moves to the middle.  Past
+// kDecayRangeMax even the middle reference overflows fp32, and the kernels
+// report the call through the device range flag.
+constexpr float kDecayRefMin = 60.f;
+constexpr float kDecayRangeMax = 160.f;
+__device__ __forceinline__ float decay_ref(float g_last) {
+  return fabsf(g_last) > kDecayRefMin ? 0.5f * g_last : 0.f;
+}
+
 }  // namespace kda

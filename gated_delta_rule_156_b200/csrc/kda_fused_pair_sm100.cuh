@@ -42,7 +42,9 @@ namespace kda {
 namespace pair {
 
 using namespace sm100;
-using ws::invert_unit_lower;
+using ws::invert_unit_lower_tc;
+using ws::kGcFloats;
+using ws::rescale_qt;
 using ws::kBarCons;
 using ws::kBarProd;
 using ws::kC;
@@ -172,8 +174,9 @@ struct PairLayout {
   static constexpr uint32_t s_kb = NP * 16384;      // Kb, two 8 KB panels
   static constexpr uint32_t s_pp = s_kb + 16384;    // P
   static constexpr uint32_t s_tp = s_pp + 8192;     // T'
-  static constexpr uint32_t s_gc = s_tp + 8192;     // exp(g_C), DK floats
-  static constexpr uint32_t copy_bytes = s_gc + DK * 4;
+  static constexpr uint32_t s_gc = s_tp + 8192;     // package vector
+  static constexpr uint32_t gc_bytes = kGcFloats<DK> * 4;
+  static constexpr uint32_t copy_bytes = s_gc + gc_bytes;
   static constexpr uint32_t slot = (copy_bytes + 1023) & ~1023u;
   // The package goes to the peer in three parts, each as soon as it exists
   // and the peer's slot is free: Qt, Kb, P and exp(g_C) (early), T' (after
@@ -181,7 +184,7 @@ struct PairLayout {
   // stays out (zero in every slot from the start).
   static constexpr uint32_t kb_bytes = DK == 64 ? 8192 : 16384;
   static constexpr uint32_t push_bytes =
-      NP * 8192 /* Qt */ + kb_bytes + 8192 /* P */ + DK * 4 + 8192 /* T' */ +
+      NP * 8192 /* Qt */ + kb_bytes + 8192 /* P */ + gc_bytes + 8192 /* T' */ +
       NP * 8192 /* W */;
   // producer-private
   static constexpr uint32_t afp = 2 * slot;         // 64 x kFS fp32
@@ -200,12 +203,13 @@ struct PairLayout {
   static constexpr uint32_t t_u = 64 + DK;
   static constexpr uint32_t t_d3 = 128 + DK;
   static constexpr uint32_t t_s = 192 + DK;
-  static_assert(t_s + 64 <= 512, "TMEM columns");
+  static constexpr uint32_t t_d3b = 256 + DK;  // MMA3/MMA5 of odd chunks
+  static_assert(t_d3b + 64 <= 512, "TMEM columns");
   static_assert(slot % 1024 == 0 && sop % 1024 == 0 && dop % 1024 == 0 &&
                     vbuf % 1024 == 0,
                 "swizzle atoms");
   static_assert(copy_bytes % 16 == 0 && push_bytes < (1u << 20), "push size");
-  static_assert((DK * 4) % 16 == 0, "exp(g_C) copy size");
+  static_assert(gc_bytes % 16 == 0, "package vector copy size");
   static_assert(bytes + 1024 <= 232448, "shared memory");
 };
 
@@ -241,6 +245,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 14);
   // q/k loads issued per slot: [0..1] by the producer, [2..3] by the consumer
   int* issued = reinterpret_cast<int*>(bars + 15);
+  // the consumer's four warps have written the next chunk's bf16 state
+  uint64_t* bar_sop = bars + 17;
 
   const int tid = threadIdx.x, warp = tid >> 5;
   const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
@@ -269,6 +275,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mbar_init(bar_m1, 1);
     mbar_init(bar_m2, 1);
     mbar_init(bar_cm, 1);
+    mbar_init(bar_sop, 4);
     *abort_flag = 0;
     for (int i = 0; i < 4; ++i) issued[i] = 0;
     fence_mbar_init();
@@ -416,7 +423,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                        pbar);
         copy_to_peer(pdst + Lay::s_kb, slot + Lay::s_kb, Lay::kb_bytes, pbar);
         copy_to_peer(pdst + Lay::s_pp, slot + Lay::s_pp, 8192, pbar);
-        copy_to_peer(pdst + Lay::s_gc, slot + Lay::s_gc, DK * 4, pbar);
+        copy_to_peer(pdst + Lay::s_gc, slot + Lay::s_gc, Lay::gc_bytes, pbar);
         sent_early = true;
       };
       if (copier) slot_ok = sent_early = sent_tp = false;
@@ -472,11 +479,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           st_chunks<4>(pp, rr, 4 * colh, v);
         }
       }
+      // MMA1 has read Qt: back to the chunk-start q e^g where rho != 0
+      if (gc[2 * DK] != 0.f) rescale_qt<Lay::NP>(kq, gc + DK, t);
       tc_fence_before();
-      fence_proxy_async();  // P, to the copy engine
+      fence_proxy_async();  // P and Qt, to the copy engine
       named_sync(kBarProd, kProd);
 
-      invert_unit_lower(afp, tfp, reinterpret_cast<float*>(sm + Lay::msc), t);
+      invert_unit_lower_tc(afp, tfp, reinterpret_cast<float*>(sm + Lay::msc), t);
 
       {  // T' = Tm Diag(beta), rows masked to the lower triangle
         const int rr = t & 63, qc = t >> 6;
@@ -521,12 +530,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      if (row_t < 64) {  // W rows (bf16) over the Kt rows of the slot
+      if (row_t < 64) {  // W rows (bf16) over the Kt rows of the slot:
+        // T' (k e^(g-rho)) scaled by exp(rho) per column = T' (k e^g)
 #pragma unroll
         for (int jj = 0; jj < DK / 64; ++jj) {
           const int hh = colh * (DK / 64) + jj;
           float v[32];
           tmem_ld32(tmem + lane_base + Lay::t_w + 32 * hh, v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] *= gc[DK + 32 * hh + i];
           st_chunks<4>(kq + (hh >> 1) * 16384, row_t, 4 * (hh & 1), v);
         }
       }
@@ -594,6 +606,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     v_issued = nch > 0 ? 1 : 0;
     uint32_t ph_cm = 0;
     int n = 0;
+    // Per chunk n: thread 0 issues U = T' V and MMA3 as soon as the package,
+    // V and the bf16 state S_n are in place; Delta; MMA4 and MMA5; then the
+    // state S_(n+1) = exp(g_C) S is written as the bf16 operand first (the
+    // four warps announce it on bar_sop, which releases the next MMA3) and
+    // back to TMEM after, and the outputs of chunk n are stored from their
+    // TMEM buffer (two buffers, alternating by chunk) while the next MMA3
+    // runs.
     for (; n < nch; ++n) {
       const int s = ((n + (int)r) >> 1) & 1;
       const bool own = (n & 1) == (int)r;
@@ -606,6 +625,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       uint8_t* tp = slot + Lay::s_tp;
       const float* gc = reinterpret_cast<const float*>(slot + Lay::s_gc);
       uint8_t* vb = vbuf + (n & 1) * 8192;
+      const uint32_t d3 = (n & 1) ? Lay::t_d3b : Lay::t_d3;
       if (n + 1 < nch) {  // V of the next chunk (its buffer was freed by n - 1)
         if (c == 0) issue_v(n + 1);
         v_issued = n + 2;
@@ -613,34 +633,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // own chunk j = n >> 1 is the (j >> 1)-th own use of its slot; peer
       // chunk i = n >> 1 the (i >> 1)-th peer use
       const uint32_t par = (uint32_t)(n >> 2) & 1u;
-      bool ok = wait_cluster((own ? full : pfull) + s, par, abort_flag);
-      ok = ok && wait_or_abort<false>(bar_v + (n & 1), (uint32_t)(n >> 1) & 1u,
-                                      abort_flag);
-      if (named_sync_or(kBarCons, kCons, !ok)) {
-        failed = true;
-        break;
-      }
-      tc_fence_after();
-
-      // ---- U = T' V ; [W; Qt] . S
-      if (c == 0) {
-        if (!own) fence_proxy_async();  // the peer's stores, to the MMA reads
-        const uint32_t idesc = idesc_bf16(128, 64, false, true);
+      bool ok = true;
+      if (c == 0) {  // ---- U = T' V ; [W; Qt] . S
+        ok = wait_cluster((own ? full : pfull) + s, par, abort_flag);
+        ok = ok && wait_or_abort<false>(bar_v + (n & 1),
+                                        (uint32_t)(n >> 1) & 1u, abort_flag);
+        if (n > 0)
+          ok = ok && wait_or_abort<false>(bar_sop, (uint32_t)(n - 1) & 1u,
+                                          abort_flag);
+        if (ok) {
+          tc_fence_after();
+          if (!own) fence_proxy_async();  // the peer's stores, to the MMA reads
+          const uint32_t idesc = idesc_bf16(128, 64, false, true);
 #pragma unroll
-        for (int ks = 0; ks < kC / 16; ++ks)
-          mma_bf16(tmem + Lay::t_u, desc_sw128(smem_u32(tp) + ks * 32, 16, 1024),
-                   desc_sw128(smem_u32(vb) + ks * 2048, 8192, 1024), idesc,
-                   ks > 0);
+          for (int ks = 0; ks < kC / 16; ++ks)
+            mma_bf16(tmem + Lay::t_u,
+                     desc_sw128(smem_u32(tp) + ks * 32, 16, 1024),
+                     desc_sw128(smem_u32(vb) + ks * 2048, 8192, 1024), idesc,
+                     ks > 0);
 #pragma unroll
-        for (int ks = 0; ks < DK / 16; ++ks)
-          mma_bf16(tmem + Lay::t_d3,
-                   desc_sw128(smem_u32(kq) + (ks >> 2) * 16384 + (ks & 3) * 32,
-                              16, 1024),
-                   desc_sw128(smem_u32(sop) + ks * 2048, 8192, 1024), idesc,
-                   ks > 0);
-        mma_commit(bar_cm);
+          for (int ks = 0; ks < DK / 16; ++ks)
+            mma_bf16(tmem + d3,
+                     desc_sw128(smem_u32(kq) + (ks >> 2) * 16384 + (ks & 3) * 32,
+                                16, 1024),
+                     desc_sw128(smem_u32(sop) + ks * 2048, 8192, 1024), idesc,
+                     ks > 0);
+          mma_commit(bar_cm);
+        } else {
+          raise_abort();  // the other threads leave their wait below
+        }
       }
-      ok = wait_or_abort<false>(bar_cm, ph_cm, abort_flag);
+      ok = ok && wait_or_abort<false>(bar_cm, ph_cm, abort_flag);
       ph_cm ^= 1;
       if (named_sync_or(kBarCons, kCons, !ok)) {
         failed = true;
@@ -654,13 +677,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int hf = 0; hf < 2; ++hf) {
           float uu[32], wsv[32];
           tmem_ld32(tmem + lane_base + Lay::t_u + 32 * hf, uu);
-          tmem_ld32(tmem + lane_base + Lay::t_d3 + 32 * hf, wsv);
+          tmem_ld32(tmem + lane_base + d3 + 32 * hf, wsv);
 #pragma unroll
           for (int i = 0; i < 32; ++i) uu[i] -= wsv[i];
           st_chunks<4>(dop, c, 4 * hf, uu);
         }
       }
       const float gamma = owns_state ? gc[c] : 1.f;
+      if (owns_state && gc[2 * DK] != 0.f) {
+        // S_C = e^(g_C - rho) (e^rho S_0 + Kb^T Delta): pre-scale the state
+        const float er = gc[DK + c];
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          float v[32];
+          tmem_ld32(tmem + lane_base + Lay::t_s + 32 * hf, v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] *= er;
+          tmem_st32(tmem + lane_base + Lay::t_s + 32 * hf, v);
+        }
+        tmem_wait_st();
+      }
       tc_fence_before();
       fence_proxy_async();
       named_sync(kBarCons, kCons);
@@ -675,7 +711,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const uint64_t bd = desc_sw128(smem_u32(dop) + ks * 2048, 8192, 1024);
           mma_bf16(tmem + Lay::t_s,
                    desc_sw128(smem_u32(kb) + ks * 2048, 8192, 1024), bd, i4, 1u);
-          mma_bf16(tmem + Lay::t_d3,
+          mma_bf16(tmem + d3,
                    desc_sw128(smem_u32(pp) - 8192 + ks * 32, 16, 1024), bd, i5,
                    1u);
         }
@@ -697,13 +733,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
       }
 
-      // ---- outputs (rows 64-127) and the state rescale by exp(g_C)
+      // ---- S <- exp(g_C) S: the bf16 operand of the next MMA3 first, then
+      // TMEM (the store completes before the next MMA4 is issued)
+      if (owns_state) {
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          float v[32];
+          tmem_ld32(tmem + lane_base + Lay::t_s + 32 * hf, v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] *= gamma;
+          st_chunks<4>(sop, c, 4 * hf, v);
+          tmem_st32(tmem + lane_base + Lay::t_s + 32 * hf, v);
+        }
+      }
+      fence_proxy_async();
+      tc_fence_before();
+      __syncwarp();
+      if ((c & 31) == 0) mbar_arrive(bar_sop);
+
+      // ---- outputs (rows 64-127 of this chunk's buffer), overlapping the
+      // next chunk's MMA3
       if (c >= 64) {
         const int rr = c - 64;
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
           float o[32];
-          tmem_ld32(tmem + lane_base + Lay::t_d3 + 32 * hf, o);
+          tmem_ld32(tmem + lane_base + d3 + 32 * hf, o);
           if (rr < L) {
             uint4* dst = reinterpret_cast<uint4*>(
                 p.out + ((size_t)(tok0 + rr) * p.H + h) * p.dv + j0 + 32 * hf);
@@ -719,21 +774,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (owns_state) {
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          float v[32];
-          tmem_ld32(tmem + lane_base + Lay::t_s + 32 * hf, v);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] *= gamma;
-          tmem_st32(tmem + lane_base + Lay::t_s + 32 * hf, v);
-          st_chunks<4>(sop, c, 4 * hf, v);
-        }
-        tmem_wait_st();
-      }
+      if (owns_state) tmem_wait_st();
       tc_fence_before();
-      fence_proxy_async();
-      named_sync(kBarCons, kCons);
     }
     if (failed) {
       if (c == 0) {

@@ -30,6 +30,9 @@ namespace kda {
 
 // Set by a kernel whose bounded wait gave up (read and cleared on the host).
 __device__ int g_fused_timeout = 0;
+// Set when a chunk's decay exceeds the factorisation's range (read and
+// cleared on the host).
+__device__ int g_fused_range = 0;
 
 namespace {
 
@@ -150,6 +153,16 @@ cudaError_t fused_take_timeout(cudaStream_t stream, int* flag) {
       cudaSuccess)
     return e;
   return cudaMemcpyToSymbol(g_fused_timeout, &zero, sizeof(int));
+}
+
+cudaError_t fused_take_range(cudaStream_t stream, int* flag) {
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return e;
+  int zero = 0;
+  if ((e = cudaMemcpyFromSymbol(flag, g_fused_range, sizeof(int))) !=
+      cudaSuccess)
+    return e;
+  return cudaMemcpyToSymbol(g_fused_range, &zero, sizeof(int));
 }
 
 cudaError_t launch_fused(const ChunkArgs& a, void* workspace,

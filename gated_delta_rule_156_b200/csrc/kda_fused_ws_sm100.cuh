@@ -22,7 +22,7 @@
 // device-side timeout flag and the tensor-map helper).
 #pragma once
 
-#include "kda_inverse.cuh"
+#include "kda_inverse_tc.cuh"
 
 namespace kda {
 namespace ws {
@@ -36,6 +36,11 @@ constexpr int kCons = 128;  // consumer threads (warps 8-11)
 constexpr int kThreads = kProd + kCons;
 constexpr int kBarProd = kBarInv, kBarCons = 2;  // named barrier ids
 static_assert(kProd == kInvThreads, "the inverse runs on the producer");
+
+// Floats of a chunk's package vector: exp(g_C - rho) and exp(rho) per
+// channel, the "some rho != 0" word, padding to 16 bytes.
+template <int DK>
+constexpr int kGcFloats = 2 * DK + 4;
 
 template <int DK>
 struct WsLayout {
@@ -57,7 +62,12 @@ struct WsLayout {
   static constexpr uint32_t sop = pp + 2 * 8192;            // S, DK rows
   static constexpr uint32_t dop = sop + DK * 128;           // Delta, 64 rows
   static constexpr uint32_t misc = dop + 8192;
-  static constexpr uint32_t bytes = misc + 2048;  // betas, gcs, barriers
+  // betas [2][64], package vectors [2][kGcFloats], barriers
+  static constexpr uint32_t gcs = 512;
+  static constexpr uint32_t bars = gcs + 2 * kGcFloats<DK> * 4;
+  static constexpr uint32_t bytes = misc + 3072;
+  static_assert(bars + 128 <= 3072, "misc area");
+  static_assert(bytes + 1024 <= 232448, "shared memory");
   static constexpr uint32_t tx_qk = 2 * NP * 8192;
   // TMEM columns: D1 (two buffers), W, U (two slots), D3, S
   static constexpr uint32_t t_d1 = 0;
@@ -172,6 +182,29 @@ __device__ __forceinline__ void ldg_f1_if(float& v, const float* p, bool pred) {
       : "r"((uint32_t)pred), "l"(p));
 }
 
+// Rows 64-127 (Qt) of the NP 64-column panels of a [Kt; Qt] operand, scaled
+// in place by exp(rho) per column (gr): Qt = q e^(g - rho) becomes the
+// chunk-start q e^g.  256 threads, 16 bytes at a time.
+template <int NP>
+__device__ __forceinline__ void rescale_qt(uint8_t* kq, const float* gr, int t) {
+#pragma unroll
+  for (int i = 0; i < 2 * NP; ++i) {
+    const int x = t + 256 * i;
+    const int pnl = x >> 9, rr = 64 + ((x & 511) >> 3), ch = x & 7;
+    uint4* p = reinterpret_cast<uint4*>(kq + pnl * 16384 + rr * 128 +
+                                        ((ch ^ (rr & 7)) << 4));
+    uint4 w = *p;
+    __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&w);
+    const float* f = gr + pnl * 64 + ch * 8;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 v = __bfloat1622float2(h2[j]);
+      h2[j] = __floats2bfloat162_rn(v.x * f[2 * j], v.y * f[2 * j + 1]);
+    }
+    *p = w;
+  }
+}
+
 template <int N>
 __device__ __forceinline__ void st_chunks(uint8_t* panel, int row, int c0,
                                           const float* v) {
@@ -189,10 +222,16 @@ __device__ __forceinline__ void st_chunks(uint8_t* panel, int row, int c0,
 
 // The producer prologue of one chunk, over all 256 producer threads: turns
 // the log(alpha) rows held in registers (raw gate logits with the prologue)
-// into the running decay g, writes exp(g_C) per channel to gc, and the
-// decay-scaled bf16 operands Kt = k e^g and Qt = q e^g (rows 0-63 and 64-127
-// of the [Kt; Qt] panel pkq) and Kb = k e^-g (panel pkb) from the raw q and k
-// rows at pq and pk.  Thread t owns channels 4 cg .. 4 cg + 3 of rows
+// into the running decay g and, with the per-channel reference rho =
+// decay_ref(g_C), writes the decay-scaled bf16 operands Kt = k e^(g-rho) and
+// Qt = q e^(g-rho) (rows 0-63 and 64-127 of the [Kt; Qt] panel pkq) and
+// Kb = k e^(rho-g) (panel pkb) from the raw q and k rows at pq and pk.  The
+// package vector gc (kGcFloats floats) receives exp(g_C - rho) per channel,
+// then exp(rho) per channel, then a nonzero word when some channel of the
+// chunk has rho != 0 (its Qt rows and W columns are then rescaled by exp(rho)
+// to the chunk-start operands, and its state pre-scaled, see rescale_qt and
+// the consumers).  A chunk whose decay leaves the supported range raises
+// g_fused_range.  Thread t owns channels 4 cg .. 4 cg + 3 of rows
 // rb RPT .. rb RPT + RPT - 1; rows at or past L are written as zeros.  pq and
 // pk may be the same bytes as the destination rows (in-place transform): each
 // element is read and rewritten by the same thread.  `red` is DK * NRB
@@ -248,10 +287,27 @@ __device__ __forceinline__ void prologue_rows(float4* la_reg, float* red,
     tot[0] += y.x; tot[1] += y.y; tot[2] += y.z; tot[3] += y.w;
   }
   constexpr float kLog2e = 1.4426950408889634f;
-  if (rb == 0)
-    *reinterpret_cast<float4*>(gc + 4 * cg) =
-        make_float4(ex2_approx(tot[0] * kLog2e), ex2_approx(tot[1] * kLog2e),
-                    ex2_approx(tot[2] * kLog2e), ex2_approx(tot[3] * kLog2e));
+  float rho[4];
+  bool shifted = false, out_of_range = false;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    rho[c] = decay_ref(tot[c]);
+    shifted |= rho[c] != 0.f;
+    out_of_range |= fabsf(tot[c]) > kDecayRangeMax;
+  }
+  if (t < 32) {  // warp 0 holds every channel (rb 0, and rb 1 when DK = 64)
+    const bool any = __any_sync(0xffffffffu, shifted);
+    if (rb == 0) {
+      *reinterpret_cast<float4*>(gc + 4 * cg) = make_float4(
+          ex2_approx((tot[0] - rho[0]) * kLog2e), ex2_approx((tot[1] - rho[1]) * kLog2e),
+          ex2_approx((tot[2] - rho[2]) * kLog2e), ex2_approx((tot[3] - rho[3]) * kLog2e));
+      *reinterpret_cast<float4*>(gc + DK + 4 * cg) = make_float4(
+          ex2_approx(rho[0] * kLog2e), ex2_approx(rho[1] * kLog2e),
+          ex2_approx(rho[2] * kLog2e), ex2_approx(rho[3] * kLog2e));
+      if (out_of_range) atomicExch(&g_fused_range, 1);
+    }
+    if (t == 0) gc[2 * DK] = any ? 1.f : 0.f;
+  }
 #pragma unroll
   for (int i = 0; i < RPT; ++i) {
     const int r = rb * RPT + i;
@@ -265,12 +321,12 @@ __device__ __forceinline__ void prologue_rows(float4* la_reg, float* red,
     if (GATE == kGateChannel) {
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        const float x = g[c] * kLog2e;
+        const float x = (g[c] - rho[c]) * kLog2e;
         e[c] = valid ? ex2_approx(x) : 0.f;
         ie[c] = valid ? ex2_approx(-x) : 0.f;
       }
     } else {  // one decay for the whole row: two exponentials per row
-      const float x = g[0] * kLog2e;
+      const float x = (g[0] - rho[0]) * kLog2e;
       const float e0 = !valid ? 0.f : GATE == kGateHead ? ex2_approx(x) : 1.f;
       const float i0 = !valid ? 0.f : GATE == kGateHead ? ex2_approx(-x) : 1.f;
 #pragma unroll
@@ -347,8 +403,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sop = sm + Lay::sop;
   uint8_t* dop = sm + Lay::dop;
   float* betas = reinterpret_cast<float*>(sm + Lay::misc);          // [2][64]
-  float* gcs = reinterpret_cast<float*>(sm + Lay::misc + 512);      // [2][DK]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Lay::misc + 1536);
+  float* gcs = reinterpret_cast<float*>(sm + Lay::misc + Lay::gcs);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Lay::misc + Lay::bars);
+  constexpr int GCF = kGcFloats<DK>;
   uint64_t* bar_in = bars + 0;
   uint64_t* bar_v = bars + 1;
   uint64_t* bar_m1 = bars + 2;  // [2] MMA1 into D1 buffer b
@@ -468,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool has_next = m + 1 < nch;
       uint8_t* kq = sm + Lay::kq + s * Lay::kq_stride;
       uint8_t* kb = sm + Lay::kb + s * 16384;
-      float* gc = gcs + s * DK;
+      float* gc = gcs + s * GCF;
       if (t < kC) betas[s * 64 + t] = beta_next;
       beta_next = 0.f;
       ldg_f1_if(beta_next, p.beta + (size_t)(tok0 + kC + t) * p.H + h,
@@ -536,10 +593,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           st_chunks<4>(pp, r, 4 * colh, v);
         }
       }
+      // MMA1 has read Qt: back to the chunk-start q e^g where rho != 0
+      if (gcs[s * GCF + 2 * DK] != 0.f) rescale_qt<Lay::NP>(kq, gcs + s * GCF + DK, t);
       tc_fence_before();
       named_sync(kBarProd, kProd);
 
-      invert_unit_lower(afp, tfp, reinterpret_cast<float*>(sm + Lay::msc), t);
+      invert_unit_lower_tc(afp, tfp, reinterpret_cast<float*>(sm + Lay::msc), t);
 
       {  // T' = Tm Diag(beta), rows masked to the lower triangle
         const int r = t & 63, qc = t >> 6;
@@ -596,12 +655,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         issue_v(tok0 + kC);
         v_pending = true;
       }
-      if (row_t < 64) {  // W rows (bf16) over the Kt rows of the slot
+      if (row_t < 64) {  // W rows (bf16) over the Kt rows of the slot:
+        // T' (k e^(g-rho)) scaled by exp(rho) per column = T' (k e^g)
+        const float* gr = gcs + s * GCF + DK;
 #pragma unroll
         for (int j = 0; j < DK / 64; ++j) {
           const int hh = colh * (DK / 64) + j;
           float v[32];
           tmem_ld32(tmem + lane_base + Lay::t_w + 32 * hh, v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] *= gr[32 * hh + i];
           st_chunks<4>(kq + (hh >> 1) * 16384, row_t, 4 * (hh & 1), v);
         }
       }
@@ -697,7 +760,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           st_chunks<4>(dop, c, 4 * hf, uu);
         }
       }
-      const float gamma = owns_state ? gcs[s * DK + c] : 1.f;
+      const float gamma = owns_state ? gcs[s * GCF + c] : 1.f;
+      if (owns_state && gcs[s * GCF + 2 * DK] != 0.f) {
+        // S_C = e^(g_C - rho) (e^rho S_0 + Kb^T Delta): pre-scale the state
+        const float er = gcs[s * GCF + DK + c];
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          float v[32];
+          tmem_ld32(tmem + lane_base + Lay::t_s + 32 * hf, v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] *= er;
+          tmem_st32(tmem + lane_base + Lay::t_s + 32 * hf, v);
+        }
+        tmem_wait_st();
+      }
       tc_fence_before();
       fence_proxy_async();
       named_sync(kBarCons, kCons);

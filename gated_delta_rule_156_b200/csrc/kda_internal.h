@@ -131,6 +131,13 @@ int fused_kernel_count(const ChunkArgs& a);
 cudaError_t fused_take_timeout(cudaStream_t stream, int* flag);
 // The same for the sequence split's tensor-core correction (kda_split.cu).
 cudaError_t split_take_timeout(cudaStream_t stream, int* flag);
+// Synchronises `stream`, then reads and clears the flag a chunkwise kernel
+// sets when a chunk's total log-decay on some channel exceeds
+// kDecayRangeMax (the fused kernels, the four-stage pipeline and the
+// backward pass each keep their own).
+cudaError_t fused_take_range(cudaStream_t stream, int* flag);
+cudaError_t staged_take_range(cudaStream_t stream, int* flag);
+cudaError_t bwd_take_range(cudaStream_t stream, int* flag);
 // Diagnostic: one CTA whose bounded wait runs out after limit_us.
 cudaError_t launch_timeout_probe(int limit_us, cudaStream_t stream);
 cudaError_t launch_fused(const ChunkArgs& a, void* workspace,

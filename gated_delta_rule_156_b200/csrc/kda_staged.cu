@@ -9,6 +9,9 @@
 //   g_r  = sum_{i<=r} l_i                          (1) cumulative log-decay
 //   Kt   = k * exp(g), Kb = k * exp(-g), Qt = q * exp(g), Kh = k * exp(g_C - g)
 //   A    = strictly_lower(Diag(b) Kt Kb^T)         (2) intra-chunk factors
+// (A and lower_incl(Qt Kb^T) only need exp(g_r - g_i) for i <= r; they are
+// formed from k exp(g - rho) and k exp(rho - g) with the per-channel
+// reference rho of decay_ref, so strong gates stay inside the fp32 range.)
 //   Tm   = (I + A)^-1    blocked: 16 x 16 diagonal blocks by forward
 //                        substitution, the blocks below by recursive doubling
 //   W    = Tm Diag(b) Kt,  U = Tm Diag(b) V
@@ -25,6 +28,10 @@
 #include "kda_inverse.cuh"
 
 namespace kda {
+
+// Set when a chunk's decay exceeds the factorisation's range (read and
+// cleared on the host).
+__device__ int g_staged_range = 0;
 
 namespace {
 
@@ -177,18 +184,25 @@ __global__ void __launch_bounds__(kThreads)
   float* Msc = Tm + 64 * ws::kFS;  // [1024] scratch of the inverse
   float* bs = Msc + 1024;          // [C]
   float* gl = bs + C;              // [dk] g at the chunk's last row
+  float* rho = gl + dk;            // [dk] reference of the A factorisation
 
-  for (int c = tid; c < dk; c += kThreads)
+  for (int c = tid; c < dk; c += kThreads) {
     gl[c] = g[((size_t)(tok0 + L - 1) * H + h) * dk + c];
+    rho[c] = decay_ref(gl[c]);
+    if (fabsf(gl[c]) > kDecayRangeMax) atomicExch(&g_staged_range, 1);
+  }
   __syncthreads();
+  // Kt holds k exp(g - rho) and Kb k exp(rho - g): their products are the
+  // exact exp(g_r - g_i) factors of A; W is rescaled by exp(rho) below to the
+  // chunk-start Kt = k exp(g).
   for (int idx = tid; idx < C * dk; idx += kThreads) {
     const int r = idx / dk, c = idx % dk;
     float kt = 0.f, kb = 0.f;
     if (r < L) {
       const size_t gi = ((size_t)(tok0 + r) * H + h) * dk + c;
       const float kv = to_f32(k[gi]), gv = g[gi];
-      kt = kv * __expf(gv);
-      kb = kv * __expf(-gv);
+      kt = kv * __expf(gv - rho[c]);
+      kb = kv * __expf(rho[c] - gv);
       kh_out[gi] = kv * __expf(gl[c] - gv);
     }
     Kt[r * ldk + c] = kt;
@@ -284,7 +298,7 @@ __global__ void __launch_bounds__(kThreads)
         const size_t ru = ((size_t)(tok0 + r) * H + h) * dv;
 #pragma unroll
         for (int b = 0; b < 8; ++b) {
-          if (b < nw) w_out[rw + tj + 16 * b] = aw[a][b];
+          if (b < nw) w_out[rw + tj + 16 * b] = aw[a][b] * __expf(rho[tj + 16 * b]);
           if (b < nu) u_out[ru + tj + 16 * b] = au[a][b];
         }
       }
@@ -474,15 +488,21 @@ __global__ void __launch_bounds__(kThreads)
   float* P = Kb + C * ldk;        // [C][C]
   float* S = P + C * C;           // [dk][kDvTile]
   float* D = S + dk * kDvTile;    // [C][kDvTile]
+  float* rho = D + C * kDvTile;   // [dk] reference of the P factorisation
 
+  for (int c = tid; c < dk; c += kThreads)
+    rho[c] = decay_ref(g[((size_t)(tok0 + L - 1) * H + h) * dk + c]);
+  __syncthreads();
+  // Qt holds q exp(g - rho), Kb k exp(rho - g); the state rows are scaled by
+  // exp(rho) so that Qt S is the chunk-start q exp(g) S.
   for (int idx = tid; idx < C * dk; idx += kThreads) {
     const int r = idx / dk, c = idx % dk;
     float qt = 0.f, kb = 0.f;
     if (r < L) {
       const size_t gi = ((size_t)(tok0 + r) * H + h) * dk + c;
       const float gv = g[gi];
-      qt = to_f32(q[gi]) * __expf(gv);
-      kb = to_f32(k[gi]) * __expf(-gv);
+      qt = to_f32(q[gi]) * __expf(gv - rho[c]);
+      kb = to_f32(k[gi]) * __expf(rho[c] - gv);
     }
     Qt[r * ldk + c] = qt;
     Kb[r * ldk + c] = kb;
@@ -490,7 +510,7 @@ __global__ void __launch_bounds__(kThreads)
   const size_t cbase = ((size_t)cid * H + h) * dk * dv;
   for (int idx = tid; idx < dk * kDvTile; idx += kThreads) {
     const int c = idx / kDvTile, jj = idx % kDvTile;
-    S[idx] = s_chunks[cbase + (size_t)c * dv + j0 + jj];
+    S[idx] = s_chunks[cbase + (size_t)c * dv + j0 + jj] * __expf(rho[c]);
   }
   for (int idx = tid; idx < C * kDvTile; idx += kThreads) {
     const int r = idx / kDvTile, jj = idx % kDvTile;
@@ -554,7 +574,7 @@ cudaError_t run(const ChunkArgs& a, void* workspace, cudaStream_t stream,
     const dim3 grid((unsigned)nch, H);
 
     const size_t sm2 = 4 * ((size_t)2 * C * (dk + 1) + (size_t)C * dv +
-                            2 * 64 * ws::kFS + 1024 + C + dk);
+                            2 * 64 * ws::kFS + 1024 + C + 2 * dk);
     if ((e = set_smem(intra_kernel<IO>, sm2)) != cudaSuccess) return e;
     intra_kernel<IO><<<grid, kThreads, sm2, stream>>>(
         k, v, a.beta, w.g, w.w, w.u, w.kh, cu, w.chunk_off, a.n_seqs, a.T, H,
@@ -582,7 +602,7 @@ cudaError_t run(const ChunkArgs& a, void* workspace, cudaStream_t stream,
 
   if (nch > 0 && part == Part::kAll) {
     const size_t sm4 = 4 * (2 * (size_t)C * (dk + 1) + (size_t)C * C +
-                            (size_t)dk * kDvTile + (size_t)C * kDvTile);
+                            (size_t)dk * kDvTile + (size_t)C * kDvTile + dk);
     if ((e = set_smem(output_kernel<IO>, sm4)) != cudaSuccess) return e;
     output_kernel<IO><<<dim3((unsigned)nch, H, dv / kDvTile), kThreads, sm4,
                         stream>>>(q, k, w.g, w.u, w.s, out, cu, w.chunk_off,
@@ -621,6 +641,16 @@ cudaError_t launch_staged_part(const ChunkArgs& a, void* workspace,
   const Part part = state_pass ? Part::kStatePass : Part::kPrefix;
   return a.bf16 ? run<__nv_bfloat16>(a, workspace, stream, part)
                 : run<float>(a, workspace, stream, part);
+}
+
+cudaError_t staged_take_range(cudaStream_t stream, int* flag) {
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return e;
+  if ((e = cudaMemcpyFromSymbol(flag, g_staged_range, sizeof(int))) !=
+      cudaSuccess)
+    return e;
+  const int zero = 0;
+  return cudaMemcpyToSymbol(g_staged_range, &zero, sizeof(int));
 }
 
 cudaError_t launch_staged(const ChunkArgs& a, void* workspace,

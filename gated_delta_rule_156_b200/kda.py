@@ -15,7 +15,8 @@ from . import build as _build
 KDA_OK = 0
 KDA_BF16, KDA_F32 = 0, 1
 STATUS_NAMES = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED",
-                3: "KDA_ERR_MISALIGNED", 4: "KDA_ERR_CUDA", 5: "KDA_ERR_TIMEOUT"}
+                3: "KDA_ERR_MISALIGNED", 4: "KDA_ERR_CUDA", 5: "KDA_ERR_TIMEOUT",
+                6: "KDA_ERR_RANGE"}
 
 # Entry points declared in include/kda.h (kept in sync by tests).
 EXPORTS = ("kda_chunk_fwd", "kda_chunk_fwd_staged", "kda_recurrent_step",

@@ -40,9 +40,17 @@
  *     before anything is launched; no exception crosses the ABI.
  *   - Supported sizes: d_k, d_v in {32, 64, 128}; chunk in {16, 32, 64}.
  *     Others return KDA_ERR_UNSUPPORTED.
- *   - Numerical range: the chunkwise path factorises the decay inside a chunk,
- *     which is exact for |sum of l over one chunk| up to about 80 per channel
- *     (fp32 exponent range).  Gates stronger than that are not supported.
+ *   - Numerical range: the chunkwise path factorises the decay inside a
+ *     chunk as exp(g_r - g_i) = exp(g_r - rho) exp(rho - g_i), with g the
+ *     running sum of l inside the chunk.  Per key channel, rho is the chunk
+ *     start while |g_C| (the channel's total log-decay over the chunk) is at
+ *     most 60, and g_C / 2 above that, so no factor exceeds exp(|g_C| / 2).
+ *     Results are exact up to rounding for |g_C| <= 160 on every channel of
+ *     every chunk: for chunk 64, any gate with alpha >= 0.082 on every token
+ *     qualifies (the pages' worked gate of 0.2 included).  A chunk beyond
+ *     that makes the call's outputs unspecified and sets a device flag that
+ *     kda_device_status reports as KDA_ERR_RANGE.  kda_recurrent_step has no
+ *     such limit.
  */
 #ifndef KDA_H_
 #define KDA_H_
@@ -68,7 +76,9 @@ typedef enum {
   KDA_ERR_UNSUPPORTED = 2, /* valid request outside the supported sizes    */
   KDA_ERR_MISALIGNED = 3,  /* a pointer is not 16-byte aligned             */
   KDA_ERR_CUDA = 4,        /* a CUDA call failed; see kda_last_cuda_error  */
-  KDA_ERR_TIMEOUT = 5      /* a bounded device-side wait gave up           */
+  KDA_ERR_TIMEOUT = 5,     /* a bounded device-side wait gave up           */
+  KDA_ERR_RANGE = 6        /* a chunk's decay exceeded the supported range
+                              (reported by kda_device_status)              */
 } kda_status;
 
 typedef enum { KDA_BF16 = 0, KDA_F32 = 1 } kda_dtype;
@@ -312,9 +322,11 @@ KDA_API const char* kda_status_string(kda_status status);
 
 /* Synchronises `stream` and reports whether any kernel of this library on
  * this device gave up a bounded device-side wait since the last call
- * (KDA_ERR_TIMEOUT; the flag is cleared), else KDA_OK.  The kernels never
- * wait without a time limit; a wait that runs out abandons the rest of that
- * CTA's work and leaves its outputs unspecified. */
+ * (KDA_ERR_TIMEOUT), else whether a chunkwise call met a chunk whose decay
+ * exceeded the supported range (KDA_ERR_RANGE, see "Numerical range"
+ * above), else KDA_OK.  The flags are cleared.  The kernels never wait
+ * without a time limit; a wait that runs out abandons the rest of that CTA's
+ * work and leaves its outputs unspecified. */
 KDA_API kda_status kda_device_status(cudaStream_t stream);
 
 /* kda_chunk_bwd -- the backward pass of kda_chunk_fwd (per-key-channel gate,
@@ -343,7 +355,11 @@ KDA_API kda_status kda_device_status(cudaStream_t stream);
  * another output (KDA_ERR_INVALID_ARG).  All arithmetic is fp32; the call
  * re-runs the forward's chunk stages and allocates its fp32 workspace from
  * the stream-ordered pool (kda_chunk_bwd_plan reports its size).  Stream
- * ordered: returns after queueing the kernels. */
+ * ordered: returns after queueing the kernels.
+ * Numerical range: the backward keeps the chunk-start factorisation of the
+ * decay, exact while |g_C| <= 80 on every channel of every chunk (g_C as
+ * under "Numerical range" above); beyond that its outputs are unspecified
+ * and kda_device_status reports KDA_ERR_RANGE. */
 KDA_API kda_status kda_chunk_bwd(const kda_shape* shape, const void* q,
                                  const void* k, const void* v,
                                  const float* log_alpha, const float* beta,

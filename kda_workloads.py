@@ -9,6 +9,7 @@ Recipe (every config uses seed 1000 + config id unless told otherwise):
   v          ~ N(0, 1)
   beta       = sigmoid(N(0, 1))                     one per token and head
   log_alpha  = logsigmoid(N(0, 1)) / 16             one per token, head, key channel
+               (the divisor is a parameter of draw(); strong-gate tests use 1)
   state      ~ N(0, 0.1) (standard deviation 0.1) where the config has one
 Draw order from one torch.Generator: q, k, v, beta, log_alpha, state.  The
 lengths of the packed config are drawn first from a separate CPU generator,
@@ -52,12 +53,14 @@ def _unit(x):
 
 
 def draw(lead, H, dk, dv, *, io="bf16", scale_q=False, n_states=None,
-         device="cpu", seed=0, state_std=0.1):
+         device="cpu", seed=0, state_std=0.1, gate_divisor=16.0):
     """Draw one set of KDA inputs with leading shape ``lead`` (e.g. (B, T)).
 
     Returns dict(q, k, v [lead, H, d] in the io dtype; log_alpha [lead, H, dk]
     and beta [lead, H] in fp32; initial_state [n_states, H, dk, dv] fp32 or
-    None).
+    None).  ``gate_divisor`` divides the logsigmoid gate (16 in every named
+    config; 1 gives the undivided logsigmoid(N(0, 1)) gate, whose decay over
+    a 64-token chunk is about 16 times stronger).
     """
     g = torch.Generator(device=device).manual_seed(int(seed))
     dt = DTYPES[io]
@@ -70,7 +73,8 @@ def draw(lead, H, dk, dv, *, io="bf16", scale_q=False, n_states=None,
     k = _unit(torch.randn(shape_k, **opts))
     v = torch.randn(shape_v, **opts)
     beta = torch.sigmoid(torch.randn(tuple(lead) + (H,), **opts))
-    log_alpha = torch.nn.functional.logsigmoid(torch.randn(shape_k, **opts)) / 16
+    log_alpha = (torch.nn.functional.logsigmoid(torch.randn(shape_k, **opts))
+                 / gate_divisor)
     state = None
     if n_states:
         state = torch.randn((n_states, H, dk, dv), **opts) * state_std

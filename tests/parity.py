@@ -78,3 +78,25 @@ def sample_units(n_seqs, H, count, seed=0, must=()):
 
 def nan_like(t):
     return torch.full_like(t, float("nan"))
+
+
+def check_units(name, got, ref, tol, unit_axes):
+    """Whole-tensor comparison that also bounds every unit: rel-L2 over the
+    whole tensor and over each slice that fixes the ``unit_axes`` (e.g. each
+    (sequence, head)), max-abs over everything.  Returns (whole rel-L2,
+    worst unit rel-L2, max-abs)."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert got.shape == ref.shape, (name, got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), f"{name}: non-finite"
+    whole = rel_l2(got, ref)
+    red = tuple(i for i in range(got.ndim) if i not in unit_axes)
+    num = np.sqrt(np.sum((got - ref) ** 2, axis=red))
+    den = np.sqrt(np.sum(ref ** 2, axis=red))
+    per = np.where(den > 0, num / np.where(den > 0, den, 1.0), num)
+    worst = float(np.max(per)) if per.size else 0.0
+    m = max_abs(got, ref) if got.size else 0.0
+    assert whole <= tol, f"{name}: rel-L2 {whole:.3e} > {tol:.0e} (max-abs {m:.3e})"
+    assert worst <= tol, (f"{name}: worst unit rel-L2 {worst:.3e} > {tol:.0e} "
+                          f"at {np.unravel_index(np.argmax(per), per.shape)}")
+    return whole, worst, m

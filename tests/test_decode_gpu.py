@@ -77,16 +77,15 @@ def test_zero_tokens_keeps_state():
     assert torch.equal(state, s0)
 
 
-def test_config4_full_size_sampled():
+def test_config4_full_size_every_element():
     """256 sequences x 32 heads, d = 128, 64 consecutive steps with the state
-    updated in place (the benchmarked launch); every output and the final
-    state of sampled (sequence, head) units against the oracle, everything
-    else checked finite."""
+    updated in place (the benchmarked launch): every output of every step and
+    the whole final state against the fp64 oracle run over all 8192
+    (sequence, head) units (about a second on 16 host cores)."""
     d = W.make(4, device=DEV)
     cfg = d["cfg"]
-    N, H, S = cfg["N"], cfg["H"], cfg["steps"]
-    units = PY.sample_units(N, H, 48, seed=4, must=[(0, 0), (N - 1, H - 1)])
-    s0 = {u: d["initial_state"][u[0], u[1]].clone() for u in units}
+    S = cfg["steps"]
+    s0 = PY.host64(d["initial_state"])
     state = d["initial_state"]
     outs = []
     for s in range(S):
@@ -96,17 +95,9 @@ def test_config4_full_size_sampled():
                                      d["beta"][s][:, None], state))
     torch.cuda.synchronize()
     out = torch.cat(outs, 1)                      # [N, S, H, dv]
-    assert torch.isfinite(out.float()).all() and torch.isfinite(state).all()
-    errs = []
-    for (n, h) in units:
-        o, f = kda_oracle.recurrent(
-            PY.host64(d["q"][:, n, h])[None, :, None],
-            PY.host64(d["k"][:, n, h])[None, :, None],
-            PY.host64(d["v"][:, n, h])[None, :, None],
-            PY.host64(d["log_alpha"][:, n, h])[None, :, None],
-            PY.host64(d["beta"][:, n, h])[None, :, None],
-            PY.host64(s0[(n, h)])[None, None])
-        errs.append(PY.check(f"out[{n},{h}]", PY.host64(out[n, :, h]), o[0, :, 0],
-                             PY.TOL_BF16)[0])
-        PY.check(f"state[{n},{h}]", PY.host64(state[n, h]), f[0, 0], PY.TOL_BF16)
-    assert np.max(errs) < PY.TOL_BF16
+    # the oracle sees each sequence's 64 steps as one 64-token sequence
+    tr = lambda x: np.ascontiguousarray(np.swapaxes(PY.host64(x), 0, 1))  # noqa: E731
+    ro, rs = kda_oracle.recurrent(tr(d["q"]), tr(d["k"]), tr(d["v"]),
+                                  tr(d["log_alpha"]), tr(d["beta"]), s0)
+    PY.check_units("out", PY.host64(out), ro, PY.TOL_BF16, unit_axes=(0, 2))
+    PY.check_units("state", PY.host64(state), rs, PY.TOL_BF16, unit_axes=(0, 1))
