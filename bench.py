@@ -182,6 +182,36 @@ def oracle_time(args_, min_seconds):
             return done, el
 
 
+def oracle_single_thread(seconds):
+    """The oracle timed on ONE host thread (OMP_NUM_THREADS=1, in a child
+    process so the parent's OpenMP runtime keeps its thread count) on whole
+    (sequence, head) units of the prefill workload; returns the tokens/s
+    record, or None if the child failed."""
+    env = dict(os.environ, OMP_NUM_THREADS="1")
+    try:
+        r = subprocess.run(
+            [sys.executable, os.path.abspath(__file__), "--oracle-child",
+             str(seconds)], env=env, capture_output=True, text=True,
+            timeout=max(120.0, 10 * seconds))
+        rec = json.loads(r.stdout.strip().splitlines()[-1])
+    except Exception:
+        return None
+    H = W.CONFIGS[PREFILL_CFG]["H"]
+    T = W.CONFIGS[PREFILL_CFG]["T"]
+    return {"value": rec["token_heads"] / rec["seconds"] / H, "unit": "tokens/s",
+            "cores": rec["threads"], "kind": "oracle",
+            "sample": f"{rec['token_heads'] // T} whole (sequence, head) units "
+                      f"of {T} tokens in {rec['seconds']:.1f} s on "
+                      f"{rec['threads']} thread; tokens/s = token-heads/s / H={H}"}
+
+
+def oracle_child(seconds):
+    from oracle import kda_oracle
+    n, el = oracle_time(oracle_inputs(1), seconds)
+    print(json.dumps({"token_heads": n, "seconds": el,
+                      "threads": kda_oracle.num_threads()}), flush=True)
+
+
 def run_reference(args, world, rank):
     """The reference arm: the fp64 CPU oracle as it stands, on host cores."""
     if rank != 0:
@@ -573,7 +603,9 @@ def run_kda(args, world, rank, local):
                "sample": f"{n // T} whole (sequence, head) units of {T} tokens "
                          f"(d_k=d_v={dk}) of the prefill workload in {el:.1f} s "
                          f"on {threads} threads; tokens/s = token-heads/s / "
-                         f"H={H}"}
+                         f"H={H}",
+               "single_thread": oracle_single_thread(
+                   max(2.0, args.cpu_seconds / 3))}
 
     traffic = load_traffic()
     if rank == 0:
@@ -583,6 +615,11 @@ def run_kda(args, world, rank, local):
             "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
+            "tensor_peak_frac": achieved_tf / pk["bf16_tflops"],
+            "hbm_frac": achieved_gbs / pk["hbm_gbs"],
+            "decode_gbs": d_gbs,
+            "decode_hbm_frac": d_launch_gbs / pk["hbm_gbs"],
+            "decode_us_per_step": d_step_ms * 1e3,
             "config": {
                 "workload": f"kda_chunk_fwd prefill B={B} T={T} H={H} "
                             f"d_k=d_v={dk} C={C} bf16 (Kimi-Linear-shaped "
@@ -592,7 +629,6 @@ def run_kda(args, world, rank, local):
                 "l2": "inputs larger than L2 (no flush)",
                 "path": K.chunk_fwd_path(B, T, H, dk, dv, C, torch.bfloat16),
             },
-            "tensor_peak_frac": achieved_tf / pk["bf16_tflops"],
             "roofline": {
                 "bound": "hbm", "achieved": achieved_gbs,
                 "peak": pk["hbm_gbs"], "unit": "GB/s",
@@ -729,12 +765,17 @@ def main():
                     default=None,
                     help="profiling aid: run one workload's warm-up and timed "
                          "launches only (no e2e, no CPU baseline, no JSON line)")
+    ap.add_argument("--oracle-child", type=float, default=None,
+                    help=argparse.SUPPRESS)
     ap.add_argument("--seq-len", type=int, default=None,
                     help="with --only prefill/backward/split: tokens per "
                          "sequence (default: the workload's own, 8192 for "
                          "prefill and backward, 131072 for the split's one "
                          "sequence of H=8), for a smaller profiler capture")
     args = ap.parse_args()
+    if args.oracle_child is not None:
+        oracle_child(args.oracle_child)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     world = int(os.environ.get("WORLD_SIZE", "1"))

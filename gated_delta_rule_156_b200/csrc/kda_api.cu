@@ -571,6 +571,30 @@ kda_status kda_selftest_timeout(int limit_us, cudaStream_t stream) {
   return e == cudaSuccess ? KDA_OK : cuda_fail(e);
 }
 
+kda_status kda_workspace_pool(size_t* reserved_bytes, size_t* used_bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  keep_pool_memory();
+  cudaMemPool_t pool;
+  if ((e = cudaDeviceGetDefaultMemPool(&pool, dev)) != cudaSuccess)
+    return cuda_fail(e);
+  uint64_t v = 0;
+  if (reserved_bytes) {
+    if ((e = cudaMemPoolGetAttribute(pool, cudaMemPoolAttrReservedMemCurrent,
+                                     &v)) != cudaSuccess)
+      return cuda_fail(e);
+    *reserved_bytes = (size_t)v;
+  }
+  if (used_bytes) {
+    if ((e = cudaMemPoolGetAttribute(pool, cudaMemPoolAttrUsedMemCurrent, &v)) !=
+        cudaSuccess)
+      return cuda_fail(e);
+    *used_bytes = (size_t)v;
+  }
+  return KDA_OK;
+}
+
 int kda_last_cuda_error(void) { return g_last_cuda_error; }
 
 int kda_version(void) { return 100; }

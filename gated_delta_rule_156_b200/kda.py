@@ -25,7 +25,7 @@ EXPORTS = ("kda_chunk_fwd", "kda_chunk_fwd_staged", "kda_recurrent_step",
            "kda_chunk_fwd_staged_noalloc", "kda_chunk_fwd_gated",
            "kda_recurrent_step_gated", "kda_chunk_fwd_ex",
            "kda_recurrent_step_ex", "kda_selftest_timeout", "kda_chunk_bwd",
-           "kda_chunk_bwd_plan", "kda_chunk_fwd_split",
+           "kda_chunk_bwd_plan", "kda_chunk_fwd_split", "kda_workspace_pool",
            "kda_chunk_fwd_split_plan")
 GATES = {"channel": 0, "head": 1, "none": 2}
 
@@ -133,6 +133,9 @@ def library():
         lib.kda_device_status.argtypes = [vp]
         lib.kda_status_string.restype = ctypes.c_char_p
         lib.kda_status_string.argtypes = [ctypes.c_int]
+        lib.kda_workspace_pool.restype = ctypes.c_int
+        lib.kda_workspace_pool.argtypes = [ctypes.POINTER(ctypes.c_size_t),
+                                           ctypes.POINTER(ctypes.c_size_t)]
         lib.kda_last_cuda_error.restype = ctypes.c_int
         lib.kda_last_cuda_error.argtypes = []
         lib.kda_version.restype = ctypes.c_int
@@ -401,6 +404,16 @@ def selftest_umma(A, B, a_mn, b_mn, panel_rows=None, stream=None):
     if st != KDA_OK:
         raise KdaError(st, "kda_selftest_umma")
     return D
+
+
+def workspace_pool():
+    """(reserved, used) bytes of the device memory pool the library's
+    stream-ordered workspace comes from (kda_workspace_pool)."""
+    r, u = ctypes.c_size_t(), ctypes.c_size_t()
+    st = library().kda_workspace_pool(ctypes.byref(r), ctypes.byref(u))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_workspace_pool")
+    return r.value, u.value
 
 
 def device_status(stream=None):

@@ -448,6 +448,23 @@ KDA_API kda_status kda_chunk_fwd_split_plan(const kda_shape* shape, int gate,
  * kda_device_status on this stream returns KDA_ERR_TIMEOUT. */
 KDA_API kda_status kda_selftest_timeout(int limit_us, cudaStream_t stream);
 
+/*
+ * kda_workspace_pool -- where the stream-ordered workspace lives.  The
+ * paths that need workspace (the four-stage pipeline, the packed layout's
+ * longest-first order, the sequence split and the backward pass) take it
+ * with cudaMallocAsync from the current device's default memory pool and
+ * give it back with cudaFreeAsync on the same stream.  The library sets that
+ * pool's release threshold to the maximum on first use, so freed workspace
+ * stays cached in the pool: after the first call of a given size, repeated
+ * calls reuse the pool's memory and reserve nothing new from the device.
+ * Calls on different streams never share a workspace.
+ *   reserved_bytes : out, memory the pool currently holds (may be NULL).
+ *   used_bytes     : out, memory of the pool in use right now (may be NULL).
+ * Reads the current device's pool; launches nothing.
+ */
+KDA_API kda_status kda_workspace_pool(size_t* reserved_bytes,
+                                      size_t* used_bytes);
+
 /* The cudaError_t value behind the most recent KDA_ERR_CUDA on this thread
  * (0 if none). */
 KDA_API int kda_last_cuda_error(void);
