@@ -137,7 +137,9 @@ kda_status validate_chunk(const kda_shape* s, const void* q, const void* k,
   return KDA_OK;
 }
 
-kda_status run_with_workspace(size_t bytes, cudaStream_t stream, bool fused,
+enum class Path { kStaged, kFused, kTwoPass };
+
+kda_status run_with_workspace(size_t bytes, cudaStream_t stream, Path path,
                               const kda::ChunkArgs& a) {
   void* ws = nullptr;
   cudaError_t e;
@@ -146,8 +148,9 @@ kda_status run_with_workspace(size_t bytes, cudaStream_t stream, bool fused,
     if ((e = cudaMallocAsync(&ws, bytes, stream)) != cudaSuccess)
       return cuda_fail(e);
   }
-  e = fused ? kda::launch_fused(a, ws, stream)
-            : kda::launch_staged(a, ws, stream);
+  e = path == Path::kFused     ? kda::launch_fused(a, ws, stream)
+      : path == Path::kTwoPass ? kda::launch_twopass(a, ws, stream)
+                               : kda::launch_staged(a, ws, stream);
   if (ws) {
     const cudaError_t f = cudaFreeAsync(ws, stream);
     if (e == cudaSuccess) e = f;
@@ -207,8 +210,8 @@ kda_status kda_chunk_fwd(const kda_shape* shape, const void* q, const void* k,
                                        final_state, &a);
   if (st != KDA_OK) return st;
   if (kda::fused_supported(a))
-    return run_with_workspace(kda::fused_workspace_bytes(a), stream, true, a);
-  return run_with_workspace(kda::staged_workspace_bytes(a), stream, false, a);
+    return run_with_workspace(kda::fused_workspace_bytes(a), stream, Path::kFused, a);
+  return run_with_workspace(kda::staged_workspace_bytes(a), stream, Path::kStaged, a);
 }
 
 kda_status kda_chunk_fwd_split(const kda_shape* shape, int gate, const void* q,
@@ -283,7 +286,7 @@ kda_status kda_chunk_fwd_staged(const kda_shape* shape, const void* q,
                                        initial_state, cu_seqlens, out,
                                        final_state, &a);
   if (st != KDA_OK) return st;
-  return run_with_workspace(kda::staged_workspace_bytes(a), stream, false, a);
+  return run_with_workspace(kda::staged_workspace_bytes(a), stream, Path::kStaged, a);
 }
 
 kda_status kda_chunk_bwd(const kda_shape* shape, const void* q, const void* k,
@@ -392,8 +395,8 @@ kda_status kda_chunk_fwd_gated(const kda_shape* shape, int gate, const void* q,
                                        final_state, &a, gate);
   if (st != KDA_OK) return st;
   if (!staged && kda::fused_supported(a))
-    return run_with_workspace(kda::fused_workspace_bytes(a), stream, true, a);
-  return run_with_workspace(kda::staged_workspace_bytes(a), stream, false, a);
+    return run_with_workspace(kda::fused_workspace_bytes(a), stream, Path::kFused, a);
+  return run_with_workspace(kda::staged_workspace_bytes(a), stream, Path::kStaged, a);
 }
 
 }  // extern "C"
@@ -428,8 +431,33 @@ kda_status kda_chunk_fwd_ex(const kda_shape* shape, int gate,
   if (st != KDA_OK) return st;
   if (!set_prologue(prologue, &a.pro)) return KDA_ERR_INVALID_ARG;
   if (!staged && kda::fused_supported(a))
-    return run_with_workspace(kda::fused_workspace_bytes(a), stream, true, a);
-  return run_with_workspace(kda::staged_workspace_bytes(a), stream, false, a);
+    return run_with_workspace(kda::fused_workspace_bytes(a), stream, Path::kFused, a);
+  return run_with_workspace(kda::staged_workspace_bytes(a), stream, Path::kStaged, a);
+}
+
+kda_status kda_chunk_fwd_twopass(const kda_shape* shape, int gate,
+                                 const kda_prologue* prologue, const void* q,
+                                 const void* k, const void* v,
+                                 const float* gate_tensor, const float* beta,
+                                 const float* initial_state,
+                                 const int32_t* cu_seqlens, void* out,
+                                 float* final_state, cudaStream_t stream) {
+  kda::ChunkArgs a{};
+  const kda_status st = validate_chunk(shape, q, k, v, gate_tensor, beta,
+                                       initial_state, cu_seqlens, out,
+                                       final_state, &a, gate);
+  if (st != KDA_OK) return st;
+  if (!set_prologue(prologue, &a.pro)) return KDA_ERR_INVALID_ARG;
+  if (!kda::fused_supported(a)) {
+    // nothing to do for an empty request; other shapes are unsupported here
+    if (a.bf16 && a.chunk == 64 && (a.dk == 64 || a.dk == 128) &&
+        (a.dv == 64 || a.dv == 128))
+      return run_with_workspace(kda::staged_workspace_bytes(a), stream,
+                                Path::kStaged, a);
+    return KDA_ERR_UNSUPPORTED;
+  }
+  return run_with_workspace(kda::twopass_workspace_bytes(a), stream,
+                            Path::kTwoPass, a);
 }
 
 kda_status kda_chunk_fwd_staged_noalloc(

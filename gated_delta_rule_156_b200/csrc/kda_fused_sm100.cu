@@ -102,6 +102,7 @@ bool make_tile_map(CUtensorMap* m, const void* base, int d, int H, int tokens) {
 
 #include "kda_fused_ws_sm100.cuh"
 #include "kda_fused_pair_sm100.cuh"
+#include "kda_twopass_sm100.cuh"
 
 namespace kda {
 namespace {
@@ -163,6 +164,17 @@ cudaError_t fused_take_range(cudaStream_t stream, int* flag) {
       cudaSuccess)
     return e;
   return cudaMemcpyToSymbol(g_fused_range, &zero, sizeof(int));
+}
+
+size_t twopass_workspace_bytes(const ChunkArgs& a) {
+  return twopass::workspace_bytes(a);
+}
+
+int twopass_kernel_count(const ChunkArgs& a) { return a.cu_seqlens ? 4 : 2; }
+
+cudaError_t launch_twopass(const ChunkArgs& a, void* workspace,
+                           cudaStream_t stream) {
+  return twopass::launch(a, workspace, stream);
 }
 
 cudaError_t launch_fused(const ChunkArgs& a, void* workspace,

@@ -142,6 +142,14 @@ cudaError_t bwd_take_range(cudaStream_t stream, int* flag);
 cudaError_t launch_timeout_probe(int limit_us, cudaStream_t stream);
 cudaError_t launch_fused(const ChunkArgs& a, void* workspace,
                          cudaStream_t stream);
+// Two-pass tensor-core prefill (kda_twopass_sm100.cuh, in the fused
+// translation unit): a parallel factorisation pass writing one package per
+// (chunk, head) into `workspace`, then the chain kernel.  Same shapes as the
+// fused kernel.
+size_t twopass_workspace_bytes(const ChunkArgs& a);
+int twopass_kernel_count(const ChunkArgs& a);
+cudaError_t launch_twopass(const ChunkArgs& a, void* workspace,
+                           cudaStream_t stream);
 
 // Upper bound on the number of chunks of a request (packed sequences may each
 // add one partial chunk).

@@ -26,6 +26,7 @@ EXPORTS = ("kda_chunk_fwd", "kda_chunk_fwd_staged", "kda_recurrent_step",
            "kda_recurrent_step_gated", "kda_chunk_fwd_ex",
            "kda_recurrent_step_ex", "kda_selftest_timeout", "kda_chunk_bwd",
            "kda_chunk_bwd_plan", "kda_chunk_fwd_split", "kda_workspace_pool",
+           "kda_chunk_fwd_twopass",
            "kda_chunk_fwd_split_plan")
 GATES = {"channel": 0, "head": 1, "none": 2}
 
@@ -98,6 +99,10 @@ def library():
         lib.kda_chunk_fwd_ex.argtypes = [
             ctypes.POINTER(KdaShape), ctypes.c_int, ctypes.POINTER(KdaPrologue),
             vp, vp, vp, fp, fp, fp, vp, vp, fp, ctypes.c_int, vp]
+        lib.kda_chunk_fwd_twopass.restype = ctypes.c_int
+        lib.kda_chunk_fwd_twopass.argtypes = [
+            ctypes.POINTER(KdaShape), ctypes.c_int, ctypes.POINTER(KdaPrologue),
+            vp, vp, vp, fp, fp, fp, vp, vp, fp, vp]
         lib.kda_recurrent_step_ex.restype = ctypes.c_int
         lib.kda_recurrent_step_ex.argtypes = [
             ctypes.POINTER(KdaShape), ctypes.c_int, ctypes.POINTER(KdaPrologue),
@@ -174,7 +179,7 @@ def _stream(stream):
 
 def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
               chunk=64, out=None, final_state=None, staged=False, stream=None,
-              gate="channel", prologue=None):
+              gate="channel", prologue=None, twopass=False):
     """Chunkwise KDA forward (kda_chunk_fwd / kda_chunk_fwd_staged, or
     kda_chunk_fwd_gated when ``gate`` is not "channel").
 
@@ -184,7 +189,8 @@ def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
     [N, H, d_k, d_v] fp32 or None; cu_seqlens int32 [N + 1] or None (then
     B == 1 and T is the packed total).  ``prologue`` (dict, see
     kda_prologue) normalises q and k and/or maps gate logits in-kernel
-    (kda_chunk_fwd_ex).  Returns (out, final_state).
+    (kda_chunk_fwd_ex).  ``twopass`` evaluates it as a factorisation pass
+    and a chain kernel (kda_chunk_fwd_twopass).  Returns (out, final_state).
     """
     B, T, H, dk = q.shape
     dv = v.shape[-1]
@@ -204,6 +210,16 @@ def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
         _check_dev(name, t, dt)
     shape = KdaShape(B, T, H, dk, dv, chunk, n if cu_seqlens is not None else 0,
                      _io(q))
+    if twopass:  # kda_chunk_fwd_twopass: factorisation pass, then the chain
+        pro = None if prologue is None else _prologue(prologue)
+        st = library().kda_chunk_fwd_twopass(
+            ctypes.byref(shape), GATES[gate],
+            None if pro is None else ctypes.byref(pro), _ptr(q), _ptr(k),
+            _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(initial_state),
+            _ptr(cu_seqlens), _ptr(out), _ptr(final_state), _stream(stream))
+        if st != KDA_OK:
+            raise KdaError(st, "kda_chunk_fwd_twopass")
+        return out, final_state
     if prologue is not None:
         pro = _prologue(prologue)
         st = library().kda_chunk_fwd_ex(

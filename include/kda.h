@@ -225,6 +225,33 @@ KDA_API kda_status kda_recurrent_step_ex(const kda_shape* shape, int gate,
                                          float* state_inout, void* out,
                                          cudaStream_t stream);
 
+/*
+ * kda_chunk_fwd_twopass -- the chunkwise prefill of kda_chunk_fwd_ex
+ * evaluated in two tensor-core passes instead of one fused kernel:
+ *   (1) a factorisation pass with one CTA per (chunk, head), all side by
+ *       side: the decay-scaled operands, A and P, T' = (I + A)^-1 Diag(beta)
+ *       and W = T' K~ of every chunk, written to a workspace as one package
+ *       per (chunk, head) (about 66 KB at d_k = 128);
+ *   (2) a chain kernel per (sequence, head, 64-column d_v tile) that reads
+ *       the packages in order and runs only the serial state and output
+ *       products, with the fp32 state in tensor memory.
+ * Same arguments, layouts and results (up to rounding order) as
+ * kda_chunk_fwd_ex without the `staged` flag.  bf16 io with d_k, d_v in
+ * {64, 128} and chunk 64 only (KDA_ERR_UNSUPPORTED otherwise).  Workspace:
+ * stream-ordered, max_chunks * H * 66,560 bytes at d_k = 128 (plus the
+ * packed layout's order and chunk offsets).
+ */
+KDA_API kda_status kda_chunk_fwd_twopass(const kda_shape* shape, int gate,
+                                         const kda_prologue* prologue,
+                                         const void* q, const void* k,
+                                         const void* v,
+                                         const float* gate_tensor,
+                                         const float* beta,
+                                         const float* initial_state,
+                                         const int32_t* cu_seqlens, void* out,
+                                         float* final_state,
+                                         cudaStream_t stream);
+
 /* Size in bytes of the fixed device scratch array behind
  * kda_chunk_fwd_staged_noalloc (16 MiB). */
 #define KDA_NOALLOC_SCRATCH_BYTES (16u << 20)
