@@ -10,8 +10,8 @@
 // one bulk copy.  No CTA waits for another, so the factorisation of all
 // chunks runs side by side on every SM instead of along each sequence.
 //
-// Pass 2, chain_kernel: one CTA of 128 threads per (sequence, head,
-// 64-column d_v tile).  Per chunk it bulk-loads the package (two ahead,
+// Pass 2, chain_kernel: one CTA of 256 threads per (sequence, head,
+// 64-column d_v tile), two threads per TMEM lane (32 columns each).  Per chunk it bulk-loads the package (two ahead,
 // double-buffered) and V, and runs the paired kernel's consumer steps:
 // U = T' V and [W; Qt] S (MMA3), Delta = U - W S, S += Kb^T Delta (MMA4) and
 // the outputs P Delta + Qt S (MMA5), then S <- exp(g_C - rho) S.  The fp32
@@ -47,7 +47,7 @@ using ws::tmem_wait_st;
 using ws::wait_or_abort;
 
 constexpr int kFactorThreads = 256;
-constexpr int kChainThreads = 128;
+constexpr int kChainThreads = 256;
 constexpr int kBarAll = 3;  // named barrier id of a whole CTA
 
 __device__ __forceinline__ void bulk_store(void* gdst, const void* src,
@@ -134,7 +134,10 @@ __global__ void __launch_bounds__(kFactorThreads, 2)
   const int colh = warp >> 2, row_t = t & 127;
   const int cg = t % NCG, rb = t / NCG;
   const int pnl = cg >> 4;
-  const int cid = blockIdx.x, h = blockIdx.y;
+  // heads fastest: neighbouring CTAs read adjacent columns of the same rows
+  const int h = (int)(blockIdx.x % (unsigned)p.H);
+  const int cid = (int)(blockIdx.x / (unsigned)p.H);
+  uint8_t* gpk = p.packages + ((size_t)cid * p.H + h) * PL::slot;
   int seq = 0, tok0 = 0, L = 0;
   const int nc = (p.T + kC - 1) / kC;
   const bool valid = locate_chunk(cid, p.cu, p.chunk_off, p.n_seqs, p.T, kC,
@@ -249,7 +252,18 @@ __global__ void __launch_bounds__(kFactorThreads, 2)
       // MMA1 has read Qt: back to the chunk-start q e^g where rho != 0
       if (gc[2 * DK] != 0.f) rescale_qt<PL::NP>(kq, gc + DK, t);
       tc_fence_before();
+      fence_proxy_async();
       named_sync(kBarAll, kFactorThreads);
+      if (t == 0) {  // Qt, Kb, P and the package vector are final: store them
+        // now, under the inverse (W and T' follow at the end)
+#pragma unroll
+        for (int q = 0; q < (int)PL::NP; ++q)
+          bulk_store(gpk + q * 16384 + 8192, kq + q * 16384 + 8192, 8192);
+        bulk_store(gpk + PL::s_kb, kb, 16384);  // (d_k = 64: its zero panel too)
+        bulk_store(gpk + PL::s_pp, pp, 8192);
+        bulk_store(gpk + PL::s_gc, gc, PL::gc_bytes);
+        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+      }
 
       invert_unit_lower_tc(afp, tfp, msc, t);
 
@@ -300,9 +314,11 @@ __global__ void __launch_bounds__(kFactorThreads, 2)
       tc_fence_before();
       fence_proxy_async();
       named_sync(kBarAll, kFactorThreads);
-      if (t == 0) {  // the package to HBM
-        bulk_store(p.packages + ((size_t)cid * p.H + h) * PL::slot, slot,
-                   PL::copy_bytes);
+      if (t == 0) {  // W and T' to HBM; every store completes before exit
+#pragma unroll
+        for (int q = 0; q < (int)PL::NP; ++q)
+          bulk_store(gpk + q * 16384, kq + q * 16384, 8192);
+        bulk_store(gpk + PL::s_tp, tp, 8192);
         bulk_commit_wait_all();
       }
     } else if (t == 0) {
@@ -355,7 +371,10 @@ __global__ void __launch_bounds__(kChainThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 6);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 7);
 
+  // eight warps: thread c owns TMEM lane (row) c % 128 and the 32 columns
+  // 32 (c / 128) .. + 31 of the 64-column tile
   const int c = threadIdx.x, warp = c >> 5;
+  const int row = c & 127, half = c >> 7;
   const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
   const int n_tiles = p.dv / kDvt;
   const int tile = blockIdx.x % n_tiles;
@@ -368,7 +387,7 @@ __global__ void __launch_bounds__(kChainThreads, 1)
   const int nch = (end - start + kC - 1) / kC;
   const int cid0 = p.cu ? p.chunk_off[seq] : seq * ((p.T + kC - 1) / kC);
   auto slot_of = [&](int s) { return sm + Lay::slots + s * PL::slot; };
-  const bool owns_state = c < DK;
+  const bool owns_state = row < DK;
 
   if (c == 0) {
     prefetch_tmap(&tm_v);
@@ -377,7 +396,7 @@ __global__ void __launch_bounds__(kChainThreads, 1)
       mbar_init(bar_v + s, 1);
     }
     mbar_init(bar_cm, 1);
-    mbar_init(bar_sop, 4);
+    mbar_init(bar_sop, kChainThreads / 32);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -412,25 +431,22 @@ __global__ void __launch_bounds__(kChainThreads, 1)
 
   const size_t sbase = (((size_t)seq * p.H + h) * DK) * p.dv + j0;
   if (owns_state) {  // initial state into TMEM (fp32) and the bf16 operand
+    float v[32];
+    if (p.s_init) {
+      const float4* src = reinterpret_cast<const float4*>(
+          p.s_init + sbase + (size_t)row * p.dv + 32 * half);
 #pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
-      float v[32];
-      if (p.s_init) {
-        const float4* src = reinterpret_cast<const float4*>(
-            p.s_init + sbase + (size_t)c * p.dv + 32 * hf);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float4 x = src[i];
-          v[4 * i] = x.x; v[4 * i + 1] = x.y; v[4 * i + 2] = x.z;
-          v[4 * i + 3] = x.w;
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = 0.f;
+      for (int i = 0; i < 8; ++i) {
+        const float4 x = src[i];
+        v[4 * i] = x.x; v[4 * i + 1] = x.y; v[4 * i + 2] = x.z;
+        v[4 * i + 3] = x.w;
       }
-      tmem_st32(tmem + lane_base + Lay::t_s + 32 * hf, v);
-      st_chunks<4>(sop, c, 4 * hf, v);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = 0.f;
     }
+    tmem_st32(tmem + lane_base + Lay::t_s + 32 * half, v);
+    st_chunks<4>(sop, row, 4 * half, v);
     tmem_wait_st();
   }
   tc_fence_before();
@@ -495,29 +511,23 @@ __global__ void __launch_bounds__(kChainThreads, 1)
     tc_fence_after();
 
     // ---- Delta = U - W S (rows 0-63)
-    if (c < 64) {
+    if (row < 64) {
+      float uu[32], wsv[32];
+      tmem_ld32(tmem + lane_base + Lay::t_u + 32 * half, uu);
+      tmem_ld32(tmem + lane_base + d3 + 32 * half, wsv);
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        float uu[32], wsv[32];
-        tmem_ld32(tmem + lane_base + Lay::t_u + 32 * hf, uu);
-        tmem_ld32(tmem + lane_base + d3 + 32 * hf, wsv);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) uu[i] -= wsv[i];
-        st_chunks<4>(dop, c, 4 * hf, uu);
-      }
+      for (int i = 0; i < 32; ++i) uu[i] -= wsv[i];
+      st_chunks<4>(dop, row, 4 * half, uu);
     }
-    const float gamma = owns_state ? gc[c] : 1.f;
+    const float gamma = owns_state ? gc[row] : 1.f;
     if (owns_state && gc[2 * DK] != 0.f) {
       // S_C = e^(g_C - rho) (e^rho S_0 + Kb^T Delta): pre-scale the state
-      const float er = gc[DK + c];
+      const float er = gc[DK + row];
+      float v[32];
+      tmem_ld32(tmem + lane_base + Lay::t_s + 32 * half, v);
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        float v[32];
-        tmem_ld32(tmem + lane_base + Lay::t_s + 32 * hf, v);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] *= er;
-        tmem_st32(tmem + lane_base + Lay::t_s + 32 * hf, v);
-      }
+      for (int i = 0; i < 32; ++i) v[i] *= er;
+      tmem_st32(tmem + lane_base + Lay::t_s + 32 * half, v);
       tmem_wait_st();
     }
     tc_fence_before();
@@ -556,15 +566,12 @@ __global__ void __launch_bounds__(kChainThreads, 1)
     // ---- S <- exp(g_C - rho) S: the bf16 operand of the next MMA3 first,
     // then TMEM (the store completes before the next MMA4 is issued)
     if (owns_state) {
+      float v[32];
+      tmem_ld32(tmem + lane_base + Lay::t_s + 32 * half, v);
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        float v[32];
-        tmem_ld32(tmem + lane_base + Lay::t_s + 32 * hf, v);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] *= gamma;
-        st_chunks<4>(sop, c, 4 * hf, v);
-        tmem_st32(tmem + lane_base + Lay::t_s + 32 * hf, v);
-      }
+      for (int i = 0; i < 32; ++i) v[i] *= gamma;
+      st_chunks<4>(sop, row, 4 * half, v);
+      tmem_st32(tmem + lane_base + Lay::t_s + 32 * half, v);
     }
     fence_proxy_async();
     tc_fence_before();
@@ -573,24 +580,21 @@ __global__ void __launch_bounds__(kChainThreads, 1)
 
     // ---- outputs (rows 64-127 of this chunk's buffer), overlapping the next
     // chunk's MMA3
-    if (c >= 64) {
-      const int rr = c - 64;
+    if (row >= 64) {
+      const int rr = row - 64;
+      float o[32];
+      tmem_ld32(tmem + lane_base + d3 + 32 * half, o);
+      if (rr < L) {
+        uint4* dst = reinterpret_cast<uint4*>(
+            p.out + ((size_t)(tok0 + rr) * p.H + h) * p.dv + j0 + 32 * half);
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        float o[32];
-        tmem_ld32(tmem + lane_base + d3 + 32 * hf, o);
-        if (rr < L) {
-          uint4* dst = reinterpret_cast<uint4*>(
-              p.out + ((size_t)(tok0 + rr) * p.H + h) * p.dv + j0 + 32 * hf);
-#pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            uint4 w;
-            w.x = pack_bf16x2(o[8 * ch + 0], o[8 * ch + 1]);
-            w.y = pack_bf16x2(o[8 * ch + 2], o[8 * ch + 3]);
-            w.z = pack_bf16x2(o[8 * ch + 4], o[8 * ch + 5]);
-            w.w = pack_bf16x2(o[8 * ch + 6], o[8 * ch + 7]);
-            dst[ch] = w;
-          }
+        for (int ch = 0; ch < 4; ++ch) {
+          uint4 w;
+          w.x = pack_bf16x2(o[8 * ch + 0], o[8 * ch + 1]);
+          w.y = pack_bf16x2(o[8 * ch + 2], o[8 * ch + 3]);
+          w.z = pack_bf16x2(o[8 * ch + 4], o[8 * ch + 5]);
+          w.w = pack_bf16x2(o[8 * ch + 6], o[8 * ch + 7]);
+          dst[ch] = w;
         }
       }
     }
@@ -608,16 +612,13 @@ __global__ void __launch_bounds__(kChainThreads, 1)
     }
   } else if (owns_state) {
     tc_fence_after();
+    float v[32];
+    tmem_ld32(tmem + lane_base + Lay::t_s + 32 * half, v);
+    float4* dst = reinterpret_cast<float4*>(p.s_final + sbase +
+                                            (size_t)row * p.dv + 32 * half);
 #pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
-      float v[32];
-      tmem_ld32(tmem + lane_base + Lay::t_s + 32 * hf, v);
-      float4* dst = reinterpret_cast<float4*>(p.s_final + sbase +
-                                              (size_t)c * p.dv + 32 * hf);
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-    }
+    for (int i = 0; i < 8; ++i)
+      dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
   }
   tc_fence_before();
   __syncthreads();
@@ -693,8 +694,8 @@ cudaError_t run(const ChunkArgs& a, void* workspace, cudaStream_t stream) {
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)smem1)) != cudaSuccess)
     return e;
-  factor_kernel<DK, GATE><<<dim3((unsigned)nchunks, a.H), kFactorThreads,
-                            smem1, stream>>>(tq, tk, p);
+  factor_kernel<DK, GATE><<<(unsigned)(nchunks * a.H), kFactorThreads, smem1,
+                            stream>>>(tq, tk, p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const size_t smem2 = ChainLayout<DK>::bytes + 1024;
   if ((e = cudaFuncSetAttribute(chain_kernel<DK>,
