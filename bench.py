@@ -367,6 +367,31 @@ def run_kda(args, world, rank, local):
         "tensor_frac": pflops / (h_launch * 1e-3) / 1e12 / pk["bf16_tflops"],
     }
 
+    # ---- the one-kernel paired path (kda_chunk_fwd_paired: no workspace)
+    # on the same inputs, for the A/B against the two-pass default ---------
+    def prefill_paired(_i):
+        K.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], None,
+                    None, chunk=C, out=out, final_state=fin, paired=True)
+
+    for i in range(args.warmup):
+        prefill_paired(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    pms_, pper = timed(prefill_paired, args.steps, stream)
+    barrier(world)
+    pms_ = max_over_ranks(pms_, world)
+    p_launch = statistics.mean(pper)
+    paired_line = {
+        "value": world * B * T / (pms_ / args.steps * 1e-3), "unit": "tokens/s",
+        "ms_per_step": pms_ / args.steps,
+        "workload": "as the prefill, through kda_chunk_fwd_paired (one "
+                    "kernel, cluster pairs, no workspace)",
+        "hbm": {"achieved": pbytes / (p_launch * 1e-3) / 1e9, "unit": "GB/s",
+                "frac": pbytes / (p_launch * 1e-3) / 1e9 / pk["hbm_gbs"]},
+        "tensor_frac": pflops / (p_launch * 1e-3) / 1e12 / pk["bf16_tflops"],
+        "headline_speedup_over_paired": (pms_ / args.steps) / ms_step,
+    }
+
     # ---- in-kernel input prologue on raw inputs: q, k L2-normalised (and q
     # scaled) and log(alpha) = logsigmoid(x) / 16 from raw gate logits x ------
     g_raw = torch.Generator(device=dev).manual_seed(4242 + rank)
@@ -656,6 +681,7 @@ def run_kda(args, world, rank, local):
                 "gpu_launches": args.steps,
             },
             "prefill_head_gate": head_gate,
+            "prefill_paired": paired_line,
             "prefill_packed_long": packed_long,
             "prefill_split": prefill_split,
             "backward": backward_line,
@@ -667,7 +693,8 @@ def run_kda(args, world, rank, local):
                                 "step i's compute and download"},
             "gpu_launches": n_kernels * args.steps,
             "gpu_launches_note": "kernel launches inside the headline prefill "
-                                 "timed region (one fused kernel per call)",
+                                 "timed region (per call: the factorisation "
+                                 "pass and the chain kernel)",
             "clocks": clk,
             "cpu_baseline": cpu,
         }

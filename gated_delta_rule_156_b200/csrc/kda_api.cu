@@ -210,7 +210,7 @@ kda_status kda_chunk_fwd(const kda_shape* shape, const void* q, const void* k,
                                        final_state, &a);
   if (st != KDA_OK) return st;
   if (kda::fused_supported(a))
-    return run_with_workspace(kda::fused_workspace_bytes(a), stream, Path::kFused, a);
+    return run_with_workspace(kda::twopass_workspace_bytes(a), stream, Path::kTwoPass, a);
   return run_with_workspace(kda::staged_workspace_bytes(a), stream, Path::kStaged, a);
 }
 
@@ -395,7 +395,7 @@ kda_status kda_chunk_fwd_gated(const kda_shape* shape, int gate, const void* q,
                                        final_state, &a, gate);
   if (st != KDA_OK) return st;
   if (!staged && kda::fused_supported(a))
-    return run_with_workspace(kda::fused_workspace_bytes(a), stream, Path::kFused, a);
+    return run_with_workspace(kda::twopass_workspace_bytes(a), stream, Path::kTwoPass, a);
   return run_with_workspace(kda::staged_workspace_bytes(a), stream, Path::kStaged, a);
 }
 
@@ -431,7 +431,7 @@ kda_status kda_chunk_fwd_ex(const kda_shape* shape, int gate,
   if (st != KDA_OK) return st;
   if (!set_prologue(prologue, &a.pro)) return KDA_ERR_INVALID_ARG;
   if (!staged && kda::fused_supported(a))
-    return run_with_workspace(kda::fused_workspace_bytes(a), stream, Path::kFused, a);
+    return run_with_workspace(kda::twopass_workspace_bytes(a), stream, Path::kTwoPass, a);
   return run_with_workspace(kda::staged_workspace_bytes(a), stream, Path::kStaged, a);
 }
 
@@ -458,6 +458,30 @@ kda_status kda_chunk_fwd_twopass(const kda_shape* shape, int gate,
   }
   return run_with_workspace(kda::twopass_workspace_bytes(a), stream,
                             Path::kTwoPass, a);
+}
+
+kda_status kda_chunk_fwd_paired(const kda_shape* shape, int gate,
+                                const kda_prologue* prologue, const void* q,
+                                const void* k, const void* v,
+                                const float* gate_tensor, const float* beta,
+                                const float* initial_state,
+                                const int32_t* cu_seqlens, void* out,
+                                float* final_state, cudaStream_t stream) {
+  kda::ChunkArgs a{};
+  const kda_status st = validate_chunk(shape, q, k, v, gate_tensor, beta,
+                                       initial_state, cu_seqlens, out,
+                                       final_state, &a, gate);
+  if (st != KDA_OK) return st;
+  if (!set_prologue(prologue, &a.pro)) return KDA_ERR_INVALID_ARG;
+  if (!kda::fused_supported(a)) {
+    if (a.bf16 && a.chunk == 64 && (a.dk == 64 || a.dk == 128) &&
+        (a.dv == 64 || a.dv == 128))
+      return run_with_workspace(kda::staged_workspace_bytes(a), stream,
+                                Path::kStaged, a);
+    return KDA_ERR_UNSUPPORTED;
+  }
+  return run_with_workspace(kda::fused_workspace_bytes(a), stream,
+                            Path::kFused, a);
 }
 
 kda_status kda_chunk_fwd_staged_noalloc(
@@ -556,13 +580,13 @@ kda_status kda_chunk_fwd_plan(const kda_shape* shape, int packed, int staged,
   kda::ChunkArgs a{};
   fill_args(shape, n_seqs, &a);
   a.cu_seqlens = packed ? reinterpret_cast<const int32_t*>(16) : nullptr;
-  const bool fused = !staged && kda::fused_supported(a);
-  if (path) *path = fused ? 1 : 0;
-  if (kernels) *kernels = fused ? kda::fused_kernel_count(a)
-                                : kda::staged_kernel_count(a);
+  const bool tc = !staged && kda::fused_supported(a);
+  if (path) *path = tc ? 2 : 0;
+  if (kernels) *kernels = tc ? kda::twopass_kernel_count(a)
+                             : kda::staged_kernel_count(a);
   if (workspace_bytes)
-    *workspace_bytes = fused ? kda::fused_workspace_bytes(a)
-                             : kda::staged_workspace_bytes(a);
+    *workspace_bytes = tc ? kda::twopass_workspace_bytes(a)
+                          : kda::staged_workspace_bytes(a);
   return KDA_OK;
 }
 

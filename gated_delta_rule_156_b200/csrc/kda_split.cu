@@ -96,17 +96,19 @@ ChunkArgs trans_args(const ChunkArgs& a, const SplitGeom& g, const SplitWs& w) {
   return t;
 }
 
+// The value and transition runs take kda_chunk_fwd's own evaluation: the
+// two-pass tensor-core path where it applies, else the four-stage pipeline.
 size_t run_workspace(const ChunkArgs& a) {
-  return fused_supported(a) ? fused_workspace_bytes(a)
+  return fused_supported(a) ? twopass_workspace_bytes(a)
                             : staged_workspace_bytes(a);
 }
 
 int run_kernels(const ChunkArgs& a) {
-  return fused_supported(a) ? fused_kernel_count(a) : staged_kernel_count(a);
+  return fused_supported(a) ? twopass_kernel_count(a) : staged_kernel_count(a);
 }
 
 cudaError_t run_forward(const ChunkArgs& a, void* ws, cudaStream_t s) {
-  return fused_supported(a) ? launch_fused(a, ws, s) : launch_staged(a, ws, s);
+  return fused_supported(a) ? launch_twopass(a, ws, s) : launch_staged(a, ws, s);
 }
 
 // Sizes and kernel counts depend on whether cu_seqlens is present, not on its

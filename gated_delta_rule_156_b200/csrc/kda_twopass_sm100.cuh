@@ -324,6 +324,7 @@ __global__ void __launch_bounds__(kFactorThreads, 2)
     } else if (t == 0) {
       atomicExch(&g_fused_timeout, 1);
       mbar_wait(bar_in, 0, 100000000ull);  // the q/k load, if still in flight
+      bulk_commit_wait_all();  // the early package stores read shared memory
     }
   }
   tc_fence_before();

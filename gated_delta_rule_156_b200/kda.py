@@ -26,7 +26,7 @@ EXPORTS = ("kda_chunk_fwd", "kda_chunk_fwd_staged", "kda_recurrent_step",
            "kda_recurrent_step_gated", "kda_chunk_fwd_ex",
            "kda_recurrent_step_ex", "kda_selftest_timeout", "kda_chunk_bwd",
            "kda_chunk_bwd_plan", "kda_chunk_fwd_split", "kda_workspace_pool",
-           "kda_chunk_fwd_twopass",
+           "kda_chunk_fwd_twopass", "kda_chunk_fwd_paired",
            "kda_chunk_fwd_split_plan")
 GATES = {"channel": 0, "head": 1, "none": 2}
 
@@ -99,10 +99,13 @@ def library():
         lib.kda_chunk_fwd_ex.argtypes = [
             ctypes.POINTER(KdaShape), ctypes.c_int, ctypes.POINTER(KdaPrologue),
             vp, vp, vp, fp, fp, fp, vp, vp, fp, ctypes.c_int, vp]
-        lib.kda_chunk_fwd_twopass.restype = ctypes.c_int
-        lib.kda_chunk_fwd_twopass.argtypes = [
-            ctypes.POINTER(KdaShape), ctypes.c_int, ctypes.POINTER(KdaPrologue),
-            vp, vp, vp, fp, fp, fp, vp, vp, fp, vp]
+        for name in ("kda_chunk_fwd_twopass", "kda_chunk_fwd_paired"):
+            fn = getattr(lib, name)
+            fn.restype = ctypes.c_int
+            fn.argtypes = [
+                ctypes.POINTER(KdaShape), ctypes.c_int,
+                ctypes.POINTER(KdaPrologue), vp, vp, vp, fp, fp, fp, vp, vp,
+                fp, vp]
         lib.kda_recurrent_step_ex.restype = ctypes.c_int
         lib.kda_recurrent_step_ex.argtypes = [
             ctypes.POINTER(KdaShape), ctypes.c_int, ctypes.POINTER(KdaPrologue),
@@ -179,7 +182,7 @@ def _stream(stream):
 
 def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
               chunk=64, out=None, final_state=None, staged=False, stream=None,
-              gate="channel", prologue=None, twopass=False):
+              gate="channel", prologue=None, twopass=False, paired=False):
     """Chunkwise KDA forward (kda_chunk_fwd / kda_chunk_fwd_staged, or
     kda_chunk_fwd_gated when ``gate`` is not "channel").
 
@@ -189,8 +192,10 @@ def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
     [N, H, d_k, d_v] fp32 or None; cu_seqlens int32 [N + 1] or None (then
     B == 1 and T is the packed total).  ``prologue`` (dict, see
     kda_prologue) normalises q and k and/or maps gate logits in-kernel
-    (kda_chunk_fwd_ex).  ``twopass`` evaluates it as a factorisation pass
-    and a chain kernel (kda_chunk_fwd_twopass).  Returns (out, final_state).
+    (kda_chunk_fwd_ex).  ``twopass`` forces the factorisation pass + chain
+    kernel (kda_chunk_fwd_twopass, the default for bf16 d in {64, 128},
+    chunk 64); ``paired`` the one-kernel cluster-pair path
+    (kda_chunk_fwd_paired).  Returns (out, final_state).
     """
     B, T, H, dk = q.shape
     dv = v.shape[-1]
@@ -210,15 +215,16 @@ def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
         _check_dev(name, t, dt)
     shape = KdaShape(B, T, H, dk, dv, chunk, n if cu_seqlens is not None else 0,
                      _io(q))
-    if twopass:  # kda_chunk_fwd_twopass: factorisation pass, then the chain
+    if twopass or paired:  # an explicit tensor-core evaluation
+        name = "kda_chunk_fwd_twopass" if twopass else "kda_chunk_fwd_paired"
         pro = None if prologue is None else _prologue(prologue)
-        st = library().kda_chunk_fwd_twopass(
+        st = getattr(library(), name)(
             ctypes.byref(shape), GATES[gate],
             None if pro is None else ctypes.byref(pro), _ptr(q), _ptr(k),
             _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(initial_state),
             _ptr(cu_seqlens), _ptr(out), _ptr(final_state), _stream(stream))
         if st != KDA_OK:
-            raise KdaError(st, "kda_chunk_fwd_twopass")
+            raise KdaError(st, name)
         return out, final_state
     if prologue is not None:
         pro = _prologue(prologue)
@@ -384,7 +390,7 @@ def recurrent_step(q, k, v, log_alpha, beta, state, out=None, stream=None,
 def chunk_fwd_plan(B, T, H, dk, dv, chunk, dtype, packed=False, n_seqs=0,
                    staged=False):
     """(path, kernels, workspace_bytes) of a chunk_fwd call of this shape:
-    path is "fused" or "staged"; no device work is done."""
+    path is "twopass" or "staged"; no device work is done."""
     io = KDA_BF16 if dtype == torch.bfloat16 else KDA_F32
     shape = KdaShape(B, T, H, dk, dv, chunk, n_seqs if packed else 0, io)
     path, kern, ws = ctypes.c_int(), ctypes.c_int(), ctypes.c_size_t()
@@ -393,7 +399,8 @@ def chunk_fwd_plan(B, T, H, dk, dv, chunk, dtype, packed=False, n_seqs=0,
                                       ctypes.byref(kern), ctypes.byref(ws))
     if st != KDA_OK:
         raise KdaError(st, "kda_chunk_fwd_plan")
-    return ("fused" if path.value == 1 else "staged"), kern.value, ws.value
+    return ({2: "twopass", 1: "fused"}.get(path.value, "staged"), kern.value,
+            ws.value)
 
 
 def chunk_fwd_kernel_count(B, T, H, dk, dv, chunk, dtype, packed=False):

@@ -120,9 +120,12 @@ typedef struct {
  *   out           : [B, T, H, d_v] io dtype, written.
  *   final_state   : [N, H, d_k, d_v] fp32, written (may equal initial_state).
  *
- * bf16 inputs with d_k, d_v in {64, 128} and chunk = 64 run the fused
- * tensor-core kernel; every other supported request runs the four-stage
- * kernel pipeline of kda_chunk_fwd_staged.  fp32 state throughout.
+ * bf16 inputs with d_k, d_v in {64, 128} and chunk = 64 run the two-pass
+ * tensor-core evaluation of kda_chunk_fwd_twopass (a factorisation pass over
+ * every (chunk, head), then the serial chain; stream-ordered workspace of
+ * one package per (chunk, head), see kda_chunk_fwd_plan); every other
+ * supported request runs the four-stage kernel pipeline of
+ * kda_chunk_fwd_staged.  fp32 state throughout.
  */
 KDA_API kda_status kda_chunk_fwd(const kda_shape* shape, const void* q, const void* k,
                          const void* v, const float* log_alpha,
@@ -252,6 +255,29 @@ KDA_API kda_status kda_chunk_fwd_twopass(const kda_shape* shape, int gate,
                                          float* final_state,
                                          cudaStream_t stream);
 
+/*
+ * kda_chunk_fwd_paired -- the same chunkwise prefill as kda_chunk_fwd_ex
+ * (without its `staged` flag) in ONE tensor-core kernel and no workspace
+ * (the packed layout needs 4 bytes per sequence for its longest-first
+ * order): per (sequence, head) a cluster of two CTAs, one per 64-column
+ * tile of d_v, that factorise alternate chunks and hand each chunk's
+ * package to the other over distributed shared memory while each runs the
+ * state chain of its own tile.  Slower than the two-pass default on every
+ * measured shape (see the design notes); kept for callers that must not
+ * hold the two-pass workspace.  bf16 io with d_k, d_v in {64, 128} and chunk
+ * 64 (d_v = 64: one CTA per head); KDA_ERR_UNSUPPORTED otherwise.
+ */
+KDA_API kda_status kda_chunk_fwd_paired(const kda_shape* shape, int gate,
+                                        const kda_prologue* prologue,
+                                        const void* q, const void* k,
+                                        const void* v,
+                                        const float* gate_tensor,
+                                        const float* beta,
+                                        const float* initial_state,
+                                        const int32_t* cu_seqlens, void* out,
+                                        float* final_state,
+                                        cudaStream_t stream);
+
 /* Size in bytes of the fixed device scratch array behind
  * kda_chunk_fwd_staged_noalloc (16 MiB). */
 #define KDA_NOALLOC_SCRATCH_BYTES (16u << 20)
@@ -317,8 +343,9 @@ KDA_API kda_status kda_recurrent_step(const kda_shape* shape, const void* q,
  * (staged = 1) would evaluate a request of this shape; launches nothing and
  * touches no device memory.
  *   packed          : nonzero when cu_seqlens will be passed.
- *   path            : out, 1 = fused tensor-core kernel, 0 = four-stage fp32
- *                     pipeline (may be NULL).
+ *   path            : out, 2 = two-pass tensor-core evaluation
+ *                     (kda_chunk_fwd_twopass), 0 = four-stage fp32 pipeline
+ *                     (may be NULL).
  *   kernels         : out, kernel launches one call makes (may be NULL).
  *   workspace_bytes : out, stream-ordered workspace one call allocates (may be
  *                     NULL).

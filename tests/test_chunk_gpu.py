@@ -151,8 +151,9 @@ def test_exact_recall_fp32(path):
 
 @pytest.mark.parametrize("dk,dv", [(128, 128), (64, 64), (64, 128), (128, 64)])
 def test_bf16_takes_fused_path(dk, dv):
-    path, kernels, _ = K.chunk_fwd_plan(1, 128, 2, dk, dv, 64, torch.bfloat16)
-    assert path == "fused" and kernels == 1
+    # the two-pass tensor-core evaluation: factorisation pass + chain kernel
+    path, kernels, ws = K.chunk_fwd_plan(1, 128, 2, dk, dv, 64, torch.bfloat16)
+    assert path == "twopass" and kernels == 2 and ws > 0
     d = W.draw((2, 130), 2, dk, dv, io="bf16", n_states=2, device=DEV, seed=dk + dv)
     out, fin = run(d, "auto", 64)
     assert K.device_status() == 0

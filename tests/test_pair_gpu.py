@@ -1,10 +1,13 @@
-"""The paired fused prefill (d_v = 128: the two 64-column tiles of a head run
-as a 2-CTA cluster and factorise alternate chunks) on the chunk counts that
-exercise its slot hand-over: sequences with no chunk, one chunk (the second
-CTA factorises nothing), two and three chunks (the first sends before the
-peer has anything to release), and longer ones with a ragged tail; for both
-key widths, every gate layout and the input prologue, against the fp64
-oracle."""
+"""The tensor-core prefill paths on the chunk counts that exercise their
+hand-overs: sequences with no chunk, one chunk, two and three chunks, and
+longer ones with a ragged tail; for both key widths, every gate layout and
+the input prologue, against the fp64 oracle.  Each test runs both
+evaluations: the paired one-kernel path (kda_chunk_fwd_paired: the two
+64-column tiles of a head run as a 2-CTA cluster and factorise alternate
+chunks; the second CTA of a one-chunk sequence factorises nothing, and with
+two or three chunks the first sends before the peer has anything to
+release) and the two-pass default (kda_chunk_fwd: the factorisation pass
+writes one package per (chunk, head), the chain kernel reads them)."""
 import numpy as np
 import pytest
 import torch
@@ -37,19 +40,29 @@ def oracle_packed(d, la_full):
                                 seq_offsets=d["offs"])
 
 
-@pytest.mark.parametrize("dk", [128, 64])
-def test_pair_path_is_taken(dk):
-    path, kernels, _ = K.chunk_fwd_plan(1, sum(LENGTHS), 3, dk, 128, 64,
-                                        torch.bfloat16, packed=True,
-                                        n_seqs=len(LENGTHS))
-    assert path == "fused" and kernels == 2  # order kernel + the pair kernel
+PATHS = ["paired", "twopass"]
+
+
+def call(path, *args, **kw):
+    return K.chunk_fwd(*args, paired=(path == "paired"), **kw)
 
 
 @pytest.mark.parametrize("dk", [128, 64])
-def test_pair_packed_chunk_counts(dk):
+def test_default_path_is_twopass(dk):
+    # order and chunk offsets of the packed layout, the factorisation pass,
+    # the chain kernel
+    path, kernels, ws = K.chunk_fwd_plan(1, sum(LENGTHS), 3, dk, 128, 64,
+                                         torch.bfloat16, packed=True,
+                                         n_seqs=len(LENGTHS))
+    assert path == "twopass" and kernels == 4 and ws > 0
+
+
+@pytest.mark.parametrize("path", PATHS)
+@pytest.mark.parametrize("dk", [128, 64])
+def test_pair_packed_chunk_counts(dk, path):
     d = packed(dk, seed=100 + dk)
-    out, fin = K.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"],
-                           d["initial_state"], d["cu"], chunk=64)
+    out, fin = call(path, d["q"], d["k"], d["v"], d["log_alpha"], d["beta"],
+                    d["initial_state"], d["cu"], chunk=64)
     assert K.device_status() == 0
     ro, rs = oracle_packed(d, d["log_alpha"])
     PY.check("out", PY.host64(out[0]), ro, PY.TOL_BF16)
@@ -58,8 +71,9 @@ def test_pair_packed_chunk_counts(dk):
     assert torch.equal(fin[4], d["initial_state"][4])
 
 
+@pytest.mark.parametrize("path", PATHS)
 @pytest.mark.parametrize("mode", ["head", "none"])
-def test_pair_gate_layouts(mode):
+def test_pair_gate_layouts(mode, path):
     d = packed(128, seed=7)
     if mode == "none":
         lg, la_full = None, torch.zeros_like(d["log_alpha"])
@@ -68,15 +82,16 @@ def test_pair_gate_layouts(mode):
         lg = (torch.nn.functional.logsigmoid(
             torch.randn(d["beta"].shape, generator=g, device=DEV)) / 16)
         la_full = lg[..., None].expand_as(d["log_alpha"]).contiguous()
-    out, fin = K.chunk_fwd(d["q"], d["k"], d["v"], lg, d["beta"],
-                           d["initial_state"], d["cu"], chunk=64, gate=mode)
+    out, fin = call(path, d["q"], d["k"], d["v"], lg, d["beta"],
+                    d["initial_state"], d["cu"], chunk=64, gate=mode)
     assert K.device_status() == 0
     ro, rs = oracle_packed(d, la_full)
     PY.check("out", PY.host64(out[0]), ro, PY.TOL_BF16)
     PY.check("final", PY.host64(fin), rs, PY.TOL_BF16)
 
 
-def test_pair_prologue():
+@pytest.mark.parametrize("path", PATHS)
+def test_pair_prologue(path):
     # raw (unnormalised) q, k and gate logits; the kernel normalises, scales
     # q by 1/sqrt(d_k) and maps the logits to log(alpha) = logsigmoid(x) / 16
     d = packed(128, seed=21)
@@ -86,8 +101,8 @@ def test_pair_prologue():
     logits = torch.randn(d["log_alpha"].shape, generator=g, device=DEV)
     pro = dict(normalize_qk=True, q_scale=128 ** -0.5, gate_logits=True,
                gate_scale=1.0 / 16)
-    out, fin = K.chunk_fwd(q_raw, k_raw, d["v"], logits, d["beta"],
-                           d["initial_state"], d["cu"], chunk=64, prologue=pro)
+    out, fin = call(path, q_raw, k_raw, d["v"], logits, d["beta"],
+                    d["initial_state"], d["cu"], chunk=64, prologue=pro)
     assert K.device_status() == 0
     qn, kn, la = kda_oracle.prologue(PY.host64(q_raw), PY.host64(k_raw),
                                      PY.host64(logits), normalize_qk=True,
@@ -101,23 +116,25 @@ def test_pair_prologue():
     PY.check("final", PY.host64(fin), rs, PY.TOL_BF16)
 
 
+@pytest.mark.parametrize("path", PATHS)
 @pytest.mark.parametrize("T", [64, 128, 192])
-def test_pair_dense_short(T):
+def test_pair_dense_short(T, path):
     # one, two and three chunks per sequence, no cu_seqlens
     d = W.draw((3, T), 2, 128, 128, io="bf16", n_states=3, device=DEV, seed=T)
-    out, fin = K.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"],
-                           d["initial_state"], None, chunk=64)
+    out, fin = call(path, d["q"], d["k"], d["v"], d["log_alpha"], d["beta"],
+                    d["initial_state"], None, chunk=64)
     assert K.device_status() == 0
     ro, rs = PY.oracle_dense(d)
     PY.check("out", PY.host64(out), ro, PY.TOL_BF16)
     PY.check("final", PY.host64(fin), rs, PY.TOL_BF16)
 
 
-def test_pair_is_deterministic():
+@pytest.mark.parametrize("path", PATHS)
+def test_pair_is_deterministic(path):
     # no atomics and a fixed hand-over order: two runs agree bit for bit
     d = packed(128, seed=5)
-    runs = [K.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"],
-                        d["initial_state"], d["cu"], chunk=64) for _ in range(2)]
+    runs = [call(path, d["q"], d["k"], d["v"], d["log_alpha"], d["beta"],
+                 d["initial_state"], d["cu"], chunk=64) for _ in range(2)]
     torch.cuda.synchronize()
     assert torch.equal(runs[0][0], runs[1][0])
     assert torch.equal(runs[0][1], runs[1][1])
