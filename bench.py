@@ -61,6 +61,28 @@ def prefill_flops(B, T, H, dk, dv, C):
     return B * T * H * (6 * dk * dv + 6 * C * dk + 4 * C * dv)
 
 
+def twopass_package_bytes(dk):
+    """Bytes of one (chunk, head) package that the two-pass prefill writes in
+    its factorisation pass and reads in its chain kernel: [W; Q~] (d_k/64
+    panels of 16 KiB), Kb (16 KiB), P and T' (8 KiB each) and the package
+    vector of 2 d_k + 4 floats."""
+    return (dk // 64) * 16384 + 16384 + 8192 + 8192 + (2 * dk + 4) * 4
+
+
+def twopass_design_bytes(B, T, H, dk, dv, C=64):
+    """HBM bytes of the two-pass design per call (dense layout): the
+    factorisation pass reads q, k (bf16), log_alpha and beta (fp32) and
+    writes one package per (chunk, head); the chain kernel reads each
+    package once (its d_v tiles run side by side and share it through L2)
+    and v, and writes o (bf16) and the fp32 final state.  Returns
+    (factor bytes, chain bytes)."""
+    th = B * T * H
+    pk = B * ((T + C - 1) // C) * H * twopass_package_bytes(dk)
+    factor = th * (2 * dk * 2 + dk * 4 + 4) + pk
+    chain = pk + th * dv * 2 * 2 + B * H * dk * dv * 4
+    return factor, chain
+
+
 def decode_bytes(N, H, dk, dv, io_bytes=2):
     """Algorithmic HBM bytes of one decode step: the fp32 state read and
     written, q, k, v, o (io dtype), log_alpha (fp32), beta (fp32)."""
@@ -250,9 +272,10 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
-def timed(fn, steps, stream):
+def timed(fn, steps, stream, events=None):
     """Run fn() `steps` times between CUDA events recorded on `stream`;
-    returns (total ms, per-step ms list)."""
+    returns (total ms, per-step ms list).  `events`, if given, receives the
+    steps + 1 boundary events."""
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
     ev[0].record(stream)
     for i in range(steps):
@@ -260,6 +283,8 @@ def timed(fn, steps, stream):
         ev[i + 1].record(stream)
     ev[-1].synchronize()
     per = [ev[i].elapsed_time(ev[i + 1]) for i in range(steps)]
+    if events is not None:
+        events.extend(ev)
     return ev[0].elapsed_time(ev[-1]), per
 
 
@@ -285,20 +310,46 @@ def run_kda(args, world, rank, local):
     out = torch.empty((B, T, H, dv), dtype=torch.bfloat16, device=dev)
     fin = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
 
-    def prefill(_i):
+    path = K.chunk_fwd_path(B, T, H, dk, dv, C, torch.bfloat16)
+    # two-pass calls record an event between their factorisation pass and
+    # their chain kernel: one per timed step, so the passes are timed apart
+    mids = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for m in mids:
+        m.record(stream)
+
+    def prefill(i):
+        if path == "twopass":
+            K.profile_pass_event(mids[i] if i < len(mids) else None)
         K.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], None,
                     None, chunk=C, out=out, final_state=fin)
 
     for i in range(args.warmup):
-        prefill(i)
+        prefill(args.steps + i)
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
     t0 = time.time()
-    ms, per = timed(prefill, args.steps, stream)
+    bounds = []
+    ms, per = timed(prefill, args.steps, stream, events=bounds)
     torch.cuda.synchronize()
+    K.profile_pass_event(None)
     clocks.mark(t0, time.time())
     barrier(world)
+    passes = None
+    if path == "twopass":
+        f_ms = statistics.mean(bounds[i].elapsed_time(mids[i])
+                               for i in range(args.steps))
+        c_ms = statistics.mean(mids[i].elapsed_time(bounds[i + 1])
+                               for i in range(args.steps))
+        f_b, c_b = twopass_design_bytes(B, T, H, dk, dv, C)
+        passes = [
+            {"kernel": "factor_kernel", "ms": f_ms, "design_bytes": f_b,
+             "achieved_gbs": f_b / (f_ms * 1e-3) / 1e9,
+             "frac": f_b / (f_ms * 1e-3) / 1e9 / pk["hbm_gbs"]},
+            {"kernel": "chain_kernel", "ms": c_ms, "design_bytes": c_b,
+             "achieved_gbs": c_b / (c_ms * 1e-3) / 1e9,
+             "frac": c_b / (c_ms * 1e-3) / 1e9 / pk["hbm_gbs"]},
+        ]
     ms = max_over_ranks(ms, world)
     ms_step = ms / args.steps
     launch_ms = statistics.mean(per)
@@ -652,7 +703,7 @@ def run_kda(args, world, rank, local):
                 "global_batch": B * world, "seq_len": T,
                 "parallelism": f"dp{world} (independent replicas)",
                 "l2": "inputs larger than L2 (no flush)",
-                "path": K.chunk_fwd_path(B, T, H, dk, dv, C, torch.bfloat16),
+                "path": path,
             },
             "roofline": {
                 "bound": "hbm", "achieved": achieved_gbs,
@@ -662,6 +713,15 @@ def run_kda(args, world, rank, local):
                 "peak_source": pk_kind,
                 "algorithmic_bytes_per_launch": pbytes,
                 "launch_ms": launch_ms,
+                "kernel": "the prefill call: factor_kernel then chain_kernel "
+                          "(per-kernel times in `passes`)",
+                "design_bytes_per_launch": (sum(p_["design_bytes"]
+                                                for p_ in passes)
+                                            if passes else None),
+                "design_frac": (sum(p_["design_bytes"] for p_ in passes)
+                                / (launch_ms * 1e-3) / 1e9 / pk["hbm_gbs"]
+                                if passes else None),
+                "passes": passes,
                 "tensor": {"achieved": achieved_tf, "peak": pk["bf16_tflops"],
                            "unit": "TFLOP/s",
                            "frac": achieved_tf / pk["bf16_tflops"],

@@ -647,6 +647,11 @@ kda_status kda_workspace_pool(size_t* reserved_bytes, size_t* used_bytes) {
   return KDA_OK;
 }
 
+kda_status kda_profile_pass_event(void* event) {
+  kda::set_pass_event(static_cast<cudaEvent_t>(event));
+  return KDA_OK;
+}
+
 int kda_last_cuda_error(void) { return g_last_cuda_error; }
 
 int kda_version(void) { return 100; }

@@ -172,6 +172,12 @@ size_t twopass_workspace_bytes(const ChunkArgs& a) {
 
 int twopass_kernel_count(const ChunkArgs& a) { return a.cu_seqlens ? 4 : 2; }
 
+namespace {
+thread_local cudaEvent_t t_pass_event = nullptr;
+}  // namespace
+void set_pass_event(cudaEvent_t e) { t_pass_event = e; }
+cudaEvent_t pass_event() { return t_pass_event; }
+
 cudaError_t launch_twopass(const ChunkArgs& a, void* workspace,
                            cudaStream_t stream) {
   return twopass::launch(a, workspace, stream);

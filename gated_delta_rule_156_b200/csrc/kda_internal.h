@@ -150,6 +150,11 @@ size_t twopass_workspace_bytes(const ChunkArgs& a);
 int twopass_kernel_count(const ChunkArgs& a);
 cudaError_t launch_twopass(const ChunkArgs& a, void* workspace,
                            cudaStream_t stream);
+// Profiling aid: an event the calling thread's two-pass launches record on
+// their stream between the factorisation pass and the chain kernel (null:
+// none).
+void set_pass_event(cudaEvent_t e);
+cudaEvent_t pass_event();
 
 // Upper bound on the number of chunks of a request (packed sequences may each
 // add one partial chunk).

@@ -65,6 +65,14 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* gsrc,
       "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
+// Until the bulk stores committed so far have read their shared-memory
+// source (the global writes complete on their own before the grid ends).
+__device__ __forceinline__ void bulk_commit_wait_read() {
+  asm volatile(
+      "cp.async.bulk.commit_group;\n\t"
+      "cp.async.bulk.wait_group.read 0;" ::
+          : "memory");
+}
 __device__ __forceinline__ void bulk_commit_wait_all() {
   asm volatile(
       "cp.async.bulk.commit_group;\n\t"
@@ -314,12 +322,13 @@ __global__ void __launch_bounds__(kFactorThreads, 2)
       tc_fence_before();
       fence_proxy_async();
       named_sync(kBarAll, kFactorThreads);
-      if (t == 0) {  // W and T' to HBM; every store completes before exit
+      if (t == 0) {  // W and T' to HBM; every store has read shared memory
+        // before exit
 #pragma unroll
         for (int q = 0; q < (int)PL::NP; ++q)
           bulk_store(gpk + q * 16384, kq + q * 16384, 8192);
         bulk_store(gpk + PL::s_tp, tp, 8192);
-        bulk_commit_wait_all();
+        bulk_commit_wait_read();
       }
     } else if (t == 0) {
       atomicExch(&g_fused_timeout, 1);
@@ -698,6 +707,8 @@ cudaError_t run(const ChunkArgs& a, void* workspace, cudaStream_t stream) {
   factor_kernel<DK, GATE><<<(unsigned)(nchunks * a.H), kFactorThreads, smem1,
                             stream>>>(tq, tk, p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (cudaEvent_t ev = pass_event())
+    if ((e = cudaEventRecord(ev, stream)) != cudaSuccess) return e;
   const size_t smem2 = ChainLayout<DK>::bytes + 1024;
   if ((e = cudaFuncSetAttribute(chain_kernel<DK>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,

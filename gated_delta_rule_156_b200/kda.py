@@ -27,7 +27,7 @@ EXPORTS = ("kda_chunk_fwd", "kda_chunk_fwd_staged", "kda_recurrent_step",
            "kda_recurrent_step_ex", "kda_selftest_timeout", "kda_chunk_bwd",
            "kda_chunk_bwd_plan", "kda_chunk_fwd_split", "kda_workspace_pool",
            "kda_chunk_fwd_twopass", "kda_chunk_fwd_paired",
-           "kda_chunk_fwd_split_plan")
+           "kda_chunk_fwd_split_plan", "kda_profile_pass_event")
 GATES = {"channel": 0, "head": 1, "none": 2}
 
 
@@ -144,6 +144,8 @@ def library():
         lib.kda_workspace_pool.restype = ctypes.c_int
         lib.kda_workspace_pool.argtypes = [ctypes.POINTER(ctypes.c_size_t),
                                            ctypes.POINTER(ctypes.c_size_t)]
+        lib.kda_profile_pass_event.restype = ctypes.c_int
+        lib.kda_profile_pass_event.argtypes = [ctypes.c_void_p]
         lib.kda_last_cuda_error.restype = ctypes.c_int
         lib.kda_last_cuda_error.argtypes = []
         lib.kda_version.restype = ctypes.c_int
@@ -427,6 +429,19 @@ def selftest_umma(A, B, a_mn, b_mn, panel_rows=None, stream=None):
     if st != KDA_OK:
         raise KdaError(st, "kda_selftest_umma")
     return D
+
+
+def profile_pass_event(event):
+    """Set (a torch.cuda.Event, already recorded once so that it exists) or
+    clear (None) the event that two-pass calls on this thread record between
+    their factorisation pass and their chain kernel
+    (kda_profile_pass_event)."""
+    h = None if event is None else ctypes.c_void_p(event.cuda_event)
+    if event is not None and not event.cuda_event:
+        raise ValueError("record the event once before passing it")
+    st = library().kda_profile_pass_event(h)
+    if st != 0:
+        raise KdaError(st, "kda_profile_pass_event")
 
 
 def workspace_pool():

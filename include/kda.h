@@ -519,6 +519,21 @@ KDA_API kda_status kda_selftest_timeout(int limit_us, cudaStream_t stream);
 KDA_API kda_status kda_workspace_pool(size_t* reserved_bytes,
                                       size_t* used_bytes);
 
+/*
+ * kda_profile_pass_event -- profiling aid for the two-pass prefill.  While
+ * `event` (a cudaEvent_t created by the caller, passed as void*) is set, every
+ * call made on this thread that runs the two-pass path (kda_chunk_fwd,
+ * kda_chunk_fwd_gated, kda_chunk_fwd_ex and kda_chunk_fwd_twopass on the
+ * bf16 shapes of the fused kernels, and the segment runs of
+ * kda_chunk_fwd_split) records it on its stream between the factorisation
+ * pass and the chain kernel, so that events recorded before and after the
+ * call time the two passes apart.  NULL clears it.  The event stays owned by
+ * the caller and must outlive the calls that record it.  Other paths ignore
+ * it.  Always returns KDA_OK; a failed record surfaces as the call's
+ * KDA_ERR_CUDA.
+ */
+KDA_API kda_status kda_profile_pass_event(void* event);
+
 /* The cudaError_t value behind the most recent KDA_ERR_CUDA on this thread
  * (0 if none). */
 KDA_API int kda_last_cuda_error(void);

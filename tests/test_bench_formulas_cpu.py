@@ -60,3 +60,24 @@ def test_prefill_flops_are_the_chunk_products():
     per_chunk = sum(2 * m * n * k for m, n, k in products)
     expect = B * H * (T // C) * per_chunk
     assert bench.prefill_flops(B, T, H, dk, dv, C) == expect == 94_489_280_512
+
+
+def test_twopass_design_bytes_count_the_package_round_trip():
+    # package: [W; Q~] panels (64 tokens x 64 channels, bf16, both halves),
+    # Kb (two 8 KiB panels), P and T' (64 x 64 bf16), and the vector of
+    # exp(g_C - rho), exp(rho) per channel plus the rho flag and padding
+    for dk in (64, 128):
+        panels = (dk // 64) * 2 * 64 * 64 * 2
+        expect = panels + 2 * 64 * 64 * 2 + 2 * (64 * 64 * 2) + (2 * dk + 4) * 4
+        assert bench.twopass_package_bytes(dk) == expect
+    assert bench.twopass_package_bytes(128) == 66_576
+    B, T, H, dk, dv = 2, 8192, 32, 128, 128
+    d = W.make(2, device="cpu")
+    inputs = nbytes(d["q"], d["k"], d["log_alpha"], d["beta"])
+    packages = B * (T // 64) * H * 66_576
+    out = torch.empty(B, T, H, dv, dtype=torch.bfloat16)
+    fin = torch.empty(B, H, dk, dv, dtype=torch.float32)
+    f, c = bench.twopass_design_bytes(B, T, H, dk, dv)
+    assert f == inputs + packages
+    assert c == packages + nbytes(d["v"], out, fin)
+    assert f + c == 1_902_379_008

@@ -124,3 +124,31 @@ def test_twopass_unsupported_shapes_rejected():
     with pytest.raises(K.KdaError):
         K.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"],
                     d["initial_state"], None, chunk=64, twopass=True)
+
+
+@pytest.mark.gpu
+def test_pass_event_times_the_two_passes_apart():
+    """kda_profile_pass_event: an event recorded between the factorisation
+    pass and the chain kernel splits the call's time into two positive
+    parts that add up to the whole."""
+    d = W.make(2, device="cuda")
+    out = torch.empty(d["v"].shape, dtype=torch.bfloat16, device="cuda")
+    fin = torch.empty((2, 32, 128, 128), dtype=torch.float32, device="cuda")
+    e0, mid, e1 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+    mid.record()
+    K.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], None, None,
+                chunk=64, out=out, final_state=fin)
+    e0.record()
+    K.profile_pass_event(mid)
+    try:
+        K.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], None,
+                    None, chunk=64, out=out, final_state=fin)
+    finally:
+        K.profile_pass_event(None)
+    e1.record()
+    torch.cuda.synchronize()
+    a, b, whole = e0.elapsed_time(mid), mid.elapsed_time(e1), e0.elapsed_time(e1)
+    assert a > 0 and b > 0
+    assert abs(a + b - whole) <= 1e-3 * whole + 1e-3
+    with pytest.raises(ValueError):
+        K.profile_pass_event(torch.cuda.Event())  # never recorded
