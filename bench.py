@@ -684,6 +684,8 @@ def run_kda(args, world, rank, local):
                    max(2.0, args.cpu_seconds / 3))}
 
     traffic = load_traffic()
+    for p_ in passes or []:
+        p_["traffic"] = traffic.get("prefill/kernels", {}).get(p_["kernel"])
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s",
@@ -835,6 +837,8 @@ def load_traffic():
                     h.update(src.read())
             if h.hexdigest() == rec["sha256"]:
                 out[name] = rec["bytes"]
+                if "kernels" in rec:  # per-kernel bytes of a multi-kernel call
+                    out[name + "/kernels"] = rec["kernels"]
     except Exception:
         return {}
     return out
