@@ -2,13 +2,14 @@
 // every (chunk, head) as one fully parallel pass, then the serial state chain
 // as a second kernel that only runs the state and output products.
 //
-// Pass 1, factor_kernel: one CTA of 256 threads per (chunk, head), two CTAs
-// per SM.  It forms the same chunk package the paired kernel hands from its
-// producer to its consumers (kda_fused_pair_sm100.cuh): [W; Qt] (W over Kt),
-// Kb, P, T' and the package vector (exp(g_C - rho), exp(rho), the rho flag),
-// in the same shared-memory layout, and writes it to an HBM workspace with
-// one bulk copy.  No CTA waits for another, so the factorisation of all
-// chunks runs side by side on every SM instead of along each sequence.
+// Pass 1, factor_kernel: CTAs of 256 threads, two per SM, each taking up to
+// four consecutive (chunk, head) items in turn.  Per item it forms the same
+// chunk package the paired kernel hands from its producer to its consumers
+// (kda_fused_pair_sm100.cuh): [W; Qt] (W over Kt), Kb, P, T' and the package
+// vector (exp(g_C - rho), exp(rho), the rho flag), in the same shared-memory
+// layout, and writes it to an HBM workspace with bulk copies.  No CTA waits
+// for another, so the factorisation of all chunks runs side by side on every
+// SM instead of along each sequence.
 //
 // Pass 2, chain_kernel: one CTA of 256 threads per (sequence, head,
 // 64-column d_v tile), two threads per TMEM lane (32 columns each).  Per chunk it bulk-loads the package (two ahead,
@@ -92,6 +93,8 @@ struct TwoPassParams {
   const int32_t* order;      // packed layout: longest sequence first
   uint8_t* packages;         // [max_chunks][H] packages of Lay::slot bytes
   int n_seqs, T, H, dv;
+  int n_items;        // (chunk, head) factorisations: max_chunks * H
+  int items_per_cta;  // consecutive items one factorisation CTA takes
 };
 
 template <int DK>
@@ -136,20 +139,13 @@ __global__ void __launch_bounds__(kFactorThreads, 2)
   uint64_t* bar_m2 = bars + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 4);
+  uint64_t* bar_fin = bars + 5;  // failure path: MMAs in flight drained
 
   const int t = threadIdx.x, warp = t >> 5;
   const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
   const int colh = warp >> 2, row_t = t & 127;
   const int cg = t % NCG, rb = t / NCG;
   const int pnl = cg >> 4;
-  // heads fastest: neighbouring CTAs read adjacent columns of the same rows
-  const int h = (int)(blockIdx.x % (unsigned)p.H);
-  const int cid = (int)(blockIdx.x / (unsigned)p.H);
-  uint8_t* gpk = p.packages + ((size_t)cid * p.H + h) * PL::slot;
-  int seq = 0, tok0 = 0, L = 0;
-  const int nc = (p.T + kC - 1) / kC;
-  const bool valid = locate_chunk(cid, p.cu, p.chunk_off, p.n_seqs, p.T, kC,
-                                  &seq, &tok0, &L);
 
   if (t == 0) {
     prefetch_tmap(&tm_q);
@@ -157,6 +153,7 @@ __global__ void __launch_bounds__(kFactorThreads, 2)
     mbar_init(bar_in, 1);
     mbar_init(bar_m1, 1);
     mbar_init(bar_m2, 1);
+    mbar_init(bar_fin, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -174,9 +171,22 @@ __global__ void __launch_bounds__(kFactorThreads, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  (void)nc;
 
-  if (valid) {
+  // The CTA takes items_per_cta consecutive items (chunk, head), heads
+  // fastest, so that neighbouring CTAs read adjacent columns of the same
+  // token rows; its set-up is paid once for all of them.  Each barrier
+  // completes once per item, so its parity alternates with the items done.
+  uint32_t ph = 0;
+  const int item0 = (int)blockIdx.x * p.items_per_cta;
+  const int item_end = min(item0 + p.items_per_cta, p.n_items);
+  for (int item = item0; item < item_end; ++item) {
+    const int h = item % p.H;
+    const int cid = item / p.H;
+    uint8_t* gpk = p.packages + ((size_t)cid * p.H + h) * PL::slot;
+    int seq = 0, tok0 = 0, L = 0;
+    if (!locate_chunk(cid, p.cu, p.chunk_off, p.n_seqs, p.T, kC, &seq, &tok0,
+                      &L))
+      continue;
     if (t == 0) {  // raw q and k: k over the Kt rows, q over the Qt rows
       mbar_arrive_expect_tx(bar_in, PL::tx_qk);
 #pragma unroll
@@ -208,7 +218,7 @@ __global__ void __launch_bounds__(kFactorThreads, 2)
       ldg_f1_if(b, p.beta + (size_t)(tok0 + t) * p.H + h, t < L);
       betas[t] = b;
     }
-    bool ok = wait_or_abort<true>(bar_in, 0, abort_flag);
+    bool ok = wait_or_abort<true>(bar_in, ph, abort_flag);
     bool failed = named_sync_or(kBarAll, kFactorThreads, !ok);
     if (!failed) {
       // ---- prologue, in place over the raw q and k
@@ -230,7 +240,7 @@ __global__ void __launch_bounds__(kFactorThreads, 2)
         }
         mma_commit(bar_m1);
       }
-      ok = wait_or_abort<false>(bar_m1, 0, abort_flag);
+      ok = wait_or_abort<false>(bar_m1, ph, abort_flag);
       failed = named_sync_or(kBarAll, kFactorThreads, !ok);
     }
     if (!failed) {
@@ -302,7 +312,7 @@ __global__ void __launch_bounds__(kFactorThreads, 2)
                    ks > 0);
         mma_commit(bar_m2);
       }
-      ok = wait_or_abort<false>(bar_m2, 0, abort_flag);
+      ok = wait_or_abort<false>(bar_m2, ph, abort_flag);
       failed = named_sync_or(kBarAll, kFactorThreads, !ok);
     }
     if (!failed) {
@@ -322,18 +332,24 @@ __global__ void __launch_bounds__(kFactorThreads, 2)
       tc_fence_before();
       fence_proxy_async();
       named_sync(kBarAll, kFactorThreads);
-      if (t == 0) {  // W and T' to HBM; every store has read shared memory
-        // before exit
+      if (t == 0) {  // W and T' to HBM; the next item's loads (or the
+        // exit) wait until every store has read shared memory
 #pragma unroll
         for (int q = 0; q < (int)PL::NP; ++q)
           bulk_store(gpk + q * 16384, kq + q * 16384, 8192);
         bulk_store(gpk + PL::s_tp, tp, 8192);
         bulk_commit_wait_read();
       }
-    } else if (t == 0) {
-      atomicExch(&g_fused_timeout, 1);
-      mbar_wait(bar_in, 0, 100000000ull);  // the q/k load, if still in flight
-      bulk_commit_wait_all();  // the early package stores read shared memory
+      ph ^= 1;
+    } else {
+      if (t == 0) {
+        atomicExch(&g_fused_timeout, 1);
+        mbar_wait(bar_in, ph, 100000000ull);  // the q/k load, if in flight
+        mma_commit(bar_fin);                  // and the MMAs
+        mbar_wait(bar_fin, 0, 100000000ull);
+        bulk_commit_wait_all();  // the early package stores read shared memory
+      }
+      break;  // failed is the same in every thread
     }
   }
   tc_fence_before();
@@ -704,8 +720,22 @@ cudaError_t run(const ChunkArgs& a, void* workspace, cudaStream_t stream) {
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)smem1)) != cudaSuccess)
     return e;
-  factor_kernel<DK, GATE><<<(unsigned)(nchunks * a.H), kFactorThreads, smem1,
-                            stream>>>(tq, tk, p);
+  p.n_items = (int)(nchunks * a.H);
+  {  // items per CTA: 4, 2 or 1, whichever still leaves two resident waves
+    int dev = 0, sms = 0, per_sm = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount,
+                                    dev)) != cudaSuccess ||
+        (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+             &per_sm, factor_kernel<DK, GATE>, kFactorThreads, smem1)) !=
+            cudaSuccess)
+      return e;
+    const int64_t wave = (int64_t)sms * (per_sm > 0 ? per_sm : 1);
+    p.items_per_cta = p.n_items >= 8 * wave ? 4 : p.n_items >= 4 * wave ? 2 : 1;
+  }
+  const unsigned grid1 =
+      (unsigned)((p.n_items + p.items_per_cta - 1) / p.items_per_cta);
+  factor_kernel<DK, GATE><<<grid1, kFactorThreads, smem1, stream>>>(tq, tk, p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (cudaEvent_t ev = pass_event())
     if ((e = cudaEventRecord(ev, stream)) != cudaSuccess) return e;
