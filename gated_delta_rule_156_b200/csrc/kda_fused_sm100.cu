@@ -170,6 +170,20 @@ size_t twopass_workspace_bytes(const ChunkArgs& a) {
   return twopass::workspace_bytes(a);
 }
 
+size_t twopass_chain_workspace_bytes(const ChunkArgs& a) {
+  return twopass::workspace_bytes(a, true);
+}
+
+int twopass_chain_kernel_count(const ChunkArgs& a) {
+  return a.cu_seqlens ? 3 : 1;
+}
+
+const void* twopass_packages(const ChunkArgs& a, const void* workspace,
+                             int64_t first_chunk) {
+  return twopass::packages_in(a, const_cast<void*>(workspace)) +
+         (size_t)first_chunk * a.H * twopass::package_slot(a.dk);
+}
+
 int twopass_kernel_count(const ChunkArgs& a) { return a.cu_seqlens ? 4 : 2; }
 
 namespace {
@@ -179,8 +193,14 @@ void set_pass_event(cudaEvent_t e) { t_pass_event = e; }
 cudaEvent_t pass_event() { return t_pass_event; }
 
 cudaError_t launch_twopass(const ChunkArgs& a, void* workspace,
-                           cudaStream_t stream) {
-  return twopass::launch(a, workspace, stream);
+                           cudaStream_t stream, cudaEvent_t factor_done) {
+  return twopass::launch(a, workspace, stream, nullptr, factor_done);
+}
+
+cudaError_t launch_twopass_chain(const ChunkArgs& a, void* workspace,
+                                 const void* packages, cudaStream_t stream) {
+  return twopass::launch(a, workspace, stream,
+                         static_cast<const uint8_t*>(packages), nullptr);
 }
 
 cudaError_t launch_fused(const ChunkArgs& a, void* workspace,

@@ -149,7 +149,20 @@ cudaError_t launch_fused(const ChunkArgs& a, void* workspace,
 size_t twopass_workspace_bytes(const ChunkArgs& a);
 int twopass_kernel_count(const ChunkArgs& a);
 cudaError_t launch_twopass(const ChunkArgs& a, void* workspace,
-                           cudaStream_t stream);
+                           cudaStream_t stream,
+                           cudaEvent_t factor_done = nullptr);
+// The chain kernel alone, over packages another call's factorisation pass
+// wrote (the layouts must agree chunk for chunk from `packages` on): for a
+// run whose q, k, log alpha and beta are a shifted copy of that call's.  Its
+// workspace holds only the packed layout's order and offsets.
+size_t twopass_chain_workspace_bytes(const ChunkArgs& a);
+int twopass_chain_kernel_count(const ChunkArgs& a);
+cudaError_t launch_twopass_chain(const ChunkArgs& a, void* workspace,
+                                 const void* packages, cudaStream_t stream);
+// Where the package of chunk `first_chunk` (of a's layout) starts in a
+// two-pass workspace.
+const void* twopass_packages(const ChunkArgs& a, const void* workspace,
+                             int64_t first_chunk);
 // Profiling aid: an event the calling thread's two-pass launches record on
 // their stream between the factorisation pass and the chain kernel (null:
 // none).

@@ -17,10 +17,13 @@
 //   (3) scan: S_in(1) = S_end(0); S_in(j+1) = M_end(j) S_in(j) + S_end|0(j);
 //       the last step gives the final state;
 //   (4) correction: o_t += S_in(j)^T X_t for the tokens of segments 1..n-1.
-// Steps (1) and (2) run the library's own prefill kernels (fused or
-// four-stage, as kda_chunk_fwd would pick for their shapes); (3) is an fp32
-// kernel below, and (4) a tcgen05 product for bf16 io with d in {64, 128}
-// (an fp32 register-blocked product otherwise).
+// Steps (1) and (2) run the library's own prefill kernels (two-pass or
+// four-stage, as kda_chunk_fwd would pick for their shapes).  On the two-pass
+// path step (2) runs only its chain kernel, over the packages step (1)'s
+// factorisation pass wrote: the transition run's q, k, log alpha and beta are
+// step (1)'s from segment 1 on, and a package does not depend on v.  (3) is
+// an fp32 kernel below, and (4) a tcgen05 product for bf16 io with d in
+// {64, 128} (an fp32 register-blocked product otherwise).
 #include <mutex>
 #include <type_traits>
 
@@ -111,6 +114,19 @@ cudaError_t run_forward(const ChunkArgs& a, void* ws, cudaStream_t s) {
   return fused_supported(a) ? launch_twopass(a, ws, s) : launch_staged(a, ws, s);
 }
 
+// On the two-pass path the transition run reads the value run's packages:
+// its q, k, log alpha and beta are the value run's from segment 1 on, and a
+// package does not depend on v, so only its chain kernel runs.
+bool shares_packages(const ChunkArgs& value) { return fused_supported(value); }
+size_t trans_workspace(const ChunkArgs& value, const ChunkArgs& trans) {
+  return shares_packages(value) ? twopass_chain_workspace_bytes(trans)
+                                : run_workspace(trans);
+}
+int trans_kernels(const ChunkArgs& value, const ChunkArgs& trans) {
+  return shares_packages(value) ? twopass_chain_kernel_count(trans)
+                                : run_kernels(trans);
+}
+
 // Sizes and kernel counts depend on whether cu_seqlens is present, not on its
 // contents: while planning (no workspace yet) the offsets point at a tag.
 const int32_t kPlanTag = 0;
@@ -146,7 +162,7 @@ SplitWs carve_split(const ChunkArgs& a, const SplitGeom& g, void* base,
   // the two runs' own workspaces: sized for the packed layout they run in
   const SplitWs probe = tagged(w);
   w.ws_val = take(run_workspace(value_args(a, g, probe)));
-  w.ws_tr = take(run_workspace(trans_args(a, g, probe)));
+  w.ws_tr = take(trans_workspace(value_args(a, g, probe), trans_args(a, g, probe)));
   if (total) *total = off;
   return w;
 }
@@ -648,17 +664,45 @@ cudaError_t run_split(const ChunkArgs& a, const SplitGeom& g, void* workspace,
   };
   if ((e = cudaEventRecord(fork, stream)) != cudaSuccess) return done(e);
   if ((e = cudaStreamWaitEvent(side, fork, 0)) != cudaSuccess) return done(e);
-  // whatever fails below, `stream` waits for the side stream before the
-  // caller can release the workspace
-  const cudaError_t e_tr = run_forward(trans_args(a, g, w), w.ws_tr, side);
-  const cudaError_t e_rec = cudaEventRecord(join, side);
-  const cudaError_t e_val =
-      e_tr == cudaSuccess ? run_forward(value_args(a, g, w), w.ws_val, stream)
-                          : cudaSuccess;
-  const cudaError_t e_wait =
-      e_rec == cudaSuccess ? cudaStreamWaitEvent(stream, join, 0) : e_rec;
-  for (cudaError_t r : {e_tr, e_rec, e_val, e_wait})
-    if (r != cudaSuccess) return done(r);
+  const ChunkArgs va = value_args(a, g, w), ta = trans_args(a, g, w);
+  if (shares_packages(va)) {
+    // the value run on `stream`; once its factorisation pass is done, the
+    // transition run's chain on the side stream over the same packages from
+    // segment 1 on (segment 0 holds Ls / C chunks)
+    cudaEvent_t factored = nullptr;
+    if ((e = cudaEventCreateWithFlags(&factored, cudaEventDisableTiming)) !=
+        cudaSuccess)
+      return done(e);
+    const cudaError_t e_val = launch_twopass(va, w.ws_val, stream, factored);
+    const cudaError_t e_dep =
+        e_val == cudaSuccess ? cudaStreamWaitEvent(side, factored, 0) : e_val;
+    const cudaError_t e_tr =
+        e_dep == cudaSuccess
+            ? launch_twopass_chain(
+                  ta, w.ws_tr,
+                  twopass_packages(va, w.ws_val, (int64_t)(g.Ls / a.chunk)),
+                  side)
+            : cudaSuccess;
+    // whatever failed, `stream` waits for the side stream before the
+    // caller can release the workspace
+    const cudaError_t e_rec = cudaEventRecord(join, side);
+    const cudaError_t e_wait =
+        e_rec == cudaSuccess ? cudaStreamWaitEvent(stream, join, 0) : e_rec;
+    cudaEventDestroy(factored);
+    for (cudaError_t r : {e_val, e_dep, e_tr, e_rec, e_wait})
+      if (r != cudaSuccess) return done(r);
+  } else {
+    // whatever fails below, `stream` waits for the side stream before the
+    // caller can release the workspace
+    const cudaError_t e_tr = run_forward(ta, w.ws_tr, side);
+    const cudaError_t e_rec = cudaEventRecord(join, side);
+    const cudaError_t e_val =
+        e_tr == cudaSuccess ? run_forward(va, w.ws_val, stream) : cudaSuccess;
+    const cudaError_t e_wait =
+        e_rec == cudaSuccess ? cudaStreamWaitEvent(stream, join, 0) : e_rec;
+    for (cudaError_t r : {e_tr, e_rec, e_val, e_wait})
+      if (r != cudaSuccess) return done(r);
+  }
   done(cudaSuccess);
 
   // (3) scan, (4) correction
@@ -735,8 +779,8 @@ int split_kernel_count(const ChunkArgs& a, const SplitGeom& g) {
   if (g.k <= 1) return run_kernels(a);
   const SplitWs w = tagged(SplitWs{});
   // setup, the two runs, scan, correction
-  return 1 + run_kernels(value_args(a, g, w)) + run_kernels(trans_args(a, g, w)) +
-         2;
+  return 1 + run_kernels(value_args(a, g, w)) +
+         trans_kernels(value_args(a, g, w), trans_args(a, g, w)) + 2;
 }
 
 cudaError_t launch_split(const ChunkArgs& a, const SplitGeom& g, void* workspace,

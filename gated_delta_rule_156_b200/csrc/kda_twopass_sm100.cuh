@@ -668,23 +668,37 @@ __global__ void chunk_offsets_kernel(const int32_t* __restrict__ cu, int n_seqs,
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Workspace: the longest-first order and the chunk offsets (packed layout),
-// then one package per (chunk, head).
-inline size_t workspace_bytes(const ChunkArgs& a) {
-  const size_t slot = a.dk == 128 ? PairLayout<128>::slot : PairLayout<64>::slot;
-  size_t off = 0;
-  if (a.cu_seqlens)
-    off = align256((size_t)a.n_seqs * 4) + align256(((size_t)a.n_seqs + 1) * 4);
-  return off + (size_t)max_chunks(a) * a.H * slot;
+// then one package per (chunk, head) unless the chain reads packages kept
+// elsewhere (chain_only).
+inline size_t package_slot(int dk) {
+  return dk == 128 ? PairLayout<128>::slot : PairLayout<64>::slot;
+}
+inline size_t index_bytes(const ChunkArgs& a) {
+  return a.cu_seqlens
+             ? align256((size_t)a.n_seqs * 4) + align256(((size_t)a.n_seqs + 1) * 4)
+             : 0;
+}
+inline size_t workspace_bytes(const ChunkArgs& a, bool chain_only = false) {
+  return index_bytes(a) +
+         (chain_only ? 0 : (size_t)max_chunks(a) * a.H * package_slot(a.dk));
+}
+inline uint8_t* packages_in(const ChunkArgs& a, void* workspace) {
+  return static_cast<uint8_t*>(workspace) + index_bytes(a);
 }
 
+// One call: the packed layout's order and chunk offsets, then (unless
+// `packages` is given) the factorisation pass into the workspace, an event
+// (factor_done, if given) and the chain kernel.  With `packages` given only
+// the chain runs, reading the packages there: chunk c of this call's layout,
+// head h, at packages + (c * H + h) * slot.
 template <int DK, int GATE>
-cudaError_t run(const ChunkArgs& a, void* workspace, cudaStream_t stream) {
-  using PL = PairLayout<DK>;
+cudaError_t run(const ChunkArgs& a, void* workspace, cudaStream_t stream,
+                const uint8_t* packages, cudaEvent_t factor_done) {
   const int tokens = a.cu_seqlens ? a.T : a.n_seqs * a.T;
   CUtensorMap tq, tk, tv;
-  if (!make_tile_map(&tq, a.q, DK, a.H, tokens) ||
-      !make_tile_map(&tk, a.k, DK, a.H, tokens) ||
-      !make_tile_map(&tv, a.v, a.dv, a.H, tokens))
+  if (!make_tile_map(&tv, a.v, a.dv, a.H, tokens)) return cudaErrorInvalidValue;
+  if (!packages && (!make_tile_map(&tq, a.q, DK, a.H, tokens) ||
+                    !make_tile_map(&tk, a.k, DK, a.H, tokens)))
     return cudaErrorInvalidValue;
   TwoPassParams p{};
   p.pro = a.pro;
@@ -711,34 +725,41 @@ cudaError_t run(const ChunkArgs& a, void* workspace, cudaStream_t stream) {
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     p.order = order;
     p.chunk_off = coff;
-    ws += align256((size_t)a.n_seqs * 4) + align256(((size_t)a.n_seqs + 1) * 4);
   }
-  p.packages = ws;
-  const int64_t nchunks = max_chunks(a);
-  const size_t smem1 = FactorLayout<DK>::bytes + 1024;
-  if ((e = cudaFuncSetAttribute(factor_kernel<DK, GATE>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)smem1)) != cudaSuccess)
-    return e;
-  p.n_items = (int)(nchunks * a.H);
-  {  // items per CTA: 4, 2 or 1, whichever still leaves two resident waves
-    int dev = 0, sms = 0, per_sm = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
-        (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount,
-                                    dev)) != cudaSuccess ||
-        (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-             &per_sm, factor_kernel<DK, GATE>, kFactorThreads, smem1)) !=
-            cudaSuccess)
+  if (packages) {
+    p.packages = const_cast<uint8_t*>(packages);
+  } else {
+    p.packages = packages_in(a, workspace);
+    const int64_t nchunks = max_chunks(a);
+    const size_t smem1 = FactorLayout<DK>::bytes + 1024;
+    if ((e = cudaFuncSetAttribute(factor_kernel<DK, GATE>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)smem1)) != cudaSuccess)
       return e;
-    const int64_t wave = (int64_t)sms * (per_sm > 0 ? per_sm : 1);
-    p.items_per_cta = p.n_items >= 8 * wave ? 4 : p.n_items >= 4 * wave ? 2 : 1;
+    p.n_items = (int)(nchunks * a.H);
+    {  // items per CTA: 4, 2 or 1, whichever still leaves two resident waves
+      int dev = 0, sms = 0, per_sm = 0;
+      if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
+          (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount,
+                                      dev)) != cudaSuccess ||
+          (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+               &per_sm, factor_kernel<DK, GATE>, kFactorThreads, smem1)) !=
+              cudaSuccess)
+        return e;
+      const int64_t wave = (int64_t)sms * (per_sm > 0 ? per_sm : 1);
+      p.items_per_cta =
+          p.n_items >= 8 * wave ? 4 : p.n_items >= 4 * wave ? 2 : 1;
+    }
+    const unsigned grid1 =
+        (unsigned)((p.n_items + p.items_per_cta - 1) / p.items_per_cta);
+    factor_kernel<DK, GATE><<<grid1, kFactorThreads, smem1, stream>>>(tq, tk,
+                                                                      p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (cudaEvent_t ev = pass_event())
+      if ((e = cudaEventRecord(ev, stream)) != cudaSuccess) return e;
+    if (factor_done)
+      if ((e = cudaEventRecord(factor_done, stream)) != cudaSuccess) return e;
   }
-  const unsigned grid1 =
-      (unsigned)((p.n_items + p.items_per_cta - 1) / p.items_per_cta);
-  factor_kernel<DK, GATE><<<grid1, kFactorThreads, smem1, stream>>>(tq, tk, p);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  if (cudaEvent_t ev = pass_event())
-    if ((e = cudaEventRecord(ev, stream)) != cudaSuccess) return e;
   const size_t smem2 = ChainLayout<DK>::bytes + 1024;
   if ((e = cudaFuncSetAttribute(chain_kernel<DK>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -746,20 +767,23 @@ cudaError_t run(const ChunkArgs& a, void* workspace, cudaStream_t stream) {
     return e;
   const unsigned grid2 = (unsigned)a.n_seqs * a.H * (a.dv / kDvt);
   chain_kernel<DK><<<grid2, kChainThreads, smem2, stream>>>(tv, p);
-  (void)sizeof(PL);
   return cudaGetLastError();
 }
 
 inline cudaError_t launch(const ChunkArgs& a, void* workspace,
-                          cudaStream_t stream) {
+                          cudaStream_t stream, const uint8_t* packages = nullptr,
+                          cudaEvent_t factor_done = nullptr) {
   if (a.gate == kGateHead)
-    return a.dk == 128 ? run<128, kGateHead>(a, workspace, stream)
-                       : run<64, kGateHead>(a, workspace, stream);
+    return a.dk == 128
+               ? run<128, kGateHead>(a, workspace, stream, packages, factor_done)
+               : run<64, kGateHead>(a, workspace, stream, packages, factor_done);
   if (a.gate == kGateNone)
-    return a.dk == 128 ? run<128, kGateNone>(a, workspace, stream)
-                       : run<64, kGateNone>(a, workspace, stream);
-  return a.dk == 128 ? run<128, kGateChannel>(a, workspace, stream)
-                     : run<64, kGateChannel>(a, workspace, stream);
+    return a.dk == 128
+               ? run<128, kGateNone>(a, workspace, stream, packages, factor_done)
+               : run<64, kGateNone>(a, workspace, stream, packages, factor_done);
+  return a.dk == 128
+             ? run<128, kGateChannel>(a, workspace, stream, packages, factor_done)
+             : run<64, kGateChannel>(a, workspace, stream, packages, factor_done);
 }
 
 }  // namespace twopass

@@ -450,7 +450,9 @@ KDA_API kda_status kda_chunk_bwd_plan(const kda_shape* shape, int packed,
  *   3. scans: S_in(1) = S_end(0), S_in(j+1) = M_end(j) S_in(j) + S_end|0(j);
  *      the last step writes final_state;
  *   4. adds S_in(j)^T (M_t^T q_t) to the outputs of segments 1..n-1.
- * Steps 1 and 2 run the path kda_chunk_fwd picks for their shapes.  Step 3
+ * Steps 1 and 2 run the path kda_chunk_fwd picks for their shapes; on the
+ * two-pass path step 2 runs only its chain kernel, over the packages step 1
+ * wrote (a package does not depend on v).  Step 3
  * is fp32.  Step 4 runs on the tensor cores (bf16 operands, fp32
  * accumulation) for bf16 io with d_k, d_v in {64, 128}, and in fp32
  * otherwise.  Segments are ceil(chunks / n_segments) chunks long, rounded

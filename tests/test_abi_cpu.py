@@ -73,11 +73,16 @@ def test_backward_plan(lib):
 def test_split_plan(lib):
     import torch
     # plan: segments of ceil(chunks / n) chunks; the kernels are the setup,
-    # both runs (four launches each on the two-pass packed path: order,
-    # chunk offsets, factorisation, chain), scan and fix
+    # the value run (order, chunk offsets, factorisation, chain on the
+    # two-pass packed path), the transition run (order, chunk offsets and a
+    # chain over the value run's packages), scan and fix
     seg, kern, ws = K.chunk_fwd_split_plan(131072, 8, 128, 128, 64,
                                            torch.bfloat16, 4)
-    assert seg == 4 and kern == 1 + 4 + 4 + 2 and ws > 0
+    assert seg == 4 and kern == 1 + 4 + 3 + 2 and ws > 0
+    # the fp32 path runs both four-stage pipelines in full
+    seg32, kern32, _ = K.chunk_fwd_split_plan(131072, 8, 128, 128, 64,
+                                              torch.float32, 4)
+    assert seg32 == 4 and kern32 > kern
     seg, kern, ws = K.chunk_fwd_split_plan(1000, 2, 64, 64, 64,
                                            torch.float32, 7)
     assert seg == 6  # 16 chunks in segments of 3
