@@ -69,7 +69,8 @@ __global__ void __launch_bounds__((DV / 4) * kRowGroups)
                   : gate == kGateHead  ? log_alpha[tok * H + h]
                                        : 0.f;
         if (pro.gate_logits && gate != kGateNone)  // scale * logsigmoid(l)
-          l = pro.gate_scale * (fminf(l, 0.f) - log1pf(__expf(-fabsf(l))));
+          // log1p(e) as log(1 + e), e <= 1: under 6e-8 apart
+          l = pro.gate_scale * (fminf(l, 0.f) - __logf(1.f + __expf(-fabsf(l))));
         s_a[c] = __expf(l);
       }
     }

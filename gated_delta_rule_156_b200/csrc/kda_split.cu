@@ -728,7 +728,7 @@ cudaError_t run_split(const ChunkArgs& a, const SplitGeom& g, void* workspace,
 
 int split_auto_segments(const ChunkArgs& a, int num_sms) {
   // CTAs one segment's chain occupies: one per head and 64-wide value tile
-  // (the paired kernel's two CTAs at d_v = 128); the transition run has
+  // (the chain kernel's two CTAs at d_v = 128); the transition run has
   // d_v = d_k, so take the wider of the two
   const int wide = a.dv > a.dk ? a.dv : a.dk;
   const int per_seg = a.H * (wide > 64 ? wide / 64 : 1);
