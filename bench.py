@@ -563,7 +563,8 @@ def run_kda(args, world, rank, local):
         del ds, outs, fins
 
     # ---- backward pass of the prefill workload: every input's gradient for
-    # a random output gradient (fp32 arithmetic, chunkwise) ----------------
+    # a random output gradient (chunkwise; fp32 products, the forward's
+    # state pass on the tensor cores for bf16 inputs) -----------------------
     gdo = torch.randn(d["v"].shape, generator=torch.Generator(device=dev)
                       .manual_seed(77 + rank), device=dev).bfloat16()
 
@@ -590,7 +591,7 @@ def run_kda(args, world, rank, local):
         "value": world * B * T / (bwms / bw_steps * 1e-3), "unit": "tokens/s",
         "ms_per_step": bwms / bw_steps, "steps": bw_steps,
         "workload": "kda_chunk_bwd on the prefill workload (dq, dk, dv, "
-                    "dlog_alpha, dbeta), fp32 arithmetic",
+                    "dlog_alpha, dbeta), fp32 products, tensor-core state pass",
         "hbm": {"achieved": bw_bytes / (bw_launch * 1e-3) / 1e9, "unit": "GB/s",
                 "frac": bw_bytes / (bw_launch * 1e-3) / 1e9 / pk["hbm_gbs"],
                 "algorithmic_bytes_per_launch": bw_bytes},

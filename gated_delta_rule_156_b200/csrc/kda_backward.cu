@@ -1,4 +1,6 @@
-// Chunkwise backward pass of the KDA forward, all arithmetic in fp32 (SIMT).
+// Chunkwise backward pass of the KDA forward, in fp32 SIMT arithmetic except
+// for the forward's state pass with bf16 inputs in 64-token chunks, which is
+// the tensor-core two-pass forward (bf16 operands, fp32 accumulators).
 //
 // The gradients of L = <dO, O> + <dS_T, S_T> follow from the chain rule
 // applied to each line of the chunkwise forward (the forward's own chunk
@@ -29,7 +31,9 @@
 //   - stage (1) of the four-stage forward (g);
 //   - a prep kernel per (chunk, head): Kt, Kb, Qt, b Kt, P and Tm, plus the
 //     forward's own W, U and Kh, so the forward's stage (2) is not run;
-//   - the forward's state pass (stage 3): Delta and every chunk-start state;
+//   - the forward's state pass: Delta and every chunk-start state (stage 3
+//     of the four-stage forward, or the two-pass forward with its outputs
+//     switched off);
 //   - the two products that do not depend on dS, Qt^T dO and P^T dO;
 //   - the reverse chain per (sequence, head, 32-column d_v tile), which
 //     keeps only dDelta and the dS update in its serial loop and takes
@@ -61,6 +65,7 @@ struct BwdWs {
   StagedView fv;
   void* staged;                   // the forward's workspace
   float* fin;                     // scratch final state of the forward
+  void* tp;                       // the two-pass forward's workspace, or null
   float *kt, *kb, *qt, *bkt;      // [tokens, H, dk]
   float *v32, *bv, *do32, *dd;    // [tokens, H, dv]
   float *tm, *pp;                 // [chunks, H, C, C]
@@ -83,6 +88,14 @@ ChunkArgs forward_args(const BwdArgs& a, float* fin) {
   return f;
 }
 
+// The forward's state pass runs as the tensor-core two-pass forward where
+// that path takes the shape (bf16 inputs, 64-token chunks, d_k and d_v in
+// {64, 128}); its bf16 operands sit inside the bf16 tolerance.  fp32 inputs
+// keep the fp32 SIMT pass.
+bool tensor_state_pass(const ChunkArgs& f) {
+  return fused_supported(f) && max_chunks(f) > 0;
+}
+
 BwdWs carve_bwd(const BwdArgs& a, void* base, size_t* total) {
   const ChunkArgs& f = a.f;
   const size_t tokens =
@@ -100,6 +113,7 @@ BwdWs carve_bwd(const BwdArgs& a, void* base, size_t* total) {
   w.fin = take(4 * (size_t)f.n_seqs * H * dk * dv);
   const ChunkArgs fa = forward_args(a, nullptr);
   w.staged = take(staged_workspace_bytes(fa));
+  w.tp = tensor_state_pass(fa) ? take(twopass_workspace_bytes(fa)) : nullptr;
   const size_t tdk = 4 * tokens * H * dk, tdv = 4 * tokens * H * dv;
   const size_t sq = 4 * nch * H * C * C, st = 4 * nch * H * dk * dv;
   w.kt = take(tdk); w.kb = take(tdk); w.qt = take(tdk); w.bkt = take(tdk);
@@ -866,9 +880,14 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   // the forward's serial state pass: chunk-start states, Delta over U, and
-  // the final state
-  if ((e = launch_staged_part(f, w.staged, &w.fv, true, stream)) != cudaSuccess)
-    return e;
+  // the final state; with bf16 inputs in 64-token chunks the tensor-core
+  // two-pass forward, which writes the states and Delta in fp32 from its
+  // accumulators and no outputs
+  e = tensor_state_pass(f)
+          ? launch_twopass_save(f, w.tp, const_cast<float*>(w.fv.s), w.fv.d,
+                                stream)
+          : launch_staged_part(f, w.staged, &w.fv, true, stream);
+  if (e != cudaSuccess) return e;
 
   auto tok = [](float* p, int cols, int t = 0) { return MatRef{p, kTok, cols, t}; };
   auto sq = [&](float* p, int t = 0) { return MatRef{p, kSq, C, t}; };
@@ -994,10 +1013,13 @@ int bwd_kernel_count(const BwdArgs& a) {
   const ChunkArgs f = forward_args(a, nullptr);
   if (f.n_seqs == 0 || f.H == 0) return 0;
   const bool any = max_chunks(f) > 0;
-  // the plan (packed layout), the forward's state pass and the reverse
-  // chain always; with any chunk also the cumulative log-decay, prep, the
-  // batched products and the final combination
-  return (f.cu_seqlens ? 1 : 0) + 2 + (any ? 1 + 1 + kBmmOps + 1 : 0);
+  // the plan (packed layout), the forward's state pass (one SIMT kernel, or
+  // the two-pass forward's launches) and the reverse chain always; with any
+  // chunk also the cumulative log-decay, prep, the batched products and the
+  // final combination
+  const int state = tensor_state_pass(f) ? twopass_kernel_count(f) : 1;
+  return (f.cu_seqlens ? 1 : 0) + state + 1 +
+         (any ? 1 + 1 + kBmmOps + 1 : 0);
 }
 
 cudaError_t launch_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {

@@ -105,7 +105,8 @@ cudaError_t launch_split(const ChunkArgs& a, const SplitGeom& g, void* workspace
 
 // Chunkwise backward pass (kda_backward.cu): the gradients of
 // L = <d_out, out> + <d_final_state, final_state> with respect to q, k, v,
-// log(alpha), beta and the initial state, all arithmetic in fp32.
+// log(alpha), beta and the initial state, in fp32 arithmetic (the forward's
+// state pass with bf16 inputs in 64-token chunks runs on the tensor cores).
 struct BwdArgs {
   ChunkArgs f;                  // forward arguments; f.out, f.final_state unused
   const void* d_out;            // [tokens, H, dv], io dtype
@@ -159,6 +160,14 @@ size_t twopass_chain_workspace_bytes(const ChunkArgs& a);
 int twopass_chain_kernel_count(const ChunkArgs& a);
 cudaError_t launch_twopass_chain(const ChunkArgs& a, void* workspace,
                                  const void* packages, cudaStream_t stream);
+// The two-pass forward for the backward pass: a.out may be null (no outputs
+// written); every chunk-start state goes to save_s [max_chunks, H, dk, dv]
+// and Delta = U - W S_0 to save_delta [tokens, H, dv], both fp32, in the
+// chunk numbering of the packed layout's offsets (the dense layout: sequence
+// s, chunk c -> s * ceil(T / C) + c).
+cudaError_t launch_twopass_save(const ChunkArgs& a, void* workspace,
+                                float* save_s, float* save_delta,
+                                cudaStream_t stream);
 // Where the package of chunk `first_chunk` (of a's layout) starts in a
 // two-pass workspace.
 const void* twopass_packages(const ChunkArgs& a, const void* workspace,
