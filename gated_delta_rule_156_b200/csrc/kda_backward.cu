@@ -1,6 +1,7 @@
 // Chunkwise backward pass of the KDA forward, in fp32 SIMT arithmetic except
-// for the forward's state pass with bf16 inputs in 64-token chunks, which is
-// the tensor-core two-pass forward (bf16 operands, fp32 accumulators).
+// with bf16 inputs in 64-token chunks: there the forward's state pass is the
+// tensor-core two-pass forward (bf16 operands, fp32 accumulators) and the
+// reverse chain runs on the tensor cores in tf32 (kda_bwd_chain_tc.cuh).
 //
 // The gradients of L = <dO, O> + <dS_T, S_T> follow from the chain rule
 // applied to each line of the chunkwise forward (the forward's own chunk
@@ -35,7 +36,8 @@
 //     of the four-stage forward, or the two-pass forward with its outputs
 //     switched off);
 //   - the two products that do not depend on dS, Qt^T dO and P^T dO;
-//   - the reverse chain per (sequence, head, 32-column d_v tile), which
+//   - the reverse chain per (sequence, head, 32-column d_v tile; 64 columns
+//     on the tensor cores), which
 //     keeps only dDelta and the dS update in its serial loop and takes
 //     gam * d gam = rowsum(S_next * dS_C) from the next chunk's start state
 //     (S_next = Diag(gam)(S_0 + Kb^T Delta));
@@ -66,6 +68,7 @@ struct BwdWs {
   void* staged;                   // the forward's workspace
   float* fin;                     // scratch final state of the forward
   void* tp;                       // the two-pass forward's workspace, or null
+  float* wt;                      // W^T per chunk [chunks, H, dk, C], or null
   float *kt, *kb, *qt, *bkt;      // [tokens, H, dk]
   float *v32, *bv, *do32, *dd;    // [tokens, H, dv]
   float *tm, *pp;                 // [chunks, H, C, C]
@@ -95,6 +98,13 @@ ChunkArgs forward_args(const BwdArgs& a, float* fin) {
 bool tensor_state_pass(const ChunkArgs& f) {
   return fused_supported(f) && max_chunks(f) > 0;
 }
+// The reverse chain on the tensor cores (tf32) under the same condition, as
+// long as the rows of W^T stay within a tensor map's signed 32-bit
+// coordinates.
+bool tensor_chain(const ChunkArgs& f) {
+  return tensor_state_pass(f) &&
+         max_chunks(f) * f.H * f.dk < ((int64_t)1 << 31);
+}
 
 BwdWs carve_bwd(const BwdArgs& a, void* base, size_t* total) {
   const ChunkArgs& f = a.f;
@@ -114,6 +124,9 @@ BwdWs carve_bwd(const BwdArgs& a, void* base, size_t* total) {
   const ChunkArgs fa = forward_args(a, nullptr);
   w.staged = take(staged_workspace_bytes(fa));
   w.tp = tensor_state_pass(fa) ? take(twopass_workspace_bytes(fa)) : nullptr;
+  w.wt = tensor_chain(fa)
+             ? take(4 * (size_t)max_chunks(fa) * f.H * f.dk * f.chunk)
+             : nullptr;
   const size_t tdk = 4 * tokens * H * dk, tdv = 4 * tokens * H * dv;
   const size_t sq = 4 * nch * H * C * C, st = 4 * nch * H * dk * dv;
   w.kt = take(tdk); w.kb = take(tdk); w.qt = take(tdk); w.bkt = take(tdk);
@@ -145,12 +158,13 @@ __host__ __device__ constexpr int prep_region(int C, int dk, int dv) {
 // M)^-1 by recursive doubling, and the forward's W = Tm Diag(b) Kt, U =
 // Tm Diag(b) V and Kh = k exp(g_C - g) for the state pass.
 template <typename IO>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 2)  // two CTAs per SM
     prep_kernel(const IO* __restrict__ q, const IO* __restrict__ k,
                 const IO* __restrict__ v, const float* __restrict__ beta,
                 const IO* __restrict__ dout, const float* __restrict__ g,
                 BwdWs w, float* __restrict__ w_out, float* __restrict__ u_out,
-                float* __restrict__ kh_out, const int32_t* cu, const int32_t* chunk_off, int n_seqs,
+                float* __restrict__ kh_out, float* __restrict__ wt_out,
+                const int32_t* cu, const int32_t* chunk_off, int n_seqs,
                 int T, int H, int dk, int dv, int C) {
   const int cid = blockIdx.x;
   int seq, tok0, L;
@@ -328,6 +342,26 @@ __global__ void __launch_bounds__(kThreads)
         for (int b = 0; b < 8; ++b)
           if (b < nx) out[ro + tj + 16 * b] = acc[a][b];
       }
+    }
+    if (pass == 0 && wt_out) {
+      // W^T for the tensor-core chain, staged transposed in the dead A
+      // region (column index XOR the row's low bits against bank
+      // conflicts) and written out coalesced at the end
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 8; ++b)
+          if (a < nr && b < nx) {
+            const int r = ti + 16 * a, col = tj + 16 * b;
+            A[col * C + (r ^ (col & 31))] = acc[a][b];
+          }
+    }
+  }
+  if (wt_out) {  // W^T [dk][C] of this chunk from the A region, zero past L
+    const size_t tb = ((size_t)cid * H + h) * dk * C;
+    for (int idx = tid; idx < dk * C; idx += kThreads) {
+      const int col = idx / C, r = idx % C;
+      wt_out[tb + idx] = r < L ? A[col * C + (r ^ (col & 31))] : 0.f;
     }
   }
 }
@@ -875,8 +909,8 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
     prep_kernel<IO><<<grid, kThreads, smp, stream>>>(
         static_cast<const IO*>(f.q), static_cast<const IO*>(f.k),
         static_cast<const IO*>(f.v), f.beta, static_cast<const IO*>(a.d_out),
-        w.fv.g, w, w.fv.w, w.fv.d, w.fv.kh, cu, co, f.n_seqs, f.T, H, dk, dv,
-        C);
+        w.fv.g, w, w.fv.w, w.fv.d, w.fv.kh, w.wt, cu, co, f.n_seqs, f.T, H,
+        dk, dv, C);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   // the forward's serial state pass: chunk-start states, Delta over U, and
@@ -936,7 +970,30 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
     KDA_BMM(bmm(tok(w.pdo, dv), sq(w.pp, 1), tok(w.do32, dv), kDimDv, kDimL,
                 kMaskNone, 1.f, 0))
   }
-  {
+  if (w.wt) {  // on the tensor cores (tf32), one CTA per 64 d_v columns
+    RevChainArgs r{};
+    r.kb = w.kb;
+    r.wt = w.wt;
+    r.qdo = w.qdo;
+    r.pdo = w.pdo;
+    r.s = w.fv.s;
+    r.fin = w.fin;
+    r.gam = w.gam;
+    r.d_final = a.d_final_state;
+    r.gst = w.gst;
+    r.dd = w.dd;
+    r.dgam = w.dgam;
+    r.d_init = a.d_initial_state;
+    r.cu = cu;
+    r.chunk_off = co;
+    r.n_seqs = f.n_seqs;
+    r.T = f.T;
+    r.H = H;
+    r.dk = dk;
+    r.dv = dv;
+    r.n_chunks = nch;
+    if ((e = launch_rev_chain_tc(r, stream)) != cudaSuccess) return e;
+  } else {
     constexpr int tp = kChainTile + 1;
     const size_t smc = 4 * ((size_t)dk * tp + 2 * (size_t)C * (dk + 1) +
                             (size_t)C * tp + dk);

@@ -103,6 +103,7 @@ bool make_tile_map(CUtensorMap* m, const void* base, int d, int H, int tokens) {
 #include "kda_fused_ws_sm100.cuh"
 #include "kda_fused_pair_sm100.cuh"
 #include "kda_twopass_sm100.cuh"
+#include "kda_bwd_chain_tc.cuh"
 
 namespace kda {
 namespace {
@@ -224,6 +225,51 @@ cudaError_t launch_fused(const ChunkArgs& a, void* workspace,
   // factorisation as a cluster pair; d_v = 64: one CTA per head.
   if (a.dv == 2 * ws::kDvt) return pair::launch_fused_pair(a, order, stream);
   return ws::launch_fused_ws(a, order, stream);
+}
+
+namespace {
+template <int DK>
+cudaError_t run_rev_chain_tc(const RevChainArgs& a, cudaStream_t stream) {
+  using Lay = bwdtc::Layout<DK>;
+  const int tokens = a.cu ? a.T : a.n_seqs * a.T;
+  CUtensorMap tkb, twt;
+  if (!make_map(&tkb, a.kb, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, DK, a.H,
+                tokens, 32, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  {  // W^T: rows (chunk, head, channel) of 64 token columns, box 32 x DK
+    auto enc = encode_fn();
+    if (!enc) return cudaErrorInvalidValue;
+    cuuint64_t dims[2] = {64, (cuuint64_t)a.n_chunks * a.H * DK};
+    cuuint64_t strides[1] = {64 * 4};
+    cuuint32_t box[2] = {32, (cuuint32_t)DK};
+    cuuint32_t es[2] = {1, 1};
+    if (enc(&twt, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+            const_cast<float*>(a.wt), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  bwdtc::Params p{a.qdo, a.pdo, a.s, a.fin, a.gam, a.d_final, a.gst, a.dd,
+                  a.dgam, a.d_init, a.cu, a.chunk_off, a.n_seqs, a.T, a.H,
+                  a.dv};
+  const size_t smem = Lay::bytes + 1024;
+  cudaError_t e;
+  if ((e = cudaFuncSetAttribute(bwdtc::rev_chain_kernel<DK>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)smem)) != cudaSuccess)
+    return e;
+  const unsigned grid = (unsigned)a.n_seqs * a.H * (a.dv / bwdtc::kTile);
+  bwdtc::rev_chain_kernel<DK><<<grid, bwdtc::kThreads, smem, stream>>>(
+      tkb, twt, p);
+  return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_rev_chain_tc(const RevChainArgs& a, cudaStream_t stream) {
+  if (a.dk == 128) return run_rev_chain_tc<128>(a, stream);
+  if (a.dk == 64) return run_rev_chain_tc<64>(a, stream);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace kda

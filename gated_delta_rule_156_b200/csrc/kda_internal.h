@@ -103,10 +103,36 @@ int split_kernel_count(const ChunkArgs& a, const SplitGeom& g);
 cudaError_t launch_split(const ChunkArgs& a, const SplitGeom& g, void* workspace,
                          cudaStream_t stream);
 
+// The backward pass's reverse state-gradient chain on the tensor cores
+// (kda_bwd_chain_tc.cuh, tf32 products): 64-token chunks, d_k and d_v in
+// {64, 128}.  Inputs and outputs are the backward workspace's fp32 arrays;
+// wt is W transposed per chunk, [chunks, H, d_k, 64] with zero columns past
+// each chunk's last token.
+struct RevChainArgs {
+  const float* kb;       // Kb [tokens, H, dk]
+  const float* wt;       // W^T [chunks, H, dk, 64]
+  const float* qdo;      // Qt^T dO [chunks, H, dk, dv]
+  const float* pdo;      // P^T dO [tokens, H, dv]
+  const float* s;        // chunk-start states [chunks, H, dk, dv]
+  const float* fin;      // final states [n_seqs, H, dk, dv]
+  const float* gam;      // exp(g_C) [chunks, H, dk]
+  const float* d_final;  // or null
+  float* gst;            // G out [chunks, H, dk, dv]
+  float* dd;             // dDelta out [tokens, H, dv]
+  float* dgam;           // gam * d gam partials [chunks, H, dv / 32, dk]
+  float* d_init;         // or null
+  const int32_t* cu;
+  const int32_t* chunk_off;
+  int n_seqs, T, H, dk, dv;
+  int64_t n_chunks;
+};
+cudaError_t launch_rev_chain_tc(const RevChainArgs& a, cudaStream_t stream);
+
 // Chunkwise backward pass (kda_backward.cu): the gradients of
 // L = <d_out, out> + <d_final_state, final_state> with respect to q, k, v,
-// log(alpha), beta and the initial state, in fp32 arithmetic (the forward's
-// state pass with bf16 inputs in 64-token chunks runs on the tensor cores).
+// log(alpha), beta and the initial state, in fp32 arithmetic (with bf16
+// inputs in 64-token chunks the forward's state pass and the reverse chain
+// run on the tensor cores).
 struct BwdArgs {
   ChunkArgs f;                  // forward arguments; f.out, f.final_state unused
   const void* d_out;            // [tokens, H, dv], io dtype

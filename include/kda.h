@@ -410,8 +410,9 @@ KDA_API kda_status kda_device_status(cudaStream_t stream);
  * aligned (KDA_ERR_MISALIGNED otherwise).  No output may overlap an input or
  * another output (KDA_ERR_INVALID_ARG).  All arithmetic is fp32 except for
  * bf16 inputs with chunk 64, where the forward's state pass (chunk-start
- * states and Delta) is the two-pass tensor-core forward: bf16 operands, fp32
- * accumulators, within the bf16 tolerance of 1e-2 relative L2; the call
+ * states and Delta) is the two-pass tensor-core forward (bf16 operands, fp32
+ * accumulators) and the reverse state-gradient chain runs on the tensor
+ * cores in tf32, within the bf16 tolerance of 1e-2 relative L2; the call
  * re-runs the forward's chunk stages and allocates its fp32 workspace from
  * the stream-ordered pool (kda_chunk_bwd_plan reports its size).  Stream
  * ordered: returns after queueing the kernels.
