@@ -17,11 +17,15 @@
 //
 // One CTA of 256 threads per (sequence, head, 64-column d_v tile); thread c
 // owns TMEM lane c % 128 and 32 columns 32 (c / 128) .. + 31.  dS stays in
-// TMEM from the first step to the last.  Kb and W^T (written transposed by
-// the backward's prep kernel) arrive by TMA one chunk ahead into two
-// buffers; G and -dDelta are written by the epilogues straight into the
-// K-major B operands of the two MMAs.  tf32 operands need K-major layouts on
-// both sides, hence the transposed copy of W.
+// TMEM from the first step to the last.  Every tile moves by TMA, so global
+// traffic is coalesced although each thread owns one row: Kb and W^T
+// (written transposed by the backward's prep kernel) for the products,
+// Qt^T dO, the next start state and P^T dO for the epilogues, each fetched
+// for the next chunk as soon as its buffer is free; G and dDelta are written
+// in place of Qt^T dO and P^T dO and stored by TMA.  The epilogues also write
+// G and -dDelta straight into the K-major B operands of the two products.
+// tf32 operands need K-major layouts on both sides, hence the transposed
+// copy of W.
 namespace kda {
 namespace bwdtc {
 
@@ -69,14 +73,9 @@ __device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t adesc,
 }
 
 struct Params {
-  const float* qdo;      // Qt^T dO      [chunks, H, dk, dv]
-  const float* pdo;      // P^T dO       [tokens, H, dv]
-  const float* s;        // start states [chunks, H, dk, dv]
-  const float* fin;      // final states [n_seqs, H, dk, dv]
   const float* gam;      // exp(g_C)     [chunks, H, dk]
   const float* d_final;  // [n_seqs, H, dk, dv] or null (zero)
-  float* gst;            // G            [chunks, H, dk, dv]
-  float* dd;             // dDelta       [tokens, H, dv]
+  float* dd;             // dDelta [tokens, H, dv] (ragged chunks' rows)
   float* dgam;           // partials     [chunks, H, dv / 32, dk]
   float* d_init;         // [n_seqs, H, dk, dv] or null
   const int32_t* cu;
@@ -84,43 +83,88 @@ struct Params {
   int n_seqs, T, H, dv;
 };
 
+// The fp32 tensor maps (128-byte swizzle, boxes 32 columns wide): Kb and
+// P^T dO / dDelta over [tokens, H, d] (64-token boxes); W^T over
+// [chunks * H * dk, 64]; Qt^T dO, the start states, G over
+// [chunks * H * dk, dv] and the final states over [n_seqs * H * dk, dv]
+// (d_k-row boxes).
+struct Maps {
+  CUtensorMap kb, wt, qdo, s, fin, pdo, gst, dd;
+};
+
 template <int DK>
 struct Layout {
   // Kb: DK / 32 panels of 64 token rows x 128 B, plus one more panel of
   // padding, since the M = 128 product reads 128 rows from each panel start
   static constexpr uint32_t kb_bytes = (DK / 32 + 1) * 8192;
+  static constexpr uint32_t kb = 0;
   // W^T: two panels (tokens 0-31, 32-63) of 128 rows (d_k, padded) x 128 B
-  static constexpr uint32_t wt_bytes = 2 * 16384;
-  static constexpr uint32_t kb = 0;                       // two buffers
-  static constexpr uint32_t wt = kb + 2 * kb_bytes;       // two buffers
-  static constexpr uint32_t gop = wt + 2 * wt_bytes;      // G: 64 rows (j) x DK
+  static constexpr uint32_t wt = kb + kb_bytes;
+  static constexpr uint32_t gop = wt + 2 * 16384;        // G: 64 rows (j) x DK
   static constexpr uint32_t dop = gop + (DK / 32) * 8192; // -dDelta: 64 x 64
-  static constexpr uint32_t misc = dop + 2 * 8192;
+  // Qt^T dO (then G) and the next start state: two panels (32 columns
+  // each) of DK rows x 128 B; P^T dO (then dDelta): two of 64 rows
+  static constexpr uint32_t qt = dop + 2 * 8192;
+  static constexpr uint32_t st = qt + 2 * DK * 128;
+  static constexpr uint32_t pt = st + 2 * DK * 128;
+  static constexpr uint32_t misc = pt + 2 * 8192;
   static constexpr uint32_t bytes = misc + 256;
   static constexpr uint32_t kb_tx = (DK / 32) * 8192;
   static constexpr uint32_t wt_tx = 2 * DK * 128;
+  static constexpr uint32_t qt_tx = 2 * DK * 128;
+  static constexpr uint32_t pt_tx = 2 * 8192;
   static constexpr uint32_t t_ds = 0, t_dd = 64;  // TMEM columns
   static_assert(bytes + 1024 <= 232448, "shared memory");
 };
 
+__device__ __forceinline__ void tma_store_2d(const void* tmap, const void* src,
+                                             int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], "
+      "[%1];" ::"l"(reinterpret_cast<uint64_t>(tmap)),
+      "r"(sm100::smem_u32(src)), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void tma_store_3d(const void* tmap, const void* src,
+                                             int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, "
+      "%4}], [%1];" ::"l"(reinterpret_cast<uint64_t>(tmap)),
+      "r"(sm100::smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Until every bulk store committed so far has read its shared-memory source.
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 template <int DK>
 __global__ void __launch_bounds__(kThreads, 1)
-    rev_chain_kernel(const __grid_constant__ CUtensorMap tm_kb,
-                     const __grid_constant__ CUtensorMap tm_wt,
-                     const Params p) {
+    rev_chain_kernel(const __grid_constant__ Maps m, const Params p) {
   using namespace sm100;
   using Lay = Layout<DK>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* kb = sm + Lay::kb;
+  uint8_t* wt = sm + Lay::wt;
   uint8_t* gop = sm + Lay::gop;
   uint8_t* dop = sm + Lay::dop;
+  uint8_t* qt = sm + Lay::qt;
+  uint8_t* st = sm + Lay::st;
+  uint8_t* pt = sm + Lay::pt;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Lay::misc);
-  uint64_t* kb_full = bars;      // two
-  uint64_t* wt_full = bars + 2;  // two
-  uint64_t* bar_mma = bars + 4;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 5);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 6);
+  // one barrier per operand buffer, each completing once per step
+  enum { kKb, kWt, kQt, kSt, kPt, kNbuf };
+  uint64_t* bar_mma = bars + kNbuf;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNbuf + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + kNbuf + 2);
 
   const int c = threadIdx.x, warp = c >> 5;
   const int row = c & 127, half = c >> 7;
@@ -129,22 +173,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tile = blockIdx.x % n_tiles;
   const int h = (blockIdx.x / n_tiles) % p.H;
   const int seq = blockIdx.x / (n_tiles * p.H);
-  const int j0 = tile * kTile + 32 * half;  // this thread's first column
+  const int jt = tile * kTile;              // the tile's first column
+  const int j0 = jt + 32 * half;            // this thread's first column
   int start, end;
   seq_range(p.cu, seq, p.T, &start, &end);
   const int nch = (end - start + kC - 1) / kC;
   const int cid0 = p.cu ? p.chunk_off[seq] : seq * ((p.T + kC - 1) / kC);
   const bool owns_state = row < DK;
   const size_t sbase = ((size_t)seq * p.H + h) * DK * p.dv;
+  // rows of the d_k-row maps
+  auto crow = [&](int n) { return (int)(((size_t)(cid0 + n) * p.H + h) * DK); };
 
   if (c == 0) {
-    prefetch_tmap(&tm_kb);
-    prefetch_tmap(&tm_wt);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(kb_full + b, 1);
-      mbar_init(wt_full + b, 1);
-    }
-    mbar_init(bar_mma, 1);
+    prefetch_tmap(&m.kb);
+    prefetch_tmap(&m.wt);
+    prefetch_tmap(&m.qdo);
+    prefetch_tmap(&m.s);
+    prefetch_tmap(&m.pdo);
+    for (int i = 0; i < kNbuf + 1; ++i) mbar_init(bars + i, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -157,26 +203,55 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // step s handles chunk nch - 1 - s; its operands sit in buffer s & 1
-  auto issue = [&](int s) {
-    const int n = nch - 1 - s;
-    const int b = s & 1;
-    uint8_t* kb = sm + Lay::kb + b * Lay::kb_bytes;
-    uint8_t* wt = sm + Lay::wt + b * Lay::wt_bytes;
-    mbar_arrive_expect_tx(kb_full + b, Lay::kb_tx);
+  // Loads of step s (chunk nch - 1 - s), issued by thread 0 only; `issued`
+  // counts the loads of each buffer (one outstanding at most).
+  int issued[kNbuf] = {0, 0, 0, 0, 0};
+  auto load_kb = [&](int s) {
+    mbar_arrive_expect_tx(bars + kKb, Lay::kb_tx);
     for (int q = 0; q < DK / 32; ++q)
-      tma_load_3d(kb + q * 8192, &tm_kb, kb_full + b, 32 * q, h,
-                  start + n * kC);
-    mbar_arrive_expect_tx(wt_full + b, Lay::wt_tx);
-    const int wrow = (int)(((size_t)(cid0 + n) * p.H + h) * DK);
-    for (int q = 0; q < 2; ++q)
-      tma_load_2d(wt + q * 16384, &tm_wt, wt_full + b, 32 * q, wrow);
+      tma_load_3d(kb + q * 8192, &m.kb, bars + kKb, 32 * q, h,
+                  start + (nch - 1 - s) * kC);
+    ++issued[kKb];
   };
-  int issued = 0;
-  if (c == 0) {
-    for (int s = 0; s < 2 && s < nch; ++s) issue(s);
+  auto load_wt = [&](int s) {
+    mbar_arrive_expect_tx(bars + kWt, Lay::wt_tx);
+    for (int q = 0; q < 2; ++q)
+      tma_load_2d(wt + q * 16384, &m.wt, bars + kWt, 32 * q, crow(nch - 1 - s));
+    ++issued[kWt];
+  };
+  auto load_qt = [&](int s) {
+    mbar_arrive_expect_tx(bars + kQt, Lay::qt_tx);
+    for (int q = 0; q < 2; ++q)
+      tma_load_2d(qt + q * DK * 128, &m.qdo, bars + kQt, jt + 32 * q,
+                  crow(nch - 1 - s));
+    ++issued[kQt];
+  };
+  auto load_st = [&](int s) {  // the start state of chunk nch - s (or final)
+    mbar_arrive_expect_tx(bars + kSt, Lay::qt_tx);
+    for (int q = 0; q < 2; ++q) {
+      if (s == 0)
+        tma_load_2d(st + q * DK * 128, &m.fin, bars + kSt, jt + 32 * q,
+                    (int)(((size_t)seq * p.H + h) * DK));
+      else
+        tma_load_2d(st + q * DK * 128, &m.s, bars + kSt, jt + 32 * q,
+                    crow(nch - s));
+    }
+    ++issued[kSt];
+  };
+  auto load_pt = [&](int s) {
+    mbar_arrive_expect_tx(bars + kPt, Lay::pt_tx);
+    for (int q = 0; q < 2; ++q)
+      tma_load_3d(pt + q * 8192, &m.pdo, bars + kPt, jt + 32 * q, h,
+                  start + (nch - 1 - s) * kC);
+    ++issued[kPt];
+  };
+  if (c == 0 && nch > 0) {
+    load_st(0);
+    load_qt(0);
+    load_kb(0);
+    load_pt(0);
+    load_wt(0);
   }
-  issued = nch < 2 ? nch : 2;
 
   if (owns_state) {  // dS of the last chunk: the final-state gradient
     float v[32];
@@ -200,80 +275,86 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
 
-  // Per-thread operands of one step's epilogues, loaded a phase ahead of
-  // their use: Qt^T dO, the next start state and gam for G (step s + 1's
-  // are fetched during step s's second product), P^T dO for dDelta (fetched
-  // while the first product runs).
-  float qd[32], sn[32], gmv = 0.f;
-  auto load_state_operands = [&](int s_) {
-    const int n = nch - 1 - s_, cid = cid0 + n;
-    const size_t cbase = ((size_t)cid * p.H + h) * DK * p.dv;
-    const float4* q4 = reinterpret_cast<const float4*>(
-        p.qdo + cbase + (size_t)row * p.dv + j0);
-    const float* snx = n + 1 < nch ? p.s + cbase + (size_t)p.H * DK * p.dv
-                                   : p.fin + sbase;
-    const float4* s4 =
-        reinterpret_cast<const float4*>(snx + (size_t)row * p.dv + j0);
+  // this thread's 128-byte row inside a swizzled operand panel
+  auto ld_row = [](const uint8_t* panel, int r, float* v) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float4 x = q4[i], y = s4[i];
-      qd[4 * i] = x.x; qd[4 * i + 1] = x.y; qd[4 * i + 2] = x.z;
-      qd[4 * i + 3] = x.w;
-      sn[4 * i] = y.x; sn[4 * i + 1] = y.y; sn[4 * i + 2] = y.z;
-      sn[4 * i + 3] = y.w;
+    for (int k = 0; k < 8; ++k) {
+      const float4 x = *reinterpret_cast<const float4*>(
+          panel + r * 128 + ((k ^ (r & 7)) << 4));
+      v[4 * k] = x.x; v[4 * k + 1] = x.y; v[4 * k + 2] = x.z;
+      v[4 * k + 3] = x.w;
     }
-    gmv = p.gam[((size_t)cid * p.H + h) * DK + row];
   };
-  if (owns_state && nch > 0) load_state_operands(0);
+  auto st_row = [](uint8_t* panel, int r, const float* v) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      *reinterpret_cast<float4*>(panel + r * 128 + ((k ^ (r & 7)) << 4)) =
+          make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+  };
 
+  float gmv = (owns_state && nch > 0)
+                  ? p.gam[((size_t)(cid0 + nch - 1) * p.H + h) * DK + row]
+                  : 0.f;
   uint32_t ph_mma = 0;
   bool failed = false;
   int s = 0;
   for (; s < nch; ++s) {
-    const int n = nch - 1 - s, b = s & 1;
+    const int n = nch - 1 - s;
     const int cid = cid0 + n, tok0 = start + n * kC;
     const int L = min(kC, end - tok0);
-    const size_t cbase = ((size_t)cid * p.H + h) * DK * p.dv;
+    const uint32_t par = (uint32_t)s & 1u;
+    bool ok = true;
 
     // ---- G = Diag(gam) dS, gam * d gam; TMEM dS <- G + Qt^T dO
     if (owns_state) {
-      float v[32];
-      tmem_ld32(tmem + lane_base + Lay::t_ds + 32 * half, v);
-      float part = 0.f;
+      ok = wait_or_abort<false>(bars + kSt, par, abort_flag) &&
+           wait_or_abort<false>(bars + kQt, par, abort_flag);
+      if (ok) {
+        float v[32], x[32];
+        tmem_ld32(tmem + lane_base + Lay::t_ds + 32 * half, v);
+        ld_row(st + half * DK * 128, row, x);
+        float part = 0.f;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) part += sn[i] * v[i];
-      p.dgam[(((size_t)cid * p.H + h) * (p.dv / 32) + j0 / 32) * DK + row] =
-          part;
+        for (int i = 0; i < 32; ++i) part += x[i] * v[i];
+        p.dgam[(((size_t)cid * p.H + h) * (p.dv / 32) + j0 / 32) * DK + row] =
+            part;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] *= gmv;
-      float4* g4 = reinterpret_cast<float4*>(p.gst + cbase +
-                                             (size_t)row * p.dv + j0);
+        for (int i = 0; i < 32; ++i) v[i] *= gmv;
+        // B operand of product 1: element (k = row, n = column), K-major
+        // panels of 32 rows (d_k) each
+        uint8_t* panel = gop + (row >> 5) * 8192;
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        g4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-      // B operand of product 1: element (k = row, n = column), K-major
-      // panels of 32 rows (d_k) each
-      uint8_t* panel = gop + (row >> 5) * 8192;
+        for (int i = 0; i < 32; ++i)
+          *reinterpret_cast<float*>(panel + swz32(32 * half + i, row & 31)) =
+              v[i];
+        uint8_t* qp = qt + half * DK * 128;
+        ld_row(qp, row, x);
+        st_row(qp, row, v);  // G, stored by TMA below
 #pragma unroll
-      for (int i = 0; i < 32; ++i)
-        *reinterpret_cast<float*>(panel + swz32(32 * half + i, row & 31)) = v[i];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] += qd[i];
-      tmem_st32(tmem + lane_base + Lay::t_ds + 32 * half, v);
-      tmem_wait_st();
+        for (int i = 0; i < 32; ++i) v[i] += x[i];
+        tmem_st32(tmem + lane_base + Lay::t_ds + 32 * half, v);
+        tmem_wait_st();
+      } else {
+        *abort_flag = 1;
+      }
+      if (n > 0) gmv = p.gam[((size_t)(cid - 1) * p.H + h) * DK + row];
     }
     fence_proxy_async();
     tc_fence_before();
-    __syncthreads();
+    if (named_sync_or(kBarAll, kThreads, !ok)) {
+      failed = true;
+      break;
+    }
 
-    // ---- product 1: D = Kb G (rows 0-63 meaningful)
-    bool ok = true;
+    // ---- product 1: D = Kb G (rows 0-63 meaningful); G out; next loads
     if (c == 0) {
       tc_fence_after();
-      ok = wait_or_abort<false>(kb_full + b, (uint32_t)(s >> 1) & 1u,
-                                abort_flag);
+      for (int q = 0; q < 2; ++q)
+        tma_store_2d(&m.gst, qt + q * DK * 128, jt + 32 * q, crow(n));
+      bulk_commit();
+      if (s + 1 < nch) load_st(s + 1);
+      ok = wait_or_abort<false>(bars + kKb, par, abort_flag);
       if (ok) {
-        const uint8_t* kb = sm + Lay::kb + b * Lay::kb_bytes;
         constexpr uint32_t id = idesc_tf32(128, kTile);
 #pragma unroll
         for (int ks = 0; ks < DK / 8; ++ks)
@@ -284,20 +365,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                               16, 1024),
                    id, ks > 0);
         mma_commit(bar_mma);
+        bulk_wait_read();  // G has left the Qt^T dO buffer
+        if (s + 1 < nch) load_qt(s + 1);
       } else {
         *abort_flag = 1;
-      }
-    }
-    float pd[32];
-    const bool in = row < L;
-    if (row < kC) {
-      const float4* p4 = reinterpret_cast<const float4*>(
-          p.pdo + ((size_t)(tok0 + (in ? row : 0)) * p.H + h) * p.dv + j0);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float4 x = in ? p4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-        pd[4 * i] = x.x; pd[4 * i + 1] = x.y; pd[4 * i + 2] = x.z;
-        pd[4 * i + 3] = x.w;
       }
     }
     ok = ok && wait_or_abort<false>(bar_mma, ph_mma, abort_flag);
@@ -307,37 +378,56 @@ __global__ void __launch_bounds__(kThreads, 1)
       break;
     }
     tc_fence_after();
+    if (c == 0 && s + 1 < nch) load_kb(s + 1);
 
     // ---- dDelta = Kb G + P^T dO (token rows 0-63; zero past the chunk)
     if (row < kC) {
-      float d[32];
-      tmem_ld32(tmem + lane_base + Lay::t_dd + 32 * half, d);
+      ok = wait_or_abort<false>(bars + kPt, par, abort_flag);
+      if (ok) {
+        float d[32], x[32];
+        const bool in = row < L;
+        uint8_t* pp = pt + half * 8192;
+        ld_row(pp, row, x);
+        tmem_ld32(tmem + lane_base + Lay::t_dd + 32 * half, d);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) d[i] = in ? d[i] + pd[i] : 0.f;
-      if (in) {
-        float4* d4 = reinterpret_cast<float4*>(
-            p.dd + ((size_t)(tok0 + row) * p.H + h) * p.dv + j0);
+        for (int i = 0; i < 32; ++i) d[i] = in ? d[i] + x[i] : 0.f;
+        if (L < kC && in) {  // a ragged chunk: the rows past it belong to
+                             // the next sequence, so no box store
+          float4* d4 = reinterpret_cast<float4*>(
+              p.dd + ((size_t)(tok0 + row) * p.H + h) * p.dv + j0);
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          d4[i] = make_float4(d[4 * i], d[4 * i + 1], d[4 * i + 2], d[4 * i + 3]);
+          for (int i = 0; i < 8; ++i)
+            d4[i] =
+                make_float4(d[4 * i], d[4 * i + 1], d[4 * i + 2], d[4 * i + 3]);
+        }
+        st_row(pp, row, d);
+        // B operand of product 2, negated: element (k = token, n = column)
+        uint8_t* panel = dop + (row >> 5) * 8192;
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          *reinterpret_cast<float*>(panel + swz32(32 * half + i, row & 31)) =
+              -d[i];
+      } else {
+        *abort_flag = 1;
       }
-      // B operand of product 2, negated: element (k = token, n = column)
-      uint8_t* panel = dop + (row >> 5) * 8192;
-#pragma unroll
-      for (int i = 0; i < 32; ++i)
-        *reinterpret_cast<float*>(panel + swz32(32 * half + i, row & 31)) = -d[i];
     }
     fence_proxy_async();
     tc_fence_before();
-    __syncthreads();
+    if (named_sync_or(kBarAll, kThreads, !ok)) {
+      failed = true;
+      break;
+    }
 
-    // ---- product 2: dS += W^T (-dDelta)
+    // ---- product 2: dS += W^T (-dDelta); dDelta out; next loads
     if (c == 0) {
       tc_fence_after();
-      ok = wait_or_abort<false>(wt_full + b, (uint32_t)(s >> 1) & 1u,
-                                abort_flag);
+      if (L == kC) {
+        for (int q = 0; q < 2; ++q)
+          tma_store_3d(&m.dd, pt + q * 8192, jt + 32 * q, h, tok0);
+        bulk_commit();
+      }
+      ok = wait_or_abort<false>(bars + kWt, par, abort_flag);
       if (ok) {
-        const uint8_t* wt = sm + Lay::wt + b * Lay::wt_bytes;
         constexpr uint32_t id = idesc_tf32(128, kTile);
 #pragma unroll
         for (int ks = 0; ks < kC / 8; ++ks)
@@ -348,11 +438,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                               16, 1024),
                    id, 1u);
         mma_commit(bar_mma);
+        bulk_wait_read();  // dDelta has left the P^T dO buffer
+        if (s + 1 < nch) load_pt(s + 1);
       } else {
         *abort_flag = 1;
       }
     }
-    if (owns_state && s + 1 < nch) load_state_operands(s + 1);
     ok = ok && wait_or_abort<false>(bar_mma, ph_mma, abort_flag);
     ph_mma ^= 1;
     if (named_sync_or(kBarAll, kThreads, !ok)) {
@@ -360,19 +451,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       break;
     }
     tc_fence_after();
-    // both buffers b are free again: the operands of step s + 2
-    if (s + 2 < nch) {
-      if (c == 0) issue(s + 2);
-      issued = s + 3;
-    }
+    if (c == 0 && s + 1 < nch) load_wt(s + 1);
   }
   if (failed) {
     if (c == 0) {
       atomicExch(&g_fused_timeout, 1);
-      for (int m = s; m < issued; ++m) {  // copies still in flight
-        mbar_wait(kb_full + (m & 1), (uint32_t)(m >> 1) & 1u, 100000000ull);
-        mbar_wait(wt_full + (m & 1), (uint32_t)(m >> 1) & 1u, 100000000ull);
-      }
+#pragma unroll
+      for (int b = 0; b < kNbuf; ++b)  // the copy still in flight, if any
+        if (issued[b] > 0)
+          mbar_wait(bars + b, (uint32_t)(issued[b] - 1) & 1u, 100000000ull);
     }
   } else if (owns_state && p.d_init) {
     float v[32];
@@ -383,6 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 8; ++i)
       dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
   }
+  if (c == 0) bulk_wait_all();
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 128);

@@ -228,31 +228,41 @@ cudaError_t launch_fused(const ChunkArgs& a, void* workspace,
 }
 
 namespace {
+// 2-D fp32 map over `rows` rows of `cols` floats, box of 32 columns x
+// `box_rows` rows, 128-byte swizzle.
+bool make_rows_map(CUtensorMap* m, const float* base, int64_t rows, int cols,
+                   int box_rows) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * 4};
+  cuuint32_t box[2] = {32, (cuuint32_t)box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base),
+             dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int DK>
 cudaError_t run_rev_chain_tc(const RevChainArgs& a, cudaStream_t stream) {
   using Lay = bwdtc::Layout<DK>;
   const int tokens = a.cu ? a.T : a.n_seqs * a.T;
-  CUtensorMap tkb, twt;
-  if (!make_map(&tkb, a.kb, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, DK, a.H,
-                tokens, 32, CU_TENSOR_MAP_SWIZZLE_128B))
+  const int64_t crows = a.n_chunks * a.H * DK;
+  const auto F32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  const auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
+  bwdtc::Maps m;
+  if (!make_map(&m.kb, a.kb, F32, 4, DK, a.H, tokens, 32, SW) ||
+      !make_map(&m.pdo, a.pdo, F32, 4, a.dv, a.H, tokens, 32, SW) ||
+      !make_map(&m.dd, a.dd, F32, 4, a.dv, a.H, tokens, 32, SW) ||
+      !make_rows_map(&m.wt, a.wt, crows, 64, DK) ||
+      !make_rows_map(&m.qdo, a.qdo, crows, a.dv, DK) ||
+      !make_rows_map(&m.s, a.s, crows, a.dv, DK) ||
+      !make_rows_map(&m.gst, a.gst, crows, a.dv, DK) ||
+      !make_rows_map(&m.fin, a.fin, (int64_t)a.n_seqs * a.H * DK, a.dv, DK))
     return cudaErrorInvalidValue;
-  {  // W^T: rows (chunk, head, channel) of 64 token columns, box 32 x DK
-    auto enc = encode_fn();
-    if (!enc) return cudaErrorInvalidValue;
-    cuuint64_t dims[2] = {64, (cuuint64_t)a.n_chunks * a.H * DK};
-    cuuint64_t strides[1] = {64 * 4};
-    cuuint32_t box[2] = {32, (cuuint32_t)DK};
-    cuuint32_t es[2] = {1, 1};
-    if (enc(&twt, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
-            const_cast<float*>(a.wt), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
-  }
-  bwdtc::Params p{a.qdo, a.pdo, a.s, a.fin, a.gam, a.d_final, a.gst, a.dd,
-                  a.dgam, a.d_init, a.cu, a.chunk_off, a.n_seqs, a.T, a.H,
-                  a.dv};
+  bwdtc::Params p{a.gam, a.d_final, a.dd, a.dgam, a.d_init, a.cu,
+                  a.chunk_off, a.n_seqs, a.T, a.H, a.dv};
   const size_t smem = Lay::bytes + 1024;
   cudaError_t e;
   if ((e = cudaFuncSetAttribute(bwdtc::rev_chain_kernel<DK>,
@@ -260,8 +270,7 @@ cudaError_t run_rev_chain_tc(const RevChainArgs& a, cudaStream_t stream) {
                                 (int)smem)) != cudaSuccess)
     return e;
   const unsigned grid = (unsigned)a.n_seqs * a.H * (a.dv / bwdtc::kTile);
-  bwdtc::rev_chain_kernel<DK><<<grid, bwdtc::kThreads, smem, stream>>>(
-      tkb, twt, p);
+  bwdtc::rev_chain_kernel<DK><<<grid, bwdtc::kThreads, smem, stream>>>(m, p);
   return cudaGetLastError();
 }
 }  // namespace
