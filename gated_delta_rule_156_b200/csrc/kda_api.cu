@@ -606,14 +606,15 @@ const char* kda_status_string(kda_status status) {
 
 kda_status kda_device_status(cudaStream_t stream) {
   int flag = 0, split_flag = 0, range_fused = 0, range_staged = 0,
-      range_bwd = 0;
+      range_bwd = 0, bwd_flag = 0;
   cudaError_t e = kda::fused_take_timeout(stream, &flag);
   if (e == cudaSuccess) e = kda::split_take_timeout(stream, &split_flag);
   if (e == cudaSuccess) e = kda::fused_take_range(stream, &range_fused);
   if (e == cudaSuccess) e = kda::staged_take_range(stream, &range_staged);
   if (e == cudaSuccess) e = kda::bwd_take_range(stream, &range_bwd);
+  if (e == cudaSuccess) e = kda::bwd_take_timeout(stream, &bwd_flag);
   if (e != cudaSuccess) return cuda_fail(e);
-  if (flag || split_flag) return KDA_ERR_TIMEOUT;
+  if (flag || split_flag || bwd_flag) return KDA_ERR_TIMEOUT;
   return range_fused || range_staged || range_bwd ? KDA_ERR_RANGE : KDA_OK;
 }
 

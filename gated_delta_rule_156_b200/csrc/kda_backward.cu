@@ -48,6 +48,7 @@
 #include "kda_common.cuh"
 #include "kda_internal.h"
 #include "kda_inverse.cuh"
+#include "sm100_ptx.cuh"
 
 namespace kda {
 
@@ -55,6 +56,8 @@ namespace kda {
 // the host).  The backward keeps the chunk-start factorisation (k e^g and
 // k e^-g), which stays inside the fp32 range while |g_C| <= kBwdDecayMax.
 __device__ int g_bwd_range = 0;
+// Set when a bounded wait of the backward's tensor-core products gave up.
+__device__ int g_bwd_timeout = 0;
 constexpr float kBwdDecayMax = 80.f;
 
 namespace {
@@ -154,9 +157,10 @@ __host__ __device__ constexpr int prep_region(int C, int dk, int dv) {
 
 // Per (chunk, head): Kt, Kb, Qt, b Kt and fp32 copies of V, b V, dO; gam;
 // M = Kt Kb^T (strictly lower, kept only on chip), P = lower_incl(Qt Kb^T),
-// Tm = (I + Diag(b)
-// M)^-1 by recursive doubling, and the forward's W = Tm Diag(b) Kt, U =
-// Tm Diag(b) V and Kh = k exp(g_C - g) for the state pass.
+// Tm = (I + Diag(b) M)^-1 by recursive doubling, and the forward's
+// W = Tm Diag(b) Kt; for the SIMT state pass also U = Tm Diag(b) V and
+// Kh = k exp(g_C - g) (u_out, kh_out null otherwise), and for the
+// tensor-core chain W^T per chunk (wt_out, else null).
 template <typename IO>
 __global__ void __launch_bounds__(kThreads, 2)  // two CTAs per SM
     prep_kernel(const IO* __restrict__ q, const IO* __restrict__ k,
@@ -207,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 2)  // two CTAs per SM
       w.kb[gi] = kb;
       w.qt[gi] = qt;
       w.bkt[gi] = bs[r] * kt;
-      kh_out[gi] = kv * __expf(gl[c] - gv);
+      if (kh_out) kh_out[gi] = kv * __expf(gl[c] - gv);
     }
     Kt[r * ldk + c] = kt;
     Kb[r * ldk + c] = kb;
@@ -302,7 +306,8 @@ __global__ void __launch_bounds__(kThreads, 2)  // two CTAs per SM
   __syncthreads();
   // W = (Tm Diag(b)) Kt, then U = (Tm Diag(b)) V with V over Kt, each over
   // i = 0 .. C - 1 (the terms above the diagonal are exact zeros)
-  for (int pass = 0; pass < 2; ++pass) {
+  // (U only for the SIMT state pass; the two-pass forward forms its own)
+  for (int pass = 0; pass < (u_out ? 2 : 1); ++pass) {
     const float* X = pass == 0 ? Kt : V;
     const int ldx = pass == 0 ? ldk : dv;
     const int nx = (pass == 0 ? dk : dv) / 16, cols = pass == 0 ? dk : dv;
@@ -851,6 +856,210 @@ cudaError_t set_smem(K kernel, size_t bytes) {
 
 // Launch one batched product with the thread blocking its padded shape asks
 // for: RM = md / 16 rows and RN = nd / 16 columns per thread.
+// op(A) (rows i, contraction t) as a K-major tf32 operand: 128-byte-swizzled
+// panels of 32 t each, `rows` x 128 B per panel.  Source A[i][t]: each thread
+// moves one 16-byte vector of a source row.
+__device__ __forceinline__ void stage_km_direct(const Src& s, int rows, int cols,
+                                                uint8_t* dst, int panel,
+                                                int tid) {
+  const int cv = cols >> 2, units = rows * cv;
+  for (int base = 0; base < units; base += 4 * kThreads) {
+    float4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int idx = base + u * kThreads + tid;
+      v[u] = idx < units ? ld_src4(s, idx / cv, (idx % cv) * 4)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int idx = base + u * kThreads + tid;
+      if (idx < units) {
+        const int r = idx / cv, c = (idx % cv) * 4;
+        *reinterpret_cast<float4*>(dst + (c >> 5) * panel +
+                                   sm100::swz32(r, c & 31)) = v[u];
+      }
+    }
+  }
+}
+// The same operand from a source stored the other way round, S[t][i]
+// (source rows = t): consecutive threads take consecutive source rows, each
+// reading 32 contiguous bytes, so the scalar shared stores of a warp fill one
+// 128-byte panel row.
+__device__ __forceinline__ void stage_km_transposed(const Src& s, int rows,
+                                                    int cols, uint8_t* dst,
+                                                    int panel, int tid) {
+  const int units = rows * (cols >> 3);
+  for (int base = 0; base < units; base += 2 * kThreads) {
+    float4 v[2][2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int idx = base + u * kThreads + tid;
+      const int r = idx % rows, c = (idx / rows) * 8;
+      const bool in = idx < units;
+      v[u][0] = in ? ld_src4(s, r, c) : make_float4(0.f, 0.f, 0.f, 0.f);
+      v[u][1] = in ? ld_src4(s, r, c + 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int idx = base + u * kThreads + tid;
+      if (idx < units) {
+        const int r = idx % rows, c = (idx / rows) * 8;
+        uint8_t* d = dst + (r >> 5) * panel;
+        const float x[8] = {v[u][0].x, v[u][0].y, v[u][0].z, v[u][0].w,
+                            v[u][1].x, v[u][1].y, v[u][1].z, v[u][1].w};
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          *reinterpret_cast<float*>(d + sm100::swz32(c + q, r & 31)) = x[q];
+      }
+    }
+  }
+}
+
+// Tensor-core form of bmm_kernel for bf16 inputs in 64-token chunks (every
+// dimension 64 or 128): per (chunk, head), each term's op(A) and op(B) are
+// staged as K-major tf32 operands and multiplied by tcgen05 kind::tf32 into
+// one TMEM accumulator of MD x ND; the epilogue applies alpha, the mask and
+// the accumulation as bmm_kernel does.  MD = 64 uses the M = 64 shape, whose
+// rows 16 q .. 16 q + 15 land in TMEM lanes 32 q .. 32 q + 15.
+template <int MD, int ND>
+__global__ void __launch_bounds__(kThreads, MD == 64 ? 2 : 1)
+    bmm_tc_kernel(BmmOp op, const int32_t* cu, const int32_t* chunk_off,
+                  int n_seqs, int T, int H, int dk, int dv, int C) {
+  using namespace sm100;
+  const int cid = blockIdx.x;
+  int seq, tok0, L;
+  if (!locate_chunk(cid, cu, chunk_off, n_seqs, T, C, &seq, &tok0, &L)) return;
+  const int h = blockIdx.y, tid = threadIdx.x, warp = tid >> 5;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  constexpr int kPanA = MD * 128, kPanB = ND * 128;
+  uint8_t* As = sm;                 // up to four panels
+  uint8_t* Bs = sm + 4 * kPanA;     // up to four panels
+  uint64_t* bar = reinterpret_cast<uint64_t*>(Bs + 4 * kPanB);
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 1);
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tslot, ND);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+  bool ok = true;
+  for (int term = 0; term < op.nterms && ok; ++term) {
+    const BmmTerm tm = term == 0 ? op.term[0]
+                       : term == 1 ? op.term[1] : op.term[2];
+    const int kd = tm.kd;
+    const Src sa = src_of(tm.a, cid, h, tok0, L, H, C, dk);
+    const Src sb = src_of(tm.b, cid, h, tok0, L, H, C, dk);
+    if (tm.a.trans) stage_km_transposed(sa, kd, MD, As, kPanA, tid);  // A[t][i]
+    else stage_km_direct(sa, MD, kd, As, kPanA, tid);                 // A[i][t]
+    if (tm.b.trans) stage_km_direct(sb, ND, kd, Bs, kPanB, tid);      // B[j][t]
+    else stage_km_transposed(sb, kd, ND, Bs, kPanB, tid);             // B[t][j]
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      constexpr uint32_t id = idesc_tf32(MD, ND);
+      for (int ks = 0; ks < kd / 8; ++ks)
+        mma_tf32(tmem,
+                 desc_sw128(smem_u32(As) + (ks >> 2) * kPanA + (ks & 3) * 32,
+                            16, 1024),
+                 desc_sw128(smem_u32(Bs) + (ks >> 2) * kPanB + (ks & 3) * 32,
+                            16, 1024),
+                 id, (term > 0 || ks > 0) ? 1u : 0u);
+      mma_commit(bar);
+    }
+    // the operands are read once the products complete: the next term may
+    // then restage them
+    ok = __syncthreads_and(mbar_wait(bar, (uint32_t)term & 1u, 2000000000ull));
+    tc_fence_after();
+  }
+  if (!ok) {
+    if (tid == 0) atomicExch(&g_bwd_timeout, 1);
+  } else {
+    const int m = dim_of(op.m, L, dk, dv), n = dim_of(op.n, L, dk, dv);
+    const Src so = src_of(op.out, cid, h, tok0, L, H, C, dk);
+    const int lane = tid & 31, q = warp & 3, chalf = tid >> 7;
+    const int i = MD == 128 ? 32 * q + lane : (lane < 16 ? 16 * q + lane : MD);
+    const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16);
+#pragma unroll
+    for (int cc = 0; cc < ND / 64; ++cc) {
+      const int j0 = chalf * (ND / 2) + 32 * cc;
+      float x[32];
+      tmem_ld32(taddr + j0, x);
+      if (i < m && j0 < n) {
+#pragma unroll
+        for (int b = 0; b < 32; ++b) {
+          const int j = j0 + b;
+          x[b] *= op.alpha;
+          if ((op.mask == kMaskLowerIncl && j > i) ||
+              (op.mask == kMaskStrictLower && j >= i))
+            x[b] = 0.f;
+        }
+        float* o = so.p + (size_t)i * so.stride + j0;
+        if (j0 + 32 <= n) {
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            float4* o4 = reinterpret_cast<float4*>(o + 4 * v);
+            float4 y = make_float4(x[4 * v], x[4 * v + 1], x[4 * v + 2],
+                                   x[4 * v + 3]);
+            if (op.accumulate) {
+              const float4 z = *o4;
+              y.x += z.x;
+              y.y += z.y;
+              y.z += z.z;
+              y.w += z.w;
+            }
+            *o4 = y;
+          }
+        } else {
+#pragma unroll
+          for (int b = 0; b < 32; ++b)
+            if (j0 + b < n) o[b] = op.accumulate ? o[b] + x[b] : x[b];
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, ND);
+}
+
+template <int MD, int ND>
+cudaError_t launch_bmm_tc_t(const BmmOp& op, dim3 grid, cudaStream_t stream,
+                            const int32_t* cu, const int32_t* co, int n_seqs,
+                            int T, int H, int dk, int dv, int C) {
+  const size_t smem = 4 * (size_t)(MD + ND) * 128 + 1024 + 64;
+  cudaError_t e = set_smem(bmm_tc_kernel<MD, ND>, smem);
+  if (e != cudaSuccess) return e;
+  bmm_tc_kernel<MD, ND><<<grid, kThreads, smem, stream>>>(op, cu, co, n_seqs,
+                                                          T, H, dk, dv, C);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bmm_tc(const BmmOp& op, int C, dim3 grid,
+                          cudaStream_t stream, const int32_t* cu,
+                          const int32_t* co, int n_seqs, int T, int H, int dk,
+                          int dv) {
+  if (op.md == 64 && op.nd == 64)
+    return launch_bmm_tc_t<64, 64>(op, grid, stream, cu, co, n_seqs, T, H, dk, dv, C);
+  if (op.md == 64 && op.nd == 128)
+    return launch_bmm_tc_t<64, 128>(op, grid, stream, cu, co, n_seqs, T, H, dk, dv, C);
+  if (op.md == 128 && op.nd == 64)
+    return launch_bmm_tc_t<128, 64>(op, grid, stream, cu, co, n_seqs, T, H, dk, dv, C);
+  if (op.md == 128 && op.nd == 128)
+    return launch_bmm_tc_t<128, 128>(op, grid, stream, cu, co, n_seqs, T, H, dk, dv, C);
+  return cudaErrorInvalidValue;
+}
+
 template <int RM, int RN>
 cudaError_t launch_bmm_t(const BmmOp& op, size_t smem, dim3 grid,
                          cudaStream_t stream, const int32_t* cu,
@@ -909,8 +1118,9 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
     prep_kernel<IO><<<grid, kThreads, smp, stream>>>(
         static_cast<const IO*>(f.q), static_cast<const IO*>(f.k),
         static_cast<const IO*>(f.v), f.beta, static_cast<const IO*>(a.d_out),
-        w.fv.g, w, w.fv.w, w.fv.d, w.fv.kh, w.wt, cu, co, f.n_seqs, f.T, H,
-        dk, dv, C);
+        w.fv.g, w, w.fv.w, tensor_state_pass(f) ? nullptr : w.fv.d,
+        tensor_state_pass(f) ? nullptr : w.fv.kh, w.wt, cu, co, f.n_seqs, f.T,
+        H, dk, dv, C);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   // the forward's serial state pass: chunk-start states, Delta over U, and
@@ -946,6 +1156,9 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
     op.alpha = alpha;
     op.accumulate = accumulate;
     const int kd = max(t0.kd, max(nterms > 1 ? t1.kd : 0, nterms > 2 ? t2.kd : 0));
+    if (w.wt)  // bf16 inputs in 64-token chunks: on the tensor cores (tf32)
+      return launch_bmm_tc(op, C, grid, stream, cu, co, f.n_seqs, f.T, H, dk,
+                           dv);
     const size_t smem = 4 * (size_t)kd * ((op.md + 4) + (op.nd + 4));
     return launch_bmm(op, C, smem, grid, stream, cu, co, f.n_seqs, f.T, H, dk,
                       dv);
@@ -1058,6 +1271,16 @@ cudaError_t bwd_take_range(cudaStream_t stream, int* flag) {
     return e;
   const int zero = 0;
   return cudaMemcpyToSymbol(g_bwd_range, &zero, sizeof(int));
+}
+
+cudaError_t bwd_take_timeout(cudaStream_t stream, int* flag) {
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return e;
+  if ((e = cudaMemcpyFromSymbol(flag, g_bwd_timeout, sizeof(int))) !=
+      cudaSuccess)
+    return e;
+  const int zero = 0;
+  return cudaMemcpyToSymbol(g_bwd_timeout, &zero, sizeof(int));
 }
 
 size_t bwd_workspace_bytes(const BwdArgs& a) {

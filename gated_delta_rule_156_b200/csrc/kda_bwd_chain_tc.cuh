@@ -29,6 +29,9 @@
 namespace kda {
 namespace bwdtc {
 
+using sm100::idesc_tf32;
+using sm100::mma_tf32;
+using sm100::swz32;
 using ws::named_sync_or;
 using ws::tmem_st32;
 using ws::tmem_wait_st;
@@ -39,17 +42,6 @@ constexpr int kTile = 64;     // d_v columns per CTA
 constexpr int kThreads = 256;
 constexpr int kBarAll = 1;
 
-__host__ __device__ constexpr uint32_t idesc_tf32(int M, int N) {
-  return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(N >> 3) << 17) |
-         ((uint32_t)(M >> 4) << 24);
-}
-
-// fp32 element (row, c) of a 128-byte-swizzled panel whose rows hold 32 fp32
-// (K-major: rows along M or N, 32 consecutive k per row).
-__device__ __forceinline__ uint32_t swz32(int row, int c) {
-  return (uint32_t)(row * 128 + (((c >> 2) ^ (row & 7)) << 4) + ((c & 3) << 2));
-}
-
 __device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap,
                                             uint64_t* bar, int c0, int c1) {
   asm volatile(
@@ -57,18 +49,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap,
       "bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(sm100::smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1),
       "r"(sm100::smem_u32(bar))
-      : "memory");
-}
-
-__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t adesc,
-                                         uint64_t bdesc, uint32_t idesc,
-                                         uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(
-          d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 

@@ -165,6 +165,7 @@ cudaError_t split_take_timeout(cudaStream_t stream, int* flag);
 cudaError_t fused_take_range(cudaStream_t stream, int* flag);
 cudaError_t staged_take_range(cudaStream_t stream, int* flag);
 cudaError_t bwd_take_range(cudaStream_t stream, int* flag);
+cudaError_t bwd_take_timeout(cudaStream_t stream, int* flag);
 // Diagnostic: one CTA whose bounded wait runs out after limit_us.
 cudaError_t launch_timeout_probe(int limit_us, cudaStream_t stream);
 cudaError_t launch_fused(const ChunkArgs& a, void* workspace,

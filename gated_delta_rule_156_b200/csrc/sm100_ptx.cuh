@@ -196,6 +196,33 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn,
          ((uint32_t)(M >> 4) << 24);
 }
 
+// Instruction descriptor of kind::tf32 with fp32 (read as tf32) A and B and
+// an fp32 accumulator, both operands K-major (the only layout kind::tf32
+// takes).
+__host__ __device__ constexpr uint32_t idesc_tf32(int M, int N) {
+  return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t adesc,
+                                         uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Byte offset of fp32 element (row, c) inside one 128-byte-swizzled panel
+// whose rows hold 32 fp32 (K-major: rows along M or N, 32 consecutive k per
+// row): 16-byte chunk index XOR (row mod 8).
+__device__ __forceinline__ uint32_t swz32(int row, int c) {
+  return (uint32_t)(row * 128 + (((c >> 2) ^ (row & 7)) << 4) + ((c & 3) << 2));
+}
+
 // Byte offset of element (row, col) inside one 128-byte-swizzled panel whose
 // rows are 64 bf16 (128 B) wide: 16-byte chunk index XOR (row mod 8).
 __device__ __forceinline__ uint32_t sw128_off(int row, int col) {
