@@ -363,6 +363,7 @@ __global__ void __launch_bounds__(kThreads, 2)  // two CTAs per SM
     }
   }
   if (wt_out) {  // W^T [dk][C] of this chunk from the A region, zero past L
+    __syncthreads();  // every thread's part of W^T is staged
     const size_t tb = ((size_t)cid * H + h) * dk * C;
     for (int idx = tid; idx < dk * C; idx += kThreads) {
       const int col = idx / C, r = idx % C;
@@ -859,20 +860,25 @@ cudaError_t set_smem(K kernel, size_t bytes) {
 // op(A) (rows i, contraction t) as a K-major tf32 operand: 128-byte-swizzled
 // panels of 32 t each, `rows` x 128 B per panel.  Source A[i][t]: each thread
 // moves one 16-byte vector of a source row.
+// 16-byte loads each thread keeps in flight while staging (the staging is
+// bound by their latency).
+// (Eight and four measured slower than four and two.)
+constexpr int kDirectBatch = 4, kTransBatch = 2;
+
 __device__ __forceinline__ void stage_km_direct(const Src& s, int rows, int cols,
                                                 uint8_t* dst, int panel,
                                                 int tid) {
   const int cv = cols >> 2, units = rows * cv;
-  for (int base = 0; base < units; base += 4 * kThreads) {
-    float4 v[4];
+  for (int base = 0; base < units; base += kDirectBatch * kThreads) {
+    float4 v[kDirectBatch];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < kDirectBatch; ++u) {
       const int idx = base + u * kThreads + tid;
       v[u] = idx < units ? ld_src4(s, idx / cv, (idx % cv) * 4)
                          : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < kDirectBatch; ++u) {
       const int idx = base + u * kThreads + tid;
       if (idx < units) {
         const int r = idx / cv, c = (idx % cv) * 4;
@@ -890,10 +896,10 @@ __device__ __forceinline__ void stage_km_transposed(const Src& s, int rows,
                                                     int cols, uint8_t* dst,
                                                     int panel, int tid) {
   const int units = rows * (cols >> 3);
-  for (int base = 0; base < units; base += 2 * kThreads) {
-    float4 v[2][2];
+  for (int base = 0; base < units; base += kTransBatch * kThreads) {
+    float4 v[kTransBatch][2];
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
+    for (int u = 0; u < kTransBatch; ++u) {
       const int idx = base + u * kThreads + tid;
       const int r = idx % rows, c = (idx / rows) * 8;
       const bool in = idx < units;
@@ -901,7 +907,7 @@ __device__ __forceinline__ void stage_km_transposed(const Src& s, int rows,
       v[u][1] = in ? ld_src4(s, r, c + 4) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
+    for (int u = 0; u < kTransBatch; ++u) {
       const int idx = base + u * kThreads + tid;
       if (idx < units) {
         const int r = idx % rows, c = (idx / rows) * 8;

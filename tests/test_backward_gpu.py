@@ -103,3 +103,26 @@ def test_backward_config2_sampled():
             None, PY.host64(unit(do)), PY.host64(dsT[s:s + 1, h:h + 1]))
         mine = [unit(x) for x in got[:5]] + [got[5][s:s + 1, h:h + 1]]
         compare(mine, ref, PY.TOL_BF16)
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_backward_is_deterministic(io):
+    # two calls on the same inputs agree bit for bit: every kernel of the
+    # backward (the tensor-core ones included) reduces in a fixed order, so a
+    # difference can only come from a race
+    lengths = [130, 64, 5, 200]
+    T = sum(lengths)
+    d = W.draw((1, T), 3, 128, 128, io=io, n_states=len(lengths), device=DEV,
+               seed=91)
+    offs = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
+    cu = torch.tensor(offs, dtype=torch.int32, device=DEV)
+    do, dsT = grads_in(d, seed=92)
+    runs = []
+    for _ in range(3):
+        got = K.chunk_bwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"],
+                          d["initial_state"], cu, do, dsT, chunk=64)
+        torch.cuda.synchronize()
+        runs.append([x.clone() for x in got if x is not None])
+    for later in runs[1:]:
+        for name, a, b in zip(NAMES, runs[0], later):
+            assert torch.equal(a, b), f"{name} differs between two calls"
