@@ -48,6 +48,7 @@
 #include "kda_common.cuh"
 #include "kda_internal.h"
 #include "kda_inverse.cuh"
+#include "kda_tmap.h"
 #include "sm100_ptx.cuh"
 
 namespace kda {
@@ -922,15 +923,26 @@ __device__ __forceinline__ void stage_km_transposed(const Src& s, int rows,
   }
 }
 
+// Tensor maps of the operands that TMA stages: [term][0 = A, 1 = B].
+struct BmmMaps {
+  CUtensorMap m[3][2];
+};
+
 // Tensor-core form of bmm_kernel for bf16 inputs in 64-token chunks (every
 // dimension 64 or 128): per (chunk, head), each term's op(A) and op(B) are
 // staged as K-major tf32 operands and multiplied by tcgen05 kind::tf32 into
 // one TMEM accumulator of MD x ND; the epilogue applies alpha, the mask and
 // the accumulation as bmm_kernel does.  MD = 64 uses the M = 64 shape, whose
 // rows 16 q .. 16 q + 15 land in TMEM lanes 32 q .. 32 q + 15.
+// Operands already K-major in memory (token rows or states whose rows are
+// M or N) arrive by TMA, one 32-column box per panel (bit 2 term + side of
+// tma_mask); the threads stage the others meanwhile.  A token box's rows
+// past the chunk are other tokens (or zero past the tensor): they only
+// reach output rows or columns past m or n, which are not stored.
 template <int MD, int ND>
 __global__ void __launch_bounds__(kThreads, MD == 64 ? 2 : 1)
-    bmm_tc_kernel(BmmOp op, const int32_t* cu, const int32_t* chunk_off,
+    bmm_tc_kernel(BmmOp op, const __grid_constant__ BmmMaps maps,
+                  int tma_mask, const int32_t* cu, const int32_t* chunk_off,
                   int n_seqs, int T, int H, int dk, int dv, int C) {
   using namespace sm100;
   const int cid = blockIdx.x;
@@ -944,9 +956,11 @@ __global__ void __launch_bounds__(kThreads, MD == 64 ? 2 : 1)
   uint8_t* As = sm;                 // up to four panels
   uint8_t* Bs = sm + 4 * kPanA;     // up to four panels
   uint64_t* bar = reinterpret_cast<uint64_t*>(Bs + 4 * kPanB);
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 1);
+  uint64_t* tbar = bar + 1;  // TMA operand copies
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 2);
   if (tid == 0) {
     mbar_init(bar, 1);
+    mbar_init(tbar, 1);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -958,16 +972,47 @@ __global__ void __launch_bounds__(kThreads, MD == 64 ? 2 : 1)
   tc_fence_after();
   const uint32_t tmem = *tslot;
   bool ok = true;
+  int tphase = 0;
   for (int term = 0; term < op.nterms && ok; ++term) {
     const BmmTerm tm = term == 0 ? op.term[0]
                        : term == 1 ? op.term[1] : op.term[2];
     const int kd = tm.kd;
+    const bool ta = (tma_mask >> (2 * term)) & 1;
+    const bool tb = (tma_mask >> (2 * term + 1)) & 1;
+    if (tid == 0 && (ta || tb)) {
+      mbar_arrive_expect_tx(
+          tbar, (ta ? (kd / 32) * kPanA : 0) + (tb ? (kd / 32) * kPanB : 0));
+      for (int side = 0; side < 2; ++side) {
+        if (!(side == 0 ? ta : tb)) continue;
+        const MatRef& x = side == 0 ? tm.a : tm.b;
+        uint8_t* dst = side == 0 ? As : Bs;
+        const int pan = side == 0 ? kPanA : kPanB;
+        for (int q = 0; q < kd / 32; ++q) {
+          if (x.kind == kTok)
+            tma_load_3d(dst + q * pan, &maps.m[term][side], tbar, 32 * q, h,
+                        tok0);
+          else
+            tma_load_2d(dst + q * pan, &maps.m[term][side], tbar, 32 * q,
+                        (int)(((size_t)cid * H + h) * dk));
+        }
+      }
+    }
     const Src sa = src_of(tm.a, cid, h, tok0, L, H, C, dk);
     const Src sb = src_of(tm.b, cid, h, tok0, L, H, C, dk);
-    if (tm.a.trans) stage_km_transposed(sa, kd, MD, As, kPanA, tid);  // A[t][i]
-    else stage_km_direct(sa, MD, kd, As, kPanA, tid);                 // A[i][t]
-    if (tm.b.trans) stage_km_direct(sb, ND, kd, Bs, kPanB, tid);      // B[j][t]
-    else stage_km_transposed(sb, kd, ND, Bs, kPanB, tid);             // B[t][j]
+    if (!ta) {
+      if (tm.a.trans) stage_km_transposed(sa, kd, MD, As, kPanA, tid);  // A[t][i]
+      else stage_km_direct(sa, MD, kd, As, kPanA, tid);                 // A[i][t]
+    }
+    if (!tb) {
+      if (tm.b.trans) stage_km_direct(sb, ND, kd, Bs, kPanB, tid);  // B[j][t]
+      else stage_km_transposed(sb, kd, ND, Bs, kPanB, tid);         // B[t][j]
+    }
+    if (ta || tb) {
+      ok = __syncthreads_and(mbar_wait(tbar, (uint32_t)tphase & 1u,
+                                       2000000000ull));
+      ++tphase;
+      if (!ok) break;
+    }
     fence_proxy_async();
     tc_fence_before();
     __syncthreads();
@@ -1040,29 +1085,58 @@ __global__ void __launch_bounds__(kThreads, MD == 64 ? 2 : 1)
 }
 
 template <int MD, int ND>
-cudaError_t launch_bmm_tc_t(const BmmOp& op, dim3 grid, cudaStream_t stream,
-                            const int32_t* cu, const int32_t* co, int n_seqs,
-                            int T, int H, int dk, int dv, int C) {
+cudaError_t launch_bmm_tc_t(const BmmOp& op, const BmmMaps& maps, int mask,
+                            dim3 grid, cudaStream_t stream, const int32_t* cu,
+                            const int32_t* co, int n_seqs, int T, int H,
+                            int dk, int dv, int C) {
   const size_t smem = 4 * (size_t)(MD + ND) * 128 + 1024 + 64;
   cudaError_t e = set_smem(bmm_tc_kernel<MD, ND>, smem);
   if (e != cudaSuccess) return e;
-  bmm_tc_kernel<MD, ND><<<grid, kThreads, smem, stream>>>(op, cu, co, n_seqs,
-                                                          T, H, dk, dv, C);
+  bmm_tc_kernel<MD, ND><<<grid, kThreads, smem, stream>>>(
+      op, maps, mask, cu, co, n_seqs, T, H, dk, dv, C);
   return cudaGetLastError();
+}
+
+// The maps of the operands stored K-major with M or N as their rows: token
+// rows (their rows are the chunk's tokens, M or N = 64) and states whose
+// rows are d_k.  Square per-chunk operands stay with the threads, which zero
+// their entries past the chunk's length.
+int bmm_tc_maps(const BmmOp& op, BmmMaps* maps, int tokens, int64_t nch,
+                int H, int dk) {
+  int mask = 0;
+  for (int t = 0; t < op.nterms; ++t)
+    for (int side = 0; side < 2; ++side) {
+      const MatRef& x = side == 0 ? op.term[t].a : op.term[t].b;
+      const bool direct = side == 0 ? !x.trans : x.trans;
+      const int rows = side == 0 ? op.md : op.nd;  // the box's rows
+      if (!direct || op.term[t].kd != x.cols) continue;
+      bool ok = false;
+      if (x.kind == kTok && rows == 64)
+        ok = make_f32_tok_map(&maps->m[t][side], x.p, x.cols, H, tokens);
+      else if (x.kind == kState && rows == dk)
+        ok = make_f32_rows_map(&maps->m[t][side], x.p, nch * H * dk, x.cols,
+                               dk);
+      if (ok) mask |= 1 << (2 * t + side);
+    }
+  return mask;
 }
 
 cudaError_t launch_bmm_tc(const BmmOp& op, int C, dim3 grid,
                           cudaStream_t stream, const int32_t* cu,
                           const int32_t* co, int n_seqs, int T, int H, int dk,
-                          int dv) {
-  if (op.md == 64 && op.nd == 64)
-    return launch_bmm_tc_t<64, 64>(op, grid, stream, cu, co, n_seqs, T, H, dk, dv, C);
-  if (op.md == 64 && op.nd == 128)
-    return launch_bmm_tc_t<64, 128>(op, grid, stream, cu, co, n_seqs, T, H, dk, dv, C);
-  if (op.md == 128 && op.nd == 64)
-    return launch_bmm_tc_t<128, 64>(op, grid, stream, cu, co, n_seqs, T, H, dk, dv, C);
-  if (op.md == 128 && op.nd == 128)
-    return launch_bmm_tc_t<128, 128>(op, grid, stream, cu, co, n_seqs, T, H, dk, dv, C);
+                          int dv, int64_t nch) {
+  BmmMaps maps;
+  const int mask =
+      bmm_tc_maps(op, &maps, cu ? T : n_seqs * T, nch, H, dk);
+#define KDA_TC(M_, N_)                                                    \
+  if (op.md == M_ && op.nd == N_)                                         \
+    return launch_bmm_tc_t<M_, N_>(op, maps, mask, grid, stream, cu, co,  \
+                                   n_seqs, T, H, dk, dv, C);
+  KDA_TC(64, 64)
+  KDA_TC(64, 128)
+  KDA_TC(128, 64)
+  KDA_TC(128, 128)
+#undef KDA_TC
   return cudaErrorInvalidValue;
 }
 
@@ -1164,7 +1238,7 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
     const int kd = max(t0.kd, max(nterms > 1 ? t1.kd : 0, nterms > 2 ? t2.kd : 0));
     if (w.wt)  // bf16 inputs in 64-token chunks: on the tensor cores (tf32)
       return launch_bmm_tc(op, C, grid, stream, cu, co, f.n_seqs, f.T, H, dk,
-                           dv);
+                           dv, nch);
     const size_t smem = 4 * (size_t)kd * ((op.md + 4) + (op.nd + 4));
     return launch_bmm(op, C, smem, grid, stream, cu, co, f.n_seqs, f.T, H, dk,
                       dv);

@@ -30,6 +30,7 @@ namespace kda {
 namespace bwdtc {
 
 using sm100::idesc_tf32;
+using sm100::tma_load_2d;
 using sm100::mma_tf32;
 using sm100::swz32;
 using ws::named_sync_or;
@@ -41,16 +42,6 @@ constexpr int kC = 64;        // chunk length
 constexpr int kTile = 64;     // d_v columns per CTA
 constexpr int kThreads = 256;
 constexpr int kBarAll = 1;
-
-__device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap,
-                                            uint64_t* bar, int c0, int c1) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::"
-      "bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(sm100::smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1),
-      "r"(sm100::smem_u32(bar))
-      : "memory");
-}
 
 struct Params {
   const float* gam;      // exp(g_C)     [chunks, H, dk]

@@ -24,6 +24,7 @@
 
 #include "kda_common.cuh"
 #include "kda_internal.h"
+#include "kda_tmap.h"
 #include "sm100_ptx.cuh"
 
 namespace kda {
@@ -279,6 +280,17 @@ cudaError_t launch_rev_chain_tc(const RevChainArgs& a, cudaStream_t stream) {
   if (a.dk == 128) return run_rev_chain_tc<128>(a, stream);
   if (a.dk == 64) return run_rev_chain_tc<64>(a, stream);
   return cudaErrorInvalidValue;
+}
+
+bool make_f32_tok_map(CUtensorMap* m, const float* base, int cols, int H,
+                      int tokens) {
+  return make_map(m, base, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, cols, H, tokens,
+                  32, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+bool make_f32_rows_map(CUtensorMap* m, const float* base, int64_t rows,
+                       int cols, int box_rows) {
+  return make_rows_map(m, base, rows, cols, box_rows);
 }
 
 }  // namespace kda
