@@ -808,21 +808,42 @@ __global__ void __launch_bounds__(kThreads)
   const int h = blockIdx.y, tid = threadIdx.x, ntile = dv / kChainTile;
   extern __shared__ float sm[];
   float* dg = sm;  // [C][dk]
-  for (int idx = tid; idx < L * dk; idx += kThreads) {
-    const int r = idx / dk;
-    const size_t gi = ((size_t)(tok0 + r) * H + h) * dk + idx % dk;
+  // four consecutive channels per thread and step (d_k, d_v multiples of 4)
+  auto ld4 = [](const float* p) { return *reinterpret_cast<const float4*>(p); };
+  const int dk4 = dk / 4, dv4 = dv / 4;
+  for (int idx = tid; idx < L * dk4; idx += kThreads) {
+    const int r = idx / dk4, c = (idx % dk4) * 4;
+    const size_t gi = ((size_t)(tok0 + r) * H + h) * dk + c;
     const float b = beta[(size_t)(tok0 + r) * H + h];
-    const float dKt = b * w.dbk[gi];
-    const float dKb = w.dkb[gi], dQt = w.dqt[gi];
-    const float gv = g[gi], e = __expf(gv), ie = __expf(-gv);
-    dk_out[gi] = from_f32<IO>(dKt * e + dKb * ie);
-    dq[gi] = from_f32<IO>(dQt * e);
-    dg[idx] = dKt * w.kt[gi] + dQt * w.qt[gi] - dKb * w.kb[gi];
+    const float4 bk = ld4(w.dbk + gi), kb4 = ld4(w.dkb + gi),
+                 qt4 = ld4(w.dqt + gi), g4 = ld4(g + gi), kt = ld4(w.kt + gi),
+                 qt = ld4(w.qt + gi), kb = ld4(w.kb + gi);
+    const float dKt[4] = {b * bk.x, b * bk.y, b * bk.z, b * bk.w};
+    const float dKb[4] = {kb4.x, kb4.y, kb4.z, kb4.w};
+    const float dQt[4] = {qt4.x, qt4.y, qt4.z, qt4.w};
+    const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
+    const float ktv[4] = {kt.x, kt.y, kt.z, kt.w};
+    const float qtv[4] = {qt.x, qt.y, qt.z, qt.w};
+    const float kbv[4] = {kb.x, kb.y, kb.z, kb.w};
+    float o[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float e = __expf(gv[u]), ie = __expf(-gv[u]);
+      dk_out[gi + u] = from_f32<IO>(dKt[u] * e + dKb[u] * ie);
+      dq[gi + u] = from_f32<IO>(dQt[u] * e);
+      o[u] = dKt[u] * ktv[u] + dQt[u] * qtv[u] - dKb[u] * kbv[u];
+    }
+    *reinterpret_cast<float4*>(dg + r * dk + c) = make_float4(o[0], o[1], o[2], o[3]);
   }
-  for (int idx = tid; idx < L * dv; idx += kThreads) {
-    const int r = idx / dv;
-    const size_t gi = ((size_t)(tok0 + r) * H + h) * dv + idx % dv;
-    dv_out[gi] = from_f32<IO>(beta[(size_t)(tok0 + r) * H + h] * w.dbv[gi]);
+  for (int idx = tid; idx < L * dv4; idx += kThreads) {
+    const int r = idx / dv4, c = (idx % dv4) * 4;
+    const size_t gi = ((size_t)(tok0 + r) * H + h) * dv + c;
+    const float b = beta[(size_t)(tok0 + r) * H + h];
+    const float4 x = ld4(w.dbv + gi);
+    dv_out[gi] = from_f32<IO>(b * x.x);
+    dv_out[gi + 1] = from_f32<IO>(b * x.y);
+    dv_out[gi + 2] = from_f32<IO>(b * x.z);
+    dv_out[gi + 3] = from_f32<IO>(b * x.w);
   }
   __syncthreads();
   for (int c = tid; c < dk; c += kThreads) {
@@ -856,16 +877,14 @@ cudaError_t set_smem(K kernel, size_t bytes) {
                               (int)bytes);
 }
 
-// Launch one batched product with the thread blocking its padded shape asks
-// for: RM = md / 16 rows and RN = nd / 16 columns per thread.
+// 16-byte loads each thread keeps in flight while staging a tensor-core
+// operand (the staging is bound by their latency; eight and four measured
+// slower than four and two).
+constexpr int kDirectBatch = 4, kTransBatch = 2;
+
 // op(A) (rows i, contraction t) as a K-major tf32 operand: 128-byte-swizzled
 // panels of 32 t each, `rows` x 128 B per panel.  Source A[i][t]: each thread
 // moves one 16-byte vector of a source row.
-// 16-byte loads each thread keeps in flight while staging (the staging is
-// bound by their latency).
-// (Eight and four measured slower than four and two.)
-constexpr int kDirectBatch = 4, kTransBatch = 2;
-
 __device__ __forceinline__ void stage_km_direct(const Src& s, int rows, int cols,
                                                 uint8_t* dst, int panel,
                                                 int tid) {
@@ -1140,6 +1159,8 @@ cudaError_t launch_bmm_tc(const BmmOp& op, int C, dim3 grid,
   return cudaErrorInvalidValue;
 }
 
+// Launch one batched product with the thread blocking its padded shape asks
+// for: RM = md / 16 rows and RN = nd / 16 columns per thread.
 template <int RM, int RN>
 cudaError_t launch_bmm_t(const BmmOp& op, size_t smem, dim3 grid,
                          cudaStream_t stream, const int32_t* cu,
