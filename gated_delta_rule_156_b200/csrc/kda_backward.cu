@@ -73,6 +73,9 @@ struct BwdWs {
   float* fin;                     // scratch final state of the forward
   void* tp;                       // the two-pass forward's workspace, or null
   float* wt;                      // W^T per chunk [chunks, H, dk, C], or null
+  // transposed per-chunk copies for the tensor-core products (or null):
+  // [chunks, H, d, C], zero past each chunk's last token; ddT holds -dDelta^T
+  float *qtT, *kbT, *bktT, *doT, *ddT;
   float *kt, *kb, *qt, *bkt;      // [tokens, H, dk]
   float *v32, *bv, *do32, *dd;    // [tokens, H, dv]
   float *tm, *pp;                 // [chunks, H, C, C]
@@ -107,7 +110,7 @@ bool tensor_state_pass(const ChunkArgs& f) {
 // coordinates.
 bool tensor_chain(const ChunkArgs& f) {
   return tensor_state_pass(f) &&
-         max_chunks(f) * f.H * f.dk < ((int64_t)1 << 31);
+         max_chunks(f) * f.H * (f.dk > f.dv ? f.dk : f.dv) < ((int64_t)1 << 31);
 }
 
 BwdWs carve_bwd(const BwdArgs& a, void* base, size_t* total) {
@@ -131,6 +134,15 @@ BwdWs carve_bwd(const BwdArgs& a, void* base, size_t* total) {
   w.wt = tensor_chain(fa)
              ? take(4 * (size_t)max_chunks(fa) * f.H * f.dk * f.chunk)
              : nullptr;
+  if (tensor_chain(fa)) {
+    const size_t tk = 4 * (size_t)max_chunks(fa) * f.H * f.dk * f.chunk;
+    const size_t tv = 4 * (size_t)max_chunks(fa) * f.H * f.dv * f.chunk;
+    w.qtT = take(tk);
+    w.kbT = take(tk);
+    w.bktT = take(tk);
+    w.doT = take(tv);
+    w.ddT = take(tv);
+  }
   const size_t tdk = 4 * tokens * H * dk, tdv = 4 * tokens * H * dv;
   const size_t sq = 4 * nch * H * C * C, st = 4 * nch * H * dk * dv;
   w.kt = take(tdk); w.kb = take(tdk); w.qt = take(tdk); w.bkt = take(tdk);
@@ -237,6 +249,16 @@ __global__ void __launch_bounds__(kThreads, 2)  // two CTAs per SM
   for (int c = tid; c < dk; c += kThreads)
     w.gam[((size_t)cid * H + h) * dk + c] = __expf(gl[c]);
   __syncthreads();
+  if (w.qtT) {  // transposed per-chunk copies for the tensor-core products
+    const size_t tb = ((size_t)cid * H + h) * dk * C;
+    for (int idx = tid; idx < dk * C; idx += kThreads) {
+      const int c = idx / C, r = idx % C;  // a warp reads one padded column
+      const bool in = r < L;
+      w.qtT[tb + idx] = in ? Qt[r * ldk + c] : 0.f;
+      w.kbT[tb + idx] = in ? Kb[r * ldk + c] : 0.f;
+      w.bktT[tb + idx] = in ? bs[r] * Kt[r * ldk + c] : 0.f;
+    }
+  }
   const size_t sqb = ((size_t)cid * H + h) * C * C;
   // Thread (ti, tj) owns rows ti + 16 a and columns tj + 16 b of each
   // product, so the padded rows give conflict-free loads.
@@ -369,6 +391,22 @@ __global__ void __launch_bounds__(kThreads, 2)  // two CTAs per SM
     for (int idx = tid; idx < dk * C; idx += kThreads) {
       const int col = idx / C, r = idx % C;
       wt_out[tb + idx] = r < L ? A[col * C + (r ^ (col & 31))] : 0.f;
+    }
+  }
+  if (w.doT) {
+    // dO^T per chunk: dO staged row-wise (column index XOR the row's low
+    // bits) in the Kt region, which nothing reads after W is formed
+    __syncthreads();
+    for (int idx = tid; idx < C * dv; idx += kThreads) {
+      const int r = idx / dv, c = idx % dv;
+      Kt[r * dv + (c ^ (r & 31))] =
+          r < L ? to_f32(dout[((size_t)(tok0 + r) * H + h) * dv + c]) : 0.f;
+    }
+    __syncthreads();
+    const size_t tb = ((size_t)cid * H + h) * dv * C;
+    for (int idx = tid; idx < dv * C; idx += kThreads) {
+      const int c = idx / C, r = idx % C;
+      w.doT[tb + idx] = Kt[r * dv + (c ^ (r & 31))];
     }
   }
 }
@@ -561,7 +599,9 @@ __global__ void __launch_bounds__(kThreads)
 // [tokens, H, cols] (rows are the chunk's tokens), a per-chunk square
 // [chunks, H, C, C], or a per-chunk state [chunks, H, dk, dv].  m, n and the
 // contraction length are each L, d_k or d_v.
-enum MatKind { kTok = 0, kSq = 1, kState = 2 };
+// kTokT: a per-chunk transposed copy of token rows, [chunks, H, cols, C]
+// (rows = the channels, C token columns).
+enum MatKind { kTok = 0, kSq = 1, kState = 2, kTokT = 3 };
 enum Dim { kDimL = 0, kDimDk = 1, kDimDv = 2 };
 enum Mask { kMaskNone = 0, kMaskLowerIncl = 1, kMaskStrictLower = 2 };
 
@@ -607,6 +647,8 @@ __device__ __forceinline__ Src src_of(const MatRef& x, int cid, int h,
                x.cols};
   if (x.kind == kSq)
     return Src{x.p + ((size_t)cid * H + h) * C * C, (size_t)C, L, L};
+  if (x.kind == kTokT)
+    return Src{x.p + ((size_t)cid * H + h) * x.cols * C, (size_t)C, x.cols, L};
   return Src{x.p + ((size_t)cid * H + h) * dk * x.cols, (size_t)x.cols, dk,
              x.cols};
 }
@@ -1010,9 +1052,10 @@ __global__ void __launch_bounds__(kThreads, MD == 64 ? 2 : 1)
           if (x.kind == kTok)
             tma_load_3d(dst + q * pan, &maps.m[term][side], tbar, 32 * q, h,
                         tok0);
-          else
+          else  // states: d_k rows; transposed copies: x.cols rows
             tma_load_2d(dst + q * pan, &maps.m[term][side], tbar, 32 * q,
-                        (int)(((size_t)cid * H + h) * dk));
+                        (int)(((size_t)cid * H + h) *
+                              (x.kind == kState ? dk : x.cols)));
         }
       }
     }
@@ -1117,9 +1160,10 @@ cudaError_t launch_bmm_tc_t(const BmmOp& op, const BmmMaps& maps, int mask,
 }
 
 // The maps of the operands stored K-major with M or N as their rows: token
-// rows (their rows are the chunk's tokens, M or N = 64) and states whose
-// rows are d_k.  Square per-chunk operands stay with the threads, which zero
-// their entries past the chunk's length.
+// rows (their rows are the chunk's tokens, M or N = 64), states whose rows
+// are d_k, and the transposed per-chunk copies (rows = channels, K = the 64
+// tokens, zero past the chunk).  Square per-chunk operands stay with the
+// threads, which zero their entries past the chunk's length.
 int bmm_tc_maps(const BmmOp& op, BmmMaps* maps, int tokens, int64_t nch,
                 int H, int dk) {
   int mask = 0;
@@ -1128,13 +1172,16 @@ int bmm_tc_maps(const BmmOp& op, BmmMaps* maps, int tokens, int64_t nch,
       const MatRef& x = side == 0 ? op.term[t].a : op.term[t].b;
       const bool direct = side == 0 ? !x.trans : x.trans;
       const int rows = side == 0 ? op.md : op.nd;  // the box's rows
-      if (!direct || op.term[t].kd != x.cols) continue;
+      if (!direct) continue;
       bool ok = false;
-      if (x.kind == kTok && rows == 64)
+      if (x.kind == kTok && rows == 64 && op.term[t].kd == x.cols)
         ok = make_f32_tok_map(&maps->m[t][side], x.p, x.cols, H, tokens);
-      else if (x.kind == kState && rows == dk)
+      else if (x.kind == kState && rows == dk && op.term[t].kd == x.cols)
         ok = make_f32_rows_map(&maps->m[t][side], x.p, nch * H * dk, x.cols,
                                dk);
+      else if (x.kind == kTokT && rows == x.cols && op.term[t].kd == 64)
+        ok = make_f32_rows_map(&maps->m[t][side], x.p, nch * H * x.cols, 64,
+                               x.cols);
       if (ok) mask |= 1 << (2 * t + side);
     }
   return mask;
@@ -1235,6 +1282,11 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
 
   auto tok = [](float* p, int cols, int t = 0) { return MatRef{p, kTok, cols, t}; };
+  // token rows contracted over the tokens: the transposed per-chunk copy on
+  // the tensor-core path (op = its transpose, K-major there), else the rows
+  auto tokc = [&](float* rows, float* copy, int cols) {
+    return copy ? MatRef{copy, kTokT, cols, 1} : MatRef{rows, kTok, cols, 0};
+  };
   auto sq = [&](float* p, int t = 0) { return MatRef{p, kSq, C, t}; };
   auto stt = [&](const float* p, int t = 0) {
     return MatRef{const_cast<float*>(p), kState, dv, t};
@@ -1279,10 +1331,12 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
   if ((e = __VA_ARGS__) != cudaSuccess) return e;
   if (nch > 0) {
     // the chain's terms that do not depend on dS: Qt^T dO and P^T dO
-    const BmmTerm tq = term(tok(w.qt, dk, 1), tok(w.do32, dv), kDimL);
+    const BmmTerm tq =
+        term(w.qtT ? MatRef{w.qtT, kTokT, dk, 0} : tok(w.qt, dk, 1),
+             tokc(w.do32, w.doT, dv), kDimL);
     KDA_BMM(bmm2(stt(w.qdo), tq, tq, 1, kDimDk, kDimDv, kMaskNone, 1.f, 0))
-    KDA_BMM(bmm(tok(w.pdo, dv), sq(w.pp, 1), tok(w.do32, dv), kDimDv, kDimL,
-                kMaskNone, 1.f, 0))
+    KDA_BMM(bmm(tok(w.pdo, dv), sq(w.pp, 1), tokc(w.do32, w.doT, dv), kDimDv,
+                kDimL, kMaskNone, 1.f, 0))
   }
   if (w.wt) {  // on the tensor cores (tf32), one CTA per 64 d_v columns
     RevChainArgs r{};
@@ -1297,6 +1351,7 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
     r.gst = w.gst;
     r.dd = w.dd;
     r.dgam = w.dgam;
+    r.ddT = w.ddT;
     r.d_init = a.d_initial_state;
     r.cu = cu;
     r.chunk_off = co;
@@ -1325,7 +1380,7 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
               kMaskLowerIncl, 1.f, 0))
   // dQt = dO S_0^T + dP Kb
   KDA_BMM(bmm2(tok(w.dqt, dk), term(tok(w.do32, dv), stt(S0, 1), kDimDv),
-               term(sq(w.dp), tok(w.kb, dk), kDimL), 2, kDimL, kDimDk,
+               term(sq(w.dp), tokc(w.kb, w.kbT, dk), kDimL), 2, kDimL, kDimDk,
                kMaskNone, 1.f, 0))
   // dW = -dDelta S_0^T
   KDA_BMM(bmm(tok(w.dw, dk), tok(w.dd, dv), stt(S0, 1), kDimDk, kDimDv,
@@ -1335,8 +1390,9 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
                term(tok(w.dd, dv), tok(w.bv, dv, 1), kDimDv), 2, kDimL, kDimL,
                kMaskNone, 1.f, 0))
   // Tm^T dDelta and Tm^T dTm
-  KDA_BMM(bmm(tok(w.dbv, dv), sq(w.tm, 1), tok(w.dd, dv), kDimDv, kDimL,
-              kMaskNone, 1.f, 0))
+  // (the transposed copy of dDelta is negated)
+  KDA_BMM(bmm(tok(w.dbv, dv), sq(w.tm, 1), tokc(w.dd, w.ddT, dv), kDimDv,
+              kDimL, kMaskNone, w.ddT ? -1.f : 1.f, 0))
   KDA_BMM(bmm(sq(w.tmp), sq(w.tm, 1), sq(w.dtm), kDimL, kDimL, kMaskNone, 1.f,
               0))
   // dA = strictly_lower(-(Tm^T dTm) Tm^T)
@@ -1344,12 +1400,13 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
               -1.f, 0))
   // dKt / b = Tm^T dW + dA Kb
   KDA_BMM(bmm2(tok(w.dbk, dk), term(sq(w.tm, 1), tok(w.dw, dk), kDimL),
-               term(sq(w.da), tok(w.kb, dk), kDimL), 2, kDimL, kDimDk,
+               term(sq(w.da), tokc(w.kb, w.kbT, dk), kDimL), 2, kDimL, kDimDk,
                kMaskNone, 1.f, 0))
   // dKb = Delta G^T + dP^T Qt + dA^T (b Kt)
   KDA_BMM(bmm3(tok(w.dkb, dk), term(tok(De, dv), stt(w.gst, 1), kDimDv),
-               term(sq(w.dp, 1), tok(w.qt, dk), kDimL),
-               term(sq(w.da, 1), tok(w.bkt, dk), kDimL), 3, kDimL, kDimDk,
+               term(sq(w.dp, 1), tokc(w.qt, w.qtT, dk), kDimL),
+               term(sq(w.da, 1), tokc(w.bkt, w.bktT, dk), kDimL), 3, kDimL,
+               kDimDk,
                kMaskNone, 1.f, 0))
 #undef KDA_BMM
   const size_t smf = 4 * (size_t)C * dk;

@@ -52,15 +52,16 @@ struct Params {
   const int32_t* cu;
   const int32_t* chunk_off;
   int n_seqs, T, H, dv;
+  int store_ddt;         // also store -dDelta^T per chunk (map ddt)
 };
 
 // The fp32 tensor maps (128-byte swizzle, boxes 32 columns wide): Kb and
 // P^T dO / dDelta over [tokens, H, d] (64-token boxes); W^T over
 // [chunks * H * dk, 64]; Qt^T dO, the start states, G over
 // [chunks * H * dk, dv] and the final states over [n_seqs * H * dk, dv]
-// (d_k-row boxes).
+// (d_k-row boxes); -dDelta^T over [chunks * H * dv, 64] (64-row boxes).
 struct Maps {
-  CUtensorMap kb, wt, qdo, s, fin, pdo, gst, dd;
+  CUtensorMap kb, wt, qdo, s, fin, pdo, gst, dd, ddt;
 };
 
 template <int DK>
@@ -395,6 +396,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (L == kC) {
         for (int q = 0; q < 2; ++q)
           tma_store_3d(&m.dd, pt + q * 8192, jt + 32 * q, h, tok0);
+        bulk_commit();
+      }
+      if (p.store_ddt) {  // the B panels: -dDelta^T, zero past the chunk
+        for (int q = 0; q < 2; ++q)
+          tma_store_2d(&m.ddt, dop + q * 8192, 32 * q,
+                       (int)(((size_t)cid * p.H + h) * p.dv + jt));
         bulk_commit();
       }
       ok = wait_or_abort<false>(bars + kWt, par, abort_flag);

@@ -260,10 +260,11 @@ cudaError_t run_rev_chain_tc(const RevChainArgs& a, cudaStream_t stream) {
       !make_rows_map(&m.qdo, a.qdo, crows, a.dv, DK) ||
       !make_rows_map(&m.s, a.s, crows, a.dv, DK) ||
       !make_rows_map(&m.gst, a.gst, crows, a.dv, DK) ||
-      !make_rows_map(&m.fin, a.fin, (int64_t)a.n_seqs * a.H * DK, a.dv, DK))
+      !make_rows_map(&m.fin, a.fin, (int64_t)a.n_seqs * a.H * DK, a.dv, DK) ||
+      (a.ddT && !make_rows_map(&m.ddt, a.ddT, a.n_chunks * a.H * a.dv, 64, 64)))
     return cudaErrorInvalidValue;
   bwdtc::Params p{a.gam, a.d_final, a.dd, a.dgam, a.d_init, a.cu,
-                  a.chunk_off, a.n_seqs, a.T, a.H, a.dv};
+                  a.chunk_off, a.n_seqs, a.T, a.H, a.dv, a.ddT ? 1 : 0};
   const size_t smem = Lay::bytes + 1024;
   cudaError_t e;
   if ((e = cudaFuncSetAttribute(bwdtc::rev_chain_kernel<DK>,

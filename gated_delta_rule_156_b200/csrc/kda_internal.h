@@ -120,6 +120,7 @@ struct RevChainArgs {
   float* gst;            // G out [chunks, H, dk, dv]
   float* dd;             // dDelta out [tokens, H, dv]
   float* dgam;           // gam * d gam partials [chunks, H, dv / 32, dk]
+  float* ddT;            // -dDelta^T per chunk [chunks, H, dv, 64], or null
   float* d_init;         // or null
   const int32_t* cu;
   const int32_t* chunk_off;
