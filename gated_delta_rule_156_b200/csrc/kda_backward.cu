@@ -171,9 +171,10 @@ __host__ __device__ constexpr int prep_region(int C, int dk, int dv) {
 // Per (chunk, head): Kt, Kb, Qt, b Kt and fp32 copies of V, b V, dO; gam;
 // M = Kt Kb^T (strictly lower, kept only on chip), P = lower_incl(Qt Kb^T),
 // Tm = (I + Diag(b) M)^-1 by recursive doubling, and the forward's
-// W = Tm Diag(b) Kt; for the SIMT state pass also U = Tm Diag(b) V and
-// Kh = k exp(g_C - g) (u_out, kh_out null otherwise), and for the
-// tensor-core chain W^T per chunk (wt_out, else null).
+// W = Tm Diag(b) Kt: row-major for the SIMT chain (w_out, else null), and
+// W^T per chunk for the tensor-core chain (wt_out, else null); for the SIMT
+// state pass also U = Tm Diag(b) V and Kh = k exp(g_C - g) (u_out, kh_out
+// null otherwise).
 template <typename IO>
 __global__ void __launch_bounds__(kThreads, 2)  // two CTAs per SM
     prep_kernel(const IO* __restrict__ q, const IO* __restrict__ k,
@@ -364,7 +365,7 @@ __global__ void __launch_bounds__(kThreads, 2)  // two CTAs per SM
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
       const int r = ti + 16 * a;
-      if (a < nr && r < L) {
+      if (out && a < nr && r < L) {
         const size_t ro = ((size_t)(tok0 + r) * H + h) * cols;
 #pragma unroll
         for (int b = 0; b < 8; ++b)
@@ -1266,7 +1267,8 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
     prep_kernel<IO><<<grid, kThreads, smp, stream>>>(
         static_cast<const IO*>(f.q), static_cast<const IO*>(f.k),
         static_cast<const IO*>(f.v), f.beta, static_cast<const IO*>(a.d_out),
-        w.fv.g, w, w.fv.w, tensor_state_pass(f) ? nullptr : w.fv.d,
+        w.fv.g, w, w.wt ? nullptr : w.fv.w,
+        tensor_state_pass(f) ? nullptr : w.fv.d,
         tensor_state_pass(f) ? nullptr : w.fv.kh, w.wt, cu, co, f.n_seqs, f.T,
         H, dk, dv, C);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
