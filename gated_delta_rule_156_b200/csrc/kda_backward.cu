@@ -412,6 +412,254 @@ __global__ void __launch_bounds__(kThreads, 2)  // two CTAs per SM
   }
 }
 
+// prep on the tensor cores, for bf16 inputs in 64-token chunks (the
+// tensor-core backward): the same outputs as prep_kernel in that mode, with
+// its three products as tcgen05 kind::tf32 MMAs on 128-byte-swizzled
+// K-major fp32 panels: M = Kt Kb^T and P = Qt Kb^T (M = 64 shape, K = d_k),
+// then W = T' Kt (K = the 64 tokens, Kt transposed in shared memory).  The
+// inverse stays the SIMT recursive doubling.  W goes out only as W^T per
+// chunk.  Shared memory: the Kt panels, then one region that holds the Qt
+// and Kb panels, later the inverse's tiles, then T' and Kt^T, then dO for
+// its transposed copy.
+template <int DK>
+struct PrepTcLayout {
+  static constexpr uint32_t kt = 0;                   // DK / 32 panels, 8 KB
+  static constexpr uint32_t r2 = DK * 256;            // Qt | Kb panels ...
+  static constexpr uint32_t qt = r2, kb = r2 + DK * 256;
+  static constexpr uint32_t am = r2;                  // [64][kFS] fp32
+  static constexpr uint32_t msc = r2 + 64 * ws::kFS * 4;
+  static constexpr uint32_t tm = msc + 4096;          // [64][kFS] fp32
+  static constexpr uint32_t tp = r2 + 40960;          // T': two 8 KB panels
+  static constexpr uint32_t ktt = r2;                 // Kt^T: two DK-row panels
+  static constexpr uint32_t r2_bytes =
+      2 * DK * 256 > 57344 ? 2 * DK * 256 : 57344;
+  static constexpr uint32_t misc = r2 + r2_bytes;     // barrier, TMEM slot
+  static constexpr uint32_t bs = misc + 64;           // [64] beta
+  static constexpr uint32_t gl = bs + 256;            // [DK] g at the last row
+  static constexpr uint32_t bytes = gl + DK * 4;
+  static_assert(tm + 64 * ws::kFS * 4 <= tp, "inverse tiles below T'");
+  static_assert(ktt + 2 * DK * 128 <= tp, "Kt^T below T'");
+  static_assert(tp + 16384 <= r2 + r2_bytes, "T' inside the region");
+};
+
+template <int DK>
+__global__ void __launch_bounds__(kThreads, 2)
+    prep_tc_kernel(const __nv_bfloat16* __restrict__ q,
+                   const __nv_bfloat16* __restrict__ k,
+                   const __nv_bfloat16* __restrict__ v,
+                   const float* __restrict__ beta,
+                   const __nv_bfloat16* __restrict__ dout,
+                   const float* __restrict__ g, BwdWs w,
+                   const int32_t* cu, const int32_t* chunk_off, int n_seqs,
+                   int T, int H, int dv) {
+  using namespace sm100;
+  using Lay = PrepTcLayout<DK>;
+  constexpr int C = 64;
+  const int cid = blockIdx.x;
+  int seq, tok0, L;
+  if (!locate_chunk(cid, cu, chunk_off, n_seqs, T, C, &seq, &tok0, &L)) return;
+  const int h = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* KT = sm + Lay::kt;
+  uint8_t* QT = sm + Lay::qt;
+  uint8_t* KB = sm + Lay::kb;
+  float* Am = reinterpret_cast<float*>(sm + Lay::am);
+  float* Msc = reinterpret_cast<float*>(sm + Lay::msc);
+  float* Tm = reinterpret_cast<float*>(sm + Lay::tm);
+  uint8_t* TP = sm + Lay::tp;
+  uint8_t* KTT = sm + Lay::ktt;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + Lay::misc);
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 1);
+  float* bs = reinterpret_cast<float*>(sm + Lay::bs);
+  float* gl = reinterpret_cast<float*>(sm + Lay::gl);
+  auto pel = [](uint8_t* panels, int r, int c) {  // (row r, column c)
+    return reinterpret_cast<float*>(panels + (c >> 5) * 8192 +
+                                    swz32(r, c & 31));
+  };
+
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tslot, 128);
+    tmem_relinquish();
+  }
+  for (int r = tid; r < C; r += kThreads)
+    bs[r] = r < L ? beta[(size_t)(tok0 + r) * H + h] : 0.f;
+  for (int c = tid; c < DK; c += kThreads) {
+    gl[c] = g[((size_t)(tok0 + L - 1) * H + h) * DK + c];
+    if (fabsf(gl[c]) > kBwdDecayMax) atomicExch(&g_bwd_range, 1);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+
+  // ---- Kt, Kb, Qt: the workspace rows and the operand panels
+  for (int idx = tid; idx < C * DK; idx += kThreads) {
+    const int r = idx / DK, c = idx % DK;
+    float kt = 0.f, kb = 0.f, qt = 0.f;
+    if (r < L) {
+      const size_t gi = ((size_t)(tok0 + r) * H + h) * DK + c;
+      const float kv = to_f32(k[gi]), qv = to_f32(q[gi]), gv = g[gi];
+      const float e = __expf(gv), ie = __expf(-gv);
+      kt = kv * e;
+      kb = kv * ie;
+      qt = qv * e;
+      w.kt[gi] = kt;
+      w.kb[gi] = kb;
+      w.qt[gi] = qt;
+      w.bkt[gi] = bs[r] * kt;
+    }
+    *pel(KT, r, c) = kt;
+    *pel(KB, r, c) = kb;
+    *pel(QT, r, c) = qt;
+  }
+  for (int idx = tid; idx < L * dv; idx += kThreads) {
+    const int r = idx / dv;
+    const size_t gi = ((size_t)(tok0 + r) * H + h) * dv + idx % dv;
+    const float vv = to_f32(v[gi]);
+    w.v32[gi] = vv;
+    w.bv[gi] = bs[r] * vv;
+    w.do32[gi] = to_f32(dout[gi]);
+  }
+  for (int c = tid; c < DK; c += kThreads)
+    w.gam[((size_t)cid * H + h) * DK + c] = __expf(gl[c]);
+  fence_proxy_async();
+  tc_fence_before();
+  __syncthreads();
+
+  // ---- M = Kt Kb^T (TMEM columns 0-63), P = Qt Kb^T (64-127)
+  if (tid == 0) {
+    tc_fence_after();
+    constexpr uint32_t id = idesc_tf32(64, 64);
+#pragma unroll
+    for (int ks = 0; ks < DK / 8; ++ks) {
+      const uint32_t o = (ks >> 2) * 8192 + (ks & 3) * 32;
+      const uint64_t bd = desc_sw128(smem_u32(KB) + o, 16, 1024);
+      mma_tf32(tmem, desc_sw128(smem_u32(KT) + o, 16, 1024), bd, id, ks > 0);
+      mma_tf32(tmem + 64, desc_sw128(smem_u32(QT) + o, 16, 1024), bd, id,
+               ks > 0);
+    }
+    mma_commit(bar);
+  }
+  // the transposed copies meanwhile (reads only)
+  {
+    const size_t tb = ((size_t)cid * H + h) * DK * C;
+    for (int idx = tid; idx < DK * C; idx += kThreads) {
+      const int c = idx / C, r = idx % C;
+      w.qtT[tb + idx] = *pel(QT, r, c);
+      w.kbT[tb + idx] = *pel(KB, r, c);
+      w.bktT[tb + idx] = bs[r] * *pel(KT, r, c);
+    }
+  }
+  bool ok = __syncthreads_and(mbar_wait(bar, 0, 2000000000ull));
+  tc_fence_after();
+  if (ok) {
+    // ---- A = Diag(b) strictly_lower(M) for the inverse; P out
+    for (int idx = tid; idx < 64 * ws::kFS; idx += kThreads) {
+      Am[idx] = 0.f;
+      Tm[idx] = 0.f;
+    }
+    __syncthreads();
+    const int qd = warp & 3, half = warp >> 2, r = 16 * qd + lane;
+    float mv[32], pv[32];
+    tmem_ld32(tmem + ((uint32_t)(32 * qd) << 16) + 32 * half, mv);
+    tmem_ld32(tmem + ((uint32_t)(32 * qd) << 16) + 64 + 32 * half, pv);
+    if (lane < 16) {  // M = 64 accumulator rows 16 qd .. 16 qd + 15
+      const size_t sqb = ((size_t)cid * H + h) * C * C;
+      float* pr = w.pp + sqb + r * C + 32 * half;
+#pragma unroll
+      for (int u = 0; u < 32; ++u) {
+        const int i = 32 * half + u;
+        Am[r * ws::kFS + i] = (r < L && i < r) ? bs[r] * mv[u] : 0.f;
+        pv[u] = (r < L && i <= r) ? pv[u] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        reinterpret_cast<float4*>(pr)[u] =
+            make_float4(pv[4 * u], pv[4 * u + 1], pv[4 * u + 2], pv[4 * u + 3]);
+    }
+    tc_fence_before();
+    __syncthreads();
+    // ---- Tm = (I + A)^-1; T' = Tm Diag(b) as the A panels of W = T' Kt
+    ws::invert_unit_lower(Am, Tm, Msc, tid);
+    __syncthreads();
+    {
+      const size_t sqb = ((size_t)cid * H + h) * C * C;
+      for (int idx = tid; idx < C * C; idx += kThreads) {
+        const int rr = idx / C, i = idx % C;
+        const float t = Tm[rr * ws::kFS + i];
+        w.tm[sqb + idx] = t;
+        *pel(TP, rr, i) = t * bs[i];
+      }
+    }
+    __syncthreads();
+    // Kt^T as the K-major B panels of W (rows = channels, K = tokens)
+    for (int idx = tid; idx < C * DK; idx += kThreads) {
+      const int c = idx / C, i = idx % C;
+      *reinterpret_cast<float*>(KTT + (i >> 5) * (DK * 128) + swz32(c, i & 31)) =
+          *pel(KT, i, c);
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      constexpr uint32_t id = idesc_tf32(64, DK);
+#pragma unroll
+      for (int ks = 0; ks < C / 8; ++ks)
+        mma_tf32(tmem,
+                 desc_sw128(smem_u32(TP) + (ks >> 2) * 8192 + (ks & 3) * 32,
+                            16, 1024),
+                 desc_sw128(smem_u32(KTT) + (ks >> 2) * (DK * 128) +
+                                (ks & 3) * 32,
+                            16, 1024),
+                 id, ks > 0);
+      mma_commit(bar);
+    }
+    ok = __syncthreads_and(mbar_wait(bar, 1, 2000000000ull));
+    tc_fence_after();
+  }
+  if (ok) {
+    // ---- W^T out: thread row r holds W[r][columns], zero past L
+    const int qd = warp & 3, half = warp >> 2, r = 16 * qd + lane;
+    const size_t tb = ((size_t)cid * H + h) * DK * C;
+#pragma unroll
+    for (int cc = 0; cc < DK / 64; ++cc) {
+      const int j0 = half * (DK / 2) + 32 * cc;
+      float wv[32];
+      tmem_ld32(tmem + ((uint32_t)(32 * qd) << 16) + j0, wv);
+      if (lane < 16) {
+#pragma unroll
+        for (int u = 0; u < 32; ++u)
+          w.wt[tb + (size_t)(j0 + u) * C + r] = r < L ? wv[u] : 0.f;
+      }
+    }
+    // ---- dO^T per chunk, staged row-wise (XOR-swizzled) in the region
+    float* Ds = reinterpret_cast<float*>(sm + Lay::r2);
+    for (int idx = tid; idx < C * dv; idx += kThreads) {
+      const int rr = idx / dv, c = idx % dv;
+      Ds[rr * dv + (c ^ (rr & 31))] =
+          rr < L ? to_f32(dout[((size_t)(tok0 + rr) * H + h) * dv + c]) : 0.f;
+    }
+    __syncthreads();
+    const size_t tv = ((size_t)cid * H + h) * dv * C;
+    for (int idx = tid; idx < dv * C; idx += kThreads) {
+      const int c = idx / C, rr = idx % C;
+      w.doT[tv + idx] = Ds[rr * dv + (c ^ (rr & 31))];
+    }
+  } else if (tid == 0) {
+    atomicExch(&g_bwd_timeout, 1);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 128);
+}
+
 // The reverse chain over one sequence's chunks for one head and one 32-wide
 // column tile of d_v (92 KB of shared memory at d = 128, so two CTAs share an
 // SM and a B=2, H=32 layer's 256 CTAs run as one wave).  Per chunk (last first), with dS the gradient of the
@@ -1262,8 +1510,30 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
   const dim3 grid((unsigned)(nch > 0 ? nch : 1), H);
 
   if (nch > 0) {
+    const bool tc = w.wt && sizeof(IO) == 2;
     const size_t smp = 4 * (3 * (size_t)prep_region(C, dk, dv) + C + dk);
-    if ((e = set_smem(prep_kernel<IO>, smp)) != cudaSuccess) return e;
+    if (tc) {  // bf16 inputs in 64-token chunks: prep on the tensor cores
+      const __nv_bfloat16* b16[4] = {
+          reinterpret_cast<const __nv_bfloat16*>(f.q),
+          reinterpret_cast<const __nv_bfloat16*>(f.k),
+          reinterpret_cast<const __nv_bfloat16*>(f.v),
+          reinterpret_cast<const __nv_bfloat16*>(a.d_out)};
+      if (dk == 128) {
+        const size_t sz = PrepTcLayout<128>::bytes + 1024;
+        if ((e = set_smem(prep_tc_kernel<128>, sz)) != cudaSuccess) return e;
+        prep_tc_kernel<128><<<grid, kThreads, sz, stream>>>(
+            b16[0], b16[1], b16[2], f.beta, b16[3], w.fv.g, w, cu, co,
+            f.n_seqs, f.T, H, dv);
+      } else {
+        const size_t sz = PrepTcLayout<64>::bytes + 1024;
+        if ((e = set_smem(prep_tc_kernel<64>, sz)) != cudaSuccess) return e;
+        prep_tc_kernel<64><<<grid, kThreads, sz, stream>>>(
+            b16[0], b16[1], b16[2], f.beta, b16[3], w.fv.g, w, cu, co,
+            f.n_seqs, f.T, H, dv);
+      }
+    } else if ((e = set_smem(prep_kernel<IO>, smp)) != cudaSuccess) {
+      return e;
+    } else {
     prep_kernel<IO><<<grid, kThreads, smp, stream>>>(
         static_cast<const IO*>(f.q), static_cast<const IO*>(f.k),
         static_cast<const IO*>(f.v), f.beta, static_cast<const IO*>(a.d_out),
@@ -1271,6 +1541,7 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
         tensor_state_pass(f) ? nullptr : w.fv.d,
         tensor_state_pass(f) ? nullptr : w.fv.kh, w.wt, cu, co, f.n_seqs, f.T,
         H, dk, dv, C);
+    }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   // the forward's serial state pass: chunk-start states, Delta over U, and
