@@ -71,7 +71,6 @@ struct BwdWs {
   StagedView fv;
   void* staged;                   // the forward's workspace
   float* fin;                     // scratch final state of the forward
-  void* tp;                       // the two-pass forward's workspace, or null
   float* wt;                      // W^T per chunk [chunks, H, dk, C], or null
   // transposed per-chunk copies for the tensor-core products (or null):
   // [chunks, H, d, C], zero past each chunk's last token; ddT holds -dDelta^T
@@ -98,18 +97,16 @@ ChunkArgs forward_args(const BwdArgs& a, float* fin) {
   return f;
 }
 
-// The forward's state pass runs as the tensor-core two-pass forward where
-// that path takes the shape (bf16 inputs, 64-token chunks, d_k and d_v in
-// {64, 128}); its bf16 operands sit inside the bf16 tolerance.  fp32 inputs
-// keep the fp32 SIMT pass.
-bool tensor_state_pass(const ChunkArgs& f) {
-  return fused_supported(f) && max_chunks(f) > 0;
-}
-// The reverse chain on the tensor cores (tf32) under the same condition, as
-// long as the rows of W^T stay within a tensor map's signed 32-bit
-// coordinates.
+// The tensor-core path (prep, the reverse chain and the batched products in
+// tf32) where the shape allows it: bf16 inputs, 64-token chunks, d_k and d_v
+// in {64, 128}, and rows of the per-chunk copies within a tensor map's
+// signed 32-bit coordinates.  The forward's state pass stays the fp32 SIMT
+// pass on every path: with bf16 operands in the state (the two-pass
+// forward's chain, tried) dlog_alpha missed the 1e-2 bar under strong gates
+// (1.9e-2 for the undivided logsigmoid gate), where its reverse sum of
+// differences amplifies the state's rounding.
 bool tensor_chain(const ChunkArgs& f) {
-  return tensor_state_pass(f) &&
+  return fused_supported(f) && max_chunks(f) > 0 &&
          max_chunks(f) * f.H * (f.dk > f.dv ? f.dk : f.dv) < ((int64_t)1 << 31);
 }
 
@@ -130,7 +127,6 @@ BwdWs carve_bwd(const BwdArgs& a, void* base, size_t* total) {
   w.fin = take(4 * (size_t)f.n_seqs * H * dk * dv);
   const ChunkArgs fa = forward_args(a, nullptr);
   w.staged = take(staged_workspace_bytes(fa));
-  w.tp = tensor_state_pass(fa) ? take(twopass_workspace_bytes(fa)) : nullptr;
   w.wt = tensor_chain(fa)
              ? take(4 * (size_t)max_chunks(fa) * f.H * f.dk * f.chunk)
              : nullptr;
@@ -414,13 +410,14 @@ __global__ void __launch_bounds__(kThreads, 2)  // two CTAs per SM
 
 // prep on the tensor cores, for bf16 inputs in 64-token chunks (the
 // tensor-core backward): the same outputs as prep_kernel in that mode, with
-// its three products as tcgen05 kind::tf32 MMAs on 128-byte-swizzled
+// its four products as tcgen05 kind::tf32 MMAs on 128-byte-swizzled
 // K-major fp32 panels: M = Kt Kb^T and P = Qt Kb^T (M = 64 shape, K = d_k),
-// then W = T' Kt (K = the 64 tokens, Kt transposed in shared memory).  The
-// inverse stays the SIMT recursive doubling.  W goes out only as W^T per
-// chunk.  Shared memory: the Kt panels, then one region that holds the Qt
-// and Kb panels, later the inverse's tiles, then T' and Kt^T, then dO for
-// its transposed copy.
+// then W = T' Kt and U = T' V (K = the 64 tokens, Kt and V transposed in
+// shared memory).  The inverse stays the SIMT recursive doubling.  W goes
+// out row-major (for the state pass) and as W^T per chunk.  Shared memory:
+// the Kt panels, then one region that holds the Qt and Kb panels, later the
+// inverse's tiles, then T' and Kt^T, then V^T, then dO for its transposed
+// copy.
 template <int DK>
 struct PrepTcLayout {
   static constexpr uint32_t kt = 0;                   // DK / 32 panels, 8 KB
@@ -484,7 +481,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(tslot, 128);
+    tmem_alloc(tslot, 256);
     tmem_relinquish();
   }
   for (int r = tid; r < C; r += kThreads)
@@ -513,6 +510,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       w.kb[gi] = kb;
       w.qt[gi] = qt;
       w.bkt[gi] = bs[r] * kt;
+      w.fv.kh[gi] = kv * __expf(gl[c] - gv);
     }
     *pel(KT, r, c) = kt;
     *pel(KB, r, c) = kb;
@@ -625,7 +623,31 @@ __global__ void __launch_bounds__(kThreads, 2)
     tc_fence_after();
   }
   if (ok) {
-    // ---- W^T out: thread row r holds W[r][columns], zero past L
+    // ---- V^T as the K-major B panels of U = T' V (Kt^T is read), then U
+    uint8_t* VT = sm + Lay::r2;
+    for (int idx = tid; idx < C * dv; idx += kThreads) {
+      const int s = idx / dv, j = idx % dv;
+      *reinterpret_cast<float*>(VT + (s >> 5) * (dv * 128) + swz32(j, s & 31)) =
+          s < L ? to_f32(v[((size_t)(tok0 + s) * H + h) * dv + j]) : 0.f;
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t id = idesc_tf32(64, dv);
+#pragma unroll
+      for (int ks = 0; ks < C / 8; ++ks)
+        mma_tf32(tmem + DK,
+                 desc_sw128(smem_u32(TP) + (ks >> 2) * 8192 + (ks & 3) * 32,
+                            16, 1024),
+                 desc_sw128(smem_u32(VT) + (ks >> 2) * (dv * 128) +
+                                (ks & 3) * 32,
+                            16, 1024),
+                 id, ks > 0);
+      mma_commit(bar);
+    }
+    // ---- W out, row-major and as W^T: thread row r holds W[r][columns]
     const int qd = warp & 3, half = warp >> 2, r = 16 * qd + lane;
     const size_t tb = ((size_t)cid * H + h) * DK * C;
 #pragma unroll
@@ -637,6 +659,33 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
         for (int u = 0; u < 32; ++u)
           w.wt[tb + (size_t)(j0 + u) * C + r] = r < L ? wv[u] : 0.f;
+        if (r < L) {
+          float4* wr = reinterpret_cast<float4*>(
+              w.fv.w + ((size_t)(tok0 + r) * H + h) * DK + j0);
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            wr[u] = make_float4(wv[4 * u], wv[4 * u + 1], wv[4 * u + 2],
+                                wv[4 * u + 3]);
+        }
+      }
+    }
+    ok = __syncthreads_and(mbar_wait(bar, 0, 2000000000ull));
+    tc_fence_after();
+  }
+  if (ok) {
+    const int qd = warp & 3, half = warp >> 2, r = 16 * qd + lane;
+    // ---- U out (row-major, the state pass turns it into Delta)
+    for (int cc = 0; cc < dv / 64; ++cc) {
+      const int j0 = half * (dv / 2) + 32 * cc;
+      float uv[32];
+      tmem_ld32(tmem + ((uint32_t)(32 * qd) << 16) + DK + j0, uv);
+      if (lane < 16 && r < L) {
+        float4* ur = reinterpret_cast<float4*>(
+            w.fv.d + ((size_t)(tok0 + r) * H + h) * dv + j0);
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          ur[u] = make_float4(uv[4 * u], uv[4 * u + 1], uv[4 * u + 2],
+                              uv[4 * u + 3]);
       }
     }
     // ---- dO^T per chunk, staged row-wise (XOR-swizzled) in the region
@@ -657,7 +706,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, 128);
+  if (warp == 0) tmem_dealloc(tmem, 256);
 }
 
 // The reverse chain over one sequence's chunks for one head and one 32-wide
@@ -1537,22 +1586,15 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
     prep_kernel<IO><<<grid, kThreads, smp, stream>>>(
         static_cast<const IO*>(f.q), static_cast<const IO*>(f.k),
         static_cast<const IO*>(f.v), f.beta, static_cast<const IO*>(a.d_out),
-        w.fv.g, w, w.wt ? nullptr : w.fv.w,
-        tensor_state_pass(f) ? nullptr : w.fv.d,
-        tensor_state_pass(f) ? nullptr : w.fv.kh, w.wt, cu, co, f.n_seqs, f.T,
-        H, dk, dv, C);
+        w.fv.g, w, w.fv.w, w.fv.d, w.fv.kh, w.wt, cu, co, f.n_seqs, f.T, H, dk,
+        dv, C);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  // the forward's serial state pass: chunk-start states, Delta over U, and
-  // the final state; with bf16 inputs in 64-token chunks the tensor-core
-  // two-pass forward, which writes the states and Delta in fp32 from its
-  // accumulators and no outputs
-  e = tensor_state_pass(f)
-          ? launch_twopass_save(f, w.tp, const_cast<float*>(w.fv.s), w.fv.d,
-                                stream)
-          : launch_staged_part(f, w.staged, &w.fv, true, stream);
-  if (e != cudaSuccess) return e;
+  // the forward's serial state pass (fp32): chunk-start states, Delta over
+  // U, and the final state
+  if ((e = launch_staged_part(f, w.staged, &w.fv, true, stream)) != cudaSuccess)
+    return e;
 
   auto tok = [](float* p, int cols, int t = 0) { return MatRef{p, kTok, cols, t}; };
   // token rows contracted over the tokens: the transposed per-chunk copy on
@@ -1724,13 +1766,10 @@ int bwd_kernel_count(const BwdArgs& a) {
   const ChunkArgs f = forward_args(a, nullptr);
   if (f.n_seqs == 0 || f.H == 0) return 0;
   const bool any = max_chunks(f) > 0;
-  // the plan (packed layout), the forward's state pass (one SIMT kernel, or
-  // the two-pass forward's launches) and the reverse chain always; with any
-  // chunk also the cumulative log-decay, prep, the batched products and the
-  // final combination
-  const int state = tensor_state_pass(f) ? twopass_kernel_count(f) : 1;
-  return (f.cu_seqlens ? 1 : 0) + state + 1 +
-         (any ? 1 + 1 + kBmmOps + 1 : 0);
+  // the plan (packed layout), the forward's state pass and the reverse chain
+  // always; with any chunk also the cumulative log-decay, prep, the batched
+  // products and the final combination
+  return (f.cu_seqlens ? 1 : 0) + 2 + (any ? 1 + 1 + kBmmOps + 1 : 0);
 }
 
 cudaError_t launch_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {

@@ -199,13 +199,6 @@ cudaError_t launch_twopass(const ChunkArgs& a, void* workspace,
   return twopass::launch(a, workspace, stream, nullptr, factor_done);
 }
 
-cudaError_t launch_twopass_save(const ChunkArgs& a, void* workspace,
-                                float* save_s, float* save_delta,
-                                cudaStream_t stream) {
-  return twopass::launch(a, workspace, stream, nullptr, nullptr, save_s,
-                         save_delta);
-}
-
 cudaError_t launch_twopass_chain(const ChunkArgs& a, void* workspace,
                                  const void* packages, cudaStream_t stream) {
   return twopass::launch(a, workspace, stream,

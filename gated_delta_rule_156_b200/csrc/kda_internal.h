@@ -188,14 +188,6 @@ size_t twopass_chain_workspace_bytes(const ChunkArgs& a);
 int twopass_chain_kernel_count(const ChunkArgs& a);
 cudaError_t launch_twopass_chain(const ChunkArgs& a, void* workspace,
                                  const void* packages, cudaStream_t stream);
-// The two-pass forward for the backward pass: a.out may be null (no outputs
-// written); every chunk-start state goes to save_s [max_chunks, H, dk, dv]
-// and Delta = U - W S_0 to save_delta [tokens, H, dv], both fp32, in the
-// chunk numbering of the packed layout's offsets (the dense layout: sequence
-// s, chunk c -> s * ceil(T / C) + c).
-cudaError_t launch_twopass_save(const ChunkArgs& a, void* workspace,
-                                float* save_s, float* save_delta,
-                                cudaStream_t stream);
 // Where the package of chunk `first_chunk` (of a's layout) starts in a
 // two-pass workspace.
 const void* twopass_packages(const ChunkArgs& a, const void* workspace,

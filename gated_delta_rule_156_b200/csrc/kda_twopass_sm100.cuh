@@ -95,11 +95,6 @@ struct TwoPassParams {
   int n_seqs, T, H, dv;
   int n_items;        // (chunk, head) factorisations: max_chunks * H
   int items_per_cta;  // consecutive items one factorisation CTA takes
-  // optional, for the backward pass: every chunk-start state
-  // [max_chunks, H, DK, dv] and Delta = U - W S_0 [tokens, H, dv], fp32; out
-  // may then be null (no outputs written)
-  float* save_s;
-  float* save_delta;
 };
 
 template <int DK>
@@ -478,14 +473,6 @@ __global__ void __launch_bounds__(kChainThreads, 1)
     }
     tmem_st32(tmem + lane_base + Lay::t_s + 32 * half, v);
     st_chunks<4>(sop, row, 4 * half, v);
-    if (p.save_s && nch > 0) {  // chunk 0's start state
-      float4* dst = reinterpret_cast<float4*>(
-          p.save_s + (((size_t)cid0 * p.H + h) * DK + row) * p.dv + j0 +
-          32 * half);
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-    }
     tmem_wait_st();
   }
   tc_fence_before();
@@ -557,15 +544,6 @@ __global__ void __launch_bounds__(kChainThreads, 1)
 #pragma unroll
       for (int i = 0; i < 32; ++i) uu[i] -= wsv[i];
       st_chunks<4>(dop, row, 4 * half, uu);
-      if (p.save_delta && row < L) {
-        float4* dst = reinterpret_cast<float4*>(
-            p.save_delta + ((size_t)(tok0 + row) * p.H + h) * p.dv + j0 +
-            32 * half);
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          dst[i] = make_float4(uu[4 * i], uu[4 * i + 1], uu[4 * i + 2],
-                               uu[4 * i + 3]);
-      }
     }
     const float gamma = owns_state ? gc[row] : 1.f;
     if (owns_state && gc[2 * DK] != 0.f) {
@@ -620,14 +598,6 @@ __global__ void __launch_bounds__(kChainThreads, 1)
       for (int i = 0; i < 32; ++i) v[i] *= gamma;
       st_chunks<4>(sop, row, 4 * half, v);
       tmem_st32(tmem + lane_base + Lay::t_s + 32 * half, v);
-      if (p.save_s && n + 1 < nch) {  // the next chunk's start state
-        float4* dst = reinterpret_cast<float4*>(
-            p.save_s + (((size_t)(cid0 + n + 1) * p.H + h) * DK + row) * p.dv +
-            j0 + 32 * half);
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-      }
     }
     fence_proxy_async();
     tc_fence_before();
@@ -640,7 +610,7 @@ __global__ void __launch_bounds__(kChainThreads, 1)
       const int rr = row - 64;
       float o[32];
       tmem_ld32(tmem + lane_base + d3 + 32 * half, o);
-      if (rr < L && p.out) {
+      if (rr < L) {
         uint4* dst = reinterpret_cast<uint4*>(
             p.out + ((size_t)(tok0 + rr) * p.H + h) * p.dv + j0 + 32 * half);
 #pragma unroll
@@ -723,8 +693,7 @@ inline uint8_t* packages_in(const ChunkArgs& a, void* workspace) {
 // head h, at packages + (c * H + h) * slot.
 template <int DK, int GATE>
 cudaError_t run(const ChunkArgs& a, void* workspace, cudaStream_t stream,
-                const uint8_t* packages, cudaEvent_t factor_done,
-                float* save_s, float* save_delta) {
+                const uint8_t* packages, cudaEvent_t factor_done) {
   const int tokens = a.cu_seqlens ? a.T : a.n_seqs * a.T;
   CUtensorMap tq, tk, tv;
   if (!make_tile_map(&tv, a.v, a.dv, a.H, tokens)) return cudaErrorInvalidValue;
@@ -743,8 +712,6 @@ cudaError_t run(const ChunkArgs& a, void* workspace, cudaStream_t stream,
   p.T = a.T;
   p.H = a.H;
   p.dv = a.dv;
-  p.save_s = save_s;
-  p.save_delta = save_delta;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   cudaError_t e;
   if (a.cu_seqlens) {
@@ -805,17 +772,18 @@ cudaError_t run(const ChunkArgs& a, void* workspace, cudaStream_t stream,
 
 inline cudaError_t launch(const ChunkArgs& a, void* workspace,
                           cudaStream_t stream, const uint8_t* packages = nullptr,
-                          cudaEvent_t factor_done = nullptr,
-                          float* save_s = nullptr, float* save_delta = nullptr) {
-#define KDA_TP_RUN(D, G) \
-  run<D, G>(a, workspace, stream, packages, factor_done, save_s, save_delta)
+                          cudaEvent_t factor_done = nullptr) {
   if (a.gate == kGateHead)
-    return a.dk == 128 ? KDA_TP_RUN(128, kGateHead) : KDA_TP_RUN(64, kGateHead);
+    return a.dk == 128
+               ? run<128, kGateHead>(a, workspace, stream, packages, factor_done)
+               : run<64, kGateHead>(a, workspace, stream, packages, factor_done);
   if (a.gate == kGateNone)
-    return a.dk == 128 ? KDA_TP_RUN(128, kGateNone) : KDA_TP_RUN(64, kGateNone);
-  return a.dk == 128 ? KDA_TP_RUN(128, kGateChannel)
-                     : KDA_TP_RUN(64, kGateChannel);
-#undef KDA_TP_RUN
+    return a.dk == 128
+               ? run<128, kGateNone>(a, workspace, stream, packages, factor_done)
+               : run<64, kGateNone>(a, workspace, stream, packages, factor_done);
+  return a.dk == 128
+             ? run<128, kGateChannel>(a, workspace, stream, packages, factor_done)
+             : run<64, kGateChannel>(a, workspace, stream, packages, factor_done);
 }
 
 }  // namespace twopass

@@ -63,12 +63,13 @@ def test_fake_address_validation_in_a_process_without_gpus():
 def test_backward_plan(lib):
     import torch
     kern, ws = K.chunk_bwd_plan(2, 8192, 32, 128, 128, 64, torch.bfloat16)
-    # cumsum, prep, the state pass (factorisation and chain of the two-pass
-    # forward), 2 + 9 products, the chain, final
-    assert kern == 17 and ws > 0
-    # fp32 inputs keep the one-kernel SIMT state pass
-    kern_f, _ = K.chunk_bwd_plan(2, 8192, 32, 128, 128, 64, torch.float32)
+    # cumsum, prep, the state pass, 2 + 9 products, the chain, final (the
+    # tensor-core kernels replace the SIMT ones one for one)
+    assert kern == 16 and ws > 0
+    kern_f, ws_f = K.chunk_bwd_plan(2, 8192, 32, 128, 128, 64, torch.float32)
     assert kern_f == 16
+    # the tensor-core path keeps W^T and the transposed per-chunk copies too
+    assert ws > ws_f
     kern_p, _ = K.chunk_bwd_plan(1, 300, 2, 64, 64, 32, torch.float32,
                                  packed=True, n_seqs=3)
     assert kern_p == 17

@@ -142,3 +142,29 @@ def test_backward_strong_gate_and_range():
                 d["initial_state"], None, do, dsT, chunk=64)
     assert K.device_status() == KDA_ERR_RANGE
     assert K.device_status() == KDA_OK
+
+
+def test_backward_tensor_core_path_strong_gate_and_range():
+    from oracle import kda_oracle
+    # bf16 inputs in 64-token chunks take the tensor-core backward (the
+    # two-pass state pass, tf32 prep, chain and products): the undivided
+    # logsigmoid gate against the oracle, and the 0.2 gate held for a chunk
+    # reported as out of range
+    d = W.draw((2, 150), 2, 128, 128, io="bf16", n_states=2, device=DEV,
+               seed=23, gate_divisor=1.0)
+    g = torch.Generator(device=DEV).manual_seed(24)
+    do = torch.randn(d["v"].shape, generator=g, device=DEV).bfloat16()
+    dsT = torch.randn(d["initial_state"].shape, generator=g, device=DEV)
+    got = K.chunk_bwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"],
+                      d["initial_state"], None, do, dsT, chunk=64)
+    assert K.device_status() == KDA_OK
+    ref = kda_oracle.recurrent_bwd(*(PY.host64(x) for x in (
+        d["q"], d["k"], d["v"], d["log_alpha"], d["beta"],
+        d["initial_state"], do, dsT)))
+    for name, x, r in zip(("dq", "dk", "dv", "dla", "db", "ds0"), got, ref):
+        PY.check(name, PY.host64(x).reshape(r.shape), r, PY.TOL_BF16)
+    d["log_alpha"][0, 64:128, :, 5] = math.log(0.2)
+    K.chunk_bwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"],
+                d["initial_state"], None, do, dsT, chunk=64)
+    assert K.device_status() == KDA_ERR_RANGE
+    assert K.device_status() == KDA_OK
