@@ -75,6 +75,7 @@ struct BwdWs {
   // transposed per-chunk copies for the tensor-core products (or null):
   // [chunks, H, d, C], zero past each chunk's last token; ddT holds -dDelta^T
   float *qtT, *kbT, *bktT, *doT, *ddT;
+  float* khT;  // Kh^T per chunk [chunks, H, dk, C] for the state pass, tf32
   float *kt, *kb, *qt, *bkt;      // [tokens, H, dk]
   float *v32, *bv, *do32, *dd;    // [tokens, H, dv]
   float *tm, *pp;                 // [chunks, H, C, C]
@@ -138,6 +139,7 @@ BwdWs carve_bwd(const BwdArgs& a, void* base, size_t* total) {
     w.bktT = take(tk);
     w.doT = take(tv);
     w.ddT = take(tv);
+    w.khT = take(tk);
   }
   const size_t tdk = 4 * tokens * H * dk, tdv = 4 * tokens * H * dv;
   const size_t sq = 4 * nch * H * C * C, st = 4 * nch * H * dk * dv;
@@ -510,7 +512,6 @@ __global__ void __launch_bounds__(kThreads, 2)
       w.kb[gi] = kb;
       w.qt[gi] = qt;
       w.bkt[gi] = bs[r] * kt;
-      w.fv.kh[gi] = kv * __expf(gl[c] - gv);
     }
     *pel(KT, r, c) = kt;
     *pel(KB, r, c) = kb;
@@ -549,9 +550,12 @@ __global__ void __launch_bounds__(kThreads, 2)
     const size_t tb = ((size_t)cid * H + h) * DK * C;
     for (int idx = tid; idx < DK * C; idx += kThreads) {
       const int c = idx / C, r = idx % C;
+      const float kb = *pel(KB, r, c);
       w.qtT[tb + idx] = *pel(QT, r, c);
-      w.kbT[tb + idx] = *pel(KB, r, c);
+      w.kbT[tb + idx] = kb;
       w.bktT[tb + idx] = bs[r] * *pel(KT, r, c);
+      // Kh = k exp(g_C - g) = Kb exp(g_C), rounded to the nearest tf32
+      w.khT[tb + idx] = sm100::tf32_rna(kb * __expf(gl[c]));
     }
   }
   bool ok = __syncthreads_and(mbar_wait(bar, 0, 2000000000ull));
@@ -659,13 +663,14 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
         for (int u = 0; u < 32; ++u)
           w.wt[tb + (size_t)(j0 + u) * C + r] = r < L ? wv[u] : 0.f;
-        if (r < L) {
+        if (r < L) {  // rounded to the nearest tf32 for the state pass
           float4* wr = reinterpret_cast<float4*>(
               w.fv.w + ((size_t)(tok0 + r) * H + h) * DK + j0);
 #pragma unroll
           for (int u = 0; u < 8; ++u)
-            wr[u] = make_float4(wv[4 * u], wv[4 * u + 1], wv[4 * u + 2],
-                                wv[4 * u + 3]);
+            wr[u] = make_float4(
+                sm100::tf32_rna(wv[4 * u]), sm100::tf32_rna(wv[4 * u + 1]),
+                sm100::tf32_rna(wv[4 * u + 2]), sm100::tf32_rna(wv[4 * u + 3]));
         }
       }
     }
@@ -1591,10 +1596,31 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  // the forward's serial state pass (fp32): chunk-start states, Delta over
-  // U, and the final state
-  if ((e = launch_staged_part(f, w.staged, &w.fv, true, stream)) != cudaSuccess)
-    return e;
+  // the forward's serial state pass: chunk-start states, Delta over U, and
+  // the final state (fp32 SIMT, or on the tensor cores with fp32-grade
+  // operands: hi + lo tf32 parts of S and Delta)
+  if (w.khT) {
+    StateChainArgs sa{};
+    sa.w = w.fv.w;
+    sa.u = w.fv.d;
+    sa.khT = w.khT;
+    sa.gam = w.gam;
+    sa.s = const_cast<float*>(w.fv.s);
+    sa.s_init = f.initial_state;
+    sa.s_final = w.fin;
+    sa.cu = cu;
+    sa.chunk_off = w.fv.chunk_off;
+    sa.n_seqs = f.n_seqs;
+    sa.T = f.T;
+    sa.H = f.H;
+    sa.dk = f.dk;
+    sa.dv = f.dv;
+    sa.n_chunks = max_chunks(f);
+    e = launch_state_chain_tc(sa, stream);
+  } else {
+    e = launch_staged_part(f, w.staged, &w.fv, true, stream);
+  }
+  if (e != cudaSuccess) return e;
 
   auto tok = [](float* p, int cols, int t = 0) { return MatRef{p, kTok, cols, t}; };
   // token rows contracted over the tokens: the transposed per-chunk copy on

@@ -30,6 +30,7 @@ namespace kda {
 namespace bwdtc {
 
 using sm100::idesc_tf32;
+using sm100::tf32_rna;
 using sm100::tma_load_2d;
 using sm100::mma_tf32;
 using sm100::swz32;
@@ -447,6 +448,372 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int i = 0; i < 8; ++i)
       dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+  }
+  if (c == 0) bulk_wait_all();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 128);
+}
+
+// ---------------------------------------------------------------------------
+// The forward's state pass for the backward, on the tensor cores: per chunk,
+// walking each sequence forward (the chunkwise form "You Could Have Come Up
+// with Kimi Delta Attention", daily.dev, Summary):
+//   Delta = U - W S           (product A: M = 64 tokens, N = 64, K = d_k)
+//   S    <- Diag(gam) S + Kh^T Delta, Kh = k exp(g_C - g)
+//                             (product B: M = d_k, N = 64, K = 64 tokens)
+// storing every chunk-start state, Delta over U, and the final state.  The
+// state's rounding is amplified in dlog_alpha under strong gates (its reverse
+// sum of differences of terms that grow like exp|g|), so this pass keeps
+// fp32-grade operands: S and Delta, formed here, enter their products as a
+// tf32 high part plus the tf32 remainder (two MMAs each), and W and Kh^T
+// arrive from prep already rounded to the nearest tf32.  One CTA of 256
+// threads per (sequence, head, 64-column d_v tile), S in TMEM throughout;
+// W, U and Kh^T by TMA into one buffer each, refilled as soon as it is free;
+// Delta stored by TMA in place of U (thread stores for a ragged last chunk),
+// each chunk-start state by TMA from a staging tile.
+
+struct StateParams {
+  const float* gam;      // exp(g_C) [chunks, H, dk]
+  const float* s_init;   // [n_seqs, H, dk, dv] or null (zero)
+  float* s_final;        // [n_seqs, H, dk, dv]
+  float* dd;             // Delta over U [tokens, H, dv] (ragged chunks' rows)
+  const int32_t* cu;
+  const int32_t* chunk_off;
+  int n_seqs, T, H, dv;
+};
+
+// W and U / Delta over [tokens, H, d] (64-token boxes); Kh^T over
+// [chunks * H * dk, 64] and the chunk-start states over [chunks * H * dk, dv]
+// (d_k-row boxes).
+struct StateMaps {
+  CUtensorMap w, u, kht, s;
+};
+
+template <int DK>
+struct StateLayout {
+  static constexpr uint32_t wb = 0;                          // W + pad panel
+  static constexpr uint32_t ub = wb + (DK / 32 + 1) * 8192;  // U / Delta
+  static constexpr uint32_t kb = ub + 2 * 8192;              // Kh^T, 128 rows
+  static constexpr uint32_t shi = kb + 2 * 16384;            // S, B operand
+  static constexpr uint32_t slo = shi + (DK / 32) * 8192;
+  static constexpr uint32_t dhi = slo + (DK / 32) * 8192;    // Delta, B operand
+  static constexpr uint32_t dlo = dhi + 2 * 8192;
+  static constexpr uint32_t sst = dlo + 2 * 8192;            // S staging
+  static constexpr uint32_t misc = sst + 2 * DK * 128;
+  static constexpr uint32_t bytes = misc + 256;
+  static constexpr uint32_t w_tx = (DK / 32) * 8192;
+  static constexpr uint32_t u_tx = 2 * 8192;
+  static constexpr uint32_t k_tx = 2 * DK * 128;
+  static constexpr uint32_t t_s = 0, t_d = 64;  // TMEM columns
+  static_assert(bytes + 1024 <= 232448, "shared memory");
+};
+
+template <int DK>
+__global__ void __launch_bounds__(kThreads, 1)
+    state_chain_kernel(const __grid_constant__ StateMaps m,
+                       const StateParams p) {
+  using namespace sm100;
+  using Lay = StateLayout<DK>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* wb = sm + Lay::wb;
+  uint8_t* ub = sm + Lay::ub;
+  uint8_t* kb = sm + Lay::kb;
+  uint8_t* shi = sm + Lay::shi;
+  uint8_t* slo = sm + Lay::slo;
+  uint8_t* dhi = sm + Lay::dhi;
+  uint8_t* dlo = sm + Lay::dlo;
+  uint8_t* sst = sm + Lay::sst;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Lay::misc);
+  enum { kW, kU, kK, kNbuf };
+  uint64_t* bar_mma = bars + kNbuf;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNbuf + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + kNbuf + 2);
+
+  const int c = threadIdx.x, warp = c >> 5;
+  const int row = c & 127, half = c >> 7;
+  const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+  const int n_tiles = p.dv / kTile;
+  const int tile = blockIdx.x % n_tiles;
+  const int h = (blockIdx.x / n_tiles) % p.H;
+  const int seq = blockIdx.x / (n_tiles * p.H);
+  const int jt = tile * kTile, j0 = jt + 32 * half;
+  int start, end;
+  seq_range(p.cu, seq, p.T, &start, &end);
+  const int nch = (end - start + kC - 1) / kC;
+  const int cid0 = p.cu ? p.chunk_off[seq] : seq * ((p.T + kC - 1) / kC);
+  const bool owns_state = row < DK;
+  const size_t sbase = ((size_t)seq * p.H + h) * DK * p.dv;
+  auto crow = [&](int n) { return (int)(((size_t)(cid0 + n) * p.H + h) * DK); };
+
+  if (c == 0) {
+    prefetch_tmap(&m.w);
+    prefetch_tmap(&m.u);
+    prefetch_tmap(&m.kht);
+    prefetch_tmap(&m.s);
+    for (int i = 0; i < kNbuf + 1; ++i) mbar_init(bars + i, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  int issued[kNbuf] = {0, 0, 0};
+  auto load_w = [&](int n) {
+    mbar_arrive_expect_tx(bars + kW, Lay::w_tx);
+    for (int q = 0; q < DK / 32; ++q)
+      tma_load_3d(wb + q * 8192, &m.w, bars + kW, 32 * q, h, start + n * kC);
+    ++issued[kW];
+  };
+  auto load_u = [&](int n) {
+    mbar_arrive_expect_tx(bars + kU, Lay::u_tx);
+    for (int q = 0; q < 2; ++q)
+      tma_load_3d(ub + q * 8192, &m.u, bars + kU, jt + 32 * q, h,
+                  start + n * kC);
+    ++issued[kU];
+  };
+  auto load_k = [&](int n) {
+    mbar_arrive_expect_tx(bars + kK, Lay::k_tx);
+    for (int q = 0; q < 2; ++q)
+      tma_load_2d(kb + q * 16384, &m.kht, bars + kK, 32 * q, crow(n));
+    ++issued[kK];
+  };
+  if (c == 0 && nch > 0) {
+    load_w(0);
+    load_u(0);
+    load_k(0);
+  }
+  auto ld_row = [](const uint8_t* panel, int r, float* v) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float4 x = *reinterpret_cast<const float4*>(
+          panel + r * 128 + ((k ^ (r & 7)) << 4));
+      v[4 * k] = x.x; v[4 * k + 1] = x.y; v[4 * k + 2] = x.z;
+      v[4 * k + 3] = x.w;
+    }
+  };
+  auto st_row = [](uint8_t* panel, int r, const float* v) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      *reinterpret_cast<float4*>(panel + r * 128 + ((k ^ (r & 7)) << 4)) =
+          make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+  };
+  // S (this thread's row, 32 columns) into the K-major B panels of product A
+  // as tf32 high part and remainder, and into the staging tile
+  auto put_state = [&](const float* v, bool stage) {
+    uint8_t* ph = shi + (row >> 5) * 8192;
+    uint8_t* pl = slo + (row >> 5) * 8192;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float hi = tf32_rna(v[i]);
+      *reinterpret_cast<float*>(ph + swz32(32 * half + i, row & 31)) = hi;
+      *reinterpret_cast<float*>(pl + swz32(32 * half + i, row & 31)) =
+          v[i] - hi;
+    }
+    if (stage) st_row(sst + half * DK * 128, row, v);
+  };
+
+  // ---- the start state
+  if (owns_state) {
+    float v[32];
+    if (p.s_init) {
+      const float4* src = reinterpret_cast<const float4*>(
+          p.s_init + sbase + (size_t)row * p.dv + j0);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float4 x = src[i];
+        v[4 * i] = x.x; v[4 * i + 1] = x.y; v[4 * i + 2] = x.z;
+        v[4 * i + 3] = x.w;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = 0.f;
+    }
+    tmem_st32(tmem + lane_base + Lay::t_s + 32 * half, v);
+    put_state(v, nch > 0);
+    if (nch == 0) {  // an empty sequence: the final state is the start state
+      float4* dst = reinterpret_cast<float4*>(p.s_final + sbase +
+                                              (size_t)row * p.dv + j0);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    }
+    tmem_wait_st();
+  }
+  fence_proxy_async();
+  tc_fence_before();
+  __syncthreads();
+  if (c == 0 && nch > 0) {
+    tc_fence_after();
+    for (int q = 0; q < 2; ++q)
+      tma_store_2d(&m.s, sst + q * DK * 128, jt + 32 * q, crow(0));
+    bulk_commit();
+  }
+
+  uint32_t ph_mma = 0;
+  bool failed = false;
+  int n = 0;
+  for (; n < nch; ++n) {
+    const int cid = cid0 + n, tok0 = start + n * kC;
+    const int L = min(kC, end - tok0);
+    const uint32_t par = (uint32_t)n & 1u;
+    bool ok = true;
+
+    // ---- product A: D = W S (rows 0-63 meaningful)
+    if (c == 0) {
+      tc_fence_after();
+      ok = wait_or_abort<false>(bars + kW, par, abort_flag);
+      if (ok) {
+        constexpr uint32_t id = idesc_tf32(128, kTile);
+#pragma unroll
+        for (int ks = 0; ks < DK / 8; ++ks) {
+          const uint32_t o = (ks >> 2) * 8192 + (ks & 3) * 32;
+          const uint64_t ad = desc_sw128(smem_u32(wb) + o, 16, 1024);
+          mma_tf32(tmem + Lay::t_d, ad, desc_sw128(smem_u32(shi) + o, 16, 1024),
+                   id, ks > 0);
+          mma_tf32(tmem + Lay::t_d, ad, desc_sw128(smem_u32(slo) + o, 16, 1024),
+                   id, 1u);
+        }
+        mma_commit(bar_mma);
+      } else {
+        *abort_flag = 1;
+      }
+    }
+    const float gmv =
+        owns_state ? p.gam[((size_t)cid * p.H + h) * DK + row] : 0.f;
+    ok = ok && wait_or_abort<false>(bar_mma, ph_mma, abort_flag);
+    ph_mma ^= 1;
+    if (named_sync_or(kBarAll, kThreads, !ok)) {
+      failed = true;
+      break;
+    }
+    tc_fence_after();
+    if (c == 0 && n + 1 < nch) load_w(n + 1);
+
+    // ---- Delta = U - W S (token rows; zero past the chunk); S <- gam S
+    if (row < kC) {
+      ok = wait_or_abort<false>(bars + kU, par, abort_flag);
+      if (ok) {
+        float d[32], u[32];
+        const bool in = row < L;
+        uint8_t* up = ub + half * 8192;
+        ld_row(up, row, u);
+        tmem_ld32(tmem + lane_base + Lay::t_d + 32 * half, d);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) d[i] = in ? u[i] - d[i] : 0.f;
+        if (L < kC && in) {  // a ragged chunk: no box store past it
+          float4* d4 = reinterpret_cast<float4*>(
+              p.dd + ((size_t)(tok0 + row) * p.H + h) * p.dv + j0);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            d4[i] =
+                make_float4(d[4 * i], d[4 * i + 1], d[4 * i + 2], d[4 * i + 3]);
+        }
+        st_row(up, row, d);
+        uint8_t* ph = dhi + (row >> 5) * 8192;
+        uint8_t* pl = dlo + (row >> 5) * 8192;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float hi = tf32_rna(d[i]);
+          *reinterpret_cast<float*>(ph + swz32(32 * half + i, row & 31)) = hi;
+          *reinterpret_cast<float*>(pl + swz32(32 * half + i, row & 31)) =
+              d[i] - hi;
+        }
+      } else {
+        *abort_flag = 1;
+      }
+    }
+    if (owns_state) {
+      float v[32];
+      tmem_ld32(tmem + lane_base + Lay::t_s + 32 * half, v);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] *= gmv;
+      tmem_st32(tmem + lane_base + Lay::t_s + 32 * half, v);
+      tmem_wait_st();
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    if (named_sync_or(kBarAll, kThreads, !ok)) {
+      failed = true;
+      break;
+    }
+
+    // ---- product B: S += Kh^T Delta; Delta out; next U
+    if (c == 0) {
+      tc_fence_after();
+      if (L == kC) {
+        for (int q = 0; q < 2; ++q)
+          tma_store_3d(&m.u, ub + q * 8192, jt + 32 * q, h, tok0);
+        bulk_commit();
+      }
+      ok = wait_or_abort<false>(bars + kK, par, abort_flag);
+      if (ok) {
+        constexpr uint32_t id = idesc_tf32(128, kTile);
+#pragma unroll
+        for (int ks = 0; ks < kC / 8; ++ks) {
+          const uint64_t ad = desc_sw128(
+              smem_u32(kb) + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+          const uint32_t o = (ks >> 2) * 8192 + (ks & 3) * 32;
+          mma_tf32(tmem + Lay::t_s, ad, desc_sw128(smem_u32(dhi) + o, 16, 1024),
+                   id, 1u);
+          mma_tf32(tmem + Lay::t_s, ad, desc_sw128(smem_u32(dlo) + o, 16, 1024),
+                   id, 1u);
+        }
+        mma_commit(bar_mma);
+        bulk_wait_read();  // Delta and the last state have left shared memory
+        if (n + 1 < nch) load_u(n + 1);
+      } else {
+        *abort_flag = 1;
+      }
+    }
+    ok = ok && wait_or_abort<false>(bar_mma, ph_mma, abort_flag);
+    ph_mma ^= 1;
+    if (named_sync_or(kBarAll, kThreads, !ok)) {
+      failed = true;
+      break;
+    }
+    tc_fence_after();
+    if (c == 0 && n + 1 < nch) load_k(n + 1);
+
+    // ---- the next chunk's start state (or the final state)
+    if (owns_state) {
+      float v[32];
+      tmem_ld32(tmem + lane_base + Lay::t_s + 32 * half, v);
+      if (n + 1 < nch) {
+        put_state(v, true);
+      } else {
+        float4* dst = reinterpret_cast<float4*>(p.s_final + sbase +
+                                                (size_t)row * p.dv + j0);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          dst[i] =
+              make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+      }
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    if (c == 0 && n + 1 < nch) {
+      tc_fence_after();
+      for (int q = 0; q < 2; ++q)
+        tma_store_2d(&m.s, sst + q * DK * 128, jt + 32 * q, crow(n + 1));
+      bulk_commit();
+    }
+  }
+  if (failed && c == 0) {
+    atomicExch(&g_fused_timeout, 1);
+#pragma unroll
+    for (int b = 0; b < kNbuf; ++b)  // the copy still in flight, if any
+      if (issued[b] > 0)
+        mbar_wait(bars + b, (uint32_t)(issued[b] - 1) & 1u, 100000000ull);
   }
   if (c == 0) bulk_wait_all();
   tc_fence_before();

@@ -270,6 +270,39 @@ cudaError_t run_rev_chain_tc(const RevChainArgs& a, cudaStream_t stream) {
 }
 }  // namespace
 
+template <int DK>
+cudaError_t run_state_chain_tc(const StateChainArgs& a, cudaStream_t stream) {
+  using Lay = bwdtc::StateLayout<DK>;
+  const int tokens = a.cu ? a.T : a.n_seqs * a.T;
+  const int64_t crows = a.n_chunks * a.H * DK;
+  const auto F32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  const auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
+  bwdtc::StateMaps m;
+  if (!make_map(&m.w, a.w, F32, 4, DK, a.H, tokens, 32, SW) ||
+      !make_map(&m.u, a.u, F32, 4, a.dv, a.H, tokens, 32, SW) ||
+      !make_rows_map(&m.kht, a.khT, crows, 64, DK) ||
+      !make_rows_map(&m.s, a.s, crows, a.dv, DK))
+    return cudaErrorInvalidValue;
+  bwdtc::StateParams p{a.gam, a.s_init, a.s_final, a.u, a.cu, a.chunk_off,
+                       a.n_seqs, a.T, a.H, a.dv};
+  const size_t smem = Lay::bytes + 1024;
+  cudaError_t e;
+  if ((e = cudaFuncSetAttribute(bwdtc::state_chain_kernel<DK>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)smem)) != cudaSuccess)
+    return e;
+  const unsigned grid = (unsigned)a.n_seqs * a.H * (a.dv / bwdtc::kTile);
+  bwdtc::state_chain_kernel<DK><<<grid, bwdtc::kThreads, smem, stream>>>(m, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_state_chain_tc(const StateChainArgs& a,
+                                  cudaStream_t stream) {
+  if (a.dk == 128) return run_state_chain_tc<128>(a, stream);
+  if (a.dk == 64) return run_state_chain_tc<64>(a, stream);
+  return cudaErrorInvalidValue;
+}
+
 cudaError_t launch_rev_chain_tc(const RevChainArgs& a, cudaStream_t stream) {
   if (a.dk == 128) return run_rev_chain_tc<128>(a, stream);
   if (a.dk == 64) return run_rev_chain_tc<64>(a, stream);

@@ -129,6 +129,25 @@ struct RevChainArgs {
 };
 cudaError_t launch_rev_chain_tc(const RevChainArgs& a, cudaStream_t stream);
 
+// The backward pass's copy of the forward's state pass on the tensor cores
+// (kda_bwd_chain_tc.cuh): Delta = U - W S over u in place, every chunk-start
+// state into s, the final state into s_final; W and Kh^T rounded to tf32 by
+// prep, S and Delta split into tf32 high part and remainder.
+struct StateChainArgs {
+  const float* w;        // W [tokens, H, dk]
+  float* u;              // U in, Delta out [tokens, H, dv]
+  const float* khT;      // Kh^T per chunk [chunks, H, dk, 64]
+  const float* gam;      // exp(g_C) [chunks, H, dk]
+  float* s;              // chunk-start states [chunks, H, dk, dv]
+  const float* s_init;   // [n_seqs, H, dk, dv] or null
+  float* s_final;        // [n_seqs, H, dk, dv]
+  const int32_t* cu;
+  const int32_t* chunk_off;
+  int n_seqs, T, H, dk, dv;
+  int64_t n_chunks;
+};
+cudaError_t launch_state_chain_tc(const StateChainArgs& a, cudaStream_t stream);
+
 // Chunkwise backward pass (kda_backward.cu): the gradients of
 // L = <d_out, out> + <d_final_state, final_state> with respect to q, k, v,
 // log(alpha), beta and the initial state, in fp32 arithmetic (with bf16

@@ -227,6 +227,14 @@ __device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t adesc,
       : "memory");
 }
 
+// x rounded to the nearest tf32 (ties away from zero), as an fp32 value:
+// what a kind::tf32 product then reads of it is exact.
+__device__ __forceinline__ float tf32_rna(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
+}
+
 // Byte offset of fp32 element (row, c) inside one 128-byte-swizzled panel
 // whose rows hold 32 fp32 (K-major: rows along M or N, 32 consecutive k per
 // row): 16-byte chunk index XOR (row mod 8).
