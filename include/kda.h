@@ -410,9 +410,9 @@ KDA_API kda_status kda_device_status(cudaStream_t stream);
  * aligned (KDA_ERR_MISALIGNED otherwise).  No output may overlap an input or
  * another output (KDA_ERR_INVALID_ARG).  All arithmetic is fp32 except for
  * bf16 inputs with chunk 64 (d_k, d_v in {64, 128}): there every product
- * but the forward's state pass runs on the tensor cores in tf32 (10-bit
- * mantissa, fp32 accumulation), within the bf16 tolerance of 1e-2 relative
- * L2 (a bounded wait that gives up is reported by kda_device_status as
+ * runs on the tensor cores in tf32 (10-bit mantissa, fp32 accumulation; the
+ * forward's state pass with high and low tf32 parts of its state and Delta),
+ * within the bf16 tolerance of 1e-2 relative L2 (a bounded wait that gives up is reported by kda_device_status as
  * KDA_ERR_TIMEOUT); the call
  * re-runs the forward's chunk stages and allocates its fp32 workspace from
  * the stream-ordered pool (kda_chunk_bwd_plan reports its size).  Stream
