@@ -1,7 +1,8 @@
 // Chunkwise backward pass of the KDA forward, in fp32 SIMT arithmetic except
-// with bf16 inputs in 64-token chunks: there the forward's state pass is the
-// tensor-core two-pass forward (bf16 operands, fp32 accumulators) and the
-// reverse chain runs on the tensor cores in tf32 (kda_bwd_chain_tc.cuh).
+// with bf16 inputs in 64-token chunks: there every product runs on the
+// tensor cores in tf32 (prep and the batched products here, the forward's
+// state pass and the reverse chain in kda_bwd_chain_tc.cuh; the state pass
+// with high and low tf32 parts of its state and Delta).
 //
 // The gradients of L = <dO, O> + <dS_T, S_T> follow from the chain rule
 // applied to each line of the chunkwise forward (the forward's own chunk
@@ -33,8 +34,7 @@
 //   - a prep kernel per (chunk, head): Kt, Kb, Qt, b Kt, P and Tm, plus the
 //     forward's own W, U and Kh, so the forward's stage (2) is not run;
 //   - the forward's state pass: Delta and every chunk-start state (stage 3
-//     of the four-stage forward, or the two-pass forward with its outputs
-//     switched off);
+//     of the four-stage forward, or its tensor-core form);
 //   - the two products that do not depend on dS, Qt^T dO and P^T dO;
 //   - the reverse chain per (sequence, head, 32-column d_v tile; 64 columns
 //     on the tensor cores), which
@@ -98,14 +98,14 @@ ChunkArgs forward_args(const BwdArgs& a, float* fin) {
   return f;
 }
 
-// The tensor-core path (prep, the reverse chain and the batched products in
-// tf32) where the shape allows it: bf16 inputs, 64-token chunks, d_k and d_v
-// in {64, 128}, and rows of the per-chunk copies within a tensor map's
-// signed 32-bit coordinates.  The forward's state pass stays the fp32 SIMT
-// pass on every path: with bf16 operands in the state (the two-pass
-// forward's chain, tried) dlog_alpha missed the 1e-2 bar under strong gates
-// (1.9e-2 for the undivided logsigmoid gate), where its reverse sum of
-// differences amplifies the state's rounding.
+// The tensor-core path (every product in tf32) where the shape allows it:
+// bf16 inputs, 64-token chunks, d_k and d_v in {64, 128}, and rows of the
+// per-chunk copies within a tensor map's signed 32-bit coordinates.  The
+// state pass there keeps fp32-grade operands (high and low tf32 parts):
+// with bf16 operands in the state (the two-pass forward's chain, tried)
+// dlog_alpha missed the 1e-2 bar under strong gates (1.9e-2 for the
+// undivided logsigmoid gate), where its reverse sum of differences amplifies
+// the state's rounding.
 bool tensor_chain(const ChunkArgs& f) {
   return fused_supported(f) && max_chunks(f) > 0 &&
          max_chunks(f) * f.H * (f.dk > f.dv ? f.dk : f.dv) < ((int64_t)1 << 31);

@@ -151,8 +151,7 @@ cudaError_t launch_state_chain_tc(const StateChainArgs& a, cudaStream_t stream);
 // Chunkwise backward pass (kda_backward.cu): the gradients of
 // L = <d_out, out> + <d_final_state, final_state> with respect to q, k, v,
 // log(alpha), beta and the initial state, in fp32 arithmetic (with bf16
-// inputs in 64-token chunks the forward's state pass and the reverse chain
-// run on the tensor cores).
+// inputs in 64-token chunks every product runs on the tensor cores in tf32).
 struct BwdArgs {
   ChunkArgs f;                  // forward arguments; f.out, f.final_state unused
   const void* d_out;            // [tokens, H, dv], io dtype
