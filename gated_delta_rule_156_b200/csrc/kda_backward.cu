@@ -497,33 +497,58 @@ __global__ void __launch_bounds__(kThreads, 2)
   tc_fence_after();
   const uint32_t tmem = *tslot;
 
-  // ---- Kt, Kb, Qt: the workspace rows and the operand panels
-  for (int idx = tid; idx < C * DK; idx += kThreads) {
-    const int r = idx / DK, c = idx % DK;
-    float kt = 0.f, kb = 0.f, qt = 0.f;
+  // ---- Kt, Kb, Qt: the workspace rows and the operand panels, four
+  // channels per thread and step (8-byte bf16 and 16-byte fp32 accesses)
+  auto ld_bf4 = [](const __nv_bfloat16* p, float* x) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
+    const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
+    x[0] = __low2float(a); x[1] = __high2float(a);
+    x[2] = __low2float(b); x[3] = __high2float(b);
+  };
+  auto st4 = [](float* p, const float* x) {
+    *reinterpret_cast<float4*>(p) = make_float4(x[0], x[1], x[2], x[3]);
+  };
+  for (int idx = tid; idx < C * DK / 4; idx += kThreads) {
+    const int r = idx / (DK / 4), c = (idx % (DK / 4)) * 4;
+    float kt[4] = {0.f, 0.f, 0.f, 0.f}, kb[4] = {0.f, 0.f, 0.f, 0.f},
+          qt[4] = {0.f, 0.f, 0.f, 0.f};
     if (r < L) {
       const size_t gi = ((size_t)(tok0 + r) * H + h) * DK + c;
-      const float kv = to_f32(k[gi]), qv = to_f32(q[gi]), gv = g[gi];
-      const float e = __expf(gv), ie = __expf(-gv);
-      kt = kv * e;
-      kb = kv * ie;
-      qt = qv * e;
-      w.kt[gi] = kt;
-      w.kb[gi] = kb;
-      w.qt[gi] = qt;
-      w.bkt[gi] = bs[r] * kt;
+      float kv[4], qv[4];
+      ld_bf4(k + gi, kv);
+      ld_bf4(q + gi, qv);
+      const float4 g4 = *reinterpret_cast<const float4*>(g + gi);
+      const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
+      float bk[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float e = __expf(gv[u]), ie = __expf(-gv[u]);
+        kt[u] = kv[u] * e;
+        kb[u] = kv[u] * ie;
+        qt[u] = qv[u] * e;
+        bk[u] = bs[r] * kt[u];
+      }
+      st4(w.kt + gi, kt);
+      st4(w.kb + gi, kb);
+      st4(w.qt + gi, qt);
+      st4(w.bkt + gi, bk);
     }
-    *pel(KT, r, c) = kt;
-    *pel(KB, r, c) = kb;
-    *pel(QT, r, c) = qt;
+    st4(pel(KT, r, c), kt);
+    st4(pel(KB, r, c), kb);
+    st4(pel(QT, r, c), qt);
   }
-  for (int idx = tid; idx < L * dv; idx += kThreads) {
-    const int r = idx / dv;
-    const size_t gi = ((size_t)(tok0 + r) * H + h) * dv + idx % dv;
-    const float vv = to_f32(v[gi]);
-    w.v32[gi] = vv;
-    w.bv[gi] = bs[r] * vv;
-    w.do32[gi] = to_f32(dout[gi]);
+  for (int idx = tid; idx < L * dv / 4; idx += kThreads) {
+    const int r = idx / (dv / 4);
+    const size_t gi = ((size_t)(tok0 + r) * H + h) * dv + (idx % (dv / 4)) * 4;
+    float vv[4], dd[4], bvv[4];
+    ld_bf4(v + gi, vv);
+    ld_bf4(dout + gi, dd);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) bvv[u] = bs[r] * vv[u];
+    st4(w.v32 + gi, vv);
+    st4(w.bv + gi, bvv);
+    st4(w.do32 + gi, dd);
   }
   for (int c = tid; c < DK; c += kThreads)
     w.gam[((size_t)cid * H + h) * DK + c] = __expf(gl[c]);
