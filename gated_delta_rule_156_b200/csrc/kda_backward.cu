@@ -654,10 +654,14 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (ok) {
     // ---- V^T as the K-major B panels of U = T' V (Kt^T is read), then U
     uint8_t* VT = sm + Lay::r2;
-    for (int idx = tid; idx < C * dv; idx += kThreads) {
-      const int s = idx / dv, j = idx % dv;
-      *reinterpret_cast<float*>(VT + (s >> 5) * (dv * 128) + swz32(j, s & 31)) =
-          s < L ? to_f32(v[((size_t)(tok0 + s) * H + h) * dv + j]) : 0.f;
+    for (int idx = tid; idx < C * dv / 4; idx += kThreads) {
+      const int s = idx / (dv / 4), j = (idx % (dv / 4)) * 4;
+      float x[4] = {0.f, 0.f, 0.f, 0.f};
+      if (s < L) ld_bf4(v + ((size_t)(tok0 + s) * H + h) * dv + j, x);
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        *reinterpret_cast<float*>(VT + (s >> 5) * (dv * 128) +
+                                  swz32(j + u, s & 31)) = x[u];
     }
     fence_proxy_async();
     tc_fence_before();
@@ -720,10 +724,12 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     // ---- dO^T per chunk, staged row-wise (XOR-swizzled) in the region
     float* Ds = reinterpret_cast<float*>(sm + Lay::r2);
-    for (int idx = tid; idx < C * dv; idx += kThreads) {
-      const int rr = idx / dv, c = idx % dv;
-      Ds[rr * dv + (c ^ (rr & 31))] =
-          rr < L ? to_f32(dout[((size_t)(tok0 + rr) * H + h) * dv + c]) : 0.f;
+    for (int idx = tid; idx < C * dv / 4; idx += kThreads) {
+      const int rr = idx / (dv / 4), c = (idx % (dv / 4)) * 4;
+      float x[4] = {0.f, 0.f, 0.f, 0.f};
+      if (rr < L) ld_bf4(dout + ((size_t)(tok0 + rr) * H + h) * dv + c, x);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) Ds[rr * dv + ((c + u) ^ (rr & 31))] = x[u];
     }
     __syncthreads();
     const size_t tv = ((size_t)cid * H + h) * dv * C;
