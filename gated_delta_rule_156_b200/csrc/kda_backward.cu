@@ -1335,7 +1335,7 @@ struct BmmMaps {
 // past the chunk are other tokens (or zero past the tensor): they only
 // reach output rows or columns past m or n, which are not stored.
 template <int MD, int ND>
-__global__ void __launch_bounds__(kThreads, MD == 64 ? 2 : 1)
+__global__ void __launch_bounds__(kThreads, MD == 64 ? 3 : 1)
     bmm_tc_kernel(BmmOp op, const __grid_constant__ BmmMaps maps,
                   int tma_mask, const int32_t* cu, const int32_t* chunk_off,
                   int n_seqs, int T, int H, int dk, int dv, int C) {
@@ -1348,9 +1348,14 @@ __global__ void __launch_bounds__(kThreads, MD == 64 ? 2 : 1)
   uint8_t* sm = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   constexpr int kPanA = MD * 128, kPanB = ND * 128;
-  uint8_t* As = sm;                 // up to four panels
-  uint8_t* Bs = sm + 4 * kPanA;     // up to four panels
-  uint64_t* bar = reinterpret_cast<uint64_t*>(Bs + 4 * kPanB);
+  // panels per operand: the longest contraction of the op's terms / 32
+  int npan = 1;
+  for (int t = 0; t < op.nterms; ++t)
+    npan = max(npan, (t == 0 ? op.term[0].kd : t == 1 ? op.term[1].kd
+                                                       : op.term[2].kd) / 32);
+  uint8_t* As = sm;                  // npan panels
+  uint8_t* Bs = sm + npan * kPanA;   // npan panels
+  uint64_t* bar = reinterpret_cast<uint64_t*>(Bs + npan * kPanB);
   uint64_t* tbar = bar + 1;  // TMA operand copies
   uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 2);
   if (tid == 0) {
@@ -1485,7 +1490,12 @@ cudaError_t launch_bmm_tc_t(const BmmOp& op, const BmmMaps& maps, int mask,
                             dim3 grid, cudaStream_t stream, const int32_t* cu,
                             const int32_t* co, int n_seqs, int T, int H,
                             int dk, int dv, int C) {
-  const size_t smem = 4 * (size_t)(MD + ND) * 128 + 1024 + 64;
+  // shared memory for the longest contraction of the op's terms: ops that
+  // contract over 64 only fit twice as many CTAs on an SM
+  int kdmax = 32;
+  for (int t = 0; t < op.nterms; ++t)
+    kdmax = op.term[t].kd > kdmax ? op.term[t].kd : kdmax;
+  const size_t smem = (size_t)(kdmax / 32) * (MD + ND) * 128 + 1024 + 64;
   cudaError_t e = set_smem(bmm_tc_kernel<MD, ND>, smem);
   if (e != cudaSuccess) return e;
   bmm_tc_kernel<MD, ND><<<grid, kThreads, smem, stream>>>(
