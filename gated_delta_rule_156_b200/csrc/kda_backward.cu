@@ -1335,7 +1335,7 @@ struct BmmMaps {
 // past the chunk are other tokens (or zero past the tensor): they only
 // reach output rows or columns past m or n, which are not stored.
 template <int MD, int ND>
-__global__ void __launch_bounds__(kThreads, MD == 64 ? 3 : 1)
+__global__ void __launch_bounds__(kThreads, 3)
     bmm_tc_kernel(BmmOp op, const __grid_constant__ BmmMaps maps,
                   int tma_mask, const int32_t* cu, const int32_t* chunk_off,
                   int n_seqs, int T, int H, int dk, int dv, int C) {
