@@ -37,6 +37,7 @@ def compare(got, ref, tol):
 @pytest.mark.parametrize("io", ["f32", "bf16"])
 @pytest.mark.parametrize("dk,dv,C,T", [(32, 32, 16, 77), (64, 64, 32, 150),
                                        (128, 128, 64, 130), (64, 128, 64, 200),
+                                       (128, 64, 64, 150), (64, 64, 64, 64),
                                        (128, 32, 16, 40)])
 def test_backward_dense(io, dk, dv, C, T):
     d = W.draw((2, T), 2, dk, dv, io=io, n_states=2, device=DEV,
