@@ -529,9 +529,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         qt[u] = qv[u] * e;
         bk[u] = bs[r] * kt[u];
       }
-      st4(w.kt + gi, kt);
-      st4(w.kb + gi, kb);
-      st4(w.qt + gi, qt);
+      st4(w.kb + gi, kb);  // (Kt and Qt rows: the final kernel recomputes them)
       st4(w.bkt + gi, bk);
     }
     st4(pel(KT, r, c), kt);
@@ -1172,7 +1170,8 @@ __global__ void __launch_bounds__(kThreads, RM * RN >= 64 ? 1 : 3)
 // Per (chunk, head): the input gradients from the products above.
 template <typename IO>
 __global__ void __launch_bounds__(kThreads)
-    final_kernel(BwdWs w, const float* __restrict__ beta,
+    final_kernel(BwdWs w, const IO* __restrict__ q, const IO* __restrict__ k,
+                 const float* __restrict__ beta,
                  const float* __restrict__ g, IO* __restrict__ dq,
                  IO* __restrict__ dk_out, IO* __restrict__ dv_out,
                  float* __restrict__ dla, float* __restrict__ dbeta,
@@ -1183,33 +1182,42 @@ __global__ void __launch_bounds__(kThreads)
   if (!locate_chunk(cid, cu, chunk_off, n_seqs, T, C, &seq, &tok0, &L)) return;
   const int h = blockIdx.y, tid = threadIdx.x, ntile = dv / kChainTile;
   extern __shared__ float sm[];
-  float* dg = sm;  // [C][dk]
-  // four consecutive channels per thread and step (d_k, d_v multiples of 4)
+  float* dg = sm;          // [C][dk]
+  float* pb = sm + C * dk; // [C][dk / 4] partials of rowsum(dKt/b * Kt)
+  // four consecutive channels per thread and step (d_k, d_v multiples of 4);
+  // Kt, Kb and Qt are recomputed from k, q and g exactly as prep forms them
   auto ld4 = [](const float* p) { return *reinterpret_cast<const float4*>(p); };
+  auto ld4io = [](const IO* p, float* x) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) x[u] = to_f32(p[u]);
+  };
   const int dk4 = dk / 4, dv4 = dv / 4;
   for (int idx = tid; idx < L * dk4; idx += kThreads) {
     const int r = idx / dk4, c = (idx % dk4) * 4;
     const size_t gi = ((size_t)(tok0 + r) * H + h) * dk + c;
     const float b = beta[(size_t)(tok0 + r) * H + h];
     const float4 bk = ld4(w.dbk + gi), kb4 = ld4(w.dkb + gi),
-                 qt4 = ld4(w.dqt + gi), g4 = ld4(g + gi), kt = ld4(w.kt + gi),
-                 qt = ld4(w.qt + gi), kb = ld4(w.kb + gi);
-    const float dKt[4] = {b * bk.x, b * bk.y, b * bk.z, b * bk.w};
+                 qt4 = ld4(w.dqt + gi), g4 = ld4(g + gi);
+    float kv[4], qv[4];
+    ld4io(k + gi, kv);
+    ld4io(q + gi, qv);
+    const float dbk[4] = {bk.x, bk.y, bk.z, bk.w};
     const float dKb[4] = {kb4.x, kb4.y, kb4.z, kb4.w};
     const float dQt[4] = {qt4.x, qt4.y, qt4.z, qt4.w};
     const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
-    const float ktv[4] = {kt.x, kt.y, kt.z, kt.w};
-    const float qtv[4] = {qt.x, qt.y, qt.z, qt.w};
-    const float kbv[4] = {kb.x, kb.y, kb.z, kb.w};
-    float o[4];
+    float o[4], part = 0.f;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const float e = __expf(gv[u]), ie = __expf(-gv[u]);
-      dk_out[gi + u] = from_f32<IO>(dKt[u] * e + dKb[u] * ie);
+      const float kt = kv[u] * e, kb = kv[u] * ie, qt = qv[u] * e;
+      const float dKt = b * dbk[u];
+      dk_out[gi + u] = from_f32<IO>(dKt * e + dKb[u] * ie);
       dq[gi + u] = from_f32<IO>(dQt[u] * e);
-      o[u] = dKt[u] * ktv[u] + dQt[u] * qtv[u] - dKb[u] * kbv[u];
+      o[u] = dKt * kt + dQt[u] * qt - dKb[u] * kb;
+      part += dbk[u] * kt;
     }
     *reinterpret_cast<float4*>(dg + r * dk + c) = make_float4(o[0], o[1], o[2], o[3]);
+    pb[r * dk4 + c / 4] = part;
   }
   for (int idx = tid; idx < L * dv4; idx += kThreads) {
     const int r = idx / dv4, c = (idx % dv4) * 4;
@@ -1236,10 +1244,9 @@ __global__ void __launch_bounds__(kThreads)
   // d beta: one warp per row, lanes across the row, then a shuffle sum
   const int warp = tid >> 5, lane = tid & 31;
   for (int r = warp; r < L; r += kThreads / 32) {
-    const size_t rk = ((size_t)(tok0 + r) * H + h) * dk;
     const size_t rv = ((size_t)(tok0 + r) * H + h) * dv;
     float acc = 0.f;
-    for (int c = lane; c < dk; c += 32) acc += w.dbk[rk + c] * w.kt[rk + c];
+    for (int c = lane; c < dk4; c += 32) acc += pb[r * dk4 + c];
     for (int j = lane; j < dv; j += 32) acc += w.dbv[rv + j] * w.v32[rv + j];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
@@ -1791,10 +1798,11 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
                kDimDk,
                kMaskNone, 1.f, 0))
 #undef KDA_BMM
-  const size_t smf = 4 * (size_t)C * dk;
+  const size_t smf = 4 * (size_t)C * dk + (size_t)C * dk;
   if ((e = set_smem(final_kernel<IO>, smf)) != cudaSuccess) return e;
   final_kernel<IO><<<grid, kThreads, smf, stream>>>(
-      w, f.beta, w.fv.g, static_cast<IO*>(a.dq), static_cast<IO*>(a.dk),
+      w, static_cast<const IO*>(f.q), static_cast<const IO*>(f.k), f.beta,
+      w.fv.g, static_cast<IO*>(a.dq), static_cast<IO*>(a.dk),
       static_cast<IO*>(a.dv), a.d_log_alpha, a.d_beta, cu, co, f.n_seqs, f.T,
       H, dk, dv, C);
   return cudaGetLastError();
