@@ -76,8 +76,8 @@ struct BwdWs {
   // [chunks, H, d, C], zero past each chunk's last token; ddT holds -dDelta^T
   float *qtT, *kbT, *bktT, *doT, *ddT;
   float* khT;  // Kh^T per chunk [chunks, H, dk, C] for the state pass, tf32
-  float *kt, *kb, *qt, *bkt;      // [tokens, H, dk]
-  float *v32, *bv, *do32, *dd;    // [tokens, H, dv]
+  float *kb, *qt, *bkt;           // [tokens, H, dk]; qt on the SIMT path only
+  float *bv, *do32, *dd;          // [tokens, H, dv]
   float *tm, *pp;                 // [chunks, H, C, C]
   float *gam;                     // [chunks, H, dk]
   float *gst;                     // G = Diag(gam) dS_C, [chunks, H, dk, dv]
@@ -143,8 +143,10 @@ BwdWs carve_bwd(const BwdArgs& a, void* base, size_t* total) {
   }
   const size_t tdk = 4 * tokens * H * dk, tdv = 4 * tokens * H * dv;
   const size_t sq = 4 * nch * H * C * C, st = 4 * nch * H * dk * dv;
-  w.kt = take(tdk); w.kb = take(tdk); w.qt = take(tdk); w.bkt = take(tdk);
-  w.v32 = take(tdv); w.bv = take(tdv); w.do32 = take(tdv); w.dd = take(tdv);
+  w.kb = take(tdk);
+  w.qt = tensor_chain(fa) ? nullptr : take(tdk);
+  w.bkt = take(tdk);
+  w.bv = take(tdv); w.do32 = take(tdv); w.dd = take(tdv);
   w.tm = take(sq); w.pp = take(sq);
   w.gam = take(4 * nch * H * dk);
   w.gst = take(st);
@@ -219,7 +221,6 @@ __global__ void __launch_bounds__(kThreads, 2)  // two CTAs per SM
       kt = kv * e;
       kb = kv * ie;
       qt = qv * e;
-      w.kt[gi] = kt;
       w.kb[gi] = kb;
       w.qt[gi] = qt;
       w.bkt[gi] = bs[r] * kt;
@@ -240,7 +241,6 @@ __global__ void __launch_bounds__(kThreads, 2)  // two CTAs per SM
     if (idx < C * dv && r < L) {
       const size_t gi = ((size_t)(tok0 + r) * H + h) * dv + idx % dv;
       vr[u] = to_f32(v[gi]);
-      w.v32[gi] = vr[u];
       w.bv[gi] = bs[r] * vr[u];
       w.do32[gi] = to_f32(dout[gi]);
     }
@@ -544,7 +544,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     ld_bf4(dout + gi, dd);
 #pragma unroll
     for (int u = 0; u < 4; ++u) bvv[u] = bs[r] * vv[u];
-    st4(w.v32 + gi, vv);
     st4(w.bv + gi, bvv);
     st4(w.do32 + gi, dd);
   }
@@ -1171,7 +1170,7 @@ __global__ void __launch_bounds__(kThreads, RM * RN >= 64 ? 1 : 3)
 template <typename IO>
 __global__ void __launch_bounds__(kThreads)
     final_kernel(BwdWs w, const IO* __restrict__ q, const IO* __restrict__ k,
-                 const float* __restrict__ beta,
+                 const IO* __restrict__ v, const float* __restrict__ beta,
                  const float* __restrict__ g, IO* __restrict__ dq,
                  IO* __restrict__ dk_out, IO* __restrict__ dv_out,
                  float* __restrict__ dla, float* __restrict__ dbeta,
@@ -1247,7 +1246,7 @@ __global__ void __launch_bounds__(kThreads)
     const size_t rv = ((size_t)(tok0 + r) * H + h) * dv;
     float acc = 0.f;
     for (int c = lane; c < dk4; c += 32) acc += pb[r * dk4 + c];
-    for (int j = lane; j < dv; j += 32) acc += w.dbv[rv + j] * w.v32[rv + j];
+    for (int j = lane; j < dv; j += 32) acc += w.dbv[rv + j] * to_f32(v[rv + j]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     if (lane == 0) dbeta[(size_t)(tok0 + r) * H + h] = acc;
@@ -1801,7 +1800,8 @@ cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
   const size_t smf = 4 * (size_t)C * dk + (size_t)C * dk;
   if ((e = set_smem(final_kernel<IO>, smf)) != cudaSuccess) return e;
   final_kernel<IO><<<grid, kThreads, smf, stream>>>(
-      w, static_cast<const IO*>(f.q), static_cast<const IO*>(f.k), f.beta,
+      w, static_cast<const IO*>(f.q), static_cast<const IO*>(f.k),
+      static_cast<const IO*>(f.v), f.beta,
       w.fv.g, static_cast<IO*>(a.dq), static_cast<IO*>(a.dk),
       static_cast<IO*>(a.dv), a.d_log_alpha, a.d_beta, cu, co, f.n_seqs, f.T,
       H, dk, dv, C);
