@@ -1,8 +1,12 @@
-// Reverse state-gradient chain of the chunkwise backward pass on the tensor
-// cores (tcgen05 kind::tf32, fp32 operands in 128-byte-swizzled shared
-// memory, fp32 accumulators in TMEM).  Included by kda_fused_sm100.cu, whose
-// tensor-map encoder and device timeout flag it shares.
+// The two serial chains of the chunkwise backward pass on the tensor cores
+// (tcgen05 kind::tf32, fp32 operands in 128-byte-swizzled shared memory,
+// fp32 accumulators in TMEM): the reverse state-gradient chain
+// (rev_chain_kernel, below) and the backward's copy of the forward's state
+// pass (state_chain_kernel, at the end of the file).  Included by
+// kda_fused_sm100.cu, whose tensor-map encoder and device timeout flag they
+// share.
 //
+// The reverse chain:
 // Per chunk, walking each sequence's chunks from last to first, with dS the
 // gradient of the state leaving the chunk (the chain rule applied to the
 // chunkwise form S_C = Diag(gam)(S_0 + Kb^T Delta), Delta = U - W S_0; "You
@@ -12,8 +16,9 @@
 //   G      = Diag(gam) dS
 //   dDelta = Kb G + P^T dO                 (MMA 1: M = 64 tokens, K = d_k)
 //   dS    <- G + Qt^T dO - W^T dDelta      (MMA 2: M = d_k, K = 64 tokens)
-// G, dDelta and the gam * d gam partials go to the workspace for the batched
-// products that follow; the last dS is the initial-state gradient.
+// G, dDelta (and -dDelta^T per chunk) and the gam * d gam partials go to the
+// workspace for the batched products that follow; the last dS is the
+// initial-state gradient.
 //
 // One CTA of 256 threads per (sequence, head, 64-column d_v tile); thread c
 // owns TMEM lane c % 128 and 32 columns 32 (c / 128) .. + 31.  dS stays in
