@@ -75,17 +75,19 @@ def test_backward_packed_with_empty_and_short(io):
     assert torch.equal(got[5][1], dsT[1])
 
 
-def test_backward_without_states():
-    # no initial state (zeros) and no final-state gradient
-    d = W.draw((1, 100), 3, 64, 64, io="f32", n_states=None, device=DEV, seed=5)
+@pytest.mark.parametrize("io,C", [("f32", 32), ("bf16", 64)])
+def test_backward_without_states(io, C):
+    # no initial state (zeros) and no final-state gradient; bf16 in 64-token
+    # chunks takes the tensor-core path
+    d = W.draw((1, 100), 3, 64, 64, io=io, n_states=None, device=DEV, seed=5)
     do, _ = grads_in(d, seed=6, with_final=False)
     got = K.chunk_bwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], None,
-                      None, do, None, chunk=32)
+                      None, do, None, chunk=C)
     torch.cuda.synchronize()
     ref = kda_oracle.recurrent_bwd(*(PY.host64(d[n]) for n in
                                      ("q", "k", "v", "log_alpha", "beta")),
                                    None, PY.host64(do), None)
-    compare(got, ref, PY.TOL_F32)
+    compare(got, ref, PY.TOL_F32 if io == "f32" else PY.TOL_BF16)
 
 
 def test_backward_config2_sampled():
