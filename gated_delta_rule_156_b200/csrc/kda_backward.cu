@@ -570,14 +570,26 @@ __global__ void __launch_bounds__(kThreads, 2)
   // the transposed copies meanwhile (reads only)
   {
     const size_t tb = ((size_t)cid * H + h) * DK * C;
-    for (int idx = tid; idx < DK * C; idx += kThreads) {
-      const int c = idx / C, r = idx % C;
-      const float kb = *pel(KB, r, c);
-      w.qtT[tb + idx] = *pel(QT, r, c);
-      w.kbT[tb + idx] = kb;
-      w.bktT[tb + idx] = bs[r] * *pel(KT, r, c);
-      // Kh = k exp(g_C - g) = Kb exp(g_C), rounded to the nearest tf32
-      w.khT[tb + idx] = sm100::tf32_rna(kb * __expf(gl[c]));
+    // a thread reads four consecutive channels of one token row (16-byte
+    // shared loads) and writes them to four transposed rows; a warp covers
+    // 32 consecutive tokens, so each global store is one 128-byte segment
+    for (int idx = tid; idx < DK / 4 * C; idx += kThreads) {
+      const int r = idx % C, c = (idx / C) * 4;
+      const float4 q4 = *reinterpret_cast<const float4*>(pel(QT, r, c));
+      const float4 b4 = *reinterpret_cast<const float4*>(pel(KB, r, c));
+      const float4 t4 = *reinterpret_cast<const float4*>(pel(KT, r, c));
+      const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
+      const float kbv[4] = {b4.x, b4.y, b4.z, b4.w};
+      const float ktv[4] = {t4.x, t4.y, t4.z, t4.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const size_t o = tb + (size_t)(c + u) * C + r;
+        w.qtT[o] = qv[u];
+        w.kbT[o] = kbv[u];
+        w.bktT[o] = bs[r] * ktv[u];
+        // Kh = k exp(g_C - g) = Kb exp(g_C), rounded to the nearest tf32
+        w.khT[o] = sm100::tf32_rna(kbv[u] * __expf(gl[c + u]));
+      }
     }
   }
   bool ok = __syncthreads_and(mbar_wait(bar, 0, 2000000000ull));
