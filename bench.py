@@ -563,8 +563,8 @@ def run_kda(args, world, rank, local):
         del ds, outs, fins
 
     # ---- backward pass of the prefill workload: every input's gradient for
-    # a random output gradient (chunkwise; fp32 products, the forward's
-    # state pass on the tensor cores for bf16 inputs) -----------------------
+    # a random output gradient (chunkwise, fp32 arithmetic; with bf16 inputs
+    # every product runs on the tensor cores in tf32) -----------------------
     gdo = torch.randn(d["v"].shape, generator=torch.Generator(device=dev)
                       .manual_seed(77 + rank), device=dev).bfloat16()
 
@@ -591,7 +591,8 @@ def run_kda(args, world, rank, local):
         "value": world * B * T / (bwms / bw_steps * 1e-3), "unit": "tokens/s",
         "ms_per_step": bwms / bw_steps, "steps": bw_steps,
         "workload": "kda_chunk_bwd on the prefill workload (dq, dk, dv, "
-                    "dlog_alpha, dbeta), fp32 products, tensor-core state pass",
+                    "dlog_alpha, dbeta), every product on tcgen05 in tf32 "
+                    "(the state pass with high and low parts)",
         "hbm": {"achieved": bw_bytes / (bw_launch * 1e-3) / 1e9, "unit": "GB/s",
                 "frac": bw_bytes / (bw_launch * 1e-3) / 1e9 / pk["hbm_gbs"],
                 "algorithmic_bytes_per_launch": bw_bytes},
