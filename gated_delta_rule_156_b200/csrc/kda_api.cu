@@ -1,6 +1,7 @@
 // C-ABI boundary of libkda.so: argument validation, workspace, dispatch.
 // Every argument error is found here, on the host, before anything launches.
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <atomic>
@@ -48,6 +49,24 @@ void keep_pool_memory() {
     cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &thr);
   }
   done_mask.fetch_or(bit);
+}
+
+// Stream-ordered workspace for one call.  With KDA_WORKSPACE_FILL set to a
+// byte value (0-255) the workspace is first filled with that byte: a test
+// aid, since with 127 every fp32 word reads 3.4e38 and a kernel that read a
+// place before writing it would turn its results non-finite or far off.
+cudaError_t take_workspace(size_t bytes, cudaStream_t stream, void** ws) {
+  *ws = nullptr;
+  if (!bytes) return cudaSuccess;
+  keep_pool_memory();
+  cudaError_t e = cudaMallocAsync(ws, bytes, stream);
+  if (e != cudaSuccess) {
+    *ws = nullptr;
+    return e;
+  }
+  const char* fill = getenv("KDA_WORKSPACE_FILL");
+  if (fill && *fill) e = cudaMemsetAsync(*ws, atoi(fill) & 255, bytes, stream);
+  return e;
 }
 
 // Shape-only checks shared by the launch entry points and the planner.
@@ -143,10 +162,9 @@ kda_status run_with_workspace(size_t bytes, cudaStream_t stream, Path path,
                               const kda::ChunkArgs& a) {
   void* ws = nullptr;
   cudaError_t e;
-  if (bytes) {
-    keep_pool_memory();
-    if ((e = cudaMallocAsync(&ws, bytes, stream)) != cudaSuccess)
-      return cuda_fail(e);
+  if ((e = take_workspace(bytes, stream, &ws)) != cudaSuccess) {
+    if (ws) cudaFreeAsync(ws, stream);
+    return cuda_fail(e);
   }
   e = path == Path::kFused     ? kda::launch_fused(a, ws, stream)
       : path == Path::kTwoPass ? kda::launch_twopass(a, ws, stream)
@@ -239,10 +257,9 @@ kda_status kda_chunk_fwd_split(const kda_shape* shape, int gate, const void* q,
   const size_t bytes = kda::split_workspace_bytes(a, g);
   void* ws = nullptr;
   cudaError_t e;
-  if (bytes) {
-    keep_pool_memory();
-    if ((e = cudaMallocAsync(&ws, bytes, stream)) != cudaSuccess)
-      return cuda_fail(e);
+  if ((e = take_workspace(bytes, stream, &ws)) != cudaSuccess) {
+    if (ws) cudaFreeAsync(ws, stream);
+    return cuda_fail(e);
   }
   e = kda::launch_split(a, g, ws, stream);
   if (ws) {
@@ -355,10 +372,9 @@ kda_status kda_chunk_bwd(const kda_shape* shape, const void* q, const void* k,
   void* ws = nullptr;
   cudaError_t e;
   const size_t bytes = kda::bwd_workspace_bytes(b);
-  if (bytes) {
-    keep_pool_memory();
-    if ((e = cudaMallocAsync(&ws, bytes, stream)) != cudaSuccess)
-      return cuda_fail(e);
+  if ((e = take_workspace(bytes, stream, &ws)) != cudaSuccess) {
+    if (ws) cudaFreeAsync(ws, stream);
+    return cuda_fail(e);
   }
   e = kda::launch_bwd(b, ws, stream);
   if (ws) {

@@ -45,6 +45,8 @@
 //     operands staged in shared memory and merged into multi-term launches;
 //   - a last kernel that combines them into the input gradients.
 // Channel gate, no input prologue.
+#include <algorithm>
+
 #include "kda_common.cuh"
 #include "kda_internal.h"
 #include "kda_inverse.cuh"
@@ -117,46 +119,123 @@ BwdWs carve_bwd(const BwdArgs& a, void* base, size_t* total) {
       f.cu_seqlens ? (size_t)f.T : (size_t)f.n_seqs * (size_t)f.T;
   const size_t H = f.H, dk = f.dk, dv = f.dv, C = f.chunk;
   const size_t nch = (size_t)max_chunks(f);
-  size_t off = 0;
-  char* p = static_cast<char*>(base);
-  auto take = [&](size_t bytes) {
-    char* r = p ? p + off : nullptr;
-    off = align256(off + bytes);
-    return reinterpret_cast<float*>(r);
-  };
-  BwdWs w{};
-  w.fin = take(4 * (size_t)f.n_seqs * H * dk * dv);
   const ChunkArgs fa = forward_args(a, nullptr);
-  w.staged = take(staged_workspace_bytes(fa));
-  w.wt = tensor_chain(fa)
-             ? take(4 * (size_t)max_chunks(fa) * f.H * f.dk * f.chunk)
-             : nullptr;
-  if (tensor_chain(fa)) {
-    const size_t tk = 4 * (size_t)max_chunks(fa) * f.H * f.dk * f.chunk;
-    const size_t tv = 4 * (size_t)max_chunks(fa) * f.H * f.dv * f.chunk;
-    w.qtT = take(tk);
-    w.kbT = take(tk);
-    w.bktT = take(tk);
-    w.doT = take(tv);
-    w.ddT = take(tv);
-    w.khT = take(tk);
-  }
   const size_t tdk = 4 * tokens * H * dk, tdv = 4 * tokens * H * dv;
   const size_t sq = 4 * nch * H * C * C, st = 4 * nch * H * dk * dv;
-  w.kb = take(tdk);
-  w.qt = tensor_chain(fa) ? nullptr : take(tdk);
-  w.bkt = take(tdk);
-  w.bv = take(tdv); w.do32 = take(tdv); w.dd = take(tdv);
-  w.tm = take(sq); w.pp = take(sq);
-  w.gam = take(4 * nch * H * dk);
-  w.gst = take(st);
-  w.dgam = take(4 * nch * H * (dv / 32) * dk);
-  w.dp = take(sq); w.dtm = take(sq); w.tmp = take(sq); w.da = take(sq);
-  w.dqt = take(tdk); w.dkb = take(tdk); w.dw = take(tdk); w.dbk = take(tdk);
-  w.dbv = take(tdv);
-  w.qdo = take(st);
-  w.pdo = take(tdv);
-  if (total) *total = off;
+  const size_t fin = 4 * (size_t)f.n_seqs * H * dk * dv;
+  const size_t gam = 4 * nch * H * dk, dgam = 4 * nch * H * (dv / 32) * dk;
+  char* p = static_cast<char*>(base);
+  BwdWs w{};
+  if (!tensor_chain(fa)) {  // fp32 SIMT path: every array apart
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+      char* r = p ? p + off : nullptr;
+      off = align256(off + bytes);
+      return reinterpret_cast<float*>(r);
+    };
+    w.fin = take(fin);
+    w.staged = take(staged_workspace_bytes(fa));
+    w.kb = take(tdk); w.qt = take(tdk); w.bkt = take(tdk);
+    w.bv = take(tdv); w.do32 = take(tdv); w.dd = take(tdv);
+    w.tm = take(sq); w.pp = take(sq);
+    w.gam = take(gam);
+    w.gst = take(st);
+    w.dgam = take(dgam);
+    w.dp = take(sq); w.dtm = take(sq); w.tmp = take(sq); w.da = take(sq);
+    w.dqt = take(tdk); w.dkb = take(tdk); w.dw = take(tdk); w.dbk = take(tdk);
+    w.dbv = take(tdv);
+    w.qdo = take(st);
+    w.pdo = take(tdv);
+    if (total) *total = off;
+    return w;
+  }
+  // Tensor-core path: arrays share memory where their lifetimes (from the
+  // launch that first writes one to the last launch that reads it, both
+  // included) do not overlap.  The launches, in order:
+  enum {
+    kPrefix,  // chunk offsets (packed layout), g
+    kPrep,    // prep_tc_kernel
+    kState,   // the forward's state pass
+    kQdo, kPdo,
+    kRev,     // reverse chain
+    kDp, kDqt, kDw, kDtm, kDbv, kTmp, kDa, kDbk, kDkb,  // batched products
+    kFinal
+  };
+  const size_t tk = 4 * nch * H * dk * C, tv = 4 * nch * H * dv * C;
+  struct Arr {
+    float** ptr;
+    size_t bytes;
+    int first, last;
+  };
+  float *staged = nullptr, *sw = nullptr, *su = nullptr, *ss = nullptr;
+  const Arr arr[] = {
+      {&staged, staged_prefix_bytes(fa), kPrefix, kFinal},
+      {&w.fin, fin, kState, kRev},
+      {&sw, tdk, kPrep, kState},  // W, row-major
+      {&su, tdv, kPrep, kDkb},    // U, then Delta in place
+      {&ss, st, kState, kDw},     // chunk-start states
+      {&w.wt, tk, kPrep, kRev},
+      {&w.qtT, tk, kPrep, kDkb},
+      {&w.kbT, tk, kPrep, kDbk},
+      {&w.bktT, tk, kPrep, kDkb},
+      {&w.doT, tv, kPrep, kPdo},
+      {&w.ddT, tv, kRev, kDbv},
+      {&w.khT, tk, kPrep, kState},
+      {&w.kb, tdk, kPrep, kRev},
+      {&w.bkt, tdk, kPrep, kDtm},
+      {&w.bv, tdv, kPrep, kDtm},
+      {&w.do32, tdv, kPrep, kDqt},
+      {&w.dd, tdv, kRev, kDtm},
+      {&w.tm, sq, kPrep, kDbk},
+      {&w.pp, sq, kPrep, kPdo},
+      {&w.gam, gam, kPrep, kRev},
+      {&w.gst, st, kRev, kDkb},
+      {&w.dgam, dgam, kRev, kFinal},
+      {&w.dp, sq, kDp, kDkb},
+      {&w.dtm, sq, kDtm, kTmp},
+      {&w.tmp, sq, kTmp, kDa},
+      {&w.da, sq, kDa, kDkb},
+      {&w.dqt, tdk, kDqt, kFinal},
+      {&w.dkb, tdk, kDkb, kFinal},
+      {&w.dw, tdk, kDw, kDbk},
+      {&w.dbk, tdk, kDbk, kFinal},
+      {&w.dbv, tdv, kDbv, kFinal},
+      {&w.qdo, st, kQdo, kRev},
+      {&w.pdo, tdv, kPdo, kRev},
+  };
+  constexpr int n = sizeof(arr) / sizeof(arr[0]);
+  // first fit, largest arrays first: each goes to the lowest offset free of
+  // every array placed before it whose lifetime it shares
+  int order[n], live[n];
+  size_t offs[n];
+  for (int i = 0; i < n; ++i) order[i] = i;
+  std::stable_sort(order, order + n, [&](int x, int y) {
+    return arr[x].bytes > arr[y].bytes;
+  });
+  size_t top = 0;
+  for (int r = 0; r < n; ++r) {
+    const Arr& x = arr[order[r]];
+    int nl = 0;
+    for (int s = 0; s < r; ++s) {
+      const Arr& y = arr[order[s]];
+      if (y.first <= x.last && x.first <= y.last) live[nl++] = order[s];
+    }
+    std::sort(live, live + nl, [&](int i, int j) { return offs[i] < offs[j]; });
+    size_t off = 0;
+    for (int s = 0; s < nl; ++s) {
+      if (off + x.bytes <= offs[live[s]]) break;
+      off = std::max(off, align256(offs[live[s]] + arr[live[s]].bytes));
+    }
+    offs[order[r]] = off;
+    top = std::max(top, align256(off + x.bytes));
+  }
+  for (int i = 0; i < n; ++i)
+    *arr[i].ptr = p ? reinterpret_cast<float*>(p + offs[i]) : nullptr;
+  w.staged = staged;
+  w.fv.w = sw;
+  w.fv.d = su;
+  w.fv.s = ss;
+  if (total) *total = top;
   return w;
 }
 
@@ -1613,9 +1692,17 @@ template <typename IO>
 cudaError_t run_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream) {
   BwdWs w = carve_bwd(a, workspace, nullptr);
   const ChunkArgs f = forward_args(a, w.fin);
-  // the forward's plan and cumulative log-decay
+  // the forward's plan and cumulative log-decay (on the tensor-core path W,
+  // U and the states have their own places in the shared workspace)
+  const StagedView packed = w.fv;
   cudaError_t e = launch_staged_part(f, w.staged, &w.fv, false, stream);
   if (e != cudaSuccess) return e;
+  if (packed.s) {
+    w.fv.w = packed.w;
+    w.fv.d = packed.d;
+    w.fv.kh = nullptr;
+    w.fv.s = packed.s;
+  }
   const int C = f.chunk, H = f.H, dk = f.dk, dv = f.dv;
   const int64_t nch = max_chunks(f);
   const int32_t* cu = f.cu_seqlens;

@@ -72,7 +72,9 @@ cudaError_t launch_staged(const ChunkArgs& a, void* workspace,
 // With state_pass true: the serial state pass, which turns U into
 // Delta = U - W S_0 in place, stores every chunk-start state
 // [max_chunks, H, dk, dv] in view->s and the final state in a.final_state.
-// All fp32; channel gate, no prologue.
+// All fp32; channel gate, no prologue.  With state_pass false only the first
+// staged_prefix_bytes(a) bytes of the workspace are touched (the chunk
+// offsets and g); view->w, d, kh and s then point past them.
 struct StagedView {
   const int32_t* chunk_off;
   const float* g;
@@ -84,6 +86,7 @@ struct StagedView {
 cudaError_t launch_staged_part(const ChunkArgs& a, void* workspace,
                                StagedView* view, bool state_pass,
                                cudaStream_t stream);
+size_t staged_prefix_bytes(const ChunkArgs& a);
 
 // Sequence-split prefill of one long sequence (kda_split.cu): k segments of
 // Ls tokens (a multiple of the chunk; the last one takes the rest) evaluated

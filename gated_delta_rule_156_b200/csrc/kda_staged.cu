@@ -57,7 +57,8 @@ struct Ws {
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-Ws carve(const ChunkArgs& a, void* base, size_t* total) {
+Ws carve(const ChunkArgs& a, void* base, size_t* total,
+         size_t* prefix = nullptr) {
   const size_t tokens =
       a.cu_seqlens ? (size_t)a.T : (size_t)a.n_seqs * (size_t)a.T;
   const size_t H = a.H;
@@ -78,6 +79,7 @@ Ws carve(const ChunkArgs& a, void* base, size_t* total) {
   }
   w.chunk_off = reinterpret_cast<int32_t*>(take(4 * (size_t)(a.n_seqs + 1)));
   w.g = reinterpret_cast<float*>(take(4 * tokens * H * a.dk));
+  if (prefix) *prefix = off;
   w.w = reinterpret_cast<float*>(take(4 * tokens * H * a.dk));
   w.u = reinterpret_cast<float*>(take(4 * tokens * H * a.dv));
   w.kh = reinterpret_cast<float*>(take(4 * tokens * H * a.dk));
@@ -618,6 +620,12 @@ size_t staged_workspace_bytes(const ChunkArgs& a) {
   size_t total = 0;
   carve(a, nullptr, &total);
   return total;
+}
+
+size_t staged_prefix_bytes(const ChunkArgs& a) {
+  size_t total = 0, prefix = 0;
+  carve(a, nullptr, &total, &prefix);
+  return prefix;
 }
 
 int staged_kernel_count(const ChunkArgs& a) {

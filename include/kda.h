@@ -415,7 +415,9 @@ KDA_API kda_status kda_device_status(cudaStream_t stream);
  * within the bf16 tolerance of 1e-2 relative L2 (a bounded wait that gives up is reported by kda_device_status as
  * KDA_ERR_TIMEOUT); the call
  * re-runs the forward's chunk stages and allocates its fp32 workspace from
- * the stream-ordered pool (kda_chunk_bwd_plan reports its size).  Stream
+ * the stream-ordered pool (kda_chunk_bwd_plan reports its size; on the
+ * tensor-core path intermediates whose lifetimes do not overlap share
+ * memory, about 5.3 GB at B=2, T=8192, H=32, d=128).  Stream
  * ordered: returns after queueing the kernels.
  * Numerical range: the backward keeps the chunk-start factorisation of the
  * decay, exact while |g_C| <= 80 on every channel of every chunk (g_C as
@@ -520,7 +522,10 @@ KDA_API kda_status kda_selftest_timeout(int limit_us, cudaStream_t stream);
  * pool's release threshold to the maximum on first use, so freed workspace
  * stays cached in the pool: after the first call of a given size, repeated
  * calls reuse the pool's memory and reserve nothing new from the device.
- * Calls on different streams never share a workspace.
+ * Calls on different streams never share a workspace.  With the
+ * environment variable KDA_WORKSPACE_FILL set to a byte value (0-255), each
+ * call first fills its workspace with that byte (a test aid: no kernel may
+ * read a place of it before writing it, so the results must not change).
  *   reserved_bytes : out, memory the pool currently holds (may be NULL).
  *   used_bytes     : out, memory of the pool in use right now (may be NULL).
  * Reads the current device's pool; launches nothing.

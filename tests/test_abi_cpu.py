@@ -68,8 +68,14 @@ def test_backward_plan(lib):
     assert kern == 16 and ws > 0
     kern_f, ws_f = K.chunk_bwd_plan(2, 8192, 32, 128, 128, 64, torch.float32)
     assert kern_f == 16
-    # the tensor-core path keeps W^T and the transposed per-chunk copies too
-    assert ws > ws_f
+    # the tensor-core path keeps W^T and the transposed per-chunk copies too,
+    # but its arrays share memory where their lifetimes do not overlap: less
+    # than the fp32 path, which keeps every array apart, and at least what
+    # the reverse chain alone reads and writes (Kb, W^T, Qt^T dO, P^T dO,
+    # the chunk-start states, G, dDelta, its transposed copy)
+    assert ws < ws_f
+    tok, st = 4 * 2 * 8192 * 32 * 128, 4 * 2 * 128 * 32 * 128 * 128
+    assert ws >= 5 * tok + 3 * st
     kern_p, _ = K.chunk_bwd_plan(1, 300, 2, 64, 64, 32, torch.float32,
                                  packed=True, n_seqs=3)
     assert kern_p == 17

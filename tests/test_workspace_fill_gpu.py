@@ -1,0 +1,95 @@
+"""No kernel reads a place of its workspace before writing it.
+
+Every call that needs workspace takes it from the stream-ordered pool, where
+it holds whatever an earlier call left.  With KDA_WORKSPACE_FILL=127 the
+library first fills it with the byte 0x7F, so each fp32 word reads 3.4e38: a
+read before the write would turn results non-finite or far off.  A read whose
+value is only multiplied by zero (a masked row of a product) stays harmless,
+as it is with any finite leftover.  So each call must return exactly what it
+returns without the fill.  This matters most for the backward pass, whose
+arrays share memory where their lifetimes do not overlap."""
+import numpy as np
+import pytest
+import torch
+
+import kda_workloads as W
+from gated_delta_rule_156_b200 import kda as K
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def same_with_fill(fn, monkeypatch):
+    monkeypatch.delenv("KDA_WORKSPACE_FILL", raising=False)
+    ref = [x.clone() for x in fn() if x is not None]
+    torch.cuda.synchronize()
+    monkeypatch.setenv("KDA_WORKSPACE_FILL", "127")
+    got = [x.clone() for x in fn() if x is not None]
+    torch.cuda.synchronize()
+    monkeypatch.delenv("KDA_WORKSPACE_FILL")
+    assert K.device_status() == 0
+    for i, (a, b) in enumerate(zip(ref, got)):
+        assert torch.isfinite(b.float()).all(), f"output {i} not finite"
+        assert torch.equal(a, b), f"output {i} changed under the fill"
+
+
+def grads(d, seed):
+    g = torch.Generator(device=DEV).manual_seed(seed)
+    do = torch.randn(d["v"].shape, generator=g, device=DEV).to(d["v"].dtype)
+    s = d["initial_state"]
+    ds = None if s is None else torch.randn(s.shape, generator=g, device=DEV)
+    return do, ds
+
+
+@pytest.mark.parametrize("io,chunk,dk,dv", [("bf16", 64, 128, 128),
+                                            ("bf16", 64, 64, 128),
+                                            ("f32", 16, 32, 64)])
+def test_backward_dense(io, chunk, dk, dv, monkeypatch):
+    d = W.draw((2, 200), 3, dk, dv, io=io, n_states=2, device=DEV, seed=91)
+    do, ds = grads(d, 92)
+    same_with_fill(lambda: K.chunk_bwd(
+        d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["initial_state"],
+        None, do, ds, chunk=chunk), monkeypatch)
+
+
+@pytest.mark.parametrize("io", ["bf16", "f32"])
+def test_backward_packed(io, monkeypatch):
+    lengths = [5, 0, 64, 1, 130, 63, 200]
+    d = W.draw((1, sum(lengths)), 2, 64, 64, io=io, n_states=len(lengths),
+               device=DEV, seed=93)
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lengths)]),
+                      dtype=torch.int32, device=DEV)
+    do, ds = grads(d, 94)
+    same_with_fill(lambda: K.chunk_bwd(
+        d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["initial_state"],
+        cu, do, ds, chunk=64), monkeypatch)
+
+
+def test_backward_without_states(monkeypatch):
+    d = W.draw((1, 300), 4, 128, 128, io="bf16", n_states=None, device=DEV,
+               seed=95)
+    do, _ = grads(d, 96)
+    same_with_fill(lambda: K.chunk_bwd(
+        d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], None, None, do,
+        None, chunk=64, want_initial_state=False), monkeypatch)
+
+
+@pytest.mark.parametrize("io,chunk,staged", [("bf16", 64, False),
+                                             ("f32", 16, True)])
+def test_prefill_packed(io, chunk, staged, monkeypatch):
+    lengths = [100, 0, 33, 64, 7, 300]
+    d = W.draw((1, sum(lengths)), 3, 64, 64, io=io, n_states=len(lengths),
+               device=DEV, seed=97)
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lengths)]),
+                      dtype=torch.int32, device=DEV)
+    same_with_fill(lambda: K.chunk_fwd(
+        d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["initial_state"],
+        cu, chunk=chunk, staged=staged), monkeypatch)
+
+
+def test_prefill_split(monkeypatch):
+    d = W.draw((1, 3000), 4, 128, 128, io="bf16", n_states=1, device=DEV,
+               seed=99)
+    same_with_fill(lambda: K.chunk_fwd_split(
+        d["q"], d["k"], d["v"], d["log_alpha"], d["beta"],
+        d["initial_state"], n_segments=3), monkeypatch)
