@@ -1277,9 +1277,29 @@ __global__ void __launch_bounds__(kThreads)
   // four consecutive channels per thread and step (d_k, d_v multiples of 4);
   // Kt, Kb and Qt are recomputed from k, q and g exactly as prep forms them
   auto ld4 = [](const float* p) { return *reinterpret_cast<const float4*>(p); };
+  // four consecutive io values as one 8-byte (bf16) or 16-byte (fp32) access
   auto ld4io = [](const IO* p, float* x) {
-#pragma unroll
-    for (int u = 0; u < 4; ++u) x[u] = to_f32(p[u]);
+    if constexpr (sizeof(IO) == 2) {
+      const uint2 u = *reinterpret_cast<const uint2*>(p);
+      const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+      const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+      x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
+    } else {
+      const float4 f = *reinterpret_cast<const float4*>(p);
+      x[0] = f.x; x[1] = f.y; x[2] = f.z; x[3] = f.w;
+    }
+  };
+  auto st4io = [](IO* p, const float* x) {
+    if constexpr (sizeof(IO) == 2) {
+      const __nv_bfloat162 a = __floats2bfloat162_rn(x[0], x[1]);
+      const __nv_bfloat162 b = __floats2bfloat162_rn(x[2], x[3]);
+      uint2 u;
+      u.x = *reinterpret_cast<const uint32_t*>(&a);
+      u.y = *reinterpret_cast<const uint32_t*>(&b);
+      *reinterpret_cast<uint2*>(p) = u;
+    } else {
+      *reinterpret_cast<float4*>(p) = make_float4(x[0], x[1], x[2], x[3]);
+    }
   };
   const int dk4 = dk / 4, dv4 = dv / 4;
   for (int idx = tid; idx < L * dk4; idx += kThreads) {
@@ -1295,17 +1315,19 @@ __global__ void __launch_bounds__(kThreads)
     const float dKb[4] = {kb4.x, kb4.y, kb4.z, kb4.w};
     const float dQt[4] = {qt4.x, qt4.y, qt4.z, qt4.w};
     const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
-    float o[4], part = 0.f;
+    float o[4], gk[4], gq[4], part = 0.f;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const float e = __expf(gv[u]), ie = __expf(-gv[u]);
       const float kt = kv[u] * e, kb = kv[u] * ie, qt = qv[u] * e;
       const float dKt = b * dbk[u];
-      dk_out[gi + u] = from_f32<IO>(dKt * e + dKb[u] * ie);
-      dq[gi + u] = from_f32<IO>(dQt[u] * e);
+      gk[u] = dKt * e + dKb[u] * ie;
+      gq[u] = dQt[u] * e;
       o[u] = dKt * kt + dQt[u] * qt - dKb[u] * kb;
       part += dbk[u] * kt;
     }
+    st4io(dk_out + gi, gk);
+    st4io(dq + gi, gq);
     *reinterpret_cast<float4*>(dg + r * dk + c) = make_float4(o[0], o[1], o[2], o[3]);
     pb[r * dk4 + c / 4] = part;
   }
@@ -1314,10 +1336,8 @@ __global__ void __launch_bounds__(kThreads)
     const size_t gi = ((size_t)(tok0 + r) * H + h) * dv + c;
     const float b = beta[(size_t)(tok0 + r) * H + h];
     const float4 x = ld4(w.dbv + gi);
-    dv_out[gi] = from_f32<IO>(b * x.x);
-    dv_out[gi + 1] = from_f32<IO>(b * x.y);
-    dv_out[gi + 2] = from_f32<IO>(b * x.z);
-    dv_out[gi + 3] = from_f32<IO>(b * x.w);
+    const float y[4] = {b * x.x, b * x.y, b * x.z, b * x.w};
+    st4io(dv_out + gi, y);
   }
   __syncthreads();
   for (int c = tid; c < dk; c += kThreads) {
