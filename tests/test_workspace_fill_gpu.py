@@ -93,3 +93,19 @@ def test_prefill_split(monkeypatch):
     same_with_fill(lambda: K.chunk_fwd_split(
         d["q"], d["k"], d["v"], d["log_alpha"], d["beta"],
         d["initial_state"], n_segments=3), monkeypatch)
+
+
+@pytest.mark.parametrize("gate,io,chunk", [("channel", "f32", 32),
+                                           ("head", "bf16", 64)])
+def test_staged_prefill_with_input_prologue(gate, io, chunk, monkeypatch):
+    # the staged pipeline writes normalised q, k and log(alpha) into its
+    # workspace first, then its four stages read them back
+    d = W.draw((2, 140), 2, 64, 64, io=io, n_states=2, device=DEV, seed=101)
+    g = torch.Generator(device=DEV).manual_seed(102)
+    logits = torch.randn(d["log_alpha"].shape if gate == "channel"
+                         else d["beta"].shape, generator=g, device=DEV)
+    pro = dict(normalize_qk=True, q_scale=0.125, gate_logits=True,
+               gate_scale=1 / 16)
+    same_with_fill(lambda: K.chunk_fwd(
+        d["q"], d["k"], d["v"], logits, d["beta"], d["initial_state"], None,
+        chunk=chunk, staged=True, gate=gate, prologue=pro), monkeypatch)
