@@ -500,9 +500,10 @@ struct StateLayout {
   static constexpr uint32_t wb = 0;                          // W + pad panel
   static constexpr uint32_t ub = wb + (DK / 32 + 1) * 8192;  // U / Delta
   static constexpr uint32_t kb = ub + 2 * 8192;              // Kh^T, 128 rows
-  static constexpr uint32_t shi = kb + 2 * 16384;            // S, B operand
-  static constexpr uint32_t slo = shi + (DK / 32) * 8192;
-  static constexpr uint32_t dhi = slo + (DK / 32) * 8192;    // Delta, B operand
+  // S as the B operand of product A: per 32-row K panel, 64 N-rows of the
+  // tf32 high part then 64 of the remainder (one N = 128 operand)
+  static constexpr uint32_t sop = kb + 2 * 16384;
+  static constexpr uint32_t dhi = sop + (DK / 32) * 16384;   // Delta, B operand
   static constexpr uint32_t dlo = dhi + 2 * 8192;
   static constexpr uint32_t sst = dlo + 2 * 8192;            // S staging
   static constexpr uint32_t misc = sst + 2 * DK * 128;
@@ -510,7 +511,8 @@ struct StateLayout {
   static constexpr uint32_t w_tx = (DK / 32) * 8192;
   static constexpr uint32_t u_tx = 2 * 8192;
   static constexpr uint32_t k_tx = 2 * DK * 128;
-  static constexpr uint32_t t_s = 0, t_d = 64;  // TMEM columns
+  // TMEM columns: S; W S_hi and W S_lo side by side
+  static constexpr uint32_t t_s = 0, t_d = 64;
   static_assert(bytes + 1024 <= 232448, "shared memory");
 };
 
@@ -526,8 +528,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* wb = sm + Lay::wb;
   uint8_t* ub = sm + Lay::ub;
   uint8_t* kb = sm + Lay::kb;
-  uint8_t* shi = sm + Lay::shi;
-  uint8_t* slo = sm + Lay::slo;
+  uint8_t* sop = sm + Lay::sop;
   uint8_t* dhi = sm + Lay::dhi;
   uint8_t* dlo = sm + Lay::dlo;
   uint8_t* sst = sm + Lay::sst;
@@ -563,7 +564,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(tmem_slot, 128);
+    tmem_alloc(tmem_slot, 256);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -614,8 +615,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // S (this thread's row, 32 columns) into the K-major B panels of product A
   // as tf32 high part and remainder, and into the staging tile
   auto put_state = [&](const float* v, bool stage) {
-    uint8_t* ph = shi + (row >> 5) * 8192;
-    uint8_t* pl = slo + (row >> 5) * 8192;
+    uint8_t* ph = sop + (row >> 5) * 16384;
+    uint8_t* pl = ph + 8192;
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       const float hi = tf32_rna(v[i]);
@@ -677,15 +678,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       ok = wait_or_abort<false>(bars + kW, par, abort_flag);
       if (ok) {
-        constexpr uint32_t id = idesc_tf32(128, kTile);
+        // one N = 128 MMA per K step: W S_hi in columns 0-63 of the
+        // accumulator, W S_lo in 64-127 (an MMA below N = 128 costs about
+        // as much as one at N = 128)
+        constexpr uint32_t id = idesc_tf32(128, 2 * kTile);
 #pragma unroll
         for (int ks = 0; ks < DK / 8; ++ks) {
-          const uint32_t o = (ks >> 2) * 8192 + (ks & 3) * 32;
-          const uint64_t ad = desc_sw128(smem_u32(wb) + o, 16, 1024);
-          mma_tf32(tmem + Lay::t_d, ad, desc_sw128(smem_u32(shi) + o, 16, 1024),
+          const uint64_t ad = desc_sw128(
+              smem_u32(wb) + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
+          mma_tf32(tmem + Lay::t_d, ad,
+                   desc_sw128(smem_u32(sop) + (ks >> 2) * 16384 + (ks & 3) * 32,
+                              16, 1024),
                    id, ks > 0);
-          mma_tf32(tmem + Lay::t_d, ad, desc_sw128(smem_u32(slo) + o, 16, 1024),
-                   id, 1u);
         }
         mma_commit(bar_mma);
       } else {
@@ -707,13 +711,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (row < kC) {
       ok = wait_or_abort<false>(bars + kU, par, abort_flag);
       if (ok) {
-        float d[32], u[32];
+        float d[32], dl[32], u[32];
         const bool in = row < L;
         uint8_t* up = ub + half * 8192;
         ld_row(up, row, u);
         tmem_ld32(tmem + lane_base + Lay::t_d + 32 * half, d);
+        tmem_ld32(tmem + lane_base + Lay::t_d + 64 + 32 * half, dl);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) d[i] = in ? u[i] - d[i] : 0.f;
+        for (int i = 0; i < 32; ++i) d[i] = in ? u[i] - (d[i] + dl[i]) : 0.f;
         if (L < kC && in) {  // a ragged chunk: no box store past it
           float4* d4 = reinterpret_cast<float4*>(
               p.dd + ((size_t)(tok0 + row) * p.H + h) * p.dv + j0);
@@ -823,7 +828,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (c == 0) bulk_wait_all();
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, 128);
+  if (warp == 0) tmem_dealloc(tmem, 256);
 }
 
 }  // namespace bwdtc
