@@ -471,7 +471,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // state's rounding is amplified in dlog_alpha under strong gates (its reverse
 // sum of differences of terms that grow like exp|g|), so this pass keeps
 // fp32-grade operands: S and Delta, formed here, enter their products as a
-// tf32 high part plus the tf32 remainder (two MMAs each), and W and Kh^T
+// tf32 high part plus the tf32 remainder (product A takes both parts of S
+// as one N = 128 operand, product B two MMAs per step), and W and Kh^T
 // arrive from prep already rounded to the nearest tf32.  One CTA of 256
 // threads per (sequence, head, 64-column d_v tile), S in TMEM throughout;
 // W, U and Kh^T by TMA into one buffer each, refilled as soon as it is free;
