@@ -1451,16 +1451,16 @@ struct BmmMaps {
 // tma_mask); the threads stage the others meanwhile.  A token box's rows
 // past the chunk are other tokens (or zero past the tensor): they only
 // reach output rows or columns past m or n, which are not stored.
+// A CTA takes `per_cta` consecutive (chunk, head) items, heads fastest, and
+// pays its set-up (barriers, TMEM allocation) once for all of them.
 template <int MD, int ND>
 __global__ void __launch_bounds__(kThreads, 3)
     bmm_tc_kernel(BmmOp op, const __grid_constant__ BmmMaps maps,
                   int tma_mask, const int32_t* cu, const int32_t* chunk_off,
-                  int n_seqs, int T, int H, int dk, int dv, int C) {
+                  int n_seqs, int T, int H, int dk, int dv, int C,
+                  int64_t n_items, int per_cta) {
   using namespace sm100;
-  const int cid = blockIdx.x;
-  int seq, tok0, L;
-  if (!locate_chunk(cid, cu, chunk_off, n_seqs, T, C, &seq, &tok0, &L)) return;
-  const int h = blockIdx.y, tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -1489,118 +1489,138 @@ __global__ void __launch_bounds__(kThreads, 3)
   tc_fence_after();
   const uint32_t tmem = *tslot;
   bool ok = true;
-  int tphase = 0;
-  for (int term = 0; term < op.nterms && ok; ++term) {
-    const BmmTerm tm = term == 0 ? op.term[0]
-                       : term == 1 ? op.term[1] : op.term[2];
-    const int kd = tm.kd;
-    const bool ta = (tma_mask >> (2 * term)) & 1;
-    const bool tb = (tma_mask >> (2 * term + 1)) & 1;
-    if (tid == 0 && (ta || tb)) {
-      mbar_arrive_expect_tx(
-          tbar, (ta ? (kd / 32) * kPanA : 0) + (tb ? (kd / 32) * kPanB : 0));
-      for (int side = 0; side < 2; ++side) {
-        if (!(side == 0 ? ta : tb)) continue;
-        const MatRef& x = side == 0 ? tm.a : tm.b;
-        uint8_t* dst = side == 0 ? As : Bs;
-        const int pan = side == 0 ? kPanA : kPanB;
-        for (int q = 0; q < kd / 32; ++q) {
-          if (x.kind == kTok)
-            tma_load_3d(dst + q * pan, &maps.m[term][side], tbar, 32 * q, h,
-                        tok0);
-          else  // states: d_k rows; transposed copies: x.cols rows
-            tma_load_2d(dst + q * pan, &maps.m[term][side], tbar, 32 * q,
-                        (int)(((size_t)cid * H + h) *
-                              (x.kind == kState ? dk : x.cols)));
+  uint32_t tphase = 0, mphase = 0;  // completions of tbar and bar so far
+  const int64_t item0 = (int64_t)blockIdx.x * per_cta;
+  const int64_t item_end = min(item0 + per_cta, n_items);
+  for (int64_t item = item0; item < item_end && ok; ++item) {
+    const int cid = (int)(item / H), h = (int)(item % H);
+    int seq, tok0, L;
+    if (!locate_chunk(cid, cu, chunk_off, n_seqs, T, C, &seq, &tok0, &L))
+      continue;
+    for (int term = 0; term < op.nterms && ok; ++term) {
+      const BmmTerm tm = term == 0 ? op.term[0]
+                         : term == 1 ? op.term[1] : op.term[2];
+      const int kd = tm.kd;
+      const bool ta = (tma_mask >> (2 * term)) & 1;
+      const bool tb = (tma_mask >> (2 * term + 1)) & 1;
+      if (tid == 0 && (ta || tb)) {
+        mbar_arrive_expect_tx(
+            tbar, (ta ? (kd / 32) * kPanA : 0) + (tb ? (kd / 32) * kPanB : 0));
+        for (int side = 0; side < 2; ++side) {
+          if (!(side == 0 ? ta : tb)) continue;
+          const MatRef& x = side == 0 ? tm.a : tm.b;
+          uint8_t* dst = side == 0 ? As : Bs;
+          const int pan = side == 0 ? kPanA : kPanB;
+          for (int q = 0; q < kd / 32; ++q) {
+            if (x.kind == kTok)
+              tma_load_3d(dst + q * pan, &maps.m[term][side], tbar, 32 * q, h,
+                          tok0);
+            else  // states: d_k rows; transposed copies: x.cols rows
+              tma_load_2d(dst + q * pan, &maps.m[term][side], tbar, 32 * q,
+                          (int)(((size_t)cid * H + h) *
+                                (x.kind == kState ? dk : x.cols)));
+          }
+        }
+      }
+      const Src sa = src_of(tm.a, cid, h, tok0, L, H, C, dk);
+      const Src sb = src_of(tm.b, cid, h, tok0, L, H, C, dk);
+      if (!ta) {
+        if (tm.a.trans)  // A[t][i]
+          stage_km_transposed(sa, kd, MD, As, kPanA, tid);
+        else  // A[i][t]
+          stage_km_direct(sa, MD, kd, As, kPanA, tid);
+      }
+      if (!tb) {
+        if (tm.b.trans)  // B[j][t]
+          stage_km_direct(sb, ND, kd, Bs, kPanB, tid);
+        else  // B[t][j]
+          stage_km_transposed(sb, kd, ND, Bs, kPanB, tid);
+      }
+      if (ta || tb) {
+        ok = __syncthreads_and(mbar_wait(tbar, tphase & 1u, 2000000000ull));
+        ++tphase;
+        if (!ok) break;
+      }
+      fence_proxy_async();
+      tc_fence_before();
+      __syncthreads();
+      if (tid == 0) {
+        tc_fence_after();
+        constexpr uint32_t id = idesc_tf32(MD, ND);
+        for (int ks = 0; ks < kd / 8; ++ks)
+          mma_tf32(tmem,
+                   desc_sw128(smem_u32(As) + (ks >> 2) * kPanA + (ks & 3) * 32,
+                              16, 1024),
+                   desc_sw128(smem_u32(Bs) + (ks >> 2) * kPanB + (ks & 3) * 32,
+                              16, 1024),
+                   id, (term > 0 || ks > 0) ? 1u : 0u);
+        mma_commit(bar);
+      }
+      // the operands are read once the products complete: the next term may
+      // then restage them
+      ok = __syncthreads_and(mbar_wait(bar, mphase & 1u, 2000000000ull));
+      ++mphase;
+      tc_fence_after();
+    }
+    if (!ok) {
+      if (tid == 0) atomicExch(&g_bwd_timeout, 1);
+    } else {
+      const int m = dim_of(op.m, L, dk, dv), n = dim_of(op.n, L, dk, dv);
+      const Src so = src_of(op.out, cid, h, tok0, L, H, C, dk);
+      const int lane = tid & 31, q = warp & 3, chalf = tid >> 7;
+      const int i =
+          MD == 128 ? 32 * q + lane : (lane < 16 ? 16 * q + lane : MD);
+      const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16);
+  #pragma unroll
+      for (int cc = 0; cc < ND / 64; ++cc) {
+        const int j0 = chalf * (ND / 2) + 32 * cc;
+        float x[32];
+        tmem_ld32(taddr + j0, x);
+        if (i < m && j0 < n) {
+  #pragma unroll
+          for (int b = 0; b < 32; ++b) {
+            const int j = j0 + b;
+            x[b] *= op.alpha;
+            if ((op.mask == kMaskLowerIncl && j > i) ||
+                (op.mask == kMaskStrictLower && j >= i))
+              x[b] = 0.f;
+          }
+          float* o = so.p + (size_t)i * so.stride + j0;
+          if (j0 + 32 <= n) {
+  #pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              float4* o4 = reinterpret_cast<float4*>(o + 4 * v);
+              float4 y = make_float4(x[4 * v], x[4 * v + 1], x[4 * v + 2],
+                                     x[4 * v + 3]);
+              if (op.accumulate) {
+                const float4 z = *o4;
+                y.x += z.x;
+                y.y += z.y;
+                y.z += z.z;
+                y.w += z.w;
+              }
+              *o4 = y;
+            }
+          } else {
+  #pragma unroll
+            for (int b = 0; b < 32; ++b)
+              if (j0 + b < n) o[b] = op.accumulate ? o[b] + x[b] : x[b];
+          }
         }
       }
     }
-    const Src sa = src_of(tm.a, cid, h, tok0, L, H, C, dk);
-    const Src sb = src_of(tm.b, cid, h, tok0, L, H, C, dk);
-    if (!ta) {
-      if (tm.a.trans) stage_km_transposed(sa, kd, MD, As, kPanA, tid);  // A[t][i]
-      else stage_km_direct(sa, MD, kd, As, kPanA, tid);                 // A[i][t]
-    }
-    if (!tb) {
-      if (tm.b.trans) stage_km_direct(sb, ND, kd, Bs, kPanB, tid);  // B[j][t]
-      else stage_km_transposed(sb, kd, ND, Bs, kPanB, tid);         // B[t][j]
-    }
-    if (ta || tb) {
-      ok = __syncthreads_and(mbar_wait(tbar, (uint32_t)tphase & 1u,
-                                       2000000000ull));
-      ++tphase;
-      if (!ok) break;
-    }
-    fence_proxy_async();
+    // this item's TMEM reads end before the next item's products start
     tc_fence_before();
     __syncthreads();
-    if (tid == 0) {
-      tc_fence_after();
-      constexpr uint32_t id = idesc_tf32(MD, ND);
-      for (int ks = 0; ks < kd / 8; ++ks)
-        mma_tf32(tmem,
-                 desc_sw128(smem_u32(As) + (ks >> 2) * kPanA + (ks & 3) * 32,
-                            16, 1024),
-                 desc_sw128(smem_u32(Bs) + (ks >> 2) * kPanB + (ks & 3) * 32,
-                            16, 1024),
-                 id, (term > 0 || ks > 0) ? 1u : 0u);
-      mma_commit(bar);
-    }
-    // the operands are read once the products complete: the next term may
-    // then restage them
-    ok = __syncthreads_and(mbar_wait(bar, (uint32_t)term & 1u, 2000000000ull));
     tc_fence_after();
-  }
-  if (!ok) {
-    if (tid == 0) atomicExch(&g_bwd_timeout, 1);
-  } else {
-    const int m = dim_of(op.m, L, dk, dv), n = dim_of(op.n, L, dk, dv);
-    const Src so = src_of(op.out, cid, h, tok0, L, H, C, dk);
-    const int lane = tid & 31, q = warp & 3, chalf = tid >> 7;
-    const int i = MD == 128 ? 32 * q + lane : (lane < 16 ? 16 * q + lane : MD);
-    const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16);
-#pragma unroll
-    for (int cc = 0; cc < ND / 64; ++cc) {
-      const int j0 = chalf * (ND / 2) + 32 * cc;
-      float x[32];
-      tmem_ld32(taddr + j0, x);
-      if (i < m && j0 < n) {
-#pragma unroll
-        for (int b = 0; b < 32; ++b) {
-          const int j = j0 + b;
-          x[b] *= op.alpha;
-          if ((op.mask == kMaskLowerIncl && j > i) ||
-              (op.mask == kMaskStrictLower && j >= i))
-            x[b] = 0.f;
-        }
-        float* o = so.p + (size_t)i * so.stride + j0;
-        if (j0 + 32 <= n) {
-#pragma unroll
-          for (int v = 0; v < 8; ++v) {
-            float4* o4 = reinterpret_cast<float4*>(o + 4 * v);
-            float4 y = make_float4(x[4 * v], x[4 * v + 1], x[4 * v + 2],
-                                   x[4 * v + 3]);
-            if (op.accumulate) {
-              const float4 z = *o4;
-              y.x += z.x;
-              y.y += z.y;
-              y.z += z.z;
-              y.w += z.w;
-            }
-            *o4 = y;
-          }
-        } else {
-#pragma unroll
-          for (int b = 0; b < 32; ++b)
-            if (j0 + b < n) o[b] = op.accumulate ? o[b] + x[b] : x[b];
-        }
-      }
-    }
-  }
+  }  // items
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, ND);
 }
+
+// Items (chunk, head) one tensor-core product CTA takes in turn.
+constexpr int kBmmItems = 4;
 
 template <int MD, int ND>
 cudaError_t launch_bmm_tc_t(const BmmOp& op, const BmmMaps& maps, int mask,
@@ -1615,8 +1635,13 @@ cudaError_t launch_bmm_tc_t(const BmmOp& op, const BmmMaps& maps, int mask,
   const size_t smem = (size_t)(kdmax / 32) * (MD + ND) * 128 + 1024 + 64;
   cudaError_t e = set_smem(bmm_tc_kernel<MD, ND>, smem);
   if (e != cudaSuccess) return e;
-  bmm_tc_kernel<MD, ND><<<grid, kThreads, smem, stream>>>(
-      op, maps, mask, cu, co, n_seqs, T, H, dk, dv, C);
+  // kBmmItems consecutive items per CTA while that leaves at least two
+  // resident waves of CTAs (three per SM on 148 SMs), else one
+  const int64_t items = (int64_t)grid.x * grid.y;
+  const int per = items >= (int64_t)kBmmItems * 2 * 3 * 148 ? kBmmItems : 1;
+  const unsigned ctas = (unsigned)((items + per - 1) / per);
+  bmm_tc_kernel<MD, ND><<<ctas, kThreads, smem, stream>>>(
+      op, maps, mask, cu, co, n_seqs, T, H, dk, dv, C, items, per);
   return cudaGetLastError();
 }
 
