@@ -1619,7 +1619,9 @@ __global__ void __launch_bounds__(kThreads, 3)
   if (warp == 0) tmem_dealloc(tmem, ND);
 }
 
-// Items (chunk, head) one tensor-core product CTA takes in turn.
+// Items (chunk, head) one tensor-core product CTA takes in turn at most (the
+// A/B on B = 2, T = 8192, H = 32, d = 128: 1 item 5.86 ms, 2 5.69, 4 5.66,
+// 8 5.87 ms for the whole backward).
 constexpr int kBmmItems = 4;
 
 template <int MD, int ND>
@@ -1635,10 +1637,19 @@ cudaError_t launch_bmm_tc_t(const BmmOp& op, const BmmMaps& maps, int mask,
   const size_t smem = (size_t)(kdmax / 32) * (MD + ND) * 128 + 1024 + 64;
   cudaError_t e = set_smem(bmm_tc_kernel<MD, ND>, smem);
   if (e != cudaSuccess) return e;
-  // kBmmItems consecutive items per CTA while that leaves at least two
-  // resident waves of CTAs (three per SM on 148 SMs), else one
+  // items per CTA: 4, 2 or 1, whichever still leaves two resident waves
   const int64_t items = (int64_t)grid.x * grid.y;
-  const int per = items >= (int64_t)kBmmItems * 2 * 3 * 148 ? kBmmItems : 1;
+  int dev = 0, sms = 0, per_sm = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
+      (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) !=
+          cudaSuccess ||
+      (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+           &per_sm, bmm_tc_kernel<MD, ND>, kThreads, smem)) != cudaSuccess)
+    return e;
+  const int64_t wave = (int64_t)sms * (per_sm > 0 ? per_sm : 1);
+  const int per = items >= 2 * kBmmItems * wave ? kBmmItems
+                  : items >= kBmmItems * wave   ? kBmmItems / 2
+                                                : 1;
   const unsigned ctas = (unsigned)((items + per - 1) / per);
   bmm_tc_kernel<MD, ND><<<ctas, kThreads, smem, stream>>>(
       op, maps, mask, cu, co, n_seqs, T, H, dk, dv, C, items, per);
