@@ -398,6 +398,32 @@ kda_status kda_chunk_bwd_plan(const kda_shape* shape, int packed, int* kernels,
   return KDA_OK;
 }
 
+kda_status kda_chunk_bwd_layout(const kda_shape* shape, int packed, int cap,
+                                size_t* offsets, size_t* sizes,
+                                int* first_launch, int* last_launch,
+                                int* count) {
+  if (!count || cap < 0) return KDA_ERR_INVALID_ARG;
+  if (cap > 0 && (!offsets || !sizes || !first_launch || !last_launch))
+    return KDA_ERR_INVALID_ARG;
+  int n_seqs = 0;
+  const kda_status st = validate_chunk_shape(shape, packed != 0, &n_seqs);
+  if (st != KDA_OK) return st;
+  kda::BwdArgs b{};
+  fill_args(shape, n_seqs, &b.f);
+  static const int32_t kTag = 0;  // only tells the planner the layout
+  b.f.cu_seqlens = packed ? &kTag : nullptr;
+  kda::BwdArray arr[64];
+  const int n = kda::bwd_workspace_layout(b, arr, 64);
+  for (int i = 0; i < n && i < cap && i < 64; ++i) {
+    offsets[i] = arr[i].offset;
+    sizes[i] = arr[i].bytes;
+    first_launch[i] = arr[i].first;
+    last_launch[i] = arr[i].last;
+  }
+  *count = n;
+  return KDA_OK;
+}
+
 kda_status kda_chunk_fwd_gated(const kda_shape* shape, int gate, const void* q,
                                const void* k, const void* v,
                                const float* log_gate, const float* beta,

@@ -113,7 +113,8 @@ bool tensor_chain(const ChunkArgs& f) {
          max_chunks(f) * f.H * (f.dk > f.dv ? f.dk : f.dv) < ((int64_t)1 << 31);
 }
 
-BwdWs carve_bwd(const BwdArgs& a, void* base, size_t* total) {
+BwdWs carve_bwd(const BwdArgs& a, void* base, size_t* total,
+                BwdArray* info = nullptr, int cap = 0, int* count = nullptr) {
   const ChunkArgs& f = a.f;
   const size_t tokens =
       f.cu_seqlens ? (size_t)f.T : (size_t)f.n_seqs * (size_t)f.T;
@@ -147,6 +148,7 @@ BwdWs carve_bwd(const BwdArgs& a, void* base, size_t* total) {
     w.qdo = take(st);
     w.pdo = take(tdv);
     if (total) *total = off;
+    if (count) *count = 0;
     return w;
   }
   // Tensor-core path: arrays share memory where their lifetimes (from the
@@ -231,6 +233,9 @@ BwdWs carve_bwd(const BwdArgs& a, void* base, size_t* total) {
   }
   for (int i = 0; i < n; ++i)
     *arr[i].ptr = p ? reinterpret_cast<float*>(p + offs[i]) : nullptr;
+  for (int i = 0; i < n && i < cap; ++i)
+    info[i] = BwdArray{offs[i], arr[i].bytes, arr[i].first, arr[i].last};
+  if (count) *count = n;
   w.staged = staged;
   w.fv.w = sw;
   w.fv.d = su;
@@ -1990,6 +1995,13 @@ size_t bwd_workspace_bytes(const BwdArgs& a) {
   size_t total = 0;
   carve_bwd(a, nullptr, &total);
   return total;
+}
+
+int bwd_workspace_layout(const BwdArgs& a, BwdArray* out, int cap) {
+  size_t total = 0;
+  int count = 0;
+  carve_bwd(a, nullptr, &total, out, out ? cap : 0, &count);
+  return count;
 }
 
 int bwd_kernel_count(const BwdArgs& a) {

@@ -168,6 +168,16 @@ struct BwdArgs {
 };
 size_t bwd_workspace_bytes(const BwdArgs& a);
 int bwd_kernel_count(const BwdArgs& a);
+// One array of the backward's workspace: its byte offset and size, and the
+// first and last launch of the call (in launch order) that touch it.
+struct BwdArray {
+  size_t offset, bytes;
+  int first, last;
+};
+// The arrays of a backward call's workspace, the first `cap` of them into
+// `out`; returns how many there are: 0 on the fp32 path, whose arrays never
+// share memory.
+int bwd_workspace_layout(const BwdArgs& a, BwdArray* out, int cap);
 cudaError_t launch_bwd(const BwdArgs& a, void* workspace, cudaStream_t stream);
 
 // Fused tensor-core prefill (kda_fused_sm100.cu): bf16 io, dk, dv in

@@ -27,7 +27,8 @@ EXPORTS = ("kda_chunk_fwd", "kda_chunk_fwd_staged", "kda_recurrent_step",
            "kda_recurrent_step_ex", "kda_selftest_timeout", "kda_chunk_bwd",
            "kda_chunk_bwd_plan", "kda_chunk_fwd_split", "kda_workspace_pool",
            "kda_chunk_fwd_twopass", "kda_chunk_fwd_paired",
-           "kda_chunk_fwd_split_plan", "kda_profile_pass_event")
+           "kda_chunk_fwd_split_plan", "kda_profile_pass_event",
+           "kda_chunk_bwd_layout")
 GATES = {"channel": 0, "head": 1, "none": 2}
 
 
@@ -133,6 +134,12 @@ def library():
         lib.kda_chunk_bwd_plan.argtypes = [
             ctypes.POINTER(KdaShape), ctypes.c_int, ctypes.POINTER(ctypes.c_int),
             ctypes.POINTER(ctypes.c_size_t)]
+        lib.kda_chunk_bwd_layout.restype = ctypes.c_int
+        lib.kda_chunk_bwd_layout.argtypes = [
+            ctypes.POINTER(KdaShape), ctypes.c_int, ctypes.c_int,
+            ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t),
+            ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int),
+            ctypes.POINTER(ctypes.c_int)]
         lib.kda_selftest_umma.restype = ctypes.c_int
         lib.kda_selftest_umma.argtypes = [ctypes.c_int] * 5 + [vp, vp, vp, vp]
         lib.kda_selftest_timeout.restype = ctypes.c_int
@@ -351,6 +358,25 @@ def chunk_bwd_plan(B, T, H, dk, dv, chunk, dtype, packed=False, n_seqs=0):
     if st != KDA_OK:
         raise KdaError(st, "kda_chunk_bwd_plan")
     return kern.value, ws.value
+
+
+def chunk_bwd_layout(B, T, H, dk, dv, chunk, dtype, packed=False, n_seqs=0):
+    """The workspace arrays of a chunk_bwd call of this shape, as (offset,
+    bytes, first launch, last launch) tuples (kda_chunk_bwd_layout); empty on
+    the fp32 path, whose arrays are all apart."""
+    io = KDA_BF16 if dtype == torch.bfloat16 else KDA_F32
+    shape = KdaShape(B, T, H, dk, dv, chunk, n_seqs if packed else 0, io)
+    cap = 64
+    offs, sizes = (ctypes.c_size_t * cap)(), (ctypes.c_size_t * cap)()
+    first, last, count = (ctypes.c_int * cap)(), (ctypes.c_int * cap)(), \
+        ctypes.c_int()
+    st = library().kda_chunk_bwd_layout(ctypes.byref(shape), int(packed), cap,
+                                        offs, sizes, first, last,
+                                        ctypes.byref(count))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_chunk_bwd_layout")
+    return [(offs[i], sizes[i], first[i], last[i])
+            for i in range(min(count.value, cap))]
 
 
 def recurrent_step(q, k, v, log_alpha, beta, state, out=None, stream=None,

@@ -438,6 +438,25 @@ KDA_API kda_status kda_chunk_bwd(const kda_shape* shape, const void* q,
 KDA_API kda_status kda_chunk_bwd_plan(const kda_shape* shape, int packed,
                                       int* kernels, size_t* workspace_bytes);
 
+/* kda_chunk_bwd_layout -- how a kda_chunk_bwd call of this shape lays out its
+ * workspace; no device work.  On the tensor-core path (bf16, chunk 64, d_k
+ * and d_v in {64, 128}) the call's intermediate arrays share memory where
+ * their lifetimes do not overlap.  For each array i < min(*count, cap) it
+ * writes its byte offset in the workspace, its size in bytes, and the first
+ * and last launch of the call (numbered in launch order) that touch it; two
+ * arrays whose launch ranges overlap never share a byte.  *count receives
+ * the number of arrays (0 on the fp32 path, whose arrays are all apart).
+ *   shape, packed : as kda_chunk_bwd_plan.
+ *   cap           : room in each output array (0: count only).
+ *   offsets, sizes, first_launch, last_launch : host arrays of cap entries
+ *                   (may be NULL when cap is 0).
+ * KDA_ERR_INVALID_ARG for a NULL count, a negative cap, or NULL arrays with
+ * cap > 0; shape errors as kda_chunk_bwd_plan. */
+KDA_API kda_status kda_chunk_bwd_layout(const kda_shape* shape, int packed,
+                                        int cap, size_t* offsets,
+                                        size_t* sizes, int* first_launch,
+                                        int* last_launch, int* count);
+
 /*
  * kda_chunk_fwd_split -- the chunkwise prefill of ONE long sequence (dense
  * layout, shape->B == 1, no cu_seqlens), evaluated as n_segments segments

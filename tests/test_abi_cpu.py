@@ -81,6 +81,34 @@ def test_backward_plan(lib):
     assert kern_p == 17
 
 
+@pytest.mark.parametrize("B,T,H,dk,dv,packed,n_seqs", [
+    (2, 8192, 32, 128, 128, False, 0),   # the prefill workload
+    (1, 2048, 4, 64, 64, False, 0),
+    (2, 200, 3, 64, 128, False, 0),      # ragged last chunk, d_k != d_v
+    (1, 300, 2, 128, 64, True, 3),       # packed layout
+])
+def test_backward_workspace_layout(lib, B, T, H, dk, dv, packed, n_seqs):
+    import torch
+    arrays = K.chunk_bwd_layout(B, T, H, dk, dv, 64, torch.bfloat16,
+                                packed=packed, n_seqs=n_seqs)
+    _, ws = K.chunk_bwd_plan(B, T, H, dk, dv, 64, torch.bfloat16,
+                             packed=packed, n_seqs=n_seqs)
+    assert len(arrays) > 20
+    assert max(o + b for o, b, _, _ in arrays) <= ws
+    for o, b, f, l in arrays:
+        assert o % 256 == 0 and b > 0 and 0 <= f <= l
+    # arrays whose launch ranges overlap never share a byte
+    for i, (oi, bi, fi, li) in enumerate(arrays):
+        for oj, bj, fj, lj in arrays[i + 1:]:
+            if fi <= lj and fj <= li:
+                assert oi + bi <= oj or oj + bj <= oi, (i, oi, bi, oj, bj)
+    # and the packing does share memory: the arrays' sum exceeds the workspace
+    assert sum(b for _, b, _, _ in arrays) > ws
+    # the fp32 path keeps every array apart and reports none
+    assert K.chunk_bwd_layout(B, T, H, dk, dv, 64, torch.float32,
+                              packed=packed, n_seqs=n_seqs) == []
+
+
 def test_split_plan(lib):
     import torch
     # plan: segments of ceil(chunks / n) chunks; the kernels are the setup,
